@@ -1,0 +1,377 @@
+"""Pins of the CPU oracle against things other than itself: closed forms,
+brute force on tiny inputs, library routines, error bounds and invariants.
+
+Each test names the part of the layer it pins.  A plausible mistake in the
+oracle (a dropped term, a wrong sign or index, a transposed operand, a wrong
+tie rule) fails at least one of them.
+"""
+import itertools
+import math
+
+import numpy as np
+import pytest
+
+import oracle
+import synth
+
+U32 = 2.0 ** -24  # unit roundoff of fp32
+
+
+def ulp_dist(a, b):
+    """Distance in fp32 ulps between two positive fp32 arrays."""
+    ai = np.asarray(a, np.float32).view(np.int32).astype(np.int64)
+    bi = np.asarray(b, np.float32).view(np.int32).astype(np.int64)
+    return np.abs(ai - bi)
+
+
+# ----------------------------------------------------------------------------- exp
+
+def test_exp_within_2ulp_of_libm_dense_sweep():
+    x = np.linspace(-87.0, 88.0, 2_000_001, dtype=np.float32)
+    y = oracle.expf(x)
+    ref = np.exp(x.astype(np.float64)).astype(np.float32)  # correctly rounded to fp32 in practice
+    assert ulp_dist(y, ref).max() <= 2
+
+
+def test_exp_special_values_and_clamp():
+    assert oracle.expf(np.float32(0.0))[0] == 1.0
+    assert ulp_dist(oracle.expf(np.float32(1.0)), np.float32(math.e))[0] <= 1
+    # arguments beyond the range are clamped to [-87, 88]
+    assert oracle.expf(np.float32(-200.0))[0] == oracle.expf(np.float32(-87.0))[0]
+    assert oracle.expf(np.float32(500.0))[0] == oracle.expf(np.float32(88.0))[0]
+    # e^a e^-a = 1 within a few ulp on random arguments
+    a = synth.uniform(11, 1, (10000,), -40.0, 40.0)
+    prod = oracle.expf(a).astype(np.float64) * oracle.expf(-a).astype(np.float64)
+    assert np.abs(prod - 1.0).max() < 6 * U32
+
+
+# ----------------------------------------------------------------------------- quantisation
+
+def test_quant_handcrafted_halves_and_zero_row():
+    # amax 127 gives scale exactly 1, so q = rint(v) with ties to even
+    row = np.array([127.0, 2.5, 3.5, -2.5, -3.5, 0.5, -0.5, 1.5, 126.5, -127.0], np.float32)
+    q, s = oracle.quantize_rows(row[None, :])
+    assert s[0] == 1.0
+    assert q[0].tolist() == [127, 2, 4, -2, -4, 0, 0, 2, 126, -127]
+    q, s = oracle.quantize_rows(np.zeros((1, 16), np.float32))
+    assert s[0] == 0.0 and not q.any()
+
+
+def test_quant_error_bound_and_full_range():
+    v = synth.normal(12, 1, (200, 333), std=3.0)
+    v[7] *= 1e-30          # tiny row
+    v[9, :] = 0.0
+    v[9, 5] = -2.0         # single non-zero entry
+    q, s = oracle.quantize_rows(v)
+    for r in range(v.shape[0]):
+        amax = np.abs(v[r]).max()
+        assert s[r] == np.float32(amax) / np.float32(127.0)
+        err = np.abs(v[r].astype(np.float64) - q[r].astype(np.float64) * float(s[r]))
+        # half a step, plus the rounding of v/s
+        assert err.max() <= float(s[r]) * (0.5 + 1e-5)
+        assert np.abs(q[r]).max() == 127
+    assert q[9, 5] == -127 and np.count_nonzero(q[9]) == 1
+
+
+# ----------------------------------------------------------------------------- smoothing
+
+def test_smoothing_identity_fp64():
+    """(X diag(s)^-1)(diag(s) W) = X W for the oracle's scales."""
+    x = synth.normal(13, 1, (16, 64)).astype(np.float64)
+    w = synth.normal(13, 2, (64, 32), std=0.02).astype(np.float64)
+    ax = np.abs(x).max(0).astype(np.float32)
+    aw = np.abs(w).max(1).astype(np.float32)
+    s, inv = oracle.smooth_scales(ax, aw, 0.6)
+    s64 = s.astype(np.float64)
+    lhs = (x / s64) @ (s64[:, None] * w)
+    assert np.abs(lhs - x @ w).max() <= 1e-12 * np.abs(x @ w).max()
+
+
+def test_smoothing_closed_forms():
+    ax = np.array([4.0, 9.0, 0.25, 0.0, 2.0], np.float32)
+    aw = np.array([1.0, 4.0, 0.04, 3.0, 0.0], np.float32)
+    # alpha = 1: s = max|X|;  alpha = 0: s = 1 / max|W|  (both floored at 1e-5)
+    s1, _ = oracle.smooth_scales(ax, aw, 1.0)
+    assert np.allclose(s1, np.maximum(ax, np.float32(1e-5)), rtol=1e-7)
+    s0, _ = oracle.smooth_scales(ax, aw, 0.0)
+    assert np.allclose(s0, 1.0 / np.maximum(aw, np.float32(1e-5)).astype(np.float64), rtol=1e-7)
+    # alpha = 1/2 balances the two: max|X_j| / s_j == max|W_j| * s_j
+    s, inv = oracle.smooth_scales(ax[:3], aw[:3], 0.5)
+    assert np.allclose(ax[:3] / s, aw[:3] * s, rtol=1e-6)
+    assert np.allclose(s.astype(np.float64) * inv, 1.0, atol=2 * U32)
+
+
+def test_weight_quant_is_per_output_channel_of_smoothed_weights():
+    d, f = 32, 24
+    w = synth.normal(14, 3, (d, f), std=0.02)
+    s = np.linspace(0.5, 3.0, d).astype(np.float32)
+    q, sw = oracle.quantize_gateup_expert(w, s)
+    assert q.shape == (f, d)
+    ws = (s[:, None] * w).astype(np.float32)           # W'[j][n] = s_j W[j][n]
+    for n in range(f):
+        assert sw[n] == np.float32(np.abs(ws[:, n]).max()) / np.float32(127.0)
+        assert np.abs(ws[:, n] - q[n] * sw[n]).max() <= sw[n] * 0.50001
+    qd, swd = oracle.quantize_down_expert(w.T.copy())   # [f][d] -> channels over d
+    assert qd.shape == (d, f)
+    for n in range(d):
+        assert swd[n] == np.float32(np.abs(w.T[:, n]).max()) / np.float32(127.0)
+
+
+# ----------------------------------------------------------------------------- router
+
+def test_router_logits_within_dot_error_bound():
+    T, d, E = 8, 512, 16
+    x = synth.normal(15, 1, (T, d))
+    x[:, 3] *= 30.0
+    wr = synth.normal(15, 2, (d, E), std=0.02)
+    lg = oracle.router_logits(x, wr)
+    ref = x.astype(np.float64) @ wr.astype(np.float64)
+    bound = d * U32 * (np.abs(x).astype(np.float64) @ np.abs(wr).astype(np.float64))
+    assert np.all(np.abs(lg - ref) <= bound)
+
+
+def test_router_logits_order_is_the_stated_one():
+    """Hand-made exact cases that tell the stated order (32 lane chains over
+    j = 32 i + p, then the xor butterfly 16, 8, 4, 2, 1) apart from a plain
+    sequential sum: 2^25 + 1 loses the 1 in fp32, so where a +1 lands decides
+    the result."""
+    d = 64
+    big = 2.0 ** 25
+
+    def logit(prods):
+        x = np.zeros((1, d), np.float32)
+        w = np.zeros((d, 1), np.float32)
+        for j, v in prods.items():
+            x[0, j], w[j, 0] = 1.0, v
+        return float(oracle.router_logits(x, w)[0, 0])
+
+    # integer partial sums below 2^24 are exact in any order
+    x = (np.arange(d) % 7).astype(np.float32)[None, :]
+    w = (np.arange(d) % 5).astype(np.float32)[:, None]
+    assert oracle.router_logits(x, w)[0, 0] == float((x[0] * w[:, 0]).sum())
+    # lane 0 chains j = 0 and j = 32 (cancel exactly), lane 1 holds j = 1
+    assert logit({0: big, 32: -big, 1: 1.0}) == 1.0        # sequential j order gives 0
+    assert logit({0: big, 1: -big, 32: 1.0}) == 0.0        # sequential j order gives 1
+    # butterfly: lane 0 meets lane 16 first, lane 1 only at the last step
+    assert logit({0: big, 16: -big, 1: 1.0}) == 1.0        # sequential lane order gives 0
+    assert logit({0: big, 1: -big, 16: 1.0}) == 0.0        # sequential lane order gives 1
+
+
+def _brute_topk(l, k):
+    """Brute force over all k-subsets: the chosen set maximises the sum of its
+    logits (fp64); among equal sums the lexicographically smallest index tuple
+    wins; slots are ordered by logit descending, index ascending."""
+    E = len(l)
+    best, best_key = None, None
+    for S in itertools.combinations(range(E), k):
+        key = (-sum(float(l[e]) for e in S), S)
+        if best_key is None or key < best_key:
+            best, best_key = S, key
+    return sorted(best, key=lambda e: (-float(l[e]), e))
+
+
+def test_topk_brute_force_all_subsets_tiny_config():
+    w = synth.WORKLOADS["tiny"]
+    data = synth.make_data(w)
+    lg = oracle.router_logits(data.x, data.w_router)
+    idx, wt = oracle.topk_softmax(lg, w.k)
+    for t in range(w.T):
+        assert idx[t].tolist() == _brute_topk(lg[t], w.k)
+
+
+def test_topk_ties_go_to_lowest_index():
+    w = synth.WORKLOADS["tiny"]
+    data = synth.make_data(w)
+    wr = data.w_router.copy()
+    wr[:, 5] = wr[:, 2]   # experts 2 and 5 always tie
+    wr[:, 7] = wr[:, 2]   # and 7
+    lg = oracle.router_logits(data.x, wr)
+    assert np.array_equal(lg[:, 2], lg[:, 5]) and np.array_equal(lg[:, 2], lg[:, 7])
+    idx, _ = oracle.topk_softmax(lg, 2)
+    for t in range(w.T):
+        assert idx[t].tolist() == _brute_topk(lg[t], 2)
+        if 5 in idx[t] or 7 in idx[t]:
+            assert 2 in idx[t]          # 5 or 7 only ever come with (after) 2
+    # all-equal logits: slots are 0..k-1 with equal weights 1/k
+    idx, wt = oracle.topk_softmax(np.zeros((3, 8), np.float32), 4)
+    assert idx.tolist() == [[0, 1, 2, 3]] * 3 and np.all(wt == np.float32(0.25))
+
+
+def test_gate_weights_softmax_over_selected():
+    lg = synth.normal(16, 1, (500, 64), std=2.0)
+    bias = synth.zipf_bias(16, 64)
+    idx, w = oracle.topk_softmax(lg, 4, bias)
+    l = lg.astype(np.float64) + bias.astype(np.float32).astype(np.float64)
+    for t in range(0, 500, 7):
+        assert idx[t].tolist() == sorted(range(64), key=lambda e: (-np.float32(lg[t, e] + bias[e]), e))[:4]
+    sel = np.take_along_axis(l, idx.astype(np.int64), 1)
+    ref = np.exp(sel - sel[:, :1])
+    ref /= ref.sum(1, keepdims=True)
+    assert np.abs(w - ref).max() < 8 * U32
+    assert np.abs(w.astype(np.float64).sum(1) - 1.0).max() <= 4 * U32
+    assert np.all(np.diff(w, axis=1) <= 0)   # rank order
+    # without renormalisation the weights are the full softmax restricted to the k slots
+    idx2, w2 = oracle.topk_softmax(lg, 4, bias, renormalize=False)
+    full = np.exp(l - l.max(1, keepdims=True))
+    full /= full.sum(1, keepdims=True)
+    assert np.abs(w2 - np.take_along_axis(full, idx2.astype(np.int64), 1)).max() < 8 * U32
+
+
+# ----------------------------------------------------------------------------- permutation
+
+def test_permute_matches_stable_sort_and_round_trips():
+    T, k, E = 300, 4, 16
+    idx = np.stack([synth.permutation(17, 100 + t, E)[:k] for t in range(T)]).astype(np.int32)
+    idx[:50] = np.array([3, 0, 1, 2])        # a crowded expert
+    offsets, row2ts, ts2row = oracle.permute(idx, E)
+    flat = idx.reshape(-1)
+    order = np.argsort(flat, kind="stable")  # library stable sort by expert
+    assert np.array_equal(row2ts, order)
+    counts = np.bincount(flat, minlength=E)
+    assert np.array_equal(np.diff(offsets), counts) and offsets[-1] == T * k
+    assert np.array_equal(row2ts[ts2row.reshape(-1)], np.arange(T * k))
+    for e in range(E):
+        rows = row2ts[offsets[e]:offsets[e + 1]]
+        assert np.all(flat[rows] == e) and np.all(np.diff(rows // k) > 0)
+
+
+def test_capacity_drops_in_token_order():
+    T, k, E = 200, 3, 8
+    rng_keys = synth.bits(18, 1, T * k)
+    idx = np.zeros((T, k), np.int32)
+    for t in range(T):                       # skewed: expert 0 very hot
+        choices = []
+        for s in range(k):
+            c = int(rng_keys[t * k + s] % 4) if s == 0 else int(rng_keys[t * k + s] % E)
+            while c in choices:
+                c = (c + 1) % E
+            choices.append(c)
+        idx[t] = choices
+    cap = oracle.capacity(1.25, T, k, E)
+    assert cap == math.ceil(1.25 * T * k / E)
+    offsets, row2ts, ts2row = oracle.permute(idx, E, cap)
+    # brute-force simulation in (token, slot) order
+    seen = [0] * E
+    kept = np.zeros((T, k), bool)
+    for t in range(T):
+        for s in range(k):
+            e = idx[t, s]
+            if seen[e] < cap:
+                seen[e] += 1
+                kept[t, s] = True
+    assert np.array_equal(ts2row >= 0, kept)
+    counts = np.bincount(idx.reshape(-1), minlength=E)
+    assert np.array_equal(np.diff(offsets), np.minimum(counts, cap))
+    assert np.array_equal(row2ts[ts2row[kept]], np.flatnonzero(kept.reshape(-1)))
+    assert oracle.capacity(0.0, T, k, E) == -1
+    assert oracle.capacity(1.25, 4096, 8, 256) == 160
+
+
+# ----------------------------------------------------------------------------- GEMM
+
+def test_int8_gemm_equals_int64_matmul():
+    a = (synth.bits(19, 1, 37 * 300) % 255).astype(np.int64) - 127
+    b = (synth.bits(19, 2, 29 * 300) % 255).astype(np.int64) - 127
+    a = a.reshape(37, 300)
+    b = b.reshape(29, 300)
+    a[0] = 127
+    b[0] = 127
+    b[1] = -127
+    c = oracle.gemm_i8(a.astype(np.int8), b.astype(np.int8))
+    assert np.array_equal(c.astype(np.int64), a @ b.T)
+
+
+# ----------------------------------------------------------------------------- whole layer
+
+def _integer_layer(T, d, E, k, f, seed):
+    """Inputs on which quantisation is exact: integer-valued X rows with
+    |x| max exactly 127, integer weights with every output channel's max 127."""
+    def ints(tid, shape):
+        v = (synth.bits(seed, tid, int(np.prod(shape))) % 255).astype(np.int64) - 127
+        return v.reshape(shape)
+    x = ints(1, (T, d))
+    x[:, 0] = 127
+    wg = ints(2, (E, d, f)); wg[:, 0, :] = 127
+    wu = ints(3, (E, d, f)); wu[:, 1, :] = -127
+    wd = ints(4, (E, f, d)); wd[:, 0, :] = 127
+    # scale the weights so that the dequantised gate/up land in SiLU's interesting range
+    return x, wg, wu, wd
+
+
+def test_whole_layer_closed_form_integer_case():
+    T, d, E, k, f = 24, 64, 4, 2, 32
+    x, wg, wu, wd = _integer_layer(T, d, E, k, f, 20)
+    prep = oracle.prepare(wg.astype(np.float32), wu.astype(np.float32), wd.astype(np.float32),
+                          x.astype(np.float32), 0.5, smooth=False)
+    assert np.all(prep.sw_gate == 1.0) and np.all(prep.sw_up == 1.0) and np.all(prep.sw_down == 1.0)
+    assert np.array_equal(prep.wq_gate.astype(np.int64), wg.transpose(0, 2, 1))
+    assert np.array_equal(prep.wq_down.astype(np.int64), wd.transpose(0, 2, 1))
+    logits = synth.normal(20, 9, (T, E))
+    rt = oracle.route(x.astype(np.float32), k, E, logits=logits)
+    y, dbg = oracle.moe_tokens(x.astype(np.float32), prep, rt)
+    assert np.all(dbg["sx"] == 1.0) and np.array_equal(dbg["xq"].astype(np.int64), x)
+    for t in range(T):
+        for s in range(k):
+            e = rt.idx[t, s]
+            g64 = x[t] @ wg[e]                       # exact integer dot products
+            u64 = x[t] @ wu[e]
+            assert np.array_equal(dbg["acc1"][t, s, :f], g64)
+            assert np.array_equal(dbg["acc1"][t, s, f:], u64)
+            # SwiGLU in fp64 from the exact integers (|acc| < 2^24: the fp32 casts are exact)
+            g = g64.astype(np.float64)
+            with np.errstate(over="ignore"):
+                h64 = g / (1.0 + np.exp(-g)) * u64
+            sh = float(dbg["sh"][t, s])
+            assert abs(sh - np.abs(h64).max() / 127.0) <= 4e-7 * sh
+            q64 = h64 / sh
+            hq = dbg["hq"][t, s].astype(np.int64)
+            near_half = np.abs(np.abs(q64 - np.floor(q64)) - 0.5) < 1e-4
+            assert np.all((hq == np.clip(np.rint(q64), -127, 127)) | near_half)
+            assert np.abs(hq - q64).max() <= 0.5 + 1e-4
+            acc2 = hq @ wd[e]
+            assert np.array_equal(dbg["acc2"][t, s], acc2)
+            o = acc2.astype(np.float64) * sh * float(rt.w[t, s])
+            assert np.allclose(dbg["o"][t, s], o, rtol=4 * U32, atol=0)
+        o_sum = dbg["o"][t].astype(np.float64).sum(0)
+        assert np.allclose(y[t], o_sum, rtol=1e-6, atol=1e-6 * np.abs(o_sum).max())
+
+
+def test_dense_special_case_e1_k1():
+    """E = 1, k = 1 is a dense W8A8 SwiGLU FFN: routing weight exactly 1, every
+    token on expert 0, output = FFN(x) up to W8A8 noise."""
+    T, d, f = 16, 128, 64
+    x = synth.normal(21, 1, (T, d))
+    wg = synth.normal(21, 2, (1, d, f), std=0.2)
+    wu = synth.normal(21, 3, (1, d, f), std=0.2)
+    wd = synth.normal(21, 4, (1, f, d), std=0.2)
+    prep = oracle.prepare(wg, wu, wd, x, 0.5)
+    rt = oracle.route(x, 1, 1, logits=np.zeros((T, 1), np.float32))
+    assert np.all(rt.w == 1.0) and np.all(rt.idx == 0)
+    y, _ = oracle.moe_tokens(x, prep, rt)
+    x64 = x.astype(np.float64)
+    g = x64 @ wg[0].astype(np.float64)
+    u = x64 @ wu[0].astype(np.float64)
+    ref = (g / (1 + np.exp(-g)) * u) @ wd[0].astype(np.float64)
+    rel = np.abs(y - ref).max() / np.abs(ref).max()
+    assert rel < 3e-2, rel
+
+
+def test_moe_vs_unquantised_fp64_sanity():
+    """Tiny config: the W8A8 layer tracks the unquantised fp64 MoE with the same
+    routing to within W8A8 noise (normwise ~1e-2)."""
+    w = synth.WORKLOADS["tiny"]
+    wts = synth.make_weights(w)
+    data = synth.make_data(w)
+    prep = oracle.prepare(wts.w_gate, wts.w_up, wts.w_down, wts.calib_x, w.alpha)
+    rt = oracle.route(data.x, w.k, w.E, w_router=data.w_router)
+    y, _ = oracle.moe_tokens(data.x, prep, rt)
+    x64 = data.x.astype(np.float64)
+    ref = np.zeros_like(x64)
+    for t in range(w.T):
+        for s in range(w.k):
+            e = rt.idx[t, s]
+            g = x64[t] @ wts.w_gate[e].astype(np.float64)
+            u = x64[t] @ wts.w_up[e].astype(np.float64)
+            ref[t] += rt.w[t, s] * ((g / (1 + np.exp(-g)) * u) @ wts.w_down[e].astype(np.float64))
+    rel = np.linalg.norm(y - ref) / np.linalg.norm(ref)
+    assert rel < 5e-2, rel
