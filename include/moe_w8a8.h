@@ -1,0 +1,204 @@
+/*
+ * moe_w8a8 -- C ABI of the B200 (sm_100a) W8A8 mixture-of-experts FFN layer.
+ *
+ * The layer (one MoE FFN block):
+ *   gate:    logits l = X W_router (+ bias), top-k experts per token with the
+ *            lowest index winning ties, softmax over the k selected logits.
+ *   sort:    the (token, slot) pairs grouped by expert in token order, an
+ *            optional per-expert capacity dropping late arrivals.
+ *   quant:   X smoothed by 1/s (SmoothQuant) and quantised to INT8 per token.
+ *   experts: for each expert, INT8 x INT8 -> INT32 grouped GEMMs against
+ *            per-output-channel INT8 weights; gate/up dequantised, SwiGLU,
+ *            h requantised to INT8 per row; down dequantised and scaled by
+ *            the routing weight.
+ *   combine: the k expert outputs of each token summed in slot order.
+ * Sources, by page title and section:
+ *   "MiniMax-M3 W8A8 on K100AI" (mhpq.cn, MetaInfer practice notes):
+ *     s1.2 W8A8 = INT8 weights x INT8 activations on the INT8 GEMM path with
+ *     integer accumulation and dequantisation back to FP16/BF16; s3.2 quant
+ *     config (8-bit weights per output channel, 8-bit activations per token,
+ *     SmoothQuant with alpha 0.6); s4.3 keep consecutive matmuls in the INT8
+ *     domain, fuse the expert FFN, pool device memory; s6.1/s6.4 smoothing
+ *     and per-token quantisation against activation outliers.
+ *   "Day0 adaptation of ultra-large model inference" (ruibaoantu.com),
+ *     section 4, MoE operator fusion: gate, sort, grouped GEMM, un-sort and
+ *     weighted sum in few kernels; top-k must equal the reference including
+ *     its tie-break rule; section 2 item 2: capacity factor, dropped tokens.
+ *
+ * Conventions for every call:
+ *   - Pointers marked "device" are CUDA device pointers on the current
+ *     device; "host" pointers are ordinary host memory.  The caller owns
+ *     every buffer it passes; the library owns the prepared-weights handle
+ *     until moe_w8a8_destroy.
+ *   - Work is enqueued on the given stream and is asynchronous; no call
+ *     synchronises the stream except moe_w8a8_prepare (which needs the
+ *     smoothing statistics on the host) and moe_w8a8_check_status.
+ *   - Arguments are validated before anything is enqueued; on an error the
+ *     call returns a status and enqueues nothing.  No call throws or exits.
+ *   - Shapes: d and f multiples of 128, 1 <= top_k <= min(8, n_experts),
+ *     n_experts <= 256, T >= 0 (T = 0 is a no-op).  Other shapes return
+ *     MOE_ERR_UNSUPPORTED_SHAPE.
+ */
+#ifndef MOE_W8A8_H
+#define MOE_W8A8_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* moe_stream_t; /* same object as cudaStream_t; NULL = legacy stream */
+
+typedef enum {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARG = 1,          /* null pointer, bad enum, alpha outside [0, 1] ...      */
+    MOE_ERR_UNSUPPORTED_SHAPE = 2,    /* see the shape rules above                             */
+    MOE_ERR_WORKSPACE_TOO_SMALL = 3,  /* workspace_bytes < moe_w8a8_workspace_size(w, T)       */
+    MOE_ERR_CUDA = 4,                 /* a CUDA runtime call failed                            */
+    MOE_ERR_TIMEOUT = 5,              /* a bounded device-side wait ran out (status word)      */
+    MOE_ERR_OOM = 6                   /* device allocation in moe_w8a8_prepare failed          */
+} moe_status;
+
+enum { MOE_F32 = 0, MOE_BF16 = 1 };
+
+/* Expert GEMM path: AUTO picks STREAM for small row counts (weight-bandwidth
+ * bound: each active expert's INT8 weights are read once with 128-bit loads)
+ * and TENSOR otherwise (tcgen05 kind::i8 grouped GEMMs). */
+enum { MOE_PATH_AUTO = 0, MOE_PATH_STREAM = 1, MOE_PATH_TENSOR = 2 };
+
+typedef struct {
+    int32_t d;                /* hidden size                                                  */
+    int32_t f;                /* expert FFN intermediate size                                 */
+    int32_t n_experts;        /* E                                                            */
+    int32_t top_k;            /* k                                                            */
+    float alpha;              /* SmoothQuant migration strength, in [0, 1] (pages use 0.6)     */
+    float capacity_factor;    /* <= 0: no capacity; else C = ceil(cf * T * k / E) per expert  */
+    int32_t renormalize;      /* 1: softmax over the k selected logits; 0: over all E          */
+    int32_t in_dtype;         /* MOE_F32 or MOE_BF16: X                                       */
+    int32_t out_dtype;        /* MOE_F32 or MOE_BF16: Y                                       */
+} moe_w8a8_config;
+
+typedef struct moe_w8a8_weights moe_w8a8_weights; /* opaque, library-owned */
+
+/* Optional intermediates for parity checks (device pointers, each may be NULL).
+ * R = number of kept (token, slot) rows, at most T*k.  Rows are ordered by
+ * expert, then token.  Channel order is canonical: acc1 holds gate channels
+ * 0..f-1 then up channels 0..f-1. */
+typedef struct {
+    float* logits;       /* [T][E]  router logits incl. bias                          */
+    int32_t* topk_idx;   /* [T][k]                                                    */
+    float* topk_w;       /* [T][k]                                                    */
+    int32_t* offsets;    /* [E+1]   first row of each expert; offsets[E] = R          */
+    int32_t* row2ts;     /* [T*k]   row -> t*k + slot (first R entries valid)          */
+    int32_t* ts2row;     /* [T*k]   (t, slot) -> row, -1 when dropped by capacity      */
+    int8_t* xq;          /* [T][d]  INT8 smoothed activations                          */
+    float* sx;           /* [T]     per-token activation scales                        */
+    int32_t* acc1;       /* [T*k][2f] gate|up INT32 accumulators (first R rows)        */
+    int8_t* hq;          /* [T*k][f]  INT8 h                                           */
+    float* sh;           /* [T*k]     per-row h scales                                 */
+    int32_t* acc2;       /* [T*k][d]  down-projection INT32 accumulators               */
+    float* o;            /* [T*k][d]  weighted expert outputs, fp32                    */
+} moe_w8a8_debug;
+
+/*
+ * Calibration statistic for SmoothQuant (mhpq.cn page s3.2: calibration
+ * samples -> per-channel activation range): absmax[j] = max(absmax[j],
+ * max_r |x[r][j]|) over `rows` activation rows x [rows][d] (device, dtype
+ * MOE_F32 or MOE_BF16).  absmax [d] (device, fp32) is updated in place, so
+ * the calibration set may come in several batches; start it at zero.
+ */
+moe_status moe_w8a8_calibrate_absmax(const void* x, int64_t rows, int32_t d, int32_t dtype,
+                                     float* absmax, moe_stream_t stream);
+
+/*
+ * Fold SmoothQuant into the expert weights and quantise them (mhpq.cn page
+ * s3.2, s6.1; formula s_j = max|X_j|^alpha / max|W_j|^(1-alpha)).
+ *   w_gate, w_up  device fp32 [E][d][f]   (gate = x W_gate[e])
+ *   w_down        device fp32 [E][f][d]
+ *   w_router      device fp32 [d][E]      (copied; used unquantised)
+ *   act_absmax    device fp32 [d]         (from moe_w8a8_calibrate_absmax)
+ * max|W_j| is taken over the gate and up weights of every expert.  Gate and
+ * up weights are smoothed and quantised per output channel; down weights
+ * per output channel without smoothing.  The inputs may be freed afterwards.
+ * Synchronises `stream` once (the O(d) scale computation runs on the host
+ * in fp64).  Allocates the handle's device memory (3 d f E bytes of INT8
+ * weights plus scales); returns MOE_ERR_OOM if that fails.
+ */
+moe_status moe_w8a8_prepare(const moe_w8a8_config* cfg, const float* w_gate, const float* w_up,
+                            const float* w_down, const float* w_router, const float* act_absmax,
+                            moe_stream_t stream, moe_w8a8_weights** out);
+
+/* Bytes of device workspace moe_w8a8_forward needs for up to max_tokens
+ * tokens (0 on a NULL handle or negative max_tokens). */
+size_t moe_w8a8_workspace_size(const moe_w8a8_weights* w, int32_t max_tokens);
+
+/*
+ * Run the layer on T tokens.
+ *   x              device [T][d], cfg.in_dtype
+ *   router_bias    device fp32 [E] added to every token's logits, or NULL
+ *   router_logits  device fp32 [T][E] used instead of X W_router, or NULL
+ *   y              device [T][d], cfg.out_dtype
+ *   workspace      device, >= moe_w8a8_workspace_size(w, T) bytes, 256-byte aligned
+ *   dbg            NULL, or device pointers receiving intermediates
+ * Allocates nothing; all scratch lives in the caller's workspace.  Calls
+ * that share a workspace must not overlap on the device.
+ */
+moe_status moe_w8a8_forward(const moe_w8a8_weights* w, const void* x, int32_t T,
+                            const float* router_bias, const float* router_logits, void* y,
+                            void* workspace, size_t workspace_bytes, const moe_w8a8_debug* dbg,
+                            moe_stream_t stream);
+
+/*
+ * moe_w8a8_forward from host memory: copies x (and router_logits /
+ * router_bias when given) host -> device into the workspace, runs the
+ * layer, and copies y device -> host, all enqueued on `stream`.  Host
+ * buffers should be page-locked for the copies to be asynchronous; y is
+ * valid once the stream has been synchronised.
+ */
+moe_status moe_w8a8_forward_host(const moe_w8a8_weights* w, const void* x_host, int32_t T,
+                                 const float* router_bias_host, const float* router_logits_host,
+                                 void* y_host, void* workspace, size_t workspace_bytes,
+                                 moe_stream_t stream);
+
+/* Select the expert GEMM path (MOE_PATH_*). */
+moe_status moe_w8a8_set_path(moe_w8a8_weights* w, int32_t path);
+
+/* Row count at or below which MOE_PATH_AUTO uses the streaming path. */
+moe_status moe_w8a8_set_stream_threshold(moe_w8a8_weights* w, int32_t max_rows);
+
+/* Smoothing scales s [d] copied to host memory. */
+moe_status moe_w8a8_get_smooth_scales(const moe_w8a8_weights* w, float* s_host);
+
+/*
+ * Copy the prepared weights out in canonical layout (device pointers, each
+ * may be NULL): wq_gate, wq_up INT8 [E][f][d]; sw_gate, sw_up fp32 [E][f];
+ * wq_down INT8 [E][d][f]; sw_down fp32 [E][d]; inv_s fp32 [d].
+ */
+moe_status moe_w8a8_export_weights(const moe_w8a8_weights* w, int8_t* wq_gate, int8_t* wq_up,
+                                   float* sw_gate, float* sw_up, int8_t* wq_down, float* sw_down,
+                                   float* inv_s, moe_stream_t stream);
+
+/*
+ * Synchronise `stream` and read the handle's device status word: MOE_OK,
+ * or MOE_ERR_TIMEOUT when a bounded wait in a kernel ran out since the last
+ * check (the word is then cleared), or MOE_ERR_CUDA on a pending CUDA error.
+ */
+moe_status moe_w8a8_check_status(const moe_w8a8_weights* w, moe_stream_t stream);
+
+/* Free the handle and its device memory (NULL is a no-op).  The caller makes
+ * sure no enqueued forward still uses it. */
+void moe_w8a8_destroy(moe_w8a8_weights* w);
+
+/* Static description of a status code. */
+const char* moe_status_string(moe_status s);
+
+/* Number of kernels the last successful forward on this handle enqueued. */
+int32_t moe_w8a8_last_launch_count(const moe_w8a8_weights* w);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_W8A8_H */

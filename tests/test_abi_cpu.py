@@ -1,0 +1,93 @@
+"""The C-ABI library without a GPU: it builds, loads, exports every entry
+point the public header declares, and its host-side argument checks return
+the documented statuses before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "moe_w8a8.h")
+
+
+@pytest.fixture(scope="module")
+def M():
+    from w8a8_quantized_moe_b200 import build
+    build.build()
+    import w8a8_quantized_moe_b200 as mod
+    return mod
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*[A-Za-z_][\w\s\*]*?\b(moe_\w+)\s*\(", text, flags=re.M)))
+
+
+def test_header_declares_the_binding_exports(M):
+    assert declared_functions() == sorted(M.EXPORTS)
+
+
+def test_every_declared_symbol_is_exported(M):
+    lib = M.lib()
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+    nm = os.popen(f"nm -D --defined-only {M.LIB_PATH}").read()
+    for name in declared_functions():
+        assert re.search(rf"\bT {name}\b", nm), name
+
+
+def test_status_strings(M):
+    assert M.moe_status_string(M.MOE_OK) == "ok"
+    assert M.moe_status_string(M.MOE_ERR_WORKSPACE_TOO_SMALL) == "workspace too small"
+    assert M.moe_status_string(99) == "unknown status"
+
+
+def test_host_side_argument_checks(M):
+    L = M.lib()
+    out = ctypes.c_void_p()
+    cfg = M.make_config(4096, 1536, 64, 4)
+    z = ctypes.c_void_p(16)   # never dereferenced: the checks fail first
+    # null config / null output handle / bad enum / bad alpha / bad shapes
+    assert L.moe_w8a8_prepare(None, z, z, z, z, z, None, ctypes.byref(out)) == M.MOE_ERR_INVALID_ARG
+    assert L.moe_w8a8_prepare(ctypes.byref(cfg), z, z, z, z, z, None, None) == M.MOE_ERR_INVALID_ARG
+    for field, value, status in [("alpha", -0.1, M.MOE_ERR_INVALID_ARG),
+                                 ("alpha", 1.5, M.MOE_ERR_INVALID_ARG),
+                                 ("in_dtype", 7, M.MOE_ERR_INVALID_ARG),
+                                 ("renormalize", 2, M.MOE_ERR_INVALID_ARG),
+                                 ("d", 4000, M.MOE_ERR_UNSUPPORTED_SHAPE),
+                                 ("f", 100, M.MOE_ERR_UNSUPPORTED_SHAPE),
+                                 ("n_experts", 300, M.MOE_ERR_UNSUPPORTED_SHAPE),
+                                 ("top_k", 9, M.MOE_ERR_UNSUPPORTED_SHAPE),
+                                 ("top_k", 0, M.MOE_ERR_UNSUPPORTED_SHAPE)]:
+        c = M.make_config(4096, 1536, 64, 4)
+        setattr(c, field, value)
+        assert L.moe_w8a8_prepare(ctypes.byref(c), z, z, z, z, z, None, ctypes.byref(out)) == status, field
+    c = M.make_config(256, 512, 4, 8)   # k > E
+    assert L.moe_w8a8_prepare(ctypes.byref(c), z, z, z, z, z, None, ctypes.byref(out)) == \
+        M.MOE_ERR_UNSUPPORTED_SHAPE
+    # missing weight pointers
+    assert L.moe_w8a8_prepare(ctypes.byref(cfg), None, z, z, z, z, None, ctypes.byref(out)) == \
+        M.MOE_ERR_INVALID_ARG
+    # handle-less calls
+    assert L.moe_w8a8_workspace_size(None, 32) == 0
+    assert L.moe_w8a8_forward(None, z, 32, None, None, z, z, 1 << 20, None, None) == M.MOE_ERR_INVALID_ARG
+    assert L.moe_w8a8_forward_host(None, z, 32, None, None, z, z, 1 << 20, None) == M.MOE_ERR_INVALID_ARG
+    assert L.moe_w8a8_set_path(None, 1) == M.MOE_ERR_INVALID_ARG
+    assert L.moe_w8a8_get_smooth_scales(None, z) == M.MOE_ERR_INVALID_ARG
+    assert L.moe_w8a8_check_status(None, None) == M.MOE_ERR_INVALID_ARG
+    assert L.moe_w8a8_calibrate_absmax(z, 4, 16, 5, z, None) == M.MOE_ERR_INVALID_ARG
+    assert L.moe_w8a8_calibrate_absmax(z, -1, 16, 0, z, None) == M.MOE_ERR_INVALID_ARG
+    assert L.moe_w8a8_last_launch_count(None) == 0
+    L.moe_w8a8_destroy(None)
+
+
+def test_product_path_does_not_touch_the_oracle():
+    """The library sources and the binding never name the oracle."""
+    pkg = os.path.join(ROOT, "w8a8_quantized_moe_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for fn in files:
+            if fn.endswith((".py", ".cu", ".cuh", ".h")):
+                text = open(os.path.join(dirpath, fn)).read()
+                assert "oracle" not in text.lower(), fn

@@ -1,0 +1,182 @@
+"""GPU parity: the CUDA library (through the C ABI) against the CPU oracle on
+the same seeded inputs.  Integer stages and the fixed-order float stages must
+match bit for bit; the output within the stated tolerance."""
+import dataclasses
+
+import numpy as np
+import pytest
+
+import oracle
+import synth
+from tests import harness as H
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def M():
+    from w8a8_quantized_moe_b200 import build
+    build.build()
+    import w8a8_quantized_moe_b200 as mod
+    return mod
+
+
+def run_case(M, wl, wts=None, data=None, tokens=None, path=None, W=None, prep=None):
+    wts = synth.make_weights(wl) if wts is None else wts
+    data = synth.make_data(wl) if data is None else data
+    if prep is None:
+        prep = H.oracle_prepare(wl, wts)
+    if W is None:
+        W = H.gpu_prepare(wl, wts)
+        H.compare_prepare(W, prep)
+    rt = H.oracle_route(wl, data)
+    y, dbg = H.gpu_forward(W, wl, data, path=path)
+    T = data.x.shape[0]
+    toks = np.arange(T) if tokens is None else np.asarray(tokens)
+    y_ref, odbg = oracle.moe_tokens(data.x, prep, rt, tokens=toks, out_bf16=wl.in_bf16)
+    err = H.compare_stages(wl, rt, dbg, y, y_ref, odbg, toks, bias=data.router_bias)
+    return err, y, y_ref, rt, dbg
+
+
+def test_tiny_layer_all_stages(M):
+    wl = synth.WORKLOADS["tiny"]
+    err, y, y_ref, _, _ = run_case(M, wl, path=M.MOE_PATH_STREAM)
+    assert np.array_equal(y, y_ref)   # the stated fp32 chain is reproduced bit for bit
+
+
+@pytest.fixture(scope="module")
+def decode_setup(M):
+    wl = synth.WORKLOADS["decode"]
+    wts = synth.make_weights(wl)
+    prep = H.oracle_prepare(wl, wts)
+    W = H.gpu_prepare(wl, wts)
+    return wl, wts, prep, W
+
+
+def test_decode_prepare_bit_exact(M, decode_setup):
+    wl, wts, prep, W = decode_setup
+    H.compare_prepare(W, prep)
+
+
+def test_decode_layer_all_stages(M, decode_setup):
+    wl, wts, prep, W = decode_setup
+    err, y, y_ref, rt, _ = run_case(M, wl, wts=wts, W=W, prep=prep)
+    assert np.array_equal(y, y_ref)
+    assert len(np.unique(rt.idx)) > 40    # most experts active, as in a decode step
+
+
+@pytest.mark.parametrize("T", [1, 37, 200])
+def test_ragged_token_counts(M, T):
+    wl = dataclasses.replace(synth.WORKLOADS["tiny"], T=T, data_seed=100 + T)
+    err, y, y_ref, _, _ = run_case(M, wl, path=M.MOE_PATH_STREAM)
+    assert np.array_equal(y, y_ref)
+
+
+def _tiny_with_logits(T, logits, seed=5, **kw):
+    wl = dataclasses.replace(synth.WORKLOADS["tiny"], T=T, data_seed=seed, **kw)
+    data = synth.make_data(wl)
+    data.router_logits = np.ascontiguousarray(logits, dtype=np.float32)
+    return wl, data
+
+
+def test_all_tokens_on_one_expert_and_empty_experts(M):
+    T, E = 50, 8
+    logits = np.zeros((T, E), np.float32)
+    logits[:, 3] = 5.0
+    logits[:, 6] = 4.0
+    wl, data = _tiny_with_logits(T, logits)
+    _, _, _, rt, dbg = run_case(M, wl, data=data, path=M.MOE_PATH_STREAM)
+    counts = np.diff(rt.offsets)
+    assert counts[3] == T and counts[6] == T and counts.sum() == 2 * T
+
+
+def test_exact_ties_resolve_to_lowest_index(M):
+    T, E = 40, 8
+    logits = np.zeros((T, E), np.float32)
+    logits[::2, [1, 4, 7]] = 2.0      # three-way tie for the top-2
+    logits[1::2, :] = 1.0             # all equal
+    wl, data = _tiny_with_logits(T, logits)
+    _, _, _, rt, dbg = run_case(M, wl, data=data, path=M.MOE_PATH_STREAM)
+    assert dbg["topk_idx"][0].tolist() == [1, 4]
+    assert dbg["topk_idx"][1].tolist() == [0, 1]
+
+
+def test_zero_token_rows(M):
+    wl = dataclasses.replace(synth.WORKLOADS["tiny"], T=16, data_seed=9)
+    data = synth.make_data(wl)
+    data.x[3] = 0.0
+    data.x[7] = 0.0
+    err, y, y_ref, _, dbg = run_case(M, wl, data=data, path=M.MOE_PATH_STREAM)
+    assert dbg["sx"][3] == 0.0 and not dbg["xq"][3].any()
+    assert np.array_equal(y, y_ref)
+
+
+def test_capacity_drops_overflow_in_token_order(M):
+    T, E = 120, 8
+    rng = synth.uniform(31, 1, (T, E))
+    logits = rng.copy()
+    logits[:, 2] += 1.0                # expert 2 very popular
+    wl, data = _tiny_with_logits(T, logits, capacity_factor=1.25)
+    _, _, _, rt, dbg = run_case(M, wl, data=data, path=M.MOE_PATH_STREAM)
+    cap = oracle.capacity(1.25, T, wl.k, E)
+    assert np.diff(rt.offsets).max() == cap
+    assert (rt.ts2row < 0).sum() > 0
+
+
+def test_zipf_bias_and_no_renormalise_paths_match(M):
+    wl = dataclasses.replace(synth.WORKLOADS["tiny"], T=48, data_seed=12, zipf_s=1.1)
+    run_case(M, wl, path=M.MOE_PATH_STREAM)
+
+
+def test_run_to_run_determinism(M, decode_setup):
+    wl, wts, prep, W = decode_setup
+    data = synth.make_data(wl)
+    y1, d1 = H.gpu_forward(W, wl, data)
+    y2, d2 = H.gpu_forward(W, wl, data)
+    assert np.array_equal(y1, y2)
+    for k in d1:
+        assert np.array_equal(d1[k], d2[k]), k
+
+
+def test_forward_host_matches_device_forward(M, decode_setup):
+    import torch
+    wl, wts, prep, W = decode_setup
+    data = synth.make_data(wl)
+    y_dev, _ = H.gpu_forward(W, wl, data, debug=False)
+    T = wl.T
+    ws = torch.empty(M.moe_w8a8_workspace_size(W, T), dtype=torch.uint8, device="cuda")
+    x_host = torch.from_numpy(data.x_bits.view(np.int16)).pin_memory()
+    lg_host = torch.from_numpy(data.router_logits).pin_memory()
+    y_host = torch.empty((T, wl.d), dtype=torch.int16).pin_memory()
+    M.moe_w8a8_forward_host(W, x_host, T, None, lg_host, y_host, ws)
+    torch.cuda.synchronize()
+    y = (y_host.numpy().view(np.uint16).astype(np.uint32) << 16).view(np.float32)
+    assert np.array_equal(y, y_dev)
+
+
+def test_error_statuses(M, decode_setup):
+    import torch
+    wl, wts, prep, W = decode_setup
+    data = synth.make_data(wl)
+    x = H.x_tensor(wl, data)
+    y = torch.empty((wl.T, wl.d), dtype=torch.bfloat16, device="cuda")
+    need = M.moe_w8a8_workspace_size(W, wl.T)
+    small = torch.empty(need - 256, dtype=torch.uint8, device="cuda")
+    with pytest.raises(M.MoeError) as e:
+        M.moe_w8a8_forward(W, x, wl.T, None, H.to_dev(data.router_logits), y, small)
+    assert e.value.status == M.MOE_ERR_WORKSPACE_TOO_SMALL
+    ws = torch.empty(need, dtype=torch.uint8, device="cuda")
+    with pytest.raises(M.MoeError) as e:
+        M.moe_w8a8_forward(W, x, -1, None, None, y, ws)
+    assert e.value.status == M.MOE_ERR_INVALID_ARG
+    M.moe_w8a8_forward(W, x, 0, None, None, y, ws)          # T = 0 is a no-op
+    bad = M.make_config(wl.d, 100, wl.E, wl.k)
+    z = torch.zeros(1, device="cuda")
+    with pytest.raises(M.MoeError) as e:
+        M.moe_w8a8_prepare(bad, z, z, z, z, z)
+    assert e.value.status == M.MOE_ERR_UNSUPPORTED_SHAPE
+    bad = M.make_config(wl.d, wl.f, wl.E, wl.k, alpha=1.5)
+    with pytest.raises(M.MoeError) as e:
+        M.moe_w8a8_prepare(bad, z, z, z, z, z)
+    assert e.value.status == M.MOE_ERR_INVALID_ARG
+    M.moe_w8a8_check_status(W)

@@ -1,0 +1,282 @@
+"""Python binding of ``libmoe_w8a8.so``, the B200 W8A8 mixture-of-experts layer.
+
+Argument marshalling only: every function here has the name of the C entry
+point it calls (see ``include/moe_w8a8.h``), turns tensors into pointers,
+checks their dtype / device / contiguity, and raises ``MoeError`` on a
+non-OK status.  All of the layer's work runs in the library's CUDA kernels;
+there is no fallback, and importing a missing library fails loudly.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmoe_w8a8.so")
+
+MOE_OK = 0
+MOE_ERR_INVALID_ARG = 1
+MOE_ERR_UNSUPPORTED_SHAPE = 2
+MOE_ERR_WORKSPACE_TOO_SMALL = 3
+MOE_ERR_CUDA = 4
+MOE_ERR_TIMEOUT = 5
+MOE_ERR_OOM = 6
+
+MOE_F32 = 0
+MOE_BF16 = 1
+
+MOE_PATH_AUTO = 0
+MOE_PATH_STREAM = 1
+MOE_PATH_TENSOR = 2
+
+# Every entry point declared in include/moe_w8a8.h.
+EXPORTS = (
+    "moe_w8a8_calibrate_absmax", "moe_w8a8_prepare", "moe_w8a8_workspace_size",
+    "moe_w8a8_forward", "moe_w8a8_forward_host", "moe_w8a8_set_path",
+    "moe_w8a8_set_stream_threshold", "moe_w8a8_get_smooth_scales", "moe_w8a8_export_weights",
+    "moe_w8a8_check_status", "moe_w8a8_destroy", "moe_status_string",
+    "moe_w8a8_last_launch_count",
+)
+
+
+class MoeError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {moe_status_string(status)} (status {status})")
+
+
+class moe_w8a8_config(ctypes.Structure):
+    _fields_ = [("d", ctypes.c_int32), ("f", ctypes.c_int32), ("n_experts", ctypes.c_int32),
+                ("top_k", ctypes.c_int32), ("alpha", ctypes.c_float),
+                ("capacity_factor", ctypes.c_float), ("renormalize", ctypes.c_int32),
+                ("in_dtype", ctypes.c_int32), ("out_dtype", ctypes.c_int32)]
+
+
+_DBG_FIELDS = ("logits", "topk_idx", "topk_w", "offsets", "row2ts", "ts2row", "xq", "sx", "acc1",
+               "hq", "sh", "acc2", "o")
+
+
+class moe_w8a8_debug(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in _DBG_FIELDS]
+
+
+_lib = None
+
+
+def lib():
+    """Load the library (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: build it with "
+                              "`python -m w8a8_quantized_moe_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i32, i64, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
+        cfgp = ctypes.POINTER(moe_w8a8_config)
+        sig = {
+            "moe_w8a8_calibrate_absmax": ([vp, i64, i32, i32, vp, vp], i32),
+            "moe_w8a8_prepare": ([cfgp, vp, vp, vp, vp, vp, vp, ctypes.POINTER(vp)], i32),
+            "moe_w8a8_workspace_size": ([vp, i32], sz),
+            "moe_w8a8_forward": ([vp, vp, i32, vp, vp, vp, vp, sz, vp, vp], i32),
+            "moe_w8a8_forward_host": ([vp, vp, i32, vp, vp, vp, vp, sz, vp], i32),
+            "moe_w8a8_set_path": ([vp, i32], i32),
+            "moe_w8a8_set_stream_threshold": ([vp, i32], i32),
+            "moe_w8a8_get_smooth_scales": ([vp, vp], i32),
+            "moe_w8a8_export_weights": ([vp, vp, vp, vp, vp, vp, vp, vp, vp], i32),
+            "moe_w8a8_check_status": ([vp, vp], i32),
+            "moe_w8a8_destroy": ([vp], None),
+            "moe_status_string": ([i32], ctypes.c_char_p),
+            "moe_w8a8_last_launch_count": ([vp], i32),
+        }
+        for name, (args, res) in sig.items():
+            fn = getattr(L, name)
+            fn.argtypes = args
+            fn.restype = res
+        _lib = L
+    return _lib
+
+
+# ------------------------------------------------------------------ marshalling helpers
+
+def _torch():
+    import torch
+    return torch
+
+
+def _dev_ptr(t, dtype=None, name="tensor", allow_none=False):
+    if t is None:
+        if allow_none:
+            return None
+        raise ValueError(f"{name} is required")
+    torch = _torch()
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _host_ptr(a, name="array", allow_none=False):
+    if a is None:
+        if allow_none:
+            return None
+        raise ValueError(f"{name} is required")
+    try:
+        import numpy as np
+        if isinstance(a, np.ndarray):
+            if not a.flags["C_CONTIGUOUS"]:
+                raise ValueError(f"{name} must be C-contiguous")
+            return ctypes.c_void_p(a.ctypes.data)
+    except ImportError:  # pragma: no cover
+        pass
+    torch = _torch()
+    if isinstance(a, torch.Tensor) and not a.is_cuda and a.is_contiguous():
+        return ctypes.c_void_p(a.data_ptr())
+    raise TypeError(f"{name} must be a contiguous host array")
+
+
+def _stream(stream):
+    if stream is None:
+        torch = _torch()
+        return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    if isinstance(stream, int):
+        return ctypes.c_void_p(stream)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _check(status: int, where: str):
+    if status != MOE_OK:
+        raise MoeError(status, where)
+
+
+def _act_dtype(code: int):
+    torch = _torch()
+    return torch.bfloat16 if code == MOE_BF16 else torch.float32
+
+
+# ------------------------------------------------------------------ entry points
+
+def moe_status_string(status: int) -> str:
+    return lib().moe_status_string(int(status)).decode()
+
+
+def moe_w8a8_calibrate_absmax(x, absmax, stream=None):
+    torch = _torch()
+    dt = MOE_BF16 if x.dtype == torch.bfloat16 else MOE_F32
+    _check(lib().moe_w8a8_calibrate_absmax(_dev_ptr(x, name="x"), x.shape[0], x.shape[1], dt,
+                                           _dev_ptr(absmax, torch.float32, "absmax"),
+                                           _stream(stream)), "moe_w8a8_calibrate_absmax")
+
+
+class Weights:
+    """Owner of a prepared-weights handle (destroyed with the object)."""
+
+    def __init__(self, handle: ctypes.c_void_p, cfg: moe_w8a8_config):
+        self.handle = handle
+        self.cfg = cfg
+
+    def __del__(self):
+        if getattr(self, "handle", None) and _lib is not None:
+            _lib.moe_w8a8_destroy(self.handle)
+            self.handle = None
+
+
+def make_config(d, f, n_experts, top_k, alpha=0.6, capacity_factor=0.0, renormalize=True,
+                in_dtype=MOE_BF16, out_dtype=MOE_BF16) -> moe_w8a8_config:
+    return moe_w8a8_config(d, f, n_experts, top_k, alpha, capacity_factor, 1 if renormalize else 0,
+                           in_dtype, out_dtype)
+
+
+def moe_w8a8_prepare(cfg: moe_w8a8_config, w_gate, w_up, w_down, w_router, act_absmax,
+                     stream=None) -> Weights:
+    torch = _torch()
+    f32 = torch.float32
+    h = ctypes.c_void_p()
+    _check(lib().moe_w8a8_prepare(ctypes.byref(cfg), _dev_ptr(w_gate, f32, "w_gate"),
+                                  _dev_ptr(w_up, f32, "w_up"), _dev_ptr(w_down, f32, "w_down"),
+                                  _dev_ptr(w_router, f32, "w_router"),
+                                  _dev_ptr(act_absmax, f32, "act_absmax"), _stream(stream),
+                                  ctypes.byref(h)), "moe_w8a8_prepare")
+    return Weights(h, cfg)
+
+
+def moe_w8a8_workspace_size(w: Weights, max_tokens: int) -> int:
+    return int(lib().moe_w8a8_workspace_size(w.handle, int(max_tokens)))
+
+
+def _debug_struct(dbg: dict | None):
+    if not dbg:
+        return None, None
+    s = moe_w8a8_debug()
+    for n in _DBG_FIELDS:
+        t = dbg.get(n)
+        setattr(s, n, None if t is None else _dev_ptr(t, name=f"dbg.{n}").value)
+    return s, ctypes.byref(s)
+
+
+def moe_w8a8_forward(w: Weights, x, T: int, router_bias, router_logits, y, workspace,
+                     dbg: dict | None = None, stream=None):
+    torch = _torch()
+    _s, dptr = _debug_struct(dbg)
+    _check(lib().moe_w8a8_forward(
+        w.handle, _dev_ptr(x, _act_dtype(w.cfg.in_dtype), "x"), int(T),
+        _dev_ptr(router_bias, torch.float32, "router_bias", True),
+        _dev_ptr(router_logits, torch.float32, "router_logits", True),
+        _dev_ptr(y, _act_dtype(w.cfg.out_dtype), "y"), _dev_ptr(workspace, name="workspace"),
+        workspace.numel() * workspace.element_size(), dptr, _stream(stream)), "moe_w8a8_forward")
+
+
+def moe_w8a8_forward_host(w: Weights, x_host, T: int, router_bias_host, router_logits_host,
+                          y_host, workspace, stream=None):
+    _check(lib().moe_w8a8_forward_host(
+        w.handle, _host_ptr(x_host, "x_host"), int(T),
+        _host_ptr(router_bias_host, "router_bias_host", True),
+        _host_ptr(router_logits_host, "router_logits_host", True), _host_ptr(y_host, "y_host"),
+        _dev_ptr(workspace, name="workspace"), workspace.numel() * workspace.element_size(),
+        _stream(stream)), "moe_w8a8_forward_host")
+
+
+def moe_w8a8_set_path(w: Weights, path: int):
+    _check(lib().moe_w8a8_set_path(w.handle, int(path)), "moe_w8a8_set_path")
+
+
+def moe_w8a8_set_stream_threshold(w: Weights, max_rows: int):
+    _check(lib().moe_w8a8_set_stream_threshold(w.handle, int(max_rows)),
+           "moe_w8a8_set_stream_threshold")
+
+
+def moe_w8a8_get_smooth_scales(w: Weights):
+    import numpy as np
+    out = np.empty(w.cfg.d, dtype=np.float32)
+    _check(lib().moe_w8a8_get_smooth_scales(w.handle, ctypes.c_void_p(out.ctypes.data)),
+           "moe_w8a8_get_smooth_scales")
+    return out
+
+
+def moe_w8a8_export_weights(w: Weights, stream=None) -> dict:
+    torch = _torch()
+    c = w.cfg
+    E, d, f = c.n_experts, c.d, c.f
+    dev = torch.device("cuda")
+    out = dict(wq_gate=torch.empty((E, f, d), dtype=torch.int8, device=dev),
+               wq_up=torch.empty((E, f, d), dtype=torch.int8, device=dev),
+               sw_gate=torch.empty((E, f), dtype=torch.float32, device=dev),
+               sw_up=torch.empty((E, f), dtype=torch.float32, device=dev),
+               wq_down=torch.empty((E, d, f), dtype=torch.int8, device=dev),
+               sw_down=torch.empty((E, d), dtype=torch.float32, device=dev),
+               inv_s=torch.empty((d,), dtype=torch.float32, device=dev))
+    _check(lib().moe_w8a8_export_weights(w.handle, *(ctypes.c_void_p(out[k].data_ptr()) for k in
+                                                     ("wq_gate", "wq_up", "sw_gate", "sw_up",
+                                                      "wq_down", "sw_down", "inv_s")),
+                                         _stream(stream)), "moe_w8a8_export_weights")
+    return out
+
+
+def moe_w8a8_check_status(w: Weights, stream=None):
+    _check(lib().moe_w8a8_check_status(w.handle, _stream(stream)), "moe_w8a8_check_status")
+
+
+def moe_w8a8_last_launch_count(w: Weights) -> int:
+    return int(lib().moe_w8a8_last_launch_count(w.handle))

@@ -1,0 +1,139 @@
+// Device-side helpers shared by the kernels of the W8A8 MoE layer.
+//
+// Every floating-point step that decides an integer (a quantised code, a
+// top-k choice) is written with explicit round-to-nearest intrinsics so that
+// the compiler cannot contract or reorder it: the layer's specification fixes
+// each of those operations as one IEEE fp32 operation in a stated order.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace moe {
+
+constexpr int kWarp = 32;
+
+// ---------------------------------------------------------------------------
+// exp by Cody & Waite range reduction and a degree-7 Taylor polynomial.
+// x is clamped to [-87, 88]; x = n ln2 + r with n = rint(x log2 e); ln2 is
+// split into a head with 16 significant bits (n * head exact for |n| < 256)
+// and an fp32 tail; e^r = sum_{i<=7} r^i / i! in Horner form (|r| <= ln2/2);
+// 2^n is assembled from exponent bits (n in [-126, 127], always normal).
+// This fixed sequence is what makes SiLU and the gate softmax reproducible
+// bit for bit against a CPU evaluation of the same steps.
+// ---------------------------------------------------------------------------
+namespace expc {
+constexpr double kLn2 = 0.69314718055994530941723212145818;
+constexpr double fact(int i) { return i <= 1 ? 1.0 : i * fact(i - 1); }
+constexpr float kLog2e = (float)(1.0 / kLn2);
+constexpr float kLn2Hi = (float)((double)(long long)(kLn2 * 65536.0) / 65536.0);
+constexpr float kLn2Lo = (float)(kLn2 - (double)kLn2Hi);
+constexpr float kC0 = (float)(1.0 / fact(0)), kC1 = (float)(1.0 / fact(1));
+constexpr float kC2 = (float)(1.0 / fact(2)), kC3 = (float)(1.0 / fact(3));
+constexpr float kC4 = (float)(1.0 / fact(4)), kC5 = (float)(1.0 / fact(5));
+constexpr float kC6 = (float)(1.0 / fact(6)), kC7 = (float)(1.0 / fact(7));
+}  // namespace expc
+
+__device__ __forceinline__ float moe_exp(float x) {
+    using namespace expc;
+    x = fminf(fmaxf(x, -87.0f), 88.0f);
+    const float n = rintf(__fmul_rn(x, kLog2e));
+    float r = __fmaf_rn(-n, kLn2Hi, x);
+    r = __fmaf_rn(-n, kLn2Lo, r);
+    float p = kC7;
+    p = __fmaf_rn(p, r, kC6);
+    p = __fmaf_rn(p, r, kC5);
+    p = __fmaf_rn(p, r, kC4);
+    p = __fmaf_rn(p, r, kC3);
+    p = __fmaf_rn(p, r, kC2);
+    p = __fmaf_rn(p, r, kC1);
+    p = __fmaf_rn(p, r, kC0);
+    const int ni = __float2int_rn(n);
+    return __fmul_rn(p, __int_as_float((ni + 127) << 23));
+}
+
+// silu(g) = g / (1 + e^-g)
+__device__ __forceinline__ float moe_silu(float g) {
+    return __fdiv_rn(g, __fadd_rn(1.0f, moe_exp(-g)));
+}
+
+// Symmetric INT8 code of v for scale s > 0: rint(v / s), ties to even, clamped
+// to [-127, 127].  Callers handle s == 0 (all-zero vector -> code 0).
+__device__ __forceinline__ int quant_code(float v, float s) {
+    int q = __float2int_rn(__fdiv_rn(v, s));
+    return max(-127, min(127, q));
+}
+
+// Pack four INT8 codes (low byte first).
+__device__ __forceinline__ uint32_t pack4(int a, int b, int c, int d) {
+    return (uint32_t)(a & 0xff) | ((uint32_t)(b & 0xff) << 8) | ((uint32_t)(c & 0xff) << 16) |
+           ((uint32_t)(d & 0xff) << 24);
+}
+
+__device__ __forceinline__ float bf16_bits_to_f32(uint16_t h) {
+    return __uint_as_float((uint32_t)h << 16);
+}
+
+// fp32 -> bf16 round to nearest even (finite inputs).
+__device__ __forceinline__ uint16_t f32_to_bf16_bits(float v) {
+    return __bfloat16_as_ushort(__float2bfloat16_rn(v));
+}
+
+// Streaming 128-bit global load that does not allocate in L1 (weights are
+// read once per launch).
+__device__ __forceinline__ int4 ld_stream_v4(const void* p) {
+    int4 r;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.s32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+                 : "l"(p));
+    return r;
+}
+
+__device__ __forceinline__ int dp4a(int a, int b, int c) { return __dp4a(a, b, c); }
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+
+__device__ __forceinline__ int warp_sum_i(int v) {
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+// Max of non-negative floats over a block (blockDim.x multiple of 32, <= 1024).
+// Exact: max does not depend on the order.  `red` needs 32 floats.
+__device__ __forceinline__ float block_max_nonneg(float v, float* red) {
+    v = warp_max(v);
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    __syncthreads();
+    if (lane == 0) red[wid] = v;
+    __syncthreads();
+    const int nw = blockDim.x >> 5;
+    float m = lane < nw ? red[lane] : 0.0f;
+    m = warp_max(m);
+    return m;
+}
+
+// Load 8 consecutive activations as fp32 (in_dtype: 0 fp32, 1 bf16).
+__device__ __forceinline__ void load8_act(const void* x, int64_t idx, int in_dtype, float v[8]) {
+    if (in_dtype == 1) {
+        const int4 raw = *reinterpret_cast<const int4*>(reinterpret_cast<const uint16_t*>(x) + idx);
+        const uint32_t w[4] = {(uint32_t)raw.x, (uint32_t)raw.y, (uint32_t)raw.z, (uint32_t)raw.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            v[2 * i] = __uint_as_float(w[i] << 16);
+            v[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+        }
+    } else {
+        const float4 a = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(x) + idx);
+        const float4 b = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(x) + idx + 4);
+        v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+        v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+    }
+}
+
+}  // namespace moe

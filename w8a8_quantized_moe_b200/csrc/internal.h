@@ -1,0 +1,97 @@
+// Internal declarations of the W8A8 MoE library: the prepared-weights handle,
+// the workspace layout and the kernel launchers (one per .cu file group).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/moe_w8a8.h"
+
+struct moe_w8a8_weights {
+    moe_w8a8_config cfg;
+    int device;
+    int num_sms;
+    int path;               // MOE_PATH_*
+    int stream_max_rows;    // AUTO: streaming path when T*k <= this
+    int last_launches;
+    // prepared weights (device)
+    int8_t* w_gu;     // [E][2f][d]: per 128-channel block, 128 gate rows then 128 up rows
+    int8_t* w_dn;     // [E][d][f]
+    float* sw_gate;   // [E][f]
+    float* sw_up;     // [E][f]
+    float* sw_dn;     // [E][d]
+    float* inv_s;     // [d]
+    float* w_router;  // [d][E]
+    float* s_host;    // [d] (host)
+    int32_t* status;  // device status word
+    // tensor maps of the weights for the tensor-core path (built at prepare)
+    CUtensorMap tm_w_gu;
+    CUtensorMap tm_w_dn;
+    bool tmaps_ok;
+};
+
+namespace moe {
+
+constexpr int kGuBlock = 128;       // gate/up interleave block (channels)
+constexpr int kPermChunk = 2048;    // (t, slot) entries per permute block
+constexpr int kMaxK = 8;
+constexpr int kMaxE = 256;
+
+// Byte offsets of the forward workspace for T tokens.
+struct WsLayout {
+    size_t x_stage, y_stage, logits_stage, bias_stage;   // forward_host staging
+    size_t logits, topk_idx, topk_w;
+    size_t hist, offsets, meta, active, tiles;
+    size_t row2ts, ts2row;
+    size_t xq, sx, aq;
+    size_t acc1, hq, sh, o;
+    size_t total;
+};
+WsLayout ws_layout(const moe_w8a8_weights* w, int T);
+
+// meta[] words written by the permute scatter kernel
+enum { META_R = 0, META_NACTIVE = 1, META_NTILES = 2, META_WORDS = 8 };
+constexpr int kTileM = 128;   // rows per tensor-core tile
+
+// ------------------------------------------------------------------ kernels
+cudaError_t launch_calib_absmax(const void* x, int64_t rows, int d, int dtype, float* absmax,
+                                cudaStream_t s);
+cudaError_t launch_gateup_input_absmax(const float* w_gate, const float* w_up, int E, int d, int f,
+                                       float* aw, cudaStream_t s);
+// Quantise column-major channels: W [E][K][N] fp32 (input j, output n), optional
+// per-input smoothing s[K]; channel n goes to out row map(n) of [E][rows][K].
+cudaError_t launch_quantize_channels(const float* w, const float* smooth, int E, int K, int N,
+                                     int8_t* out, int out_rows, int row_block, int row_stride,
+                                     int row_base, float* sw, cudaStream_t s);
+cudaError_t launch_export_gateup(const int8_t* w_gu, int E, int d, int f, int8_t* gate,
+                                 int8_t* up, cudaStream_t s);
+
+cudaError_t launch_router_logits(const void* x, int in_dtype, const float* wr, int T, int d, int E,
+                                 float* logits, cudaStream_t s);
+cudaError_t launch_topk(const float* logits, const float* bias, int T, int E, int k, int renorm,
+                        int32_t* idx, float* wts, float* logits_out, cudaStream_t s);
+cudaError_t launch_permute(const int32_t* idx, int T, int k, int E, int cap, int32_t* hist,
+                           int32_t* offsets, int32_t* row2ts, int32_t* ts2row, int32_t* meta,
+                           int32_t* active, int32_t* tiles, cudaStream_t s);
+cudaError_t launch_smooth_quant(const void* x, int in_dtype, const float* inv_s, int T, int d,
+                                int k, const int32_t* ts2row, int8_t* xq, float* sx, int8_t* aq,
+                                cudaStream_t s);
+
+cudaError_t launch_stream_gateup(const moe_w8a8_weights* w, int T, const int8_t* xq,
+                                 const int32_t* row2ts, const int32_t* offsets,
+                                 const int32_t* active, const int32_t* meta, int32_t* acc1,
+                                 cudaStream_t s);
+cudaError_t launch_swiglu_requant(const moe_w8a8_weights* w, const int32_t* acc1,
+                                  const int32_t* row2ts, const int32_t* topk_idx,
+                                  const float* sx, const int32_t* meta, int max_rows, int8_t* hq,
+                                  float* sh, cudaStream_t s);
+cudaError_t launch_stream_down(const moe_w8a8_weights* w, int T, const int8_t* hq,
+                               const float* sh, const int32_t* row2ts, const float* topk_w,
+                               const int32_t* offsets, const int32_t* active, const int32_t* meta,
+                               float* o, int32_t* acc2_dbg, cudaStream_t s);
+cudaError_t launch_combine(const float* o, const int32_t* ts2row, int T, int k, int d,
+                           int out_dtype, void* y, cudaStream_t s);
+
+}  // namespace moe

@@ -1,0 +1,335 @@
+// Gate, top-k, sort-by-expert and smoothed per-token quantisation.
+// ("Day0 adaptation of ultra-large model inference", section 4: gate ->
+// sort -> grouped GEMM -> un-sort -> weighted sum, with top-k routing equal to
+// the reference including its tie-break; section 2 item 2: capacity factor.
+// "MiniMax-M3 W8A8 on K100AI", s3.2 / s6.4: smoothing and per-token INT8.)
+#include "common.cuh"
+#include "internal.h"
+
+namespace moe {
+namespace {
+
+// ---------------------------------------------------------------------------
+// Router logits in the stated fp32 order: for each (t, e), lane p of a warp
+// owns partial sum p = fma chain over i ascending of x[t][32i+p] W[32i+p][e]
+// from +0; the 32 partials are combined by xor-butterfly 16, 8, 4, 2, 1.
+// A warp computes a block of 4 tokens x 16 experts (64 chains per lane).
+// ---------------------------------------------------------------------------
+constexpr int kRtTok = 4;    // tokens per warp
+constexpr int kRtExp = 16;   // experts per warp
+constexpr int kRtWarps = 8;
+
+__global__ void __launch_bounds__(kRtWarps * 32) router_logits_kernel(
+    const void* __restrict__ x, int in_dtype, const float* __restrict__ wr, int T, int d, int E,
+    float* __restrict__ logits) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int n_eg = (E + kRtExp - 1) / kRtExp;
+    const int wid = blockIdx.x * kRtWarps + warp;   // global warp id
+    const int tg = wid / n_eg, eg = wid % n_eg;
+    const int t0 = tg * kRtTok, e0 = eg * kRtExp;
+    if (t0 >= T) return;
+    float acc[kRtTok][kRtExp];
+#pragma unroll
+    for (int a = 0; a < kRtTok; ++a)
+#pragma unroll
+        for (int b = 0; b < kRtExp; ++b) acc[a][b] = 0.0f;
+    const int nchunks = d / 32;
+    for (int i = 0; i < nchunks; ++i) {
+        const int j = 32 * i + lane;
+        float xv[kRtTok];
+#pragma unroll
+        for (int a = 0; a < kRtTok; ++a) {
+            const int t = min(t0 + a, T - 1);
+            xv[a] = in_dtype == MOE_BF16
+                        ? bf16_bits_to_f32(reinterpret_cast<const uint16_t*>(x)[(int64_t)t * d + j])
+                        : reinterpret_cast<const float*>(x)[(int64_t)t * d + j];
+        }
+        const float* wrow = wr + (int64_t)j * E + e0;
+#pragma unroll
+        for (int b = 0; b < kRtExp; ++b) {
+            const float wv = (e0 + b < E) ? __ldg(wrow + b) : 0.0f;
+#pragma unroll
+            for (int a = 0; a < kRtTok; ++a) acc[a][b] = __fmaf_rn(xv[a], wv, acc[a][b]);
+        }
+    }
+#pragma unroll
+    for (int a = 0; a < kRtTok; ++a)
+#pragma unroll
+        for (int b = 0; b < kRtExp; ++b) {
+            float v = acc[a][b];
+#pragma unroll
+            for (int o = 16; o >= 1; o >>= 1) v = __fadd_rn(v, __shfl_xor_sync(0xffffffffu, v, o));
+            acc[a][b] = v;
+        }
+    // every lane now holds all 64 logits; lane q writes entries q and q + 32
+#pragma unroll
+    for (int v = 0; v < kRtTok * kRtExp; ++v) {
+        if ((v & 31) != lane) continue;
+        const int a = v / kRtExp, b = v % kRtExp;
+        const int t = t0 + a, e = e0 + b;
+        if (t < T && e < E) logits[(int64_t)t * E + e] = acc[a][b];
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Top-k + gate weights, one warp per token.  l_e = logit + bias_e; k rounds of
+// a warp argmax on (l descending, e ascending); w = softmax of the selected
+// logits (renormalised) with the layer's exp, sum in slot order.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ bool better(float v, int i, float v2, int i2) {
+    return v > v2 || (v == v2 && i < i2);
+}
+
+__global__ void topk_kernel(const float* __restrict__ logits, const float* __restrict__ bias, int T,
+                            int E, int k, int renorm, int32_t* __restrict__ idx,
+                            float* __restrict__ wts, float* __restrict__ logits_out) {
+    __shared__ float lsh[8][kMaxE];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int t = blockIdx.x * 8 + warp;
+    if (t >= T) return;
+    constexpr int kPer = kMaxE / 32;
+    float l[kPer];
+    bool taken[kPer];
+#pragma unroll
+    for (int m = 0; m < kPer; ++m) {
+        const int e = lane + 32 * m;
+        float v = -INFINITY;
+        if (e < E) {
+            v = logits[(int64_t)t * E + e];
+            if (bias) v = __fadd_rn(v, bias[e]);
+            if (logits_out) logits_out[(int64_t)t * E + e] = v;
+            lsh[warp][e] = v;
+        }
+        l[m] = v;
+        taken[m] = e >= E;
+    }
+    float sel_v[kMaxK];
+    int sel_i[kMaxK];
+#pragma unroll
+    for (int s = 0; s < kMaxK; ++s) {
+        if (s >= k) break;
+        float bv = -INFINITY;
+        int bi = 0x7fffffff;
+#pragma unroll
+        for (int m = 0; m < kPer; ++m) {
+            const int e = lane + 32 * m;
+            if (!taken[m] && better(l[m], e, bv, bi)) { bv = l[m]; bi = e; }
+        }
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) {
+            const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+            const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+            if (better(ov, oi, bv, bi)) { bv = ov; bi = oi; }
+        }
+#pragma unroll
+        for (int m = 0; m < kPer; ++m)
+            if (lane + 32 * m == bi) taken[m] = true;
+        sel_v[s] = bv;
+        sel_i[s] = bi;
+    }
+    __syncwarp();
+    if (lane == 0) {
+        const float lmax = sel_v[0];
+        float z = 0.0f;
+        if (renorm) {
+            for (int s = 0; s < k; ++s) z = __fadd_rn(z, moe_exp(__fsub_rn(sel_v[s], lmax)));
+        } else {
+            for (int e = 0; e < E; ++e) z = __fadd_rn(z, moe_exp(__fsub_rn(lsh[warp][e], lmax)));
+        }
+        for (int s = 0; s < k; ++s) {
+            idx[(int64_t)t * k + s] = sel_i[s];
+            wts[(int64_t)t * k + s] = __fdiv_rn(moe_exp(__fsub_rn(sel_v[s], lmax)), z);
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Sort by expert: histogram per chunk of kPermChunk entries (t*k + slot
+// order), then a scatter in which every block derives the global expert
+// offsets and its own prefix from the histogram and ranks its entries stably
+// (warp match + per-warp counts).  Entry i of expert e gets position
+// pos = #(earlier entries of e); it is kept when pos < capacity.
+// ---------------------------------------------------------------------------
+__global__ void perm_hist_kernel(const int32_t* __restrict__ idx, int n, int E,
+                                 int32_t* __restrict__ hist) {
+    __shared__ int cnt[kMaxE];
+    for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[e] = 0;
+    __syncthreads();
+    const int base = blockIdx.x * kPermChunk;
+    for (int i = threadIdx.x; i < kPermChunk; i += blockDim.x)
+        if (base + i < n) atomicAdd(&cnt[idx[base + i]], 1);
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += blockDim.x) hist[(int64_t)blockIdx.x * E + e] = cnt[e];
+}
+
+constexpr int kPermThreads = 256;
+
+__global__ void __launch_bounds__(kPermThreads) perm_scatter_kernel(
+    const int32_t* __restrict__ idx, int n, int E, int cap, int nblk,
+    const int32_t* __restrict__ hist, int32_t* __restrict__ offsets, int32_t* __restrict__ row2ts,
+    int32_t* __restrict__ ts2row, int32_t* __restrict__ meta, int32_t* __restrict__ active,
+    int32_t* __restrict__ tiles) {
+    __shared__ int pre[kMaxE], off[kMaxE + 1], running[kMaxE], kept[kMaxE];
+    __shared__ int wcnt[kPermThreads / 32][kMaxE];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    for (int e = tid; e < E; e += blockDim.x) {
+        int tot = 0, before = 0;
+        for (int b = 0; b < nblk; ++b) {
+            const int h = hist[(int64_t)b * E + e];
+            tot += h;
+            if (b < (int)blockIdx.x) before += h;
+        }
+        pre[e] = before;
+        kept[e] = cap < 0 ? tot : min(tot, cap);
+        running[e] = 0;
+    }
+    __syncthreads();
+    if (tid == 0) {
+        int acc = 0;
+        for (int e = 0; e < E; ++e) { off[e] = acc; acc += kept[e]; }
+        off[E] = acc;
+    }
+    __syncthreads();
+    if (blockIdx.x == 0 && tid == 0) {
+        int na = 0, nt = 0;
+        for (int e = 0; e <= E; ++e) offsets[e] = off[e];
+        for (int e = 0; e < E; ++e) {
+            if (kept[e] == 0) continue;
+            active[na++] = e;
+            for (int m = 0; m * kTileM < kept[e]; ++m) {
+                tiles[2 * nt] = e;
+                tiles[2 * nt + 1] = off[e] + m * kTileM;
+                ++nt;
+            }
+        }
+        meta[META_R] = off[E];
+        meta[META_NACTIVE] = na;
+        meta[META_NTILES] = nt;
+    }
+    const int base = blockIdx.x * kPermChunk;
+    for (int r0 = 0; r0 < kPermChunk; r0 += kPermThreads) {
+        for (int i = tid; i < (kPermThreads / 32) * E; i += blockDim.x) (&wcnt[0][0])[i] = 0;
+        __syncthreads();
+        const int i = base + r0 + tid;
+        const bool valid = i < n;
+        const int e = valid ? idx[i] : -1;
+        const unsigned m = __match_any_sync(0xffffffffu, e);
+        const int rank_w = __popc(m & ((1u << lane) - 1u));
+        if (valid && rank_w == 0) wcnt[warp][e] = __popc(m);
+        __syncthreads();
+        if (valid) {
+            int rank = running[e] + rank_w;
+            for (int w2 = 0; w2 < warp; ++w2) rank += wcnt[w2][e];
+            const int pos = pre[e] + rank;
+            if (cap < 0 || pos < cap) {
+                const int row = off[e] + pos;
+                ts2row[i] = row;
+                row2ts[row] = i;
+            } else {
+                ts2row[i] = -1;
+            }
+        }
+        __syncthreads();
+        for (int e2 = tid; e2 < E; e2 += blockDim.x) {
+            int s = 0;
+            for (int w2 = 0; w2 < kPermThreads / 32; ++w2) s += wcnt[w2][e2];
+            running[e2] += s;
+        }
+        __syncthreads();
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Smoothed per-token quantisation: x' = fp32(x * inv_s); sx = amax/127;
+// q = rint(x'/sx) clamped to +-127.  One block per token; each thread owns
+// groups of 8 channels.  Writes xq[t] and, when aq is given, the copy of the
+// token's codes into every kept (t, slot) row of the expert-sorted matrix.
+// ---------------------------------------------------------------------------
+constexpr int kSqThreads = 256;
+constexpr int kSqMaxGroups = 8;   // d <= 256 * 8 * 8 = 16384
+
+__global__ void __launch_bounds__(kSqThreads) smooth_quant_kernel(
+    const void* __restrict__ x, int in_dtype, const float* __restrict__ inv_s, int d, int k,
+    const int32_t* __restrict__ ts2row, int8_t* __restrict__ xq, float* __restrict__ sx,
+    int8_t* __restrict__ aq) {
+    __shared__ float red[32];
+    const int t = blockIdx.x;
+    const int ng = d / 8;
+    float v[kSqMaxGroups][8];
+    float m = 0.0f;
+#pragma unroll
+    for (int gi = 0; gi < kSqMaxGroups; ++gi) {
+        const int g = threadIdx.x + gi * kSqThreads;
+        if (g < ng) {
+            load8_act(x, (int64_t)t * d + g * 8, in_dtype, v[gi]);
+            const float4 s0 = *reinterpret_cast<const float4*>(inv_s + g * 8);
+            const float4 s1 = *reinterpret_cast<const float4*>(inv_s + g * 8 + 4);
+            const float sv[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                v[gi][c] = __fmul_rn(v[gi][c], sv[c]);
+                m = fmaxf(m, fabsf(v[gi][c]));
+            }
+        }
+    }
+    const float amax = block_max_nonneg(m, red);
+    const float s = amax > 0.0f ? __fdiv_rn(amax, 127.0f) : 0.0f;
+    if (threadIdx.x == 0) sx[t] = s;
+    int rows[kMaxK];
+    if (aq)
+        for (int sl = 0; sl < k; ++sl) rows[sl] = ts2row[(int64_t)t * k + sl];
+#pragma unroll
+    for (int gi = 0; gi < kSqMaxGroups; ++gi) {
+        const int g = threadIdx.x + gi * kSqThreads;
+        if (g < ng) {
+            int q[8];
+#pragma unroll
+            for (int c = 0; c < 8; ++c) q[c] = s > 0.0f ? quant_code(v[gi][c], s) : 0;
+            const uint2 packed = make_uint2(pack4(q[0], q[1], q[2], q[3]), pack4(q[4], q[5], q[6], q[7]));
+            *reinterpret_cast<uint2*>(xq + (int64_t)t * d + g * 8) = packed;
+            if (aq)
+                for (int sl = 0; sl < k; ++sl)
+                    if (rows[sl] >= 0)
+                        *reinterpret_cast<uint2*>(aq + (int64_t)rows[sl] * d + g * 8) = packed;
+        }
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_router_logits(const void* x, int in_dtype, const float* wr, int T, int d, int E,
+                                 float* logits, cudaStream_t s) {
+    const int n_eg = (E + kRtExp - 1) / kRtExp;
+    const int64_t warps = (int64_t)((T + kRtTok - 1) / kRtTok) * n_eg;
+    const int blocks = (int)((warps + kRtWarps - 1) / kRtWarps);
+    router_logits_kernel<<<blocks, kRtWarps * 32, 0, s>>>(x, in_dtype, wr, T, d, E, logits);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_topk(const float* logits, const float* bias, int T, int E, int k, int renorm,
+                        int32_t* idx, float* wts, float* logits_out, cudaStream_t s) {
+    topk_kernel<<<(T + 7) / 8, 256, 0, s>>>(logits, bias, T, E, k, renorm, idx, wts, logits_out);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_permute(const int32_t* idx, int T, int k, int E, int cap, int32_t* hist,
+                           int32_t* offsets, int32_t* row2ts, int32_t* ts2row, int32_t* meta,
+                           int32_t* active, int32_t* tiles, cudaStream_t s) {
+    const int n = T * k;
+    const int nblk = (n + kPermChunk - 1) / kPermChunk;
+    perm_hist_kernel<<<nblk, 256, 0, s>>>(idx, n, E, hist);
+    cudaError_t err = cudaGetLastError();
+    if (err != cudaSuccess) return err;
+    perm_scatter_kernel<<<nblk, kPermThreads, 0, s>>>(idx, n, E, cap, nblk, hist, offsets, row2ts,
+                                                      ts2row, meta, active, tiles);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_smooth_quant(const void* x, int in_dtype, const float* inv_s, int T, int d,
+                                int k, const int32_t* ts2row, int8_t* xq, float* sx, int8_t* aq,
+                                cudaStream_t s) {
+    smooth_quant_kernel<<<T, kSqThreads, 0, s>>>(x, in_dtype, inv_s, d, k, ts2row, xq, sx, aq);
+    return cudaGetLastError();
+}
+
+}  // namespace moe

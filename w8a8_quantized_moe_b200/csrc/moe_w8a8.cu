@@ -1,0 +1,392 @@
+// C ABI of the W8A8 MoE layer: argument checks, the prepared-weights handle,
+// the workspace layout and the launch sequence of one forward.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdlib>
+#include <cstring>
+#include <vector>
+
+#include "internal.h"
+
+using namespace moe;
+
+namespace {
+
+constexpr size_t kAlign = 256;
+inline size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+moe_status check_config(const moe_w8a8_config* c) {
+    if (!c) return MOE_ERR_INVALID_ARG;
+    if (!(c->alpha >= 0.0f && c->alpha <= 1.0f)) return MOE_ERR_INVALID_ARG;
+    if (c->in_dtype != MOE_F32 && c->in_dtype != MOE_BF16) return MOE_ERR_INVALID_ARG;
+    if (c->out_dtype != MOE_F32 && c->out_dtype != MOE_BF16) return MOE_ERR_INVALID_ARG;
+    if (c->renormalize != 0 && c->renormalize != 1) return MOE_ERR_INVALID_ARG;
+    if (std::isnan(c->capacity_factor)) return MOE_ERR_INVALID_ARG;
+    if (c->d <= 0 || c->f <= 0 || c->n_experts <= 0 || c->top_k <= 0) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (c->d % 128 || c->f % 128) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (c->d > 16384 || c->f > 16384) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (c->n_experts > kMaxE || c->top_k > kMaxK || c->top_k > c->n_experts) return MOE_ERR_UNSUPPORTED_SHAPE;
+    return MOE_OK;
+}
+
+// Capacity per expert: ceil(cf * T * k / E) in fp64, -1 for none.
+int capacity_of(const moe_w8a8_config& c, int T) {
+    if (!(c.capacity_factor > 0.0f)) return -1;
+    return (int)std::ceil((double)c.capacity_factor * (double)((int64_t)T * c.top_k) / (double)c.n_experts);
+}
+
+int choose_path(const moe_w8a8_weights* w, int T) {
+    if (w->path != MOE_PATH_AUTO) return w->path;
+    return (int64_t)T * w->cfg.top_k <= w->stream_max_rows ? MOE_PATH_STREAM : MOE_PATH_TENSOR;
+}
+
+void free_handle(moe_w8a8_weights* w) {
+    if (!w) return;
+    cudaFree(w->w_gu);
+    cudaFree(w->w_dn);
+    cudaFree(w->sw_gate);
+    cudaFree(w->sw_up);
+    cudaFree(w->sw_dn);
+    cudaFree(w->inv_s);
+    cudaFree(w->w_router);
+    cudaFree(w->status);
+    std::free(w->s_host);
+    delete w;
+}
+
+#define CUDA_TRY(expr)                                  \
+    do {                                                \
+        cudaError_t err_ = (expr);                      \
+        if (err_ != cudaSuccess) return MOE_ERR_CUDA;   \
+    } while (0)
+
+}  // namespace
+
+namespace moe {
+
+WsLayout ws_layout(const moe_w8a8_weights* w, int T) {
+    const moe_w8a8_config& c = w->cfg;
+    const int E = c.n_experts, k = c.top_k, d = c.d, f = c.f;
+    const size_t tk = (size_t)T * k;
+    const size_t in_b = c.in_dtype == MOE_BF16 ? 2 : 4, out_b = c.out_dtype == MOE_BF16 ? 2 : 4;
+    const size_t nblk = (tk + kPermChunk - 1) / kPermChunk;
+    const size_t max_tiles = (tk + kTileM - 1) / kTileM + E;
+    const bool stream = choose_path(w, T) == MOE_PATH_STREAM;
+    WsLayout L{};
+    size_t p = 0;
+    auto take = [&](size_t bytes) { size_t at = p; p = align_up(p + bytes); return at; };
+    L.x_stage = take((size_t)T * d * in_b);
+    L.y_stage = take((size_t)T * d * out_b);
+    L.logits_stage = take((size_t)T * E * 4);
+    L.bias_stage = take((size_t)E * 4);
+    L.logits = take((size_t)T * E * 4);
+    L.topk_idx = take(tk * 4);
+    L.topk_w = take(tk * 4);
+    L.hist = take(nblk * E * 4);
+    L.offsets = take((size_t)(E + 1) * 4);
+    L.meta = take(META_WORDS * 4);
+    L.active = take((size_t)E * 4);
+    L.tiles = take(max_tiles * 8);
+    L.row2ts = take(tk * 4);
+    L.ts2row = take(tk * 4);
+    L.xq = take((size_t)T * d);
+    L.sx = take((size_t)T * 4);
+    L.aq = take(stream ? 0 : tk * d);
+    L.acc1 = take(stream ? tk * 2 * f * 4 : 0);
+    L.hq = take(tk * f);
+    L.sh = take(tk * 4);
+    L.o = take(tk * d * 4);
+    L.total = p;
+    return L;
+}
+
+}  // namespace moe
+
+extern "C" {
+
+const char* moe_status_string(moe_status s) {
+    switch (s) {
+        case MOE_OK: return "ok";
+        case MOE_ERR_INVALID_ARG: return "invalid argument";
+        case MOE_ERR_UNSUPPORTED_SHAPE: return "unsupported shape";
+        case MOE_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
+        case MOE_ERR_CUDA: return "CUDA error";
+        case MOE_ERR_TIMEOUT: return "device wait timed out";
+        case MOE_ERR_OOM: return "device allocation failed";
+    }
+    return "unknown status";
+}
+
+moe_status moe_w8a8_calibrate_absmax(const void* x, int64_t rows, int32_t d, int32_t dtype,
+                                     float* absmax, moe_stream_t stream) {
+    if (!absmax || rows < 0 || (rows > 0 && !x)) return MOE_ERR_INVALID_ARG;
+    if (dtype != MOE_F32 && dtype != MOE_BF16) return MOE_ERR_INVALID_ARG;
+    if (d <= 0) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (launch_calib_absmax(x, rows, d, dtype, absmax, (cudaStream_t)stream) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    return MOE_OK;
+}
+
+moe_status moe_w8a8_prepare(const moe_w8a8_config* cfg, const float* w_gate, const float* w_up,
+                            const float* w_down, const float* w_router, const float* act_absmax,
+                            moe_stream_t stream, moe_w8a8_weights** out) {
+    if (!out) return MOE_ERR_INVALID_ARG;
+    *out = nullptr;
+    moe_status st = check_config(cfg);
+    if (st != MOE_OK) return st;
+    if (!w_gate || !w_up || !w_down || !w_router || !act_absmax) return MOE_ERR_INVALID_ARG;
+    const moe_w8a8_config c = *cfg;
+    const int E = c.n_experts, d = c.d, f = c.f;
+    cudaStream_t s = (cudaStream_t)stream;
+
+    moe_w8a8_weights* w = new moe_w8a8_weights();
+    w->cfg = c;
+    w->path = MOE_PATH_AUTO;
+    w->stream_max_rows = 512;
+    if (cudaGetDevice(&w->device) != cudaSuccess ||
+        cudaDeviceGetAttribute(&w->num_sms, cudaDevAttrMultiProcessorCount, w->device) != cudaSuccess) {
+        free_handle(w);
+        return MOE_ERR_CUDA;
+    }
+    const size_t n_gu = (size_t)E * 2 * f * d, n_dn = (size_t)E * d * f;
+    bool ok = cudaMalloc(&w->w_gu, n_gu) == cudaSuccess && cudaMalloc(&w->w_dn, n_dn) == cudaSuccess &&
+              cudaMalloc(&w->sw_gate, (size_t)E * f * 4) == cudaSuccess &&
+              cudaMalloc(&w->sw_up, (size_t)E * f * 4) == cudaSuccess &&
+              cudaMalloc(&w->sw_dn, (size_t)E * d * 4) == cudaSuccess &&
+              cudaMalloc(&w->inv_s, (size_t)d * 4) == cudaSuccess &&
+              cudaMalloc(&w->w_router, (size_t)d * E * 4) == cudaSuccess &&
+              cudaMalloc(&w->status, 64) == cudaSuccess;
+    w->s_host = (float*)std::malloc((size_t)d * 4);
+    float* tmp = nullptr;   // aw [d] then s [d] on the device
+    ok = ok && w->s_host && cudaMalloc(&tmp, (size_t)2 * d * 4) == cudaSuccess;
+    if (!ok) {
+        cudaGetLastError();
+        cudaFree(tmp);
+        free_handle(w);
+        return MOE_ERR_OOM;
+    }
+    auto fail = [&](moe_status code) {
+        cudaFree(tmp);
+        free_handle(w);
+        return code;
+    };
+    float* aw_dev = tmp;
+    float* s_dev = tmp + d;
+    if (cudaMemsetAsync(w->status, 0, 64, s) != cudaSuccess ||
+        cudaMemsetAsync(aw_dev, 0, (size_t)d * 4, s) != cudaSuccess ||
+        launch_gateup_input_absmax(w_gate, w_up, E, d, f, aw_dev, s) != cudaSuccess)
+        return fail(MOE_ERR_CUDA);
+    std::vector<float> aw(d), ax(d), inv(d);
+    if (cudaMemcpyAsync(aw.data(), aw_dev, (size_t)d * 4, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+        cudaMemcpyAsync(ax.data(), act_absmax, (size_t)d * 4, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+        cudaStreamSynchronize(s) != cudaSuccess)
+        return fail(MOE_ERR_CUDA);
+    // SmoothQuant scales, fp64 on the host: s_j = ax^alpha / aw^(1-alpha), both
+    // statistics floored at 1e-5; inv_s_j = fp32(1 / s_j).
+    const double a = (double)c.alpha;
+    const double floor_v = (double)1e-5f;
+    for (int j = 0; j < d; ++j) {
+        const double xv = ax[j] > 1e-5f ? (double)ax[j] : floor_v;
+        const double wv = aw[j] > 1e-5f ? (double)aw[j] : floor_v;
+        w->s_host[j] = (float)(std::pow(xv, a) / std::pow(wv, 1.0 - a));
+        inv[j] = (float)(1.0 / (double)w->s_host[j]);
+    }
+    if (cudaMemcpyAsync(s_dev, w->s_host, (size_t)d * 4, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+        cudaMemcpyAsync(w->inv_s, inv.data(), (size_t)d * 4, cudaMemcpyHostToDevice, s) != cudaSuccess)
+        return fail(MOE_ERR_CUDA);
+    // gate -> rows [blk*256, blk*256+128), up -> rows [blk*256+128, blk*256+256)
+    if (launch_quantize_channels(w_gate, s_dev, E, d, f, w->w_gu, 2 * f, kGuBlock, 2 * kGuBlock, 0,
+                                 w->sw_gate, s) != cudaSuccess ||
+        launch_quantize_channels(w_up, s_dev, E, d, f, w->w_gu, 2 * f, kGuBlock, 2 * kGuBlock,
+                                 kGuBlock, w->sw_up, s) != cudaSuccess ||
+        launch_quantize_channels(w_down, nullptr, E, f, d, w->w_dn, d, d, d, 0, w->sw_dn, s) !=
+            cudaSuccess ||
+        cudaMemcpyAsync(w->w_router, w_router, (size_t)d * E * 4, cudaMemcpyDeviceToDevice, s) !=
+            cudaSuccess ||
+        cudaStreamSynchronize(s) != cudaSuccess)
+        return fail(MOE_ERR_CUDA);
+    cudaFree(tmp);
+    *out = w;
+    return MOE_OK;
+}
+
+size_t moe_w8a8_workspace_size(const moe_w8a8_weights* w, int32_t max_tokens) {
+    if (!w || max_tokens < 0) return 0;
+    return ws_layout(w, max_tokens).total;
+}
+
+static moe_status forward_impl(const moe_w8a8_weights* w, const void* x, int T, const float* bias,
+                               const float* given_logits, void* y, char* ws,
+                               const moe_w8a8_debug* dbg, cudaStream_t s) {
+    const moe_w8a8_config& c = w->cfg;
+    const int E = c.n_experts, k = c.top_k, d = c.d, f = c.f;
+    const WsLayout L = ws_layout(w, T);
+    const int path = choose_path(w, T);
+    int launches = 0;
+    auto P = [&](size_t off) { return (void*)(ws + off); };
+    float* logits = (float*)P(L.logits);
+    int32_t* idx = (int32_t*)P(L.topk_idx);
+    float* wts = (float*)P(L.topk_w);
+    int32_t* offsets = (int32_t*)P(L.offsets);
+    int32_t* meta = (int32_t*)P(L.meta);
+    int32_t* active = (int32_t*)P(L.active);
+    int32_t* tiles = (int32_t*)P(L.tiles);
+    int32_t* row2ts = (int32_t*)P(L.row2ts);
+    int32_t* ts2row = (int32_t*)P(L.ts2row);
+    int8_t* xq = (int8_t*)P(L.xq);
+    float* sx = (float*)P(L.sx);
+    int8_t* hq = (int8_t*)P(L.hq);
+    float* sh = (float*)P(L.sh);
+    float* o = (float*)P(L.o);
+    const size_t tk = (size_t)T * k;
+
+    const float* lsrc = given_logits;
+    if (!lsrc) {
+        CUDA_TRY(launch_router_logits(x, c.in_dtype, w->w_router, T, d, E, logits, s));
+        ++launches;
+        lsrc = logits;
+    }
+    CUDA_TRY(launch_topk(lsrc, bias, T, E, k, c.renormalize, idx, wts, dbg ? dbg->logits : nullptr, s));
+    ++launches;
+    CUDA_TRY(launch_permute(idx, T, k, E, capacity_of(c, T), (int32_t*)P(L.hist), offsets, row2ts,
+                            ts2row, meta, active, tiles, s));
+    launches += 2;
+    if (path == MOE_PATH_STREAM) {
+        CUDA_TRY(launch_smooth_quant(x, c.in_dtype, w->inv_s, T, d, k, ts2row, xq, sx, nullptr, s));
+        int32_t* acc1 = (int32_t*)P(L.acc1);
+        CUDA_TRY(launch_stream_gateup(w, T, xq, row2ts, offsets, active, meta, acc1, s));
+        CUDA_TRY(launch_swiglu_requant(w, acc1, row2ts, idx, sx, meta, (int)tk, hq, sh, s));
+        CUDA_TRY(launch_stream_down(w, T, hq, sh, row2ts, wts, offsets, active, meta, o,
+                                    dbg ? dbg->acc2 : nullptr, s));
+        launches += 4;
+        if (dbg && dbg->acc1)
+            CUDA_TRY(cudaMemcpyAsync(dbg->acc1, acc1, tk * 2 * f * 4, cudaMemcpyDeviceToDevice, s));
+    } else {
+        return MOE_ERR_UNSUPPORTED_SHAPE;
+    }
+    CUDA_TRY(launch_combine(o, ts2row, T, k, d, c.out_dtype, y, s));
+    ++launches;
+    if (dbg) {
+        auto cp = [&](void* dst, const void* src, size_t bytes) {
+            return dst ? cudaMemcpyAsync(dst, src, bytes, cudaMemcpyDeviceToDevice, s) : cudaSuccess;
+        };
+        CUDA_TRY(cp(dbg->topk_idx, idx, tk * 4));
+        CUDA_TRY(cp(dbg->topk_w, wts, tk * 4));
+        CUDA_TRY(cp(dbg->offsets, offsets, (size_t)(E + 1) * 4));
+        CUDA_TRY(cp(dbg->row2ts, row2ts, tk * 4));
+        CUDA_TRY(cp(dbg->ts2row, ts2row, tk * 4));
+        CUDA_TRY(cp(dbg->xq, xq, (size_t)T * d));
+        CUDA_TRY(cp(dbg->sx, sx, (size_t)T * 4));
+        CUDA_TRY(cp(dbg->hq, hq, tk * f));
+        CUDA_TRY(cp(dbg->sh, sh, tk * 4));
+        CUDA_TRY(cp(dbg->o, o, tk * d * 4));
+    }
+    const_cast<moe_w8a8_weights*>(w)->last_launches = launches;
+    return MOE_OK;
+}
+
+moe_status moe_w8a8_forward(const moe_w8a8_weights* w, const void* x, int32_t T,
+                            const float* router_bias, const float* router_logits, void* y,
+                            void* workspace, size_t workspace_bytes, const moe_w8a8_debug* dbg,
+                            moe_stream_t stream) {
+    if (!w || T < 0) return MOE_ERR_INVALID_ARG;
+    if (T == 0) return MOE_OK;
+    if (!x || !y || !workspace) return MOE_ERR_INVALID_ARG;
+    if ((uintptr_t)workspace % kAlign) return MOE_ERR_INVALID_ARG;
+    if (choose_path(w, T) == MOE_PATH_TENSOR) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (workspace_bytes < ws_layout(w, T).total) return MOE_ERR_WORKSPACE_TOO_SMALL;
+    return forward_impl(w, x, T, router_bias, router_logits, y, (char*)workspace, dbg,
+                        (cudaStream_t)stream);
+}
+
+moe_status moe_w8a8_forward_host(const moe_w8a8_weights* w, const void* x_host, int32_t T,
+                                 const float* router_bias_host, const float* router_logits_host,
+                                 void* y_host, void* workspace, size_t workspace_bytes,
+                                 moe_stream_t stream) {
+    if (!w || T < 0) return MOE_ERR_INVALID_ARG;
+    if (T == 0) return MOE_OK;
+    if (!x_host || !y_host || !workspace) return MOE_ERR_INVALID_ARG;
+    if ((uintptr_t)workspace % kAlign) return MOE_ERR_INVALID_ARG;
+    if (choose_path(w, T) == MOE_PATH_TENSOR) return MOE_ERR_UNSUPPORTED_SHAPE;
+    const WsLayout L = ws_layout(w, T);
+    if (workspace_bytes < L.total) return MOE_ERR_WORKSPACE_TOO_SMALL;
+    const moe_w8a8_config& c = w->cfg;
+    cudaStream_t s = (cudaStream_t)stream;
+    char* ws = (char*)workspace;
+    const size_t in_b = c.in_dtype == MOE_BF16 ? 2 : 4, out_b = c.out_dtype == MOE_BF16 ? 2 : 4;
+    CUDA_TRY(cudaMemcpyAsync(ws + L.x_stage, x_host, (size_t)T * c.d * in_b, cudaMemcpyHostToDevice, s));
+    const float* lg = nullptr;
+    const float* bs = nullptr;
+    if (router_logits_host) {
+        CUDA_TRY(cudaMemcpyAsync(ws + L.logits_stage, router_logits_host, (size_t)T * c.n_experts * 4,
+                                 cudaMemcpyHostToDevice, s));
+        lg = (const float*)(ws + L.logits_stage);
+    }
+    if (router_bias_host) {
+        CUDA_TRY(cudaMemcpyAsync(ws + L.bias_stage, router_bias_host, (size_t)c.n_experts * 4,
+                                 cudaMemcpyHostToDevice, s));
+        bs = (const float*)(ws + L.bias_stage);
+    }
+    moe_status st = forward_impl(w, ws + L.x_stage, T, bs, lg, ws + L.y_stage, ws, nullptr, s);
+    if (st != MOE_OK) return st;
+    CUDA_TRY(cudaMemcpyAsync(y_host, ws + L.y_stage, (size_t)T * c.d * out_b, cudaMemcpyDeviceToHost, s));
+    return MOE_OK;
+}
+
+moe_status moe_w8a8_set_path(moe_w8a8_weights* w, int32_t path) {
+    if (!w || path < MOE_PATH_AUTO || path > MOE_PATH_TENSOR) return MOE_ERR_INVALID_ARG;
+    w->path = path;
+    return MOE_OK;
+}
+
+moe_status moe_w8a8_set_stream_threshold(moe_w8a8_weights* w, int32_t max_rows) {
+    if (!w || max_rows < 0) return MOE_ERR_INVALID_ARG;
+    w->stream_max_rows = max_rows;
+    return MOE_OK;
+}
+
+moe_status moe_w8a8_get_smooth_scales(const moe_w8a8_weights* w, float* s_host) {
+    if (!w || !s_host) return MOE_ERR_INVALID_ARG;
+    std::memcpy(s_host, w->s_host, (size_t)w->cfg.d * 4);
+    return MOE_OK;
+}
+
+moe_status moe_w8a8_export_weights(const moe_w8a8_weights* w, int8_t* wq_gate, int8_t* wq_up,
+                                   float* sw_gate, float* sw_up, int8_t* wq_down, float* sw_down,
+                                   float* inv_s, moe_stream_t stream) {
+    if (!w) return MOE_ERR_INVALID_ARG;
+    const moe_w8a8_config& c = w->cfg;
+    const int E = c.n_experts, d = c.d, f = c.f;
+    cudaStream_t s = (cudaStream_t)stream;
+    if (wq_gate || wq_up) CUDA_TRY(launch_export_gateup(w->w_gu, E, d, f, wq_gate, wq_up, s));
+    auto cp = [&](void* dst, const void* src, size_t bytes) {
+        return dst ? cudaMemcpyAsync(dst, src, bytes, cudaMemcpyDeviceToDevice, s) : cudaSuccess;
+    };
+    CUDA_TRY(cp(sw_gate, w->sw_gate, (size_t)E * f * 4));
+    CUDA_TRY(cp(sw_up, w->sw_up, (size_t)E * f * 4));
+    CUDA_TRY(cp(wq_down, w->w_dn, (size_t)E * d * f));
+    CUDA_TRY(cp(sw_down, w->sw_dn, (size_t)E * d * 4));
+    CUDA_TRY(cp(inv_s, w->inv_s, (size_t)d * 4));
+    return MOE_OK;
+}
+
+moe_status moe_w8a8_check_status(const moe_w8a8_weights* w, moe_stream_t stream) {
+    if (!w) return MOE_ERR_INVALID_ARG;
+    if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return MOE_ERR_CUDA;
+    int32_t word = 0;
+    if (cudaMemcpy(&word, w->status, 4, cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ERR_CUDA;
+    if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
+    if (word != 0) {
+        if (cudaMemset(w->status, 0, 64) != cudaSuccess) return MOE_ERR_CUDA;
+        return MOE_ERR_TIMEOUT;
+    }
+    return MOE_OK;
+}
+
+void moe_w8a8_destroy(moe_w8a8_weights* w) { free_handle(w); }
+
+int32_t moe_w8a8_last_launch_count(const moe_w8a8_weights* w) { return w ? w->last_launches : 0; }
+
+}  // extern "C"
