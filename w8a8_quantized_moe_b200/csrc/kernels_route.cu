@@ -208,7 +208,7 @@ __global__ void __launch_bounds__(kPermThreads) perm_scatter_kernel(
     }
     const int base = blockIdx.x * kPermChunk;
     for (int r0 = 0; r0 < kPermChunk; r0 += kPermThreads) {
-        for (int i = tid; i < (kPermThreads / 32) * E; i += blockDim.x) (&wcnt[0][0])[i] = 0;
+        for (int i = tid; i < (kPermThreads / 32) * E; i += blockDim.x) wcnt[i / E][i % E] = 0;
         __syncthreads();
         const int i = base + r0 + tid;
         const bool valid = i < n;
@@ -221,8 +221,8 @@ __global__ void __launch_bounds__(kPermThreads) perm_scatter_kernel(
             int rank = running[e] + rank_w;
             for (int w2 = 0; w2 < warp; ++w2) rank += wcnt[w2][e];
             const int pos = pre[e] + rank;
-            if (cap < 0 || pos < cap) {
-                const int row = off[e] + pos;
+            const int row = off[e] + pos;
+            if ((cap < 0 || pos < cap) && row < off[E]) {   // row < R always holds; guard the store
                 ts2row[i] = row;
                 row2ts[row] = i;
             } else {
