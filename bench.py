@@ -1,0 +1,416 @@
+#!/usr/bin/env python
+"""Benchmark of the B200 W8A8 MoE layer: tokens/s and roofline fraction.
+
+One step = one forward of the whole layer (router/top-k, permute, smoothed
+per-token quantisation, grouped expert GEMMs with their epilogues, combine)
+over one batch of synthetic tokens already resident in HBM.  The prepared
+INT8 weights are made once, untimed (the offline preparation step).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload decode|prefill|tiny|large]
+    python bench.py --impl reference ...   # the CPU oracle as the reference arm
+
+Multi-GPU runs (torchrun, one process per GPU) are independent replicas of
+the layer on different token batches; value = all ranks' tokens / the
+slowest rank's device time.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "W8A8 MoE layer tokens/s at T=32 and T=16384; % of HBM / INT8 TC roofline"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+INT8_PER_BF16 = 2.0   # nominal dense ratio (4.5 POPS int8 / 2.25 PFLOPS bf16)
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=500)
+    p.add_argument("--warmup", type=int, default=20)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--workload", default="decode", choices=sorted(synth.WORKLOADS))
+    p.add_argument("--cpu-seconds", type=float, default=10.0,
+                   help="CPU work budget of the oracle baseline sample")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-stage-events", action="store_true")
+    return p.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as fh:
+            return json.load(fh), "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def describe(wl: synth.Workload) -> str:
+    router = "uniform random router logits" if wl.logits_uniform else "router W_g ~N(0,0.02)"
+    if wl.zipf_s:
+        router += f" + Zipf({wl.zipf_s}) expert bias"
+    cap = f", capacity factor {wl.capacity_factor}" if wl.capacity_factor > 0 else ""
+    return (f"{wl.name}: T={wl.T} tokens, d={wl.d}, E={wl.E} experts, top-{wl.k}, SwiGLU f={wl.f}, "
+            f"{'bf16' if wl.in_bf16 else 'fp32'} X with {wl.n_outliers} outlier channels x"
+            f"{wl.outlier_factor:g}, INT8 per-channel weights ~N(0,0.02), alpha {wl.alpha}, "
+            f"{router}{cap}, weight seed {wl.weight_seed}, data seed {wl.data_seed}")
+
+
+# ------------------------------------------------------------------ clocks (NVML, read only)
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons during the timed region."""
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
+
+    def __init__(self, torch_dev: int):
+        self.samples, self.reasons = [], set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thread = None
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            props = torch.cuda.get_device_properties(torch_dev)
+            try:
+                bus = f"{props.pci_domain_id:08X}:{props.pci_bus_id:02X}:{props.pci_device_id:02X}.0"
+                self.h = pynvml.nvmlDeviceGetHandleByPciBusId(bus.encode())
+            except Exception:
+                self.h = pynvml.nvmlDeviceGetHandleByIndex(torch_dev)
+            self.nv = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception as exc:  # no NVML: report that, keep going
+            self.nv = None
+            self.err = str(exc)
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for bit, name in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(0.002)
+
+    def start(self):
+        if self.nv is not None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+
+    def stop(self):
+        self._stop.set()
+        if self._thread:
+            self._thread.join()
+
+    def summary(self):
+        if self.nv is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "note": "NVML unavailable"}
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------------ byte / op model
+
+def algorithmic(wl: synth.Workload, n_active: int, R: int):
+    """Per-step algorithmic bytes and INT8 ops of the layer and of the gate/up
+    stage (the dominant stage): active experts' INT8 weights (3 d f bytes each)
+    and their fp32 scales, X in, Y out, router input; intermediates excluded."""
+    in_b = 2 if wl.in_bf16 else 4
+    w_bytes = n_active * 3 * wl.d * wl.f
+    scales = n_active * (2 * wl.f + wl.d) * 4
+    router = wl.T * wl.E * 4 if wl.logits_uniform else wl.d * wl.E * 4
+    layer = w_bytes + scales + wl.T * wl.d * in_b * 2 + router
+    gemm1 = n_active * 2 * wl.f * wl.d + wl.T * wl.d + R * 2 * wl.f * 4
+    gemm2 = n_active * wl.d * wl.f + R * wl.f + R * wl.d * 4 + n_active * wl.d * 4
+    ops = 2 * R * 3 * wl.d * wl.f
+    return dict(layer_bytes=layer, gemm1_bytes=gemm1, gemm2_bytes=gemm2, int8_ops=ops)
+
+
+# ------------------------------------------------------------------ distributed plumbing
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        backend = "nccl" if args.impl == "ours" else "gloo"
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return world, rank, local
+
+
+def max_over_ranks(v: float, world: int) -> float:
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ------------------------------------------------------------------ oracle timing
+
+def oracle_step(wl, prep, data):
+    """One oracle step on the tokens of `data`: routing of those tokens, the
+    expert FFNs and the combine.  Returns the seconds it took."""
+    import oracle
+    t0 = time.perf_counter()
+    rt = oracle.route(data.x, wl.k, wl.E, w_router=data.w_router, logits=data.router_logits,
+                      bias=data.router_bias, capacity_factor=wl.capacity_factor)
+    oracle.moe_tokens(data.x, prep, rt, out_bf16=wl.in_bf16, debug=False)
+    return time.perf_counter() - t0
+
+
+def oracle_sample_size(wl, prep, budget_s: float, steps: int) -> int:
+    """Tokens per oracle step so that `steps` steps take about budget_s."""
+    probe = synth.make_data(wl, T=1)
+    per_token = max(oracle_step(wl, prep, probe), 1e-4)
+    return int(max(1, min(wl.T, budget_s / (steps * per_token))))
+
+
+def run_reference(args, world, rank):
+    """The reference arm: the CPU oracle, as it stands, on the host cores.
+    Each step is a bounded sample (the first n tokens of the workload's
+    batch, n sized so that warm-up + timed steps take about two minutes)."""
+    if rank != 0:
+        return
+    import oracle
+    wl = synth.WORKLOADS[args.workload]
+    wts = synth.make_weights(wl)
+    prep = oracle.prepare(wts.w_gate, wts.w_up, wts.w_down, wts.calib_x, wl.alpha)
+    n_tok = oracle_sample_size(wl, prep, 120.0, args.steps + args.warmup)
+    data = synth.make_data(wl, T=n_tok)
+    for _ in range(args.warmup):
+        oracle_step(wl, prep, data)
+    secs = sum(oracle_step(wl, prep, data) for _ in range(args.steps))
+    value = n_tok * args.steps / secs
+    sample = (f"{args.steps} steps of the first {n_tok} of the {wl.T} tokens of the {wl.name} "
+              f"workload (routing of the sampled tokens, expert FFNs, combine); preparation untimed")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * secs / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "int8", "data": "synthetic",
+            "config": {"workload": describe(wl), "parallelism": "single CPU thread"},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ our arm
+
+def run_ours(args, world, rank, local):
+    import torch
+
+    import w8a8_quantized_moe_b200 as M
+    from w8a8_quantized_moe_b200 import build as B
+
+    if not os.path.exists(M.LIB_PATH):
+        B.build()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    base = synth.WORKLOADS[args.workload]
+    import dataclasses
+    # replicas: same layer weights on every rank, a different token batch per rank
+    wl = dataclasses.replace(base, data_seed=base.data_seed + 1000 * rank) if rank else base
+
+    # ---- offline preparation (untimed)
+    wts = synth.make_weights(wl)
+    data = synth.make_data(wl)
+    cfg = M.make_config(wl.d, wl.f, wl.E, wl.k, wl.alpha, wl.capacity_factor, True,
+                        M.MOE_BF16 if wl.in_bf16 else M.MOE_F32,
+                        M.MOE_BF16 if wl.in_bf16 else M.MOE_F32)
+    act = torch.bfloat16 if wl.in_bf16 else torch.float32
+
+    def host_act(v32):
+        if wl.in_bf16:
+            return torch.from_numpy(synth.f32_to_bf16_bits(v32).view(np.int16)).view(torch.bfloat16)
+        return torch.from_numpy(v32)
+
+    cal = host_act(wts.calib_x).to(dev)
+    ax = torch.zeros(wl.d, dtype=torch.float32, device=dev)
+    M.moe_w8a8_calibrate_absmax(cal, ax)
+    wg, wu, wd = (torch.from_numpy(a).to(dev) for a in (wts.w_gate, wts.w_up, wts.w_down))
+    wr = torch.from_numpy(data.w_router).to(dev)
+    W = M.moe_w8a8_prepare(cfg, wg, wu, wd, wr, ax)
+    del wg, wu, wd, cal
+    torch.cuda.empty_cache()
+
+    T = wl.T
+    x = host_act(data.x).to(dev) if not wl.in_bf16 else \
+        torch.from_numpy(data.x_bits.view(np.int16)).view(torch.bfloat16).to(dev)
+    logits = torch.from_numpy(data.router_logits).to(dev) if data.router_logits is not None else None
+    bias = torch.from_numpy(data.router_bias).to(dev) if data.router_bias is not None else None
+    y = torch.empty((T, wl.d), dtype=act, device=dev)
+    ws = torch.empty(M.moe_w8a8_workspace_size(W, T), dtype=torch.uint8, device=dev)
+
+    # routing statistics of this batch (for the byte model): one debug forward
+    offs = torch.empty(wl.E + 1, dtype=torch.int32, device=dev)
+    M.moe_w8a8_forward(W, x, T, bias, logits, y, ws, {"offsets": offs})
+    counts = np.diff(offs.cpu().numpy())
+    n_active, R = int((counts > 0).sum()), int(counts.sum())
+    alg = algorithmic(wl, n_active, R)
+
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(args.warmup):
+        M.moe_w8a8_forward(W, x, T, bias, logits, y, ws)
+    torch.cuda.synchronize(dev)
+
+    # ---- timed region: K steps, device time, max over ranks
+    K = args.steps
+    stage_events = not args.no_stage_events
+    if stage_events:
+        M.moe_w8a8_profile_start(W, K)
+    clocks = ClockSampler(local)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    clocks.start()
+    e0.record(stream)
+    for _ in range(K):
+        M.moe_w8a8_forward(W, x, T, bias, logits, y, ws)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    clocks.stop()
+    barrier(world)
+    launches_per_step = M.moe_w8a8_last_launch_count(W)
+    ms_local = e0.elapsed_time(e1)
+    ms_total = max_over_ranks(ms_local, world)
+    M.moe_w8a8_check_status(W)
+    stages = None
+    if stage_events:
+        st = M.moe_w8a8_profile_read(W, K)
+        M.moe_w8a8_profile_stop(W)
+        stages = {M.STAGE_NAMES[i]: float(st[:, i].mean()) for i in range(M.MOE_N_STAGES)}
+
+    value = world * T * K / (ms_total / 1e3)
+
+    # ---- end to end through the C ABI with host buffers (H2D + forward + D2H per step)
+    e2e = None
+    if not args.no_e2e:
+        if wl.in_bf16:
+            xh = torch.from_numpy(data.x_bits.view(np.int16)).pin_memory()
+            yh = torch.empty((T, wl.d), dtype=torch.int16).pin_memory()
+        else:
+            xh = torch.from_numpy(data.x).pin_memory()
+            yh = torch.empty((T, wl.d), dtype=torch.float32).pin_memory()
+        lh = torch.from_numpy(data.router_logits).pin_memory() if data.router_logits is not None else None
+        bh = torch.from_numpy(data.router_bias).pin_memory() if data.router_bias is not None else None
+        for _ in range(max(3, args.warmup)):
+            M.moe_w8a8_forward_host(W, xh, T, bh, lh, yh, ws)
+        torch.cuda.synchronize(dev)
+        barrier(world)
+        e0.record(stream)
+        for _ in range(K):
+            M.moe_w8a8_forward_host(W, xh, T, bh, lh, yh, ws)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier(world)
+        ms_e2e = max_over_ranks(e0.elapsed_time(e1), world)
+        h2d = xh.numel() * xh.element_size() + (lh.numel() * 4 if lh is not None else 0) + \
+            (bh.numel() * 4 if bh is not None else 0)
+        e2e = {"value": world * T * K / (ms_e2e / 1e3), "unit": "tokens/s",
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(yh.numel() * yh.element_size())}
+
+    if rank != 0:
+        return
+
+    # ---- roofline of the dominant stage, from the live stage events
+    peaks, peak_src = load_peaks()
+    roof = None
+    if stages:
+        dom = max(("gemm1", "gemm2"), key=lambda s: stages[s])
+        dom_ms = stages[dom]
+        bytes_dom = alg[f"{dom}_bytes"]
+        achieved = bytes_dom / (dom_ms / 1e3) / 1e9
+        roof = {"bound": "hbm", "kernel": f"{dom} ({'stream_gateup' if dom == 'gemm1' else 'stream_down'})",
+                "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                "peak_source": f"hbm_gbs of {peak_src}",
+                "algorithmic_bytes_per_launch": bytes_dom, "launch_ms": dom_ms}
+    layer_gbs = alg["layer_bytes"] / (ms_total / K / 1e3) / 1e9
+
+    # ---- CPU baseline: the oracle on a bounded sample of this workload (rank 0, N = 1)
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        import oracle
+        prep = oracle.prepare(wts.w_gate, wts.w_up, wts.w_down, wts.calib_x, wl.alpha)
+        n_tok = min(wl.T, 32)
+        sdata = synth.make_data(wl, T=n_tok)
+        secs, n = 0.0, 0
+        while n == 0 or secs < args.cpu_seconds:
+            secs += oracle_step(wl, prep, sdata)
+            n += 1
+        tokens = n * n_tok
+        cpu = {"value": tokens / secs, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+               "sample": f"{n} steps of the first {n_tok} of the {wl.T} tokens of the {wl.name} workload "
+                         f"({secs:.1f} s of single-thread CPU time; preparation untimed)"}
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": ms_total / K, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "int8", "data": "synthetic",
+        "config": {"workload": describe(wl), "T": T, "d": wl.d, "E": wl.E, "k": wl.k, "f": wl.f,
+                   "alpha": wl.alpha, "active_experts": n_active, "rows": R,
+                   "l2": f"inputs larger than L2: {alg['gemm1_bytes'] / 1e9 + 0:.2f} GB gate/up + "
+                         f"{alg['gemm2_bytes'] / 1e9:.2f} GB down INT8 weights streamed per step "
+                         f"vs 126 MB L2; no flush",
+                   "parallelism": "replicas" if world > 1 else "single GPU",
+                   "layer_bytes_per_step": alg["layer_bytes"], "layer_gbs": layer_gbs,
+                   "layer_hbm_frac": layer_gbs / peaks["hbm_gbs"],
+                   "int8_ops_per_step": alg["int8_ops"]},
+        "roofline": roof,
+        "stages_ms": stages,
+        "e2e": e2e,
+        "gpu_launches": launches_per_step * K,
+        "clocks": clocks.summary(),
+        "cpu_baseline": cpu,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    world, rank, local = dist_setup(args)
+    try:
+        if args.impl == "reference":
+            run_reference(args, world, rank)
+        else:
+            run_ours(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

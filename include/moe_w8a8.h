@@ -197,6 +197,39 @@ const char* moe_status_string(moe_status s);
 /* Number of kernels the last successful forward on this handle enqueued. */
 int32_t moe_w8a8_last_launch_count(const moe_w8a8_weights* w);
 
+
+/* Stages of one forward, for per-stage timing. */
+enum {
+    MOE_STAGE_ROUTER = 0,   /* router logits X W_router (skipped when logits are given) */
+    MOE_STAGE_TOPK = 1,     /* top-k + gate softmax                                     */
+    MOE_STAGE_PERMUTE = 2,  /* histogram + stable scatter by expert                     */
+    MOE_STAGE_QUANT = 3,    /* smoothing + per-token INT8 quantisation                  */
+    MOE_STAGE_GEMM1 = 4,    /* gate/up grouped GEMM                                     */
+    MOE_STAGE_REQUANT = 5,  /* SwiGLU + per-row INT8 requantisation (when not fused)    */
+    MOE_STAGE_GEMM2 = 6,    /* down grouped GEMM + dequant x routing weight             */
+    MOE_STAGE_COMBINE = 7,  /* un-sort + weighted sum                                   */
+    MOE_N_STAGES = 8
+};
+
+/*
+ * Measurement aid: from now on, record a CUDA event pair around every stage
+ * of the next max_forwards forwards on this handle, on the forward's stream
+ * (a stage that does not run records an empty interval).  Allocates the
+ * events here, never inside a forward.
+ */
+moe_status moe_w8a8_profile_start(moe_w8a8_weights* w, int32_t max_forwards);
+
+/* Synchronise the recorded events and write ms_host[i * MOE_N_STAGES + s],
+ * the time of stage s in recorded forward i, for up to `capacity` forwards.
+ * Returns the number of forwards written (negative on a CUDA error). */
+int32_t moe_w8a8_profile_read(moe_w8a8_weights* w, float* ms_host, int32_t capacity);
+
+/* Stop recording and free the events. */
+moe_status moe_w8a8_profile_stop(moe_w8a8_weights* w);
+
+/* Static name of a stage ("router", "topk", ...), or "?" . */
+const char* moe_w8a8_stage_name(int32_t stage);
+
 #ifdef __cplusplus
 }
 #endif

@@ -35,8 +35,11 @@ EXPORTS = (
     "moe_w8a8_forward", "moe_w8a8_forward_host", "moe_w8a8_set_path",
     "moe_w8a8_set_stream_threshold", "moe_w8a8_get_smooth_scales", "moe_w8a8_export_weights",
     "moe_w8a8_check_status", "moe_w8a8_destroy", "moe_status_string",
-    "moe_w8a8_last_launch_count",
+    "moe_w8a8_last_launch_count", "moe_w8a8_profile_start", "moe_w8a8_profile_read",
+    "moe_w8a8_profile_stop", "moe_w8a8_stage_name",
 )
+
+MOE_N_STAGES = 8
 
 
 class MoeError(RuntimeError):
@@ -87,6 +90,10 @@ def lib():
             "moe_w8a8_destroy": ([vp], None),
             "moe_status_string": ([i32], ctypes.c_char_p),
             "moe_w8a8_last_launch_count": ([vp], i32),
+            "moe_w8a8_profile_start": ([vp, i32], i32),
+            "moe_w8a8_profile_read": ([vp, vp, i32], i32),
+            "moe_w8a8_profile_stop": ([vp], i32),
+            "moe_w8a8_stage_name": ([i32], ctypes.c_char_p),
         }
         for name, (args, res) in sig.items():
             fn = getattr(L, name)
@@ -280,3 +287,28 @@ def moe_w8a8_check_status(w: Weights, stream=None):
 
 def moe_w8a8_last_launch_count(w: Weights) -> int:
     return int(lib().moe_w8a8_last_launch_count(w.handle))
+
+
+def moe_w8a8_profile_start(w: Weights, max_forwards: int):
+    _check(lib().moe_w8a8_profile_start(w.handle, int(max_forwards)), "moe_w8a8_profile_start")
+
+
+def moe_w8a8_profile_read(w: Weights, capacity: int):
+    """Per-stage milliseconds of the recorded forwards: numpy [n][MOE_N_STAGES]."""
+    import numpy as np
+    out = np.zeros((capacity, MOE_N_STAGES), dtype=np.float32)
+    n = lib().moe_w8a8_profile_read(w.handle, ctypes.c_void_p(out.ctypes.data), int(capacity))
+    if n < 0:
+        raise MoeError(MOE_ERR_CUDA, "moe_w8a8_profile_read")
+    return out[:n]
+
+
+def moe_w8a8_profile_stop(w: Weights):
+    _check(lib().moe_w8a8_profile_stop(w.handle), "moe_w8a8_profile_stop")
+
+
+def moe_w8a8_stage_name(stage: int) -> str:
+    return lib().moe_w8a8_stage_name(int(stage)).decode()
+
+
+STAGE_NAMES = ("router", "topk", "permute", "quant", "gemm1", "requant", "gemm2", "combine")

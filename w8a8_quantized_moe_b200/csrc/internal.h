@@ -30,6 +30,10 @@ struct moe_w8a8_weights {
     CUtensorMap tm_w_gu;
     CUtensorMap tm_w_dn;
     bool tmaps_ok;
+    // per-stage event timing (measurement aid)
+    cudaEvent_t* prof_events;   // [prof_max][MOE_N_STAGES][2]
+    int prof_max;
+    int prof_n;
 };
 
 namespace moe {

@@ -42,8 +42,17 @@ int choose_path(const moe_w8a8_weights* w, int T) {
     return (int64_t)T * w->cfg.top_k <= w->stream_max_rows ? MOE_PATH_STREAM : MOE_PATH_TENSOR;
 }
 
+void prof_free(moe_w8a8_weights* w) {
+    if (!w->prof_events) return;
+    for (int i = 0; i < w->prof_max * MOE_N_STAGES * 2; ++i) cudaEventDestroy(w->prof_events[i]);
+    delete[] w->prof_events;
+    w->prof_events = nullptr;
+    w->prof_max = w->prof_n = 0;
+}
+
 void free_handle(moe_w8a8_weights* w) {
     if (!w) return;
+    prof_free(w);
     cudaFree(w->w_gu);
     cudaFree(w->w_dn);
     cudaFree(w->sw_gate);
@@ -241,33 +250,58 @@ static moe_status forward_impl(const moe_w8a8_weights* w, const void* x, int T, 
     float* sh = (float*)P(L.sh);
     float* o = (float*)P(L.o);
     const size_t tk = (size_t)T * k;
+    moe_w8a8_weights* mw = const_cast<moe_w8a8_weights*>(w);
+    const bool prof = w->prof_events && w->prof_n < w->prof_max;
+    auto mark = [&](int stage, int edge) {
+        if (prof) cudaEventRecord(w->prof_events[(w->prof_n * MOE_N_STAGES + stage) * 2 + edge], s);
+    };
+    auto empty_stage = [&](int stage) { mark(stage, 0); mark(stage, 1); };
 
     const float* lsrc = given_logits;
     if (!lsrc) {
+        mark(MOE_STAGE_ROUTER, 0);
         CUDA_TRY(launch_router_logits(x, c.in_dtype, w->w_router, T, d, E, logits, s));
+        mark(MOE_STAGE_ROUTER, 1);
         ++launches;
         lsrc = logits;
+    } else {
+        empty_stage(MOE_STAGE_ROUTER);
     }
+    mark(MOE_STAGE_TOPK, 0);
     CUDA_TRY(launch_topk(lsrc, bias, T, E, k, c.renormalize, idx, wts, dbg ? dbg->logits : nullptr, s));
+    mark(MOE_STAGE_TOPK, 1);
     ++launches;
+    mark(MOE_STAGE_PERMUTE, 0);
     CUDA_TRY(launch_permute(idx, T, k, E, capacity_of(c, T), (int32_t*)P(L.hist), offsets, row2ts,
                             ts2row, meta, active, tiles, s));
+    mark(MOE_STAGE_PERMUTE, 1);
     launches += 2;
     if (path == MOE_PATH_STREAM) {
+        mark(MOE_STAGE_QUANT, 0);
         CUDA_TRY(launch_smooth_quant(x, c.in_dtype, w->inv_s, T, d, k, ts2row, xq, sx, nullptr, s));
+        mark(MOE_STAGE_QUANT, 1);
         int32_t* acc1 = (int32_t*)P(L.acc1);
+        mark(MOE_STAGE_GEMM1, 0);
         CUDA_TRY(launch_stream_gateup(w, T, xq, row2ts, offsets, active, meta, acc1, s));
+        mark(MOE_STAGE_GEMM1, 1);
+        mark(MOE_STAGE_REQUANT, 0);
         CUDA_TRY(launch_swiglu_requant(w, acc1, row2ts, idx, sx, meta, (int)tk, hq, sh, s));
+        mark(MOE_STAGE_REQUANT, 1);
+        mark(MOE_STAGE_GEMM2, 0);
         CUDA_TRY(launch_stream_down(w, T, hq, sh, row2ts, wts, offsets, active, meta, o,
                                     dbg ? dbg->acc2 : nullptr, s));
+        mark(MOE_STAGE_GEMM2, 1);
         launches += 4;
         if (dbg && dbg->acc1)
             CUDA_TRY(cudaMemcpyAsync(dbg->acc1, acc1, tk * 2 * f * 4, cudaMemcpyDeviceToDevice, s));
     } else {
         return MOE_ERR_UNSUPPORTED_SHAPE;
     }
+    mark(MOE_STAGE_COMBINE, 0);
     CUDA_TRY(launch_combine(o, ts2row, T, k, d, c.out_dtype, y, s));
+    mark(MOE_STAGE_COMBINE, 1);
     ++launches;
+    if (prof) ++mw->prof_n;
     if (dbg) {
         auto cp = [&](void* dst, const void* src, size_t bytes) {
             return dst ? cudaMemcpyAsync(dst, src, bytes, cudaMemcpyDeviceToDevice, s) : cudaSuccess;
@@ -283,7 +317,7 @@ static moe_status forward_impl(const moe_w8a8_weights* w, const void* x, int T, 
         CUDA_TRY(cp(dbg->sh, sh, tk * 4));
         CUDA_TRY(cp(dbg->o, o, tk * d * 4));
     }
-    const_cast<moe_w8a8_weights*>(w)->last_launches = launches;
+    mw->last_launches = launches;
     return MOE_OK;
 }
 
@@ -386,6 +420,51 @@ moe_status moe_w8a8_check_status(const moe_w8a8_weights* w, moe_stream_t stream)
 }
 
 void moe_w8a8_destroy(moe_w8a8_weights* w) { free_handle(w); }
+
+moe_status moe_w8a8_profile_start(moe_w8a8_weights* w, int32_t max_forwards) {
+    if (!w || max_forwards <= 0) return MOE_ERR_INVALID_ARG;
+    prof_free(w);
+    const int n = max_forwards * MOE_N_STAGES * 2;
+    w->prof_events = new cudaEvent_t[n];
+    for (int i = 0; i < n; ++i) {
+        if (cudaEventCreate(&w->prof_events[i]) != cudaSuccess) {
+            for (int j = 0; j < i; ++j) cudaEventDestroy(w->prof_events[j]);
+            delete[] w->prof_events;
+            w->prof_events = nullptr;
+            return MOE_ERR_CUDA;
+        }
+    }
+    w->prof_max = max_forwards;
+    w->prof_n = 0;
+    return MOE_OK;
+}
+
+int32_t moe_w8a8_profile_read(moe_w8a8_weights* w, float* ms_host, int32_t capacity) {
+    if (!w || !ms_host || capacity < 0 || !w->prof_events) return -1;
+    const int n = w->prof_n < capacity ? w->prof_n : capacity;
+    for (int i = 0; i < n; ++i)
+        for (int st = 0; st < MOE_N_STAGES; ++st) {
+            cudaEvent_t a = w->prof_events[(i * MOE_N_STAGES + st) * 2];
+            cudaEvent_t b = w->prof_events[(i * MOE_N_STAGES + st) * 2 + 1];
+            if (cudaEventSynchronize(b) != cudaSuccess) return -1;
+            float ms = 0.0f;
+            if (cudaEventElapsedTime(&ms, a, b) != cudaSuccess) return -1;
+            ms_host[i * MOE_N_STAGES + st] = ms;
+        }
+    return n;
+}
+
+moe_status moe_w8a8_profile_stop(moe_w8a8_weights* w) {
+    if (!w) return MOE_ERR_INVALID_ARG;
+    prof_free(w);
+    return MOE_OK;
+}
+
+const char* moe_w8a8_stage_name(int32_t stage) {
+    static const char* names[MOE_N_STAGES] = {"router", "topk", "permute", "quant",
+                                              "gemm1", "requant", "gemm2", "combine"};
+    return (stage >= 0 && stage < MOE_N_STAGES) ? names[stage] : "?";
+}
 
 int32_t moe_w8a8_last_launch_count(const moe_w8a8_weights* w) { return w ? w->last_launches : 0; }
 
