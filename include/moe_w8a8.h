@@ -162,6 +162,38 @@ moe_status moe_w8a8_forward_host(const moe_w8a8_weights* w, const void* x_host, 
                                  void* y_host, void* workspace, size_t workspace_bytes,
                                  moe_stream_t stream);
 
+/*
+ * moe_w8a8_forward for callers that cannot allocate device memory.
+ *
+ * No counterpart on the pages: this entry point exists for library users,
+ * not for the method.  Some callers may not call cudaMalloc at all on their
+ * request path: a serving process that plans every device byte at start-up
+ * and forbids allocation afterwards, or a plugin hosted by a framework that
+ * owns the device allocator and gives the plugin no allocation hook.  Such a
+ * caller passes only its inputs and outputs; the scratch memory comes from a
+ * fixed array compiled into this library (MOE_NOALLOC_SCRATCH_BYTES bytes of
+ * device memory, held on every GPU that loads the library until the process
+ * exits).  Nothing is allocated by this call: no cudaMalloc, no cudaFree, no
+ * allocating library routine.
+ *
+ *   x, router_bias, router_logits, y: as for moe_w8a8_forward (device).
+ * T is limited by the array: a call whose moe_w8a8_workspace_size(w, T)
+ * exceeds MOE_NOALLOC_SCRATCH_BYTES returns MOE_ERR_WORKSPACE_TOO_SMALL and
+ * enqueues nothing (for the d=4096, E=64, top-4, f=1536 decode layer that is
+ * T up to 59 tokens).
+ * The first call on a device looks up the array's device address with that
+ * device current (cudaGetSymbolAddress) and caches it; make that first call
+ * before any stream capture.  Every call on a device shares the one array,
+ * which keeps the previous call's contents (the forward writes every scratch
+ * word it later reads, so nothing needs clearing); calls that overlap on the
+ * GPU (different streams, or different threads) race on it and must be
+ * serialised by the caller.
+ */
+#define MOE_NOALLOC_SCRATCH_BYTES (8u << 20)
+moe_status moe_w8a8_forward_noalloc(const moe_w8a8_weights* w, const void* x, int32_t T,
+                                    const float* router_bias, const float* router_logits,
+                                    void* y, moe_stream_t stream);
+
 /* Select the expert GEMM path (MOE_PATH_*). */
 moe_status moe_w8a8_set_path(moe_w8a8_weights* w, int32_t path);
 

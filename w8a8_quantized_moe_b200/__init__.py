@@ -36,8 +36,10 @@ EXPORTS = (
     "moe_w8a8_set_stream_threshold", "moe_w8a8_get_smooth_scales", "moe_w8a8_export_weights",
     "moe_w8a8_check_status", "moe_w8a8_destroy", "moe_status_string",
     "moe_w8a8_last_launch_count", "moe_w8a8_profile_start", "moe_w8a8_profile_read",
-    "moe_w8a8_profile_stop", "moe_w8a8_stage_name",
+    "moe_w8a8_profile_stop", "moe_w8a8_stage_name", "moe_w8a8_forward_noalloc",
 )
+
+MOE_NOALLOC_SCRATCH_BYTES = 8 << 20
 
 MOE_N_STAGES = 8
 
@@ -94,6 +96,7 @@ def lib():
             "moe_w8a8_profile_read": ([vp, vp, i32], i32),
             "moe_w8a8_profile_stop": ([vp], i32),
             "moe_w8a8_stage_name": ([i32], ctypes.c_char_p),
+            "moe_w8a8_forward_noalloc": ([vp, vp, i32, vp, vp, vp, vp], i32),
         }
         for name, (args, res) in sig.items():
             fn = getattr(L, name)
@@ -312,3 +315,14 @@ def moe_w8a8_stage_name(stage: int) -> str:
 
 
 STAGE_NAMES = ("router", "topk", "permute", "quant", "gemm1", "requant", "gemm2", "combine")
+
+
+def moe_w8a8_forward_noalloc(w: Weights, x, T: int, router_bias, router_logits, y, stream=None):
+    """Forward for callers that cannot allocate: scratch comes from the
+    library's fixed device array (see the header); no workspace argument."""
+    torch = _torch()
+    _check(lib().moe_w8a8_forward_noalloc(
+        w.handle, _dev_ptr(x, _act_dtype(w.cfg.in_dtype), "x"), int(T),
+        _dev_ptr(router_bias, torch.float32, "router_bias", True),
+        _dev_ptr(router_logits, torch.float32, "router_logits", True),
+        _dev_ptr(y, _act_dtype(w.cfg.out_dtype), "y"), _stream(stream)), "moe_w8a8_forward_noalloc")

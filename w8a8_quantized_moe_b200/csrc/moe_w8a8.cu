@@ -6,6 +6,7 @@
 #include <cmath>
 #include <cstdlib>
 #include <cstring>
+#include <mutex>
 #include <vector>
 
 #include "internal.h"
@@ -469,3 +470,48 @@ const char* moe_w8a8_stage_name(int32_t stage) {
 int32_t moe_w8a8_last_launch_count(const moe_w8a8_weights* w) { return w ? w->last_launches : 0; }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Forward without any allocation: the scratch is a fixed device array in this
+// file.  In host code `g_noalloc_scratch` names a host-side stand-in, not a
+// device address, so its device address is looked up once per device (with
+// that device current) and only that address is handed to the kernels.
+// ---------------------------------------------------------------------------
+namespace {
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[MOE_NOALLOC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mutex;
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of the scratch array on the current device (set-up on the
+// first call per device); nullptr if the lookup fails.
+void* noalloc_scratch_for_current_device() {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    if (!g_noalloc_ptr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return nullptr;
+        g_noalloc_ptr[dev] = p;
+    }
+    return g_noalloc_ptr[dev];
+}
+
+}  // namespace
+
+extern "C" moe_status moe_w8a8_forward_noalloc(const moe_w8a8_weights* w, const void* x, int32_t T,
+                                               const float* router_bias,
+                                               const float* router_logits, void* y,
+                                               moe_stream_t stream) {
+    if (!w || T < 0) return MOE_ERR_INVALID_ARG;
+    if (T == 0) return MOE_OK;
+    if (!x || !y) return MOE_ERR_INVALID_ARG;
+    if (choose_path(w, T) == MOE_PATH_TENSOR) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (ws_layout(w, T).total > (size_t)MOE_NOALLOC_SCRATCH_BYTES) return MOE_ERR_WORKSPACE_TOO_SMALL;
+    void* scratch = noalloc_scratch_for_current_device();
+    if (!scratch) return MOE_ERR_CUDA;
+    return forward_impl(w, x, T, router_bias, router_logits, y, (char*)scratch, nullptr,
+                        (cudaStream_t)stream);
+}
