@@ -68,8 +68,13 @@ def gpu_prepare(wl: synth.Workload, wts: synth.LayerWeights, capacity_factor=Non
     return W
 
 
+DBG_ALL = ("logits", "topk_idx", "topk_w", "offsets", "row2ts", "ts2row", "xq", "sx", "acc1", "hq",
+           "sh", "acc2", "o")
+DBG_SMALL = ("logits", "topk_idx", "topk_w", "offsets", "row2ts", "ts2row", "xq", "sx", "hq", "sh")
+
+
 def gpu_forward(W, wl: synth.Workload, data: synth.LayerData, debug=True, path=None, T=None,
-                router_w=None):
+                fields=DBG_ALL):
     """Run forward; returns (y as fp32 numpy, dict of debug numpy arrays)."""
     import w8a8_quantized_moe_b200 as M
     torch = torch_mod()
@@ -99,6 +104,7 @@ def gpu_forward(W, wl: synth.Workload, data: synth.LayerData, debug=True, path=N
                    sh=torch.empty(tk, dtype=torch.float32, device=dev),
                    acc2=torch.zeros((tk, wl.d), dtype=torch.int32, device=dev),
                    o=torch.empty((tk, wl.d), dtype=torch.float32, device=dev))
+        dbg = {k: v for k, v in dbg.items() if k in fields}
     M.moe_w8a8_forward(W, x, T, bias, logits, y, ws, dbg)
     M.moe_w8a8_check_status(W)
     out = {}
@@ -164,7 +170,8 @@ def compare_stages(wl, rt: oracle.Routing, dbg: dict, y_gpu, y_ref, odbg: dict, 
             assert dbg["sh"][row] == odbg["sh"][i, s], f"h scale differs at t={t} s={s}"
             if "acc2" in dbg and dbg["acc2"] is not None:
                 assert np.array_equal(dbg["acc2"][row], odbg["acc2"][i, s]), f"acc2 differs at t={t} s={s}"
-            assert np.array_equal(dbg["o"][row], odbg["o"][i, s]), f"expert output differs at t={t} s={s}"
+            if "o" in dbg:
+                assert np.array_equal(dbg["o"][row], odbg["o"][i, s]), f"expert output differs at t={t} s={s}"
     err = max_rel_err(y_gpu[tokens], y_ref)
     assert err <= TOL[wl.in_bf16], f"output max relative error {err}"
     return err

@@ -21,7 +21,8 @@ def M():
     return mod
 
 
-def run_case(M, wl, wts=None, data=None, tokens=None, path=None, W=None, prep=None):
+def run_case(M, wl, wts=None, data=None, tokens=None, path=None, W=None, prep=None,
+             fields=H.DBG_ALL):
     wts = synth.make_weights(wl) if wts is None else wts
     data = synth.make_data(wl) if data is None else data
     if prep is None:
@@ -30,7 +31,7 @@ def run_case(M, wl, wts=None, data=None, tokens=None, path=None, W=None, prep=No
         W = H.gpu_prepare(wl, wts)
         H.compare_prepare(W, prep)
     rt = H.oracle_route(wl, data)
-    y, dbg = H.gpu_forward(W, wl, data, path=path)
+    y, dbg = H.gpu_forward(W, wl, data, path=path, fields=fields)
     T = data.x.shape[0]
     toks = np.arange(T) if tokens is None else np.asarray(tokens)
     y_ref, odbg = oracle.moe_tokens(data.x, prep, rt, tokens=toks, out_bf16=wl.in_bf16)
@@ -180,3 +181,75 @@ def test_error_statuses(M, decode_setup):
         M.moe_w8a8_prepare(bad, z, z, z, z, z)
     assert e.value.status == M.MOE_ERR_INVALID_ARG
     M.moe_w8a8_check_status(W)
+
+
+# ----------------------------------------------------------------- tensor-core (tcgen05) path
+
+@pytest.mark.parametrize("T", [64, 37, 1, 200, 1000])
+def test_tensor_path_tiny_layer(M, T):
+    wl = dataclasses.replace(synth.WORKLOADS["tiny"], T=T, data_seed=200 + T)
+    err, y, y_ref, _, _ = run_case(M, wl, path=M.MOE_PATH_TENSOR)
+    assert np.array_equal(y, y_ref)
+
+
+def test_tensor_path_decode_layer(M, decode_setup):
+    wl, wts, prep, W = decode_setup
+    try:
+        err, y, y_ref, rt, _ = run_case(M, wl, wts=wts, W=W, prep=prep, path=M.MOE_PATH_TENSOR)
+        assert np.array_equal(y, y_ref)
+    finally:
+        M.moe_w8a8_set_path(W, M.MOE_PATH_AUTO)
+
+
+def test_tensor_path_capacity_and_skew(M):
+    T, E = 300, 8
+    logits = synth.uniform(41, 1, (T, E))
+    logits[:, 5] += 1.0
+    wl, data = _tiny_with_logits(T, logits, capacity_factor=1.25)
+    _, _, _, rt, _ = run_case(M, wl, data=data, path=M.MOE_PATH_TENSOR)
+    assert (rt.ts2row < 0).sum() > 0
+
+
+def test_tensor_path_all_tokens_one_expert(M):
+    T, E = 700, 8
+    logits = np.zeros((T, E), np.float32)
+    logits[:, 2] = 3.0
+    logits[:, 7] = 2.0
+    wl, data = _tiny_with_logits(T, logits)
+    run_case(M, wl, data=data, path=M.MOE_PATH_TENSOR)
+
+
+def test_tensor_path_determinism(M):
+    wl = dataclasses.replace(synth.WORKLOADS["tiny"], T=500, data_seed=77)
+    wts = synth.make_weights(wl)
+    data = synth.make_data(wl)
+    W = H.gpu_prepare(wl, wts)
+    y1, d1 = H.gpu_forward(W, wl, data, path=M.MOE_PATH_TENSOR)
+    y2, d2 = H.gpu_forward(W, wl, data, path=M.MOE_PATH_TENSOR)
+    assert np.array_equal(y1, y2)
+    for k in d1:
+        assert np.array_equal(d1[k], d2[k]), k
+
+
+@pytest.fixture(scope="module")
+def prefill_setup(M, decode_setup):
+    _, wts, prep, _ = decode_setup      # the prefill layer reuses the decode layer's expert weights
+    wl = synth.WORKLOADS["prefill"]
+    W = H.gpu_prepare(wl, wts)
+    return wl, wts, prep, W
+
+
+def test_prefill_layer_sampled_tokens(M, prefill_setup):
+    """Full-size prefill layer (T=16384) in the launch configuration the bench
+    times (tensor path); every routing / permutation entry is checked, the
+    expert FFN and output on a spread sample of tokens."""
+    wl, wts, prep, W = prefill_setup
+    H.compare_prepare(W, prep)
+    data = synth.make_data(wl)
+    toks = np.unique(np.concatenate([np.arange(0, 16), np.arange(wl.T - 16, wl.T),
+                                     np.linspace(0, wl.T - 1, 32).astype(np.int64)]))
+    err, y, y_ref, rt, dbg = run_case(M, wl, wts=wts, data=data, W=W, prep=prep, tokens=toks,
+                                      fields=H.DBG_SMALL)
+    assert np.array_equal(y[toks], y_ref)
+    counts = np.diff(rt.offsets)
+    assert counts.min() > 600 and counts.max() < 1500    # near-balanced loads

@@ -1,0 +1,596 @@
+// Grouped INT8 GEMMs on the 5th-generation tensor cores (tcgen05, kind::i8)
+// for the expert FFN of the W8A8 MoE layer ("MiniMax-M3 W8A8 on K100AI",
+// s1.2: INT8 x INT8 on the INT8 GEMM path with integer accumulation; s4.3:
+// fuse the expert FFN and stay in INT8 between the two matmuls; "Day0
+// adaptation of ultra-large model inference", section 4: grouped GEMM over the
+// expert-sorted tokens).
+//
+// One persistent kernel per GEMM, one CTA per SM.  Tiles of 128 sorted rows
+// (one expert) x 256 output channels, K in blocks of 128 bytes:
+//   warp 0      TMA producer: A tile (128 x 128 B) and B tile (256 x 128 B) per
+//               k-block into a 4-stage shared-memory ring (128-byte swizzle)
+//   warp 1      allocates 512 TMEM columns; one thread issues tcgen05.mma
+//               (M=128, N=256, K=32 per instruction) into one of two 256-column
+//               INT32 accumulators, double-buffered so the epilogue of one tile
+//               runs under the main loop of the next
+//   warps 2..9  epilogue: tcgen05.ld of their 32-lane quarter of the
+//               accumulator, dequantisation and the fused math, global stores
+// GEMM1 epilogue: g, u dequantised (per-token x per-channel scales), h = silu(g)
+// u written in fp32 with per-row partial maxima; the CTA that completes the last
+// column tile of a 128-row tile requantises those rows to INT8 (row max over all
+// f channels) -- completion is counted with an atomic, nothing waits on another
+// CTA.  GEMM2 epilogue: o = acc2 sh sw w in fp32 per sorted row.
+//
+// Every wait on an mbarrier is bounded by the global timer; when a wait runs
+// out the kernel records MOE_ERR_TIMEOUT in the status word, stops issuing
+// work, waits (bounded) for its copies and MMAs in flight, frees its TMEM and
+// returns.
+#include <cuda.h>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace moe {
+namespace {
+
+constexpr int BM = 128, BN = 256, BK = 128;
+constexpr int kStages = 4;
+constexpr int kABytes = BM * BK;                  // 16 KB
+constexpr int kBBytes = BN * BK;                  // 32 KB
+constexpr int kStageBytes = kABytes + kBBytes;
+constexpr int kEpiWarps = 8;
+constexpr int kThreads = 64 + kEpiWarps * 32;     // 320
+constexpr uint32_t kTmemCols = 2 * BN;            // two 256-column accumulators
+constexpr uint64_t kWaitBudgetNs = 2000000000ull; // 2 s per wait
+constexpr size_t kSmemBytes = (size_t)kStages * kStageBytes + 1024 + 256;
+
+// Instruction descriptor, kind::i8: D = s32 (bits 4-5 = 2), A and B signed
+// 8-bit (bits 7-9, 10-12 = 1), both K-major, N>>3 at bit 17, M>>4 at bit 24.
+constexpr uint32_t kIdesc = (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
+                            ((uint32_t)(BM >> 4) << 24);
+
+struct Ctl {
+    uint64_t full[kStages];
+    uint64_t empty[kStages];
+    uint64_t acc_full[2];
+    uint64_t acc_empty[2];
+    uint64_t drain;
+    uint64_t ep_done;   // GEMM1: all epilogue warps finished a tile's stores
+    uint64_t ep_go;     // GEMM1: the tile's completion count has been taken
+    uint32_t tmem_base;
+    int abort;
+    int last_flag;
+};
+
+struct TcParams {
+    int N, K, n_tiles_n, f, k;
+    const int32_t* meta;
+    const int32_t* tiles;     // [m-tile][2] = (expert, first row)
+    const int32_t* offsets;   // [E+1]
+    const int32_t* row2ts;
+    const float* topk_w;
+    const float* sx;          // GEMM1: per-token activation scale
+    const float* sw0;         // GEMM1: sw_gate [E][f]; GEMM2: sw_dn [E][d]
+    const float* sw1;         // GEMM1: sw_up [E][f]
+    const float* sh;          // GEMM2: per-row h scale
+    float* h32;               // GEMM1: h [rows][f]
+    float* pamax;             // GEMM1: per-row partial max [rows][f/64]
+    int32_t* mcount;          // GEMM1: completed column tiles per row tile
+    int8_t* hq;               // GEMM1: requantised h [rows][f]
+    float* sh_out;            // GEMM1: per-row h scale
+    float* o;                 // GEMM2: [rows][d]
+    int32_t* acc_dbg;         // optional raw accumulators (canonical channel order)
+    int32_t* status;
+};
+
+// ------------------------------------------------------------------ PTX wrappers
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+    return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+                 "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+__device__ __forceinline__ uint64_t global_timer() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Bounded wait for the phase of parity `parity` to complete.  Returns false
+// (after recording the timeout) when the budget runs out or another role
+// already gave up.
+__device__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort, int32_t* status) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_timer();
+    while (true) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if (*abort) return false;
+        if (global_timer() - t0 > kWaitBudgetNs) {
+            *abort = 1;
+            atomicExch(status, (int32_t)MOE_ERR_TIMEOUT);
+            return false;
+        }
+    }
+}
+
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int x,
+                                            int y) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];" ::"r"(
+            smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y)
+        : "memory");
+}
+
+// Shared-memory matrix descriptor, K-major, 128-byte swizzle: 8-row atoms of
+// 1024 bytes (stride byte offset 1024); leading byte offset unused for this
+// layout; descriptor version 1 (bit 46); layout type 2 = SWIZZLE_128B.
+__device__ __forceinline__ uint64_t desc_sw128(uint32_t saddr) {
+    uint64_t d = (uint64_t)((saddr >> 4) & 0x3FFFu);
+    d |= (uint64_t)1 << 16;
+    d |= (uint64_t)(1024 >> 4) << 32;
+    d |= (uint64_t)1 << 46;
+    d |= (uint64_t)2 << 61;
+    return d;
+}
+
+__device__ __forceinline__ void mma_i8(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t accum) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(tmem_d),
+        "l"(adesc), "l"(bdesc), "r"(kIdesc), "r"(accum));
+}
+
+__device__ __forceinline__ void mma_commit(uint64_t* bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                     smem_u32(bar))
+                 : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+          "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+          "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+          "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+}
+
+__device__ __forceinline__ void tmem_ld_wait() {
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// ------------------------------------------------------------------ epilogues
+
+enum { EPI_SWIGLU = 0, EPI_DOWN = 1 };
+
+// GEMM1 tile: columns 0..127 of the accumulator are gate channels
+// nt*128 + c, columns 128..255 the matching up channels.
+__device__ __forceinline__ void epilogue_swiglu(const TcParams& p, uint32_t taddr, int half, int e,
+                                                int nt, int grow, bool valid, float& amax,
+                                                Ctl* ctl, int buf, int lane) {
+    const int f = p.f;
+    float sxt = 0.0f;
+    if (valid) sxt = p.sx[p.row2ts[grow] / p.k];
+    amax = 0.0f;
+#pragma unroll 1
+    for (int c = 0; c < 2; ++c) {
+        const int col0 = 64 * half + 32 * c;
+        uint32_t g[32], u[32];
+        tmem_ld32(taddr + col0, g);
+        tmem_ld32(taddr + 128 + col0, u);
+        tmem_ld_wait();
+        if (c == 1) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&ctl->acc_empty[buf]);
+        }
+        if (!valid) continue;
+        const int ch0 = nt * 128 + col0;
+        const float* swg = p.sw0 + (int64_t)e * f + ch0;
+        const float* swu = p.sw1 + (int64_t)e * f + ch0;
+        float* hrow = p.h32 + (int64_t)grow * f + ch0;
+#pragma unroll
+        for (int j = 0; j < 32; j += 4) {
+            const float4 sg = *reinterpret_cast<const float4*>(swg + j);
+            const float4 su = *reinterpret_cast<const float4*>(swu + j);
+            const float sgv[4] = {sg.x, sg.y, sg.z, sg.w}, suv[4] = {su.x, su.y, su.z, su.w};
+            float hv[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const float gf = __fmul_rn(__fmul_rn(__int2float_rn((int)g[j + q]), sxt), sgv[q]);
+                const float uf = __fmul_rn(__fmul_rn(__int2float_rn((int)u[j + q]), sxt), suv[q]);
+                hv[q] = __fmul_rn(moe_silu(gf), uf);
+                amax = fmaxf(amax, fabsf(hv[q]));
+            }
+            *reinterpret_cast<float4*>(hrow + j) = make_float4(hv[0], hv[1], hv[2], hv[3]);
+        }
+        if (p.acc_dbg) {
+            int32_t* dg = p.acc_dbg + (int64_t)grow * 2 * f + ch0;
+            for (int j = 0; j < 32; ++j) {
+                dg[j] = (int32_t)g[j];
+                dg[f + j] = (int32_t)u[j];
+            }
+        }
+    }
+}
+
+__device__ __forceinline__ void epilogue_down(const TcParams& p, uint32_t taddr, int half, int e,
+                                              int nt, int grow, bool valid, Ctl* ctl, int buf,
+                                              int lane) {
+    const int d = p.N;
+    float shr = 0.0f, wr = 0.0f;
+    if (valid) {
+        shr = p.sh[grow];
+        wr = p.topk_w[p.row2ts[grow]];
+    }
+#pragma unroll 1
+    for (int c = 0; c < 4; ++c) {
+        const int col0 = 128 * half + 32 * c;
+        uint32_t a[32];
+        tmem_ld32(taddr + col0, a);
+        tmem_ld_wait();
+        if (c == 3) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&ctl->acc_empty[buf]);
+        }
+        if (!valid) continue;
+        const int ch0 = nt * BN + col0;
+        const float* sw = p.sw0 + (int64_t)e * d + ch0;
+        float* orow = p.o + (int64_t)grow * d + ch0;
+#pragma unroll
+        for (int j = 0; j < 32; j += 4) {
+            const float4 s4 = *reinterpret_cast<const float4*>(sw + j);
+            const float sv[4] = {s4.x, s4.y, s4.z, s4.w};
+            float ov[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+                ov[q] = __fmul_rn(__fmul_rn(__fmul_rn(__int2float_rn((int)a[j + q]), shr), sv[q]), wr);
+            *reinterpret_cast<float4*>(orow + j) = make_float4(ov[0], ov[1], ov[2], ov[3]);
+        }
+        if (p.acc_dbg) {
+            int32_t* da = p.acc_dbg + (int64_t)grow * d + ch0;
+            for (int j = 0; j < 32; ++j) da[j] = (int32_t)a[j];
+        }
+    }
+}
+
+// Requantise the rows of a finished 128-row tile: sh = max over the row's
+// partial maxima / 127, codes rint(h / sh).  One warp per row.
+__device__ void requant_rows(const TcParams& p, int row0, int nrows, int ew, int lane) {
+    const int f = p.f, npart = f / 64;
+    for (int r = ew; r < nrows; r += kEpiWarps) {
+        const int grow = row0 + r;
+        float m = 0.0f;
+        for (int i = lane; i < npart; i += 32) m = fmaxf(m, __ldcg(p.pamax + (int64_t)grow * npart + i));
+        m = warp_max(m);
+        const float s = m > 0.0f ? __fdiv_rn(m, 127.0f) : 0.0f;
+        if (lane == 0) p.sh_out[grow] = s;
+        const float4* hrow = reinterpret_cast<const float4*>(p.h32 + (int64_t)grow * f);
+        uint32_t* qrow = reinterpret_cast<uint32_t*>(p.hq + (int64_t)grow * f);
+        for (int c4 = lane; c4 < f / 4; c4 += 32) {
+            const float4 h = __ldcg(hrow + c4);
+            qrow[c4] = s > 0.0f ? pack4(quant_code(h.x, s), quant_code(h.y, s), quant_code(h.z, s),
+                                        quant_code(h.w, s))
+                                : 0u;
+        }
+    }
+}
+
+// ------------------------------------------------------------------ the kernel
+
+template <int EPI>
+__global__ void __launch_bounds__(kThreads, 1)
+    tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
+                   const TcParams p) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    Ctl* ctl = reinterpret_cast<Ctl*>(smem + kStages * kStageBytes);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int num_tiles = p.meta[META_NTILES] * p.n_tiles_n;
+    const int nkb = p.K / BK;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&ctl->full[s], 1);
+            mbar_init(&ctl->empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&ctl->acc_full[b], 1);
+            mbar_init(&ctl->acc_empty[b], kEpiWarps);
+        }
+        mbar_init(&ctl->drain, 1);
+        mbar_init(&ctl->ep_done, kEpiWarps);
+        mbar_init(&ctl->ep_go, 1);
+        ctl->abort = 0;
+        ctl->last_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         smem_u32(&ctl->tmem_base)),
+                     "r"(kTmemCols));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = ctl->tmem_base;
+    volatile int* abort = &ctl->abort;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // ---------------- TMA producer
+            int s = 0;
+            uint32_t ph = 0;
+            uint32_t issued_par[kStages];
+            bool issued[kStages];
+            for (int i = 0; i < kStages; ++i) issued[i] = false;
+            bool ok = true;
+            for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+                const int mt = t / p.n_tiles_n, nt = t % p.n_tiles_n;
+                const int e = p.tiles[2 * mt], row0 = p.tiles[2 * mt + 1];
+                const int brow = e * p.N + nt * BN;
+                for (int kb = 0; kb < nkb; ++kb) {
+                    if (!mbar_wait(&ctl->empty[s], ph ^ 1, abort, p.status)) { ok = false; break; }
+                    mbar_arrive_expect_tx(&ctl->full[s], kStageBytes);
+                    uint8_t* sa = smem + s * kStageBytes;
+                    tma_load_2d(sa, &tm_a, &ctl->full[s], kb * BK, row0);
+                    tma_load_2d(sa + kABytes, &tm_b, &ctl->full[s], kb * BK, brow);
+                    issued[s] = true;
+                    issued_par[s] = ph;
+                    if (++s == kStages) { s = 0; ph ^= 1; }
+                }
+            }
+            // copies in flight land before the CTA ends (bounded)
+            for (int i = 0; i < kStages; ++i) {
+                if (!issued[i]) continue;
+                const uint64_t t0 = global_timer();
+                while (!mbar_try_wait(&ctl->full[i], issued_par[i]) && global_timer() - t0 < kWaitBudgetNs) {}
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            // ---------------- MMA issuer
+            int s = 0, buf = 0;
+            uint32_t ph = 0, aph = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+                if (!mbar_wait(&ctl->acc_empty[buf], aph ^ 1, abort, p.status)) break;
+                tc_fence_after();
+                const uint32_t d_tmem = tmem + (uint32_t)(buf * BN);
+                for (int kb = 0; kb < nkb; ++kb) {
+                    if (!mbar_wait(&ctl->full[s], ph, abort, p.status)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t a_addr = smem_u32(smem + s * kStageBytes);
+                    const uint32_t b_addr = a_addr + kABytes;
+#pragma unroll
+                    for (int kk = 0; kk < BK / 32; ++kk)
+                        mma_i8(d_tmem, desc_sw128(a_addr + kk * 32), desc_sw128(b_addr + kk * 32),
+                               (kb | kk) != 0 ? 1u : 0u);
+                    mma_commit(&ctl->empty[s]);
+                    if (++s == kStages) { s = 0; ph ^= 1; }
+                }
+                if (!ok) break;
+                mma_commit(&ctl->acc_full[buf]);
+                buf ^= 1;
+                if (buf == 0) aph ^= 1;
+            }
+            // all MMAs issued by this thread complete before TMEM is freed (bounded)
+            mma_commit(&ctl->drain);
+            const uint64_t t0 = global_timer();
+            while (!mbar_try_wait(&ctl->drain, 0) && global_timer() - t0 < kWaitBudgetNs) {}
+        }
+    } else {
+        // ---------------- epilogue warps
+        const int ew = warp - 2;                 // 0..7
+        const int quad = warp & 3;               // TMEM lanes this warp may access
+        const int half = ew >> 2;                // which half of the tile's columns
+        const int r_in_tile = quad * 32 + lane;
+        int buf = 0;
+        uint32_t aph = 0, it = 0;
+        for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++it) {
+            if (!mbar_wait(&ctl->acc_full[buf], aph, abort, p.status)) break;
+            tc_fence_after();
+            const int mt = t / p.n_tiles_n, nt = t % p.n_tiles_n;
+            const int e = p.tiles[2 * mt], row0 = p.tiles[2 * mt + 1];
+            const int nrows = min(BM, p.offsets[e + 1] - row0);
+            const int grow = row0 + r_in_tile;
+            const bool valid = r_in_tile < nrows;
+            const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(buf * BN);
+            if (EPI == EPI_SWIGLU) {
+                float amax;
+                epilogue_swiglu(p, taddr, half, e, nt, grow, valid, amax, ctl, buf, lane);
+                if (valid) p.pamax[(int64_t)grow * (p.f / 64) + nt * 2 + half] = amax;
+                // publish this warp's h and maxima, then count the column tile
+                __threadfence();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&ctl->ep_done);
+                if (ew == 0 && lane == 0) {
+                    int last = 0;
+                    if (mbar_wait(&ctl->ep_done, it & 1, abort, p.status))
+                        last = atomicAdd(p.mcount + mt, 1) == p.n_tiles_n - 1;
+                    *reinterpret_cast<volatile int*>(&ctl->last_flag) = last;
+                    mbar_arrive(&ctl->ep_go);
+                }
+                __syncwarp();
+                if (!mbar_wait(&ctl->ep_go, it & 1, abort, p.status)) break;
+                if (*reinterpret_cast<volatile int*>(&ctl->last_flag)) {
+                    // the last column tile of this row tile: every h of its rows is written
+                    __threadfence();
+                    requant_rows(p, row0, nrows, ew, lane);
+                }
+            } else {
+                epilogue_down(p, taddr, half, e, nt, grow, valid, ctl, buf, lane);
+            }
+            buf ^= 1;
+            if (buf == 0) aph ^= 1;
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols));
+    }
+}
+
+// ------------------------------------------------------------------ host side
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
+                                  CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                  CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    }
+    return fn;
+}
+
+// 2-D map over an int8 [rows][K] K-major matrix, box = box_rows x 128 bytes,
+// 128-byte swizzle (the layout the MMA descriptors expect).
+bool make_map(CUtensorMap* m, const void* base, uint64_t K, uint64_t rows, uint32_t box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[2] = {K, rows};
+    const cuuint64_t strides[1] = {K};
+    const cuuint32_t box[2] = {(cuuint32_t)BK, box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int EPI>
+cudaError_t launch(const CUtensorMap& ta, const CUtensorMap& tb, const TcParams& p, int grid,
+                   cudaStream_t s) {
+    static bool attr = false;
+    if (!attr) {
+        cudaError_t e = cudaFuncSetAttribute(tc_gemm_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)kSmemBytes);
+        if (e != cudaSuccess) return e;
+        attr = true;
+    }
+    tc_gemm_kernel<EPI><<<grid, kThreads, kSmemBytes, s>>>(ta, tb, p);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+bool tc_make_weight_maps(moe_w8a8_weights* w) {
+    const moe_w8a8_config& c = w->cfg;
+    const uint64_t E = c.n_experts, d = c.d, f = c.f;
+    return make_map(&w->tm_w_gu, w->w_gu, d, E * 2 * f, BN) && make_map(&w->tm_w_dn, w->w_dn, f, E * d, BN);
+}
+
+bool tc_supported(const moe_w8a8_config& c) { return c.d % BN == 0 && c.f % BK == 0 && c.d % BK == 0; }
+
+cudaError_t launch_tc_gemm1(const moe_w8a8_weights* w, int T, const int8_t* aq, const int32_t* meta,
+                            const int32_t* tiles, const int32_t* offsets, const int32_t* row2ts,
+                            const float* sx, float* h32, float* pamax, int32_t* mcount, int8_t* hq,
+                            float* sh, int32_t* acc_dbg, cudaStream_t s) {
+    const moe_w8a8_config& c = w->cfg;
+    CUtensorMap ta;
+    const int rows = T * c.top_k;
+    if (!make_map(&ta, aq, c.d, rows, BM)) return cudaErrorInvalidValue;
+    TcParams p{};
+    p.N = 2 * c.f;
+    p.K = c.d;
+    p.n_tiles_n = p.N / BN;
+    p.f = c.f;
+    p.k = c.top_k;
+    p.meta = meta;
+    p.tiles = tiles;
+    p.offsets = offsets;
+    p.row2ts = row2ts;
+    p.sx = sx;
+    p.sw0 = w->sw_gate;
+    p.sw1 = w->sw_up;
+    p.h32 = h32;
+    p.pamax = pamax;
+    p.mcount = mcount;
+    p.hq = hq;
+    p.sh_out = sh;
+    p.acc_dbg = acc_dbg;
+    p.status = w->status;
+    const int max_mt = (rows + BM - 1) / BM + c.n_experts;
+    const int grid = max(1, min(w->num_sms, max_mt * p.n_tiles_n));
+    return launch<EPI_SWIGLU>(ta, w->tm_w_gu, p, grid, s);
+}
+
+cudaError_t launch_tc_gemm2(const moe_w8a8_weights* w, int T, const int8_t* hq, const float* sh,
+                            const int32_t* meta, const int32_t* tiles, const int32_t* offsets,
+                            const int32_t* row2ts, const float* topk_w, float* o, int32_t* acc_dbg,
+                            cudaStream_t s) {
+    const moe_w8a8_config& c = w->cfg;
+    CUtensorMap ta;
+    const int rows = T * c.top_k;
+    if (!make_map(&ta, hq, c.f, rows, BM)) return cudaErrorInvalidValue;
+    TcParams p{};
+    p.N = c.d;
+    p.K = c.f;
+    p.n_tiles_n = p.N / BN;
+    p.f = c.f;
+    p.k = c.top_k;
+    p.meta = meta;
+    p.tiles = tiles;
+    p.offsets = offsets;
+    p.row2ts = row2ts;
+    p.topk_w = topk_w;
+    p.sw0 = w->sw_dn;
+    p.sh = sh;
+    p.o = o;
+    p.acc_dbg = acc_dbg;
+    p.status = w->status;
+    const int max_mt = (rows + BM - 1) / BM + c.n_experts;
+    const int grid = max(1, min(w->num_sms, max_mt * p.n_tiles_n));
+    return launch<EPI_DOWN>(ta, w->tm_w_dn, p, grid, s);
+}
+
+}  // namespace moe

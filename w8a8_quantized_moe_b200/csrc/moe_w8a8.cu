@@ -38,8 +38,11 @@ int capacity_of(const moe_w8a8_config& c, int T) {
     return (int)std::ceil((double)c.capacity_factor * (double)((int64_t)T * c.top_k) / (double)c.n_experts);
 }
 
+bool tensor_ok(const moe_w8a8_weights* w) { return w->tmaps_ok && tc_supported(w->cfg); }
+
 int choose_path(const moe_w8a8_weights* w, int T) {
     if (w->path != MOE_PATH_AUTO) return w->path;
+    if (!tensor_ok(w)) return MOE_PATH_STREAM;
     return (int64_t)T * w->cfg.top_k <= w->stream_max_rows ? MOE_PATH_STREAM : MOE_PATH_TENSOR;
 }
 
@@ -108,6 +111,9 @@ WsLayout ws_layout(const moe_w8a8_weights* w, int T) {
     L.hq = take(tk * f);
     L.sh = take(tk * 4);
     L.o = take(tk * d * 4);
+    L.h32 = take(stream ? 0 : tk * f * 4);
+    L.pamax = take(stream ? 0 : tk * (f / 64) * 4);
+    L.mcount = take(stream ? 0 : max_tiles * 4);
     L.total = p;
     return L;
 }
@@ -217,6 +223,7 @@ moe_status moe_w8a8_prepare(const moe_w8a8_config* cfg, const float* w_gate, con
             cudaSuccess ||
         cudaStreamSynchronize(s) != cudaSuccess)
         return fail(MOE_ERR_CUDA);
+    w->tmaps_ok = tc_make_weight_maps(w);
     cudaFree(tmp);
     *out = w;
     return MOE_OK;
@@ -273,8 +280,9 @@ static moe_status forward_impl(const moe_w8a8_weights* w, const void* x, int T, 
     mark(MOE_STAGE_TOPK, 1);
     ++launches;
     mark(MOE_STAGE_PERMUTE, 0);
+    const bool tensor = path == MOE_PATH_TENSOR;
     CUDA_TRY(launch_permute(idx, T, k, E, capacity_of(c, T), (int32_t*)P(L.hist), offsets, row2ts,
-                            ts2row, meta, active, tiles, s));
+                            ts2row, meta, active, tiles, tensor ? (int32_t*)P(L.mcount) : nullptr, s));
     mark(MOE_STAGE_PERMUTE, 1);
     launches += 2;
     if (path == MOE_PATH_STREAM) {
@@ -296,7 +304,21 @@ static moe_status forward_impl(const moe_w8a8_weights* w, const void* x, int T, 
         if (dbg && dbg->acc1)
             CUDA_TRY(cudaMemcpyAsync(dbg->acc1, acc1, tk * 2 * f * 4, cudaMemcpyDeviceToDevice, s));
     } else {
-        return MOE_ERR_UNSUPPORTED_SHAPE;
+        int8_t* aq = (int8_t*)P(L.aq);
+        mark(MOE_STAGE_QUANT, 0);
+        CUDA_TRY(launch_smooth_quant(x, c.in_dtype, w->inv_s, T, d, k, ts2row, xq, sx, aq, s));
+        mark(MOE_STAGE_QUANT, 1);
+        mark(MOE_STAGE_GEMM1, 0);
+        CUDA_TRY(launch_tc_gemm1(w, T, aq, meta, tiles, offsets, row2ts, sx, (float*)P(L.h32),
+                                 (float*)P(L.pamax), (int32_t*)P(L.mcount), hq, sh,
+                                 dbg ? dbg->acc1 : nullptr, s));
+        mark(MOE_STAGE_GEMM1, 1);
+        empty_stage(MOE_STAGE_REQUANT);
+        mark(MOE_STAGE_GEMM2, 0);
+        CUDA_TRY(launch_tc_gemm2(w, T, hq, sh, meta, tiles, offsets, row2ts, wts, o,
+                                 dbg ? dbg->acc2 : nullptr, s));
+        mark(MOE_STAGE_GEMM2, 1);
+        launches += 3;
     }
     mark(MOE_STAGE_COMBINE, 0);
     CUDA_TRY(launch_combine(o, ts2row, T, k, d, c.out_dtype, y, s));
@@ -330,7 +352,7 @@ moe_status moe_w8a8_forward(const moe_w8a8_weights* w, const void* x, int32_t T,
     if (T == 0) return MOE_OK;
     if (!x || !y || !workspace) return MOE_ERR_INVALID_ARG;
     if ((uintptr_t)workspace % kAlign) return MOE_ERR_INVALID_ARG;
-    if (choose_path(w, T) == MOE_PATH_TENSOR) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (choose_path(w, T) == MOE_PATH_TENSOR && !tensor_ok(w)) return MOE_ERR_UNSUPPORTED_SHAPE;
     if (workspace_bytes < ws_layout(w, T).total) return MOE_ERR_WORKSPACE_TOO_SMALL;
     return forward_impl(w, x, T, router_bias, router_logits, y, (char*)workspace, dbg,
                         (cudaStream_t)stream);
@@ -344,7 +366,7 @@ moe_status moe_w8a8_forward_host(const moe_w8a8_weights* w, const void* x_host, 
     if (T == 0) return MOE_OK;
     if (!x_host || !y_host || !workspace) return MOE_ERR_INVALID_ARG;
     if ((uintptr_t)workspace % kAlign) return MOE_ERR_INVALID_ARG;
-    if (choose_path(w, T) == MOE_PATH_TENSOR) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (choose_path(w, T) == MOE_PATH_TENSOR && !tensor_ok(w)) return MOE_ERR_UNSUPPORTED_SHAPE;
     const WsLayout L = ws_layout(w, T);
     if (workspace_bytes < L.total) return MOE_ERR_WORKSPACE_TOO_SMALL;
     const moe_w8a8_config& c = w->cfg;
