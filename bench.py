@@ -47,6 +47,8 @@ def parse():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-stage-events", action="store_true")
+    p.add_argument("--no-prefill", action="store_true",
+                   help="skip the extra prefill-layer measurement of the decode run")
     return p.parse_args()
 
 
@@ -228,35 +230,27 @@ def run_reference(args, world, rank):
 
 # ------------------------------------------------------------------ our arm
 
-def run_ours(args, world, rank, local):
+def measure(args, wl, world, rank, local, e2e_on=True, wts=None):
+    """Prepare the layer (untimed), then time K forwards on resident inputs,
+    with per-stage CUDA events, clock samples and an end-to-end leg."""
     import torch
 
     import w8a8_quantized_moe_b200 as M
-    from w8a8_quantized_moe_b200 import build as B
 
-    if not os.path.exists(M.LIB_PATH):
-        B.build()
-    torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    base = synth.WORKLOADS[args.workload]
-    import dataclasses
-    # replicas: same layer weights on every rank, a different token batch per rank
-    wl = dataclasses.replace(base, data_seed=base.data_seed + 1000 * rank) if rank else base
-
-    # ---- offline preparation (untimed)
-    wts = synth.make_weights(wl)
+    wts = synth.make_weights(wl) if wts is None else wts
     data = synth.make_data(wl)
     cfg = M.make_config(wl.d, wl.f, wl.E, wl.k, wl.alpha, wl.capacity_factor, True,
                         M.MOE_BF16 if wl.in_bf16 else M.MOE_F32,
                         M.MOE_BF16 if wl.in_bf16 else M.MOE_F32)
     act = torch.bfloat16 if wl.in_bf16 else torch.float32
 
-    def host_act(v32):
+    def to_act(v32):
         if wl.in_bf16:
             return torch.from_numpy(synth.f32_to_bf16_bits(v32).view(np.int16)).view(torch.bfloat16)
         return torch.from_numpy(v32)
 
-    cal = host_act(wts.calib_x).to(dev)
+    cal = to_act(wts.calib_x).to(dev)
     ax = torch.zeros(wl.d, dtype=torch.float32, device=dev)
     M.moe_w8a8_calibrate_absmax(cal, ax)
     wg, wu, wd = (torch.from_numpy(a).to(dev) for a in (wts.w_gate, wts.w_up, wts.w_down))
@@ -266,26 +260,26 @@ def run_ours(args, world, rank, local):
     torch.cuda.empty_cache()
 
     T = wl.T
-    x = host_act(data.x).to(dev) if not wl.in_bf16 else \
-        torch.from_numpy(data.x_bits.view(np.int16)).view(torch.bfloat16).to(dev)
+    x = torch.from_numpy(data.x_bits.view(np.int16)).view(torch.bfloat16).to(dev) if wl.in_bf16 \
+        else torch.from_numpy(data.x).to(dev)
     logits = torch.from_numpy(data.router_logits).to(dev) if data.router_logits is not None else None
     bias = torch.from_numpy(data.router_bias).to(dev) if data.router_bias is not None else None
     y = torch.empty((T, wl.d), dtype=act, device=dev)
     ws = torch.empty(M.moe_w8a8_workspace_size(W, T), dtype=torch.uint8, device=dev)
 
-    # routing statistics of this batch (for the byte model): one debug forward
+    # routing statistics of this batch (for the byte / op model): one debug forward
     offs = torch.empty(wl.E + 1, dtype=torch.int32, device=dev)
     M.moe_w8a8_forward(W, x, T, bias, logits, y, ws, {"offsets": offs})
     counts = np.diff(offs.cpu().numpy())
     n_active, R = int((counts > 0).sum()), int(counts.sum())
     alg = algorithmic(wl, n_active, R)
+    tensor = T * wl.k > 512
 
     stream = torch.cuda.current_stream(dev)
     for _ in range(args.warmup):
         M.moe_w8a8_forward(W, x, T, bias, logits, y, ws)
     torch.cuda.synchronize(dev)
 
-    # ---- timed region: K steps, device time, max over ranks
     K = args.steps
     stage_events = not args.no_stage_events
     if stage_events:
@@ -302,9 +296,8 @@ def run_ours(args, world, rank, local):
     torch.cuda.synchronize(dev)
     clocks.stop()
     barrier(world)
-    launches_per_step = M.moe_w8a8_last_launch_count(W)
-    ms_local = e0.elapsed_time(e1)
-    ms_total = max_over_ranks(ms_local, world)
+    launches = M.moe_w8a8_last_launch_count(W) * K
+    ms_total = max_over_ranks(e0.elapsed_time(e1), world)
     M.moe_w8a8_check_status(W)
     stages = None
     if stage_events:
@@ -312,11 +305,8 @@ def run_ours(args, world, rank, local):
         M.moe_w8a8_profile_stop(W)
         stages = {M.STAGE_NAMES[i]: float(st[:, i].mean()) for i in range(M.MOE_N_STAGES)}
 
-    value = world * T * K / (ms_total / 1e3)
-
-    # ---- end to end through the C ABI with host buffers (H2D + forward + D2H per step)
     e2e = None
-    if not args.no_e2e:
+    if e2e_on and not args.no_e2e:
         if wl.in_bf16:
             xh = torch.from_numpy(data.x_bits.view(np.int16)).pin_memory()
             yh = torch.empty((T, wl.d), dtype=torch.int16).pin_memory()
@@ -341,25 +331,80 @@ def run_ours(args, world, rank, local):
         e2e = {"value": world * T * K / (ms_e2e / 1e3), "unit": "tokens/s",
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(yh.numel() * yh.element_size())}
 
-    if rank != 0:
-        return
-
-    # ---- roofline of the dominant stage, from the live stage events
     peaks, peak_src = load_peaks()
     roof = None
     if stages:
-        dom = max(("gemm1", "gemm2"), key=lambda s: stages[s])
+        dom = max(("gemm1", "gemm2"), key=lambda k: stages[k])
         dom_ms = stages[dom]
-        bytes_dom = alg[f"{dom}_bytes"]
-        achieved = bytes_dom / (dom_ms / 1e3) / 1e9
-        roof = {"bound": "hbm", "kernel": f"{dom} ({'stream_gateup' if dom == 'gemm1' else 'stream_down'})",
-                "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": achieved / peaks["hbm_gbs"], "traffic": None,
-                "peak_source": f"hbm_gbs of {peak_src}",
-                "algorithmic_bytes_per_launch": bytes_dom, "launch_ms": dom_ms}
-    layer_gbs = alg["layer_bytes"] / (ms_total / K / 1e3) / 1e9
+        if tensor:
+            ops = 2 * R * (2 * wl.f if dom == "gemm1" else wl.f) * wl.d
+            peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]) * INT8_PER_BF16
+            achieved = ops / (dom_ms / 1e3) / 1e12
+            roof = {"bound": "tensor", "kernel": f"{dom} (tc_gemm_kernel<{0 if dom == 'gemm1' else 1}>)",
+                    "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                    "traffic": None,
+                    "peak_source": f"2 x bf16_tflops_sustained of {peak_src} (INT8 dense = 2 x bf16, nominal)",
+                    "int8_ops_per_launch": ops, "launch_ms": dom_ms,
+                    "frac_of_nominal_4500": achieved / 4500.0}
+        else:
+            b = alg[f"{dom}_bytes"]
+            achieved = b / (dom_ms / 1e3) / 1e9
+            roof = {"bound": "hbm",
+                    "kernel": f"{dom} ({'stream_gateup_kernel' if dom == 'gemm1' else 'stream_down_kernel'})",
+                    "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                    "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                    "peak_source": f"hbm_gbs of {peak_src}",
+                    "algorithmic_bytes_per_launch": b, "launch_ms": dom_ms}
+    step_s = ms_total / K / 1e3
+    layer_gbs = alg["layer_bytes"] / step_s / 1e9
+    layer_tops = alg["int8_ops"] / step_s / 1e12
+    out = {
+        "value": world * T * K / (ms_total / 1e3), "ms_per_step": ms_total / K,
+        "config": {"workload": describe(wl), "T": T, "d": wl.d, "E": wl.E, "k": wl.k, "f": wl.f,
+                   "alpha": wl.alpha, "active_experts": n_active, "rows": R,
+                   "expert_path": "tcgen05 grouped GEMM" if tensor else "weight streaming",
+                   "l2": (f"inputs larger than L2: {alg['layer_bytes'] / 1e9:.2f} GB of algorithmic "
+                          f"bytes per step (INT8 weights of the active experts, X, Y) vs 126 MB L2; "
+                          f"no flush"),
+                   "parallelism": "replicas" if world > 1 else "single GPU",
+                   "layer_bytes_per_step": alg["layer_bytes"], "layer_gbs": layer_gbs,
+                   "layer_hbm_frac": layer_gbs / peaks["hbm_gbs"],
+                   "int8_ops_per_step": alg["int8_ops"], "layer_int8_tops": layer_tops},
+        "roofline": roof, "stages_ms": stages, "e2e": e2e, "gpu_launches": launches,
+        "clocks": clocks.summary(),
+    }
+    return out, wts, W
 
-    # ---- CPU baseline: the oracle on a bounded sample of this workload (rank 0, N = 1)
+
+def run_ours(args, world, rank, local):
+    import torch
+
+    import w8a8_quantized_moe_b200 as M
+    from w8a8_quantized_moe_b200 import build as B
+
+    if not os.path.exists(M.LIB_PATH):
+        B.build()
+    torch.cuda.set_device(local)
+    import dataclasses
+    base = synth.WORKLOADS[args.workload]
+    # replicas: same layer weights on every rank, a different token batch per rank
+    wl = dataclasses.replace(base, data_seed=base.data_seed + 1000 * rank) if rank else base
+    res, wts, W = measure(args, wl, world, rank, local)
+    del W
+
+    extra = None
+    if args.workload == "decode" and not args.no_prefill:
+        pw = synth.WORKLOADS["prefill"]
+        pw = dataclasses.replace(pw, data_seed=pw.data_seed + 1000 * rank) if rank else pw
+        # the prefill layer reuses the decode layer's expert weights
+        pres, _, PW = measure(args, pw, world, rank, local, e2e_on=False, wts=wts)
+        del PW
+        torch.cuda.empty_cache()
+        extra = {"metric": "prefill layer tokens/s (T=16384)", "unit": "tokens/s", **pres}
+
+    if rank != 0:
+        return
+
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
         import oracle
@@ -370,31 +415,18 @@ def run_ours(args, world, rank, local):
         while n == 0 or secs < args.cpu_seconds:
             secs += oracle_step(wl, prep, sdata)
             n += 1
-        tokens = n * n_tok
-        cpu = {"value": tokens / secs, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+        cpu = {"value": n * n_tok / secs, "unit": "tokens/s", "cores": 1, "kind": "oracle",
                "sample": f"{n} steps of the first {n_tok} of the {wl.T} tokens of the {wl.name} workload "
                          f"({secs:.1f} s of single-thread CPU time; preparation untimed)"}
 
-    line = {
-        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
-        "warmup": args.warmup, "ms_per_step": ms_total / K, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "int8", "data": "synthetic",
-        "config": {"workload": describe(wl), "T": T, "d": wl.d, "E": wl.E, "k": wl.k, "f": wl.f,
-                   "alpha": wl.alpha, "active_experts": n_active, "rows": R,
-                   "l2": f"inputs larger than L2: {alg['gemm1_bytes'] / 1e9 + 0:.2f} GB gate/up + "
-                         f"{alg['gemm2_bytes'] / 1e9:.2f} GB down INT8 weights streamed per step "
-                         f"vs 126 MB L2; no flush",
-                   "parallelism": "replicas" if world > 1 else "single GPU",
-                   "layer_bytes_per_step": alg["layer_bytes"], "layer_gbs": layer_gbs,
-                   "layer_hbm_frac": layer_gbs / peaks["hbm_gbs"],
-                   "int8_ops_per_step": alg["int8_ops"]},
-        "roofline": roof,
-        "stages_ms": stages,
-        "e2e": e2e,
-        "gpu_launches": launches_per_step * K,
-        "clocks": clocks.summary(),
-        "cpu_baseline": cpu,
-    }
+    line = {"metric": METRIC, "value": res["value"], "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": res["ms_per_step"],
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8",
+            "data": "synthetic", "config": res["config"], "roofline": res["roofline"],
+            "stages_ms": res["stages_ms"], "e2e": res["e2e"], "gpu_launches": res["gpu_launches"],
+            "clocks": res["clocks"], "cpu_baseline": cpu}
+    if extra is not None:
+        line["prefill"] = extra
     print(json.dumps(line), flush=True)
 
 
