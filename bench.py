@@ -47,6 +47,8 @@ def parse():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-stage-events", action="store_true")
+    p.add_argument("--tokens", type=int, default=0,
+                   help="override the workload's token count T (same layer, same seeds)")
     p.add_argument("--no-prefill", action="store_true",
                    help="skip the extra prefill-layer measurement of the decode run")
     return p.parse_args()
@@ -387,6 +389,8 @@ def run_ours(args, world, rank, local):
     torch.cuda.set_device(local)
     import dataclasses
     base = synth.WORKLOADS[args.workload]
+    if args.tokens > 0:
+        base = dataclasses.replace(base, T=args.tokens)
     # replicas: same layer weights on every rank, a different token batch per rank
     wl = dataclasses.replace(base, data_seed=base.data_seed + 1000 * rank) if rank else base
     res, wts, W = measure(args, wl, world, rank, local)
