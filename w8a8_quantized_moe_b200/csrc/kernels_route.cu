@@ -10,64 +10,92 @@ namespace moe {
 namespace {
 
 // ---------------------------------------------------------------------------
-// Router logits in the stated fp32 order: for each (t, e), lane p of a warp
-// owns partial sum p = fma chain over i ascending of x[t][32i+p] W[32i+p][e]
-// from +0; the 32 partials are combined by xor-butterfly 16, 8, 4, 2, 1.
-// A warp computes a block of 4 tokens x 16 experts (64 chains per lane).
+// Router logits in the stated fp32 order: for each (t, e), partial sum p
+// (p = 0..31) is the fma chain over i ascending of x[t][32i+p] W[32i+p][e] from
+// +0, and the 32 partials are combined by xor-butterfly 16, 8, 4, 2, 1.
+// A block computes 32 tokens x 32 experts.  Lane p of every warp owns partial p
+// for a register tile of 8 tokens x 8 experts (16 warps = 4 token groups x 4
+// expert groups); X and W_router are staged in shared memory 128 channels at a
+// time, laid out [i][p][t] and [i][p][e] with padded rows so that each lane's 8
+// tokens (experts) are one conflict-free pair of 16-byte loads.
 // ---------------------------------------------------------------------------
-constexpr int kRtTok = 4;    // tokens per warp
-constexpr int kRtExp = 16;   // experts per warp
-constexpr int kRtWarps = 8;
+constexpr int kRtT = 32;         // tokens per block
+constexpr int kRtE = 32;         // experts per block
+constexpr int kRtKC = 128;       // channels per staged chunk (4 steps of i)
+constexpr int kRtPad = 36;       // padded row (floats): 16-byte aligned, rows 4 banks apart
+constexpr int kRtThreads = 512;
 
-__global__ void __launch_bounds__(kRtWarps * 32) router_logits_kernel(
+__global__ void __launch_bounds__(kRtThreads) router_logits_kernel(
     const void* __restrict__ x, int in_dtype, const float* __restrict__ wr, int T, int d, int E,
     float* __restrict__ logits) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int n_eg = (E + kRtExp - 1) / kRtExp;
-    const int wid = blockIdx.x * kRtWarps + warp;   // global warp id
-    const int tg = wid / n_eg, eg = wid % n_eg;
-    const int t0 = tg * kRtTok, e0 = eg * kRtExp;
-    if (t0 >= T) return;
-    float acc[kRtTok][kRtExp];
+    __shared__ __align__(16) float xs[kRtKC / 32][32][kRtPad];
+    __shared__ __align__(16) float ws[kRtKC / 32][32][kRtPad];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int tg = warp >> 2, eg = warp & 3;
+    const int t0 = blockIdx.x * kRtT, e0 = blockIdx.y * kRtE;
+    float acc[8][8];
 #pragma unroll
-    for (int a = 0; a < kRtTok; ++a)
+    for (int a = 0; a < 8; ++a)
 #pragma unroll
-        for (int b = 0; b < kRtExp; ++b) acc[a][b] = 0.0f;
-    const int nchunks = d / 32;
-    for (int i = 0; i < nchunks; ++i) {
-        const int j = 32 * i + lane;
-        float xv[kRtTok];
+        for (int b = 0; b < 8; ++b) acc[a][b] = 0.0f;
+    for (int c = 0; c < d; c += kRtKC) {
+        // X chunk: 32 tokens x 128 channels, one group of 8 channels per thread
+        {
+            const int tt = tid >> 4, j0 = (tid & 15) * 8;
+            const int t = t0 + tt;
+            float v[8];
+            if (t < T) {
+                load8_act(x, (int64_t)t * d + c + j0, in_dtype, v);
+            } else {
 #pragma unroll
-        for (int a = 0; a < kRtTok; ++a) {
-            const int t = min(t0 + a, T - 1);
-            xv[a] = in_dtype == MOE_BF16
-                        ? bf16_bits_to_f32(reinterpret_cast<const uint16_t*>(x)[(int64_t)t * d + j])
-                        : reinterpret_cast<const float*>(x)[(int64_t)t * d + j];
+                for (int q = 0; q < 8; ++q) v[q] = 0.0f;
+            }
+#pragma unroll
+            for (int q = 0; q < 8; ++q) xs[(j0 + q) >> 5][(j0 + q) & 31][tt] = v[q];
         }
-        const float* wrow = wr + (int64_t)j * E + e0;
-#pragma unroll
-        for (int b = 0; b < kRtExp; ++b) {
-            const float wv = (e0 + b < E) ? __ldg(wrow + b) : 0.0f;
-#pragma unroll
-            for (int a = 0; a < kRtTok; ++a) acc[a][b] = __fmaf_rn(xv[a], wv, acc[a][b]);
+        // W chunk: 128 rows x 32 experts, 16 bytes per thread (two per thread)
+        for (int idx = tid; idx < kRtKC * (kRtE / 4); idx += kRtThreads) {
+            const int row = idx >> 3, q4 = idx & 7;
+            const int e = e0 + 4 * q4;
+            const float* src = wr + (int64_t)(c + row) * E;
+            float4 v;
+            v.x = e + 0 < E ? src[e + 0] : 0.0f;
+            v.y = e + 1 < E ? src[e + 1] : 0.0f;
+            v.z = e + 2 < E ? src[e + 2] : 0.0f;
+            v.w = e + 3 < E ? src[e + 3] : 0.0f;
+            *reinterpret_cast<float4*>(&ws[row >> 5][row & 31][4 * q4]) = v;
         }
+        __syncthreads();
+#pragma unroll
+        for (int i = 0; i < kRtKC / 32; ++i) {
+            const float4 xa = *reinterpret_cast<const float4*>(&xs[i][lane][tg * 8]);
+            const float4 xb = *reinterpret_cast<const float4*>(&xs[i][lane][tg * 8 + 4]);
+            const float4 wa = *reinterpret_cast<const float4*>(&ws[i][lane][eg * 8]);
+            const float4 wb = *reinterpret_cast<const float4*>(&ws[i][lane][eg * 8 + 4]);
+            const float xv[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
+            const float wv[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
+#pragma unroll
+            for (int a = 0; a < 8; ++a)
+#pragma unroll
+                for (int b = 0; b < 8; ++b) acc[a][b] = __fmaf_rn(xv[a], wv[b], acc[a][b]);
+        }
+        __syncthreads();
     }
 #pragma unroll
-    for (int a = 0; a < kRtTok; ++a)
+    for (int a = 0; a < 8; ++a)
 #pragma unroll
-        for (int b = 0; b < kRtExp; ++b) {
+        for (int b = 0; b < 8; ++b) {
             float v = acc[a][b];
 #pragma unroll
             for (int o = 16; o >= 1; o >>= 1) v = __fadd_rn(v, __shfl_xor_sync(0xffffffffu, v, o));
             acc[a][b] = v;
         }
-    // every lane now holds all 64 logits; lane q writes entries q and q + 32
+    // every lane now holds all 64 logits of the warp's tile; lane q writes entries q and q + 32
 #pragma unroll
-    for (int v = 0; v < kRtTok * kRtExp; ++v) {
+    for (int v = 0; v < 64; ++v) {
         if ((v & 31) != lane) continue;
-        const int a = v / kRtExp, b = v % kRtExp;
-        const int t = t0 + a, e = e0 + b;
-        if (t < T && e < E) logits[(int64_t)t * E + e] = acc[a][b];
+        const int t = t0 + tg * 8 + (v >> 3), e = e0 + eg * 8 + (v & 7);
+        if (t < T && e < E) logits[(int64_t)t * E + e] = acc[v >> 3][v & 7];
     }
 }
 
@@ -206,8 +234,8 @@ __global__ void __launch_bounds__(kPermThreads) perm_scatter_kernel(
         meta[META_NACTIVE] = na;
         meta[META_NTILES] = nt;
     }
-    if (blockIdx.x == 0 && mcount)   // per-row-tile completion counters of the tensor path
-        for (int i = tid; i < max_tiles; i += blockDim.x) mcount[i] = 0;
+    if (blockIdx.x == 0 && mcount)   // tensor path: row-tile counters, requant queue head/tail/items
+        for (int i = tid; i < max_tiles * 9 + 2; i += blockDim.x) mcount[i] = 0;
     const int base = blockIdx.x * kPermChunk;
     for (int r0 = 0; r0 < kPermChunk; r0 += kPermThreads) {
         for (int i = tid; i < (kPermThreads / 32) * E; i += blockDim.x) wcnt[i / E][i % E] = 0;
@@ -301,10 +329,8 @@ __global__ void __launch_bounds__(kSqThreads) smooth_quant_kernel(
 
 cudaError_t launch_router_logits(const void* x, int in_dtype, const float* wr, int T, int d, int E,
                                  float* logits, cudaStream_t s) {
-    const int n_eg = (E + kRtExp - 1) / kRtExp;
-    const int64_t warps = (int64_t)((T + kRtTok - 1) / kRtTok) * n_eg;
-    const int blocks = (int)((warps + kRtWarps - 1) / kRtWarps);
-    router_logits_kernel<<<blocks, kRtWarps * 32, 0, s>>>(x, in_dtype, wr, T, d, E, logits);
+    dim3 grid((T + kRtT - 1) / kRtT, (E + kRtE - 1) / kRtE);
+    router_logits_kernel<<<grid, kRtThreads, 0, s>>>(x, in_dtype, wr, T, d, E, logits);
     return cudaGetLastError();
 }
 

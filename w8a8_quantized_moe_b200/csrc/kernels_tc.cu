@@ -16,10 +16,16 @@
 //   warps 2..9  epilogue: tcgen05.ld of their 32-lane quarter of the
 //               accumulator, dequantisation and the fused math, global stores
 // GEMM1 epilogue: g, u dequantised (per-token x per-channel scales), h = silu(g)
-// u written in fp32 with per-row partial maxima; the CTA that completes the last
-// column tile of a 128-row tile requantises those rows to INT8 (row max over all
-// f channels) -- completion is counted with an atomic, nothing waits on another
-// CTA.  GEMM2 epilogue: o = acc2 sh sw w in fp32 per sorted row.
+// u written in fp32 with per-row partial maxima.  Completion of a 128-row tile
+// is counted with an atomic; the CTA that completes its last column tile
+// publishes the tile's rows as 8 requantisation items (16 rows each) on a
+// device-wide queue, and every epilogue warp of every CTA claims at most one
+// item per tile it finishes (and drains the queue before exiting), so the
+// requantisation (row max over all f channels -> INT8) is spread over the GPU
+// while h is still in L2.  Nothing ever waits for another CTA.
+// GEMM2 epilogue: o = acc2 sh sw w in fp32 per sorted row.
+// Epilogue stores go through a small swizzled shared-memory buffer per warp so
+// that each global store instruction writes whole 128-byte rows.
 //
 // Every wait on an mbarrier is bounded by the global timer; when a wait runs
 // out the kernel records MOE_ERR_TIMEOUT in the status word, stops issuing
@@ -42,7 +48,10 @@ constexpr int kEpiWarps = 8;
 constexpr int kThreads = 64 + kEpiWarps * 32;     // 320
 constexpr uint32_t kTmemCols = 2 * BN;            // two 256-column accumulators
 constexpr uint64_t kWaitBudgetNs = 2000000000ull; // 2 s per wait
-constexpr size_t kSmemBytes = (size_t)kStages * kStageBytes + 1024 + 256;
+constexpr int kEpiStageBytes = 16 * 32 * 4;      // 16 rows x 32 fp32 per epilogue warp
+constexpr size_t kSmemBytes = (size_t)kStages * kStageBytes + (size_t)kEpiWarps * kEpiStageBytes + 1024 + 256;
+constexpr int kRqRows = 16;                       // rows per requantisation item
+constexpr int kRqItemsPerTile = 128 / kRqRows;
 
 // Instruction descriptor, kind::i8: D = s32 (bits 4-5 = 2), A and B signed
 // 8-bit (bits 7-9, 10-12 = 1), both K-major, N>>3 at bit 17, M>>4 at bit 24.
@@ -76,6 +85,9 @@ struct TcParams {
     float* h32;               // GEMM1: h [rows][f]
     float* pamax;             // GEMM1: per-row partial max [rows][f/64]
     int32_t* mcount;          // GEMM1: completed column tiles per row tile
+    int32_t* rq_head;         // GEMM1: requantisation queue: next item to claim
+    int32_t* rq_tail;         //        items published so far
+    int32_t* rq_items;        //        item + 1 (0 = not yet written)
     int8_t* hq;               // GEMM1: requantised h [rows][f]
     float* sh_out;            // GEMM1: per-row h scale
     float* o;                 // GEMM2: [rows][d]
@@ -201,15 +213,46 @@ __device__ __forceinline__ void tmem_ld_wait() {
 
 enum { EPI_SWIGLU = 0, EPI_DOWN = 1 };
 
+// Store a warp's 32 rows x 32 fp32 values (lane l holds row l's values v[0..31])
+// to rows gbase + l*ld (only the first nvalid rows), coalesced: two passes of 16
+// rows through a 2 KB buffer whose 16-byte chunks are XOR-swizzled by row, so
+// neither the shared-memory writes nor the reads conflict.
+__device__ __forceinline__ void store_rows32(float* stage, const uint32_t (&v)[32], float* gbase,
+                                             int64_t ld, int nvalid, int lane) {
+    float4* st4 = reinterpret_cast<float4*>(stage);
+#pragma unroll
+    for (int pass = 0; pass < 2; ++pass) {
+        if ((lane >> 4) == pass) {
+            const int r = lane & 15;
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                st4[r * 8 + (j ^ (r & 7))] = make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
+                                                         __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]));
+        }
+        __syncwarp();
+#pragma unroll
+        for (int it = 0; it < 4; ++it) {
+            const int r = it * 4 + (lane >> 3), c = lane & 7;
+            const float4 q = st4[r * 8 + (c ^ (r & 7))];
+            const int row = pass * 16 + r;
+            if (row < nvalid) reinterpret_cast<float4*>(gbase + (int64_t)row * ld)[c] = q;
+        }
+        __syncwarp();
+    }
+}
+
 // GEMM1 tile: columns 0..127 of the accumulator are gate channels
-// nt*128 + c, columns 128..255 the matching up channels.
+// nt*128 + c, columns 128..255 the matching up channels.  Each warp owns 32
+// rows (its TMEM lane quarter) and 64 of the 128 h columns.
 __device__ __forceinline__ void epilogue_swiglu(const TcParams& p, uint32_t taddr, int half, int e,
-                                                int nt, int grow, bool valid, float& amax,
+                                                int nt, int wrow0, int nvalid, float* stage,
                                                 Ctl* ctl, int buf, int lane) {
     const int f = p.f;
+    const bool valid = lane < nvalid;
+    const int grow = wrow0 + lane;
     float sxt = 0.0f;
     if (valid) sxt = p.sx[p.row2ts[grow] / p.k];
-    amax = 0.0f;
+    float amax = 0.0f;
 #pragma unroll 1
     for (int c = 0; c < 2; ++c) {
         const int col0 = 64 * half + 32 * c;
@@ -222,40 +265,42 @@ __device__ __forceinline__ void epilogue_swiglu(const TcParams& p, uint32_t tadd
             __syncwarp();
             if (lane == 0) mbar_arrive(&ctl->acc_empty[buf]);
         }
-        if (!valid) continue;
         const int ch0 = nt * 128 + col0;
         const float* swg = p.sw0 + (int64_t)e * f + ch0;
         const float* swu = p.sw1 + (int64_t)e * f + ch0;
-        float* hrow = p.h32 + (int64_t)grow * f + ch0;
-#pragma unroll
-        for (int j = 0; j < 32; j += 4) {
-            const float4 sg = *reinterpret_cast<const float4*>(swg + j);
-            const float4 su = *reinterpret_cast<const float4*>(swu + j);
-            const float sgv[4] = {sg.x, sg.y, sg.z, sg.w}, suv[4] = {su.x, su.y, su.z, su.w};
-            float hv[4];
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const float gf = __fmul_rn(__fmul_rn(__int2float_rn((int)g[j + q]), sxt), sgv[q]);
-                const float uf = __fmul_rn(__fmul_rn(__int2float_rn((int)u[j + q]), sxt), suv[q]);
-                hv[q] = __fmul_rn(moe_silu(gf), uf);
-                amax = fmaxf(amax, fabsf(hv[q]));
-            }
-            *reinterpret_cast<float4*>(hrow + j) = make_float4(hv[0], hv[1], hv[2], hv[3]);
-        }
-        if (p.acc_dbg) {
+        if (p.acc_dbg && valid) {
             int32_t* dg = p.acc_dbg + (int64_t)grow * 2 * f + ch0;
             for (int j = 0; j < 32; ++j) {
                 dg[j] = (int32_t)g[j];
                 dg[f + j] = (int32_t)u[j];
             }
         }
+        // h overwrites u in place (each u is dead once its h is formed)
+#pragma unroll
+        for (int j = 0; j < 32; j += 4) {
+            const float4 sg = *reinterpret_cast<const float4*>(swg + j);
+            const float4 su = *reinterpret_cast<const float4*>(swu + j);
+            const float sgv[4] = {sg.x, sg.y, sg.z, sg.w}, suv[4] = {su.x, su.y, su.z, su.w};
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const float gf = __fmul_rn(__fmul_rn(__int2float_rn((int)g[j + q]), sxt), sgv[q]);
+                const float uf = __fmul_rn(__fmul_rn(__int2float_rn((int)u[j + q]), sxt), suv[q]);
+                const float h = __fmul_rn(moe_silu(gf), uf);
+                if (valid) amax = fmaxf(amax, fabsf(h));
+                u[j + q] = __float_as_uint(h);
+            }
+        }
+        store_rows32(stage, u, p.h32 + (int64_t)wrow0 * f + ch0, f, nvalid, lane);
     }
+    if (valid) p.pamax[(int64_t)grow * (f / 64) + nt * 2 + half] = amax;
 }
 
 __device__ __forceinline__ void epilogue_down(const TcParams& p, uint32_t taddr, int half, int e,
-                                              int nt, int grow, bool valid, Ctl* ctl, int buf,
-                                              int lane) {
+                                              int nt, int wrow0, int nvalid, float* stage, Ctl* ctl,
+                                              int buf, int lane) {
     const int d = p.N;
+    const bool valid = lane < nvalid;
+    const int grow = wrow0 + lane;
     float shr = 0.0f, wr = 0.0f;
     if (valid) {
         shr = p.sh[grow];
@@ -272,32 +317,34 @@ __device__ __forceinline__ void epilogue_down(const TcParams& p, uint32_t taddr,
             __syncwarp();
             if (lane == 0) mbar_arrive(&ctl->acc_empty[buf]);
         }
-        if (!valid) continue;
         const int ch0 = nt * BN + col0;
         const float* sw = p.sw0 + (int64_t)e * d + ch0;
-        float* orow = p.o + (int64_t)grow * d + ch0;
+        if (p.acc_dbg && valid) {
+            int32_t* da = p.acc_dbg + (int64_t)grow * d + ch0;
+            for (int j = 0; j < 32; ++j) da[j] = (int32_t)a[j];
+        }
 #pragma unroll
         for (int j = 0; j < 32; j += 4) {
             const float4 s4 = *reinterpret_cast<const float4*>(sw + j);
             const float sv[4] = {s4.x, s4.y, s4.z, s4.w};
-            float ov[4];
 #pragma unroll
             for (int q = 0; q < 4; ++q)
-                ov[q] = __fmul_rn(__fmul_rn(__fmul_rn(__int2float_rn((int)a[j + q]), shr), sv[q]), wr);
-            *reinterpret_cast<float4*>(orow + j) = make_float4(ov[0], ov[1], ov[2], ov[3]);
+                a[j + q] = __float_as_uint(
+                    __fmul_rn(__fmul_rn(__fmul_rn(__int2float_rn((int)a[j + q]), shr), sv[q]), wr));
         }
-        if (p.acc_dbg) {
-            int32_t* da = p.acc_dbg + (int64_t)grow * d + ch0;
-            for (int j = 0; j < 32; ++j) da[j] = (int32_t)a[j];
-        }
+        store_rows32(stage, a, p.o + (int64_t)wrow0 * d + ch0, d, nvalid, lane);
     }
 }
 
-// Requantise the rows of a finished 128-row tile: sh = max over the row's
-// partial maxima / 127, codes rint(h / sh).  One warp per row.
-__device__ void requant_rows(const TcParams& p, int row0, int nrows, int ew, int lane) {
+// Requantisation item v: rows [16 (v % 8), +16) of row tile v / 8.  One warp:
+// per row, sh = max over the row's partial maxima / 127 and codes rint(h / sh).
+__device__ void requant_item(const TcParams& p, int v, int lane) {
+    const int mt = v / kRqItemsPerTile, part = v % kRqItemsPerTile;
+    const int e = p.tiles[2 * mt], row0 = p.tiles[2 * mt + 1];
+    const int nrows = min(BM, p.offsets[e + 1] - row0);
     const int f = p.f, npart = f / 64;
-    for (int r = ew; r < nrows; r += kEpiWarps) {
+    const int r1 = min(nrows, (part + 1) * kRqRows);
+    for (int r = part * kRqRows; r < r1; ++r) {
         const int grow = row0 + r;
         float m = 0.0f;
         for (int i = lane; i < npart; i += 32) m = fmaxf(m, __ldcg(p.pamax + (int64_t)grow * npart + i));
@@ -315,6 +362,35 @@ __device__ void requant_rows(const TcParams& p, int row0, int nrows, int ew, int
     }
 }
 
+// Claim the next published requantisation item (warp-uniform result, -1 when
+// the queue is empty).  The claim is a CAS on the head; the claimed slot is
+// then read until its writer has filled it (bounded).
+__device__ int rq_pop(const TcParams& p, volatile int* abort, int lane) {
+    int v = -1;
+    if (lane == 0) {
+        while (!*abort) {
+            const int h = __ldcg(p.rq_head);
+            const int t = __ldcg(p.rq_tail);
+            if (h >= t) break;
+            if (atomicCAS(p.rq_head, h, h + 1) != h) continue;
+            const uint64_t t0 = global_timer();
+            int x;
+            while ((x = __ldcg(p.rq_items + h)) == 0) {
+                if (global_timer() - t0 > kWaitBudgetNs) {
+                    *abort = 1;
+                    atomicExch(p.status, (int32_t)MOE_ERR_TIMEOUT);
+                    break;
+                }
+            }
+            v = x - 1;
+            break;
+        }
+    }
+    v = __shfl_sync(0xffffffffu, v, 0);
+    if (v >= 0) __threadfence();
+    return v;
+}
+
 // ------------------------------------------------------------------ the kernel
 
 template <int EPI>
@@ -323,7 +399,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                    const TcParams p) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
-    Ctl* ctl = reinterpret_cast<Ctl*>(smem + kStages * kStageBytes);
+    float* epi_stage = reinterpret_cast<float*>(smem + kStages * kStageBytes);
+    Ctl* ctl = reinterpret_cast<Ctl*>(smem + kStages * kStageBytes + kEpiWarps * kEpiStageBytes);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int num_tiles = p.meta[META_NTILES] * p.n_tiles_n;
     const int nkb = p.K / BK;
@@ -424,7 +501,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int ew = warp - 2;                 // 0..7
         const int quad = warp & 3;               // TMEM lanes this warp may access
         const int half = ew >> 2;                // which half of the tile's columns
-        const int r_in_tile = quad * 32 + lane;
+        float* stage = epi_stage + ew * (kEpiStageBytes / 4);
         int buf = 0;
         uint32_t aph = 0, it = 0;
         for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++it) {
@@ -433,36 +510,39 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int mt = t / p.n_tiles_n, nt = t % p.n_tiles_n;
             const int e = p.tiles[2 * mt], row0 = p.tiles[2 * mt + 1];
             const int nrows = min(BM, p.offsets[e + 1] - row0);
-            const int grow = row0 + r_in_tile;
-            const bool valid = r_in_tile < nrows;
+            const int wrow0 = row0 + quad * 32;                      // this warp's 32 rows
+            const int nvalid = max(0, min(32, nrows - quad * 32));
             const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(buf * BN);
             if (EPI == EPI_SWIGLU) {
-                float amax;
-                epilogue_swiglu(p, taddr, half, e, nt, grow, valid, amax, ctl, buf, lane);
-                if (valid) p.pamax[(int64_t)grow * (p.f / 64) + nt * 2 + half] = amax;
+                epilogue_swiglu(p, taddr, half, e, nt, wrow0, nvalid, stage, ctl, buf, lane);
                 // publish this warp's h and maxima, then count the column tile
                 __threadfence();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&ctl->ep_done);
                 if (ew == 0 && lane == 0) {
-                    int last = 0;
-                    if (mbar_wait(&ctl->ep_done, it & 1, abort, p.status))
-                        last = atomicAdd(p.mcount + mt, 1) == p.n_tiles_n - 1;
-                    *reinterpret_cast<volatile int*>(&ctl->last_flag) = last;
+                    if (mbar_wait(&ctl->ep_done, it & 1, abort, p.status) &&
+                        atomicAdd(p.mcount + mt, 1) == p.n_tiles_n - 1) {
+                        // last column tile of this row tile: its rows become requantisation items
+                        __threadfence();
+                        const int base = atomicAdd(p.rq_tail, kRqItemsPerTile);
+                        for (int i = 0; i < kRqItemsPerTile; ++i)
+                            atomicExch(p.rq_items + base + i, mt * kRqItemsPerTile + i + 1);
+                    }
                     mbar_arrive(&ctl->ep_go);
                 }
                 __syncwarp();
                 if (!mbar_wait(&ctl->ep_go, it & 1, abort, p.status)) break;
-                if (*reinterpret_cast<volatile int*>(&ctl->last_flag)) {
-                    // the last column tile of this row tile: every h of its rows is written
-                    __threadfence();
-                    requant_rows(p, row0, nrows, ew, lane);
-                }
+                const int v = rq_pop(p, abort, lane);
+                if (v >= 0) requant_item(p, v, lane);
             } else {
-                epilogue_down(p, taddr, half, e, nt, grow, valid, ctl, buf, lane);
+                epilogue_down(p, taddr, half, e, nt, wrow0, nvalid, stage, ctl, buf, lane);
             }
             buf ^= 1;
             if (buf == 0) aph ^= 1;
+        }
+        if (EPI == EPI_SWIGLU) {
+            // drain the requantisation queue (items published later are drained by their publisher)
+            for (int v = rq_pop(p, abort, lane); v >= 0; v = rq_pop(p, abort, lane)) requant_item(p, v, lane);
         }
     }
 
@@ -536,6 +616,7 @@ cudaError_t launch_tc_gemm1(const moe_w8a8_weights* w, int T, const int8_t* aq, 
                             const float* sx, float* h32, float* pamax, int32_t* mcount, int8_t* hq,
                             float* sh, int32_t* acc_dbg, cudaStream_t s) {
     const moe_w8a8_config& c = w->cfg;
+    const int max_tiles_rows = (T * c.top_k + BM - 1) / BM + c.n_experts;
     CUtensorMap ta;
     const int rows = T * c.top_k;
     if (!make_map(&ta, aq, c.d, rows, BM)) return cudaErrorInvalidValue;
@@ -555,6 +636,9 @@ cudaError_t launch_tc_gemm1(const moe_w8a8_weights* w, int T, const int8_t* aq, 
     p.h32 = h32;
     p.pamax = pamax;
     p.mcount = mcount;
+    p.rq_head = mcount + max_tiles_rows;          // layout of the zeroed sync area: counters,
+    p.rq_tail = mcount + max_tiles_rows + 1;      // head, tail, then the item slots
+    p.rq_items = mcount + max_tiles_rows + 2;
     p.hq = hq;
     p.sh_out = sh;
     p.acc_dbg = acc_dbg;

@@ -113,7 +113,7 @@ WsLayout ws_layout(const moe_w8a8_weights* w, int T) {
     L.o = take(tk * d * 4);
     L.h32 = take(stream ? 0 : tk * f * 4);
     L.pamax = take(stream ? 0 : tk * (f / 64) * 4);
-    L.mcount = take(stream ? 0 : max_tiles * 4);
+    L.mcount = take(stream ? 0 : (max_tiles * 9 + 2) * 4);   // counters, queue head/tail, items
     L.total = p;
     return L;
 }
