@@ -37,6 +37,7 @@ EXPORTS = (
     "moe_w8a8_check_status", "moe_w8a8_destroy", "moe_status_string",
     "moe_w8a8_last_launch_count", "moe_w8a8_profile_start", "moe_w8a8_profile_read",
     "moe_w8a8_profile_stop", "moe_w8a8_stage_name", "moe_w8a8_forward_noalloc",
+    "moe_w8a8_status_words",
 )
 
 MOE_NOALLOC_SCRATCH_BYTES = 8 << 20
@@ -97,6 +98,7 @@ def lib():
             "moe_w8a8_profile_stop": ([vp], i32),
             "moe_w8a8_stage_name": ([i32], ctypes.c_char_p),
             "moe_w8a8_forward_noalloc": ([vp, vp, i32, vp, vp, vp, vp], i32),
+            "moe_w8a8_status_words": ([vp, vp, i32, vp], i32),
         }
         for name, (args, res) in sig.items():
             fn = getattr(L, name)
@@ -326,3 +328,12 @@ def moe_w8a8_forward_noalloc(w: Weights, x, T: int, router_bias, router_logits, 
         _dev_ptr(router_bias, torch.float32, "router_bias", True),
         _dev_ptr(router_logits, torch.float32, "router_logits", True),
         _dev_ptr(y, _act_dtype(w.cfg.out_dtype), "y"), _stream(stream)), "moe_w8a8_forward_noalloc")
+
+
+def moe_w8a8_status_words(w: Weights, n: int = 5, stream=None):
+    """The handle's status words (code, then where a bounded wait gave up)."""
+    import numpy as np
+    out = np.zeros(n, dtype=np.int32)
+    _check(lib().moe_w8a8_status_words(w.handle, ctypes.c_void_p(out.ctypes.data), int(n),
+                                       _stream(stream)), "moe_w8a8_status_words")
+    return out

@@ -136,7 +136,19 @@ __device__ __forceinline__ uint64_t global_timer() {
 // Bounded wait for the phase of parity `parity` to complete.  Returns false
 // (after recording the timeout) when the budget runs out or another role
 // already gave up.
-__device__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort, int32_t* status) {
+// Record a timeout: status[0] = MOE_ERR_TIMEOUT; the first reporter also
+// leaves where it gave up in status[1..4] (site, block, tile iteration, extra).
+__device__ void report_timeout(int32_t* status, int site, int iter, int extra) {
+    atomicExch(status, (int32_t)MOE_ERR_TIMEOUT);
+    if (atomicCAS(status + 1, 0, site) == 0) {
+        status[2] = (int32_t)blockIdx.x;
+        status[3] = iter;
+        status[4] = extra;
+    }
+}
+
+__device__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort, int32_t* status,
+                          int site = 0, int iter = 0) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_timer();
     while (true) {
@@ -144,7 +156,7 @@ __device__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort, i
         if (*abort) return false;
         if (global_timer() - t0 > kWaitBudgetNs) {
             *abort = 1;
-            atomicExch(status, (int32_t)MOE_ERR_TIMEOUT);
+            report_timeout(status, site, iter, (int)parity);
             return false;
         }
     }
@@ -362,6 +374,14 @@ __device__ void requant_item(const TcParams& p, int v, int lane) {
     }
 }
 
+// Coherent GPU-scope load that the compiler may not hoist or merge (the queue
+// words change under other CTAs' atomics).
+__device__ __forceinline__ int ld_relaxed_gpu(const int* ptr) {
+    int v;
+    asm volatile("ld.relaxed.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(ptr) : "memory");
+    return v;
+}
+
 // Claim the next published requantisation item (warp-uniform result, -1 when
 // the queue is empty).  The claim is a CAS on the head; the claimed slot is
 // then read until its writer has filled it (bounded).
@@ -369,16 +389,16 @@ __device__ int rq_pop(const TcParams& p, volatile int* abort, int lane) {
     int v = -1;
     if (lane == 0) {
         while (!*abort) {
-            const int h = __ldcg(p.rq_head);
-            const int t = __ldcg(p.rq_tail);
+            const int h = ld_relaxed_gpu(p.rq_head);
+            const int t = ld_relaxed_gpu(p.rq_tail);
             if (h >= t) break;
             if (atomicCAS(p.rq_head, h, h + 1) != h) continue;
             const uint64_t t0 = global_timer();
             int x;
-            while ((x = __ldcg(p.rq_items + h)) == 0) {
+            while ((x = ld_relaxed_gpu(p.rq_items + h)) == 0) {
                 if (global_timer() - t0 > kWaitBudgetNs) {
                     *abort = 1;
-                    atomicExch(p.status, (int32_t)MOE_ERR_TIMEOUT);
+                    report_timeout(p.status, 7, h, t);
                     break;
                 }
             }
@@ -447,7 +467,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int e = p.tiles[2 * mt], row0 = p.tiles[2 * mt + 1];
                 const int brow = e * p.N + nt * BN;
                 for (int kb = 0; kb < nkb; ++kb) {
-                    if (!mbar_wait(&ctl->empty[s], ph ^ 1, abort, p.status)) { ok = false; break; }
+                    if (!mbar_wait(&ctl->empty[s], ph ^ 1, abort, p.status, 1, t)) { ok = false; break; }
                     mbar_arrive_expect_tx(&ctl->full[s], kStageBytes);
                     uint8_t* sa = smem + s * kStageBytes;
                     tma_load_2d(sa, &tm_a, &ctl->full[s], kb * BK, row0);
@@ -471,11 +491,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t ph = 0, aph = 0;
             bool ok = true;
             for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
-                if (!mbar_wait(&ctl->acc_empty[buf], aph ^ 1, abort, p.status)) break;
+                if (!mbar_wait(&ctl->acc_empty[buf], aph ^ 1, abort, p.status, 2, t)) break;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem + (uint32_t)(buf * BN);
                 for (int kb = 0; kb < nkb; ++kb) {
-                    if (!mbar_wait(&ctl->full[s], ph, abort, p.status)) { ok = false; break; }
+                    if (!mbar_wait(&ctl->full[s], ph, abort, p.status, 3, t)) { ok = false; break; }
                     tc_fence_after();
                     const uint32_t a_addr = smem_u32(smem + s * kStageBytes);
                     const uint32_t b_addr = a_addr + kABytes;
@@ -505,7 +525,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         int buf = 0;
         uint32_t aph = 0, it = 0;
         for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++it) {
-            if (!mbar_wait(&ctl->acc_full[buf], aph, abort, p.status)) break;
+            if (!mbar_wait(&ctl->acc_full[buf], aph, abort, p.status, 4, t)) break;
             tc_fence_after();
             const int mt = t / p.n_tiles_n, nt = t % p.n_tiles_n;
             const int e = p.tiles[2 * mt], row0 = p.tiles[2 * mt + 1];
@@ -520,7 +540,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&ctl->ep_done);
                 if (ew == 0 && lane == 0) {
-                    if (mbar_wait(&ctl->ep_done, it & 1, abort, p.status) &&
+                    if (mbar_wait(&ctl->ep_done, it & 1, abort, p.status, 5, t) &&
                         atomicAdd(p.mcount + mt, 1) == p.n_tiles_n - 1) {
                         // last column tile of this row tile: its rows become requantisation items
                         __threadfence();
@@ -531,7 +551,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     mbar_arrive(&ctl->ep_go);
                 }
                 __syncwarp();
-                if (!mbar_wait(&ctl->ep_go, it & 1, abort, p.status)) break;
+                if (!mbar_wait(&ctl->ep_go, it & 1, abort, p.status, 6, t)) break;
                 const int v = rq_pop(p, abort, lane);
                 if (v >= 0) requant_item(p, v, lane);
             } else {

@@ -442,6 +442,15 @@ moe_status moe_w8a8_check_status(const moe_w8a8_weights* w, moe_stream_t stream)
     return MOE_OK;
 }
 
+moe_status moe_w8a8_status_words(const moe_w8a8_weights* w, int32_t* words_host, int32_t n,
+                                 moe_stream_t stream) {
+    if (!w || !words_host || n < 0 || n > 16) return MOE_ERR_INVALID_ARG;
+    if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return MOE_ERR_CUDA;
+    if (n && cudaMemcpy(words_host, w->status, (size_t)n * 4, cudaMemcpyDeviceToHost) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    return MOE_OK;
+}
+
 void moe_w8a8_destroy(moe_w8a8_weights* w) { free_handle(w); }
 
 moe_status moe_w8a8_profile_start(moe_w8a8_weights* w, int32_t max_forwards) {
