@@ -224,8 +224,8 @@ moe_status moe_w8a8_check_status(const moe_w8a8_weights* w, moe_stream_t stream)
  * handle's status words to words_host[0..n) (n <= 16): word 0 is the status
  * code, words 1-4 say where the first bounded wait gave up (site: 1 producer
  * stage-free, 2 MMA accumulator-free, 3 MMA stage-full, 4 epilogue
- * accumulator-full, 5/6 epilogue tile handshake, 7 requantisation queue slot;
- * then block index, tile, and a site-specific value).  Does not clear them.
+ * accumulator-full; then block index, tile, and the awaited phase parity).
+ * Does not clear them.
  */
 moe_status moe_w8a8_status_words(const moe_w8a8_weights* w, int32_t* words_host, int32_t n,
                                  moe_stream_t stream);

@@ -51,7 +51,7 @@ struct WsLayout {
     size_t row2ts, ts2row;
     size_t xq, sx, aq;
     size_t acc1, hq, sh, o;
-    size_t h32, pamax, mcount;   // tensor path: fp32 h, per-row partial maxima, tile counters
+    size_t h32, pamax;           // tensor path: fp32 h, per-row partial maxima
     size_t total;
 };
 WsLayout ws_layout(const moe_w8a8_weights* w, int T);
@@ -79,7 +79,7 @@ cudaError_t launch_topk(const float* logits, const float* bias, int T, int E, in
                         int32_t* idx, float* wts, float* logits_out, cudaStream_t s);
 cudaError_t launch_permute(const int32_t* idx, int T, int k, int E, int cap, int32_t* hist,
                            int32_t* offsets, int32_t* row2ts, int32_t* ts2row, int32_t* meta,
-                           int32_t* active, int32_t* tiles, int32_t* mcount, cudaStream_t s);
+                           int32_t* active, int32_t* tiles, cudaStream_t s);
 cudaError_t launch_smooth_quant(const void* x, int in_dtype, const float* inv_s, int T, int d,
                                 int k, const int32_t* ts2row, int8_t* xq, float* sx, int8_t* aq,
                                 cudaStream_t s);
@@ -101,8 +101,10 @@ bool tc_make_weight_maps(moe_w8a8_weights* w);
 bool tc_supported(const moe_w8a8_config& c);
 cudaError_t launch_tc_gemm1(const moe_w8a8_weights* w, int T, const int8_t* aq, const int32_t* meta,
                             const int32_t* tiles, const int32_t* offsets, const int32_t* row2ts,
-                            const float* sx, float* h32, float* pamax, int32_t* mcount, int8_t* hq,
-                            float* sh, int32_t* acc_dbg, cudaStream_t s);
+                            const float* sx, float* h32, float* pamax, int32_t* acc_dbg,
+                            cudaStream_t s);
+cudaError_t launch_requant(const float* h32, const float* pamax, int f, const int32_t* meta,
+                           int max_rows, int8_t* hq, float* sh, cudaStream_t s);
 cudaError_t launch_tc_gemm2(const moe_w8a8_weights* w, int T, const int8_t* hq, const float* sh,
                             const int32_t* meta, const int32_t* tiles, const int32_t* offsets,
                             const int32_t* row2ts, const float* topk_w, float* o, int32_t* acc_dbg,

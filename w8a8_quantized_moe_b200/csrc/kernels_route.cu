@@ -196,7 +196,7 @@ __global__ void __launch_bounds__(kPermThreads) perm_scatter_kernel(
     const int32_t* __restrict__ idx, int n, int E, int cap, int nblk,
     const int32_t* __restrict__ hist, int32_t* __restrict__ offsets, int32_t* __restrict__ row2ts,
     int32_t* __restrict__ ts2row, int32_t* __restrict__ meta, int32_t* __restrict__ active,
-    int32_t* __restrict__ tiles, int32_t* __restrict__ mcount, int max_tiles) {
+    int32_t* __restrict__ tiles) {
     __shared__ int pre[kMaxE], off[kMaxE + 1], running[kMaxE], kept[kMaxE];
     __shared__ int wcnt[kPermThreads / 32][kMaxE];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -234,8 +234,6 @@ __global__ void __launch_bounds__(kPermThreads) perm_scatter_kernel(
         meta[META_NACTIVE] = na;
         meta[META_NTILES] = nt;
     }
-    if (blockIdx.x == 0 && mcount)   // tensor path: row-tile counters, requant queue head/tail/items
-        for (int i = tid; i < max_tiles * 9 + 2; i += blockDim.x) mcount[i] = 0;
     const int base = blockIdx.x * kPermChunk;
     for (int r0 = 0; r0 < kPermChunk; r0 += kPermThreads) {
         for (int i = tid; i < (kPermThreads / 32) * E; i += blockDim.x) wcnt[i / E][i % E] = 0;
@@ -342,15 +340,14 @@ cudaError_t launch_topk(const float* logits, const float* bias, int T, int E, in
 
 cudaError_t launch_permute(const int32_t* idx, int T, int k, int E, int cap, int32_t* hist,
                            int32_t* offsets, int32_t* row2ts, int32_t* ts2row, int32_t* meta,
-                           int32_t* active, int32_t* tiles, int32_t* mcount, cudaStream_t s) {
+                           int32_t* active, int32_t* tiles, cudaStream_t s) {
     const int n = T * k;
-    const int max_tiles = (n + kTileM - 1) / kTileM + E;
     const int nblk = (n + kPermChunk - 1) / kPermChunk;
     perm_hist_kernel<<<nblk, 256, 0, s>>>(idx, n, E, hist);
     cudaError_t err = cudaGetLastError();
     if (err != cudaSuccess) return err;
     perm_scatter_kernel<<<nblk, kPermThreads, 0, s>>>(idx, n, E, cap, nblk, hist, offsets, row2ts,
-                                                      ts2row, meta, active, tiles, mcount, max_tiles);
+                                                      ts2row, meta, active, tiles);
     return cudaGetLastError();
 }
 

@@ -16,14 +16,11 @@
 //   warps 2..9  epilogue: tcgen05.ld of their 32-lane quarter of the
 //               accumulator, dequantisation and the fused math, global stores
 // GEMM1 epilogue: g, u dequantised (per-token x per-channel scales), h = silu(g)
-// u written in fp32 with per-row partial maxima.  Completion of a 128-row tile
-// is counted with an atomic; the CTA that completes its last column tile
-// publishes the tile's rows as 8 requantisation items (16 rows each) on a
-// device-wide queue, and every epilogue warp of every CTA claims at most one
-// item per tile it finishes (and drains the queue before exiting), so the
-// requantisation (row max over all f channels -> INT8) is spread over the GPU
-// while h is still in L2.  Nothing ever waits for another CTA.
-// GEMM2 epilogue: o = acc2 sh sw w in fp32 per sorted row.
+// u written in fp32 with one partial row maximum per 64 columns; the row-wide
+// INT8 requantisation of h (max over all f channels) is a separate,
+// bandwidth-bound kernel (requant_kernel below), so no CTA ever waits for or
+// coordinates with another.  GEMM2 epilogue: o = acc2 sh sw w in fp32 per
+// sorted row.
 // Epilogue stores go through a small swizzled shared-memory buffer per warp so
 // that each global store instruction writes whole 128-byte rows.
 //
@@ -50,8 +47,7 @@ constexpr uint32_t kTmemCols = 2 * BN;            // two 256-column accumulators
 constexpr uint64_t kWaitBudgetNs = 2000000000ull; // 2 s per wait
 constexpr int kEpiStageBytes = 16 * 32 * 4;      // 16 rows x 32 fp32 per epilogue warp
 constexpr size_t kSmemBytes = (size_t)kStages * kStageBytes + (size_t)kEpiWarps * kEpiStageBytes + 1024 + 256;
-constexpr int kRqRows = 16;                       // rows per requantisation item
-constexpr int kRqItemsPerTile = 128 / kRqRows;
+
 
 // Instruction descriptor, kind::i8: D = s32 (bits 4-5 = 2), A and B signed
 // 8-bit (bits 7-9, 10-12 = 1), both K-major, N>>3 at bit 17, M>>4 at bit 24.
@@ -64,11 +60,8 @@ struct Ctl {
     uint64_t acc_full[2];
     uint64_t acc_empty[2];
     uint64_t drain;
-    uint64_t ep_done;   // GEMM1: all epilogue warps finished a tile's stores
-    uint64_t ep_go;     // GEMM1: the tile's completion count has been taken
     uint32_t tmem_base;
     int abort;
-    int last_flag;
 };
 
 struct TcParams {
@@ -84,12 +77,6 @@ struct TcParams {
     const float* sh;          // GEMM2: per-row h scale
     float* h32;               // GEMM1: h [rows][f]
     float* pamax;             // GEMM1: per-row partial max [rows][f/64]
-    int32_t* mcount;          // GEMM1: completed column tiles per row tile
-    int32_t* rq_head;         // GEMM1: requantisation queue: next item to claim
-    int32_t* rq_tail;         //        items published so far
-    int32_t* rq_items;        //        item + 1 (0 = not yet written)
-    int8_t* hq;               // GEMM1: requantised h [rows][f]
-    float* sh_out;            // GEMM1: per-row h scale
     float* o;                 // GEMM2: [rows][d]
     int32_t* acc_dbg;         // optional raw accumulators (canonical channel order)
     int32_t* status;
@@ -348,69 +335,6 @@ __device__ __forceinline__ void epilogue_down(const TcParams& p, uint32_t taddr,
     }
 }
 
-// Requantisation item v: rows [16 (v % 8), +16) of row tile v / 8.  One warp:
-// per row, sh = max over the row's partial maxima / 127 and codes rint(h / sh).
-__device__ void requant_item(const TcParams& p, int v, int lane) {
-    const int mt = v / kRqItemsPerTile, part = v % kRqItemsPerTile;
-    const int e = p.tiles[2 * mt], row0 = p.tiles[2 * mt + 1];
-    const int nrows = min(BM, p.offsets[e + 1] - row0);
-    const int f = p.f, npart = f / 64;
-    const int r1 = min(nrows, (part + 1) * kRqRows);
-    for (int r = part * kRqRows; r < r1; ++r) {
-        const int grow = row0 + r;
-        float m = 0.0f;
-        for (int i = lane; i < npart; i += 32) m = fmaxf(m, __ldcg(p.pamax + (int64_t)grow * npart + i));
-        m = warp_max(m);
-        const float s = m > 0.0f ? __fdiv_rn(m, 127.0f) : 0.0f;
-        if (lane == 0) p.sh_out[grow] = s;
-        const float4* hrow = reinterpret_cast<const float4*>(p.h32 + (int64_t)grow * f);
-        uint32_t* qrow = reinterpret_cast<uint32_t*>(p.hq + (int64_t)grow * f);
-        for (int c4 = lane; c4 < f / 4; c4 += 32) {
-            const float4 h = __ldcg(hrow + c4);
-            qrow[c4] = s > 0.0f ? pack4(quant_code(h.x, s), quant_code(h.y, s), quant_code(h.z, s),
-                                        quant_code(h.w, s))
-                                : 0u;
-        }
-    }
-}
-
-// Coherent GPU-scope load that the compiler may not hoist or merge (the queue
-// words change under other CTAs' atomics).
-__device__ __forceinline__ int ld_relaxed_gpu(const int* ptr) {
-    int v;
-    asm volatile("ld.relaxed.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(ptr) : "memory");
-    return v;
-}
-
-// Claim the next published requantisation item (warp-uniform result, -1 when
-// the queue is empty).  The claim is a CAS on the head; the claimed slot is
-// then read until its writer has filled it (bounded).
-__device__ int rq_pop(const TcParams& p, volatile int* abort, int lane) {
-    int v = -1;
-    if (lane == 0) {
-        while (!*abort) {
-            const int h = ld_relaxed_gpu(p.rq_head);
-            const int t = ld_relaxed_gpu(p.rq_tail);
-            if (h >= t) break;
-            if (atomicCAS(p.rq_head, h, h + 1) != h) continue;
-            const uint64_t t0 = global_timer();
-            int x;
-            while ((x = ld_relaxed_gpu(p.rq_items + h)) == 0) {
-                if (global_timer() - t0 > kWaitBudgetNs) {
-                    *abort = 1;
-                    report_timeout(p.status, 7, h, t);
-                    break;
-                }
-            }
-            v = x - 1;
-            break;
-        }
-    }
-    v = __shfl_sync(0xffffffffu, v, 0);
-    if (v >= 0) __threadfence();
-    return v;
-}
-
 // ------------------------------------------------------------------ the kernel
 
 template <int EPI>
@@ -435,10 +359,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&ctl->acc_empty[b], kEpiWarps);
         }
         mbar_init(&ctl->drain, 1);
-        mbar_init(&ctl->ep_done, kEpiWarps);
-        mbar_init(&ctl->ep_go, 1);
         ctl->abort = 0;
-        ctl->last_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     if (warp == 1) {
@@ -523,8 +444,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int half = ew >> 2;                // which half of the tile's columns
         float* stage = epi_stage + ew * (kEpiStageBytes / 4);
         int buf = 0;
-        uint32_t aph = 0, it = 0;
-        for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++it) {
+        uint32_t aph = 0;
+        for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
             if (!mbar_wait(&ctl->acc_full[buf], aph, abort, p.status, 4, t)) break;
             tc_fence_after();
             const int mt = t / p.n_tiles_n, nt = t % p.n_tiles_n;
@@ -533,36 +454,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int wrow0 = row0 + quad * 32;                      // this warp's 32 rows
             const int nvalid = max(0, min(32, nrows - quad * 32));
             const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(buf * BN);
-            if (EPI == EPI_SWIGLU) {
+            if (EPI == EPI_SWIGLU)
                 epilogue_swiglu(p, taddr, half, e, nt, wrow0, nvalid, stage, ctl, buf, lane);
-                // publish this warp's h and maxima, then count the column tile
-                __threadfence();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&ctl->ep_done);
-                if (ew == 0 && lane == 0) {
-                    if (mbar_wait(&ctl->ep_done, it & 1, abort, p.status, 5, t) &&
-                        atomicAdd(p.mcount + mt, 1) == p.n_tiles_n - 1) {
-                        // last column tile of this row tile: its rows become requantisation items
-                        __threadfence();
-                        const int base = atomicAdd(p.rq_tail, kRqItemsPerTile);
-                        for (int i = 0; i < kRqItemsPerTile; ++i)
-                            atomicExch(p.rq_items + base + i, mt * kRqItemsPerTile + i + 1);
-                    }
-                    mbar_arrive(&ctl->ep_go);
-                }
-                __syncwarp();
-                if (!mbar_wait(&ctl->ep_go, it & 1, abort, p.status, 6, t)) break;
-                const int v = rq_pop(p, abort, lane);
-                if (v >= 0) requant_item(p, v, lane);
-            } else {
+            else
                 epilogue_down(p, taddr, half, e, nt, wrow0, nvalid, stage, ctl, buf, lane);
-            }
             buf ^= 1;
             if (buf == 0) aph ^= 1;
-        }
-        if (EPI == EPI_SWIGLU) {
-            // drain the requantisation queue (items published later are drained by their publisher)
-            for (int v = rq_pop(p, abort, lane); v >= 0; v = rq_pop(p, abort, lane)) requant_item(p, v, lane);
         }
     }
 
@@ -571,6 +468,36 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == 1) {
         tc_fence_after();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols));
+    }
+}
+
+// ------------------------------------------------------------------ requantisation of h
+
+// One warp per sorted row: sh = max over the row's partial maxima / 127 and
+// codes rint(h / sh), ties to even, clamped to +-127 (sh = 0 gives 0).
+constexpr int kRqThreads = 256;
+
+__global__ void __launch_bounds__(kRqThreads) requant_kernel(const float* __restrict__ h32,
+                                                             const float* __restrict__ pamax, int f,
+                                                             const int32_t* __restrict__ meta,
+                                                             int8_t* __restrict__ hq,
+                                                             float* __restrict__ sh) {
+    const int lane = threadIdx.x & 31;
+    const int row = blockIdx.x * (kRqThreads / 32) + (threadIdx.x >> 5);
+    if (row >= meta[META_R]) return;
+    const int npart = f / 64;
+    float m = 0.0f;
+    for (int i = lane; i < npart; i += 32) m = fmaxf(m, pamax[(int64_t)row * npart + i]);
+    m = warp_max(m);
+    const float s = m > 0.0f ? __fdiv_rn(m, 127.0f) : 0.0f;
+    if (lane == 0) sh[row] = s;
+    const float4* hrow = reinterpret_cast<const float4*>(h32 + (int64_t)row * f);
+    uint32_t* qrow = reinterpret_cast<uint32_t*>(hq + (int64_t)row * f);
+    for (int c4 = lane; c4 < f / 4; c4 += 32) {
+        const float4 h = hrow[c4];
+        qrow[c4] = s > 0.0f ? pack4(quant_code(h.x, s), quant_code(h.y, s), quant_code(h.z, s),
+                                    quant_code(h.w, s))
+                            : 0u;
     }
 }
 
@@ -631,12 +558,19 @@ bool tc_make_weight_maps(moe_w8a8_weights* w) {
 
 bool tc_supported(const moe_w8a8_config& c) { return c.d % BN == 0 && c.f % BK == 0 && c.d % BK == 0; }
 
+cudaError_t launch_requant(const float* h32, const float* pamax, int f, const int32_t* meta,
+                           int max_rows, int8_t* hq, float* sh, cudaStream_t s) {
+    const int rows_per_block = kRqThreads / 32;
+    requant_kernel<<<(max_rows + rows_per_block - 1) / rows_per_block, kRqThreads, 0, s>>>(
+        h32, pamax, f, meta, hq, sh);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_tc_gemm1(const moe_w8a8_weights* w, int T, const int8_t* aq, const int32_t* meta,
                             const int32_t* tiles, const int32_t* offsets, const int32_t* row2ts,
-                            const float* sx, float* h32, float* pamax, int32_t* mcount, int8_t* hq,
-                            float* sh, int32_t* acc_dbg, cudaStream_t s) {
+                            const float* sx, float* h32, float* pamax, int32_t* acc_dbg,
+                            cudaStream_t s) {
     const moe_w8a8_config& c = w->cfg;
-    const int max_tiles_rows = (T * c.top_k + BM - 1) / BM + c.n_experts;
     CUtensorMap ta;
     const int rows = T * c.top_k;
     if (!make_map(&ta, aq, c.d, rows, BM)) return cudaErrorInvalidValue;
@@ -655,12 +589,6 @@ cudaError_t launch_tc_gemm1(const moe_w8a8_weights* w, int T, const int8_t* aq, 
     p.sw1 = w->sw_up;
     p.h32 = h32;
     p.pamax = pamax;
-    p.mcount = mcount;
-    p.rq_head = mcount + max_tiles_rows;          // layout of the zeroed sync area: counters,
-    p.rq_tail = mcount + max_tiles_rows + 1;      // head, tail, then the item slots
-    p.rq_items = mcount + max_tiles_rows + 2;
-    p.hq = hq;
-    p.sh_out = sh;
     p.acc_dbg = acc_dbg;
     p.status = w->status;
     const int max_mt = (rows + BM - 1) / BM + c.n_experts;

@@ -113,7 +113,6 @@ WsLayout ws_layout(const moe_w8a8_weights* w, int T) {
     L.o = take(tk * d * 4);
     L.h32 = take(stream ? 0 : tk * f * 4);
     L.pamax = take(stream ? 0 : tk * (f / 64) * 4);
-    L.mcount = take(stream ? 0 : (max_tiles * 9 + 2) * 4);   // counters, queue head/tail, items
     L.total = p;
     return L;
 }
@@ -280,9 +279,8 @@ static moe_status forward_impl(const moe_w8a8_weights* w, const void* x, int T, 
     mark(MOE_STAGE_TOPK, 1);
     ++launches;
     mark(MOE_STAGE_PERMUTE, 0);
-    const bool tensor = path == MOE_PATH_TENSOR;
     CUDA_TRY(launch_permute(idx, T, k, E, capacity_of(c, T), (int32_t*)P(L.hist), offsets, row2ts,
-                            ts2row, meta, active, tiles, tensor ? (int32_t*)P(L.mcount) : nullptr, s));
+                            ts2row, meta, active, tiles, s));
     mark(MOE_STAGE_PERMUTE, 1);
     launches += 2;
     if (path == MOE_PATH_STREAM) {
@@ -310,15 +308,16 @@ static moe_status forward_impl(const moe_w8a8_weights* w, const void* x, int T, 
         mark(MOE_STAGE_QUANT, 1);
         mark(MOE_STAGE_GEMM1, 0);
         CUDA_TRY(launch_tc_gemm1(w, T, aq, meta, tiles, offsets, row2ts, sx, (float*)P(L.h32),
-                                 (float*)P(L.pamax), (int32_t*)P(L.mcount), hq, sh,
-                                 dbg ? dbg->acc1 : nullptr, s));
+                                 (float*)P(L.pamax), dbg ? dbg->acc1 : nullptr, s));
         mark(MOE_STAGE_GEMM1, 1);
-        empty_stage(MOE_STAGE_REQUANT);
+        mark(MOE_STAGE_REQUANT, 0);
+        CUDA_TRY(launch_requant((float*)P(L.h32), (float*)P(L.pamax), f, meta, (int)tk, hq, sh, s));
+        mark(MOE_STAGE_REQUANT, 1);
         mark(MOE_STAGE_GEMM2, 0);
         CUDA_TRY(launch_tc_gemm2(w, T, hq, sh, meta, tiles, offsets, row2ts, wts, o,
                                  dbg ? dbg->acc2 : nullptr, s));
         mark(MOE_STAGE_GEMM2, 1);
-        launches += 3;
+        launches += 4;
     }
     mark(MOE_STAGE_COMBINE, 0);
     CUDA_TRY(launch_combine(o, ts2row, T, k, d, c.out_dtype, y, s));
