@@ -47,6 +47,8 @@ def parse():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-stage-events", action="store_true")
+    p.add_argument("--path", choices=["auto", "stream", "tensor"], default="auto",
+                   help="expert GEMM path: weight streaming, tcgen05 grouped GEMM, or automatic")
     p.add_argument("--tokens", type=int, default=0,
                    help="override the workload's token count T (same layer, same seeds)")
     p.add_argument("--no-prefill", action="store_true",
@@ -258,6 +260,8 @@ def measure(args, wl, world, rank, local, e2e_on=True, wts=None):
     wg, wu, wd = (torch.from_numpy(a).to(dev) for a in (wts.w_gate, wts.w_up, wts.w_down))
     wr = torch.from_numpy(data.w_router).to(dev)
     W = M.moe_w8a8_prepare(cfg, wg, wu, wd, wr, ax)
+    M.moe_w8a8_set_path(W, {"auto": M.MOE_PATH_AUTO, "stream": M.MOE_PATH_STREAM,
+                            "tensor": M.MOE_PATH_TENSOR}[args.path])
     del wg, wu, wd, cal
     torch.cuda.empty_cache()
 
@@ -275,7 +279,7 @@ def measure(args, wl, world, rank, local, e2e_on=True, wts=None):
     counts = np.diff(offs.cpu().numpy())
     n_active, R = int((counts > 0).sum()), int(counts.sum())
     alg = algorithmic(wl, n_active, R)
-    tensor = T * wl.k > 512
+    tensor = args.path == "tensor" or (args.path == "auto" and T * wl.k > 512)
 
     stream = torch.cuda.current_stream(dev)
     for _ in range(args.warmup):
