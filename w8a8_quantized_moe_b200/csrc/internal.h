@@ -80,6 +80,11 @@ cudaError_t launch_topk(const float* logits, const float* bias, int T, int E, in
 cudaError_t launch_permute(const int32_t* idx, int T, int k, int E, int cap, int32_t* hist,
                            int32_t* offsets, int32_t* row2ts, int32_t* ts2row, int32_t* meta,
                            int32_t* active, int32_t* tiles, cudaStream_t s);
+bool route_small_ok(int T, int k);
+cudaError_t launch_route_small(const float* logits, const float* bias, int T, int E, int k,
+                               int renorm, int cap, int32_t* idx, float* wts, float* logits_out,
+                               int32_t* offsets, int32_t* row2ts, int32_t* ts2row, int32_t* meta,
+                               int32_t* active, int32_t* tiles, cudaStream_t s);
 cudaError_t launch_smooth_quant(const void* x, int in_dtype, const float* inv_s, int T, int d,
                                 int k, const int32_t* ts2row, int8_t* xq, float* sx, int8_t* aq,
                                 cudaStream_t s);

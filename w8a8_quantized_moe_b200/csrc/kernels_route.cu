@@ -108,13 +108,14 @@ __device__ __forceinline__ bool better(float v, int i, float v2, int i2) {
     return v > v2 || (v == v2 && i < i2);
 }
 
-__global__ void topk_kernel(const float* __restrict__ logits, const float* __restrict__ bias, int T,
-                            int E, int k, int renorm, int32_t* __restrict__ idx,
-                            float* __restrict__ wts, float* __restrict__ logits_out) {
-    __shared__ float lsh[8][kMaxE];
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int t = blockIdx.x * 8 + warp;
-    if (t >= T) return;
+// One warp: top-k and gate weights of token t.  lsh: kMaxE floats of shared
+// scratch for this warp (used when the softmax runs over all E experts).
+// When idx_copy is given, the chosen experts are also written there.
+__device__ __forceinline__ void topk_token(const float* __restrict__ logits,
+                                           const float* __restrict__ bias, int t, int E, int k,
+                                           int renorm, int32_t* __restrict__ idx,
+                                           float* __restrict__ wts, float* __restrict__ logits_out,
+                                           float* lsh, int32_t* idx_copy, int lane) {
     constexpr int kPer = kMaxE / 32;
     float l[kPer];
     bool taken[kPer];
@@ -126,7 +127,7 @@ __global__ void topk_kernel(const float* __restrict__ logits, const float* __res
             v = logits[(int64_t)t * E + e];
             if (bias) v = __fadd_rn(v, bias[e]);
             if (logits_out) logits_out[(int64_t)t * E + e] = v;
-            lsh[warp][e] = v;
+            lsh[e] = v;
         }
         l[m] = v;
         taken[m] = e >= E;
@@ -156,28 +157,108 @@ __global__ void topk_kernel(const float* __restrict__ logits, const float* __res
         sel_i[s] = bi;
     }
     __syncwarp();
-    if (lane == 0) {
-        const float lmax = sel_v[0];
-        float z = 0.0f;
-        if (renorm) {
-            for (int s = 0; s < k; ++s) z = __fadd_rn(z, moe_exp(__fsub_rn(sel_v[s], lmax)));
-        } else {
-            for (int e = 0; e < E; ++e) z = __fadd_rn(z, moe_exp(__fsub_rn(lsh[warp][e], lmax)));
-        }
-        for (int s = 0; s < k; ++s) {
+    // slot s is handled by lane s: exp of each selected logit in parallel, the
+    // normaliser summed in slot (or expert) order by a fixed sequence of adds
+    const float lmax = sel_v[0];
+    float z = 0.0f;
+    if (renorm) {
+        for (int s = 0; s < k; ++s) z = __fadd_rn(z, moe_exp(__fsub_rn(sel_v[s], lmax)));
+    } else {
+        for (int e = 0; e < E; ++e) z = __fadd_rn(z, moe_exp(__fsub_rn(lsh[e], lmax)));
+    }
+#pragma unroll
+    for (int s = 0; s < kMaxK; ++s) {
+        if (s >= k) break;
+        if (lane == s) {
             idx[(int64_t)t * k + s] = sel_i[s];
             wts[(int64_t)t * k + s] = __fdiv_rn(moe_exp(__fsub_rn(sel_v[s], lmax)), z);
+            if (idx_copy) idx_copy[t * k + s] = sel_i[s];
         }
     }
 }
 
+__global__ void topk_kernel(const float* __restrict__ logits, const float* __restrict__ bias, int T,
+                            int E, int k, int renorm, int32_t* __restrict__ idx,
+                            float* __restrict__ wts, float* __restrict__ logits_out) {
+    __shared__ float lsh[8][kMaxE];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int t = blockIdx.x * 8 + warp;
+    if (t >= T) return;
+    topk_token(logits, bias, t, E, k, renorm, idx, wts, logits_out, lsh[warp], nullptr, lane);
+}
+
 // ---------------------------------------------------------------------------
-// Sort by expert: histogram per chunk of kPermChunk entries (t*k + slot
-// order), then a scatter in which every block derives the global expert
-// offsets and its own prefix from the histogram and ranks its entries stably
-// (warp match + per-warp counts).  Entry i of expert e gets position
-// pos = #(earlier entries of e); it is kept when pos < capacity.
+// Sort by expert.  Entry i (= t*k + slot) of expert e gets position
+// pos = #(earlier entries of e) and is kept when pos < capacity; kept rows are
+// ordered by expert, then by i.  Large inputs: a histogram per chunk of
+// kPermChunk entries, then a scatter in which every block derives the global
+// expert offsets and its own prefix from the histogram.  Small inputs: one
+// block does top-k, histogram, scan and scatter.
 // ---------------------------------------------------------------------------
+
+// Expert offsets (exclusive scan of kept counts) and the lists the expert
+// kernels read: active experts and 128-row tiles.  Written by one thread.
+__device__ void write_offsets_and_lists(const int* kept, int E, int* off, int32_t* offsets,
+                                        int32_t* meta, int32_t* active, int32_t* tiles) {
+    int acc = 0;
+    for (int e = 0; e < E; ++e) { off[e] = acc; acc += kept[e]; }
+    off[E] = acc;
+    int na = 0, nt = 0;
+    for (int e = 0; e <= E; ++e) offsets[e] = off[e];
+    for (int e = 0; e < E; ++e) {
+        if (kept[e] == 0) continue;
+        active[na++] = e;
+        for (int m = 0; m * kTileM < kept[e]; ++m) {
+            tiles[2 * nt] = e;
+            tiles[2 * nt + 1] = off[e] + m * kTileM;
+            ++nt;
+        }
+    }
+    meta[META_R] = off[E];
+    meta[META_NACTIVE] = na;
+    meta[META_NTILES] = nt;
+}
+
+// Stable ranks of entries [base, base + len) in rounds of blockDim.x: warp
+// match for ranks inside a warp, per-warp counts (wcnt, [warps][kMaxE]) for
+// ranks across warps, running per-expert totals across rounds.  pre[e]: entries
+// of e before `base`.  Block-wide; needs off[], pre[], running[] in shared.
+__device__ void scatter_entries(const int32_t* idx, int base, int len, int E, int cap,
+                                const int* pre, const int* off, int* running, int (*wcnt)[kMaxE],
+                                int32_t* __restrict__ row2ts, int32_t* __restrict__ ts2row) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
+    for (int r0 = 0; r0 < len; r0 += blockDim.x) {
+        for (int i = tid; i < nw * E; i += blockDim.x) wcnt[i / E][i % E] = 0;
+        __syncthreads();
+        const int i = base + r0 + tid;
+        const bool valid = r0 + tid < len;
+        const int e = valid ? idx[i] : -1;
+        const unsigned m = __match_any_sync(0xffffffffu, e);
+        const int rank_w = __popc(m & ((1u << lane) - 1u));
+        if (valid && rank_w == 0) wcnt[warp][e] = __popc(m);
+        __syncthreads();
+        if (valid) {
+            int rank = running[e] + rank_w;
+            for (int w2 = 0; w2 < warp; ++w2) rank += wcnt[w2][e];
+            const int pos = pre[e] + rank;
+            const int row = off[e] + pos;
+            if ((cap < 0 || pos < cap) && row < off[E]) {   // row < R always holds; guard the store
+                ts2row[i] = row;
+                row2ts[row] = i;
+            } else {
+                ts2row[i] = -1;
+            }
+        }
+        __syncthreads();
+        for (int e2 = tid; e2 < E; e2 += blockDim.x) {
+            int s = 0;
+            for (int w2 = 0; w2 < nw; ++w2) s += wcnt[w2][e2];
+            running[e2] += s;
+        }
+        __syncthreads();
+    }
+}
+
 __global__ void perm_hist_kernel(const int32_t* __restrict__ idx, int n, int E,
                                  int32_t* __restrict__ hist) {
     __shared__ int cnt[kMaxE];
@@ -199,7 +280,7 @@ __global__ void __launch_bounds__(kPermThreads) perm_scatter_kernel(
     int32_t* __restrict__ tiles) {
     __shared__ int pre[kMaxE], off[kMaxE + 1], running[kMaxE], kept[kMaxE];
     __shared__ int wcnt[kPermThreads / 32][kMaxE];
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int tid = threadIdx.x;
     for (int e = tid; e < E; e += blockDim.x) {
         int tot = 0, before = 0;
         for (int b = 0; b < nblk; ++b) {
@@ -213,58 +294,61 @@ __global__ void __launch_bounds__(kPermThreads) perm_scatter_kernel(
     }
     __syncthreads();
     if (tid == 0) {
-        int acc = 0;
-        for (int e = 0; e < E; ++e) { off[e] = acc; acc += kept[e]; }
-        off[E] = acc;
+        if (blockIdx.x == 0) {
+            write_offsets_and_lists(kept, E, off, offsets, meta, active, tiles);
+        } else {
+            int acc = 0;
+            for (int e = 0; e < E; ++e) { off[e] = acc; acc += kept[e]; }
+            off[E] = acc;
+        }
     }
     __syncthreads();
-    if (blockIdx.x == 0 && tid == 0) {
-        int na = 0, nt = 0;
-        for (int e = 0; e <= E; ++e) offsets[e] = off[e];
-        for (int e = 0; e < E; ++e) {
-            if (kept[e] == 0) continue;
-            active[na++] = e;
-            for (int m = 0; m * kTileM < kept[e]; ++m) {
-                tiles[2 * nt] = e;
-                tiles[2 * nt + 1] = off[e] + m * kTileM;
-                ++nt;
-            }
-        }
-        meta[META_R] = off[E];
-        meta[META_NACTIVE] = na;
-        meta[META_NTILES] = nt;
-    }
     const int base = blockIdx.x * kPermChunk;
-    for (int r0 = 0; r0 < kPermChunk; r0 += kPermThreads) {
-        for (int i = tid; i < (kPermThreads / 32) * E; i += blockDim.x) wcnt[i / E][i % E] = 0;
-        __syncthreads();
-        const int i = base + r0 + tid;
-        const bool valid = i < n;
-        const int e = valid ? idx[i] : -1;
-        const unsigned m = __match_any_sync(0xffffffffu, e);
-        const int rank_w = __popc(m & ((1u << lane) - 1u));
-        if (valid && rank_w == 0) wcnt[warp][e] = __popc(m);
-        __syncthreads();
-        if (valid) {
-            int rank = running[e] + rank_w;
-            for (int w2 = 0; w2 < warp; ++w2) rank += wcnt[w2][e];
-            const int pos = pre[e] + rank;
-            const int row = off[e] + pos;
-            if ((cap < 0 || pos < cap) && row < off[E]) {   // row < R always holds; guard the store
-                ts2row[i] = row;
-                row2ts[row] = i;
-            } else {
-                ts2row[i] = -1;
-            }
-        }
-        __syncthreads();
-        for (int e2 = tid; e2 < E; e2 += blockDim.x) {
-            int s = 0;
-            for (int w2 = 0; w2 < kPermThreads / 32; ++w2) s += wcnt[w2][e2];
-            running[e2] += s;
-        }
-        __syncthreads();
+    scatter_entries(idx, base, min(kPermChunk, n - base), E, cap, pre, off, running, wcnt, row2ts,
+                    ts2row);
+}
+
+// Small inputs (T*k <= kRouteSmallMax): top-k, histogram, scan and stable
+// scatter in one block of 1024 threads (warp w does tokens w, w + 32, ...).
+constexpr int kRouteSmallThreads = 1024;
+constexpr int kRouteSmallMax = 2048;
+
+struct RouteSmallSmem {
+    int32_t idx[kRouteSmallMax];
+    int pre[kMaxE], off[kMaxE + 1], running[kMaxE], kept[kMaxE];
+    union {
+        float lsh[kRouteSmallThreads / 32][kMaxE];
+        int wcnt[kRouteSmallThreads / 32][kMaxE];
+    } u;
+};
+
+__global__ void __launch_bounds__(kRouteSmallThreads) route_small_kernel(
+    const float* __restrict__ logits, const float* __restrict__ bias, int T, int E, int k,
+    int renorm, int cap, int32_t* __restrict__ idx, float* __restrict__ wts,
+    float* __restrict__ logits_out, int32_t* __restrict__ offsets, int32_t* __restrict__ row2ts,
+    int32_t* __restrict__ ts2row, int32_t* __restrict__ meta, int32_t* __restrict__ active,
+    int32_t* __restrict__ tiles) {
+    extern __shared__ __align__(16) uint8_t smem_raw[];
+    RouteSmallSmem& sm = *reinterpret_cast<RouteSmallSmem*>(smem_raw);
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int n = T * k;
+    for (int t = warp; t < T; t += kRouteSmallThreads / 32)
+        topk_token(logits, bias, t, E, k, renorm, idx, wts, logits_out, sm.u.lsh[warp], sm.idx, lane);
+    for (int e = tid; e < E; e += blockDim.x) {
+        sm.kept[e] = 0;
+        sm.pre[e] = 0;
+        sm.running[e] = 0;
     }
+    __syncthreads();
+    for (int i = tid; i < n; i += blockDim.x) atomicAdd(&sm.kept[sm.idx[i]], 1);
+    __syncthreads();
+    if (tid == 0) {
+        for (int e = 0; e < E; ++e)
+            if (cap >= 0) sm.kept[e] = min(sm.kept[e], cap);
+        write_offsets_and_lists(sm.kept, E, sm.off, offsets, meta, active, tiles);
+    }
+    __syncthreads();
+    scatter_entries(sm.idx, 0, n, E, cap, sm.pre, sm.off, sm.running, sm.u.wcnt, row2ts, ts2row);
 }
 
 // ---------------------------------------------------------------------------
@@ -273,10 +357,12 @@ __global__ void __launch_bounds__(kPermThreads) perm_scatter_kernel(
 // groups of 8 channels.  Writes xq[t] and, when aq is given, the copy of the
 // token's codes into every kept (t, slot) row of the expert-sorted matrix.
 // ---------------------------------------------------------------------------
-constexpr int kSqThreads = 256;
-constexpr int kSqMaxGroups = 8;   // d <= 256 * 8 * 8 = 16384
+constexpr int kSqMaxThreads = 1024;
+constexpr int kSqMaxGroups = 2;   // d <= 1024 threads x 2 groups x 8 = 16384
 
-__global__ void __launch_bounds__(kSqThreads) smooth_quant_kernel(
+// blockDim.x = min(1024, d / 8) threads; thread g owns channel groups g and
+// g + blockDim.x (8 channels each).
+__global__ void __launch_bounds__(kSqMaxThreads) smooth_quant_kernel(
     const void* __restrict__ x, int in_dtype, const float* __restrict__ inv_s, int d, int k,
     const int32_t* __restrict__ ts2row, int8_t* __restrict__ xq, float* __restrict__ sx,
     int8_t* __restrict__ aq) {
@@ -287,7 +373,7 @@ __global__ void __launch_bounds__(kSqThreads) smooth_quant_kernel(
     float m = 0.0f;
 #pragma unroll
     for (int gi = 0; gi < kSqMaxGroups; ++gi) {
-        const int g = threadIdx.x + gi * kSqThreads;
+        const int g = threadIdx.x + gi * blockDim.x;
         if (g < ng) {
             load8_act(x, (int64_t)t * d + g * 8, in_dtype, v[gi]);
             const float4 s0 = *reinterpret_cast<const float4*>(inv_s + g * 8);
@@ -308,7 +394,7 @@ __global__ void __launch_bounds__(kSqThreads) smooth_quant_kernel(
         for (int sl = 0; sl < k; ++sl) rows[sl] = ts2row[(int64_t)t * k + sl];
 #pragma unroll
     for (int gi = 0; gi < kSqMaxGroups; ++gi) {
-        const int g = threadIdx.x + gi * kSqThreads;
+        const int g = threadIdx.x + gi * blockDim.x;
         if (g < ng) {
             int q[8];
 #pragma unroll
@@ -351,10 +437,30 @@ cudaError_t launch_permute(const int32_t* idx, int T, int k, int E, int cap, int
     return cudaGetLastError();
 }
 
+bool route_small_ok(int T, int k) { return (int64_t)T * k <= kRouteSmallMax; }
+
+cudaError_t launch_route_small(const float* logits, const float* bias, int T, int E, int k,
+                               int renorm, int cap, int32_t* idx, float* wts, float* logits_out,
+                               int32_t* offsets, int32_t* row2ts, int32_t* ts2row, int32_t* meta,
+                               int32_t* active, int32_t* tiles, cudaStream_t s) {
+    static bool attr = false;
+    if (!attr) {
+        cudaError_t e = cudaFuncSetAttribute(route_small_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)sizeof(RouteSmallSmem));
+        if (e != cudaSuccess) return e;
+        attr = true;
+    }
+    route_small_kernel<<<1, kRouteSmallThreads, sizeof(RouteSmallSmem), s>>>(
+        logits, bias, T, E, k, renorm, cap, idx, wts, logits_out, offsets, row2ts, ts2row, meta,
+        active, tiles);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_smooth_quant(const void* x, int in_dtype, const float* inv_s, int T, int d,
                                 int k, const int32_t* ts2row, int8_t* xq, float* sx, int8_t* aq,
                                 cudaStream_t s) {
-    smooth_quant_kernel<<<T, kSqThreads, 0, s>>>(x, in_dtype, inv_s, d, k, ts2row, xq, sx, aq);
+    const int threads = max(32, min(kSqMaxThreads, d / 8));
+    smooth_quant_kernel<<<T, threads, 0, s>>>(x, in_dtype, inv_s, d, k, ts2row, xq, sx, aq);
     return cudaGetLastError();
 }
 

@@ -274,15 +274,26 @@ static moe_status forward_impl(const moe_w8a8_weights* w, const void* x, int T, 
     } else {
         empty_stage(MOE_STAGE_ROUTER);
     }
-    mark(MOE_STAGE_TOPK, 0);
-    CUDA_TRY(launch_topk(lsrc, bias, T, E, k, c.renormalize, idx, wts, dbg ? dbg->logits : nullptr, s));
-    mark(MOE_STAGE_TOPK, 1);
-    ++launches;
-    mark(MOE_STAGE_PERMUTE, 0);
-    CUDA_TRY(launch_permute(idx, T, k, E, capacity_of(c, T), (int32_t*)P(L.hist), offsets, row2ts,
-                            ts2row, meta, active, tiles, s));
-    mark(MOE_STAGE_PERMUTE, 1);
-    launches += 2;
+    if (route_small_ok(T, k)) {
+        // top-k, histogram, scan and scatter in one block
+        mark(MOE_STAGE_TOPK, 0);
+        CUDA_TRY(launch_route_small(lsrc, bias, T, E, k, c.renormalize, capacity_of(c, T), idx, wts,
+                                    dbg ? dbg->logits : nullptr, offsets, row2ts, ts2row, meta,
+                                    active, tiles, s));
+        mark(MOE_STAGE_TOPK, 1);
+        empty_stage(MOE_STAGE_PERMUTE);
+        ++launches;
+    } else {
+        mark(MOE_STAGE_TOPK, 0);
+        CUDA_TRY(launch_topk(lsrc, bias, T, E, k, c.renormalize, idx, wts, dbg ? dbg->logits : nullptr, s));
+        mark(MOE_STAGE_TOPK, 1);
+        ++launches;
+        mark(MOE_STAGE_PERMUTE, 0);
+        CUDA_TRY(launch_permute(idx, T, k, E, capacity_of(c, T), (int32_t*)P(L.hist), offsets, row2ts,
+                                ts2row, meta, active, tiles, s));
+        mark(MOE_STAGE_PERMUTE, 1);
+        launches += 2;
+    }
     if (path == MOE_PATH_STREAM) {
         mark(MOE_STAGE_QUANT, 0);
         CUDA_TRY(launch_smooth_quant(x, c.in_dtype, w->inv_s, T, d, k, ts2row, xq, sx, nullptr, s));
