@@ -473,40 +473,43 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // ------------------------------------------------------------------ requantisation of h
 
-// One block per sorted row: sh = max over the row's partial maxima / 127 and
-// codes rint(h / sh), ties to even, clamped to +-127 (sh = 0 gives 0).
-constexpr int kRqThreads = 128;
+// One warp per sorted row: sh = max over the row's partial maxima / 127 and
+// codes rint(h / sh), ties to even, clamped to +-127 (sh = 0 gives 0).  Each
+// lane issues all its loads of a batch (up to 16 x 16 bytes) before using them.
+constexpr int kRqThreads = 256;
+constexpr int kRqBatch = 16;
 
 __global__ void __launch_bounds__(kRqThreads) requant_kernel(const float* __restrict__ h32,
                                                              const float* __restrict__ pamax, int f,
                                                              const int32_t* __restrict__ meta,
                                                              int8_t* __restrict__ hq,
                                                              float* __restrict__ sh) {
-    __shared__ float red[32];
-    const int row = blockIdx.x;
+    const int lane = threadIdx.x & 31;
+    const int row = blockIdx.x * (kRqThreads / 32) + (threadIdx.x >> 5);
     if (row >= meta[META_R]) return;
-    const int npart = f / 64;
-    const float4* hrow = reinterpret_cast<const float4*>(h32 + (int64_t)row * f);
-    constexpr int kMaxPer = 16384 / 4 / kRqThreads;
-    float4 h[kMaxPer];
-#pragma unroll
-    for (int i = 0; i < kMaxPer; ++i) {
-        const int c4 = threadIdx.x + i * kRqThreads;
-        if (c4 < f / 4) h[i] = hrow[c4];
-    }
+    const int npart = f / 64, n4 = f / 4;
     float m = 0.0f;
-    for (int i = threadIdx.x; i < npart; i += kRqThreads) m = fmaxf(m, pamax[(int64_t)row * npart + i]);
-    m = block_max_nonneg(m, red);
+    for (int i = lane; i < npart; i += 32) m = fmaxf(m, pamax[(int64_t)row * npart + i]);
+    m = warp_max(m);
     const float s = m > 0.0f ? __fdiv_rn(m, 127.0f) : 0.0f;
-    if (threadIdx.x == 0) sh[row] = s;
+    if (lane == 0) sh[row] = s;
+    const float4* hrow = reinterpret_cast<const float4*>(h32 + (int64_t)row * f);
     uint32_t* qrow = reinterpret_cast<uint32_t*>(hq + (int64_t)row * f);
+    for (int b = 0; b < n4; b += 32 * kRqBatch) {
+        float4 h[kRqBatch];
 #pragma unroll
-    for (int i = 0; i < kMaxPer; ++i) {
-        const int c4 = threadIdx.x + i * kRqThreads;
-        if (c4 < f / 4)
-            qrow[c4] = s > 0.0f ? pack4(quant_code(h[i].x, s), quant_code(h[i].y, s), quant_code(h[i].z, s),
-                                        quant_code(h[i].w, s))
-                                : 0u;
+        for (int i = 0; i < kRqBatch; ++i) {
+            const int c4 = b + lane + 32 * i;
+            if (c4 < n4) h[i] = hrow[c4];
+        }
+#pragma unroll
+        for (int i = 0; i < kRqBatch; ++i) {
+            const int c4 = b + lane + 32 * i;
+            if (c4 < n4)
+                qrow[c4] = s > 0.0f ? pack4(quant_code(h[i].x, s), quant_code(h[i].y, s),
+                                            quant_code(h[i].z, s), quant_code(h[i].w, s))
+                                    : 0u;
+        }
     }
 }
 
@@ -569,7 +572,9 @@ bool tc_supported(const moe_w8a8_config& c) { return c.d % BN == 0 && c.f % BK =
 
 cudaError_t launch_requant(const float* h32, const float* pamax, int f, const int32_t* meta,
                            int max_rows, int8_t* hq, float* sh, cudaStream_t s) {
-    requant_kernel<<<max_rows, kRqThreads, 0, s>>>(h32, pamax, f, meta, hq, sh);
+    const int rows_per_block = kRqThreads / 32;
+    requant_kernel<<<(max_rows + rows_per_block - 1) / rows_per_block, kRqThreads, 0, s>>>(
+        h32, pamax, f, meta, hq, sh);
     return cudaGetLastError();
 }
 
