@@ -17,13 +17,18 @@ namespace {
 // for a register tile of 8 tokens x 8 experts (16 warps = 4 token groups x 4
 // expert groups); X and W_router are staged in shared memory 128 channels at a
 // time, laid out [i][p][t] and [i][p][e] with padded rows so that each lane's 8
-// tokens (experts) are one conflict-free pair of 16-byte loads.
+// tokens (experts) are one conflict-free pair of 16-byte loads.  The token
+// index of X is XOR-swizzled on bits 2-4 by (p / 8, i mod 2) so that the
+// staging stores (8 consecutive channels of one token per thread) do not pile
+// onto one bank; 4-token groups stay contiguous.
 // ---------------------------------------------------------------------------
 constexpr int kRtT = 32;         // tokens per block
 constexpr int kRtE = 32;         // experts per block
 constexpr int kRtKC = 128;       // channels per staged chunk (4 steps of i)
 constexpr int kRtPad = 36;       // padded row (floats): 16-byte aligned, rows 4 banks apart
 constexpr int kRtThreads = 512;
+
+__device__ __forceinline__ int rt_swz(int p, int i) { return ((((p >> 3) & 3) | ((i & 1) << 2)) << 2); }
 
 __global__ void __launch_bounds__(kRtThreads) router_logits_kernel(
     const void* __restrict__ x, int in_dtype, const float* __restrict__ wr, int T, int d, int E,
@@ -51,7 +56,10 @@ __global__ void __launch_bounds__(kRtThreads) router_logits_kernel(
                 for (int q = 0; q < 8; ++q) v[q] = 0.0f;
             }
 #pragma unroll
-            for (int q = 0; q < 8; ++q) xs[(j0 + q) >> 5][(j0 + q) & 31][tt] = v[q];
+            for (int q = 0; q < 8; ++q) {
+                const int i = (j0 + q) >> 5, pp = (j0 + q) & 31;
+                xs[i][pp][tt ^ rt_swz(pp, i)] = v[q];
+            }
         }
         // W chunk: 128 rows x 32 experts, 16 bytes per thread (two per thread)
         for (int idx = tid; idx < kRtKC * (kRtE / 4); idx += kRtThreads) {
@@ -68,8 +76,9 @@ __global__ void __launch_bounds__(kRtThreads) router_logits_kernel(
         __syncthreads();
 #pragma unroll
         for (int i = 0; i < kRtKC / 32; ++i) {
-            const float4 xa = *reinterpret_cast<const float4*>(&xs[i][lane][tg * 8]);
-            const float4 xb = *reinterpret_cast<const float4*>(&xs[i][lane][tg * 8 + 4]);
+            const int sw = rt_swz(lane, i);
+            const float4 xa = *reinterpret_cast<const float4*>(&xs[i][lane][(tg * 8) ^ sw]);
+            const float4 xb = *reinterpret_cast<const float4*>(&xs[i][lane][(tg * 8 + 4) ^ sw]);
             const float4 wa = *reinterpret_cast<const float4*>(&ws[i][lane][eg * 8]);
             const float4 wb = *reinterpret_cast<const float4*>(&ws[i][lane][eg * 8 + 4]);
             const float xv[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
@@ -197,26 +206,46 @@ __global__ void topk_kernel(const float* __restrict__ logits, const float* __res
 // ---------------------------------------------------------------------------
 
 // Expert offsets (exclusive scan of kept counts) and the lists the expert
-// kernels read: active experts and 128-row tiles.  Written by one thread.
+// kernels read: active experts and 128-row tiles.  Run by one full warp: lane
+// l owns experts [l*per, l*per + per), three exclusive warp scans place its
+// offsets, active entries and tiles.
 __device__ void write_offsets_and_lists(const int* kept, int E, int* off, int32_t* offsets,
-                                        int32_t* meta, int32_t* active, int32_t* tiles) {
-    int acc = 0;
-    for (int e = 0; e < E; ++e) { off[e] = acc; acc += kept[e]; }
-    off[E] = acc;
-    int na = 0, nt = 0;
-    for (int e = 0; e <= E; ++e) offsets[e] = off[e];
-    for (int e = 0; e < E; ++e) {
-        if (kept[e] == 0) continue;
-        active[na++] = e;
+                                        int32_t* meta, int32_t* active, int32_t* tiles, int lane) {
+    const int per = (E + 31) / 32;
+    const int e0 = min(E, lane * per), e1 = min(E, e0 + per);
+    int rows = 0, nact = 0, ntl = 0;
+    for (int e = e0; e < e1; ++e) {
+        rows += kept[e];
+        nact += kept[e] > 0;
+        ntl += (kept[e] + kTileM - 1) / kTileM;
+    }
+    int xr = rows, xa = nact, xt = ntl;   // inclusive scans
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int a = __shfl_up_sync(0xffffffffu, xr, o);
+        const int b = __shfl_up_sync(0xffffffffu, xa, o);
+        const int c = __shfl_up_sync(0xffffffffu, xt, o);
+        if (lane >= o) { xr += a; xa += b; xt += c; }
+    }
+    int r = xr - rows, na = xa - nact, nt = xt - ntl;
+    for (int e = e0; e < e1; ++e) {
+        off[e] = r;
+        offsets[e] = r;
+        if (kept[e] > 0) active[na++] = e;
         for (int m = 0; m * kTileM < kept[e]; ++m) {
             tiles[2 * nt] = e;
-            tiles[2 * nt + 1] = off[e] + m * kTileM;
+            tiles[2 * nt + 1] = r + m * kTileM;
             ++nt;
         }
+        r += kept[e];
     }
-    meta[META_R] = off[E];
-    meta[META_NACTIVE] = na;
-    meta[META_NTILES] = nt;
+    if (lane == 31) {
+        off[E] = xr;
+        offsets[E] = xr;
+        meta[META_R] = xr;
+        meta[META_NACTIVE] = xa;
+        meta[META_NTILES] = xt;
+    }
 }
 
 // Stable ranks of entries [base, base + len) in rounds of blockDim.x: warp
@@ -293,10 +322,10 @@ __global__ void __launch_bounds__(kPermThreads) perm_scatter_kernel(
         running[e] = 0;
     }
     __syncthreads();
-    if (tid == 0) {
+    if (tid < 32) {
         if (blockIdx.x == 0) {
-            write_offsets_and_lists(kept, E, off, offsets, meta, active, tiles);
-        } else {
+            write_offsets_and_lists(kept, E, off, offsets, meta, active, tiles, tid);
+        } else if (tid == 0) {
             int acc = 0;
             for (int e = 0; e < E; ++e) { off[e] = acc; acc += kept[e]; }
             off[E] = acc;
@@ -342,11 +371,10 @@ __global__ void __launch_bounds__(kRouteSmallThreads) route_small_kernel(
     __syncthreads();
     for (int i = tid; i < n; i += blockDim.x) atomicAdd(&sm.kept[sm.idx[i]], 1);
     __syncthreads();
-    if (tid == 0) {
-        for (int e = 0; e < E; ++e)
-            if (cap >= 0) sm.kept[e] = min(sm.kept[e], cap);
-        write_offsets_and_lists(sm.kept, E, sm.off, offsets, meta, active, tiles);
-    }
+    if (cap >= 0)
+        for (int e = tid; e < E; e += blockDim.x) sm.kept[e] = min(sm.kept[e], cap);
+    __syncthreads();
+    if (tid < 32) write_offsets_and_lists(sm.kept, E, sm.off, offsets, meta, active, tiles, tid);
     __syncthreads();
     scatter_entries(sm.idx, 0, n, E, cap, sm.pre, sm.off, sm.running, sm.u.wcnt, row2ts, ts2row);
 }
