@@ -108,6 +108,110 @@ __global__ void __launch_bounds__(kRtThreads) router_logits_kernel(
     }
 }
 
+// Router logits, same order, with the X and W tiles streamed into shared
+// memory by cp.async through a 3-stage ring so that global loads overlap the
+// FMAs.  X is kept as it arrives ([t][channel], bf16 or fp32); lane p reads its
+// 8 tokens' values x[t][32i+p] one element at a time (a warp reads 32
+// consecutive channels: conflict-free).  W rows are padded to 36 floats so the
+// two 16-byte loads of a lane's 8 experts do not conflict.  Needs E % 4 == 0.
+constexpr int kRaStages = 3;
+constexpr int kRaWPad = 36;
+
+template <int XB>   // bytes per X element: 2 (bf16) or 4 (fp32)
+struct RouterAsyncSmem {
+    uint8_t x[kRaStages][kRtT][kRtKC * XB];
+    float w[kRaStages][kRtKC][kRaWPad];
+};
+
+__device__ __forceinline__ void cp_async16(void* dst, const void* src, int src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(
+                     (uint32_t)__cvta_generic_to_shared(dst)),
+                 "l"(src), "r"(src_bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+template <int XB>
+__global__ void __launch_bounds__(kRtThreads) router_logits_async_kernel(
+    const void* __restrict__ x, const float* __restrict__ wr, int T, int d, int E,
+    float* __restrict__ logits) {
+    extern __shared__ __align__(16) uint8_t smem_raw[];
+    RouterAsyncSmem<XB>& sm = *reinterpret_cast<RouterAsyncSmem<XB>*>(smem_raw);
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int tg = warp >> 2, eg = warp & 3;
+    const int t0 = blockIdx.x * kRtT, e0 = blockIdx.y * kRtE;
+    const int nchunks = d / kRtKC;
+    constexpr int kXChunks = kRtT * kRtKC * XB / 16;   // 16-byte pieces of an X tile
+    constexpr int kWChunks = kRtKC * kRtE / 4;         // 16-byte pieces of a W tile
+
+    auto issue = [&](int c, int stage) {
+        for (int q = tid; q < kXChunks; q += kRtThreads) {
+            const int tt = q / (kRtKC * XB / 16), part = q % (kRtKC * XB / 16);
+            const int t = t0 + tt;
+            const uint8_t* src = reinterpret_cast<const uint8_t*>(x) +
+                                 ((int64_t)min(t, T - 1) * d + (int64_t)c * kRtKC) * XB + part * 16;
+            cp_async16(&sm.x[stage][tt][part * 16], src, t < T ? 16 : 0);
+        }
+        for (int q = tid; q < kWChunks; q += kRtThreads) {
+            const int row = q / (kRtE / 4), c4 = q % (kRtE / 4);
+            const int e = e0 + 4 * c4;
+            const float* src = wr + (int64_t)(c * kRtKC + row) * E + min(e, E - 4);
+            cp_async16(&sm.w[stage][row][4 * c4], src, e < E ? 16 : 0);
+        }
+        cp_async_commit();
+    };
+
+    float acc[8][8];
+#pragma unroll
+    for (int a = 0; a < 8; ++a)
+#pragma unroll
+        for (int b = 0; b < 8; ++b) acc[a][b] = 0.0f;
+
+    issue(0, 0);
+    if (nchunks > 1) issue(1, 1); else cp_async_commit();
+    for (int c = 0; c < nchunks; ++c) {
+        cp_async_wait<1>();
+        __syncthreads();
+        if (c + 2 < nchunks) issue(c + 2, (c + 2) % kRaStages); else cp_async_commit();
+        const int st = c % kRaStages;
+#pragma unroll
+        for (int i = 0; i < kRtKC / 32; ++i) {
+            float xv[8];
+#pragma unroll
+            for (int a = 0; a < 8; ++a) {
+                const uint8_t* px = &sm.x[st][tg * 8 + a][(32 * i + lane) * XB];
+                xv[a] = XB == 2 ? bf16_bits_to_f32(*reinterpret_cast<const uint16_t*>(px))
+                                : *reinterpret_cast<const float*>(px);
+            }
+            const float4 wa = *reinterpret_cast<const float4*>(&sm.w[st][32 * i + lane][eg * 8]);
+            const float4 wb = *reinterpret_cast<const float4*>(&sm.w[st][32 * i + lane][eg * 8 + 4]);
+            const float wv[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
+#pragma unroll
+            for (int a = 0; a < 8; ++a)
+#pragma unroll
+                for (int b = 0; b < 8; ++b) acc[a][b] = __fmaf_rn(xv[a], wv[b], acc[a][b]);
+        }
+    }
+    cp_async_wait<0>();
+#pragma unroll
+    for (int a = 0; a < 8; ++a)
+#pragma unroll
+        for (int b = 0; b < 8; ++b) {
+            float v = acc[a][b];
+#pragma unroll
+            for (int o = 16; o >= 1; o >>= 1) v = __fadd_rn(v, __shfl_xor_sync(0xffffffffu, v, o));
+            acc[a][b] = v;
+        }
+#pragma unroll
+    for (int v = 0; v < 64; ++v) {
+        if ((v & 31) != lane) continue;
+        const int t = t0 + tg * 8 + (v >> 3), e = e0 + eg * 8 + (v & 7);
+        if (t < T && e < E) logits[(int64_t)t * E + e] = acc[v >> 3][v & 7];
+    }
+}
+
 // ---------------------------------------------------------------------------
 // Top-k + gate weights, one warp per token.  l_e = logit + bias_e; k rounds of
 // a warp argmax on (l descending, e ascending); w = softmax of the selected
@@ -442,7 +546,22 @@ __global__ void __launch_bounds__(kSqMaxThreads) smooth_quant_kernel(
 cudaError_t launch_router_logits(const void* x, int in_dtype, const float* wr, int T, int d, int E,
                                  float* logits, cudaStream_t s) {
     dim3 grid((T + kRtT - 1) / kRtT, (E + kRtE - 1) / kRtE);
-    router_logits_kernel<<<grid, kRtThreads, 0, s>>>(x, in_dtype, wr, T, d, E, logits);
+    if (E % 4 == 0 && E >= 4) {
+        static bool attr = false;
+        if (!attr) {
+            cudaFuncSetAttribute(router_logits_async_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)sizeof(RouterAsyncSmem<2>));
+            cudaFuncSetAttribute(router_logits_async_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)sizeof(RouterAsyncSmem<4>));
+            attr = true;
+        }
+        if (in_dtype == MOE_BF16)
+            router_logits_async_kernel<2><<<grid, kRtThreads, sizeof(RouterAsyncSmem<2>), s>>>(x, wr, T, d, E, logits);
+        else
+            router_logits_async_kernel<4><<<grid, kRtThreads, sizeof(RouterAsyncSmem<4>), s>>>(x, wr, T, d, E, logits);
+    } else {
+        router_logits_kernel<<<grid, kRtThreads, 0, s>>>(x, in_dtype, wr, T, d, E, logits);
+    }
     return cudaGetLastError();
 }
 
