@@ -65,6 +65,20 @@ __device__ __forceinline__ int quant_code(float v, float s) {
     return max(-127, min(127, q));
 }
 
+// The same code without a division in the common case.  With r = fp32(1/s)
+// and t = fp32(v r), |t - fp32(v / s)| <= 3.0001 u |v / s| (u = 2^-24) by the
+// standard rounding-error bound, i.e. below 2.3e-5 for |v / s| <= 128.  So
+// unless t lies within 3e-5 of a half-integer, t and the IEEE quotient round
+// to the same integer; near a half-integer the IEEE quotient is formed.  The
+// result is identical to quant_code(v, s).  `r` must be fp32(1 / s), s > 0.
+__device__ __forceinline__ int quant_code_fast(float v, float s, float r) {
+    const float t = __fmul_rn(v, r);
+    const float n = rintf(t);
+    const float dist = fabsf(fabsf(__fsub_rn(t, n)) - 0.5f);
+    int q = (dist > 3.0e-5f || fabsf(t) > 130.0f) ? __float2int_rn(n) : __float2int_rn(__fdiv_rn(v, s));
+    return max(-127, min(127, q));
+}
+
 // Pack four INT8 codes (low byte first).
 __device__ __forceinline__ uint32_t pack4(int a, int b, int c, int d) {
     return (uint32_t)(a & 0xff) | ((uint32_t)(b & 0xff) << 8) | ((uint32_t)(c & 0xff) << 16) |

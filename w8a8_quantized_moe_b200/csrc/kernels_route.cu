@@ -520,6 +520,7 @@ __global__ void __launch_bounds__(kSqMaxThreads) smooth_quant_kernel(
     }
     const float amax = block_max_nonneg(m, red);
     const float s = amax > 0.0f ? __fdiv_rn(amax, 127.0f) : 0.0f;
+    const float rs = s > 0.0f ? __frcp_rn(s) : 0.0f;
     if (threadIdx.x == 0) sx[t] = s;
     int rows[kMaxK];
     if (aq)
@@ -530,7 +531,7 @@ __global__ void __launch_bounds__(kSqMaxThreads) smooth_quant_kernel(
         if (g < ng) {
             int q[8];
 #pragma unroll
-            for (int c = 0; c < 8; ++c) q[c] = s > 0.0f ? quant_code(v[gi][c], s) : 0;
+            for (int c = 0; c < 8; ++c) q[c] = s > 0.0f ? quant_code_fast(v[gi][c], s, rs) : 0;
             const uint2 packed = make_uint2(pack4(q[0], q[1], q[2], q[3]), pack4(q[4], q[5], q[6], q[7]));
             *reinterpret_cast<uint2*>(xq + (int64_t)t * d + g * 8) = packed;
             if (aq)

@@ -492,6 +492,7 @@ __global__ void __launch_bounds__(kRqThreads) requant_kernel(const float* __rest
     for (int i = lane; i < npart; i += 32) m = fmaxf(m, pamax[(int64_t)row * npart + i]);
     m = warp_max(m);
     const float s = m > 0.0f ? __fdiv_rn(m, 127.0f) : 0.0f;
+    const float rs = s > 0.0f ? __frcp_rn(s) : 0.0f;
     if (lane == 0) sh[row] = s;
     const float4* hrow = reinterpret_cast<const float4*>(h32 + (int64_t)row * f);
     uint32_t* qrow = reinterpret_cast<uint32_t*>(hq + (int64_t)row * f);
@@ -506,8 +507,8 @@ __global__ void __launch_bounds__(kRqThreads) requant_kernel(const float* __rest
         for (int i = 0; i < kRqBatch; ++i) {
             const int c4 = b + lane + 32 * i;
             if (c4 < n4)
-                qrow[c4] = s > 0.0f ? pack4(quant_code(h[i].x, s), quant_code(h[i].y, s),
-                                            quant_code(h[i].z, s), quant_code(h[i].w, s))
+                qrow[c4] = s > 0.0f ? pack4(quant_code_fast(h[i].x, s, rs), quant_code_fast(h[i].y, s, rs),
+                                            quant_code_fast(h[i].z, s, rs), quant_code_fast(h[i].w, s, rs))
                                     : 0u;
         }
     }
