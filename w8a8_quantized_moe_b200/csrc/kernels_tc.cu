@@ -474,10 +474,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 // ------------------------------------------------------------------ requantisation of h
 
 // One warp per sorted row: sh = max over the row's partial maxima / 127 and
-// codes rint(h / sh), ties to even, clamped to +-127 (sh = 0 gives 0).  Each
-// lane issues all its loads of a batch (up to 16 x 16 bytes) before using them.
+// codes rint(h / sh), ties to even, clamped to +-127 (sh = 0 gives 0).  The h
+// loads of a batch (up to 8 x 16 bytes per lane) are issued together with the
+// partial-maximum loads, before the reduction.
 constexpr int kRqThreads = 256;
-constexpr int kRqBatch = 16;
+constexpr int kRqBatch = 8;
 
 __global__ void __launch_bounds__(kRqThreads) requant_kernel(const float* __restrict__ h32,
                                                              const float* __restrict__ pamax, int f,
@@ -488,20 +489,27 @@ __global__ void __launch_bounds__(kRqThreads) requant_kernel(const float* __rest
     const int row = blockIdx.x * (kRqThreads / 32) + (threadIdx.x >> 5);
     if (row >= meta[META_R]) return;
     const int npart = f / 64, n4 = f / 4;
+    const float4* hrow = reinterpret_cast<const float4*>(h32 + (int64_t)row * f);
+    uint32_t* qrow = reinterpret_cast<uint32_t*>(hq + (int64_t)row * f);
+    float4 h[kRqBatch];
+#pragma unroll
+    for (int i = 0; i < kRqBatch; ++i) {
+        const int c4 = lane + 32 * i;
+        if (c4 < n4) h[i] = hrow[c4];
+    }
     float m = 0.0f;
     for (int i = lane; i < npart; i += 32) m = fmaxf(m, pamax[(int64_t)row * npart + i]);
     m = warp_max(m);
     const float s = m > 0.0f ? __fdiv_rn(m, 127.0f) : 0.0f;
     const float rs = s > 0.0f ? __frcp_rn(s) : 0.0f;
     if (lane == 0) sh[row] = s;
-    const float4* hrow = reinterpret_cast<const float4*>(h32 + (int64_t)row * f);
-    uint32_t* qrow = reinterpret_cast<uint32_t*>(hq + (int64_t)row * f);
     for (int b = 0; b < n4; b += 32 * kRqBatch) {
-        float4 h[kRqBatch];
+        if (b > 0) {
 #pragma unroll
-        for (int i = 0; i < kRqBatch; ++i) {
-            const int c4 = b + lane + 32 * i;
-            if (c4 < n4) h[i] = hrow[c4];
+            for (int i = 0; i < kRqBatch; ++i) {
+                const int c4 = b + lane + 32 * i;
+                if (c4 < n4) h[i] = hrow[c4];
+            }
         }
 #pragma unroll
         for (int i = 0; i < kRqBatch; ++i) {
