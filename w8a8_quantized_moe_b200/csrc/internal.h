@@ -49,7 +49,7 @@ struct WsLayout {
     size_t logits, topk_idx, topk_w;
     size_t hist, offsets, meta, active, tiles;
     size_t row2ts, ts2row;
-    size_t xq, sx;
+    size_t xq, sx, aq;
     size_t acc1, hq, sh, o;
     size_t h32, pamax;           // tensor path: fp32 h, per-row partial maxima
     size_t total;
@@ -104,7 +104,7 @@ cudaError_t launch_stream_down(const moe_w8a8_weights* w, int T, const int8_t* h
 // tensor-core path (kernels_tc.cu)
 bool tc_make_weight_maps(moe_w8a8_weights* w);
 bool tc_supported(const moe_w8a8_config& c);
-cudaError_t launch_tc_gemm1(const moe_w8a8_weights* w, int T, const int8_t* xq, const int32_t* meta,
+cudaError_t launch_tc_gemm1(const moe_w8a8_weights* w, int T, const int8_t* aq, const int32_t* meta,
                             const int32_t* tiles, const int32_t* offsets, const int32_t* row2ts,
                             const float* sx, float* h32, float* pamax, int32_t* acc_dbg,
                             cudaStream_t s);

@@ -158,19 +158,6 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, u
         : "memory");
 }
 
-// Four rows (y0..y3) of a 2-D tensor map whose box is one row high, written as
-// four consecutive 128-byte rows at dst (the map's swizzle applies as for a
-// 4-row box at that address).
-__device__ __forceinline__ void tma_gather4(void* dst, const CUtensorMap* map, uint64_t* bar, int x,
-                                            int y0, int y1, int y2, int y3) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(smem_u32(dst)),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y0), "r"(y1), "r"(y2),
-        "r"(y3)
-        : "memory");
-}
-
 // Shared-memory matrix descriptor, K-major, 128-byte swizzle: 8-row atoms of
 // 1024 bytes (stride byte offset 1024); leading byte offset unused for this
 // layout; descriptor version 1 (bit 46); layout type 2 = SWIZZLE_128B.
@@ -388,57 +375,36 @@ __global__ void __launch_bounds__(kThreads, 1)
     volatile int* abort = &ctl->abort;
 
     if (warp == 0) {
-        // ---------------- TMA producer (whole warp).  GEMM1 gathers its A rows
-        // straight from the per-token INT8 activations: lane l fetches sorted rows
-        // 4l..4l+3 of the tile (token row2ts[row] / k) with one gather4 per k-block.
-        // GEMM2 reads A (h codes, already in sorted order) as a tiled box.
-        int s = 0;
-        uint32_t ph = 0;
-        uint32_t issued_par[kStages];
-        bool issued[kStages];
-        for (int i = 0; i < kStages; ++i) issued[i] = false;
-        bool ok = true;
-        for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
-            const int mt = t / p.n_tiles_n, nt = t % p.n_tiles_n;
-            const int e = p.tiles[2 * mt], row0 = p.tiles[2 * mt + 1];
-            const int brow = e * p.N + nt * BN;
-            int arow[4] = {0, 0, 0, 0};
-            if (EPI == EPI_SWIGLU) {
-                const int nrows = min(BM, p.offsets[e + 1] - row0);
-                const int fallback = p.row2ts[row0] / p.k;
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const int r = 4 * lane + q;
-                    arow[q] = r < nrows ? p.row2ts[row0 + r] / p.k : fallback;
-                }
-            }
-            for (int kb = 0; kb < nkb; ++kb) {
-                int go = 1;
-                if (lane == 0) go = mbar_wait(&ctl->empty[s], ph ^ 1, abort, p.status, 1, t) ? 1 : 0;
-                go = __shfl_sync(0xffffffffu, go, 0);
-                if (!go) { ok = false; break; }
-                uint8_t* sa = smem + s * kStageBytes;
-                if (lane == 0) {
+        if (lane == 0) {
+            // ---------------- TMA producer
+            int s = 0;
+            uint32_t ph = 0;
+            uint32_t issued_par[kStages];
+            bool issued[kStages];
+            for (int i = 0; i < kStages; ++i) issued[i] = false;
+            bool ok = true;
+            for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+                const int mt = t / p.n_tiles_n, nt = t % p.n_tiles_n;
+                const int e = p.tiles[2 * mt], row0 = p.tiles[2 * mt + 1];
+                const int brow = e * p.N + nt * BN;
+                for (int kb = 0; kb < nkb; ++kb) {
+                    if (!mbar_wait(&ctl->empty[s], ph ^ 1, abort, p.status, 1, t)) { ok = false; break; }
                     mbar_arrive_expect_tx(&ctl->full[s], kStageBytes);
+                    uint8_t* sa = smem + s * kStageBytes;
+                    tma_load_2d(sa, &tm_a, &ctl->full[s], kb * BK, row0);
                     tma_load_2d(sa + kABytes, &tm_b, &ctl->full[s], kb * BK, brow);
-                    if (EPI != EPI_SWIGLU) tma_load_2d(sa, &tm_a, &ctl->full[s], kb * BK, row0);
                     issued[s] = true;
                     issued_par[s] = ph;
+                    if (++s == kStages) { s = 0; ph ^= 1; }
                 }
-                __syncwarp();
-                if (EPI == EPI_SWIGLU)
-                    tma_gather4(sa + lane * 4 * BK, &tm_a, &ctl->full[s], kb * BK, arow[0], arow[1],
-                                arow[2], arow[3]);
-                if (++s == kStages) { s = 0; ph ^= 1; }
             }
-        }
-        // copies in flight land before the CTA ends (bounded)
-        if (lane == 0)
+            // copies in flight land before the CTA ends (bounded)
             for (int i = 0; i < kStages; ++i) {
                 if (!issued[i]) continue;
                 const uint64_t t0 = global_timer();
                 while (!mbar_try_wait(&ctl->full[i], issued_par[i]) && global_timer() - t0 < kWaitBudgetNs) {}
             }
+        }
     } else if (warp == 1) {
         if (lane == 0) {
             // ---------------- MMA issuer
@@ -621,14 +587,14 @@ cudaError_t launch_requant(const float* h32, const float* pamax, int f, const in
     return cudaGetLastError();
 }
 
-cudaError_t launch_tc_gemm1(const moe_w8a8_weights* w, int T, const int8_t* xq, const int32_t* meta,
+cudaError_t launch_tc_gemm1(const moe_w8a8_weights* w, int T, const int8_t* aq, const int32_t* meta,
                             const int32_t* tiles, const int32_t* offsets, const int32_t* row2ts,
                             const float* sx, float* h32, float* pamax, int32_t* acc_dbg,
                             cudaStream_t s) {
     const moe_w8a8_config& c = w->cfg;
     CUtensorMap ta;
     const int rows = T * c.top_k;
-    if (!make_map(&ta, xq, c.d, T, 1)) return cudaErrorInvalidValue;   // gather4: one-row box
+    if (!make_map(&ta, aq, c.d, rows, BM)) return cudaErrorInvalidValue;
     TcParams p{};
     p.N = 2 * c.f;
     p.K = c.d;

@@ -106,6 +106,7 @@ WsLayout ws_layout(const moe_w8a8_weights* w, int T) {
     L.ts2row = take(tk * 4);
     L.xq = take((size_t)T * d);
     L.sx = take((size_t)T * 4);
+    L.aq = take(stream ? 0 : tk * d);
     L.acc1 = take(stream ? tk * 2 * f * 4 : 0);
     L.hq = take(tk * f);
     L.sh = take(tk * 4);
@@ -312,11 +313,12 @@ static moe_status forward_impl(const moe_w8a8_weights* w, const void* x, int T, 
         if (dbg && dbg->acc1)
             CUDA_TRY(cudaMemcpyAsync(dbg->acc1, acc1, tk * 2 * f * 4, cudaMemcpyDeviceToDevice, s));
     } else {
+        int8_t* aq = (int8_t*)P(L.aq);
         mark(MOE_STAGE_QUANT, 0);
-        CUDA_TRY(launch_smooth_quant(x, c.in_dtype, w->inv_s, T, d, k, ts2row, xq, sx, nullptr, s));
+        CUDA_TRY(launch_smooth_quant(x, c.in_dtype, w->inv_s, T, d, k, ts2row, xq, sx, aq, s));
         mark(MOE_STAGE_QUANT, 1);
         mark(MOE_STAGE_GEMM1, 0);
-        CUDA_TRY(launch_tc_gemm1(w, T, xq, meta, tiles, offsets, row2ts, sx, (float*)P(L.h32),
+        CUDA_TRY(launch_tc_gemm1(w, T, aq, meta, tiles, offsets, row2ts, sx, (float*)P(L.h32),
                                  (float*)P(L.pamax), dbg ? dbg->acc1 : nullptr, s));
         mark(MOE_STAGE_GEMM1, 1);
         mark(MOE_STAGE_REQUANT, 0);
