@@ -489,72 +489,64 @@ __global__ void __launch_bounds__(kRouteSmallThreads) route_small_kernel(
 // groups of 8 channels.  Writes xq[t] and, when aq is given, the copy of the
 // token's codes into every kept (t, slot) row of the expert-sorted matrix.
 // ---------------------------------------------------------------------------
-// One warp per token: lane l owns channel groups l, l + 32, ... (8 channels
-// each, d/256 groups per lane), all loads issued before the reduction; the
-// token's max is a warp shuffle reduction (no block barrier).
-constexpr int kSqThreads = 256;          // 8 tokens per block
-constexpr int kSqMaxGroups = 8;          // 8 groups (64 channels) per lane per pass
+// One block of 128 threads per token: thread i owns channel groups i, i + 128,
+// ... (8 channels each); all of a thread's loads are issued before the block
+// max (one shared-memory exchange), then the codes are written to xq[t] and,
+// for the tensor-core path, to every kept (t, slot) row of the sorted copy.
+constexpr int kSqThreads = 128;
 
+template <int kSqMaxGroups>   // groups of 8 channels per thread: d <= 128 x 8 x kSqMaxGroups
 __global__ void __launch_bounds__(kSqThreads) smooth_quant_kernel(
     const void* __restrict__ x, int in_dtype, const float* __restrict__ inv_s, int T, int d, int k,
     const int32_t* __restrict__ ts2row, int8_t* __restrict__ xq, float* __restrict__ sx,
     int8_t* __restrict__ aq) {
-    const int lane = threadIdx.x & 31;
-    const int t = blockIdx.x * (kSqThreads / 32) + (threadIdx.x >> 5);
-    if (t >= T) return;
+    __shared__ float red[kSqThreads / 32];
+    const int t = blockIdx.x, tid = threadIdx.x, lane = tid & 31;
     const int ng = d / 8;
-    int rows[kMaxK];
-    if (aq)
-        for (int sl = 0; sl < k; ++sl) rows[sl] = ts2row[(int64_t)t * k + sl];
-    // amax over the whole token first (d may exceed one pass of registers)
+    float v[kSqMaxGroups][8];
+#pragma unroll
+    for (int gi = 0; gi < kSqMaxGroups; ++gi) {
+        const int g = tid + kSqThreads * gi;
+        if (g < ng) load8_act(x, (int64_t)t * d + g * 8, in_dtype, v[gi]);
+    }
     float m = 0.0f;
-    for (int g0 = 0; g0 < ng; g0 += 32 * kSqMaxGroups) {
-        float v[kSqMaxGroups][8];
 #pragma unroll
-        for (int gi = 0; gi < kSqMaxGroups; ++gi) {
-            const int g = g0 + lane + 32 * gi;
-            if (g < ng) load8_act(x, (int64_t)t * d + g * 8, in_dtype, v[gi]);
-        }
+    for (int gi = 0; gi < kSqMaxGroups; ++gi) {
+        const int g = tid + kSqThreads * gi;
+        if (g < ng) {
+            const float4 s0 = *reinterpret_cast<const float4*>(inv_s + g * 8);
+            const float4 s1 = *reinterpret_cast<const float4*>(inv_s + g * 8 + 4);
+            const float sv[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
 #pragma unroll
-        for (int gi = 0; gi < kSqMaxGroups; ++gi) {
-            const int g = g0 + lane + 32 * gi;
-            if (g < ng) {
-                const float4 s0 = *reinterpret_cast<const float4*>(inv_s + g * 8);
-                const float4 s1 = *reinterpret_cast<const float4*>(inv_s + g * 8 + 4);
-                const float sv[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
-#pragma unroll
-                for (int c = 0; c < 8; ++c) m = fmaxf(m, fabsf(__fmul_rn(v[gi][c], sv[c])));
+            for (int c = 0; c < 8; ++c) {
+                v[gi][c] = __fmul_rn(v[gi][c], sv[c]);
+                m = fmaxf(m, fabsf(v[gi][c]));
             }
         }
     }
     m = warp_max(m);
+    if (lane == 0) red[tid >> 5] = m;
+    __syncthreads();
+#pragma unroll
+    for (int w = 0; w < kSqThreads / 32; ++w) m = fmaxf(m, red[w]);
     const float s = m > 0.0f ? __fdiv_rn(m, 127.0f) : 0.0f;
     const float rs = s > 0.0f ? __frcp_rn(s) : 0.0f;
-    if (lane == 0) sx[t] = s;
-    for (int g0 = 0; g0 < ng; g0 += 32 * kSqMaxGroups) {
-        float v[kSqMaxGroups][8];
+    if (tid == 0) sx[t] = s;
+    int rows[kMaxK];
 #pragma unroll
-        for (int gi = 0; gi < kSqMaxGroups; ++gi) {
-            const int g = g0 + lane + 32 * gi;
-            if (g < ng) load8_act(x, (int64_t)t * d + g * 8, in_dtype, v[gi]);
-        }
+    for (int sl = 0; sl < kMaxK; ++sl) rows[sl] = (aq && sl < k) ? ts2row[(int64_t)t * k + sl] : -1;
 #pragma unroll
-        for (int gi = 0; gi < kSqMaxGroups; ++gi) {
-            const int g = g0 + lane + 32 * gi;
-            if (g >= ng) continue;
-            const float4 s0 = *reinterpret_cast<const float4*>(inv_s + g * 8);
-            const float4 s1 = *reinterpret_cast<const float4*>(inv_s + g * 8 + 4);
-            const float sv[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
-            int q[8];
+    for (int gi = 0; gi < kSqMaxGroups; ++gi) {
+        const int g = tid + kSqThreads * gi;
+        if (g >= ng) continue;
+        int q[8];
 #pragma unroll
-            for (int c = 0; c < 8; ++c) q[c] = s > 0.0f ? quant_code_fast(__fmul_rn(v[gi][c], sv[c]), s, rs) : 0;
-            const uint2 packed = make_uint2(pack4(q[0], q[1], q[2], q[3]), pack4(q[4], q[5], q[6], q[7]));
-            *reinterpret_cast<uint2*>(xq + (int64_t)t * d + g * 8) = packed;
-            if (aq)
-                for (int sl = 0; sl < k; ++sl)
-                    if (rows[sl] >= 0)
-                        *reinterpret_cast<uint2*>(aq + (int64_t)rows[sl] * d + g * 8) = packed;
-        }
+        for (int c = 0; c < 8; ++c) q[c] = s > 0.0f ? quant_code_fast(v[gi][c], s, rs) : 0;
+        const uint2 packed = make_uint2(pack4(q[0], q[1], q[2], q[3]), pack4(q[4], q[5], q[6], q[7]));
+        *reinterpret_cast<uint2*>(xq + (int64_t)t * d + g * 8) = packed;
+#pragma unroll
+        for (int sl = 0; sl < kMaxK; ++sl)
+            if (rows[sl] >= 0) *reinterpret_cast<uint2*>(aq + (int64_t)rows[sl] * d + g * 8) = packed;
     }
 }
 
@@ -623,9 +615,13 @@ cudaError_t launch_route_small(const float* logits, const float* bias, int T, in
 cudaError_t launch_smooth_quant(const void* x, int in_dtype, const float* inv_s, int T, int d,
                                 int k, const int32_t* ts2row, int8_t* xq, float* sx, int8_t* aq,
                                 cudaStream_t s) {
-    const int per_block = kSqThreads / 32;
-    smooth_quant_kernel<<<(T + per_block - 1) / per_block, kSqThreads, 0, s>>>(x, in_dtype, inv_s, T, d,
-                                                                               k, ts2row, xq, sx, aq);
+    const int groups = (d / 8 + kSqThreads - 1) / kSqThreads;
+    if (groups <= 4)
+        smooth_quant_kernel<4><<<T, kSqThreads, 0, s>>>(x, in_dtype, inv_s, T, d, k, ts2row, xq, sx, aq);
+    else if (groups <= 8)
+        smooth_quant_kernel<8><<<T, kSqThreads, 0, s>>>(x, in_dtype, inv_s, T, d, k, ts2row, xq, sx, aq);
+    else
+        smooth_quant_kernel<16><<<T, kSqThreads, 0, s>>>(x, in_dtype, inv_s, T, d, k, ts2row, xq, sx, aq);
     return cudaGetLastError();
 }
 
