@@ -49,6 +49,9 @@ def parse():
     p.add_argument("--no-stage-events", action="store_true")
     p.add_argument("--path", choices=["auto", "stream", "tensor"], default="auto",
                    help="expert GEMM path: weight streaming, tcgen05 grouped GEMM, or automatic")
+    p.add_argument("--sweep", action="store_true",
+                   help="token-count x skew x alpha sweep on the decode layer's shape: one JSON line "
+                        "per point and expert path (not the headline line)")
     p.add_argument("--tokens", type=int, default=0,
                    help="override the workload's token count T (same layer, same seeds)")
     p.add_argument("--no-prefill", action="store_true",
@@ -389,6 +392,78 @@ def measure(args, wl, world, rank, local, e2e_on=True, wts=None):
     return out, wts, W
 
 
+def run_sweep(args, local):
+    """T in {1 .. 16384} x {uniform, Zipf(1.1) skew} x alpha in {0.5, 0.7} on the
+    decode layer's shape and weights (seeds 10..41): tokens/s per point for the
+    weight-streaming and the tcgen05 expert paths, with the roofline fraction of
+    the bound that applies (HBM below the machine balance, INT8 tensor above)."""
+    import torch
+
+    import w8a8_quantized_moe_b200 as M
+
+    dev = torch.device("cuda", local)
+    peaks, peak_src = load_peaks()
+    int8_peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]) * INT8_PER_BF16
+    points = synth.sweep_workloads()
+    base = synth.WORKLOADS["decode"]
+    wts = synth.make_weights(base)
+    handles = {}
+    for wl in points:
+        if wl.alpha not in handles:
+            cfg = M.make_config(wl.d, wl.f, wl.E, wl.k, wl.alpha, 0.0, True, M.MOE_BF16, M.MOE_BF16)
+            cal = torch.from_numpy(synth.f32_to_bf16_bits(wts.calib_x).view(np.int16)).view(torch.bfloat16).to(dev)
+            ax = torch.zeros(wl.d, dtype=torch.float32, device=dev)
+            M.moe_w8a8_calibrate_absmax(cal, ax)
+            wg, wu, wd = (torch.from_numpy(a).to(dev) for a in (wts.w_gate, wts.w_up, wts.w_down))
+            # one router W_g ~N(0, 0.02^2) for the whole sweep (part of the layer's weights)
+            wr = torch.from_numpy(synth.normal(base.weight_seed, synth.TID_W_ROUTER, (wl.d, wl.E),
+                                               std=0.02)).to(dev)
+            handles[wl.alpha] = M.moe_w8a8_prepare(cfg, wg, wu, wd, wr, ax)
+            del wg, wu, wd
+            torch.cuda.empty_cache()
+    stream = torch.cuda.current_stream(dev)
+    for wl in points:
+        W = handles[wl.alpha]
+        data = synth.make_data(wl)
+        T = wl.T
+        x = torch.from_numpy(data.x_bits.view(np.int16)).view(torch.bfloat16).to(dev)
+        bias = torch.from_numpy(data.router_bias).to(dev) if data.router_bias is not None else None
+        logits = None   # the layer's router computes X W_router (timed)
+        y = torch.empty((T, wl.d), dtype=torch.bfloat16, device=dev)
+        for path_name, path in (("stream", M.MOE_PATH_STREAM), ("tensor", M.MOE_PATH_TENSOR)):
+            M.moe_w8a8_set_path(W, path)
+            ws = torch.empty(M.moe_w8a8_workspace_size(W, T), dtype=torch.uint8, device=dev)
+            offs = torch.empty(wl.E + 1, dtype=torch.int32, device=dev)
+            M.moe_w8a8_forward(W, x, T, bias, logits, y, ws, {"offsets": offs})
+            counts = np.diff(offs.cpu().numpy())
+            n_active, R = int((counts > 0).sum()), int(counts.sum())
+            alg = algorithmic(wl, n_active, R)
+            steps = max(3, min(args.steps, int(2e5 / max(T, 1))))
+            for _ in range(3):
+                M.moe_w8a8_forward(W, x, T, bias, logits, y, ws)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            torch.cuda.synchronize(dev)
+            e0.record(stream)
+            for _ in range(steps):
+                M.moe_w8a8_forward(W, x, T, bias, logits, y, ws)
+            e1.record(stream)
+            torch.cuda.synchronize(dev)
+            M.moe_w8a8_check_status(W)
+            step_s = e0.elapsed_time(e1) / steps / 1e3
+            t_hbm = alg["layer_bytes"] / (peaks["hbm_gbs"] * 1e9)
+            t_tc = alg["int8_ops"] / (int8_peak * 1e12)
+            bound = "hbm" if t_hbm >= t_tc else "tensor"
+            print(json.dumps({"sweep_point": wl.name, "T": T, "skew": "zipf1.1" if wl.zipf_s else "uniform",
+                              "alpha": wl.alpha, "seed": wl.data_seed, "path": path_name,
+                              "tokens_per_s": T / step_s, "ms_per_step": step_s * 1e3,
+                              "active_experts": n_active, "rows": R, "bound": bound,
+                              "roofline_frac": max(t_hbm, t_tc) / step_s,
+                              "peak_source": f"{peak_src} (hbm_gbs, 2 x bf16_tflops_sustained)"}),
+                  flush=True)
+            del ws
+        M.moe_w8a8_set_path(W, M.MOE_PATH_AUTO)
+
+
 def run_ours(args, world, rank, local):
     import torch
 
@@ -398,6 +473,10 @@ def run_ours(args, world, rank, local):
     if not os.path.exists(M.LIB_PATH):
         B.build()
     torch.cuda.set_device(local)
+    if args.sweep:
+        if rank == 0:
+            run_sweep(args, local)
+        return
     import dataclasses
     base = synth.WORKLOADS[args.workload]
     if args.tokens > 0:
