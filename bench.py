@@ -282,7 +282,7 @@ def measure(args, wl, world, rank, local, e2e_on=True, wts=None):
     counts = np.diff(offs.cpu().numpy())
     n_active, R = int((counts > 0).sum()), int(counts.sum())
     alg = algorithmic(wl, n_active, R)
-    tensor = args.path == "tensor" or (args.path == "auto" and T * wl.k > 512)
+    tensor = args.path == "tensor" or (args.path == "auto" and T * wl.k > 32)
 
     stream = torch.cuda.current_stream(dev)
     for _ in range(args.warmup):

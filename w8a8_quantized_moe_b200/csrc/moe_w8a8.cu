@@ -159,7 +159,7 @@ moe_status moe_w8a8_prepare(const moe_w8a8_config* cfg, const float* w_gate, con
     moe_w8a8_weights* w = new moe_w8a8_weights();
     w->cfg = c;
     w->path = MOE_PATH_AUTO;
-    w->stream_max_rows = 512;
+    w->stream_max_rows = 32;   // measured crossover: streaming wins up to T*k = 32 rows
     if (cudaGetDevice(&w->device) != cudaSuccess ||
         cudaDeviceGetAttribute(&w->num_sms, cudaDevAttrMultiProcessorCount, w->device) != cudaSuccess) {
         free_handle(w);
