@@ -549,7 +549,7 @@ extern "C" moe_status moe_w8a8_forward_noalloc(const moe_w8a8_weights* w, const 
     if (!w || T < 0) return MOE_ERR_INVALID_ARG;
     if (T == 0) return MOE_OK;
     if (!x || !y) return MOE_ERR_INVALID_ARG;
-    if (choose_path(w, T) == MOE_PATH_TENSOR) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (choose_path(w, T) == MOE_PATH_TENSOR && !tensor_ok(w)) return MOE_ERR_UNSUPPORTED_SHAPE;
     if (ws_layout(w, T).total > (size_t)MOE_NOALLOC_SCRATCH_BYTES) return MOE_ERR_WORKSPACE_TOO_SMALL;
     void* scratch = noalloc_scratch_for_current_device();
     if (!scratch) return MOE_ERR_CUDA;
