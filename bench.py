@@ -34,6 +34,12 @@ METRIC = "W8A8 MoE layer tokens/s at T=32 and T=16384; % of HBM / INT8 TC roofli
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 INT8_PER_BF16 = 2.0   # nominal dense ratio (4.5 POPS int8 / 2.25 PFLOPS bf16)
 
+# DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum) of the dominant
+# kernel, from one ncu capture of the current kernel source (see profiles/).
+TRAFFIC = {
+    ("decode", 32, "tc_gemm_kernel<0>"): 706.834176e6 + 4.643584e6,
+}
+
 
 def parse():
     p = argparse.ArgumentParser()
@@ -139,16 +145,22 @@ class ClockSampler:
 
 # ------------------------------------------------------------------ byte / op model
 
-def algorithmic(wl: synth.Workload, n_active: int, R: int):
-    """Per-step algorithmic bytes and INT8 ops of the layer and of the gate/up
-    stage (the dominant stage): active experts' INT8 weights (3 d f bytes each)
-    and their fp32 scales, X in, Y out, router input; intermediates excluded."""
+def algorithmic(wl: synth.Workload, n_active: int, R: int, tensor: bool = False):
+    """Per-step algorithmic bytes and INT8 ops.  Layer: active experts' INT8
+    weights (3 d f bytes each) and their fp32 scales, X in, Y out, router input;
+    intermediates excluded.  Per GEMM launch: the weights of the active experts
+    plus that launch's own inputs and outputs (streaming path: A rows and the
+    INT32 accumulators; tensor path: sorted A rows, fp32 h + partial maxima for
+    GEMM1, h codes and fp32 expert outputs for GEMM2)."""
     in_b = 2 if wl.in_bf16 else 4
     w_bytes = n_active * 3 * wl.d * wl.f
     scales = n_active * (2 * wl.f + wl.d) * 4
     router = wl.T * wl.E * 4 if wl.logits_uniform else wl.d * wl.E * 4
     layer = w_bytes + scales + wl.T * wl.d * in_b * 2 + router
-    gemm1 = n_active * 2 * wl.f * wl.d + wl.T * wl.d + R * 2 * wl.f * 4
+    if tensor:
+        gemm1 = n_active * 2 * wl.f * wl.d + R * wl.d + R * wl.f * 4 + R * (wl.f // 64) * 4
+    else:
+        gemm1 = n_active * 2 * wl.f * wl.d + wl.T * wl.d + R * 2 * wl.f * 4
     gemm2 = n_active * wl.d * wl.f + R * wl.f + R * wl.d * 4 + n_active * wl.d * 4
     ops = 2 * R * 3 * wl.d * wl.f
     return dict(layer_bytes=layer, gemm1_bytes=gemm1, gemm2_bytes=gemm2, int8_ops=ops)
@@ -170,13 +182,22 @@ def dist_setup(args):
 
 
 def max_over_ranks(v: float, world: int) -> float:
+    """The slowest rank's time (every rank gets it)."""
     if world == 1:
         return v
     import torch
     import torch.distributed as dist
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def replica_workload(base: synth.Workload, rank: int) -> synth.Workload:
+    """Replicas: the same layer weights on every rank, a different token batch
+    (data seed) per rank."""
+    import dataclasses
+    return dataclasses.replace(base, data_seed=base.data_seed + 1000 * rank) if rank else base
 
 
 def barrier(world: int):
@@ -298,8 +319,8 @@ def measure(args, wl, world, rank, local, e2e_on=True, wts=None):
     M.moe_w8a8_forward(W, x, T, bias, logits, y, ws, {"offsets": offs})
     counts = np.diff(offs.cpu().numpy())
     n_active, R = int((counts > 0).sum()), int(counts.sum())
-    alg = algorithmic(wl, n_active, R)
     tensor = args.path == "tensor" or (args.path == "auto" and T * wl.k > 32)
+    alg = algorithmic(wl, n_active, R, tensor)
 
     stream = torch.cuda.current_stream(dev)
     for _ in range(args.warmup):
@@ -365,29 +386,31 @@ def measure(args, wl, world, rank, local, e2e_on=True, wts=None):
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(yh.numel() * yh.element_size())}
 
     peaks, peak_src = load_peaks()
+    int8_peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]) * INT8_PER_BF16
     roof = None
     if stages:
         dom = max(("gemm1", "gemm2"), key=lambda k: stages[k])
         dom_ms = stages[dom]
-        if tensor:
-            ops = 2 * R * (2 * wl.f if dom == "gemm1" else wl.f) * wl.d
-            peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]) * INT8_PER_BF16
+        kernel = (f"tc_gemm_kernel<{0 if dom == 'gemm1' else 1}>" if tensor else
+                  ("stream_gateup_kernel" if dom == "gemm1" else "stream_down_kernel"))
+        ops = 2 * R * (2 * wl.f if dom == "gemm1" else wl.f) * wl.d
+        nbytes = alg[f"{dom}_bytes"]
+        # the bound is whichever of the byte time and the INT8 op time is larger
+        if ops / (int8_peak * 1e12) > nbytes / (peaks["hbm_gbs"] * 1e9):
             achieved = ops / (dom_ms / 1e3) / 1e12
-            roof = {"bound": "tensor", "kernel": f"{dom} (tc_gemm_kernel<{0 if dom == 'gemm1' else 1}>)",
-                    "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
-                    "traffic": None,
+            roof = {"bound": "tensor", "kernel": f"{dom} ({kernel})", "achieved": achieved,
+                    "peak": int8_peak, "unit": "TFLOP/s", "frac": achieved / int8_peak,
+                    "traffic": TRAFFIC.get((wl.name, wl.T, kernel)),
                     "peak_source": f"2 x bf16_tflops_sustained of {peak_src} (INT8 dense = 2 x bf16, nominal)",
                     "int8_ops_per_launch": ops, "launch_ms": dom_ms,
                     "frac_of_nominal_4500": achieved / 4500.0}
         else:
-            b = alg[f"{dom}_bytes"]
-            achieved = b / (dom_ms / 1e3) / 1e9
-            roof = {"bound": "hbm",
-                    "kernel": f"{dom} ({'stream_gateup_kernel' if dom == 'gemm1' else 'stream_down_kernel'})",
-                    "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                    "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+            achieved = nbytes / (dom_ms / 1e3) / 1e9
+            roof = {"bound": "hbm", "kernel": f"{dom} ({kernel})", "achieved": achieved,
+                    "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
+                    "traffic": TRAFFIC.get((wl.name, wl.T, kernel)),
                     "peak_source": f"hbm_gbs of {peak_src}",
-                    "algorithmic_bytes_per_launch": b, "launch_ms": dom_ms}
+                    "algorithmic_bytes_per_launch": nbytes, "launch_ms": dom_ms}
     step_s = ms_total / K / 1e3
     layer_gbs = alg["layer_bytes"] / step_s / 1e9
     layer_tops = alg["int8_ops"] / step_s / 1e12
@@ -454,7 +477,7 @@ def run_sweep(args, local):
             M.moe_w8a8_forward(W, x, T, bias, logits, y, ws, {"offsets": offs})
             counts = np.diff(offs.cpu().numpy())
             n_active, R = int((counts > 0).sum()), int(counts.sum())
-            alg = algorithmic(wl, n_active, R)
+            alg = algorithmic(wl, n_active, R, path_name == "tensor")
             steps = max(3, min(args.steps, int(2e5 / max(T, 1))))
             for _ in range(3):
                 M.moe_w8a8_forward(W, x, T, bias, logits, y, ws)
@@ -498,15 +521,13 @@ def run_ours(args, world, rank, local):
     base = synth.WORKLOADS[args.workload]
     if args.tokens > 0:
         base = dataclasses.replace(base, T=args.tokens)
-    # replicas: same layer weights on every rank, a different token batch per rank
-    wl = dataclasses.replace(base, data_seed=base.data_seed + 1000 * rank) if rank else base
+    wl = replica_workload(base, rank)
     res, wts, W = measure(args, wl, world, rank, local)
     del W
 
     extra = None
     if args.workload == "decode" and not args.no_prefill:
-        pw = synth.WORKLOADS["prefill"]
-        pw = dataclasses.replace(pw, data_seed=pw.data_seed + 1000 * rank) if rank else pw
+        pw = replica_workload(synth.WORKLOADS["prefill"], rank)
         # the prefill layer reuses the decode layer's expert weights
         pres, _, PW = measure(args, pw, world, rank, local, e2e_on=False, wts=wts)
         del PW
