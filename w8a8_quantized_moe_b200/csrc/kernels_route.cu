@@ -33,6 +33,9 @@ __device__ __forceinline__ int rt_swz(int p, int i) { return ((((p >> 3) & 3) | 
 __global__ void __launch_bounds__(kRtThreads) router_logits_kernel(
     const void* __restrict__ x, int in_dtype, const float* __restrict__ wr, int T, int d, int E,
     float* __restrict__ logits) {
+    pdl_wait();
+    pdl_trigger();
+
     __shared__ __align__(16) float xs[kRtKC / 32][32][kRtPad];
     __shared__ __align__(16) float ws[kRtKC / 32][32][kRtPad];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -137,6 +140,9 @@ template <int XB>
 __global__ void __launch_bounds__(kRtThreads) router_logits_async_kernel(
     const void* __restrict__ x, const float* __restrict__ wr, int T, int d, int E,
     float* __restrict__ logits) {
+    pdl_wait();
+    pdl_trigger();
+
     extern __shared__ __align__(16) uint8_t smem_raw[];
     RouterAsyncSmem<XB>& sm = *reinterpret_cast<RouterAsyncSmem<XB>*>(smem_raw);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -293,6 +299,9 @@ __device__ __forceinline__ void topk_token(const float* __restrict__ logits,
 __global__ void topk_kernel(const float* __restrict__ logits, const float* __restrict__ bias, int T,
                             int E, int k, int renorm, int32_t* __restrict__ idx,
                             float* __restrict__ wts, float* __restrict__ logits_out) {
+    pdl_wait();
+    pdl_trigger();
+
     __shared__ float lsh[8][kMaxE];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int t = blockIdx.x * 8 + warp;
@@ -394,6 +403,9 @@ __device__ void scatter_entries(const int32_t* idx, int base, int len, int E, in
 
 __global__ void perm_hist_kernel(const int32_t* __restrict__ idx, int n, int E,
                                  int32_t* __restrict__ hist) {
+    pdl_wait();
+    pdl_trigger();
+
     __shared__ int cnt[kMaxE];
     for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[e] = 0;
     __syncthreads();
@@ -411,6 +423,9 @@ __global__ void __launch_bounds__(kPermThreads) perm_scatter_kernel(
     const int32_t* __restrict__ hist, int32_t* __restrict__ offsets, int32_t* __restrict__ row2ts,
     int32_t* __restrict__ ts2row, int32_t* __restrict__ meta, int32_t* __restrict__ active,
     int32_t* __restrict__ tiles) {
+    pdl_wait();
+    pdl_trigger();
+
     __shared__ int pre[kMaxE], off[kMaxE + 1], running[kMaxE], kept[kMaxE];
     __shared__ int wcnt[kPermThreads / 32][kMaxE];
     const int tid = threadIdx.x;
@@ -461,6 +476,9 @@ __global__ void __launch_bounds__(kRouteSmallThreads) route_small_kernel(
     float* __restrict__ logits_out, int32_t* __restrict__ offsets, int32_t* __restrict__ row2ts,
     int32_t* __restrict__ ts2row, int32_t* __restrict__ meta, int32_t* __restrict__ active,
     int32_t* __restrict__ tiles) {
+    pdl_wait();
+    pdl_trigger();
+
     extern __shared__ __align__(16) uint8_t smem_raw[];
     RouteSmallSmem& sm = *reinterpret_cast<RouteSmallSmem*>(smem_raw);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -500,6 +518,9 @@ __global__ void __launch_bounds__(kSqThreads) smooth_quant_kernel(
     const void* __restrict__ x, int in_dtype, const float* __restrict__ inv_s, int T, int d, int k,
     const int32_t* __restrict__ ts2row, int8_t* __restrict__ xq, float* __restrict__ sx,
     int8_t* __restrict__ aq) {
+    pdl_wait();
+    pdl_trigger();
+
     __shared__ float red[kSqThreads / 32];
     const int t = blockIdx.x, tid = threadIdx.x, lane = tid & 31;
     const int ng = d / 8;
@@ -565,19 +586,21 @@ cudaError_t launch_router_logits(const void* x, int in_dtype, const float* wr, i
             attr = true;
         }
         if (in_dtype == MOE_BF16)
-            router_logits_async_kernel<2><<<grid, kRtThreads, sizeof(RouterAsyncSmem<2>), s>>>(x, wr, T, d, E, logits);
+            return launch_pdl(router_logits_async_kernel<2>, grid, dim3(kRtThreads), sizeof(RouterAsyncSmem<2>), s,
+                              x, wr, T, d, E, logits);
         else
-            router_logits_async_kernel<4><<<grid, kRtThreads, sizeof(RouterAsyncSmem<4>), s>>>(x, wr, T, d, E, logits);
+            return launch_pdl(router_logits_async_kernel<4>, grid, dim3(kRtThreads), sizeof(RouterAsyncSmem<4>), s,
+                              x, wr, T, d, E, logits);
     } else {
-        router_logits_kernel<<<grid, kRtThreads, 0, s>>>(x, in_dtype, wr, T, d, E, logits);
+        return launch_pdl(router_logits_kernel, grid, dim3(kRtThreads), 0, s, x, in_dtype, wr, T, d, E, logits);
     }
     return cudaGetLastError();
 }
 
 cudaError_t launch_topk(const float* logits, const float* bias, int T, int E, int k, int renorm,
                         int32_t* idx, float* wts, float* logits_out, cudaStream_t s) {
-    topk_kernel<<<(T + 7) / 8, 256, 0, s>>>(logits, bias, T, E, k, renorm, idx, wts, logits_out);
-    return cudaGetLastError();
+    return launch_pdl(topk_kernel, dim3((T + 7) / 8), dim3(256), 0, s, logits, bias, T, E, k, renorm, idx,
+                      wts, logits_out);
 }
 
 cudaError_t launch_permute(const int32_t* idx, int T, int k, int E, int cap, int32_t* hist,
@@ -585,12 +608,10 @@ cudaError_t launch_permute(const int32_t* idx, int T, int k, int E, int cap, int
                            int32_t* active, int32_t* tiles, cudaStream_t s) {
     const int n = T * k;
     const int nblk = (n + kPermChunk - 1) / kPermChunk;
-    perm_hist_kernel<<<nblk, 256, 0, s>>>(idx, n, E, hist);
-    cudaError_t err = cudaGetLastError();
+    cudaError_t err = launch_pdl(perm_hist_kernel, dim3(nblk), dim3(256), 0, s, idx, n, E, hist);
     if (err != cudaSuccess) return err;
-    perm_scatter_kernel<<<nblk, kPermThreads, 0, s>>>(idx, n, E, cap, nblk, hist, offsets, row2ts,
-                                                      ts2row, meta, active, tiles);
-    return cudaGetLastError();
+    return launch_pdl(perm_scatter_kernel, dim3(nblk), dim3(kPermThreads), 0, s, idx, n, E, cap, nblk, hist,
+                      offsets, row2ts, ts2row, meta, active, tiles);
 }
 
 bool route_small_ok(int T, int k) { return (int64_t)T * k <= kRouteSmallMax; }
@@ -606,23 +627,17 @@ cudaError_t launch_route_small(const float* logits, const float* bias, int T, in
         if (e != cudaSuccess) return e;
         attr = true;
     }
-    route_small_kernel<<<1, kRouteSmallThreads, sizeof(RouteSmallSmem), s>>>(
-        logits, bias, T, E, k, renorm, cap, idx, wts, logits_out, offsets, row2ts, ts2row, meta,
-        active, tiles);
-    return cudaGetLastError();
+    return launch_pdl(route_small_kernel, dim3(1), dim3(kRouteSmallThreads), sizeof(RouteSmallSmem), s, logits,
+                      bias, T, E, k, renorm, cap, idx, wts, logits_out, offsets, row2ts, ts2row, meta,
+                      active, tiles);
 }
 
 cudaError_t launch_smooth_quant(const void* x, int in_dtype, const float* inv_s, int T, int d,
                                 int k, const int32_t* ts2row, int8_t* xq, float* sx, int8_t* aq,
                                 cudaStream_t s) {
     const int groups = (d / 8 + kSqThreads - 1) / kSqThreads;
-    if (groups <= 4)
-        smooth_quant_kernel<4><<<T, kSqThreads, 0, s>>>(x, in_dtype, inv_s, T, d, k, ts2row, xq, sx, aq);
-    else if (groups <= 8)
-        smooth_quant_kernel<8><<<T, kSqThreads, 0, s>>>(x, in_dtype, inv_s, T, d, k, ts2row, xq, sx, aq);
-    else
-        smooth_quant_kernel<16><<<T, kSqThreads, 0, s>>>(x, in_dtype, inv_s, T, d, k, ts2row, xq, sx, aq);
-    return cudaGetLastError();
+    auto kern = groups <= 4 ? smooth_quant_kernel<4> : groups <= 8 ? smooth_quant_kernel<8> : smooth_quant_kernel<16>;
+    return launch_pdl(kern, dim3(T), dim3(kSqThreads), 0, s, x, in_dtype, inv_s, T, d, k, ts2row, xq, sx, aq);
 }
 
 }  // namespace moe

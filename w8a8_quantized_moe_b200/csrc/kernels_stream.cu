@@ -77,7 +77,9 @@ __global__ void __launch_bounds__(kStThreads) stream_gateup_kernel(
     const int8_t* __restrict__ w_gu, int d, int f, int k, const int8_t* __restrict__ xq,
     const int32_t* __restrict__ row2ts, const int32_t* __restrict__ offsets,
     const int32_t* __restrict__ active, const int32_t* __restrict__ meta,
-    int32_t* __restrict__ acc1) {
+    int32_t* __restrict__ acc1) {    pdl_wait();
+    pdl_trigger();
+
     extern __shared__ __align__(16) int8_t As[];   // [kStRows][d]
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int n_units_e = (2 * f) / kGuUnit;
@@ -128,7 +130,9 @@ __global__ void __launch_bounds__(kSwThreads) swiglu_requant_kernel(
     const int32_t* __restrict__ acc1, int f, int k, const int32_t* __restrict__ row2ts,
     const int32_t* __restrict__ topk_idx, const float* __restrict__ sx,
     const float* __restrict__ sw_gate, const float* __restrict__ sw_up,
-    const int32_t* __restrict__ meta, int8_t* __restrict__ hq, float* __restrict__ sh) {
+    const int32_t* __restrict__ meta, int8_t* __restrict__ hq, float* __restrict__ sh) {    pdl_wait();
+    pdl_trigger();
+
     extern __shared__ __align__(16) float hs[];   // [f]
     __shared__ float red[32];
     const int r = blockIdx.x;
@@ -179,7 +183,9 @@ __global__ void __launch_bounds__(kStThreads) stream_down_kernel(
     const float* __restrict__ sh, const int32_t* __restrict__ row2ts,
     const float* __restrict__ topk_w, const float* __restrict__ sw_dn,
     const int32_t* __restrict__ offsets, const int32_t* __restrict__ active,
-    const int32_t* __restrict__ meta, float* __restrict__ o, int32_t* __restrict__ acc2_dbg) {
+    const int32_t* __restrict__ meta, float* __restrict__ o, int32_t* __restrict__ acc2_dbg) {    pdl_wait();
+    pdl_trigger();
+
     extern __shared__ __align__(16) int8_t As[];   // [kStRows][f]
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int n_units_e = d / kDnUnit;
@@ -222,7 +228,9 @@ __global__ void __launch_bounds__(kStThreads) stream_down_kernel(
 // Un-sort + weighted sum: y[t] = ((0 + o_slot0) + o_slot1) + ... over the kept
 // slots, in slot order, then cast to the output dtype.
 __global__ void combine_kernel(const float* __restrict__ o, const int32_t* __restrict__ ts2row,
-                               int k, int d, int out_dtype, void* __restrict__ y) {
+                               int k, int d, int out_dtype, void* __restrict__ y) {    pdl_wait();
+    pdl_trigger();
+
     const int t = blockIdx.x;
     const int n4 = blockIdx.y * blockDim.x + threadIdx.x;
     if (n4 * 4 >= d) return;
@@ -264,10 +272,9 @@ cudaError_t launch_stream_gateup(const moe_w8a8_weights* w, int T, const int8_t*
         attr = true;
     }
     const int grid = stream_grid(w, w->cfg.n_experts * (2 * f / kGuUnit));
-    stream_gateup_kernel<<<grid, kStThreads, smem, s>>>(w->w_gu, d, f, w->cfg.top_k, xq, row2ts,
-                                                        offsets, active, meta, acc1);
     (void)T;
-    return cudaGetLastError();
+    return launch_pdl(stream_gateup_kernel, dim3(grid), dim3(kStThreads), smem, s, w->w_gu, d, f,
+                      w->cfg.top_k, xq, row2ts, offsets, active, meta, acc1);
 }
 
 cudaError_t launch_swiglu_requant(const moe_w8a8_weights* w, const int32_t* acc1,
@@ -280,9 +287,8 @@ cudaError_t launch_swiglu_requant(const moe_w8a8_weights* w, const int32_t* acc1
         cudaFuncSetAttribute(swiglu_requant_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 100 * 1024);
         attr = true;
     }
-    swiglu_requant_kernel<<<max_rows, kSwThreads, (size_t)f * 4, s>>>(
-        acc1, f, w->cfg.top_k, row2ts, topk_idx, sx, w->sw_gate, w->sw_up, meta, hq, sh);
-    return cudaGetLastError();
+    return launch_pdl(swiglu_requant_kernel, dim3(max_rows), dim3(kSwThreads), (size_t)f * 4, s, acc1, f,
+                      w->cfg.top_k, row2ts, topk_idx, sx, w->sw_gate, w->sw_up, meta, hq, sh);
 }
 
 cudaError_t launch_stream_down(const moe_w8a8_weights* w, int T, const int8_t* hq, const float* sh,
@@ -292,17 +298,15 @@ cudaError_t launch_stream_down(const moe_w8a8_weights* w, int T, const int8_t* h
     const int d = w->cfg.d, f = w->cfg.f;
     const size_t smem = (size_t)kStRows * f;
     const int grid = stream_grid(w, w->cfg.n_experts * (d / kDnUnit));
-    stream_down_kernel<<<grid, kStThreads, smem, s>>>(w->w_dn, d, f, hq, sh, row2ts, topk_w,
-                                                      w->sw_dn, offsets, active, meta, o, acc2_dbg);
     (void)T;
-    return cudaGetLastError();
+    return launch_pdl(stream_down_kernel, dim3(grid), dim3(kStThreads), smem, s, w->w_dn, d, f, hq, sh,
+                      row2ts, topk_w, w->sw_dn, offsets, active, meta, o, acc2_dbg);
 }
 
 cudaError_t launch_combine(const float* o, const int32_t* ts2row, int T, int k, int d,
                            int out_dtype, void* y, cudaStream_t s) {
     dim3 grid(T, (d / 4 + 255) / 256);
-    combine_kernel<<<grid, 256, 0, s>>>(o, ts2row, k, d, out_dtype, y);
-    return cudaGetLastError();
+    return launch_pdl(combine_kernel, grid, dim3(256), 0, s, o, ts2row, k, d, out_dtype, y);
 }
 
 }  // namespace moe

@@ -346,7 +346,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     float* epi_stage = reinterpret_cast<float*>(smem + kStages * kStageBytes);
     Ctl* ctl = reinterpret_cast<Ctl*>(smem + kStages * kStageBytes + kEpiWarps * kEpiStageBytes);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int num_tiles = p.meta[META_NTILES] * p.n_tiles_n;
     const int nkb = p.K / BK;
 
     if (threadIdx.x == 0) {
@@ -373,6 +372,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     const uint32_t tmem = ctl->tmem_base;
     volatile int* abort = &ctl->abort;
+    // everything above overlaps the previous kernel; its results are read below
+    pdl_wait();
+    pdl_trigger();
+    const int num_tiles = p.meta[META_NTILES] * p.n_tiles_n;
 
     if (warp == 0) {
         if (lane == 0) {
@@ -484,7 +487,9 @@ __global__ void __launch_bounds__(kRqThreads) requant_kernel(const float* __rest
                                                              const float* __restrict__ pamax, int f,
                                                              const int32_t* __restrict__ meta,
                                                              int8_t* __restrict__ hq,
-                                                             float* __restrict__ sh) {
+                                                             float* __restrict__ sh) {    pdl_wait();
+    pdl_trigger();
+
     const int lane = threadIdx.x & 31;
     const int row = blockIdx.x * (kRqThreads / 32) + (threadIdx.x >> 5);
     if (row >= meta[META_R]) return;
@@ -565,8 +570,7 @@ cudaError_t launch(const CUtensorMap& ta, const CUtensorMap& tb, const TcParams&
         if (e != cudaSuccess) return e;
         attr = true;
     }
-    tc_gemm_kernel<EPI><<<grid, kThreads, kSmemBytes, s>>>(ta, tb, p);
-    return cudaGetLastError();
+    return launch_pdl(tc_gemm_kernel<EPI>, dim3(grid), dim3(kThreads), kSmemBytes, s, ta, tb, p);
 }
 
 }  // namespace
@@ -582,9 +586,8 @@ bool tc_supported(const moe_w8a8_config& c) { return c.d % BN == 0 && c.f % BK =
 cudaError_t launch_requant(const float* h32, const float* pamax, int f, const int32_t* meta,
                            int max_rows, int8_t* hq, float* sh, cudaStream_t s) {
     const int rows_per_block = kRqThreads / 32;
-    requant_kernel<<<(max_rows + rows_per_block - 1) / rows_per_block, kRqThreads, 0, s>>>(
-        h32, pamax, f, meta, hq, sh);
-    return cudaGetLastError();
+    return launch_pdl(requant_kernel, dim3((max_rows + rows_per_block - 1) / rows_per_block),
+                      dim3(kRqThreads), 0, s, h32, pamax, f, meta, hq, sh);
 }
 
 cudaError_t launch_tc_gemm1(const moe_w8a8_weights* w, int T, const int8_t* aq, const int32_t* meta,
