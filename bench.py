@@ -60,6 +60,9 @@ def parse():
                         "per point and expert path (not the headline line)")
     p.add_argument("--tokens", type=int, default=0,
                    help="override the workload's token count T (same layer, same seeds)")
+    p.add_argument("--act-clip", type=float, default=0.0, metavar="PERCENT",
+                   help="saturating activation clip at this percentile of the smoothed calibration "
+                        "activations (0: off)")
     p.add_argument("--no-prefill", action="store_true",
                    help="skip the extra prefill-layer measurement of the decode run")
     return p.parse_args()
@@ -303,6 +306,10 @@ def measure(args, wl, world, rank, local, e2e_on=True, wts=None):
     W = M.moe_w8a8_prepare(cfg, wg, wu, wd, wr, ax)
     M.moe_w8a8_set_path(W, {"auto": M.MOE_PATH_AUTO, "stream": M.MOE_PATH_STREAM,
                             "tensor": M.MOE_PATH_TENSOR}[args.path])
+    clip = 0.0
+    if getattr(args, "act_clip", 0.0) > 0.0:
+        clip = M.moe_w8a8_calibrate_act_clip(W, cal, args.act_clip)
+        M.moe_w8a8_set_act_clip(W, clip)
     del wg, wu, wd, cal
     torch.cuda.empty_cache()
 
@@ -429,6 +436,8 @@ def measure(args, wl, world, rank, local, e2e_on=True, wts=None):
         "roofline": roof, "stages_ms": stages, "e2e": e2e, "gpu_launches": launches,
         "clocks": clocks.summary(),
     }
+    if clip > 0.0:
+        out["config"]["act_clip"] = {"percentile": args.act_clip, "value": clip}
     return out, wts, W
 
 

@@ -200,6 +200,35 @@ moe_status moe_w8a8_set_path(moe_w8a8_weights* w, int32_t path);
 /* Row count at or below which MOE_PATH_AUTO uses the streaming path. */
 moe_status moe_w8a8_set_stream_threshold(moe_w8a8_weights* w, int32_t max_rows);
 
+/*
+ * Saturating activation clip (mhpq.cn page s6.4, the third defence against
+ * activation outliers: cut values at a threshold instead of stretching the
+ * scale to the maximum; gtnt.cn page s3.2: the threshold is a percentile of
+ * the calibration activations, 99.9 there).  With clip > 0 every forward
+ * quantises token t of the smoothed input x' = x * inv_s with the range
+ * a_t = min(max_j |x'_tj|, clip): scale a_t / 127, codes rint(x' / scale)
+ * clamped to +-127, so values beyond the clip saturate.  clip = 0 turns it
+ * off (the default).  Only the layer input is clipped, not the expert's
+ * intermediate h.  Returns MOE_ERR_INVALID_ARG for a negative or non-finite
+ * clip.  Takes effect from the next forward; do not change it while a
+ * forward on this handle may be in flight.
+ */
+moe_status moe_w8a8_set_act_clip(moe_w8a8_weights* w, float clip);
+
+/*
+ * The clip threshold from calibration rows x [rows][d] (device, dtype
+ * MOE_F32 or MOE_BF16): the nearest-rank `percent` percentile (0 < percent
+ * <= 100) of |x[r][j] * inv_s[j]| over every element, i.e. the
+ * ceil(percent/100 * rows * d)-th smallest, written to *clip_host.  Calibration
+ * helper, not part of the forward: it allocates rows * d * 4 bytes of device
+ * memory, runs one kernel, copies the values to the host and selects there,
+ * and synchronises `stream`.  Does not change the handle; pass the value to
+ * moe_w8a8_set_act_clip.
+ */
+moe_status moe_w8a8_calibrate_act_clip(const moe_w8a8_weights* w, const void* x, int64_t rows,
+                                       int32_t dtype, double percent, float* clip_host,
+                                       moe_stream_t stream);
+
 /* Smoothing scales s [d] copied to host memory. */
 moe_status moe_w8a8_get_smooth_scales(const moe_w8a8_weights* w, float* s_host);
 

@@ -54,13 +54,14 @@ def lib():
             "oracle_topk_softmax": ([vp, vp, i64, i32, i32, i32, vp, vp], None),
             "oracle_capacity": ([f32, i64, i32, i32], i32),
             "oracle_permute": ([vp, i64, i32, i32, i32, vp, vp, vp], i32),
-            "oracle_quantize_tokens": ([vp, vp, i64, i32, vp, vp], None),
+            "oracle_quantize_tokens": ([vp, vp, i64, i32, f32, vp, vp], None),
+            "oracle_act_clip_percentile": ([vp, vp, i64, i32, ctypes.c_double], f32),
             "oracle_gemm_i8": ([vp, vp, i64, i64, i64, vp], None),
             "oracle_swiglu_requant": ([vp, vp, f32, vp, vp, i32, vp, vp, vp], None),
             "oracle_down_epilogue": ([vp, f32, vp, f32, i32, vp], None),
             "oracle_round_bf16": ([f32], f32),
-            "oracle_moe_tokens": ([vp, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp,
-                                   vp, i64, i32, vp, vp, vp, vp, vp, vp, vp, vp], None),
+            "oracle_moe_tokens": ([vp, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp, vp, f32, vp, vp,
+                                   vp, vp, i64, i32, vp, vp, vp, vp, vp, vp, vp, vp], None),
         }
         for name, (args, res) in sig.items():
             fn = getattr(L, name)
@@ -174,13 +175,22 @@ def permute(idx, E: int, cap: int = -1):
     return offsets, row2ts[:R].copy(), ts2row
 
 
-def quantize_tokens(x, inv_s):
+def quantize_tokens(x, inv_s, act_clip: float = 0.0):
+    """Per-token INT8 codes of x' = x * inv_s; act_clip > 0 caps each token's
+    range at act_clip (values beyond it saturate at +-127)."""
     x = _c(x, np.float32)
     T, d = x.shape
     q = np.empty((T, d), dtype=np.int8)
     sx = np.empty(T, dtype=np.float32)
-    lib().oracle_quantize_tokens(P(x), P(_c(inv_s, np.float32)), T, d, P(q), P(sx))
+    lib().oracle_quantize_tokens(P(x), P(_c(inv_s, np.float32)), T, d, float(act_clip), P(q), P(sx))
     return q, sx
+
+
+def act_clip_percentile(x, inv_s, percent: float) -> float:
+    """Nearest-rank percentile of |x * inv_s| over every element of x [rows][d]."""
+    x = _c(x, np.float32)
+    rows, d = x.shape
+    return float(lib().oracle_act_clip_percentile(P(x), P(_c(inv_s, np.float32)), rows, d, float(percent)))
 
 
 def gemm_i8(a, b) -> np.ndarray:
@@ -279,8 +289,10 @@ def route(x, k: int, E: int, w_router=None, logits=None, bias=None, renormalize=
     return Routing(logits, idx, w, cap, offsets, row2ts, ts2row)
 
 
-def moe_tokens(x, prep: Prepared, rt: Routing, tokens=None, out_bf16=False, debug=True):
-    """Expert FFN + combine for the listed tokens (all by default)."""
+def moe_tokens(x, prep: Prepared, rt: Routing, tokens=None, out_bf16=False, debug=True,
+               act_clip: float = 0.0):
+    """Expert FFN + combine for the listed tokens (all by default); act_clip > 0
+    caps the per-token activation range (saturating clip)."""
     x = _c(x, np.float32)
     T, d = x.shape
     E, f, _ = prep.wq_gate.shape
@@ -297,7 +309,7 @@ def moe_tokens(x, prep: Prepared, rt: Routing, tokens=None, out_bf16=False, debu
     g = dbg.get
     lib().oracle_moe_tokens(P(x), d, f, E, k, P(prep.wq_gate), P(prep.wq_up), P(prep.sw_gate),
                             P(prep.sw_up), P(prep.wq_down), P(prep.sw_down), P(prep.inv_s),
-                            P(rt.idx), P(rt.w), P(_c(rt.ts2row, np.int32)), P(tok), n,
+                            float(act_clip), P(rt.idx), P(rt.w), P(_c(rt.ts2row, np.int32)), P(tok), n,
                             1 if out_bf16 else 0, P(y), P(g("xq")), P(g("sx")), P(g("acc1")),
                             P(g("hq")), P(g("sh")), P(g("acc2")), P(g("o")))
     return y, dbg

@@ -95,10 +95,14 @@ static inline int8_t quant_one(float v, float scale) {
     return (int8_t)t;
 }
 
-/* Quantise n values read with a stride; writes q contiguously. */
-static float quant_vector(const float* v, int64_t n, int64_t stride, int8_t* q) {
+/* Quantise n values read with a stride; writes q contiguously.  clip > 0    */
+/* caps the range: amax = min(max |v|, clip), so values beyond the cap        */
+/* saturate at +-127 instead of stretching the scale ([MiniMax-M3 W8A8 on     */
+/* K100AI] s6.4, third defence: saturate at a threshold).                    */
+static float quant_vector_clip(const float* v, int64_t n, int64_t stride, int8_t* q, float clip) {
     float amax = 0.0f;
     for (int64_t i = 0; i < n; ++i) amax = fmaxf(amax, fabsf(v[i * stride]));
+    if (clip > 0.0f && amax > clip) amax = clip;
     if (amax == 0.0f) {
         memset(q, 0, (size_t)n);
         return 0.0f;
@@ -106,6 +110,10 @@ static float quant_vector(const float* v, int64_t n, int64_t stride, int8_t* q) 
     float scale = amax / 127.0f;
     for (int64_t i = 0; i < n; ++i) q[i] = quant_one(v[i * stride], scale);
     return scale;
+}
+
+static float quant_vector(const float* v, int64_t n, int64_t stride, int8_t* q) {
+    return quant_vector_clip(v, n, stride, q, 0.0f);
 }
 
 void oracle_quantize_rows(const float* v, int64_t rows, int64_t n, int8_t* q, float* scale) {
@@ -303,14 +311,48 @@ int32_t oracle_permute(const int32_t* idx, int64_t T, int32_t k, int32_t E, int3
 /* ([MiniMax-M3 W8A8 on K100AI] s3.2, s6.4): x'_j = fp32(x_j * inv_s_j),    */
 /* then the symmetric INT8 rule over the d channels of the token.           */
 /* ------------------------------------------------------------------------ */
+/* act_clip > 0: the token's range is capped at act_clip (saturation of the  */
+/* smoothed values beyond it); 0: no cap.                                    */
 void oracle_quantize_tokens(const float* x, const float* inv_s, int64_t T, int32_t d,
-                            int8_t* q, float* sx) {
+                            float act_clip, int8_t* q, float* sx) {
     float* xs = (float*)malloc(sizeof(float) * (size_t)d);
     for (int64_t t = 0; t < T; ++t) {
         for (int32_t j = 0; j < d; ++j) xs[j] = inv_s ? x[t * d + j] * inv_s[j] : x[t * d + j];
-        sx[t] = quant_vector(xs, d, 1, q + t * d);
+        sx[t] = quant_vector_clip(xs, d, 1, q + t * d, act_clip);
     }
     free(xs);
+}
+
+/* ------------------------------------------------------------------------ */
+/* Clip threshold from calibration data ("One night of MoE inference         */
+/* optimisation", s3.2: the activation truncation percentile, 99.9; values   */
+/* above that quantile of the activations' range are cut).  READING: the     */
+/* percentile is taken over |x'| of every element of the calibration rows,   */
+/* x' = fp32(x * inv_s) (the values the per-token quantiser sees), with the  */
+/* nearest-rank rule: the ceil(p/100 * n)-th smallest value (p in (0, 100]). */
+/* ------------------------------------------------------------------------ */
+static int cmp_float(const void* a, const void* b) {
+    const float x = *(const float*)a, y = *(const float*)b;
+    return (x > y) - (x < y);
+}
+
+float oracle_act_clip_percentile(const float* x, const float* inv_s, int64_t rows, int32_t d,
+                                 double percent) {
+    const int64_t n = rows * d;
+    if (n <= 0) return 0.0f;
+    float* a = (float*)malloc(sizeof(float) * (size_t)n);
+    for (int64_t r = 0; r < rows; ++r)
+        for (int32_t j = 0; j < d; ++j) {
+            const float v = inv_s ? x[r * d + j] * inv_s[j] : x[r * d + j];
+            a[r * d + j] = fabsf(v);
+        }
+    qsort(a, (size_t)n, sizeof(float), cmp_float);
+    int64_t rank = (int64_t)ceil(percent / 100.0 * (double)n);
+    if (rank < 1) rank = 1;
+    if (rank > n) rank = n;
+    const float c = a[rank - 1];
+    free(a);
+    return c;
 }
 
 /* ------------------------------------------------------------------------ */
@@ -376,7 +418,8 @@ float oracle_round_bf16(float v) {
 /*
  * Inputs: x [T][d] fp32 values; quantised weights in the oracle's layout
  * (wq_gate, wq_up [E][f][d] with sw_gate, sw_up [E][f]; wq_down [E][d][f]
- * with sw_down [E][d]); inv_s [d] (NULL: no smoothing); routing already
+ * with sw_down [E][d]); inv_s [d] (NULL: no smoothing); act_clip (0: none,
+ * else the cap of the per-token range, see oracle_quantize_tokens); routing already
  * done (idx, w [T][k]; ts2row [T][k], -1 = dropped).  Computes the tokens
  * listed in tok[n_sel].  Outputs per selected token i: y [i][d] (fp32 sum
  * y = ((0 + o_slot0) + o_slot1) + ... over kept slots, then bf16-rounded if
@@ -387,7 +430,7 @@ float oracle_round_bf16(float v) {
 void oracle_moe_tokens(const float* x, int32_t d, int32_t f, int32_t E, int32_t k,
                        const int8_t* wq_gate, const int8_t* wq_up, const float* sw_gate,
                        const float* sw_up, const int8_t* wq_down, const float* sw_down,
-                       const float* inv_s, const int32_t* idx, const float* w,
+                       const float* inv_s, float act_clip, const int32_t* idx, const float* w,
                        const int32_t* ts2row, const int64_t* tok, int64_t n_sel, int32_t out_bf16,
                        float* y, int8_t* xq_out, float* sx_out, int32_t* acc1_out, int8_t* hq_out,
                        float* sh_out, int32_t* acc2_out, float* o_out) {
@@ -401,7 +444,7 @@ void oracle_moe_tokens(const float* x, int32_t d, int32_t f, int32_t E, int32_t 
     for (int64_t i = 0; i < n_sel; ++i) {
         int64_t t = tok[i];
         float sx;
-        oracle_quantize_tokens(x + t * d, inv_s, 1, d, xq, &sx);
+        oracle_quantize_tokens(x + t * d, inv_s, 1, d, act_clip, xq, &sx);
         if (xq_out) memcpy(xq_out + i * d, xq, (size_t)d);
         if (sx_out) sx_out[i] = sx;
         float* yt = y + i * d;

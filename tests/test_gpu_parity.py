@@ -201,6 +201,52 @@ def test_tensor_path_decode_layer(M, decode_setup):
         M.moe_w8a8_set_path(W, M.MOE_PATH_AUTO)
 
 
+@pytest.mark.parametrize("T", [1, 5, 13, 47])
+def test_tensor_path_decode_layer_small_batches(M, decode_setup, T):
+    """Few rows per expert on the tensor-core path (one to a dozen rows in a
+    128-row tile, fewer tiles than SMs at the smallest sizes): every
+    accumulator must still match exactly."""
+    wl0, wts, prep, W = decode_setup
+    wl = dataclasses.replace(wl0, T=T, data_seed=300 + T)
+    try:
+        err, y, y_ref, rt, dbg = run_case(M, wl, wts=wts, W=W, prep=prep, path=M.MOE_PATH_TENSOR)
+        assert np.array_equal(y, y_ref)
+    finally:
+        M.moe_w8a8_set_path(W, M.MOE_PATH_AUTO)
+
+
+@pytest.mark.parametrize("path_name", ["stream", "tensor"])
+def test_activation_clip_at_calibrated_percentile(M, decode_setup, path_name):
+    """Saturating clip of the smoothed activations at the 99.9th percentile of
+    the calibration rows: the percentile computed by the library equals the
+    oracle's order statistic, the clip binds (outlier channels saturate at
+    +-127 and token scales are capped), and every stage still matches the
+    oracle run with the same clip."""
+    import torch
+    wl, wts, prep, W = decode_setup
+    cal = torch.from_numpy(synth.f32_to_bf16_bits(wts.calib_x).view(np.int16)).view(torch.bfloat16).cuda()
+    clip = M.moe_w8a8_calibrate_act_clip(W, cal, 99.9)
+    assert clip == oracle.act_clip_percentile(wts.calib_x, prep.inv_s, 99.9)
+    path = M.MOE_PATH_STREAM if path_name == "stream" else M.MOE_PATH_TENSOR
+    M.moe_w8a8_set_act_clip(W, clip)
+    try:
+        data = synth.make_data(wl)
+        rt = H.oracle_route(wl, data)
+        y, dbg = H.gpu_forward(W, wl, data, path=path)
+        y_ref, odbg = oracle.moe_tokens(data.x, prep, rt, out_bf16=wl.in_bf16, act_clip=clip)
+        H.compare_stages(wl, rt, dbg, y, y_ref, odbg, np.arange(wl.T), bias=data.router_bias)
+        assert np.array_equal(y, y_ref)
+        capped = dbg["sx"] == np.float32(clip) / np.float32(127.0)
+        assert capped.sum() > wl.T // 2
+        assert (np.abs(dbg["xq"][capped].astype(np.int32)) == 127).sum(axis=1).min() >= 2
+    finally:
+        M.moe_w8a8_set_act_clip(W, 0.0)
+        M.moe_w8a8_set_path(W, M.MOE_PATH_AUTO)
+    with pytest.raises(M.MoeError) as e:
+        M.moe_w8a8_set_act_clip(W, -1.0)
+    assert e.value.status == M.MOE_ERR_INVALID_ARG
+
+
 def test_tensor_path_capacity_and_skew(M):
     T, E = 300, 8
     logits = synth.uniform(41, 1, (T, E))

@@ -73,6 +73,56 @@ def test_quant_error_bound_and_full_range():
     assert q[9, 5] == -127 and np.count_nonzero(q[9]) == 1
 
 
+# ----------------------------------------------------------------------------- activation clip
+
+def test_clip_at_or_above_the_range_changes_nothing():
+    x = synth.normal(14, 1, (40, 256), std=2.0)
+    inv_s = synth.uniform(14, 2, (256,)) + np.float32(0.5)
+    q0, s0 = oracle.quantize_tokens(x, inv_s)
+    top = float((np.abs(x * inv_s)).max())
+    for clip in (top, top * 2.0, 1e30):
+        q, s = oracle.quantize_tokens(x, inv_s, act_clip=clip)
+        assert np.array_equal(q, q0) and np.array_equal(s, s0)
+
+
+def test_clip_saturates_beyond_the_cap_and_keeps_half_step_inside():
+    """With the token's range capped at c: the scale is c/127 (one fp32
+    division), values within the cap are within half a step, values beyond it
+    saturate at +-127 with their sign."""
+    x = synth.normal(15, 1, (64, 512), std=1.0)
+    x[:, ::50] *= 40.0                       # outlier channels
+    c = np.float32(3.0)
+    q, s = oracle.quantize_tokens(x, None, act_clip=float(c))
+    for t in range(x.shape[0]):
+        amax = np.float32(np.abs(x[t]).max())
+        cap = min(amax, c)
+        assert s[t] == np.float32(cap) / np.float32(127.0)
+        inside = np.abs(x[t]) <= cap
+        err = np.abs(x[t][inside].astype(np.float64) - q[t][inside].astype(np.float64) * float(s[t]))
+        assert err.max() <= float(s[t]) * (0.5 + 1e-5)
+        beyond = np.abs(x[t]) > cap * np.float32(1.0001)
+        assert np.array_equal(q[t][beyond], np.where(x[t][beyond] > 0, 127, -127).astype(np.int8))
+    # a hand-made token: cap 2 -> scale 2/127, 5 and -9 saturate, 1 -> rint(63.5) = 64
+    row = np.array([[1.0, 5.0, -9.0, 2.0, -2.0, 0.0]], np.float32)
+    q, s = oracle.quantize_tokens(row, None, act_clip=2.0)
+    assert s[0] == np.float32(2.0) / np.float32(127.0)
+    assert q[0].tolist() == [int(np.rint(np.float32(1.0) / s[0])), 127, -127, 127, -127, 0]
+
+
+def test_clip_percentile_is_the_nearest_rank_order_statistic():
+    x = synth.normal(16, 1, (50, 96), std=1.5)
+    inv_s = synth.uniform(16, 2, (96,)) + np.float32(0.25)
+    a = np.sort(np.abs((x * inv_s).astype(np.float32)).ravel())
+    n = a.size
+    for p in (50.0, 99.0, 99.9, 100.0, 1e-9):
+        c = oracle.act_clip_percentile(x, inv_s, p)
+        rank = max(1, min(n, int(np.ceil(p / 100.0 * n))))
+        assert c == a[rank - 1]
+        # the defining property, counted directly
+        assert (a <= c).sum() >= rank and (a < c).sum() < rank
+    assert oracle.act_clip_percentile(x, inv_s, 100.0) == a[-1]
+
+
 # ----------------------------------------------------------------------------- smoothing
 
 def test_smoothing_identity_fp64():

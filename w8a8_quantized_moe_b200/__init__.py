@@ -37,7 +37,7 @@ EXPORTS = (
     "moe_w8a8_check_status", "moe_w8a8_destroy", "moe_status_string",
     "moe_w8a8_last_launch_count", "moe_w8a8_profile_start", "moe_w8a8_profile_read",
     "moe_w8a8_profile_stop", "moe_w8a8_stage_name", "moe_w8a8_forward_noalloc",
-    "moe_w8a8_status_words",
+    "moe_w8a8_status_words", "moe_w8a8_set_act_clip", "moe_w8a8_calibrate_act_clip",
 )
 
 MOE_NOALLOC_SCRATCH_BYTES = 8 << 20
@@ -87,6 +87,8 @@ def lib():
             "moe_w8a8_forward_host": ([vp, vp, i32, vp, vp, vp, vp, sz, vp], i32),
             "moe_w8a8_set_path": ([vp, i32], i32),
             "moe_w8a8_set_stream_threshold": ([vp, i32], i32),
+            "moe_w8a8_set_act_clip": ([vp, ctypes.c_float], i32),
+            "moe_w8a8_calibrate_act_clip": ([vp, vp, i64, i32, ctypes.c_double, vp, vp], i32),
             "moe_w8a8_get_smooth_scales": ([vp, vp], i32),
             "moe_w8a8_export_weights": ([vp, vp, vp, vp, vp, vp, vp, vp, vp], i32),
             "moe_w8a8_check_status": ([vp, vp], i32),
@@ -257,6 +259,20 @@ def moe_w8a8_set_path(w: Weights, path: int):
 def moe_w8a8_set_stream_threshold(w: Weights, max_rows: int):
     _check(lib().moe_w8a8_set_stream_threshold(w.handle, int(max_rows)),
            "moe_w8a8_set_stream_threshold")
+
+
+def moe_w8a8_set_act_clip(w: Weights, clip: float):
+    _check(lib().moe_w8a8_set_act_clip(w.handle, float(clip)), "moe_w8a8_set_act_clip")
+
+
+def moe_w8a8_calibrate_act_clip(w: Weights, x, percent: float, stream=None) -> float:
+    torch = _torch()
+    dt = MOE_BF16 if x.dtype == torch.bfloat16 else MOE_F32
+    out = ctypes.c_float(0.0)
+    _check(lib().moe_w8a8_calibrate_act_clip(w.handle, _dev_ptr(x, name="x"), x.shape[0], dt, float(percent),
+                                             ctypes.byref(out), _stream(stream)),
+           "moe_w8a8_calibrate_act_clip")
+    return float(out.value)
 
 
 def moe_w8a8_get_smooth_scales(w: Weights):

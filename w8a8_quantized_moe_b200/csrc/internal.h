@@ -15,6 +15,7 @@ struct moe_w8a8_weights {
     int num_sms;
     int path;               // MOE_PATH_*
     int stream_max_rows;    // AUTO: streaming path when T*k <= this
+    float act_clip;         // > 0: cap of each token's smoothed range (saturating clip)
     int last_launches;
     // prepared weights (device)
     int8_t* w_gu;     // [E][2f][d]: per 128-channel block, 128 gate rows then 128 up rows
@@ -85,9 +86,13 @@ cudaError_t launch_route_small(const float* logits, const float* bias, int T, in
                                int renorm, int cap, int32_t* idx, float* wts, float* logits_out,
                                int32_t* offsets, int32_t* row2ts, int32_t* ts2row, int32_t* meta,
                                int32_t* active, int32_t* tiles, cudaStream_t s);
-cudaError_t launch_smooth_quant(const void* x, int in_dtype, const float* inv_s, int T, int d,
-                                int k, const int32_t* ts2row, int8_t* xq, float* sx, int8_t* aq,
+// act_clip > 0 caps each token's range (saturating clip), 0 = off.
+cudaError_t launch_smooth_quant(const void* x, int in_dtype, const float* inv_s, float act_clip, int T,
+                                int d, int k, const int32_t* ts2row, int8_t* xq, float* sx, int8_t* aq,
                                 cudaStream_t s);
+// out[r][j] = |fp32(x[r][j] * inv_s[j])| (calibration of the activation clip)
+cudaError_t launch_scaled_abs(const void* x, int64_t rows, int d, int dtype, const float* inv_s, float* out,
+                              cudaStream_t s);
 
 cudaError_t launch_stream_gateup(const moe_w8a8_weights* w, int T, const int8_t* xq,
                                  const int32_t* row2ts, const int32_t* offsets,

@@ -32,6 +32,17 @@ __global__ void calib_absmax_kernel(const void* __restrict__ x, int64_t rows, in
     if (r1 > r0) atomic_max_nonneg(absmax + j, m);
 }
 
+// out[r][j] = |fp32(x[r][j] * inv_s[j])|: the smoothed values the per-token
+// quantiser sees, for the percentile of the activation clip.
+__global__ void scaled_abs_kernel(const void* __restrict__ x, int64_t n, int d, int dtype,
+                                  const float* __restrict__ inv_s, float* __restrict__ out) {
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+        const float v = dtype == MOE_BF16 ? bf16_bits_to_f32(reinterpret_cast<const uint16_t*>(x)[i])
+                                          : reinterpret_cast<const float*>(x)[i];
+        out[i] = fabsf(__fmul_rn(v, inv_s[i % d]));
+    }
+}
+
 // aw[j] = max over experts and output channels of |W_gate[e][j][:]|, |W_up[e][j][:]|
 // (one block per (j, e); rows are f contiguous floats).
 __global__ void gateup_input_absmax_kernel(const float* __restrict__ wg, const float* __restrict__ wu,
@@ -127,6 +138,15 @@ cudaError_t launch_calib_absmax(const void* x, int64_t rows, int d, int dtype, f
     if (rows <= 0) return cudaSuccess;
     dim3 grid((d + 255) / 256, (unsigned)(rows < 64 ? rows : 64));
     calib_absmax_kernel<<<grid, 256, 0, s>>>(x, rows, d, dtype, absmax);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_scaled_abs(const void* x, int64_t rows, int d, int dtype, const float* inv_s, float* out,
+                              cudaStream_t s) {
+    const int64_t n = rows * d;
+    if (n <= 0) return cudaSuccess;
+    const int64_t blocks = (n + 255) / 256;
+    scaled_abs_kernel<<<(unsigned)(blocks < 4096 ? blocks : 4096), 256, 0, s>>>(x, n, d, dtype, inv_s, out);
     return cudaGetLastError();
 }
 

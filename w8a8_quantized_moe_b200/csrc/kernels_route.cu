@@ -515,8 +515,8 @@ constexpr int kSqThreads = 128;
 
 template <int kSqMaxGroups>   // groups of 8 channels per thread: d <= 128 x 8 x kSqMaxGroups
 __global__ void __launch_bounds__(kSqThreads) smooth_quant_kernel(
-    const void* __restrict__ x, int in_dtype, const float* __restrict__ inv_s, int T, int d, int k,
-    const int32_t* __restrict__ ts2row, int8_t* __restrict__ xq, float* __restrict__ sx,
+    const void* __restrict__ x, int in_dtype, const float* __restrict__ inv_s, float act_clip, int T, int d,
+    int k, const int32_t* __restrict__ ts2row, int8_t* __restrict__ xq, float* __restrict__ sx,
     int8_t* __restrict__ aq) {
     pdl_wait();
     pdl_trigger();
@@ -550,6 +550,7 @@ __global__ void __launch_bounds__(kSqThreads) smooth_quant_kernel(
     __syncthreads();
 #pragma unroll
     for (int w = 0; w < kSqThreads / 32; ++w) m = fmaxf(m, red[w]);
+    if (act_clip > 0.0f) m = fminf(m, act_clip);   // saturating clip: values beyond it go to +-127
     const float s = m > 0.0f ? __fdiv_rn(m, 127.0f) : 0.0f;
     const float rs = s > 0.0f ? __frcp_rn(s) : 0.0f;
     if (tid == 0) sx[t] = s;
@@ -632,12 +633,13 @@ cudaError_t launch_route_small(const float* logits, const float* bias, int T, in
                       active, tiles);
 }
 
-cudaError_t launch_smooth_quant(const void* x, int in_dtype, const float* inv_s, int T, int d,
-                                int k, const int32_t* ts2row, int8_t* xq, float* sx, int8_t* aq,
+cudaError_t launch_smooth_quant(const void* x, int in_dtype, const float* inv_s, float act_clip, int T,
+                                int d, int k, const int32_t* ts2row, int8_t* xq, float* sx, int8_t* aq,
                                 cudaStream_t s) {
     const int groups = (d / 8 + kSqThreads - 1) / kSqThreads;
     auto kern = groups <= 4 ? smooth_quant_kernel<4> : groups <= 8 ? smooth_quant_kernel<8> : smooth_quant_kernel<16>;
-    return launch_pdl(kern, dim3(T), dim3(kSqThreads), 0, s, x, in_dtype, inv_s, T, d, k, ts2row, xq, sx, aq);
+    return launch_pdl(kern, dim3(T), dim3(kSqThreads), 0, s, x, in_dtype, inv_s, act_clip, T, d, k, ts2row, xq,
+                      sx, aq);
 }
 
 }  // namespace moe

@@ -3,6 +3,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdlib>
 #include <cstring>
@@ -296,7 +297,7 @@ static moe_status forward_impl(const moe_w8a8_weights* w, const void* x, int T, 
     }
     if (path == MOE_PATH_STREAM) {
         mark(MOE_STAGE_QUANT, 0);
-        CUDA_TRY(launch_smooth_quant(x, c.in_dtype, w->inv_s, T, d, k, ts2row, xq, sx, nullptr, s));
+        CUDA_TRY(launch_smooth_quant(x, c.in_dtype, w->inv_s, w->act_clip, T, d, k, ts2row, xq, sx, nullptr, s));
         mark(MOE_STAGE_QUANT, 1);
         int32_t* acc1 = (int32_t*)P(L.acc1);
         mark(MOE_STAGE_GEMM1, 0);
@@ -315,7 +316,7 @@ static moe_status forward_impl(const moe_w8a8_weights* w, const void* x, int T, 
     } else {
         int8_t* aq = (int8_t*)P(L.aq);
         mark(MOE_STAGE_QUANT, 0);
-        CUDA_TRY(launch_smooth_quant(x, c.in_dtype, w->inv_s, T, d, k, ts2row, xq, sx, aq, s));
+        CUDA_TRY(launch_smooth_quant(x, c.in_dtype, w->inv_s, w->act_clip, T, d, k, ts2row, xq, sx, aq, s));
         mark(MOE_STAGE_QUANT, 1);
         mark(MOE_STAGE_GEMM1, 0);
         CUDA_TRY(launch_tc_gemm1(w, T, aq, meta, tiles, offsets, row2ts, sx, (float*)P(L.h32),
@@ -411,6 +412,37 @@ moe_status moe_w8a8_set_path(moe_w8a8_weights* w, int32_t path) {
 moe_status moe_w8a8_set_stream_threshold(moe_w8a8_weights* w, int32_t max_rows) {
     if (!w || max_rows < 0) return MOE_ERR_INVALID_ARG;
     w->stream_max_rows = max_rows;
+    return MOE_OK;
+}
+
+moe_status moe_w8a8_set_act_clip(moe_w8a8_weights* w, float clip) {
+    if (!w || !(clip >= 0.0f) || !std::isfinite(clip)) return MOE_ERR_INVALID_ARG;
+    w->act_clip = clip;
+    return MOE_OK;
+}
+
+moe_status moe_w8a8_calibrate_act_clip(const moe_w8a8_weights* w, const void* x, int64_t rows,
+                                       int32_t dtype, double percent, float* clip_host,
+                                       moe_stream_t stream) {
+    if (!w || !clip_host || rows <= 0 || !x) return MOE_ERR_INVALID_ARG;
+    if (dtype != MOE_F32 && dtype != MOE_BF16) return MOE_ERR_INVALID_ARG;
+    if (!(percent > 0.0 && percent <= 100.0)) return MOE_ERR_INVALID_ARG;
+    const int d = w->cfg.d;
+    const int64_t n = rows * d;
+    cudaStream_t s = (cudaStream_t)stream;
+    float* dev = nullptr;
+    if (cudaMalloc(&dev, (size_t)n * 4) != cudaSuccess) return MOE_ERR_OOM;
+    std::vector<float> a((size_t)n);
+    cudaError_t err = launch_scaled_abs(x, rows, d, dtype, w->inv_s, dev, s);
+    if (err == cudaSuccess) err = cudaMemcpyAsync(a.data(), dev, (size_t)n * 4, cudaMemcpyDeviceToHost, s);
+    if (err == cudaSuccess) err = cudaStreamSynchronize(s);
+    cudaFree(dev);
+    if (err != cudaSuccess) return MOE_ERR_CUDA;
+    // nearest rank: the ceil(percent/100 * n)-th smallest value
+    int64_t rank = (int64_t)std::ceil(percent / 100.0 * (double)n);
+    rank = std::min<int64_t>(std::max<int64_t>(rank, 1), n);
+    std::nth_element(a.begin(), a.begin() + (rank - 1), a.end());
+    *clip_host = a[(size_t)(rank - 1)];
     return MOE_OK;
 }
 
