@@ -60,6 +60,8 @@ def parse():
                         "per point and expert path (not the headline line)")
     p.add_argument("--tokens", type=int, default=0,
                    help="override the workload's token count T (same layer, same seeds)")
+    p.add_argument("--format", choices=["int8", "e4m3"], default="int8",
+                   help="expert number format: INT8 (the pages' W8A8) or FP8 E4M3")
     p.add_argument("--act-clip", type=float, default=0.0, metavar="PERCENT",
                    help="saturating activation clip at this percentile of the smoothed calibration "
                         "activations (0: off)")
@@ -218,7 +220,10 @@ def oracle_step(wl, prep, data):
     t0 = time.perf_counter()
     rt = oracle.route(data.x, wl.k, wl.E, w_router=data.w_router, logits=data.router_logits,
                       bias=data.router_bias, capacity_factor=wl.capacity_factor)
-    oracle.moe_tokens(data.x, prep, rt, out_bf16=wl.in_bf16, debug=False)
+    if prep.wq_gate.dtype == np.uint8:     # E4M3 experts
+        oracle.moe_tokens_fp8(data.x, prep, rt, out_bf16=wl.in_bf16, debug=False)
+    else:
+        oracle.moe_tokens(data.x, prep, rt, out_bf16=wl.in_bf16, debug=False)
     return time.perf_counter() - t0
 
 
@@ -238,7 +243,8 @@ def run_reference(args, world, rank):
     import oracle
     wl = synth.WORKLOADS[args.workload]
     wts = synth.make_weights(wl)
-    prep = oracle.prepare(wts.w_gate, wts.w_up, wts.w_down, wts.calib_x, wl.alpha)
+    prepare = oracle.prepare_fp8 if args.format == "e4m3" else oracle.prepare
+    prep = prepare(wts.w_gate, wts.w_up, wts.w_down, wts.calib_x, wl.alpha)
     n_tok = oracle_sample_size(wl, prep, 120.0, args.steps + args.warmup)
     data = synth.make_data(wl, T=n_tok)
     for _ in range(args.warmup):
@@ -250,7 +256,7 @@ def run_reference(args, world, rank):
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": 1e3 * secs / args.steps, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "int8", "data": "synthetic",
+            "vs_baseline": None, "dtype": "e4m3" if args.format == "e4m3" else "int8", "data": "synthetic",
             "config": {"workload": describe(wl), "parallelism": "single CPU thread"},
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
                              "sample": sample},
@@ -273,9 +279,11 @@ def measure(args, wl, world, rank, local, e2e_on=True, wts=None):
     if wts is None and not streamed:
         wts = synth.make_weights(wl)
     data = synth.make_data(wl)
+    fp8 = getattr(args, "format", "int8") == "e4m3"
     cfg = M.make_config(wl.d, wl.f, wl.E, wl.k, wl.alpha, wl.capacity_factor, True,
                         M.MOE_BF16 if wl.in_bf16 else M.MOE_F32,
-                        M.MOE_BF16 if wl.in_bf16 else M.MOE_F32)
+                        M.MOE_BF16 if wl.in_bf16 else M.MOE_F32,
+                        M.MOE_FMT_E4M3 if fp8 else M.MOE_FMT_INT8)
     act = torch.bfloat16 if wl.in_bf16 else torch.float32
 
     def to_act(v32):
@@ -326,7 +334,7 @@ def measure(args, wl, world, rank, local, e2e_on=True, wts=None):
     M.moe_w8a8_forward(W, x, T, bias, logits, y, ws, {"offsets": offs})
     counts = np.diff(offs.cpu().numpy())
     n_active, R = int((counts > 0).sum()), int(counts.sum())
-    tensor = args.path == "tensor" or (args.path == "auto" and T * wl.k > 32)
+    tensor = args.path == "tensor" or (args.path == "auto" and (fp8 or T * wl.k > 32))
     alg = algorithmic(wl, n_active, R, tensor)
 
     stream = torch.cuda.current_stream(dev)
@@ -553,7 +561,8 @@ def run_ours(args, world, rank, local):
                          "device expert by expert, and the oracle would need all of them on the host"}
     elif world == 1 and not args.no_cpu_baseline:
         import oracle
-        prep = oracle.prepare(wts.w_gate, wts.w_up, wts.w_down, wts.calib_x, wl.alpha)
+        prepare = oracle.prepare_fp8 if args.format == "e4m3" else oracle.prepare
+        prep = prepare(wts.w_gate, wts.w_up, wts.w_down, wts.calib_x, wl.alpha)
         n_tok = min(wl.T, 32)
         sdata = synth.make_data(wl, T=n_tok)
         secs, n = 0.0, 0
@@ -566,7 +575,8 @@ def run_ours(args, world, rank, local):
 
     line = {"metric": METRIC, "value": res["value"], "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": res["ms_per_step"],
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8",
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "e4m3" if args.format == "e4m3" else "int8",
             "data": "synthetic", "config": res["config"], "roofline": res["roofline"],
             "stages_ms": res["stages_ms"], "e2e": res["e2e"], "gpu_launches": res["gpu_launches"],
             "clocks": res["clocks"], "cpu_baseline": cpu}

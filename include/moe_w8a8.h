@@ -63,9 +63,23 @@ typedef enum {
 
 enum { MOE_F32 = 0, MOE_BF16 = 1 };
 
+/* Number format of the expert weights, the quantised activations and h
+ * (ruibaoantu.com "Day0 adaptation" page, section 1: expert layers in INT8 or
+ * FP8, activations on the same precision path as the weights).
+ *   MOE_FMT_INT8: symmetric INT8, scale = amax / 127, codes rint(v / scale)
+ *                 clamped to +-127; INT32 accumulation (exact).
+ *   MOE_FMT_E4M3: FP8 E4M3 (finite-only OCP format, largest 448), scale =
+ *                 amax / 448, codes = nearest E4M3 of v / scale (ties to even,
+ *                 saturating); fp32 accumulation in the tensor cores, so the
+ *                 accumulators are not reproducible bit for bit across
+ *                 summation orders.  Tensor-core path only (MOE_PATH_STREAM is
+ *                 refused; MOE_PATH_AUTO picks the tensor path). */
+enum { MOE_FMT_INT8 = 0, MOE_FMT_E4M3 = 1 };
+
 /* Expert GEMM path: AUTO picks STREAM for small row counts (weight-bandwidth
  * bound: each active expert's INT8 weights are read once with 128-bit loads)
- * and TENSOR otherwise (tcgen05 kind::i8 grouped GEMMs). */
+ * and TENSOR otherwise (tcgen05 kind::i8 grouped GEMMs; kind::f8f6f4 for E4M3
+ * experts, which always take the TENSOR path). */
 enum { MOE_PATH_AUTO = 0, MOE_PATH_STREAM = 1, MOE_PATH_TENSOR = 2 };
 
 typedef struct {
@@ -78,6 +92,7 @@ typedef struct {
     int32_t renormalize;      /* 1: softmax over the k selected logits; 0: over all E          */
     int32_t in_dtype;         /* MOE_F32 or MOE_BF16: X                                       */
     int32_t out_dtype;        /* MOE_F32 or MOE_BF16: Y                                       */
+    int32_t expert_format;    /* MOE_FMT_INT8 (0) or MOE_FMT_E4M3 (1)                         */
 } moe_w8a8_config;
 
 typedef struct moe_w8a8_weights moe_w8a8_weights; /* opaque, library-owned */

@@ -62,6 +62,19 @@ def lib():
             "oracle_round_bf16": ([f32], f32),
             "oracle_moe_tokens": ([vp, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp, vp, f32, vp, vp,
                                    vp, vp, i64, i32, vp, vp, vp, vp, vp, vp, vp, vp], None),
+            "oracle_e4m3_round": ([f32], f32),
+            "oracle_e4m3_encode": ([f32], ctypes.c_uint8),
+            "oracle_e4m3_decode": ([ctypes.c_uint8], f32),
+            "oracle_e4m3_encode_array": ([vp, i64, vp], None),
+            "oracle_e4m3_decode_array": ([vp, i64, vp], None),
+            "oracle_quantize_rows_fp8": ([vp, i64, i64, vp, vp], None),
+            "oracle_quantize_gateup_expert_fp8": ([vp, vp, i32, i32, vp, vp], None),
+            "oracle_quantize_down_expert_fp8": ([vp, i32, i32, vp, vp], None),
+            "oracle_quantize_tokens_fp8": ([vp, vp, i64, i32, f32, vp, vp], None),
+            "oracle_gemm_fp8": ([vp, vp, i64, i64, i64, vp], None),
+            "oracle_swiglu_requant_fp8": ([vp, vp, f32, vp, vp, i32, vp, vp, vp], None),
+            "oracle_moe_tokens_fp8": ([vp, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp, vp, f32, vp, vp,
+                                       vp, vp, i64, i32, vp, vp, vp, vp, vp, vp, vp, vp], None),
         }
         for name, (args, res) in sig.items():
             fn = getattr(L, name)
@@ -312,4 +325,108 @@ def moe_tokens(x, prep: Prepared, rt: Routing, tokens=None, out_bf16=False, debu
                             float(act_clip), P(rt.idx), P(rt.w), P(_c(rt.ts2row, np.int32)), P(tok), n,
                             1 if out_bf16 else 0, P(y), P(g("xq")), P(g("sx")), P(g("acc1")),
                             P(g("hq")), P(g("sh")), P(g("acc2")), P(g("o")))
+    return y, dbg
+
+
+# ------------------------------------------------------------------ FP8 (E4M3) experts
+
+def e4m3_encode(v) -> np.ndarray:
+    """E4M3 codes (uint8) of fp32 values: nearest, ties to even, saturating at 448."""
+    v = _c(np.atleast_1d(v), np.float32)
+    q = np.empty(v.shape, dtype=np.uint8)
+    lib().oracle_e4m3_encode_array(P(v), v.size, P(q))
+    return q
+
+
+def e4m3_decode(q) -> np.ndarray:
+    q = _c(np.atleast_1d(q), np.uint8)
+    v = np.empty(q.shape, dtype=np.float32)
+    lib().oracle_e4m3_decode_array(P(q), q.size, P(v))
+    return v
+
+
+def quantize_rows_fp8(v) -> tuple[np.ndarray, np.ndarray]:
+    v = _c(v, np.float32)
+    v2 = v.reshape(-1, v.shape[-1])
+    q = np.empty(v2.shape, dtype=np.uint8)
+    s = np.empty(v2.shape[0], dtype=np.float32)
+    lib().oracle_quantize_rows_fp8(P(v2), v2.shape[0], v2.shape[1], P(q), P(s))
+    return q.reshape(v.shape), s.reshape(v.shape[:-1])
+
+
+def quantize_tokens_fp8(x, inv_s, act_clip: float = 0.0):
+    x = _c(x, np.float32)
+    T, d = x.shape
+    q = np.empty((T, d), dtype=np.uint8)
+    sx = np.empty(T, dtype=np.float32)
+    lib().oracle_quantize_tokens_fp8(P(x), P(_c(inv_s, np.float32)), T, d, float(act_clip), P(q), P(sx))
+    return q, sx
+
+
+def gemm_fp8(a, b) -> np.ndarray:
+    a, b = _c(a, np.uint8), _c(b, np.uint8)
+    M, K = a.shape
+    N = b.shape[0]
+    c = np.empty((M, N), dtype=np.float32)
+    lib().oracle_gemm_fp8(P(a), P(b), M, N, K, P(c))
+    return c
+
+
+def swiglu_requant_fp8(acc_g, acc_u, sx: float, sw_g, sw_u):
+    acc_g, acc_u = _c(acc_g, np.float32), _c(acc_u, np.float32)
+    f = acc_g.size
+    h = np.empty(f, dtype=np.float32)
+    hq = np.empty(f, dtype=np.uint8)
+    sh = np.empty(1, dtype=np.float32)
+    lib().oracle_swiglu_requant_fp8(P(acc_g), P(acc_u), sx, P(_c(sw_g, np.float32)),
+                                    P(_c(sw_u, np.float32)), f, P(h), P(hq), P(sh))
+    return h, hq, float(sh[0])
+
+
+def prepare_fp8(w_gate, w_up, w_down, calib_x, alpha: float, smooth: bool = True) -> Prepared:
+    """As prepare(), with E4M3 weight codes (uint8) and amax/448 scales."""
+    E, d, f = w_gate.shape
+    ax = channel_absmax(calib_x)
+    aw = gateup_input_absmax(w_gate, w_up)
+    s, inv_s = smooth_scales(ax, aw, alpha) if smooth else (None, None)
+    wq_gate = np.empty((E, f, d), dtype=np.uint8)
+    wq_up = np.empty((E, f, d), dtype=np.uint8)
+    sw_gate = np.empty((E, f), dtype=np.float32)
+    sw_up = np.empty((E, f), dtype=np.float32)
+    wq_down = np.empty((E, d, f), dtype=np.uint8)
+    sw_down = np.empty((E, d), dtype=np.float32)
+    L = lib()
+    for e in range(E):
+        for src, q, sw in ((w_gate[e], wq_gate[e], sw_gate[e]), (w_up[e], wq_up[e], sw_up[e])):
+            src = _c(src, np.float32)
+            L.oracle_quantize_gateup_expert_fp8(P(src), P(_c(s, np.float32)), d, f, P(q), P(sw))
+        src = _c(w_down[e], np.float32)
+        L.oracle_quantize_down_expert_fp8(P(src), f, d, P(wq_down[e]), P(sw_down[e]))
+    if not smooth:
+        s = np.ones(d, dtype=np.float32)
+    return Prepared(ax, aw, s, inv_s, wq_gate, wq_up, sw_gate, sw_up, wq_down, sw_down)
+
+
+def moe_tokens_fp8(x, prep: Prepared, rt: Routing, tokens=None, out_bf16=False, debug=True,
+                   act_clip: float = 0.0):
+    """Expert FFN + combine with E4M3 experts for the listed tokens (all by default)."""
+    x = _c(x, np.float32)
+    T, d = x.shape
+    E, f, _ = prep.wq_gate.shape
+    k = rt.idx.shape[1]
+    tok = np.arange(T, dtype=np.int64) if tokens is None else _c(tokens, np.int64)
+    n = tok.size
+    y = np.empty((n, d), dtype=np.float32)
+    dbg = {}
+    if debug:
+        dbg = dict(xq=np.empty((n, d), np.uint8), sx=np.empty(n, np.float32),
+                   acc1=np.zeros((n, k, 2 * f), np.float32), hq=np.zeros((n, k, f), np.uint8),
+                   sh=np.zeros((n, k), np.float32), acc2=np.zeros((n, k, d), np.float32),
+                   o=np.zeros((n, k, d), np.float32))
+    g = dbg.get
+    lib().oracle_moe_tokens_fp8(P(x), d, f, E, k, P(prep.wq_gate), P(prep.wq_up), P(prep.sw_gate),
+                                P(prep.sw_up), P(prep.wq_down), P(prep.sw_down), P(prep.inv_s),
+                                float(act_clip), P(rt.idx), P(rt.w), P(_c(rt.ts2row, np.int32)), P(tok), n,
+                                1 if out_bf16 else 0, P(y), P(g("xq")), P(g("sx")), P(g("acc1")),
+                                P(g("hq")), P(g("sh")), P(g("acc2")), P(g("o")))
     return y, dbg

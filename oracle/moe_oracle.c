@@ -479,3 +479,207 @@ void oracle_moe_tokens(const float* x, int32_t d, int32_t f, int32_t E, int32_t 
     }
     free(xq); free(acc_g); free(acc_u); free(hq); free(acc2); free(o);
 }
+
+/* ======================================================================== */
+/* FP8 (E4M3) experts ([Day0 adaptation] section 1: expert layers stored in  */
+/* FP8 or INT8, with the activations kept on the same precision path as the  */
+/* weights; the deployment config names FP8 experts).                        */
+/* ======================================================================== */
+
+/*
+ * E4M3, the finite-only 8-bit float of the OCP FP8 formats: 1 sign bit, 4
+ * exponent bits (bias 7), 3 mantissa bits, no infinities; exponent 1111 with
+ * mantissa 111 is NaN, so the largest finite magnitude is 1.75 * 2^8 = 448.
+ * Normal values (8 + m) 2^(e-10) for e = 1..15, subnormals m 2^-9.
+ * READING: rounding is to the nearest representable value, ties to the even
+ * code; magnitudes beyond 448 saturate to 448 (a finite input never becomes
+ * NaN); the sign is kept, so tiny negative values give -0 (code 0x80).
+ */
+
+/* Spacing of E4M3 values in the binade of a (0 < a < 448). */
+static float e4m3_step(float a) {
+    int e;
+    frexpf(a, &e);            /* a = m 2^e, m in [0.5, 1): binade 2^(e-1) */
+    int be = e - 1;
+    if (be < -6) be = -6;     /* the subnormals share the lowest binade's spacing */
+    return ldexpf(1.0f, be - 3);
+}
+
+/* The E4M3 value nearest to v (as a float). */
+float oracle_e4m3_round(float v) {
+    float a = fabsf(v);
+    float r;
+    if (a >= 448.0f) {
+        r = 448.0f;
+    } else if (a == 0.0f) {
+        r = 0.0f;
+    } else {
+        const float q = e4m3_step(a);
+        r = rintf(a / q) * q;  /* a / q is exact (q is a power of two) */
+        if (r > 448.0f) r = 448.0f;
+    }
+    return signbit(v) ? -r : r;
+}
+
+uint8_t oracle_e4m3_encode(float v) {
+    const float r = fabsf(oracle_e4m3_round(v));
+    const uint8_t s = signbit(v) ? 0x80 : 0x00;
+    if (r == 0.0f) return s;
+    int e;
+    frexpf(r, &e);
+    const int be = e - 1;
+    if (be < -6) return (uint8_t)(s | (int)(r / ldexpf(1.0f, -9)));          /* subnormal */
+    const int m = (int)(r / ldexpf(1.0f, be - 3)) - 8;
+    return (uint8_t)(s | ((be + 7) << 3) | m);
+}
+
+float oracle_e4m3_decode(uint8_t c) {
+    const int s = c >> 7, e = (c >> 3) & 15, m = c & 7;
+    float a;
+    if (e == 15 && m == 7) a = NAN;
+    else if (e == 0) a = ldexpf((float)m, -9);
+    else a = ldexpf((float)(8 + m), e - 10);
+    return s ? -a : a;
+}
+
+void oracle_e4m3_encode_array(const float* v, int64_t n, uint8_t* q) {
+    for (int64_t i = 0; i < n; ++i) q[i] = oracle_e4m3_encode(v[i]);
+}
+
+void oracle_e4m3_decode_array(const uint8_t* q, int64_t n, float* v) {
+    for (int64_t i = 0; i < n; ++i) v[i] = oracle_e4m3_decode(q[i]);
+}
+
+/* Scaled E4M3 quantisation of one vector (the FP8 counterpart of the INT8   */
+/* rule): scale = amax / 448 (fp32 division), q = e4m3(v / scale); amax == 0 */
+/* gives scale 0 and codes 0; clip > 0 caps amax as in the INT8 rule.        */
+static float quant_vector_fp8(const float* v, int64_t n, int64_t stride, uint8_t* q, float clip) {
+    float amax = 0.0f;
+    for (int64_t i = 0; i < n; ++i) amax = fmaxf(amax, fabsf(v[i * stride]));
+    if (clip > 0.0f && amax > clip) amax = clip;
+    if (amax == 0.0f) {
+        memset(q, 0, (size_t)n);
+        return 0.0f;
+    }
+    const float scale = amax / 448.0f;
+    for (int64_t i = 0; i < n; ++i) q[i] = oracle_e4m3_encode(v[i * stride] / scale);
+    return scale;
+}
+
+void oracle_quantize_rows_fp8(const float* v, int64_t rows, int64_t n, uint8_t* q, float* scale) {
+    for (int64_t r = 0; r < rows; ++r) scale[r] = quant_vector_fp8(v + r * n, n, 1, q + r * n, 0.0f);
+}
+
+/* Expert weights in E4M3, per output channel, as the INT8 quantisers above:  */
+/* gate/up from w [d][f] with the smoothing fold (q [f][d]), down from        */
+/* w [f][d] without it (q [d][f]).                                            */
+void oracle_quantize_gateup_expert_fp8(const float* w, const float* s, int32_t d, int32_t f, uint8_t* q,
+                                       float* sw) {
+    float* col = (float*)malloc(sizeof(float) * (size_t)d);
+    for (int32_t n = 0; n < f; ++n) {
+        for (int32_t j = 0; j < d; ++j) col[j] = s ? s[j] * w[(int64_t)j * f + n] : w[(int64_t)j * f + n];
+        sw[n] = quant_vector_fp8(col, d, 1, q + (int64_t)n * d, 0.0f);
+    }
+    free(col);
+}
+
+void oracle_quantize_down_expert_fp8(const float* w, int32_t f, int32_t d, uint8_t* q, float* sw) {
+    for (int32_t n = 0; n < d; ++n) sw[n] = quant_vector_fp8(w + n, f, d, q + (int64_t)n * f, 0.0f);
+}
+
+void oracle_quantize_tokens_fp8(const float* x, const float* inv_s, int64_t T, int32_t d, float act_clip,
+                                uint8_t* q, float* sx) {
+    float* xs = (float*)malloc(sizeof(float) * (size_t)d);
+    for (int64_t t = 0; t < T; ++t) {
+        for (int32_t j = 0; j < d; ++j) xs[j] = inv_s ? x[t * d + j] * inv_s[j] : x[t * d + j];
+        sx[t] = quant_vector_fp8(xs, d, 1, q + t * d, act_clip);
+    }
+    free(xs);
+}
+
+/* E4M3 x E4M3 GEMM, c[m][n] = sum_k a[m][k] b[n][k], computed exactly and  */
+/* rounded once to fp32.  Exact in fp64: every product of two E4M3 values is */
+/* a multiple of 2^-18 below 2^18, so a sum of up to 2^16 of them needs at   */
+/* most 52 significant bits.                                                 */
+void oracle_gemm_fp8(const uint8_t* a, const uint8_t* b, int64_t M, int64_t N, int64_t K, float* c) {
+    double lut[256];
+    for (int i = 0; i < 256; ++i) lut[i] = (double)oracle_e4m3_decode((uint8_t)i);
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t n = 0; n < N; ++n) {
+            double acc = 0.0;
+            const uint8_t* ar = a + m * K;
+            const uint8_t* br = b + n * K;
+            for (int64_t kk = 0; kk < K; ++kk) acc += lut[ar[kk]] * lut[br[kk]];
+            c[m * N + n] = (float)acc;
+        }
+}
+
+/* SwiGLU on the fp32 accumulators of the FP8 path, then E4M3 per row. */
+void oracle_swiglu_requant_fp8(const float* acc_g, const float* acc_u, float sx, const float* sw_g,
+                               const float* sw_u, int32_t f, float* h_out, uint8_t* hq, float* sh) {
+    float* h = (float*)malloc(sizeof(float) * (size_t)f);
+    for (int32_t n = 0; n < f; ++n) {
+        float g = (acc_g[n] * sx) * sw_g[n];
+        float u = (acc_u[n] * sx) * sw_u[n];
+        float silu = g / (1.0f + oracle_expf(-g));
+        h[n] = silu * u;
+    }
+    if (h_out) memcpy(h_out, h, sizeof(float) * (size_t)f);
+    *sh = quant_vector_fp8(h, f, 1, hq, 0.0f);
+    free(h);
+}
+
+/* The whole layer with FP8 experts: as oracle_moe_tokens, with E4M3 codes   */
+/* (uint8) for weights, tokens and h, and fp32 accumulators.                 */
+void oracle_moe_tokens_fp8(const float* x, int32_t d, int32_t f, int32_t E, int32_t k,
+                           const uint8_t* wq_gate, const uint8_t* wq_up, const float* sw_gate,
+                           const float* sw_up, const uint8_t* wq_down, const float* sw_down,
+                           const float* inv_s, float act_clip, const int32_t* idx, const float* w,
+                           const int32_t* ts2row, const int64_t* tok, int64_t n_sel, int32_t out_bf16,
+                           float* y, uint8_t* xq_out, float* sx_out, float* acc1_out, uint8_t* hq_out,
+                           float* sh_out, float* acc2_out, float* o_out) {
+    (void)E;
+    uint8_t* xq = (uint8_t*)malloc((size_t)d);
+    float* acc_g = (float*)malloc(sizeof(float) * (size_t)f);
+    float* acc_u = (float*)malloc(sizeof(float) * (size_t)f);
+    uint8_t* hq = (uint8_t*)malloc((size_t)f);
+    float* acc2 = (float*)malloc(sizeof(float) * (size_t)d);
+    float* o = (float*)malloc(sizeof(float) * (size_t)d);
+    for (int64_t i = 0; i < n_sel; ++i) {
+        const int64_t t = tok[i];
+        float sx;
+        oracle_quantize_tokens_fp8(x + t * d, inv_s, 1, d, act_clip, xq, &sx);
+        if (xq_out) memcpy(xq_out + i * d, xq, (size_t)d);
+        if (sx_out) sx_out[i] = sx;
+        float* yt = y + i * d;
+        for (int32_t n = 0; n < d; ++n) yt[n] = 0.0f;
+        for (int32_t s = 0; s < k; ++s) {
+            const int64_t ts = t * k + s;
+            const int32_t e = idx[ts];
+            const int64_t dbg = i * k + s;
+            if (ts2row[ts] < 0) {
+                if (sh_out) sh_out[dbg] = 0.0f;
+                continue;
+            }
+            oracle_gemm_fp8(xq, wq_gate + (int64_t)e * f * d, 1, f, d, acc_g);
+            oracle_gemm_fp8(xq, wq_up + (int64_t)e * f * d, 1, f, d, acc_u);
+            float sh;
+            oracle_swiglu_requant_fp8(acc_g, acc_u, sx, sw_gate + (int64_t)e * f, sw_up + (int64_t)e * f, f,
+                                      NULL, hq, &sh);
+            oracle_gemm_fp8(hq, wq_down + (int64_t)e * d * f, 1, d, f, acc2);
+            for (int32_t n = 0; n < d; ++n) o[n] = ((acc2[n] * sh) * sw_down[(int64_t)e * d + n]) * w[ts];
+            for (int32_t n = 0; n < d; ++n) yt[n] = yt[n] + o[n];
+            if (acc1_out) {
+                memcpy(acc1_out + dbg * 2 * f, acc_g, sizeof(float) * (size_t)f);
+                memcpy(acc1_out + dbg * 2 * f + f, acc_u, sizeof(float) * (size_t)f);
+            }
+            if (hq_out) memcpy(hq_out + dbg * f, hq, (size_t)f);
+            if (sh_out) sh_out[dbg] = sh;
+            if (acc2_out) memcpy(acc2_out + dbg * d, acc2, sizeof(float) * (size_t)d);
+            if (o_out) memcpy(o_out + dbg * d, o, sizeof(float) * (size_t)d);
+        }
+        if (out_bf16)
+            for (int32_t n = 0; n < d; ++n) yt[n] = oracle_round_bf16(yt[n]);
+    }
+    free(xq); free(acc_g); free(acc_u); free(hq); free(acc2); free(o);
+}

@@ -47,14 +47,15 @@ def x_tensor(wl: synth.Workload, data: synth.LayerData):
     return to_dev(data.x)
 
 
-def gpu_prepare(wl: synth.Workload, wts: synth.LayerWeights, capacity_factor=None, renormalize=True):
-    """Calibration absmax + prepare through the C ABI."""
+def gpu_prepare(wl: synth.Workload, wts: synth.LayerWeights, capacity_factor=None, renormalize=True,
+                fmt=0):
+    """Calibration absmax + prepare through the C ABI (fmt: MOE_FMT_INT8 / MOE_FMT_E4M3)."""
     import w8a8_quantized_moe_b200 as M
     torch = torch_mod()
     cfg = M.make_config(wl.d, wl.f, wl.E, wl.k, wl.alpha,
                         wl.capacity_factor if capacity_factor is None else capacity_factor,
                         renormalize, M.MOE_BF16 if wl.in_bf16 else M.MOE_F32,
-                        M.MOE_BF16 if wl.in_bf16 else M.MOE_F32)
+                        M.MOE_BF16 if wl.in_bf16 else M.MOE_F32, fmt)
     calib = synth.f32_to_bf16_bits(wts.calib_x) if wl.in_bf16 else wts.calib_x
     if wl.in_bf16:
         cal = torch.from_numpy(calib.view(np.int16)).view(torch.bfloat16).cuda()
@@ -115,7 +116,9 @@ def gpu_forward(W, wl: synth.Workload, data: synth.LayerData, debug=True, path=N
 
 # ------------------------------------------------------------------ oracle side
 
-def oracle_prepare(wl: synth.Workload, wts: synth.LayerWeights) -> oracle.Prepared:
+def oracle_prepare(wl: synth.Workload, wts: synth.LayerWeights, fmt=0) -> oracle.Prepared:
+    if fmt == 1:
+        return oracle.prepare_fp8(wts.w_gate, wts.w_up, wts.w_down, wts.calib_x, wl.alpha)
     return oracle.prepare(wts.w_gate, wts.w_up, wts.w_down, wts.calib_x, wl.alpha)
 
 
@@ -131,6 +134,8 @@ def oracle_route(wl: synth.Workload, data: synth.LayerData, capacity_factor=None
 def compare_prepare(W, prep: oracle.Prepared):
     import w8a8_quantized_moe_b200 as M
     g = {k: v.cpu().numpy() for k, v in M.moe_w8a8_export_weights(W).items()}
+    if prep.wq_gate.dtype == np.uint8:           # E4M3 codes travel in the same byte buffers
+        g = {k: (v.view(np.uint8) if v.dtype == np.int8 else v) for k, v in g.items()}
     s = M.moe_w8a8_get_smooth_scales(W)
     assert np.array_equal(s, prep.s), "smoothing scales differ"
     assert np.array_equal(g["inv_s"], prep.inv_s), "inverse smoothing scales differ"

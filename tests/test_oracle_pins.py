@@ -425,3 +425,111 @@ def test_moe_vs_unquantised_fp64_sanity():
             ref[t] += rt.w[t, s] * ((g / (1 + np.exp(-g)) * u) @ wts.w_down[e].astype(np.float64))
     rel = np.linalg.norm(y - ref) / np.linalg.norm(ref)
     assert rel < 5e-2, rel
+
+
+# ----------------------------------------------------------------------------- FP8 (E4M3)
+
+def _e4m3_table():
+    """All finite non-negative E4M3 values by code, from the format definition
+    (bias 7, 3 mantissa bits, subnormals m 2^-9, code 0x7f is NaN)."""
+    vals = []
+    for c in range(0x7f):
+        e, m = c >> 3, c & 7
+        vals.append(m * 2.0 ** -9 if e == 0 else (8 + m) * 2.0 ** (e - 10))
+    return np.array(vals)
+
+
+def _e4m3_brute(v):
+    """Nearest finite E4M3 by exhaustive search; ties go to the even code;
+    beyond 448 saturate."""
+    tab = _e4m3_table()
+    out = np.empty(len(v), np.uint8)
+    for i, x in enumerate(np.asarray(v, np.float64)):
+        a = abs(x)
+        dist = np.abs(tab - a)
+        best = np.flatnonzero(dist == dist.min())
+        c = int(best[0]) if len(best) == 1 else int([b for b in best if b % 2 == 0][0])
+        if a >= 448.0:
+            c = 0x7e
+        out[i] = c | (0x80 if np.signbit(x) else 0)
+    return out
+
+
+def test_e4m3_decode_table():
+    v = oracle.e4m3_decode(np.arange(256, dtype=np.uint8))
+    tab = _e4m3_table()
+    assert np.array_equal(v[:0x7f].astype(np.float64), tab)
+    assert np.isnan(v[0x7f]) and np.isnan(v[0xff])
+    assert np.array_equal(v[0x80:0xff], -v[:0x7f])
+    assert v[0x7e] == 448.0 and v[1] == 2.0 ** -9 and v[8] == 2.0 ** -6
+    assert np.all(np.diff(tab) > 0)
+
+
+def test_e4m3_encode_matches_exhaustive_nearest_with_ties_to_even():
+    tab = _e4m3_table()
+    mids = (tab[1:] + tab[:-1]) / 2.0
+    rng = np.random.default_rng(7)
+    dense = np.exp(rng.uniform(np.log(1e-4), np.log(600.0), 4000)).astype(np.float32)
+    special = np.array([0.0, 448.0, 449.0, 464.0, 465.0, 1e6, 2.0 ** -10, 3 * 2.0 ** -11, 1e-30], np.float32)
+    v = np.concatenate([tab.astype(np.float32), mids.astype(np.float32), dense, special])
+    v = np.concatenate([v, -v])
+    assert np.array_equal(oracle.e4m3_encode(v), _e4m3_brute(v))
+    # every code decodes and re-encodes to itself (the NaN codes excepted)
+    codes = np.array([c for c in range(256) if c & 0x7f != 0x7f], np.uint8)
+    assert np.array_equal(oracle.e4m3_encode(oracle.e4m3_decode(codes)), codes)
+
+
+def test_fp8_quant_rows_scale_and_error_bound():
+    v = synth.normal(17, 1, (100, 300), std=2.0)
+    v[5] = 0.0
+    q, s = oracle.quantize_rows_fp8(v)
+    assert s[5] == 0.0 and not q[5].any()
+    dq = oracle.e4m3_decode(q).astype(np.float64)
+    for r in range(v.shape[0]):
+        if r == 5:
+            continue
+        amax = np.abs(v[r]).max()
+        assert s[r] == np.float32(amax) / np.float32(448.0)
+        assert (q[r] & 0x7f).max() == 0x7e            # the largest value maps to +-448
+        t = v[r].astype(np.float64) / float(s[r])
+        # half a step of the value's binade (2^-4 relative for normals, 2^-10 absolute below 2^-6)
+        step = np.where(np.abs(t) >= 2.0 ** -6, 2.0 ** (np.floor(np.log2(np.maximum(np.abs(t), 1e-30))) - 3),
+                        2.0 ** -9)
+        assert np.all(np.abs(t - dq[r]) <= step / 2 * (1 + 1e-6) + 1e-7 * np.abs(t))
+
+
+def test_fp8_gemm_is_the_exact_sum_rounded_once():
+    rng = np.random.default_rng(18)
+    a = rng.integers(0, 256, (7, 333), dtype=np.uint8)
+    b = rng.integers(0, 256, (5, 333), dtype=np.uint8)
+    a[(a & 0x7f) == 0x7f] = 0
+    b[(b & 0x7f) == 0x7f] = 0
+    c = oracle.gemm_fp8(a, b)
+    va, vb = oracle.e4m3_decode(a), oracle.e4m3_decode(b)
+    from fractions import Fraction
+    for m in range(a.shape[0]):
+        for n in range(b.shape[0]):
+            exact = sum(Fraction(float(x)) * Fraction(float(y)) for x, y in zip(va[m], vb[n]))
+            assert c[m, n] == np.float32(float(exact))
+
+
+def test_fp8_dense_special_case_e1_k1():
+    """E = 1, k = 1: the layer is one dense SwiGLU FFN; the FP8 chain stays
+    within FP8 noise (a few 1e-2 relative) of the unquantised fp64 FFN."""
+    d, f, T = 128, 256, 8
+    x = synth.normal(19, 1, (T, d))
+    wg = synth.normal(19, 2, (1, d, f), std=0.05)
+    wu = synth.normal(19, 3, (1, d, f), std=0.05)
+    wd = synth.normal(19, 4, (1, f, d), std=0.05)
+    prep = oracle.prepare_fp8(wg, wu, wd, x, 0.5)
+    rt = oracle.route(x, 1, 1, logits=np.zeros((T, 1), np.float32))
+    y, dbg = oracle.moe_tokens_fp8(x, prep, rt)
+    x64 = x.astype(np.float64)
+    g = x64 @ wg[0].astype(np.float64)
+    u = x64 @ wu[0].astype(np.float64)
+    h = g / (1.0 + np.exp(-g)) * u
+    ref = h @ wd[0].astype(np.float64)
+    rel = np.abs(y - ref).max() / np.abs(ref).max()
+    assert rel < 0.1
+    # every stage's debug output decodes to values of the right scale
+    assert np.all(dbg["sx"] > 0) and np.all(dbg["sh"] > 0)

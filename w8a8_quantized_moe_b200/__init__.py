@@ -25,6 +25,9 @@ MOE_ERR_OOM = 6
 MOE_F32 = 0
 MOE_BF16 = 1
 
+MOE_FMT_INT8 = 0
+MOE_FMT_E4M3 = 1
+
 MOE_PATH_AUTO = 0
 MOE_PATH_STREAM = 1
 MOE_PATH_TENSOR = 2
@@ -55,7 +58,8 @@ class moe_w8a8_config(ctypes.Structure):
     _fields_ = [("d", ctypes.c_int32), ("f", ctypes.c_int32), ("n_experts", ctypes.c_int32),
                 ("top_k", ctypes.c_int32), ("alpha", ctypes.c_float),
                 ("capacity_factor", ctypes.c_float), ("renormalize", ctypes.c_int32),
-                ("in_dtype", ctypes.c_int32), ("out_dtype", ctypes.c_int32)]
+                ("in_dtype", ctypes.c_int32), ("out_dtype", ctypes.c_int32),
+                ("expert_format", ctypes.c_int32)]
 
 
 _DBG_FIELDS = ("logits", "topk_idx", "topk_w", "offsets", "row2ts", "ts2row", "xq", "sx", "acc1",
@@ -198,9 +202,9 @@ class Weights:
 
 
 def make_config(d, f, n_experts, top_k, alpha=0.6, capacity_factor=0.0, renormalize=True,
-                in_dtype=MOE_BF16, out_dtype=MOE_BF16) -> moe_w8a8_config:
+                in_dtype=MOE_BF16, out_dtype=MOE_BF16, expert_format=MOE_FMT_INT8) -> moe_w8a8_config:
     return moe_w8a8_config(d, f, n_experts, top_k, alpha, capacity_factor, 1 if renormalize else 0,
-                           in_dtype, out_dtype)
+                           in_dtype, out_dtype, expert_format)
 
 
 def moe_w8a8_prepare(cfg: moe_w8a8_config, w_gate, w_up, w_down, w_router, act_absmax,

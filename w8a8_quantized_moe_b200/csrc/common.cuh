@@ -7,6 +7,7 @@
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda_fp8.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -79,6 +80,26 @@ __device__ __forceinline__ int quant_code_fast(float v, float s, float r) {
     const float dist = fabsf(fabsf(__fsub_rn(t, n)) - 0.5f);
     int q = (dist > 3.0e-5f || fabsf(t) > 130.0f) ? __float2int_rn(n) : __float2int_rn(__fdiv_rn(v, s));
     return max(-127, min(127, q));
+}
+
+// E4M3 code of v: the nearest E4M3 value, ties to even, magnitudes beyond 448
+// saturated (the conversion instruction's round-to-nearest, satfinite mode).
+__device__ __forceinline__ uint32_t e4m3_code(float v) {
+    return (uint32_t)__nv_cvt_float_to_fp8(v, __NV_SATFINITE, __NV_E4M3);
+}
+
+// Expert number formats (values of moe_w8a8_config::expert_format).
+enum { FMT_INT8 = 0, FMT_E4M3 = 1 };
+
+// Largest code magnitude of a format: the scale of a vector is amax / this.
+template <int FMT>
+__device__ __forceinline__ float fmt_qmax() { return FMT == FMT_E4M3 ? 448.0f : 127.0f; }
+
+// Code byte of v for scale s > 0 (r = fp32(1 / s), used by the INT8 rule only).
+template <int FMT>
+__device__ __forceinline__ uint32_t fmt_code(float v, float s, float r) {
+    if (FMT == FMT_E4M3) return e4m3_code(__fdiv_rn(v, s));
+    return (uint32_t)quant_code_fast(v, s, r) & 0xffu;
 }
 
 // Pack four INT8 codes (low byte first).

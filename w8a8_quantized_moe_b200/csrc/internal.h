@@ -68,9 +68,10 @@ cudaError_t launch_gateup_input_absmax(const float* w_gate, const float* w_up, i
                                        float* aw, cudaStream_t s);
 // Quantise column-major channels: W [E][K][N] fp32 (input j, output n), optional
 // per-input smoothing s[K]; channel n goes to out row map(n) of [E][rows][K].
+// fmt: MOE_FMT_INT8 or MOE_FMT_E4M3 (codes stored as bytes either way)
 cudaError_t launch_quantize_channels(const float* w, const float* smooth, int E, int K, int N,
                                      int8_t* out, int out_rows, int row_block, int row_stride,
-                                     int row_base, float* sw, cudaStream_t s);
+                                     int row_base, float* sw, int fmt, cudaStream_t s);
 cudaError_t launch_export_gateup(const int8_t* w_gu, int E, int d, int f, int8_t* gate,
                                  int8_t* up, cudaStream_t s);
 
@@ -89,7 +90,7 @@ cudaError_t launch_route_small(const float* logits, const float* bias, int T, in
 // act_clip > 0 caps each token's range (saturating clip), 0 = off.
 cudaError_t launch_smooth_quant(const void* x, int in_dtype, const float* inv_s, float act_clip, int T,
                                 int d, int k, const int32_t* ts2row, int8_t* xq, float* sx, int8_t* aq,
-                                cudaStream_t s);
+                                int fmt, cudaStream_t s);
 // out[r][j] = |fp32(x[r][j] * inv_s[j])| (calibration of the activation clip)
 cudaError_t launch_scaled_abs(const void* x, int64_t rows, int d, int dtype, const float* inv_s, float* out,
                               cudaStream_t s);
@@ -114,7 +115,7 @@ cudaError_t launch_tc_gemm1(const moe_w8a8_weights* w, int T, const int8_t* aq, 
                             const float* sx, float* h32, float* pamax, int32_t* acc_dbg,
                             cudaStream_t s);
 cudaError_t launch_requant(const float* h32, const float* pamax, int f, const int32_t* meta,
-                           int max_rows, int8_t* hq, float* sh, cudaStream_t s);
+                           int max_rows, int8_t* hq, float* sh, int fmt, cudaStream_t s);
 cudaError_t launch_tc_gemm2(const moe_w8a8_weights* w, int T, const int8_t* hq, const float* sh,
                             const int32_t* meta, const int32_t* tiles, const int32_t* offsets,
                             const int32_t* row2ts, const float* topk_w, float* o, int32_t* acc_dbg,

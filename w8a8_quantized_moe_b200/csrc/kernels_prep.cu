@@ -60,10 +60,12 @@ __global__ void gateup_input_absmax_kernel(const float* __restrict__ wg, const f
 // Per-output-channel quantisation of W [E][K][N] (input j along K, output n
 // along N).  Block = (32 channels, expert), 256 threads as 8 rows x 32 columns.
 // Pass 1: amax_n = max_j |W'[j][n]| with W' = fp32(s_j * W) (s may be NULL).
-// Pass 2: codes rint(W'/sw_n) written K-major to out row map(n).
+// Pass 2: codes rint(W'/sw_n) (INT8) or e4m3(W'/sw_n) (E4M3), sw_n = amax_n /
+// 127 or / 448, written K-major to out row map(n).
 constexpr int kQCh = 32;
 constexpr int kQJ = 128;  // j-chunk staged through shared memory
 
+template <int FMT>
 __global__ void __launch_bounds__(256) quantize_channels_kernel(
     const float* __restrict__ w, const float* __restrict__ smooth, int K, int N,
     int8_t* __restrict__ out, int out_rows, int row_block, int row_stride, int row_base,
@@ -87,7 +89,7 @@ __global__ void __launch_bounds__(256) quantize_channels_kernel(
     if (ty == 0) {
         float a = red[0][tx];
         for (int i = 1; i < 8; ++i) a = fmaxf(a, red[i][tx]);
-        const float s = a > 0.0f ? __fdiv_rn(a, 127.0f) : 0.0f;
+        const float s = a > 0.0f ? __fdiv_rn(a, fmt_qmax<FMT>()) : 0.0f;
         scale_s[tx] = s;
         if (n < N) sw[(int64_t)e * N + n] = s;
     }
@@ -101,7 +103,7 @@ __global__ void __launch_bounds__(256) quantize_channels_kernel(
             if (n < N && s > 0.0f) {
                 float v = we[(int64_t)(j0 + jj) * N + n];
                 if (smooth) v = __fmul_rn(smooth[j0 + jj], v);
-                q = quant_code(v, s);
+                q = FMT == FMT_E4M3 ? (int)e4m3_code(__fdiv_rn(v, s)) : quant_code(v, s);
             }
             tile[tx][jj] = (int8_t)q;
         }
@@ -158,10 +160,14 @@ cudaError_t launch_gateup_input_absmax(const float* w_gate, const float* w_up, i
 
 cudaError_t launch_quantize_channels(const float* w, const float* smooth, int E, int K, int N,
                                      int8_t* out, int out_rows, int row_block, int row_stride,
-                                     int row_base, float* sw, cudaStream_t s) {
+                                     int row_base, float* sw, int fmt, cudaStream_t s) {
     dim3 grid((N + kQCh - 1) / kQCh, E);
-    quantize_channels_kernel<<<grid, 256, 0, s>>>(w, smooth, K, N, out, out_rows, row_block,
-                                                  row_stride, row_base, sw);
+    if (fmt == FMT_E4M3)
+        quantize_channels_kernel<FMT_E4M3><<<grid, 256, 0, s>>>(w, smooth, K, N, out, out_rows, row_block,
+                                                                row_stride, row_base, sw);
+    else
+        quantize_channels_kernel<FMT_INT8><<<grid, 256, 0, s>>>(w, smooth, K, N, out, out_rows, row_block,
+                                                                row_stride, row_base, sw);
     return cudaGetLastError();
 }
 

@@ -218,6 +218,98 @@ __global__ void __launch_bounds__(kRtThreads) router_logits_async_kernel(
     }
 }
 
+// Router logits for bf16 X and E % 32 == 0, same fixed order, with a larger
+// register tile: each lane keeps its chain position for 16 tokens x 8 experts
+// (128 accumulators), so every W value it reads from shared memory feeds 16
+// FMAs and every X value 8.  256 threads: warp w covers tokens (w >> 2) * 16
+// and experts (w & 3) * 8 of the block's 32 x 32 tile.  X ([token][channel],
+// rows padded by 16 bytes) and W (rows padded to 36 floats, so a quarter
+// warp's 16-byte loads hit distinct banks) arrive by cp.async through a
+// 3-stage ring of 256-channel chunks; a lane reads its 16 tokens' values of
+// channel 32i + lane one bf16 at a time (a warp reads 64 consecutive bytes).
+// Measured against transposed-X and 128-channel variants of the same tile
+// (identical logits): this one was the fastest, by 5%.
+constexpr int kRwThreads = 256;
+constexpr int kRwKC = 256;        // channels per staged chunk (8 steps of i)
+
+struct RouterWideSmem {
+    uint16_t x[kRaStages][kRtT][kRwKC + 8];
+    float w[kRaStages][kRwKC][kRaWPad];
+};
+
+__global__ void __launch_bounds__(kRwThreads, 1) router_logits_wide_kernel(
+    const uint16_t* __restrict__ x, const float* __restrict__ wr, int T, int d, int E,
+    float* __restrict__ logits) {
+    pdl_wait();
+    pdl_trigger();
+
+    extern __shared__ __align__(16) uint8_t smem_raw[];
+    RouterWideSmem& sm = *reinterpret_cast<RouterWideSmem*>(smem_raw);
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int tg = warp >> 2, eg = warp & 3;
+    const int t0 = blockIdx.x * kRtT, e0 = blockIdx.y * kRtE;
+    const int nchunks = d / kRwKC;
+
+    auto issue = [&](int c, int stage) {
+        for (int q = tid; q < kRtT * kRwKC / 8; q += kRwThreads) {
+            const int tt = q / (kRwKC / 8), part = q % (kRwKC / 8);
+            cp_async16(&sm.x[stage][tt][part * 8], x + (int64_t)min(t0 + tt, T - 1) * d + (int64_t)c * kRwKC + part * 8,
+                       16);
+        }
+        for (int q = tid; q < kRwKC * kRtE / 4; q += kRwThreads) {
+            const int row = q / (kRtE / 4), c4 = q % (kRtE / 4);
+            cp_async16(&sm.w[stage][row][4 * c4], wr + (int64_t)(c * kRwKC + row) * E + e0 + 4 * c4, 16);
+        }
+        cp_async_commit();
+    };
+
+    float acc[16][8];
+#pragma unroll
+    for (int a = 0; a < 16; ++a)
+#pragma unroll
+        for (int b = 0; b < 8; ++b) acc[a][b] = 0.0f;
+
+    issue(0, 0);
+    if (nchunks > 1) issue(1, 1); else cp_async_commit();
+    for (int c = 0; c < nchunks; ++c) {
+        cp_async_wait<1>();
+        __syncthreads();
+        if (c + 2 < nchunks) issue(c + 2, (c + 2) % kRaStages); else cp_async_commit();
+        const int st = c % kRaStages;
+#pragma unroll
+        for (int i = 0; i < kRwKC / 32; ++i) {
+            const int k = 32 * i + lane;
+            float xv[16];
+#pragma unroll
+            for (int a = 0; a < 16; ++a) xv[a] = __uint_as_float((uint32_t)sm.x[st][tg * 16 + a][k] << 16);
+            const float4 wa = *reinterpret_cast<const float4*>(&sm.w[st][k][eg * 8]);
+            const float4 wb = *reinterpret_cast<const float4*>(&sm.w[st][k][eg * 8 + 4]);
+            const float wv[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
+#pragma unroll
+            for (int a = 0; a < 16; ++a)
+#pragma unroll
+                for (int b = 0; b < 8; ++b) acc[a][b] = __fmaf_rn(xv[a], wv[b], acc[a][b]);
+        }
+    }
+    cp_async_wait<0>();
+#pragma unroll
+    for (int a = 0; a < 16; ++a)
+#pragma unroll
+        for (int b = 0; b < 8; ++b) {
+            float v = acc[a][b];
+#pragma unroll
+            for (int o = 16; o >= 1; o >>= 1) v = __fadd_rn(v, __shfl_xor_sync(0xffffffffu, v, o));
+            acc[a][b] = v;
+        }
+    // every lane holds all 128 logits of the warp's tile; lane q writes entries q, q+32, q+64, q+96
+#pragma unroll
+    for (int v = 0; v < 128; ++v) {
+        if ((v & 31) != lane) continue;
+        const int t = t0 + tg * 16 + (v >> 3), e = e0 + eg * 8 + (v & 7);
+        if (t < T) logits[(int64_t)t * E + e] = acc[v >> 3][v & 7];
+    }
+}
+
 // ---------------------------------------------------------------------------
 // Top-k + gate weights, one warp per token.  l_e = logit + bias_e; k rounds of
 // a warp argmax on (l descending, e ascending); w = softmax of the selected
@@ -513,7 +605,7 @@ __global__ void __launch_bounds__(kRouteSmallThreads) route_small_kernel(
 // for the tensor-core path, to every kept (t, slot) row of the sorted copy.
 constexpr int kSqThreads = 128;
 
-template <int kSqMaxGroups>   // groups of 8 channels per thread: d <= 128 x 8 x kSqMaxGroups
+template <int kSqMaxGroups, int FMT>   // groups of 8 channels per thread: d <= 128 x 8 x kSqMaxGroups
 __global__ void __launch_bounds__(kSqThreads) smooth_quant_kernel(
     const void* __restrict__ x, int in_dtype, const float* __restrict__ inv_s, float act_clip, int T, int d,
     int k, const int32_t* __restrict__ ts2row, int8_t* __restrict__ xq, float* __restrict__ sx,
@@ -551,7 +643,7 @@ __global__ void __launch_bounds__(kSqThreads) smooth_quant_kernel(
 #pragma unroll
     for (int w = 0; w < kSqThreads / 32; ++w) m = fmaxf(m, red[w]);
     if (act_clip > 0.0f) m = fminf(m, act_clip);   // saturating clip: values beyond it go to +-127
-    const float s = m > 0.0f ? __fdiv_rn(m, 127.0f) : 0.0f;
+    const float s = m > 0.0f ? __fdiv_rn(m, fmt_qmax<FMT>()) : 0.0f;
     const float rs = s > 0.0f ? __frcp_rn(s) : 0.0f;
     if (tid == 0) sx[t] = s;
     int rows[kMaxK];
@@ -563,7 +655,7 @@ __global__ void __launch_bounds__(kSqThreads) smooth_quant_kernel(
         if (g >= ng) continue;
         int q[8];
 #pragma unroll
-        for (int c = 0; c < 8; ++c) q[c] = s > 0.0f ? quant_code_fast(v[gi][c], s, rs) : 0;
+        for (int c = 0; c < 8; ++c) q[c] = s > 0.0f ? (int)fmt_code<FMT>(v[gi][c], s, rs) : 0;
         const uint2 packed = make_uint2(pack4(q[0], q[1], q[2], q[3]), pack4(q[4], q[5], q[6], q[7]));
         *reinterpret_cast<uint2*>(xq + (int64_t)t * d + g * 8) = packed;
 #pragma unroll
@@ -577,6 +669,17 @@ __global__ void __launch_bounds__(kSqThreads) smooth_quant_kernel(
 cudaError_t launch_router_logits(const void* x, int in_dtype, const float* wr, int T, int d, int E,
                                  float* logits, cudaStream_t s) {
     dim3 grid((T + kRtT - 1) / kRtT, (E + kRtE - 1) / kRtE);
+    if (in_dtype == MOE_BF16 && E % kRtE == 0 && d % kRwKC == 0 && (reinterpret_cast<uintptr_t>(x) & 15) == 0) {
+        static bool wide_attr = false;
+        if (!wide_attr) {
+            cudaError_t e = cudaFuncSetAttribute(router_logits_wide_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 (int)sizeof(RouterWideSmem));
+            if (e != cudaSuccess) return e;
+            wide_attr = true;
+        }
+        return launch_pdl(router_logits_wide_kernel, grid, dim3(kRwThreads), sizeof(RouterWideSmem), s,
+                          reinterpret_cast<const uint16_t*>(x), wr, T, d, E, logits);
+    }
     if (E % 4 == 0 && E >= 4) {
         static bool attr = false;
         if (!attr) {
@@ -635,9 +738,13 @@ cudaError_t launch_route_small(const float* logits, const float* bias, int T, in
 
 cudaError_t launch_smooth_quant(const void* x, int in_dtype, const float* inv_s, float act_clip, int T,
                                 int d, int k, const int32_t* ts2row, int8_t* xq, float* sx, int8_t* aq,
-                                cudaStream_t s) {
+                                int fmt, cudaStream_t s) {
     const int groups = (d / 8 + kSqThreads - 1) / kSqThreads;
-    auto kern = groups <= 4 ? smooth_quant_kernel<4> : groups <= 8 ? smooth_quant_kernel<8> : smooth_quant_kernel<16>;
+    auto kern = fmt == FMT_E4M3
+                    ? (groups <= 4 ? smooth_quant_kernel<4, FMT_E4M3>
+                                   : groups <= 8 ? smooth_quant_kernel<8, FMT_E4M3> : smooth_quant_kernel<16, FMT_E4M3>)
+                    : (groups <= 4 ? smooth_quant_kernel<4, FMT_INT8>
+                                   : groups <= 8 ? smooth_quant_kernel<8, FMT_INT8> : smooth_quant_kernel<16, FMT_INT8>);
     return launch_pdl(kern, dim3(T), dim3(kSqThreads), 0, s, x, in_dtype, inv_s, act_clip, T, d, k, ts2row, xq,
                       sx, aq);
 }

@@ -1,5 +1,8 @@
-// Grouped INT8 GEMMs on the 5th-generation tensor cores (tcgen05, kind::i8)
-// for the expert FFN of the W8A8 MoE layer ("MiniMax-M3 W8A8 on K100AI",
+// Grouped 8-bit GEMMs on the 5th-generation tensor cores (tcgen05: kind::i8
+// for INT8 experts with INT32 accumulators, kind::f8f6f4 for E4M3 experts with
+// fp32 accumulators; "Day0 adaptation of ultra-large model inference",
+// section 1: FP8 or INT8 expert layers) for the expert FFN of the W8A8 MoE
+// layer ("MiniMax-M3 W8A8 on K100AI",
 // s1.2: INT8 x INT8 on the INT8 GEMM path with integer accumulation; s4.3:
 // fuse the expert FFN and stay in INT8 between the two matmuls; "Day0
 // adaptation of ultra-large model inference", section 4: grouped GEMM over the
@@ -49,10 +52,14 @@ constexpr int kEpiStageBytes = 16 * 32 * 4;      // 16 rows x 32 fp32 per epilog
 constexpr size_t kSmemBytes = (size_t)kStages * kStageBytes + (size_t)kEpiWarps * kEpiStageBytes + 1024 + 256;
 
 
-// Instruction descriptor, kind::i8: D = s32 (bits 4-5 = 2), A and B signed
-// 8-bit (bits 7-9, 10-12 = 1), both K-major, N>>3 at bit 17, M>>4 at bit 24.
-constexpr uint32_t kIdesc = (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
-                            ((uint32_t)(BM >> 4) << 24);
+// Instruction descriptors (both operands K-major, N>>3 at bit 17, M>>4 at bit 24):
+//   kind::i8     D = s32 (bits 4-5 = 2), A and B signed 8-bit (bits 7-9, 10-12 = 1)
+//   kind::f8f6f4 D = f32 (bits 4-5 = 1), A and B E4M3 (bits 7-9, 10-12 = 0)
+template <int FMT>
+__host__ __device__ constexpr uint32_t idesc() {
+    return (FMT == FMT_E4M3 ? (1u << 4) : ((2u << 4) | (1u << 7) | (1u << 10))) | ((uint32_t)(BN >> 3) << 17) |
+           ((uint32_t)(BM >> 4) << 24);
+}
 
 struct Ctl {
     uint64_t full[kStages];
@@ -170,12 +177,28 @@ __device__ __forceinline__ uint64_t desc_sw128(uint32_t saddr) {
     return d;
 }
 
-__device__ __forceinline__ void mma_i8(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t accum) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(tmem_d),
-        "l"(adesc), "l"(bdesc), "r"(kIdesc), "r"(accum));
+// One M=128, N=256, K=32 MMA of 8-bit operands: INT8 (s32 accumulators) or
+// E4M3 (f32 accumulators).
+template <int FMT>
+__device__ __forceinline__ void mma_8bit(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t accum) {
+    if (FMT == FMT_E4M3)
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "setp.ne.b32 p, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(tmem_d),
+            "l"(adesc), "l"(bdesc), "r"(idesc<FMT>()), "r"(accum));
+    else
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "setp.ne.b32 p, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(tmem_d),
+            "l"(adesc), "l"(bdesc), "r"(idesc<FMT>()), "r"(accum));
+}
+
+// Accumulator word as a float: INT32 converted, fp32 reinterpreted.
+template <int FMT>
+__device__ __forceinline__ float acc_value(uint32_t a) {
+    return FMT == FMT_E4M3 ? __uint_as_float(a) : __int2float_rn((int)a);
 }
 
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
@@ -243,6 +266,7 @@ __device__ __forceinline__ void store_rows32(float* stage, const uint32_t (&v)[3
 // GEMM1 tile: columns 0..127 of the accumulator are gate channels
 // nt*128 + c, columns 128..255 the matching up channels.  Each warp owns 32
 // rows (its TMEM lane quarter) and 64 of the 128 h columns.
+template <int FMT>
 __device__ __forceinline__ void epilogue_swiglu(const TcParams& p, uint32_t taddr, int half, int e,
                                                 int nt, int wrow0, int nvalid, float* stage,
                                                 Ctl* ctl, int buf, int lane) {
@@ -282,8 +306,8 @@ __device__ __forceinline__ void epilogue_swiglu(const TcParams& p, uint32_t tadd
             const float sgv[4] = {sg.x, sg.y, sg.z, sg.w}, suv[4] = {su.x, su.y, su.z, su.w};
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
-                const float gf = __fmul_rn(__fmul_rn(__int2float_rn((int)g[j + q]), sxt), sgv[q]);
-                const float uf = __fmul_rn(__fmul_rn(__int2float_rn((int)u[j + q]), sxt), suv[q]);
+                const float gf = __fmul_rn(__fmul_rn(acc_value<FMT>(g[j + q]), sxt), sgv[q]);
+                const float uf = __fmul_rn(__fmul_rn(acc_value<FMT>(u[j + q]), sxt), suv[q]);
                 const float h = __fmul_rn(moe_silu(gf), uf);
                 if (valid) amax = fmaxf(amax, fabsf(h));
                 u[j + q] = __float_as_uint(h);
@@ -294,6 +318,7 @@ __device__ __forceinline__ void epilogue_swiglu(const TcParams& p, uint32_t tadd
     if (valid) p.pamax[(int64_t)grow * (f / 64) + nt * 2 + half] = amax;
 }
 
+template <int FMT>
 __device__ __forceinline__ void epilogue_down(const TcParams& p, uint32_t taddr, int half, int e,
                                               int nt, int wrow0, int nvalid, float* stage, Ctl* ctl,
                                               int buf, int lane) {
@@ -329,7 +354,7 @@ __device__ __forceinline__ void epilogue_down(const TcParams& p, uint32_t taddr,
 #pragma unroll
             for (int q = 0; q < 4; ++q)
                 a[j + q] = __float_as_uint(
-                    __fmul_rn(__fmul_rn(__fmul_rn(__int2float_rn((int)a[j + q]), shr), sv[q]), wr));
+                    __fmul_rn(__fmul_rn(__fmul_rn(acc_value<FMT>(a[j + q]), shr), sv[q]), wr));
         }
         store_rows32(stage, a, p.o + (int64_t)wrow0 * d + ch0, d, nvalid, lane);
     }
@@ -337,7 +362,7 @@ __device__ __forceinline__ void epilogue_down(const TcParams& p, uint32_t taddr,
 
 // ------------------------------------------------------------------ the kernel
 
-template <int EPI>
+template <int EPI, int FMT>
 __global__ void __launch_bounds__(kThreads, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                    const TcParams p) {
@@ -425,7 +450,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const uint32_t b_addr = a_addr + kABytes;
 #pragma unroll
                     for (int kk = 0; kk < BK / 32; ++kk)
-                        mma_i8(d_tmem, desc_sw128(a_addr + kk * 32), desc_sw128(b_addr + kk * 32),
+                        mma_8bit<FMT>(d_tmem, desc_sw128(a_addr + kk * 32), desc_sw128(b_addr + kk * 32),
                                (kb | kk) != 0 ? 1u : 0u);
                     mma_commit(&ctl->empty[s]);
                     if (++s == kStages) { s = 0; ph ^= 1; }
@@ -458,9 +483,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int nvalid = max(0, min(32, nrows - quad * 32));
             const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(buf * BN);
             if (EPI == EPI_SWIGLU)
-                epilogue_swiglu(p, taddr, half, e, nt, wrow0, nvalid, stage, ctl, buf, lane);
+                epilogue_swiglu<FMT>(p, taddr, half, e, nt, wrow0, nvalid, stage, ctl, buf, lane);
             else
-                epilogue_down(p, taddr, half, e, nt, wrow0, nvalid, stage, ctl, buf, lane);
+                epilogue_down<FMT>(p, taddr, half, e, nt, wrow0, nvalid, stage, ctl, buf, lane);
             buf ^= 1;
             if (buf == 0) aph ^= 1;
         }
@@ -483,6 +508,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 constexpr int kRqThreads = 256;
 constexpr int kRqBatch = 8;
 
+template <int FMT>
 __global__ void __launch_bounds__(kRqThreads) requant_kernel(const float* __restrict__ h32,
                                                              const float* __restrict__ pamax, int f,
                                                              const int32_t* __restrict__ meta,
@@ -505,7 +531,7 @@ __global__ void __launch_bounds__(kRqThreads) requant_kernel(const float* __rest
     float m = 0.0f;
     for (int i = lane; i < npart; i += 32) m = fmaxf(m, pamax[(int64_t)row * npart + i]);
     m = warp_max(m);
-    const float s = m > 0.0f ? __fdiv_rn(m, 127.0f) : 0.0f;
+    const float s = m > 0.0f ? __fdiv_rn(m, fmt_qmax<FMT>()) : 0.0f;
     const float rs = s > 0.0f ? __frcp_rn(s) : 0.0f;
     if (lane == 0) sh[row] = s;
     for (int b = 0; b < n4; b += 32 * kRqBatch) {
@@ -520,8 +546,8 @@ __global__ void __launch_bounds__(kRqThreads) requant_kernel(const float* __rest
         for (int i = 0; i < kRqBatch; ++i) {
             const int c4 = b + lane + 32 * i;
             if (c4 < n4)
-                qrow[c4] = s > 0.0f ? pack4(quant_code_fast(h[i].x, s, rs), quant_code_fast(h[i].y, s, rs),
-                                            quant_code_fast(h[i].z, s, rs), quant_code_fast(h[i].w, s, rs))
+                qrow[c4] = s > 0.0f ? pack4((int)fmt_code<FMT>(h[i].x, s, rs), (int)fmt_code<FMT>(h[i].y, s, rs),
+                                            (int)fmt_code<FMT>(h[i].z, s, rs), (int)fmt_code<FMT>(h[i].w, s, rs))
                                     : 0u;
         }
     }
@@ -560,17 +586,23 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t K, uint64_t rows, uint3
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int EPI>
-cudaError_t launch(const CUtensorMap& ta, const CUtensorMap& tb, const TcParams& p, int grid,
-                   cudaStream_t s) {
+template <int EPI, int FMT>
+cudaError_t launch_fmt(const CUtensorMap& ta, const CUtensorMap& tb, const TcParams& p, int grid,
+                       cudaStream_t s) {
     static bool attr = false;
     if (!attr) {
-        cudaError_t e = cudaFuncSetAttribute(tc_gemm_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        cudaError_t e = cudaFuncSetAttribute(tc_gemm_kernel<EPI, FMT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)kSmemBytes);
         if (e != cudaSuccess) return e;
         attr = true;
     }
-    return launch_pdl(tc_gemm_kernel<EPI>, dim3(grid), dim3(kThreads), kSmemBytes, s, ta, tb, p);
+    return launch_pdl(tc_gemm_kernel<EPI, FMT>, dim3(grid), dim3(kThreads), kSmemBytes, s, ta, tb, p);
+}
+
+template <int EPI>
+cudaError_t launch(const CUtensorMap& ta, const CUtensorMap& tb, const TcParams& p, int grid, int fmt,
+                   cudaStream_t s) {
+    return fmt == FMT_E4M3 ? launch_fmt<EPI, FMT_E4M3>(ta, tb, p, grid, s) : launch_fmt<EPI, FMT_INT8>(ta, tb, p, grid, s);
 }
 
 }  // namespace
@@ -584,10 +616,12 @@ bool tc_make_weight_maps(moe_w8a8_weights* w) {
 bool tc_supported(const moe_w8a8_config& c) { return c.d % BN == 0 && c.f % BK == 0 && c.d % BK == 0; }
 
 cudaError_t launch_requant(const float* h32, const float* pamax, int f, const int32_t* meta,
-                           int max_rows, int8_t* hq, float* sh, cudaStream_t s) {
+                           int max_rows, int8_t* hq, float* sh, int fmt, cudaStream_t s) {
     const int rows_per_block = kRqThreads / 32;
-    return launch_pdl(requant_kernel, dim3((max_rows + rows_per_block - 1) / rows_per_block),
-                      dim3(kRqThreads), 0, s, h32, pamax, f, meta, hq, sh);
+    const dim3 grid((max_rows + rows_per_block - 1) / rows_per_block);
+    if (fmt == FMT_E4M3)
+        return launch_pdl(requant_kernel<FMT_E4M3>, grid, dim3(kRqThreads), 0, s, h32, pamax, f, meta, hq, sh);
+    return launch_pdl(requant_kernel<FMT_INT8>, grid, dim3(kRqThreads), 0, s, h32, pamax, f, meta, hq, sh);
 }
 
 cudaError_t launch_tc_gemm1(const moe_w8a8_weights* w, int T, const int8_t* aq, const int32_t* meta,
@@ -617,7 +651,7 @@ cudaError_t launch_tc_gemm1(const moe_w8a8_weights* w, int T, const int8_t* aq, 
     p.status = w->status;
     const int max_mt = (rows + BM - 1) / BM + c.n_experts;
     const int grid = max(1, min(w->num_sms, max_mt * p.n_tiles_n));
-    return launch<EPI_SWIGLU>(ta, w->tm_w_gu, p, grid, s);
+    return launch<EPI_SWIGLU>(ta, w->tm_w_gu, p, grid, c.expert_format, s);
 }
 
 cudaError_t launch_tc_gemm2(const moe_w8a8_weights* w, int T, const int8_t* hq, const float* sh,
@@ -646,7 +680,7 @@ cudaError_t launch_tc_gemm2(const moe_w8a8_weights* w, int T, const int8_t* hq, 
     p.status = w->status;
     const int max_mt = (rows + BM - 1) / BM + c.n_experts;
     const int grid = max(1, min(w->num_sms, max_mt * p.n_tiles_n));
-    return launch<EPI_DOWN>(ta, w->tm_w_dn, p, grid, s);
+    return launch<EPI_DOWN>(ta, w->tm_w_dn, p, grid, c.expert_format, s);
 }
 
 }  // namespace moe

@@ -25,6 +25,7 @@ moe_status check_config(const moe_w8a8_config* c) {
     if (c->in_dtype != MOE_F32 && c->in_dtype != MOE_BF16) return MOE_ERR_INVALID_ARG;
     if (c->out_dtype != MOE_F32 && c->out_dtype != MOE_BF16) return MOE_ERR_INVALID_ARG;
     if (c->renormalize != 0 && c->renormalize != 1) return MOE_ERR_INVALID_ARG;
+    if (c->expert_format != MOE_FMT_INT8 && c->expert_format != MOE_FMT_E4M3) return MOE_ERR_INVALID_ARG;
     if (std::isnan(c->capacity_factor)) return MOE_ERR_INVALID_ARG;
     if (c->d <= 0 || c->f <= 0 || c->n_experts <= 0 || c->top_k <= 0) return MOE_ERR_UNSUPPORTED_SHAPE;
     if (c->d % 128 || c->f % 128) return MOE_ERR_UNSUPPORTED_SHAPE;
@@ -43,8 +44,17 @@ bool tensor_ok(const moe_w8a8_weights* w) { return w->tmaps_ok && tc_supported(w
 
 int choose_path(const moe_w8a8_weights* w, int T) {
     if (w->path != MOE_PATH_AUTO) return w->path;
+    if (w->cfg.expert_format == MOE_FMT_E4M3) return MOE_PATH_TENSOR;   // no streaming FP8 path
     if (!tensor_ok(w)) return MOE_PATH_STREAM;
     return (int64_t)T * w->cfg.top_k <= w->stream_max_rows ? MOE_PATH_STREAM : MOE_PATH_TENSOR;
+}
+
+// The chosen path can run this handle: the tensor path needs its tensor maps
+// and shape, the streaming path INT8 experts.
+bool path_ok(const moe_w8a8_weights* w, int T) {
+    const int path = choose_path(w, T);
+    if (path == MOE_PATH_TENSOR) return tensor_ok(w);
+    return w->cfg.expert_format == MOE_FMT_INT8;
 }
 
 void prof_free(moe_w8a8_weights* w) {
@@ -213,11 +223,12 @@ moe_status moe_w8a8_prepare(const moe_w8a8_config* cfg, const float* w_gate, con
         cudaMemcpyAsync(w->inv_s, inv.data(), (size_t)d * 4, cudaMemcpyHostToDevice, s) != cudaSuccess)
         return fail(MOE_ERR_CUDA);
     // gate -> rows [blk*256, blk*256+128), up -> rows [blk*256+128, blk*256+256)
+    const int fmt = c.expert_format;
     if (launch_quantize_channels(w_gate, s_dev, E, d, f, w->w_gu, 2 * f, kGuBlock, 2 * kGuBlock, 0,
-                                 w->sw_gate, s) != cudaSuccess ||
+                                 w->sw_gate, fmt, s) != cudaSuccess ||
         launch_quantize_channels(w_up, s_dev, E, d, f, w->w_gu, 2 * f, kGuBlock, 2 * kGuBlock,
-                                 kGuBlock, w->sw_up, s) != cudaSuccess ||
-        launch_quantize_channels(w_down, nullptr, E, f, d, w->w_dn, d, d, d, 0, w->sw_dn, s) !=
+                                 kGuBlock, w->sw_up, fmt, s) != cudaSuccess ||
+        launch_quantize_channels(w_down, nullptr, E, f, d, w->w_dn, d, d, d, 0, w->sw_dn, fmt, s) !=
             cudaSuccess ||
         cudaMemcpyAsync(w->w_router, w_router, (size_t)d * E * 4, cudaMemcpyDeviceToDevice, s) !=
             cudaSuccess ||
@@ -297,7 +308,8 @@ static moe_status forward_impl(const moe_w8a8_weights* w, const void* x, int T, 
     }
     if (path == MOE_PATH_STREAM) {
         mark(MOE_STAGE_QUANT, 0);
-        CUDA_TRY(launch_smooth_quant(x, c.in_dtype, w->inv_s, w->act_clip, T, d, k, ts2row, xq, sx, nullptr, s));
+        CUDA_TRY(launch_smooth_quant(x, c.in_dtype, w->inv_s, w->act_clip, T, d, k, ts2row, xq, sx, nullptr,
+                                     MOE_FMT_INT8, s));
         mark(MOE_STAGE_QUANT, 1);
         int32_t* acc1 = (int32_t*)P(L.acc1);
         mark(MOE_STAGE_GEMM1, 0);
@@ -316,14 +328,16 @@ static moe_status forward_impl(const moe_w8a8_weights* w, const void* x, int T, 
     } else {
         int8_t* aq = (int8_t*)P(L.aq);
         mark(MOE_STAGE_QUANT, 0);
-        CUDA_TRY(launch_smooth_quant(x, c.in_dtype, w->inv_s, w->act_clip, T, d, k, ts2row, xq, sx, aq, s));
+        CUDA_TRY(launch_smooth_quant(x, c.in_dtype, w->inv_s, w->act_clip, T, d, k, ts2row, xq, sx, aq,
+                                     c.expert_format, s));
         mark(MOE_STAGE_QUANT, 1);
         mark(MOE_STAGE_GEMM1, 0);
         CUDA_TRY(launch_tc_gemm1(w, T, aq, meta, tiles, offsets, row2ts, sx, (float*)P(L.h32),
                                  (float*)P(L.pamax), dbg ? dbg->acc1 : nullptr, s));
         mark(MOE_STAGE_GEMM1, 1);
         mark(MOE_STAGE_REQUANT, 0);
-        CUDA_TRY(launch_requant((float*)P(L.h32), (float*)P(L.pamax), f, meta, (int)tk, hq, sh, s));
+        CUDA_TRY(launch_requant((float*)P(L.h32), (float*)P(L.pamax), f, meta, (int)tk, hq, sh, c.expert_format,
+                                s));
         mark(MOE_STAGE_REQUANT, 1);
         mark(MOE_STAGE_GEMM2, 0);
         CUDA_TRY(launch_tc_gemm2(w, T, hq, sh, meta, tiles, offsets, row2ts, wts, o,
@@ -363,7 +377,7 @@ moe_status moe_w8a8_forward(const moe_w8a8_weights* w, const void* x, int32_t T,
     if (T == 0) return MOE_OK;
     if (!x || !y || !workspace) return MOE_ERR_INVALID_ARG;
     if ((uintptr_t)workspace % kAlign) return MOE_ERR_INVALID_ARG;
-    if (choose_path(w, T) == MOE_PATH_TENSOR && !tensor_ok(w)) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (!path_ok(w, T)) return MOE_ERR_UNSUPPORTED_SHAPE;
     if (workspace_bytes < ws_layout(w, T).total) return MOE_ERR_WORKSPACE_TOO_SMALL;
     return forward_impl(w, x, T, router_bias, router_logits, y, (char*)workspace, dbg,
                         (cudaStream_t)stream);
@@ -377,7 +391,7 @@ moe_status moe_w8a8_forward_host(const moe_w8a8_weights* w, const void* x_host, 
     if (T == 0) return MOE_OK;
     if (!x_host || !y_host || !workspace) return MOE_ERR_INVALID_ARG;
     if ((uintptr_t)workspace % kAlign) return MOE_ERR_INVALID_ARG;
-    if (choose_path(w, T) == MOE_PATH_TENSOR && !tensor_ok(w)) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (!path_ok(w, T)) return MOE_ERR_UNSUPPORTED_SHAPE;
     const WsLayout L = ws_layout(w, T);
     if (workspace_bytes < L.total) return MOE_ERR_WORKSPACE_TOO_SMALL;
     const moe_w8a8_config& c = w->cfg;
@@ -581,7 +595,7 @@ extern "C" moe_status moe_w8a8_forward_noalloc(const moe_w8a8_weights* w, const 
     if (!w || T < 0) return MOE_ERR_INVALID_ARG;
     if (T == 0) return MOE_OK;
     if (!x || !y) return MOE_ERR_INVALID_ARG;
-    if (choose_path(w, T) == MOE_PATH_TENSOR && !tensor_ok(w)) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (!path_ok(w, T)) return MOE_ERR_UNSUPPORTED_SHAPE;
     if (ws_layout(w, T).total > (size_t)MOE_NOALLOC_SCRATCH_BYTES) return MOE_ERR_WORKSPACE_TOO_SMALL;
     void* scratch = noalloc_scratch_for_current_device();
     if (!scratch) return MOE_ERR_CUDA;
