@@ -37,8 +37,10 @@ INT8_PER_BF16 = 2.0   # nominal dense ratio (4.5 POPS int8 / 2.25 PFLOPS bf16)
 # DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum) of the dominant
 # kernel, from one ncu capture of the current kernel source (see profiles/).
 TRAFFIC = {
-    ("decode", 32, "tc_gemm_kernel<0>"): 706.834176e6 + 4.643584e6,
+    ("decode", 32, "tc_ffn_fused_kernel"): 1060.688e6 + 6.212096e6,
 }
+
+FUSED_MAX_ROWS = 512   # T*k at or below which the tensor path runs GEMM1 + requant + GEMM2 as one launch
 
 
 def parse():
@@ -156,7 +158,8 @@ def algorithmic(wl: synth.Workload, n_active: int, R: int, tensor: bool = False)
     intermediates excluded.  Per GEMM launch: the weights of the active experts
     plus that launch's own inputs and outputs (streaming path: A rows and the
     INT32 accumulators; tensor path: sorted A rows, fp32 h + partial maxima for
-    GEMM1, h codes and fp32 expert outputs for GEMM2)."""
+    GEMM1, h codes and fp32 expert outputs for GEMM2; the fused launch of few-row
+    batches: the sum of the two)."""
     in_b = 2 if wl.in_bf16 else 4
     w_bytes = n_active * 3 * wl.d * wl.f
     scales = n_active * (2 * wl.f + wl.d) * 4
@@ -168,7 +171,9 @@ def algorithmic(wl: synth.Workload, n_active: int, R: int, tensor: bool = False)
         gemm1 = n_active * 2 * wl.f * wl.d + wl.T * wl.d + R * 2 * wl.f * 4
     gemm2 = n_active * wl.d * wl.f + R * wl.f + R * wl.d * 4 + n_active * wl.d * 4
     ops = 2 * R * 3 * wl.d * wl.f
-    return dict(layer_bytes=layer, gemm1_bytes=gemm1, gemm2_bytes=gemm2, int8_ops=ops)
+    # the fused launch (GEMM1 + requantisation + GEMM2): both GEMMs' bytes
+    return dict(layer_bytes=layer, gemm1_bytes=gemm1, gemm2_bytes=gemm2, fused_bytes=gemm1 + gemm2,
+                int8_ops=ops)
 
 
 # ------------------------------------------------------------------ distributed plumbing
@@ -335,6 +340,7 @@ def measure(args, wl, world, rank, local, e2e_on=True, wts=None):
     counts = np.diff(offs.cpu().numpy())
     n_active, R = int((counts > 0).sum()), int(counts.sum())
     tensor = args.path == "tensor" or (args.path == "auto" and (fp8 or T * wl.k > 32))
+    fused = tensor and T * wl.k <= FUSED_MAX_ROWS
     alg = algorithmic(wl, n_active, R, tensor)
 
     stream = torch.cuda.current_stream(dev)
@@ -410,6 +416,8 @@ def measure(args, wl, world, rank, local, e2e_on=True, wts=None):
                   ("stream_gateup_kernel" if dom == "gemm1" else "stream_down_kernel"))
         ops = 2 * R * (2 * wl.f if dom == "gemm1" else wl.f) * wl.d
         nbytes = alg[f"{dom}_bytes"]
+        if fused:
+            kernel, ops, nbytes = "tc_ffn_fused_kernel", alg["int8_ops"], alg["fused_bytes"]
         # the bound is whichever of the byte time and the INT8 op time is larger
         if ops / (int8_peak * 1e12) > nbytes / (peaks["hbm_gbs"] * 1e9):
             achieved = ops / (dom_ms / 1e3) / 1e12

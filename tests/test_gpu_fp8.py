@@ -140,8 +140,9 @@ def run_fp8(M, wl, wts=None, data=None, W=None, prep=None, tokens=None):
     return compare_fp8(wl, prep, rt, dbg, y, y_ref, odbg, toks, bias=data.router_bias)
 
 
-@pytest.mark.parametrize("T", [64, 1, 200])
+@pytest.mark.parametrize("T", [64, 1, 200, 300])
 def test_fp8_tiny_layer(M, T):
+    # T*k = 128, 2, 400 rows run the fused expert launch, 600 the separate ones
     wl = dataclasses.replace(synth.WORKLOADS["tiny"], T=T, data_seed=400 + T)
     run_fp8(M, wl)
 

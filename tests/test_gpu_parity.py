@@ -256,8 +256,11 @@ def test_tensor_path_capacity_and_skew(M):
     assert (rt.ts2row < 0).sum() > 0
 
 
-def test_tensor_path_all_tokens_one_expert(M):
-    T, E = 700, 8
+@pytest.mark.parametrize("T", [700, 200])
+def test_tensor_path_all_tokens_one_expert(M, T):
+    """Two experts take every token: several 128-row tiles per expert, through
+    the separate GEMM launches (T=700) and the fused one (T=200, 400 rows)."""
+    E = 8
     logits = np.zeros((T, E), np.float32)
     logits[:, 2] = 3.0
     logits[:, 7] = 2.0

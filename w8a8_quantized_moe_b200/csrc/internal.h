@@ -53,6 +53,8 @@ struct WsLayout {
     size_t xq, sx, aq;
     size_t acc1, hq, sh, o;
     size_t h32, pamax;           // tensor path: fp32 h, per-row partial maxima
+    size_t fused_sync;           // fused tensor launch: its counters and queue (cleared per forward)
+    int fused_words;             // their number (0: no fused launch)
     size_t total;
 };
 WsLayout ws_layout(const moe_w8a8_weights* w, int T);
@@ -86,7 +88,7 @@ bool route_small_ok(int T, int k);
 cudaError_t launch_route_small(const float* logits, const float* bias, int T, int E, int k,
                                int renorm, int cap, int32_t* idx, float* wts, float* logits_out,
                                int32_t* offsets, int32_t* row2ts, int32_t* ts2row, int32_t* meta,
-                               int32_t* active, int32_t* tiles, cudaStream_t s);
+                               int32_t* active, int32_t* tiles, int32_t* zero_words, int n_zero, cudaStream_t s);
 // act_clip > 0 caps each token's range (saturating clip), 0 = off.
 cudaError_t launch_smooth_quant(const void* x, int in_dtype, const float* inv_s, float act_clip, int T,
                                 int d, int k, const int32_t* ts2row, int8_t* xq, float* sx, int8_t* aq,
@@ -120,6 +122,16 @@ cudaError_t launch_tc_gemm2(const moe_w8a8_weights* w, int T, const int8_t* hq, 
                             const int32_t* meta, const int32_t* tiles, const int32_t* offsets,
                             const int32_t* row2ts, const float* topk_w, float* o, int32_t* acc_dbg,
                             cudaStream_t s);
+
+// GEMM1 + requantisation of h + GEMM2 in one persistent launch (few rows per
+// expert).  sync_words: fused_sync_words(max m-tiles) words, zeroed before the launch.
+cudaError_t launch_tc_ffn_fused(const moe_w8a8_weights* w, int T, const int8_t* aq, const int32_t* meta,
+                                const int32_t* tiles, const int32_t* offsets, const int32_t* row2ts,
+                                const float* sx, const float* topk_w, float* h32, float* pamax, int8_t* hq,
+                                float* sh, float* o, int32_t* acc1_dbg, int32_t* acc2_dbg, int32_t* sync_words,
+                                cudaStream_t s);
+inline size_t fused_sync_words(size_t max_mtiles) { return 3 * max_mtiles + 2; }
+constexpr int kFusedMaxRows = 512;   // T*k at or below which the tensor path runs the fused launch
 
 cudaError_t launch_combine(const float* o, const int32_t* ts2row, int T, int k, int d,
                            int out_dtype, void* y, cudaStream_t s);

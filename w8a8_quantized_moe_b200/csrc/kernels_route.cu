@@ -567,9 +567,11 @@ __global__ void __launch_bounds__(kRouteSmallThreads) route_small_kernel(
     int renorm, int cap, int32_t* __restrict__ idx, float* __restrict__ wts,
     float* __restrict__ logits_out, int32_t* __restrict__ offsets, int32_t* __restrict__ row2ts,
     int32_t* __restrict__ ts2row, int32_t* __restrict__ meta, int32_t* __restrict__ active,
-    int32_t* __restrict__ tiles) {
+    int32_t* __restrict__ tiles, int32_t* __restrict__ zero_words, int n_zero) {
     pdl_wait();
     pdl_trigger();
+    // counters a later kernel of this forward starts from zero (the fused expert launch)
+    for (int i = threadIdx.x; i < n_zero; i += blockDim.x) zero_words[i] = 0;
 
     extern __shared__ __align__(16) uint8_t smem_raw[];
     RouteSmallSmem& sm = *reinterpret_cast<RouteSmallSmem*>(smem_raw);
@@ -723,7 +725,8 @@ bool route_small_ok(int T, int k) { return (int64_t)T * k <= kRouteSmallMax; }
 cudaError_t launch_route_small(const float* logits, const float* bias, int T, int E, int k,
                                int renorm, int cap, int32_t* idx, float* wts, float* logits_out,
                                int32_t* offsets, int32_t* row2ts, int32_t* ts2row, int32_t* meta,
-                               int32_t* active, int32_t* tiles, cudaStream_t s) {
+                               int32_t* active, int32_t* tiles, int32_t* zero_words, int n_zero,
+                               cudaStream_t s) {
     static bool attr = false;
     if (!attr) {
         cudaError_t e = cudaFuncSetAttribute(route_small_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -733,7 +736,7 @@ cudaError_t launch_route_small(const float* logits, const float* bias, int T, in
     }
     return launch_pdl(route_small_kernel, dim3(1), dim3(kRouteSmallThreads), sizeof(RouteSmallSmem), s, logits,
                       bias, T, E, k, renorm, cap, idx, wts, logits_out, offsets, row2ts, ts2row, meta,
-                      active, tiles);
+                      active, tiles, zero_words, n_zero);
 }
 
 cudaError_t launch_smooth_quant(const void* x, int in_dtype, const float* inv_s, float act_clip, int T,

@@ -499,6 +499,320 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
+// ------------------------------------------------------------------ fused expert FFN (few rows)
+
+// Requantise the rows [row0, row0 + nrows) of h with one warp: the same
+// arithmetic as requant_kernel (sh = max of the row's partial maxima / qmax,
+// codes of h / sh).  Reads through L2 (other CTAs wrote h and the maxima).
+// Lane r finds the scale of rows r, r + 32, ... (kept in `scales`, nrows <=
+// 128); then one flat pass over the rows' h with 8 x 16-byte loads per lane
+// in flight, so a few rows cost a few L2 round trips in total.
+template <int FMT>
+__device__ void requant_rows_warp(const float* h32, const float* pamax, int f, int row0, int nrows, int8_t* hq,
+                                  float* sh, float* scales, int lane) {
+    constexpr int kB = 8;
+    const int npart = f / 64, n4 = f / 4;
+    for (int r = lane; r < nrows; r += 32) {
+        const float* pm = pamax + (int64_t)(row0 + r) * npart;
+        float m = 0.0f;
+        for (int i = 0; i < npart; ++i) m = fmaxf(m, __ldcg(pm + i));
+        const float s = m > 0.0f ? __fdiv_rn(m, fmt_qmax<FMT>()) : 0.0f;
+        scales[r] = s;
+        sh[row0 + r] = s;
+    }
+    __syncwarp();
+    const int total = nrows * n4;   // float4 groups of all rows
+    const float4* h4 = reinterpret_cast<const float4*>(h32 + (int64_t)row0 * f);
+    uint32_t* q4 = reinterpret_cast<uint32_t*>(hq + (int64_t)row0 * f);
+    for (int b = 0; b < total; b += 32 * kB) {
+        float4 h[kB];
+#pragma unroll
+        for (int i = 0; i < kB; ++i)
+            if (b + lane + 32 * i < total) h[i] = __ldcg(h4 + b + lane + 32 * i);
+#pragma unroll
+        for (int i = 0; i < kB; ++i) {
+            const int j = b + lane + 32 * i;
+            if (j < total) {
+                const float s = scales[j / n4];
+                const float rs = s > 0.0f ? __frcp_rn(s) : 0.0f;
+                q4[j] = s > 0.0f ? pack4((int)fmt_code<FMT>(h[i].x, s, rs), (int)fmt_code<FMT>(h[i].y, s, rs),
+                                         (int)fmt_code<FMT>(h[i].z, s, rs), (int)fmt_code<FMT>(h[i].w, s, rs))
+                                 : 0u;
+            }
+        }
+    }
+}
+
+__device__ __forceinline__ int atom_add_acq_rel(int32_t* p, int v) {
+    int old;
+    asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+    return old;
+}
+__device__ __forceinline__ int ld_acquire(const int32_t* p) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ void st_release(int32_t* p, int v) {
+    asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+// Orders this thread's generic-proxy global accesses with its async-proxy
+// (TMA) ones: after h codes are stored (before they are released), and after
+// they are acquired (before a TMA load reads them).
+__device__ __forceinline__ void fence_proxy_async_global() {
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+struct FusedExtra {
+    int32_t* count;   // [m-tiles] GEMM1 epilogue-warp arrivals
+    int32_t* ready;   // [m-tiles] 1 once the m-tile's h codes are written
+    int32_t* queue;   // [m-tiles] m-tiles whose h is complete, + 1, in completion order
+    int32_t* qtail;   // next free queue slot
+    int32_t* qhead;   // next queue slot a requantisation warp takes
+    int8_t* hq;       // [rows][f] h codes
+    float* sh;        // [rows] h scales
+};                    // (count, ready, queue, qtail, qhead zeroed before the launch)
+
+constexpr int kFusedThreads = kThreads + 32;   // + one requantisation warp (warp 10)
+constexpr size_t kFusedSmemBytes = kSmemBytes + kEpiStageBytes;
+
+// GEMM1 (gate/up + SwiGLU), the row-wise requantisation of h and GEMM2 (down)
+// in one persistent launch, for launches with few rows per expert (decode),
+// where both GEMMs stream weights and a separate GEMM2 launch would wait for
+// the partial last wave of GEMM1 to drain.  One tile index space: GEMM1 tiles
+// (m-tile x 256 gate/up columns) first, then GEMM2 tiles (m-tile x 256 output
+// columns), dealt round robin, so the SMs idle in GEMM1's last wave start on
+// GEMM2 tiles at once.  Dependencies are per m-tile (one expert's rows): every
+// epilogue warp that finishes a GEMM1 tile adds one to count[m]; the warp that
+// brings it to (GEMM1 column tiles x epilogue warps) appends m to a device-wide
+// queue.  Warp 10 of every CTA takes queue slots in turn, requantises that
+// m-tile's rows and releases ready[m], so requantisation runs on otherwise idle
+// warps of many CTAs and never delays an epilogue (when the epilogue warp that
+// completed an m-tile requantised it itself, it fell behind, became the last
+// arrival again, and the delays piled up).  The producer of a GEMM2 tile waits
+// for ready[m] (bounded) before loading its h codes.  A CTA's GEMM1 tiles all
+// come before its GEMM2 tiles, GEMM1 tiles wait on nothing, and the requant
+// warps wait only on GEMM1 tiles, so with every CTA resident the waits always
+// end.  Arithmetic per element is that of the two separate kernels and
+// requant_kernel, so the results are identical.
+template <int FMT>
+__global__ void __launch_bounds__(kFusedThreads, 1)
+    tc_ffn_fused_kernel(const __grid_constant__ CUtensorMap tm_a1, const __grid_constant__ CUtensorMap tm_b1,
+                        const __grid_constant__ CUtensorMap tm_a2, const __grid_constant__ CUtensorMap tm_b2,
+                        const TcParams p1, const TcParams p2, const FusedExtra fx) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    float* epi_stage = reinterpret_cast<float*>(smem + kStages * kStageBytes);
+    // the requantisation warp's scale buffer follows the epilogue warps' staging buffers
+    Ctl* ctl = reinterpret_cast<Ctl*>(smem + kStages * kStageBytes + (kEpiWarps + 1) * kEpiStageBytes);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&ctl->full[s], 1);
+            mbar_init(&ctl->empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&ctl->acc_full[b], 1);
+            mbar_init(&ctl->acc_empty[b], kEpiWarps);
+        }
+        mbar_init(&ctl->drain, 1);
+        ctl->abort = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         smem_u32(&ctl->tmem_base)),
+                     "r"(kTmemCols));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = ctl->tmem_base;
+    volatile int* abort = &ctl->abort;
+    pdl_wait();
+    pdl_trigger();
+    const int n_mt = p1.meta[META_NTILES];
+    const int w1 = n_mt * p1.n_tiles_n;
+    const int num_tiles = w1 + n_mt * p2.n_tiles_n;
+    const int arrivals = p1.n_tiles_n * kEpiWarps;   // per m-tile, when its h is complete
+
+    // tile t -> (first GEMM?, m-tile, column tile)
+    auto decode = [&](int t, bool& g1, int& mt, int& nt) {
+        g1 = t < w1;
+        const int u = g1 ? t : t - w1;
+        const int nn = g1 ? p1.n_tiles_n : p2.n_tiles_n;
+        mt = u / nn;
+        nt = u % nn;
+    };
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // ---------------- TMA producer
+            int s = 0;
+            uint32_t ph = 0;
+            uint32_t issued_par[kStages];
+            bool issued[kStages];
+            for (int i = 0; i < kStages; ++i) issued[i] = false;
+            bool ok = true;
+            for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+                bool g1;
+                int mt, nt;
+                decode(t, g1, mt, nt);
+                const TcParams& p = g1 ? p1 : p2;
+                const CUtensorMap* ma = g1 ? &tm_a1 : &tm_a2;
+                const CUtensorMap* mb = g1 ? &tm_b1 : &tm_b2;
+                const int e = p.tiles[2 * mt], row0 = p.tiles[2 * mt + 1];
+                const int brow = e * p.N + nt * BN;
+                if (!g1) {
+                    // this m-tile's h codes must be written before they are loaded
+                    const uint64_t t0 = global_timer();
+                    while (ld_acquire(fx.ready + mt) == 0) {
+                        if (*abort) { ok = false; break; }
+                        if (global_timer() - t0 > kWaitBudgetNs) {
+                            *abort = 1;
+                            report_timeout(p.status, 6, t, mt);
+                            ok = false;
+                            break;
+                        }
+                    }
+                    if (!ok) break;
+                    fence_proxy_async_global();
+                }
+                const int nkb = p.K / BK;
+                for (int kb = 0; kb < nkb; ++kb) {
+                    if (!mbar_wait(&ctl->empty[s], ph ^ 1, abort, p.status, 1, t)) { ok = false; break; }
+                    mbar_arrive_expect_tx(&ctl->full[s], kStageBytes);
+                    uint8_t* sa = smem + s * kStageBytes;
+                    tma_load_2d(sa, ma, &ctl->full[s], kb * BK, row0);
+                    tma_load_2d(sa + kABytes, mb, &ctl->full[s], kb * BK, brow);
+                    issued[s] = true;
+                    issued_par[s] = ph;
+                    if (++s == kStages) { s = 0; ph ^= 1; }
+                }
+            }
+            for (int i = 0; i < kStages; ++i) {
+                if (!issued[i]) continue;
+                const uint64_t t0 = global_timer();
+                while (!mbar_try_wait(&ctl->full[i], issued_par[i]) && global_timer() - t0 < kWaitBudgetNs) {}
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            // ---------------- MMA issuer
+            int s = 0, buf = 0;
+            uint32_t ph = 0, aph = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+                const int nkb = (t < w1 ? p1.K : p2.K) / BK;
+                if (!mbar_wait(&ctl->acc_empty[buf], aph ^ 1, abort, p1.status, 2, t)) break;
+                tc_fence_after();
+                const uint32_t d_tmem = tmem + (uint32_t)(buf * BN);
+                for (int kb = 0; kb < nkb; ++kb) {
+                    if (!mbar_wait(&ctl->full[s], ph, abort, p1.status, 3, t)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t a_addr = smem_u32(smem + s * kStageBytes);
+                    const uint32_t b_addr = a_addr + kABytes;
+#pragma unroll
+                    for (int kk = 0; kk < BK / 32; ++kk)
+                        mma_8bit<FMT>(d_tmem, desc_sw128(a_addr + kk * 32), desc_sw128(b_addr + kk * 32),
+                                      (kb | kk) != 0 ? 1u : 0u);
+                    mma_commit(&ctl->empty[s]);
+                    if (++s == kStages) { s = 0; ph ^= 1; }
+                }
+                if (!ok) break;
+                mma_commit(&ctl->acc_full[buf]);
+                buf ^= 1;
+                if (buf == 0) aph ^= 1;
+            }
+            mma_commit(&ctl->drain);
+            const uint64_t t0 = global_timer();
+            while (!mbar_try_wait(&ctl->drain, 0) && global_timer() - t0 < kWaitBudgetNs) {}
+        }
+    } else if (warp == kFusedThreads / 32 - 1) {
+        // ---------------- requantisation warp: queue slots in turn
+        float* scales = epi_stage + kEpiWarps * (kEpiStageBytes / 4);
+        while (true) {
+            int i = 0;
+            if (lane == 0) i = atomicAdd(fx.qhead, 1);
+            i = __shfl_sync(0xffffffffu, i, 0);
+            if (i >= n_mt) break;
+            int v = 0;
+            if (lane == 0) {
+                const uint64_t t0 = global_timer();
+                while ((v = ld_acquire(fx.queue + i)) == 0) {
+                    if (*abort) break;
+                    if (global_timer() - t0 > kWaitBudgetNs) {
+                        *abort = 1;
+                        report_timeout(p1.status, 7, i, 0);
+                        break;
+                    }
+                    __nanosleep(64);
+                }
+            }
+            v = __shfl_sync(0xffffffffu, v, 0);
+            if (v == 0) break;
+            (void)ld_acquire(fx.queue + i);   // each lane's own acquire of the m-tile's h
+            const int mt = v - 1;
+            const int e = p1.tiles[2 * mt], row0 = p1.tiles[2 * mt + 1];
+            const int nrows = min(BM, p1.offsets[e + 1] - row0);
+            requant_rows_warp<FMT>(p1.h32, p1.pamax, p1.f, row0, nrows, fx.hq, fx.sh, scales, lane);
+            fence_proxy_async_global();
+            __threadfence();
+            __syncwarp();
+            if (lane == 0) st_release(fx.ready + mt, 1);
+        }
+    } else {
+        // ---------------- epilogue warps
+        const int ew = warp - 2;
+        const int quad = warp & 3;
+        const int half = ew >> 2;
+        float* stage = epi_stage + ew * (kEpiStageBytes / 4);
+        int buf = 0;
+        uint32_t aph = 0;
+        for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
+            if (!mbar_wait(&ctl->acc_full[buf], aph, abort, p1.status, 4, t)) break;
+            tc_fence_after();
+            bool g1;
+            int mt, nt;
+            decode(t, g1, mt, nt);
+            const TcParams& p = g1 ? p1 : p2;
+            const int e = p.tiles[2 * mt], row0 = p.tiles[2 * mt + 1];
+            const int nrows = min(BM, p.offsets[e + 1] - row0);
+            const int wrow0 = row0 + quad * 32;
+            const int nvalid = max(0, min(32, nrows - quad * 32));
+            const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(buf * BN);
+            if (g1) {
+                epilogue_swiglu<FMT>(p1, taddr, half, e, nt, wrow0, nvalid, stage, ctl, buf, lane);
+                // this warp's share of the tile is stored: count it; the last arrival requantises
+                __threadfence();
+                __syncwarp();
+                int old = 0;
+                if (lane == 0) old = atom_add_acq_rel(fx.count + mt, 1);
+                old = __shfl_sync(0xffffffffu, old, 0);
+                if (old == arrivals - 1 && lane == 0) {
+                    // the m-tile's h is complete: hand it to the requantisation warps
+                    const int slot = atomicAdd(fx.qtail, 1);
+                    st_release(fx.queue + slot, mt + 1);
+                }
+            } else {
+                (void)ld_acquire(fx.ready + mt);   // the h scales this epilogue reads were released there
+                epilogue_down<FMT>(p2, taddr, half, e, nt, wrow0, nvalid, stage, ctl, buf, lane);
+            }
+            buf ^= 1;
+            if (buf == 0) aph ^= 1;
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols));
+    }
+}
+
 // ------------------------------------------------------------------ requantisation of h
 
 // One warp per sorted row: sh = max over the row's partial maxima / 127 and
@@ -611,6 +925,66 @@ bool tc_make_weight_maps(moe_w8a8_weights* w) {
     const moe_w8a8_config& c = w->cfg;
     const uint64_t E = c.n_experts, d = c.d, f = c.f;
     return make_map(&w->tm_w_gu, w->w_gu, d, E * 2 * f, BN) && make_map(&w->tm_w_dn, w->w_dn, f, E * d, BN);
+}
+
+template <int FMT>
+cudaError_t launch_fused_fmt(const CUtensorMap& a1, const CUtensorMap& b1, const CUtensorMap& a2,
+                             const CUtensorMap& b2, const TcParams& p1, const TcParams& p2, const FusedExtra& fx,
+                             int grid, cudaStream_t s) {
+    static bool attr = false;
+    if (!attr) {
+        cudaError_t e = cudaFuncSetAttribute(tc_ffn_fused_kernel<FMT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)kFusedSmemBytes);
+        if (e != cudaSuccess) return e;
+        attr = true;
+    }
+    return launch_pdl(tc_ffn_fused_kernel<FMT>, dim3(grid), dim3(kFusedThreads), kFusedSmemBytes, s, a1, b1, a2,
+                      b2, p1, p2, fx);
+}
+
+cudaError_t launch_tc_ffn_fused(const moe_w8a8_weights* w, int T, const int8_t* aq, const int32_t* meta,
+                                const int32_t* tiles, const int32_t* offsets, const int32_t* row2ts,
+                                const float* sx, const float* topk_w, float* h32, float* pamax, int8_t* hq,
+                                float* sh, float* o, int32_t* acc1_dbg, int32_t* acc2_dbg, int32_t* sync_words,
+                                cudaStream_t s) {
+    const moe_w8a8_config& c = w->cfg;
+    const int rows = T * c.top_k;
+    CUtensorMap a1, a2;
+    if (!make_map(&a1, aq, c.d, rows, BM) || !make_map(&a2, hq, c.f, rows, BM)) return cudaErrorInvalidValue;
+    TcParams p1{}, p2{};
+    p1.N = 2 * c.f;
+    p1.K = c.d;
+    p1.n_tiles_n = p1.N / BN;
+    p2.N = c.d;
+    p2.K = c.f;
+    p2.n_tiles_n = p2.N / BN;
+    for (TcParams* p : {&p1, &p2}) {
+        p->f = c.f;
+        p->k = c.top_k;
+        p->meta = meta;
+        p->tiles = tiles;
+        p->offsets = offsets;
+        p->row2ts = row2ts;
+        p->status = w->status;
+    }
+    p1.sx = sx;
+    p1.sw0 = w->sw_gate;
+    p1.sw1 = w->sw_up;
+    p1.h32 = h32;
+    p1.pamax = pamax;
+    p1.acc_dbg = acc1_dbg;
+    p2.topk_w = topk_w;
+    p2.sw0 = w->sw_dn;
+    p2.sh = sh;
+    p2.o = o;
+    p2.acc_dbg = acc2_dbg;
+    const int max_mt = (rows + BM - 1) / BM + c.n_experts;
+    const FusedExtra fx{sync_words, sync_words + max_mt, sync_words + 2 * max_mt, sync_words + 3 * max_mt,
+                        sync_words + 3 * max_mt + 1, hq, sh};
+    const int grid = max(1, min(w->num_sms, max_mt * (p1.n_tiles_n + p2.n_tiles_n)));
+    if (c.expert_format == FMT_E4M3)
+        return launch_fused_fmt<FMT_E4M3>(a1, w->tm_w_gu, a2, w->tm_w_dn, p1, p2, fx, grid, s);
+    return launch_fused_fmt<FMT_INT8>(a1, w->tm_w_gu, a2, w->tm_w_dn, p1, p2, fx, grid, s);
 }
 
 bool tc_supported(const moe_w8a8_config& c) { return c.d % BN == 0 && c.f % BK == 0 && c.d % BK == 0; }

@@ -57,6 +57,14 @@ bool path_ok(const moe_w8a8_weights* w, int T) {
     return w->cfg.expert_format == MOE_FMT_INT8;
 }
 
+// The tensor path runs GEMM1, the requantisation of h and GEMM2 as one
+// launch when there are few rows per expert (and the routing front end is the
+// one-block kernel, which clears the launch's counters).
+bool fused_ok(const moe_w8a8_weights* w, int T) {
+    const int64_t tk = (int64_t)T * w->cfg.top_k;
+    return tk <= kFusedMaxRows && route_small_ok(T, w->cfg.top_k);
+}
+
 void prof_free(moe_w8a8_weights* w) {
     if (!w->prof_events) return;
     for (int i = 0; i < w->prof_max * MOE_N_STAGES * 2; ++i) cudaEventDestroy(w->prof_events[i]);
@@ -124,6 +132,9 @@ WsLayout ws_layout(const moe_w8a8_weights* w, int T) {
     L.o = take(tk * d * 4);
     L.h32 = take(stream ? 0 : tk * f * 4);
     L.pamax = take(stream ? 0 : tk * (f / 64) * 4);
+    const bool fused = !stream && fused_ok(w, T);
+    L.fused_sync = take(fused ? fused_sync_words(max_tiles) * 4 : 0);
+    L.fused_words = fused ? (int)fused_sync_words(max_tiles) : 0;
     L.total = p;
     return L;
 }
@@ -289,9 +300,11 @@ static moe_status forward_impl(const moe_w8a8_weights* w, const void* x, int T, 
     if (route_small_ok(T, k)) {
         // top-k, histogram, scan and scatter in one block
         mark(MOE_STAGE_TOPK, 0);
+        const bool fused = path == MOE_PATH_TENSOR && L.fused_words > 0;
         CUDA_TRY(launch_route_small(lsrc, bias, T, E, k, c.renormalize, capacity_of(c, T), idx, wts,
                                     dbg ? dbg->logits : nullptr, offsets, row2ts, ts2row, meta,
-                                    active, tiles, s));
+                                    active, tiles, fused ? (int32_t*)P(L.fused_sync) : nullptr,
+                                    fused ? L.fused_words : 0, s));
         mark(MOE_STAGE_TOPK, 1);
         empty_stage(MOE_STAGE_PERMUTE);
         ++launches;
@@ -331,19 +344,32 @@ static moe_status forward_impl(const moe_w8a8_weights* w, const void* x, int T, 
         CUDA_TRY(launch_smooth_quant(x, c.in_dtype, w->inv_s, w->act_clip, T, d, k, ts2row, xq, sx, aq,
                                      c.expert_format, s));
         mark(MOE_STAGE_QUANT, 1);
-        mark(MOE_STAGE_GEMM1, 0);
-        CUDA_TRY(launch_tc_gemm1(w, T, aq, meta, tiles, offsets, row2ts, sx, (float*)P(L.h32),
-                                 (float*)P(L.pamax), dbg ? dbg->acc1 : nullptr, s));
-        mark(MOE_STAGE_GEMM1, 1);
-        mark(MOE_STAGE_REQUANT, 0);
-        CUDA_TRY(launch_requant((float*)P(L.h32), (float*)P(L.pamax), f, meta, (int)tk, hq, sh, c.expert_format,
-                                s));
-        mark(MOE_STAGE_REQUANT, 1);
-        mark(MOE_STAGE_GEMM2, 0);
-        CUDA_TRY(launch_tc_gemm2(w, T, hq, sh, meta, tiles, offsets, row2ts, wts, o,
-                                 dbg ? dbg->acc2 : nullptr, s));
-        mark(MOE_STAGE_GEMM2, 1);
-        launches += 4;
+        if (L.fused_words > 0) {
+            // few rows per expert: GEMM1, requantisation and GEMM2 in one launch
+            // (its time is reported as the GEMM1 stage)
+            mark(MOE_STAGE_GEMM1, 0);
+            CUDA_TRY(launch_tc_ffn_fused(w, T, aq, meta, tiles, offsets, row2ts, sx, wts, (float*)P(L.h32),
+                                         (float*)P(L.pamax), hq, sh, o, dbg ? dbg->acc1 : nullptr,
+                                         dbg ? dbg->acc2 : nullptr, (int32_t*)P(L.fused_sync), s));
+            mark(MOE_STAGE_GEMM1, 1);
+            empty_stage(MOE_STAGE_REQUANT);
+            empty_stage(MOE_STAGE_GEMM2);
+            launches += 2;
+        } else {
+            mark(MOE_STAGE_GEMM1, 0);
+            CUDA_TRY(launch_tc_gemm1(w, T, aq, meta, tiles, offsets, row2ts, sx, (float*)P(L.h32),
+                                     (float*)P(L.pamax), dbg ? dbg->acc1 : nullptr, s));
+            mark(MOE_STAGE_GEMM1, 1);
+            mark(MOE_STAGE_REQUANT, 0);
+            CUDA_TRY(launch_requant((float*)P(L.h32), (float*)P(L.pamax), f, meta, (int)tk, hq, sh,
+                                    c.expert_format, s));
+            mark(MOE_STAGE_REQUANT, 1);
+            mark(MOE_STAGE_GEMM2, 0);
+            CUDA_TRY(launch_tc_gemm2(w, T, hq, sh, meta, tiles, offsets, row2ts, wts, o,
+                                     dbg ? dbg->acc2 : nullptr, s));
+            mark(MOE_STAGE_GEMM2, 1);
+            launches += 4;
+        }
     }
     mark(MOE_STAGE_COMBINE, 0);
     CUDA_TRY(launch_combine(o, ts2row, T, k, d, c.out_dtype, y, s));
