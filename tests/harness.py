@@ -48,7 +48,7 @@ def x_tensor(wl: synth.Workload, data: synth.LayerData):
 
 
 def gpu_prepare(wl: synth.Workload, wts: synth.LayerWeights, capacity_factor=None, renormalize=True,
-                fmt=0):
+                fmt=0, w_router=None):
     """Calibration absmax + prepare through the C ABI (fmt: MOE_FMT_INT8 / MOE_FMT_E4M3)."""
     import w8a8_quantized_moe_b200 as M
     torch = torch_mod()
@@ -63,7 +63,9 @@ def gpu_prepare(wl: synth.Workload, wts: synth.LayerWeights, capacity_factor=Non
         cal = to_dev(calib)
     ax = torch.zeros(wl.d, dtype=torch.float32, device="cuda")
     M.moe_w8a8_calibrate_absmax(cal, ax)
-    wr = to_dev(synth.normal(wl.data_seed, synth.TID_W_ROUTER, (wl.d, wl.E), std=wl.weight_std))
+    if w_router is None:
+        w_router = synth.normal(wl.data_seed, synth.TID_W_ROUTER, (wl.d, wl.E), std=wl.weight_std)
+    wr = to_dev(w_router)
     W = M.moe_w8a8_prepare(cfg, to_dev(wts.w_gate), to_dev(wts.w_up), to_dev(wts.w_down), wr, ax)
     torch.cuda.synchronize()
     return W
@@ -148,14 +150,35 @@ def compare_prepare(W, prep: oracle.Prepared):
             raise AssertionError(f"{name}: {len(bad)} codes differ, first at {bad[0].tolist()}")
 
 
+def certified_router(wl: synth.Workload, T: int) -> bool:
+    """Whether the library routes this batch with the certified tensor-core
+    router (computed bf16 logits, renormalised gate, at least 1024 tokens and
+    more than 2048 (token, slot) pairs)."""
+    return wl.in_bf16 and not wl.logits_uniform and T >= 1024 and T * wl.k > 2048 and wl.d % 64 == 0
+
+
+def compare_logits(wl, rt: oracle.Routing, got, bias=None):
+    """Router logits (+ bias): bit-exact, or, where the certified router ran,
+    bit-exact for every selected expert and within 1e-4 of the row's largest
+    logit elsewhere (those entries only chose the candidates)."""
+    T = rt.idx.shape[0]
+    ref_l = rt.logits if bias is None else (rt.logits + bias[None, :]).astype(np.float32)
+    if not certified_router(wl, T):
+        assert np.array_equal(got, ref_l), "router logits differ"
+        return
+    sel = np.take_along_axis(got, rt.idx, axis=1)
+    assert np.array_equal(sel, np.take_along_axis(ref_l, rt.idx, axis=1)), "selected logits differ"
+    scale = np.abs(ref_l).max(axis=1, keepdims=True)
+    assert np.all(np.abs(got - ref_l) <= 1e-4 * scale), "approximate logits out of range"
+
+
 def compare_stages(wl, rt: oracle.Routing, dbg: dict, y_gpu, y_ref, odbg: dict, tokens,
                    bias=None):
     """Bit-exact integer stages, exact float intermediates, tolerance on y."""
     T = rt.idx.shape[0]
     k = wl.k
     tokens = np.asarray(tokens, np.int64)
-    ref_l = rt.logits if bias is None else (rt.logits + bias[None, :]).astype(np.float32)
-    assert np.array_equal(dbg["logits"], ref_l), "router logits differ"
+    compare_logits(wl, rt, dbg["logits"], bias)
     assert np.array_equal(dbg["topk_idx"], rt.idx), "top-k indices differ"
     assert np.array_equal(dbg["topk_w"], rt.w), "gate weights differ"
     assert np.array_equal(dbg["offsets"], rt.offsets), "expert offsets differ"

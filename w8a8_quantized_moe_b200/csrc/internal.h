@@ -25,12 +25,23 @@ struct moe_w8a8_weights {
     float* sw_dn;     // [E][d]
     float* inv_s;     // [d]
     float* w_router;  // [d][E]
+    // certified tensor-core router (bf16 X): W_g split into bf16 hi + lo rows
+    // [rt_epad][d] (experts padded with zero rows), W_g transposed [E][d] fp32
+    // for the exact re-evaluation, and max_e |W_g[j][e]| [d]; the last two
+    // lane-interleaved (channel 32 i + p at [i / 4][p][i % 4])
+    uint16_t* rt_hi;
+    uint16_t* rt_lo;
+    float* rt_wt;
+    float* rt_wmax;
+    int rt_epad;      // 0: no tensor-core router for this handle
     float* s_host;    // [d] (host)
     int32_t* status;  // device status word
     // tensor maps of the weights for the tensor-core path (built at prepare)
     CUtensorMap tm_w_gu;
     CUtensorMap tm_w_dn;
     bool tmaps_ok;
+    CUtensorMap tm_rt_hi;
+    CUtensorMap tm_rt_lo;
     // per-stage event timing (measurement aid)
     cudaEvent_t* prof_events;   // [prof_max][MOE_N_STAGES][2]
     int prof_max;
@@ -48,6 +59,7 @@ constexpr int kMaxE = 256;
 struct WsLayout {
     size_t x_stage, y_stage, logits_stage, bias_stage;   // forward_host staging
     size_t logits, topk_idx, topk_w;
+    size_t logits_sel;           // certified router: exact-or--inf logits [T][E]
     size_t hist, offsets, meta, active, tiles;
     size_t row2ts, ts2row;
     size_t xq, sx, aq;
@@ -111,6 +123,16 @@ cudaError_t launch_stream_down(const moe_w8a8_weights* w, int T, const int8_t* h
                                float* o, int32_t* acc2_dbg, cudaStream_t s);
 // tensor-core path (kernels_tc.cu)
 bool tc_make_weight_maps(moe_w8a8_weights* w);
+// Certified tensor-core router: approximate logits l~ [T][E] from bf16 X (this
+// file's kernels_tc.cu), then per token the candidate experts within the error
+// bound, their logits in the stated fp32 order, top-k and gate weights
+// (kernels_route.cu).  sel: [T][E] scratch.
+bool router_tc_make_maps(moe_w8a8_weights* w);
+cudaError_t launch_router_tc(const moe_w8a8_weights* w, const void* x, int T, float* approx, cudaStream_t s);
+cudaError_t launch_router_select(const moe_w8a8_weights* w, const void* x, int T, const float* approx,
+                                 const float* bias, float* sel, int32_t* idx, float* wts, float* logits_out,
+                                 cudaStream_t s);
+constexpr int kRouterTcMinTokens = 1024;   // the certified router runs from this many tokens up
 bool tc_supported(const moe_w8a8_config& c);
 cudaError_t launch_tc_gemm1(const moe_w8a8_weights* w, int T, const int8_t* aq, const int32_t* meta,
                             const int32_t* tiles, const int32_t* offsets, const int32_t* row2ts,

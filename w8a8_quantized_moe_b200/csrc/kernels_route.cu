@@ -3,6 +3,8 @@
 // sort -> grouped GEMM -> un-sort -> weighted sum, with top-k routing equal to
 // the reference including its tie-break; section 2 item 2: capacity factor.
 // "MiniMax-M3 W8A8 on K100AI", s3.2 / s6.4: smoothing and per-token INT8.)
+#include <cmath>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -402,6 +404,176 @@ __global__ void topk_kernel(const float* __restrict__ logits, const float* __res
 }
 
 // ---------------------------------------------------------------------------
+// Certified router, second step (the first is router_tc_kernel: approximate
+// logits l~ from the tensor cores).  One warp per token:
+//   S = sum_j |x_j| max_e |W_g[j][e]|  bounds sum_j |x_j| |W_g[j][e]| for every e;
+//   a_e = l~_e + bias_e; v_k = the k-th largest a_e;
+//   B = c_err S + 2^-22 (max_e |a_e| + 1) bounds |a_e - l_e| for every e, l_e
+//       being the logit in the stated fp32 order (+ bias): c_err covers the bf16
+//       split of W_g (2^-16), the fp32 order's own rounding and the tensor
+//       cores' fp32 accumulation (modelled as at most 2^-21 of the running
+//       absolute sum per MMA step); the last term the two bias additions;
+//   candidates C = { e : a_e >= v_k - 2B }.
+// An expert outside C has l_e < v_k - B <= l_j for each of the k experts j with
+// the largest a_j, so it cannot be among the top k: the top k of the exact
+// logits over C alone is the top k over all experts, ties included.  The
+// candidates' logits are computed in the stated order (lane chains, xor
+// butterfly, then + bias), the others set to -inf, and topk_token chooses and
+// weighs exactly as for fully computed logits.  logits_out (debug) receives
+// exact logits for candidates and a_e for the rest.
+// ---------------------------------------------------------------------------
+constexpr int kSelWarps = 4;
+constexpr int kSelCand = 4;   // candidates evaluated together (more: further passes)
+constexpr int kSelJ = 4;      // 16-byte steps of every candidate loaded together
+
+// W_g and max|W_g| are stored lane-interleaved: element j = 32 i + p (lane p,
+// step i) of a row sits at [i / 4][p][i % 4], so lane p reads its 4 steps
+// 4j..4j+3 with one 16-byte load and a warp reads 512 contiguous bytes.
+__device__ __forceinline__ float4 ld_lane4(const float* rowbase, int j, int lane) {
+    return __ldg(reinterpret_cast<const float4*>(rowbase) + (int64_t)j * 32 + lane);
+}
+
+__global__ void __launch_bounds__(kSelWarps * 32) router_select_kernel(
+    const uint16_t* __restrict__ x, const float* __restrict__ approx, const float* __restrict__ bias,
+    const float* __restrict__ wt, const float* __restrict__ wmax, int T, int d, int E, int k, float c_err,
+    float* __restrict__ sel, int32_t* __restrict__ idx, float* __restrict__ wts, float* __restrict__ logits_out) {
+    pdl_wait();
+    pdl_trigger();
+
+    extern __shared__ __align__(16) uint8_t smem_raw[];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    uint16_t* xs = reinterpret_cast<uint16_t*>(smem_raw) + (size_t)warp * d;   // this warp's token row
+    float* lsh = reinterpret_cast<float*>(smem_raw + (size_t)kSelWarps * d * 2) + warp * kMaxE;
+    const int t = blockIdx.x * kSelWarps + warp;
+    if (t >= T) return;
+    {
+        const int4* src = reinterpret_cast<const int4*>(x + (int64_t)t * d);
+        int4* dst = reinterpret_cast<int4*>(xs);
+        for (int i = lane; i < d / 8; i += 32) dst[i] = src[i];
+        __syncwarp();
+    }
+    const int nj = d / 128;   // 16-byte steps per lane
+    float S = 0.0f;
+#pragma unroll 8
+    for (int j = 0; j < nj; ++j) {
+        const float4 m4 = ld_lane4(wmax, j, lane);
+        const float mv[4] = {m4.x, m4.y, m4.z, m4.w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) S = fmaf(fabsf(bf16_bits_to_f32(xs[32 * (4 * j + q) + lane])), mv[q], S);
+    }
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) S += __shfl_xor_sync(0xffffffffu, S, o);
+    constexpr int kPer = kMaxE / 32;
+    float a[kPer], ex[kPer];
+    bool taken[kPer];
+    float amax = 0.0f;
+#pragma unroll
+    for (int m = 0; m < kPer; ++m) {
+        const int e = lane + 32 * m;
+        a[m] = -INFINITY;
+        ex[m] = -INFINITY;
+        if (e < E) {
+            float v = approx[(int64_t)t * E + e];
+            if (bias) v = __fadd_rn(v, bias[e]);
+            a[m] = v;
+            amax = fmaxf(amax, fabsf(v));
+        }
+        taken[m] = e >= E;
+    }
+    amax = warp_max(amax);
+    float vk = 0.0f;
+    for (int s = 0; s < k; ++s) {
+        float bv = -INFINITY;
+        int bi = 0x7fffffff;
+#pragma unroll
+        for (int m = 0; m < kPer; ++m) {
+            const int e = lane + 32 * m;
+            if (!taken[m] && better(a[m], e, bv, bi)) { bv = a[m]; bi = e; }
+        }
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) {
+            const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+            const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+            if (better(ov, oi, bv, bi)) { bv = ov; bi = oi; }
+        }
+#pragma unroll
+        for (int m = 0; m < kPer; ++m)
+            if (lane + 32 * m == bi) taken[m] = true;
+        vk = bv;
+    }
+    const float B = c_err * S * (1.0f + 0x1p-10f) + 0x1p-22f * (amax + 1.0f);
+    const float thr = vk - 2.0f * B * (1.0f + 0x1p-10f);
+    unsigned cmask[kPer];
+#pragma unroll
+    for (int m = 0; m < kPer; ++m) cmask[m] = __ballot_sync(0xffffffffu, lane + 32 * m < E && a[m] >= thr);
+    // candidates in passes of kSelCand: all their chains advance together
+    int m0 = 0;
+    while (true) {
+        int ce[kSelCand];
+        int nc = 0;
+        for (; m0 < kPer && nc < kSelCand; ) {
+            if (cmask[m0] == 0u) { ++m0; continue; }
+            const int b = __ffs(cmask[m0]) - 1;
+            cmask[m0] &= cmask[m0] - 1;
+            ce[nc++] = b + 32 * m0;
+        }
+        if (nc == 0) break;
+        float acc[kSelCand];
+#pragma unroll
+        for (int c = 0; c < kSelCand; ++c) acc[c] = 0.0f;
+        for (int j0 = 0; j0 < nj; j0 += kSelJ) {
+            // all loads of kSelJ steps of every candidate first (one L2 round trip), then the
+            // FMAs, each chain in its own channel order
+            float4 w4[kSelJ][kSelCand];
+#pragma unroll
+            for (int jj = 0; jj < kSelJ; ++jj)
+#pragma unroll
+                for (int c = 0; c < kSelCand; ++c)
+                    if (c < nc && j0 + jj < nj) w4[jj][c] = ld_lane4(wt + (int64_t)ce[c] * d, j0 + jj, lane);
+#pragma unroll
+            for (int jj = 0; jj < kSelJ; ++jj) {
+                if (j0 + jj >= nj) break;
+                float xv[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) xv[q] = bf16_bits_to_f32(xs[32 * (4 * (j0 + jj) + q) + lane]);
+#pragma unroll
+                for (int c = 0; c < kSelCand; ++c) {
+                    if (c < nc) {
+                        acc[c] = __fmaf_rn(xv[0], w4[jj][c].x, acc[c]);
+                        acc[c] = __fmaf_rn(xv[1], w4[jj][c].y, acc[c]);
+                        acc[c] = __fmaf_rn(xv[2], w4[jj][c].z, acc[c]);
+                        acc[c] = __fmaf_rn(xv[3], w4[jj][c].w, acc[c]);
+                    }
+                }
+            }
+        }
+#pragma unroll
+        for (int c = 0; c < kSelCand; ++c) {
+            if (c < nc) {
+                float v = acc[c];
+#pragma unroll
+                for (int o = 16; o >= 1; o >>= 1) v = __fadd_rn(v, __shfl_xor_sync(0xffffffffu, v, o));
+                if (bias) v = __fadd_rn(v, bias[ce[c]]);
+#pragma unroll
+                for (int m = 0; m < kPer; ++m)
+                    if (ce[c] == lane + 32 * m) ex[m] = v;
+            }
+        }
+    }
+#pragma unroll
+    for (int m = 0; m < kPer; ++m) {
+        const int e = lane + 32 * m;
+        if (e < E) {
+            const bool cand = a[m] >= thr;
+            sel[(int64_t)t * E + e] = cand ? ex[m] : -INFINITY;
+            if (logits_out) logits_out[(int64_t)t * E + e] = cand ? ex[m] : a[m];
+        }
+    }
+    __syncwarp();
+    topk_token(sel, nullptr, t, E, k, 1, idx, wts, nullptr, lsh, nullptr, lane);
+}
+
+// ---------------------------------------------------------------------------
 // Sort by expert.  Entry i (= t*k + slot) of expert e gets position
 // pos = #(earlier entries of e) and is kept when pos < capacity; kept rows are
 // ordered by expert, then by i.  Large inputs: a histogram per chunk of
@@ -701,6 +873,27 @@ cudaError_t launch_router_logits(const void* x, int in_dtype, const float* wr, i
         return launch_pdl(router_logits_kernel, grid, dim3(kRtThreads), 0, s, x, in_dtype, wr, T, d, E, logits);
     }
     return cudaGetLastError();
+}
+
+cudaError_t launch_router_select(const moe_w8a8_weights* w, const void* x, int T, const float* approx,
+                                 const float* bias, float* sel, int32_t* idx, float* wts, float* logits_out,
+                                 cudaStream_t s) {
+    const int d = w->cfg.d;
+    // bf16 split of W_g (2^-16), the stated order's own rounding ((d/32 + 6) ulps), the
+    // tensor cores' accumulation: 2 x (d/16 + 1) MMA steps, 2^-21 of the running sum each
+    const double c_err = std::ldexp(1.0, -16) + (d / 32 + 6) * std::ldexp(1.0, -24) +
+                         (2.0 * (d / 16) + 2.0) * std::ldexp(1.0, -21);
+    const size_t smem = (size_t)kSelWarps * d * 2 + (size_t)kSelWarps * kMaxE * 4;
+    static bool attr = false;
+    if (!attr) {
+        cudaError_t e = cudaFuncSetAttribute(router_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)((size_t)kSelWarps * 16384 * 2 + (size_t)kSelWarps * kMaxE * 4));
+        if (e != cudaSuccess) return e;
+        attr = true;
+    }
+    return launch_pdl(router_select_kernel, dim3((T + kSelWarps - 1) / kSelWarps), dim3(kSelWarps * 32), smem, s,
+                      reinterpret_cast<const uint16_t*>(x), approx, bias, w->rt_wt, w->rt_wmax, T, d,
+                      w->cfg.n_experts, w->cfg.top_k, (float)c_err, sel, idx, wts, logits_out);
 }
 
 cudaError_t launch_topk(const float* logits, const float* bias, int T, int E, int k, int renorm,

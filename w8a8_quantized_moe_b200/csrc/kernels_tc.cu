@@ -867,6 +867,149 @@ __global__ void __launch_bounds__(kRqThreads) requant_kernel(const float* __rest
     }
 }
 
+// ------------------------------------------------------------------ approximate router logits
+
+// Approximate router logits on the tensor cores, for the certified router:
+// l~[t][e] = sum_j x[t][j] (hi[e][j] + lo[e][j]) with W_g split into two bf16
+// parts (hi = bf16(w), lo = bf16(w - hi), so |w - hi - lo| <= 2^-16 |w|),
+// tcgen05.mma kind::f16 (bf16 x bf16, fp32 accumulators in TMEM).  One CTA per
+// 128 tokens: warp 0 loads X (128 x 64 bf16) and both W parts (EPAD x 64 bf16)
+// per k-block by TMA into a ring, warp 1 issues two MMAs per 16 channels into
+// one accumulator, warps 2-5 write the EPAD columns of their 32 rows.  These
+// values only choose candidates; the logits that decide top-k and the gate
+// weights are recomputed in the stated fp32 order (router_select_kernel).
+constexpr int kRcBK = 64;                     // bf16 channels per k-block (128 bytes)
+constexpr int kRcThreads = 192;
+constexpr int kRcABytes = BM * kRcBK * 2;     // 16 KB
+
+template <int EPAD>
+struct RcCfg {
+    static constexpr int kBBytes = EPAD * kRcBK * 2;                  // one W part
+    static constexpr int kStage = kRcABytes + 2 * kBBytes;
+    static constexpr int kStages = EPAD <= 64 ? 4 : (EPAD <= 128 ? 3 : 2);
+    static constexpr size_t kSmem = (size_t)kStages * kStage + 1024 + 256;
+    // kind::f16: D = f32 (bits 4-5 = 1), A and B bf16 (bits 7-9, 10-12 = 1), K-major
+    static constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(EPAD >> 3) << 17) |
+                                       ((uint32_t)(BM >> 4) << 24);
+};
+
+__device__ __forceinline__ void mma_bf16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                         uint32_t accum) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(tmem_d),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accum));
+}
+
+template <int EPAD>
+__global__ void __launch_bounds__(kRcThreads, 1)
+    router_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_hi,
+                     const __grid_constant__ CUtensorMap tm_lo, int T, int d, int E, float* __restrict__ approx,
+                     int32_t* status) {
+    using C = RcCfg<EPAD>;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    Ctl* ctl = reinterpret_cast<Ctl*>(smem + C::kStages * C::kStage);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int t0 = blockIdx.x * BM;
+    const int nkb = d / kRcBK;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::kStages; ++s) {
+            mbar_init(&ctl->full[s], 1);
+            mbar_init(&ctl->empty[s], 1);
+        }
+        mbar_init(&ctl->acc_full[0], 1);
+        mbar_init(&ctl->drain, 1);
+        ctl->abort = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         smem_u32(&ctl->tmem_base)),
+                     "r"((uint32_t)EPAD));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = ctl->tmem_base;
+    volatile int* abort = &ctl->abort;
+    pdl_wait();
+    pdl_trigger();
+
+    if (warp == 0) {
+        if (lane == 0) {
+            int s = 0;
+            uint32_t ph = 0;
+            uint32_t issued_par[4];
+            bool issued[4] = {false, false, false, false};
+            for (int kb = 0; kb < nkb; ++kb) {
+                if (!mbar_wait(&ctl->empty[s], ph ^ 1, abort, status, 11, kb)) break;
+                mbar_arrive_expect_tx(&ctl->full[s], C::kStage);
+                uint8_t* sa = smem + s * C::kStage;
+                tma_load_2d(sa, &tm_x, &ctl->full[s], kb * kRcBK, t0);
+                tma_load_2d(sa + kRcABytes, &tm_hi, &ctl->full[s], kb * kRcBK, 0);
+                tma_load_2d(sa + kRcABytes + C::kBBytes, &tm_lo, &ctl->full[s], kb * kRcBK, 0);
+                issued[s] = true;
+                issued_par[s] = ph;
+                if (++s == C::kStages) { s = 0; ph ^= 1; }
+            }
+            for (int i = 0; i < C::kStages; ++i) {
+                if (!issued[i]) continue;
+                const uint64_t tw = global_timer();
+                while (!mbar_try_wait(&ctl->full[i], issued_par[i]) && global_timer() - tw < kWaitBudgetNs) {}
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            int s = 0;
+            uint32_t ph = 0;
+            bool ok = true;
+            for (int kb = 0; kb < nkb; ++kb) {
+                if (!mbar_wait(&ctl->full[s], ph, abort, status, 12, kb)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t a_addr = smem_u32(smem + s * C::kStage);
+                const uint32_t hi_addr = a_addr + kRcABytes, lo_addr = hi_addr + C::kBBytes;
+#pragma unroll
+                for (int kk = 0; kk < kRcBK / 16; ++kk) {
+                    mma_bf16(tmem, desc_sw128(a_addr + kk * 32), desc_sw128(hi_addr + kk * 32), C::kIdesc,
+                             (kb | kk) != 0 ? 1u : 0u);
+                    mma_bf16(tmem, desc_sw128(a_addr + kk * 32), desc_sw128(lo_addr + kk * 32), C::kIdesc, 1u);
+                }
+                mma_commit(&ctl->empty[s]);
+                if (++s == C::kStages) { s = 0; ph ^= 1; }
+            }
+            if (ok) mma_commit(&ctl->acc_full[0]);
+            mma_commit(&ctl->drain);
+            const uint64_t tw = global_timer();
+            while (!mbar_try_wait(&ctl->drain, 0) && global_timer() - tw < kWaitBudgetNs) {}
+        }
+    } else {
+        // warps 2..5: TMEM lane quarter warp % 4 = 32 tokens each
+        const int quad = warp & 3;
+        if (mbar_wait(&ctl->acc_full[0], 0, abort, status, 13, 0)) {
+            tc_fence_after();
+            const int t = t0 + quad * 32 + lane;
+#pragma unroll 1
+            for (int c0 = 0; c0 < EPAD; c0 += 32) {
+                uint32_t v[32];
+                tmem_ld32(tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)c0, v);
+                tmem_ld_wait();
+                if (t < T)
+                    for (int j = 0; j < 32; ++j)
+                        if (c0 + j < E) approx[(int64_t)t * E + c0 + j] = __uint_as_float(v[j]);
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"((uint32_t)EPAD));
+    }
+}
+
 // ------------------------------------------------------------------ host side
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -898,6 +1041,35 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t K, uint64_t rows, uint3
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 2-D map over a bf16 [rows][K] K-major matrix, box = box_rows x 64 elements
+// (128 bytes), 128-byte swizzle.
+bool make_map_bf16(CUtensorMap* m, const void* base, uint64_t K, uint64_t rows, uint32_t box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[2] = {K, rows};
+    const cuuint64_t strides[1] = {K * 2};
+    const cuuint32_t box[2] = {(cuuint32_t)kRcBK, box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int EPAD>
+cudaError_t launch_router_tc_pad(const CUtensorMap& mx, const moe_w8a8_weights* w, int T, float* approx,
+                                 cudaStream_t s) {
+    using C = RcCfg<EPAD>;
+    static bool attr = false;
+    if (!attr) {
+        cudaError_t e = cudaFuncSetAttribute(router_tc_kernel<EPAD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)C::kSmem);
+        if (e != cudaSuccess) return e;
+        attr = true;
+    }
+    return launch_pdl(router_tc_kernel<EPAD>, dim3((T + BM - 1) / BM), dim3(kRcThreads), C::kSmem, s, mx,
+                      w->tm_rt_hi, w->tm_rt_lo, T, w->cfg.d, w->cfg.n_experts, approx, w->status);
 }
 
 template <int EPI, int FMT>
@@ -985,6 +1157,22 @@ cudaError_t launch_tc_ffn_fused(const moe_w8a8_weights* w, int T, const int8_t* 
     if (c.expert_format == FMT_E4M3)
         return launch_fused_fmt<FMT_E4M3>(a1, w->tm_w_gu, a2, w->tm_w_dn, p1, p2, fx, grid, s);
     return launch_fused_fmt<FMT_INT8>(a1, w->tm_w_gu, a2, w->tm_w_dn, p1, p2, fx, grid, s);
+}
+
+bool router_tc_make_maps(moe_w8a8_weights* w) {
+    return make_map_bf16(&w->tm_rt_hi, w->rt_hi, w->cfg.d, w->rt_epad, w->rt_epad) &&
+           make_map_bf16(&w->tm_rt_lo, w->rt_lo, w->cfg.d, w->rt_epad, w->rt_epad);
+}
+
+cudaError_t launch_router_tc(const moe_w8a8_weights* w, const void* x, int T, float* approx, cudaStream_t s) {
+    CUtensorMap mx;
+    if (!make_map_bf16(&mx, x, w->cfg.d, T, BM)) return cudaErrorInvalidValue;
+    switch (w->rt_epad) {
+        case 64: return launch_router_tc_pad<64>(mx, w, T, approx, s);
+        case 128: return launch_router_tc_pad<128>(mx, w, T, approx, s);
+        case 256: return launch_router_tc_pad<256>(mx, w, T, approx, s);
+    }
+    return cudaErrorInvalidValue;
 }
 
 bool tc_supported(const moe_w8a8_config& c) { return c.d % BN == 0 && c.f % BK == 0 && c.d % BK == 0; }

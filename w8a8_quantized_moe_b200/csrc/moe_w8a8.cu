@@ -60,6 +60,12 @@ bool path_ok(const moe_w8a8_weights* w, int T) {
 // The tensor path runs GEMM1, the requantisation of h and GEMM2 as one
 // launch when there are few rows per expert (and the routing front end is the
 // one-block kernel, which clears the launch's counters).
+// The certified tensor-core router serves large batches with computed logits
+// (the one-block routing front end keeps the FMA router).
+bool router_tc_ok(const moe_w8a8_weights* w, int T) {
+    return w->rt_epad > 0 && T >= kRouterTcMinTokens && !route_small_ok(T, w->cfg.top_k);
+}
+
 bool fused_ok(const moe_w8a8_weights* w, int T) {
     const int64_t tk = (int64_t)T * w->cfg.top_k;
     return tk <= kFusedMaxRows && route_small_ok(T, w->cfg.top_k);
@@ -83,6 +89,10 @@ void free_handle(moe_w8a8_weights* w) {
     cudaFree(w->sw_dn);
     cudaFree(w->inv_s);
     cudaFree(w->w_router);
+    cudaFree(w->rt_hi);
+    cudaFree(w->rt_lo);
+    cudaFree(w->rt_wt);
+    cudaFree(w->rt_wmax);
     cudaFree(w->status);
     std::free(w->s_host);
     delete w;
@@ -114,6 +124,7 @@ WsLayout ws_layout(const moe_w8a8_weights* w, int T) {
     L.logits_stage = take((size_t)T * E * 4);
     L.bias_stage = take((size_t)E * 4);
     L.logits = take((size_t)T * E * 4);
+    L.logits_sel = take(router_tc_ok(w, T) ? (size_t)T * E * 4 : 0);
     L.topk_idx = take(tk * 4);
     L.topk_w = take(tk * 4);
     L.hist = take(nblk * E * 4);
@@ -139,6 +150,73 @@ WsLayout ws_layout(const moe_w8a8_weights* w, int T) {
     return L;
 }
 
+}  // namespace moe
+
+namespace moe {
+namespace {
+
+// fp32 -> bf16 bits, round to nearest even (finite values).
+uint16_t bf16_rn(float v) {
+    uint32_t b;
+    std::memcpy(&b, &v, 4);
+    b += 0x7FFFu + ((b >> 16) & 1u);
+    return (uint16_t)(b >> 16);
+}
+
+float bf16_value(uint16_t h) {
+    const uint32_t b = (uint32_t)h << 16;
+    float v;
+    std::memcpy(&v, &b, 4);
+    return v;
+}
+
+// Tables of the certified tensor-core router (bf16 X, renormalised gate):
+// W_g [d][E] -> hi, lo [epad][d] bf16 with hi = bf16(w), lo = bf16(w - hi)
+// (w - hi is exact in fp32), W_g transposed [E][d], max_e |W_g[j][e]| [d].
+// Leaves rt_epad = 0 (FMA router only) when the layer does not qualify or a
+// step fails.
+void prepare_router_tc(moe_w8a8_weights* w, cudaStream_t s) {
+    const moe_w8a8_config& c = w->cfg;
+    const int d = c.d, E = c.n_experts;
+    w->rt_epad = 0;
+    if (c.in_dtype != MOE_BF16 || c.renormalize != 1 || d % 128 != 0 || E > 256) return;
+    const int epad = E <= 64 ? 64 : (E <= 128 ? 128 : 256);
+    std::vector<float> wg((size_t)d * E), wt((size_t)E * d), wmax(d, 0.0f);
+    std::vector<uint16_t> hi((size_t)epad * d, 0), lo((size_t)epad * d, 0);
+    if (cudaMemcpyAsync(wg.data(), w->w_router, wg.size() * 4, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+        cudaStreamSynchronize(s) != cudaSuccess)
+        return;
+    // wt and wmax lane-interleaved: channel j = 32 i + p at [i / 4][p][i % 4]
+    auto lane_pos = [](int j) { const int i = j / 32, p = j % 32; return (size_t)(i / 4) * 128 + p * 4 + i % 4; };
+    std::vector<float> wmax_lin(d, 0.0f);
+    for (int j = 0; j < d; ++j)
+        for (int e = 0; e < E; ++e) {
+            const float v = wg[(size_t)j * E + e];
+            const uint16_t h = bf16_rn(v);
+            hi[(size_t)e * d + j] = h;
+            lo[(size_t)e * d + j] = bf16_rn(v - bf16_value(h));
+            wt[(size_t)e * d + lane_pos(j)] = v;
+            wmax_lin[j] = std::max(wmax_lin[j], std::fabs(v));
+        }
+    for (int j = 0; j < d; ++j) wmax[lane_pos(j)] = wmax_lin[j];
+    bool ok = cudaMalloc(&w->rt_hi, hi.size() * 2) == cudaSuccess &&
+              cudaMalloc(&w->rt_lo, lo.size() * 2) == cudaSuccess &&
+              cudaMalloc(&w->rt_wt, wt.size() * 4) == cudaSuccess &&
+              cudaMalloc(&w->rt_wmax, wmax.size() * 4) == cudaSuccess;
+    ok = ok && cudaMemcpyAsync(w->rt_hi, hi.data(), hi.size() * 2, cudaMemcpyHostToDevice, s) == cudaSuccess &&
+         cudaMemcpyAsync(w->rt_lo, lo.data(), lo.size() * 2, cudaMemcpyHostToDevice, s) == cudaSuccess &&
+         cudaMemcpyAsync(w->rt_wt, wt.data(), wt.size() * 4, cudaMemcpyHostToDevice, s) == cudaSuccess &&
+         cudaMemcpyAsync(w->rt_wmax, wmax.data(), wmax.size() * 4, cudaMemcpyHostToDevice, s) == cudaSuccess &&
+         cudaStreamSynchronize(s) == cudaSuccess;
+    if (!ok) {
+        cudaGetLastError();
+        return;
+    }
+    w->rt_epad = epad;
+    if (!router_tc_make_maps(w)) w->rt_epad = 0;
+}
+
+}  // namespace
 }  // namespace moe
 
 extern "C" {
@@ -246,10 +324,12 @@ moe_status moe_w8a8_prepare(const moe_w8a8_config* cfg, const float* w_gate, con
         cudaStreamSynchronize(s) != cudaSuccess)
         return fail(MOE_ERR_CUDA);
     w->tmaps_ok = tc_make_weight_maps(w);
+    prepare_router_tc(w, s);
     cudaFree(tmp);
     *out = w;
     return MOE_OK;
 }
+
 
 size_t moe_w8a8_workspace_size(const moe_w8a8_weights* w, int32_t max_tokens) {
     if (!w || max_tokens < 0) return 0;
@@ -288,7 +368,19 @@ static moe_status forward_impl(const moe_w8a8_weights* w, const void* x, int T, 
     auto empty_stage = [&](int stage) { mark(stage, 0); mark(stage, 1); };
 
     const float* lsrc = given_logits;
-    if (!lsrc) {
+    const bool certified = !lsrc && router_tc_ok(w, T) && ((uintptr_t)x & 15) == 0;
+    if (certified) {
+        // approximate logits on the tensor cores, then per token the candidates'
+        // logits in the stated order, top-k and gate weights
+        mark(MOE_STAGE_ROUTER, 0);
+        CUDA_TRY(launch_router_tc(w, x, T, logits, s));
+        mark(MOE_STAGE_ROUTER, 1);
+        mark(MOE_STAGE_TOPK, 0);
+        CUDA_TRY(launch_router_select(w, x, T, logits, bias, (float*)P(L.logits_sel), idx, wts,
+                                      dbg ? dbg->logits : nullptr, s));
+        mark(MOE_STAGE_TOPK, 1);
+        launches += 2;
+    } else if (!lsrc) {
         mark(MOE_STAGE_ROUTER, 0);
         CUDA_TRY(launch_router_logits(x, c.in_dtype, w->w_router, T, d, E, logits, s));
         mark(MOE_STAGE_ROUTER, 1);
@@ -297,7 +389,13 @@ static moe_status forward_impl(const moe_w8a8_weights* w, const void* x, int T, 
     } else {
         empty_stage(MOE_STAGE_ROUTER);
     }
-    if (route_small_ok(T, k)) {
+    if (certified) {
+        mark(MOE_STAGE_PERMUTE, 0);
+        CUDA_TRY(launch_permute(idx, T, k, E, capacity_of(c, T), (int32_t*)P(L.hist), offsets, row2ts,
+                                ts2row, meta, active, tiles, s));
+        mark(MOE_STAGE_PERMUTE, 1);
+        launches += 2;
+    } else if (route_small_ok(T, k)) {
         // top-k, histogram, scan and scatter in one block
         mark(MOE_STAGE_TOPK, 0);
         const bool fused = path == MOE_PATH_TENSOR && L.fused_words > 0;
