@@ -159,6 +159,13 @@ size_t moe_w8a8_workspace_size(const moe_w8a8_weights* w, int32_t max_tokens);
  *   dbg            NULL, or device pointers receiving intermediates
  * Allocates nothing; all scratch lives in the caller's workspace.  Calls
  * that share a workspace must not overlap on the device.
+ * With few rows per expert (T*k <= 512 on the tensor path) the expert FFN
+ * runs as one persistent launch whose thread blocks wait on one another
+ * (one per SM, all resident at once).  Forwards issued concurrently on
+ * other streams of the same device can keep some of its blocks off the
+ * SMs; its waits are bounded (2 s) and then fail with MOE_ERR_TIMEOUT
+ * (moe_w8a8_check_status) rather than hang.  Issue such batches on one
+ * stream, or serialise the streams.
  */
 moe_status moe_w8a8_forward(const moe_w8a8_weights* w, const void* x, int32_t T,
                             const float* router_bias, const float* router_logits, void* y,
