@@ -160,12 +160,12 @@ size_t moe_w8a8_workspace_size(const moe_w8a8_weights* w, int32_t max_tokens);
  * Allocates nothing; all scratch lives in the caller's workspace.  Calls
  * that share a workspace must not overlap on the device.
  * With few rows per expert (T*k <= 512 on the tensor path) the expert FFN
- * runs as one persistent launch whose thread blocks wait on one another
- * (one per SM, all resident at once).  Forwards issued concurrently on
- * other streams of the same device can keep some of its blocks off the
- * SMs; its waits are bounded (2 s) and then fail with MOE_ERR_TIMEOUT
- * (moe_w8a8_check_status) rather than hang.  Issue such batches on one
- * stream, or serialise the streams.
+ * runs as one persistent launch whose thread blocks wait on one another's
+ * results; tiles are taken from a device-wide counter in dependency order,
+ * so every wait is on work a running block already holds and the launch
+ * progresses even when other streams keep some of its blocks off the SMs.
+ * All such waits are bounded (2 s) and report MOE_ERR_TIMEOUT
+ * (moe_w8a8_check_status) instead of hanging.
  */
 moe_status moe_w8a8_forward(const moe_w8a8_weights* w, const void* x, int32_t T,
                             const float* router_bias, const float* router_logits, void* y,

@@ -569,12 +569,21 @@ struct FusedExtra {
     int32_t* queue;   // [m-tiles] m-tiles whose h is complete, + 1, in completion order
     int32_t* qtail;   // next free queue slot
     int32_t* qhead;   // next queue slot a requantisation warp takes
+    int32_t* next;    // next tile to take (dynamic schedule)
     int8_t* hq;       // [rows][f] h codes
     float* sh;        // [rows] h scales
-};                    // (count, ready, queue, qtail, qhead zeroed before the launch)
+};                    // (count, ready, queue, qtail, qhead, next zeroed before the launch)
 
 constexpr int kFusedThreads = kThreads + 32;   // + one requantisation warp (warp 10)
-constexpr size_t kFusedSmemBytes = kSmemBytes + kEpiStageBytes;
+constexpr int kTileRing = 8;                   // tiles taken but not yet finished, per CTA
+
+// The order in which a CTA's producer took its tiles, for its MMA and epilogue warps.
+struct TileRing {
+    uint64_t full[kTileRing];    // the producer wrote tile[q]
+    uint64_t empty[kTileRing];   // the MMA thread and the 8 epilogue warps have read it
+    int tile[kTileRing];         // tile index, or -1 = no more tiles
+};
+constexpr size_t kFusedSmemBytes = kSmemBytes + kEpiStageBytes + 256;
 
 // GEMM1 (gate/up + SwiGLU), the row-wise requantisation of h and GEMM2 (down)
 // in one persistent launch, for launches with few rows per expert (decode),
@@ -582,7 +591,12 @@ constexpr size_t kFusedSmemBytes = kSmemBytes + kEpiStageBytes;
 // the partial last wave of GEMM1 to drain.  One tile index space: GEMM1 tiles
 // (m-tile x 256 gate/up columns) first, then GEMM2 tiles (m-tile x 256 output
 // columns), dealt round robin, so the SMs idle in GEMM1's last wave start on
-// GEMM2 tiles at once.  Dependencies are per m-tile (one expert's rows): every
+// GEMM2 tiles at once.  Tiles are taken from a device-wide counter in that
+// order (each CTA's producer takes the next one when it has room and hands the
+// index to its MMA and epilogue warps through a small ring), so every tile a
+// wait depends on has already been taken by a running CTA: the launch makes
+// progress even when not all its CTAs are resident.  Dependencies are per
+// m-tile (one expert's rows): every
 // epilogue warp that finishes a GEMM1 tile adds one to count[m]; the warp that
 // brings it to (GEMM1 column tiles x epilogue warps) appends m to a device-wide
 // queue.  Warp 10 of every CTA takes queue slots in turn, requantises that
@@ -590,11 +604,11 @@ constexpr size_t kFusedSmemBytes = kSmemBytes + kEpiStageBytes;
 // warps of many CTAs and never delays an epilogue (when the epilogue warp that
 // completed an m-tile requantised it itself, it fell behind, became the last
 // arrival again, and the delays piled up).  The producer of a GEMM2 tile waits
-// for ready[m] (bounded) before loading its h codes.  A CTA's GEMM1 tiles all
-// come before its GEMM2 tiles, GEMM1 tiles wait on nothing, and the requant
-// warps wait only on GEMM1 tiles, so with every CTA resident the waits always
-// end.  Arithmetic per element is that of the two separate kernels and
-// requant_kernel, so the results are identical.
+// for ready[m] (bounded) before loading its h codes.  GEMM1 tiles are all taken
+// before any GEMM2 tile, GEMM1 tiles wait on nothing, and the requant warps
+// wait only on GEMM1 tiles, so the waits always end.  Arithmetic per element
+// is that of the two separate kernels and requant_kernel, so the results are
+// identical.
 template <int FMT>
 __global__ void __launch_bounds__(kFusedThreads, 1)
     tc_ffn_fused_kernel(const __grid_constant__ CUtensorMap tm_a1, const __grid_constant__ CUtensorMap tm_b1,
@@ -605,6 +619,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
     float* epi_stage = reinterpret_cast<float*>(smem + kStages * kStageBytes);
     // the requantisation warp's scale buffer follows the epilogue warps' staging buffers
     Ctl* ctl = reinterpret_cast<Ctl*>(smem + kStages * kStageBytes + (kEpiWarps + 1) * kEpiStageBytes);
+    TileRing* ring = reinterpret_cast<TileRing*>(reinterpret_cast<uint8_t*>(ctl) + 256);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
@@ -615,6 +630,10 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
         for (int b = 0; b < 2; ++b) {
             mbar_init(&ctl->acc_full[b], 1);
             mbar_init(&ctl->acc_empty[b], kEpiWarps);
+        }
+        for (int q = 0; q < kTileRing; ++q) {
+            mbar_init(&ring->full[q], 1);
+            mbar_init(&ring->empty[q], 1 + kEpiWarps);
         }
         mbar_init(&ctl->drain, 1);
         ctl->abort = 0;
@@ -656,7 +675,17 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
             bool issued[kStages];
             for (int i = 0; i < kStages; ++i) issued[i] = false;
             bool ok = true;
-            for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+            int q = 0;
+            uint32_t rph = 0;
+            while (ok) {
+                // take the next tile and tell the MMA and epilogue warps
+                int t = atomicAdd(fx.next, 1);
+                if (t >= num_tiles) t = -1;
+                if (!mbar_wait(&ring->empty[q], rph ^ 1, abort, p1.status, 8, t)) break;
+                ring->tile[q] = t;
+                mbar_arrive(&ring->full[q]);
+                if (++q == kTileRing) { q = 0; rph ^= 1; }
+                if (t < 0) break;
                 bool g1;
                 int mt, nt;
                 decode(t, g1, mt, nt);
@@ -704,7 +733,14 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
             int s = 0, buf = 0;
             uint32_t ph = 0, aph = 0;
             bool ok = true;
-            for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+            int q = 0;
+            uint32_t rph = 0;
+            while (ok) {
+                if (!mbar_wait(&ring->full[q], rph, abort, p1.status, 9, 0)) break;
+                const int t = ring->tile[q];
+                mbar_arrive(&ring->empty[q]);
+                if (++q == kTileRing) { q = 0; rph ^= 1; }
+                if (t < 0) break;
                 const int nkb = (t < w1 ? p1.K : p2.K) / BK;
                 if (!mbar_wait(&ctl->acc_empty[buf], aph ^ 1, abort, p1.status, 2, t)) break;
                 tc_fence_after();
@@ -771,7 +807,15 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
         float* stage = epi_stage + ew * (kEpiStageBytes / 4);
         int buf = 0;
         uint32_t aph = 0;
-        for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
+        int q = 0;
+        uint32_t rph = 0;
+        while (true) {
+            if (!mbar_wait(&ring->full[q], rph, abort, p1.status, 10, 0)) break;
+            const int t = ring->tile[q];
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&ring->empty[q]);
+            if (++q == kTileRing) { q = 0; rph ^= 1; }
+            if (t < 0) break;
             if (!mbar_wait(&ctl->acc_full[buf], aph, abort, p1.status, 4, t)) break;
             tc_fence_after();
             bool g1;
@@ -1152,7 +1196,7 @@ cudaError_t launch_tc_ffn_fused(const moe_w8a8_weights* w, int T, const int8_t* 
     p2.acc_dbg = acc2_dbg;
     const int max_mt = (rows + BM - 1) / BM + c.n_experts;
     const FusedExtra fx{sync_words, sync_words + max_mt, sync_words + 2 * max_mt, sync_words + 3 * max_mt,
-                        sync_words + 3 * max_mt + 1, hq, sh};
+                        sync_words + 3 * max_mt + 1, sync_words + 3 * max_mt + 2, hq, sh};
     const int grid = max(1, min(w->num_sms, max_mt * (p1.n_tiles_n + p2.n_tiles_n)));
     if (c.expert_format == FMT_E4M3)
         return launch_fused_fmt<FMT_E4M3>(a1, w->tm_w_gu, a2, w->tm_w_dn, p1, p2, fx, grid, s);
