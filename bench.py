@@ -37,6 +37,7 @@ INT8_PER_BF16 = 2.0   # nominal dense ratio (4.5 POPS int8 / 2.25 PFLOPS bf16)
 # DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum) of the dominant
 # kernel, from one ncu capture of the current kernel source (see profiles/).
 TRAFFIC = {
+    ("decode", 32, "tc_ffn_fused_kernel"): 1060.720e6 + 6.530304e6,
 }
 
 FUSED_MAX_ROWS = 512   # T*k at or below which the tensor path runs GEMM1 + requant + GEMM2 as one launch
