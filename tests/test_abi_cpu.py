@@ -56,6 +56,8 @@ def test_host_side_argument_checks(M):
                                  ("alpha", 1.5, M.MOE_ERR_INVALID_ARG),
                                  ("in_dtype", 7, M.MOE_ERR_INVALID_ARG),
                                  ("renormalize", 2, M.MOE_ERR_INVALID_ARG),
+                                 ("expert_format", 2, M.MOE_ERR_INVALID_ARG),
+                                 ("expert_format", -1, M.MOE_ERR_INVALID_ARG),
                                  ("d", 4000, M.MOE_ERR_UNSUPPORTED_SHAPE),
                                  ("f", 100, M.MOE_ERR_UNSUPPORTED_SHAPE),
                                  ("n_experts", 300, M.MOE_ERR_UNSUPPORTED_SHAPE),
@@ -80,6 +82,9 @@ def test_host_side_argument_checks(M):
     assert L.moe_w8a8_calibrate_absmax(z, 4, 16, 5, z, None) == M.MOE_ERR_INVALID_ARG
     assert L.moe_w8a8_calibrate_absmax(z, -1, 16, 0, z, None) == M.MOE_ERR_INVALID_ARG
     assert L.moe_w8a8_last_launch_count(None) == 0
+    assert L.moe_w8a8_set_act_clip(None, 1.0) == M.MOE_ERR_INVALID_ARG
+    clip = ctypes.c_float(0.0)
+    assert L.moe_w8a8_calibrate_act_clip(None, z, 4, 1, 99.9, ctypes.byref(clip), None) == M.MOE_ERR_INVALID_ARG
     L.moe_w8a8_destroy(None)
 
 
