@@ -784,7 +784,11 @@ __global__ void __launch_bounds__(kSqThreads) smooth_quant_kernel(
     const void* __restrict__ x, int in_dtype, const float* __restrict__ inv_s, float act_clip, int T, int d,
     int k, const int32_t* __restrict__ ts2row, int8_t* __restrict__ xq, float* __restrict__ sx,
     int8_t* __restrict__ aq) {
-    pdl_wait();
+    // X is an input of the forward and xq / sx are read only by later kernels of
+    // this forward: when this kernel starts (its predecessor has passed its own
+    // wait) every kernel of the previous forward has finished, so the codes are
+    // formed while the routing kernel still runs; only the copy into the
+    // expert-sorted rows waits for the routing (ts2row).
     pdl_trigger();
 
     __shared__ float red[kSqThreads / 32];
@@ -820,9 +824,7 @@ __global__ void __launch_bounds__(kSqThreads) smooth_quant_kernel(
     const float s = m > 0.0f ? __fdiv_rn(m, fmt_qmax<FMT>()) : 0.0f;
     const float rs = s > 0.0f ? __frcp_rn(s) : 0.0f;
     if (tid == 0) sx[t] = s;
-    int rows[kMaxK];
-#pragma unroll
-    for (int sl = 0; sl < kMaxK; ++sl) rows[sl] = (aq && sl < k) ? ts2row[(int64_t)t * k + sl] : -1;
+    uint2 packed[kSqMaxGroups];
 #pragma unroll
     for (int gi = 0; gi < kSqMaxGroups; ++gi) {
         const int g = tid + kSqThreads * gi;
@@ -830,11 +832,21 @@ __global__ void __launch_bounds__(kSqThreads) smooth_quant_kernel(
         int q[8];
 #pragma unroll
         for (int c = 0; c < 8; ++c) q[c] = s > 0.0f ? (int)fmt_code<FMT>(v[gi][c], s, rs) : 0;
-        const uint2 packed = make_uint2(pack4(q[0], q[1], q[2], q[3]), pack4(q[4], q[5], q[6], q[7]));
-        *reinterpret_cast<uint2*>(xq + (int64_t)t * d + g * 8) = packed;
+        packed[gi] = make_uint2(pack4(q[0], q[1], q[2], q[3]), pack4(q[4], q[5], q[6], q[7]));
+        *reinterpret_cast<uint2*>(xq + (int64_t)t * d + g * 8) = packed[gi];
+    }
+    pdl_wait();   // the routing of this forward is complete from here on
+    if (!aq) return;
+    int rows[kMaxK];
+#pragma unroll
+    for (int sl = 0; sl < kMaxK; ++sl) rows[sl] = sl < k ? ts2row[(int64_t)t * k + sl] : -1;
+#pragma unroll
+    for (int gi = 0; gi < kSqMaxGroups; ++gi) {
+        const int g = tid + kSqThreads * gi;
+        if (g >= ng) continue;
 #pragma unroll
         for (int sl = 0; sl < kMaxK; ++sl)
-            if (rows[sl] >= 0) *reinterpret_cast<uint2*>(aq + (int64_t)rows[sl] * d + g * 8) = packed;
+            if (rows[sl] >= 0) *reinterpret_cast<uint2*>(aq + (int64_t)rows[sl] * d + g * 8) = packed[gi];
     }
 }
 
