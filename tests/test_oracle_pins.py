@@ -533,3 +533,58 @@ def test_fp8_dense_special_case_e1_k1():
     assert rel < 0.1
     # every stage's debug output decodes to values of the right scale
     assert np.all(dbg["sx"] > 0) and np.all(dbg["sh"] > 0)
+
+
+def test_fp8_whole_layer_closed_form_exact_codes():
+    """E4M3 counterpart of the integer closed form: X rows and weight columns
+    drawn from the E4M3 values with each range exactly 448, smoothing off, so
+    every scale is 1 and every code is the value itself.  Then the gate/up
+    accumulators are exact rational sums rounded once to fp32, the h codes are
+    within half an E4M3 step of h / sh, and the down accumulators are the
+    exact sums of the decoded h codes -- each checked against fp64 arithmetic
+    written here, not the oracle's routines."""
+    T, d, E, k, f = 16, 64, 3, 2, 32
+    tab = _e4m3_table()
+    vals = np.concatenate([tab[8:0x7e], -tab[8:0x7e]])       # normal E4M3 values below 448
+    rng = np.random.default_rng(21)
+
+    def draw(shape, axis):
+        a = rng.choice(vals, size=shape)                      # exact E4M3 values, |a| <= 416
+        # put an exact 448 on every row (axis=1) / column (axis=-2) so the range is 448
+        idx = rng.integers(0, a.shape[axis], size=[s for i, s in enumerate(a.shape) if i != axis % a.ndim])
+        np.put_along_axis(a, np.expand_dims(idx, axis), 448.0, axis=axis)
+        return a
+    x = draw((T, d), 1)
+    wg = np.stack([draw((d, f), 0) for _ in range(E)])
+    wu = np.stack([draw((d, f), 0) for _ in range(E)])
+    wd = np.stack([draw((f, d), 0) for _ in range(E)])
+    prep = oracle.prepare_fp8(wg.astype(np.float32), wu.astype(np.float32), wd.astype(np.float32),
+                              x.astype(np.float32), 0.5, smooth=False)
+    assert np.all(prep.sw_gate == 1.0) and np.all(prep.sw_up == 1.0) and np.all(prep.sw_down == 1.0)
+    assert np.array_equal(oracle.e4m3_decode(prep.wq_gate).astype(np.float64), wg.transpose(0, 2, 1))
+    logits = synth.normal(21, 9, (T, E))
+    rt = oracle.route(x.astype(np.float32), k, E, logits=logits)
+    y, dbg = oracle.moe_tokens_fp8(x.astype(np.float32), prep, rt)
+    assert np.all(dbg["sx"] == 1.0)
+    assert np.array_equal(oracle.e4m3_decode(dbg["xq"]).astype(np.float64), x)
+    from fractions import Fraction
+    for t in range(T):
+        for s in range(k):
+            e = rt.idx[t, s]
+            g_exact = [sum(Fraction(float(a)) * Fraction(float(b)) for a, b in zip(x[t], wg[e][:, n]))
+                       for n in range(f)]
+            assert np.array_equal(dbg["acc1"][t, s, :f], np.array([np.float32(float(v)) for v in g_exact]))
+            g = dbg["acc1"][t, s, :f].astype(np.float64)
+            u = dbg["acc1"][t, s, f:].astype(np.float64)
+            assert np.array_equal(dbg["acc1"][t, s, f:], (x[t] @ wu[e]).astype(np.float32))
+            with np.errstate(over="ignore"):
+                h64 = g / (1.0 + np.exp(-g)) * u
+            sh = float(dbg["sh"][t, s])
+            assert abs(sh - np.abs(h64).max() / 448.0) <= 1e-6 * sh
+            q = h64 / sh
+            dq = oracle.e4m3_decode(dbg["hq"][t, s]).astype(np.float64)
+            step = np.where(np.abs(q) >= 2.0 ** -6,
+                            2.0 ** (np.floor(np.log2(np.maximum(np.abs(q), 1e-30))) - 3), 2.0 ** -9)
+            assert np.all(np.abs(dq - q) <= step / 2 * (1 + 1e-4) + 1e-6 * np.abs(q))
+            acc2 = wd[e].T @ dq                                      # exact: products fit fp64
+            assert np.array_equal(dbg["acc2"][t, s], acc2.astype(np.float32))
