@@ -166,6 +166,9 @@ size_t moe_w8a8_workspace_size(const moe_w8a8_weights* w, int32_t max_tokens);
  * progresses even when other streams keep some of its blocks off the SMs.
  * All such waits are bounded (2 s) and report MOE_ERR_TIMEOUT
  * (moe_w8a8_check_status) instead of hanging.
+ * A handle from moe_w8a8_prepare_shard that does not hold every expert
+ * returns MOE_ERR_INVALID_ARG (here, in moe_w8a8_forward_host and in
+ * moe_w8a8_forward_noalloc): it runs through the moe_w8a8_ep_* calls.
  */
 moe_status moe_w8a8_forward(const moe_w8a8_weights* w, const void* x, int32_t T,
                             const float* router_bias, const float* router_logits, void* y,
@@ -265,8 +268,10 @@ moe_status moe_w8a8_export_weights(const moe_w8a8_weights* w, int8_t* wq_gate, i
 
 /*
  * Synchronise `stream` and read the handle's device status word: MOE_OK,
- * or MOE_ERR_TIMEOUT when a bounded wait in a kernel ran out since the last
- * check (the word is then cleared), or MOE_ERR_CUDA on a pending CUDA error.
+ * MOE_ERR_TIMEOUT when a bounded wait in a kernel ran out since the last
+ * check, MOE_ERR_INVALID_ARG when moe_w8a8_ep_experts received a row for an
+ * expert this handle does not hold (the word is then cleared), or
+ * MOE_ERR_CUDA on a pending CUDA error.
  */
 moe_status moe_w8a8_check_status(const moe_w8a8_weights* w, moe_stream_t stream);
 
@@ -275,8 +280,9 @@ moe_status moe_w8a8_check_status(const moe_w8a8_weights* w, moe_stream_t stream)
  * handle's status words to words_host[0..n) (n <= 16): word 0 is the status
  * code, words 1-4 say where the first bounded wait gave up (site: 1 producer
  * stage-free, 2 MMA accumulator-free, 3 MMA stage-full, 4 epilogue
- * accumulator-full; then block index, tile, and the awaited phase parity).
- * Does not clear them.
+ * accumulator-full; then block index, tile, and the awaited phase parity;
+ * site 14: a received expert-parallel row names an expert outside the
+ * handle's range, then the row index and the expert).  Does not clear them.
  */
 moe_status moe_w8a8_status_words(const moe_w8a8_weights* w, int32_t* words_host, int32_t n,
                                  moe_stream_t stream);
@@ -323,6 +329,122 @@ moe_status moe_w8a8_profile_stop(moe_w8a8_weights* w);
 
 /* Static name of a stage ("router", "topk", ...), or "?" . */
 const char* moe_w8a8_stage_name(int32_t stage);
+
+/* ------------------------------------------------------------------------
+ * Expert parallelism.  "Day0 adaptation of ultra-large model inference",
+ * section 3: the experts are spread over the GPUs and each layer moves its
+ * tokens with one All-to-All each way; section 4: the operator chain gate ->
+ * sort -> All-to-All -> grouped GEMM -> reverse All-to-All -> un-sort ->
+ * weighted sum.
+ *
+ * G ranks hold G contiguous ranges of the layer's E experts (rank g: experts
+ * [g E / G, (g + 1) E / G) when G divides E; any contiguous split works).
+ * Each rank routes and quantises its own T tokens against all E experts; the
+ * result on every rank equals moe_w8a8_forward on that rank's tokens with a
+ * handle holding all experts (the same capacity rule, applied to those T
+ * tokens).  One layer on one rank:
+ *   1. moe_w8a8_ep_dispatch: router, top-k, sort and quantisation.  Writes
+ *      the kept (token, slot) rows, expert-major and in token order within
+ *      an expert (so the rows for one rank are contiguous), to `send`, and
+ *      the per-expert row offsets [E + 1] to expert_offsets.
+ *   2. the caller exchanges, per destination rank, the rows of its experts
+ *      (one All-to-All of whole rows; row counts from expert_offsets).
+ *   3. moe_w8a8_ep_experts on the received rows (in any order): the local
+ *      experts' grouped GEMMs; writes the fp32 output row of each received
+ *      row, in the received order.
+ *   4. the caller returns the output rows to their senders (the reverse
+ *      All-to-All: every row goes back to the rank and position it came from).
+ *   5. moe_w8a8_ep_combine: each token's output as the sum of its kept slots
+ *      in slot order, from the returned rows in the order of `send`.
+ * Row layout (moe_w8a8_ep_row_bytes(w) = d + 16 bytes per row): the d INT8
+ * (or E4M3) codes of the token, then fp32 activation scale, fp32 gate weight,
+ * int32 global expert, int32 t * k + slot on the sending rank.
+ * ------------------------------------------------------------------------ */
+
+/* Bytes per dispatched row: d + 16 (0 on a NULL handle). */
+int32_t moe_w8a8_ep_row_bytes(const moe_w8a8_weights* w);
+
+/*
+ * aw[j] = max over the given n_local experts e and every output n of
+ * |w_gate[e][j][n]| and |w_up[e][j][n]|: the weight statistic of the
+ * SmoothQuant scale ("MiniMax-M3 W8A8 on K100AI" s6.1/s6.4).  The layer's aw
+ * is the maximum over all ranks (an all-reduce with MAX of this per-rank
+ * value), which every rank then passes to moe_w8a8_prepare_shard.
+ *   w_gate, w_up  device fp32 [n_local][d][f];  aw  device fp32 [d]
+ * Asynchronous on `stream`.
+ */
+moe_status moe_w8a8_gateup_absmax(const moe_w8a8_config* cfg, int32_t n_local, const float* w_gate,
+                                  const float* w_up, float* aw, moe_stream_t stream);
+
+/*
+ * moe_w8a8_prepare for experts [expert_first, expert_first + n_local) of the
+ * layer `cfg` (cfg.n_experts = all E experts).
+ *   w_gate, w_up   device fp32 [n_local][d][f] (those experts only)
+ *   w_down         device fp32 [n_local][f][d]
+ *   w_router       device fp32 [d][E] (the whole router)
+ *   act_absmax     device fp32 [d]
+ *   gateup_absmax  device fp32 [d], the layer's aw over ALL E experts (see
+ *                  moe_w8a8_gateup_absmax), so that every rank computes the
+ *                  same smoothing s and quantises its tokens identically
+ * Returns MOE_ERR_INVALID_ARG for a range outside [0, E) or a NULL pointer;
+ * otherwise as moe_w8a8_prepare.  The handle serves moe_w8a8_ep_* only
+ * (unless it holds all E experts).
+ */
+moe_status moe_w8a8_prepare_shard(const moe_w8a8_config* cfg, int32_t expert_first, int32_t n_local,
+                                  const float* w_gate, const float* w_up, const float* w_down,
+                                  const float* w_router, const float* act_absmax, const float* gateup_absmax,
+                                  moe_stream_t stream, moe_w8a8_weights** out);
+
+/* Workspace of moe_w8a8_ep_dispatch and moe_w8a8_ep_combine for up to
+ * max_tokens tokens; of moe_w8a8_ep_experts for `rows` received rows. */
+size_t moe_w8a8_ep_dispatch_workspace_size(const moe_w8a8_weights* w, int32_t max_tokens);
+size_t moe_w8a8_ep_experts_workspace_size(const moe_w8a8_weights* w, int32_t rows);
+
+/*
+ * Step 1 of the expert-parallel layer on this rank's T tokens.
+ *   x, router_bias, router_logits   as in moe_w8a8_forward
+ *   send            device [T * k][moe_w8a8_ep_row_bytes(w)] bytes, 16-byte
+ *                   aligned; rows [0, R) are written, R = expert_offsets[E]
+ *   expert_offsets  device int32 [E + 1]: the rows of expert e are
+ *                   [expert_offsets[e], expert_offsets[e + 1]) (zeros for T = 0)
+ *   workspace       device, >= moe_w8a8_ep_dispatch_workspace_size(w, T),
+ *                   256-byte aligned; it keeps the token -> row map that
+ *                   moe_w8a8_ep_combine reads, so it must not be reused in
+ *                   between
+ *   dbg             NULL, or routing intermediates (logits, topk_idx, topk_w,
+ *                   offsets, row2ts, ts2row, xq, sx)
+ */
+moe_status moe_w8a8_ep_dispatch(const moe_w8a8_weights* w, const void* x, int32_t T, const float* router_bias,
+                                const float* router_logits, void* send, int32_t* expert_offsets, void* workspace,
+                                size_t workspace_bytes, const moe_w8a8_debug* dbg, moe_stream_t stream);
+
+/*
+ * Step 3: the experts this handle holds, on R received rows.
+ *   recv      device [R][moe_w8a8_ep_row_bytes(w)] bytes, 16-byte aligned,
+ *             rows as written by moe_w8a8_ep_dispatch on any rank of the
+ *             same layer, each naming one of this handle's experts
+ *   o_rows    device fp32 [R][d], 16-byte aligned: o_rows[r] = the routing
+ *             weight x the expert's output for received row r
+ *   workspace device, >= moe_w8a8_ep_experts_workspace_size(w, R), 256-byte aligned
+ *   dbg       NULL, or the expert side's intermediates by local sorted row
+ *             (topk_idx = local expert per received row, offsets [n_local + 1],
+ *             row2ts / ts2row between received and sorted rows, sx, acc1,
+ *             hq, sh, acc2, o)
+ * A row naming an expert outside this handle's range is reported through
+ * the status word (moe_w8a8_check_status: MOE_ERR_INVALID_ARG) and its
+ * output is meaningless.  R = 0 is a no-op.
+ */
+moe_status moe_w8a8_ep_experts(const moe_w8a8_weights* w, const void* recv, int32_t R, float* o_rows,
+                               void* workspace, size_t workspace_bytes, const moe_w8a8_debug* dbg,
+                               moe_stream_t stream);
+
+/*
+ * Step 5: y [T][d] (cfg.out_dtype) from the returned rows o_rows (device fp32
+ * [R][d], in the row order of `send`; may be NULL when R = 0) and the
+ * workspace of the matching moe_w8a8_ep_dispatch with the same T.
+ */
+moe_status moe_w8a8_ep_combine(const moe_w8a8_weights* w, const float* o_rows, int32_t T, void* y,
+                               const void* workspace, size_t workspace_bytes, moe_stream_t stream);
 
 #ifdef __cplusplus
 }

@@ -47,9 +47,10 @@ def x_tensor(wl: synth.Workload, data: synth.LayerData):
     return to_dev(data.x)
 
 
-def gpu_prepare(wl: synth.Workload, wts: synth.LayerWeights, capacity_factor=None, renormalize=True,
-                fmt=0, w_router=None):
-    """Calibration absmax + prepare through the C ABI (fmt: MOE_FMT_INT8 / MOE_FMT_E4M3)."""
+def gpu_layer_tensors(wl: synth.Workload, wts: synth.LayerWeights, capacity_factor=None, renormalize=True,
+                      fmt=0, w_router=None):
+    """The config and the device inputs of prepare: (cfg, w_gate, w_up, w_down,
+    w_router, act_absmax), the calibration absmax measured through the C ABI."""
     import w8a8_quantized_moe_b200 as M
     torch = torch_mod()
     cfg = M.make_config(wl.d, wl.f, wl.E, wl.k, wl.alpha,
@@ -65,8 +66,16 @@ def gpu_prepare(wl: synth.Workload, wts: synth.LayerWeights, capacity_factor=Non
     M.moe_w8a8_calibrate_absmax(cal, ax)
     if w_router is None:
         w_router = synth.normal(wl.data_seed, synth.TID_W_ROUTER, (wl.d, wl.E), std=wl.weight_std)
-    wr = to_dev(w_router)
-    W = M.moe_w8a8_prepare(cfg, to_dev(wts.w_gate), to_dev(wts.w_up), to_dev(wts.w_down), wr, ax)
+    return cfg, to_dev(wts.w_gate), to_dev(wts.w_up), to_dev(wts.w_down), to_dev(w_router), ax
+
+
+def gpu_prepare(wl: synth.Workload, wts: synth.LayerWeights, capacity_factor=None, renormalize=True,
+                fmt=0, w_router=None):
+    """Calibration absmax + prepare through the C ABI (fmt: MOE_FMT_INT8 / MOE_FMT_E4M3)."""
+    import w8a8_quantized_moe_b200 as M
+    torch = torch_mod()
+    cfg, wg, wu, wd, wr, ax = gpu_layer_tensors(wl, wts, capacity_factor, renormalize, fmt, w_router)
+    W = M.moe_w8a8_prepare(cfg, wg, wu, wd, wr, ax)
     torch.cuda.synchronize()
     return W
 

@@ -88,6 +88,35 @@ def test_host_side_argument_checks(M):
     L.moe_w8a8_destroy(None)
 
 
+def test_expert_parallel_host_side_checks(M):
+    L = M.lib()
+    out = ctypes.c_void_p(123)
+    cfg = M.make_config(4096, 1536, 64, 4)
+    z = ctypes.c_void_p(16)   # never dereferenced: the checks fail first
+    # shard range outside [0, E), empty shard, missing layer statistic
+    for first, n in [(-1, 8), (60, 8), (0, 0), (0, 65)]:
+        assert L.moe_w8a8_prepare_shard(ctypes.byref(cfg), first, n, z, z, z, z, z, z, None,
+                                        ctypes.byref(out)) == M.MOE_ERR_INVALID_ARG, (first, n)
+        assert out.value is None
+    assert L.moe_w8a8_prepare_shard(ctypes.byref(cfg), 0, 8, z, z, z, z, z, None, None,
+                                    ctypes.byref(out)) == M.MOE_ERR_INVALID_ARG
+    assert L.moe_w8a8_prepare_shard(None, 0, 8, z, z, z, z, z, z, None, ctypes.byref(out)) == M.MOE_ERR_INVALID_ARG
+    bad = M.make_config(4000, 1536, 64, 4)
+    assert L.moe_w8a8_prepare_shard(ctypes.byref(bad), 0, 8, z, z, z, z, z, z, None,
+                                    ctypes.byref(out)) == M.MOE_ERR_UNSUPPORTED_SHAPE
+    assert L.moe_w8a8_gateup_absmax(ctypes.byref(cfg), 0, z, z, z, None) == M.MOE_ERR_INVALID_ARG
+    assert L.moe_w8a8_gateup_absmax(ctypes.byref(cfg), 65, z, z, z, None) == M.MOE_ERR_INVALID_ARG
+    assert L.moe_w8a8_gateup_absmax(ctypes.byref(cfg), 8, z, z, None, None) == M.MOE_ERR_INVALID_ARG
+    assert L.moe_w8a8_gateup_absmax(ctypes.byref(bad), 8, z, z, z, None) == M.MOE_ERR_UNSUPPORTED_SHAPE
+    # handle-less calls
+    assert L.moe_w8a8_ep_row_bytes(None) == 0
+    assert L.moe_w8a8_ep_dispatch_workspace_size(None, 32) == 0
+    assert L.moe_w8a8_ep_experts_workspace_size(None, 32) == 0
+    assert L.moe_w8a8_ep_dispatch(None, z, 32, None, None, z, z, z, 1 << 20, None, None) == M.MOE_ERR_INVALID_ARG
+    assert L.moe_w8a8_ep_experts(None, z, 32, z, z, 1 << 20, None, None) == M.MOE_ERR_INVALID_ARG
+    assert L.moe_w8a8_ep_combine(None, z, 32, z, z, 1 << 20, None) == M.MOE_ERR_INVALID_ARG
+
+
 def test_product_path_does_not_touch_the_oracle():
     """The library sources and the binding never name the oracle."""
     pkg = os.path.join(ROOT, "w8a8_quantized_moe_b200")

@@ -1,0 +1,182 @@
+"""Expert-parallel exchange on CPU.
+
+gloo ranks run ``ExpertParallelMoE`` (the same driver the GPU ranks run) with
+stand-ins for the library's three compute steps written on the oracle: the
+dispatch writes the routed, quantised rows in the library's row layout, the
+expert step evaluates each received row with the oracle's GEMMs and
+epilogues, and the combine sums slots in slot order.  Every rank's output
+must equal the oracle's single-process layer on that rank's tokens bit for
+bit, which holds only if every row reaches the rank holding its expert and
+every output row comes back to the position it left from.
+"""
+import dataclasses
+import os
+import socket
+import sys
+
+import numpy as np
+import pytest
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+class OracleStages:
+    """One rank's compute steps on the oracle (experts [first, first + n))."""
+
+    def __init__(self, wl, prep, first, n):
+        import torch
+        self.wl, self.prep, self.first, self.n = wl, prep, first, n
+        self.d, self.k, self.E = wl.d, wl.k, wl.E
+        self.row_bytes = wl.d + 16
+        self.device = torch.device("cpu")
+        self.out_dtype = torch.float32
+        self.ts2row = None
+        self.seen_experts = set()
+
+    def dispatch_workspace(self, T):
+        return 16
+
+    def experts_workspace(self, R):
+        return 16
+
+    def dispatch(self, data, T, bias, logits, send, offsets, ws):
+        import torch
+
+        import oracle
+        d, k, E, rb = self.d, self.k, self.E, self.row_bytes
+        if T == 0:
+            offsets.zero_()
+            self.ts2row = np.zeros((0, k), np.int32)
+            return
+        rt = oracle.route(data.x, k, E, w_router=data.w_router, logits=data.router_logits, bias=data.router_bias,
+                          capacity_factor=self.wl.capacity_factor)
+        xq, sx = oracle.quantize_tokens(data.x, self.prep.inv_s)
+        R = int(rt.offsets[E])
+        rows = np.zeros((T * k, rb), np.uint8)
+        for r in range(R):
+            ts = int(rt.row2ts[r])
+            t, sl = divmod(ts, k)
+            rows[r, :d] = xq[t].view(np.uint8)
+            rows[r, d:d + 8] = np.array([sx[t], rt.w[t, sl]], np.float32).view(np.uint8)
+            rows[r, d + 8:] = np.array([rt.idx[t, sl], ts], np.int32).view(np.uint8)
+        send.copy_(torch.from_numpy(rows.reshape(-1)))
+        offsets.copy_(torch.from_numpy(rt.offsets.astype(np.int32)))
+        self.ts2row = rt.ts2row
+
+    def experts(self, recv, R, o_rows, ws):
+        import torch
+
+        import oracle
+        d, p = self.d, self.prep
+        rows = recv.numpy().reshape(R, self.row_bytes)
+        for r in range(R):
+            codes = rows[r, :d].view(np.int8)
+            sx, w = rows[r, d:d + 8].view(np.float32)
+            e, _ts = rows[r, d + 8:].view(np.int32)
+            assert self.first <= e < self.first + self.n, f"row for expert {e} on the wrong rank"
+            self.seen_experts.add(int(e))
+            acc_g = oracle.gemm_i8(codes[None], p.wq_gate[e])[0]
+            acc_u = oracle.gemm_i8(codes[None], p.wq_up[e])[0]
+            _h, hq, sh = oracle.swiglu_requant(acc_g, acc_u, float(sx), p.sw_gate[e], p.sw_up[e])
+            acc2 = oracle.gemm_i8(hq[None], p.wq_down[e])[0]
+            o_rows[r] = torch.from_numpy(oracle.down_epilogue(acc2, sh, p.sw_down[e], float(w)))
+
+    def combine(self, o_rows, T, y, ws):
+        import torch
+        o = o_rows.numpy()
+        acc = np.zeros((T, self.d), np.float32)
+        for sl in range(self.k):
+            rows = self.ts2row[:, sl]
+            m = rows >= 0
+            acc[m] = acc[m] + o[rows[m]]
+        y.copy_(torch.from_numpy(acc))
+
+
+def _rank_main(rank, world, port, out_dir, case):
+    sys.path.insert(0, ROOT)
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    import datetime
+    import json
+
+    import torch.distributed as dist
+
+    import oracle
+    import synth
+    from w8a8_quantized_moe_b200.ep import ExpertParallelMoE, equal_expert_ranges
+
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=120))
+    try:
+        wl = dataclasses.replace(synth.WORKLOADS["tiny"], **case.get("wl", {}))
+        T = case.get("T", [wl.T] * world)[rank]
+        wts = synth.make_weights(wl)
+        prep = oracle.prepare(wts.w_gate, wts.w_up, wts.w_down, wts.calib_x, wl.alpha)
+        first, n = equal_expert_ranges(wl.E, world)[rank]
+        stages = OracleStages(wl, prep, first, n)
+        layer = ExpertParallelMoE(stages)
+        out = {"rows": None, "equal": True, "T": T}
+        for step in range(2):   # two layers' worth of traffic through the same buffers
+            wl_r = dataclasses.replace(wl, T=max(T, 1), data_seed=wl.data_seed + 37 * rank + 1000 * step)
+            data = synth.make_data(wl_r)
+            y = layer.forward(data, T).numpy()
+            if T:
+                rt = oracle.route(data.x, wl.k, wl.E, w_router=data.w_router, logits=data.router_logits,
+                                  bias=data.router_bias, capacity_factor=wl.capacity_factor)
+                y_ref, _ = oracle.moe_tokens(data.x, prep, rt, debug=False)
+                out["equal"] &= bool(np.array_equal(y, y_ref))
+            out["rows"] = list(layer.last_rows)
+        out["seen"] = sorted(stages.seen_experts)
+        out["range"] = [first, n]
+        with open(os.path.join(out_dir, f"r{rank}.json"), "w") as fh:
+            json.dump(out, fh)
+    finally:
+        dist.destroy_process_group()
+
+
+def _run(tmp_path, world, case):
+    import json
+    mp.start_processes(_rank_main, args=(world, _free_port(), str(tmp_path), case), nprocs=world,
+                       start_method="spawn", join=True)
+    return [json.load(open(tmp_path / f"r{i}.json")) for i in range(world)]
+
+
+def test_ep_two_ranks_uniform(tmp_path):
+    r = _run(tmp_path, 2, {})
+    assert all(x["equal"] for x in r)
+    sent = sum(x["rows"][0] for x in r)
+    assert sent == sum(x["rows"][1] for x in r) == 2 * 64 * 2   # no capacity: every slot travels
+    for x in r:
+        first, n = x["range"]
+        assert x["seen"] and all(first <= e < first + n for e in x["seen"])
+
+
+def test_ep_four_ranks_skewed_with_capacity(tmp_path):
+    # Zipf router bias piles tokens on a few experts; capacity 1.0 drops the
+    # late arrivals on the sending rank, so ranks send and receive unequal counts
+    r = _run(tmp_path, 4, {"wl": {"zipf_s": 1.5, "capacity_factor": 1.0}})
+    assert all(x["equal"] for x in r)
+    sent = [x["rows"][0] for x in r]
+    recv = [x["rows"][1] for x in r]
+    assert sum(sent) == sum(recv) < 4 * 64 * 2
+    assert len(set(recv)) > 1
+
+
+def test_ep_rank_without_tokens(tmp_path):
+    # rank 1 routes no tokens this step but still serves its experts
+    r = _run(tmp_path, 2, {"T": [64, 0]})
+    assert r[0]["equal"] and r[1]["T"] == 0
+    assert r[1]["rows"][0] == 0 and r[1]["rows"][1] > 0
+
+
+def test_expert_ranges_host_checks():
+    sys.path.insert(0, ROOT)
+    from w8a8_quantized_moe_b200.ep import equal_expert_ranges
+    assert equal_expert_ranges(64, 8) == [(8 * g, 8) for g in range(8)]
+    with pytest.raises(ValueError):
+        equal_expert_ranges(10, 4)

@@ -41,6 +41,9 @@ EXPORTS = (
     "moe_w8a8_last_launch_count", "moe_w8a8_profile_start", "moe_w8a8_profile_read",
     "moe_w8a8_profile_stop", "moe_w8a8_stage_name", "moe_w8a8_forward_noalloc",
     "moe_w8a8_status_words", "moe_w8a8_set_act_clip", "moe_w8a8_calibrate_act_clip",
+    "moe_w8a8_ep_row_bytes", "moe_w8a8_gateup_absmax", "moe_w8a8_prepare_shard",
+    "moe_w8a8_ep_dispatch_workspace_size", "moe_w8a8_ep_experts_workspace_size",
+    "moe_w8a8_ep_dispatch", "moe_w8a8_ep_experts", "moe_w8a8_ep_combine",
 )
 
 MOE_NOALLOC_SCRATCH_BYTES = 8 << 20
@@ -105,6 +108,14 @@ def lib():
             "moe_w8a8_stage_name": ([i32], ctypes.c_char_p),
             "moe_w8a8_forward_noalloc": ([vp, vp, i32, vp, vp, vp, vp], i32),
             "moe_w8a8_status_words": ([vp, vp, i32, vp], i32),
+            "moe_w8a8_ep_row_bytes": ([vp], i32),
+            "moe_w8a8_gateup_absmax": ([cfgp, i32, vp, vp, vp, vp], i32),
+            "moe_w8a8_prepare_shard": ([cfgp, i32, i32, vp, vp, vp, vp, vp, vp, vp, ctypes.POINTER(vp)], i32),
+            "moe_w8a8_ep_dispatch_workspace_size": ([vp, i32], sz),
+            "moe_w8a8_ep_experts_workspace_size": ([vp, i32], sz),
+            "moe_w8a8_ep_dispatch": ([vp, vp, i32, vp, vp, vp, vp, vp, sz, vp, vp], i32),
+            "moe_w8a8_ep_experts": ([vp, vp, i32, vp, vp, sz, vp, vp], i32),
+            "moe_w8a8_ep_combine": ([vp, vp, i32, vp, vp, sz, vp], i32),
         }
         for name, (args, res) in sig.items():
             fn = getattr(L, name)
@@ -189,11 +200,15 @@ def moe_w8a8_calibrate_absmax(x, absmax, stream=None):
 
 
 class Weights:
-    """Owner of a prepared-weights handle (destroyed with the object)."""
+    """Owner of a prepared-weights handle (destroyed with the object); it
+    holds experts [expert_first, expert_first + n_local) of the layer."""
 
-    def __init__(self, handle: ctypes.c_void_p, cfg: moe_w8a8_config):
+    def __init__(self, handle: ctypes.c_void_p, cfg: moe_w8a8_config, expert_first: int = 0,
+                 n_local: int | None = None):
         self.handle = handle
         self.cfg = cfg
+        self.expert_first = expert_first
+        self.n_local = cfg.n_experts if n_local is None else n_local
 
     def __del__(self):
         if getattr(self, "handle", None) and _lib is not None:
@@ -290,7 +305,7 @@ def moe_w8a8_get_smooth_scales(w: Weights):
 def moe_w8a8_export_weights(w: Weights, stream=None) -> dict:
     torch = _torch()
     c = w.cfg
-    E, d, f = c.n_experts, c.d, c.f
+    E, d, f = w.n_local, c.d, c.f
     dev = torch.device("cuda")
     out = dict(wq_gate=torch.empty((E, f, d), dtype=torch.int8, device=dev),
                wq_up=torch.empty((E, f, d), dtype=torch.int8, device=dev),
@@ -357,3 +372,77 @@ def moe_w8a8_status_words(w: Weights, n: int = 5, stream=None):
     _check(lib().moe_w8a8_status_words(w.handle, ctypes.c_void_p(out.ctypes.data), int(n),
                                        _stream(stream)), "moe_w8a8_status_words")
     return out
+
+
+# ------------------------------------------------------------------ expert parallelism
+
+def _nbytes(t) -> int:
+    return t.numel() * t.element_size()
+
+
+def moe_w8a8_ep_row_bytes(w: Weights) -> int:
+    return int(lib().moe_w8a8_ep_row_bytes(w.handle))
+
+
+def moe_w8a8_gateup_absmax(cfg: moe_w8a8_config, w_gate, w_up, aw, stream=None):
+    torch = _torch()
+    f32 = torch.float32
+    _check(lib().moe_w8a8_gateup_absmax(ctypes.byref(cfg), int(w_gate.shape[0]), _dev_ptr(w_gate, f32, "w_gate"),
+                                        _dev_ptr(w_up, f32, "w_up"), _dev_ptr(aw, f32, "aw"), _stream(stream)),
+           "moe_w8a8_gateup_absmax")
+
+
+def moe_w8a8_prepare_shard(cfg: moe_w8a8_config, expert_first: int, w_gate, w_up, w_down, w_router,
+                           act_absmax, gateup_absmax, stream=None) -> Weights:
+    torch = _torch()
+    f32 = torch.float32
+    n_local = int(w_gate.shape[0])
+    h = ctypes.c_void_p()
+    _check(lib().moe_w8a8_prepare_shard(ctypes.byref(cfg), int(expert_first), n_local,
+                                        _dev_ptr(w_gate, f32, "w_gate"), _dev_ptr(w_up, f32, "w_up"),
+                                        _dev_ptr(w_down, f32, "w_down"), _dev_ptr(w_router, f32, "w_router"),
+                                        _dev_ptr(act_absmax, f32, "act_absmax"),
+                                        _dev_ptr(gateup_absmax, f32, "gateup_absmax"), _stream(stream),
+                                        ctypes.byref(h)), "moe_w8a8_prepare_shard")
+    return Weights(h, cfg, int(expert_first), n_local)
+
+
+def moe_w8a8_ep_dispatch_workspace_size(w: Weights, max_tokens: int) -> int:
+    return int(lib().moe_w8a8_ep_dispatch_workspace_size(w.handle, int(max_tokens)))
+
+
+def moe_w8a8_ep_experts_workspace_size(w: Weights, rows: int) -> int:
+    return int(lib().moe_w8a8_ep_experts_workspace_size(w.handle, int(rows)))
+
+
+def moe_w8a8_ep_dispatch(w: Weights, x, T: int, router_bias, router_logits, send, expert_offsets, workspace,
+                         dbg: dict | None = None, stream=None):
+    torch = _torch()
+    _s, dptr = _debug_struct(dbg)
+    _check(lib().moe_w8a8_ep_dispatch(
+        w.handle, _dev_ptr(x, _act_dtype(w.cfg.in_dtype), "x", T == 0), int(T),
+        _dev_ptr(router_bias, torch.float32, "router_bias", True),
+        _dev_ptr(router_logits, torch.float32, "router_logits", True),
+        _dev_ptr(send, torch.uint8, "send", T == 0), _dev_ptr(expert_offsets, torch.int32, "expert_offsets"),
+        _dev_ptr(workspace, name="workspace", allow_none=T == 0),
+        0 if workspace is None else _nbytes(workspace), dptr, _stream(stream)), "moe_w8a8_ep_dispatch")
+
+
+def moe_w8a8_ep_experts(w: Weights, recv, R: int, o_rows, workspace, dbg: dict | None = None, stream=None):
+    torch = _torch()
+    if R == 0:
+        return
+    _s, dptr = _debug_struct(dbg)
+    _check(lib().moe_w8a8_ep_experts(
+        w.handle, _dev_ptr(recv, torch.uint8, "recv"), int(R), _dev_ptr(o_rows, torch.float32, "o_rows"),
+        _dev_ptr(workspace, name="workspace"), _nbytes(workspace), dptr, _stream(stream)), "moe_w8a8_ep_experts")
+
+
+def moe_w8a8_ep_combine(w: Weights, o_rows, T: int, y, workspace, stream=None):
+    torch = _torch()
+    if T == 0:
+        return
+    o_ptr = None if o_rows is None or o_rows.numel() == 0 else _dev_ptr(o_rows, torch.float32, "o_rows")
+    _check(lib().moe_w8a8_ep_combine(
+        w.handle, o_ptr, int(T), _dev_ptr(y, _act_dtype(w.cfg.out_dtype), "y"),
+        _dev_ptr(workspace, name="workspace"), _nbytes(workspace), _stream(stream)), "moe_w8a8_ep_combine")

@@ -16,13 +16,17 @@ struct moe_w8a8_weights {
     int path;               // MOE_PATH_*
     int stream_max_rows;    // AUTO: streaming path when T*k <= this
     float act_clip;         // > 0: cap of each token's smoothed range (saturating clip)
+    // experts held: global experts [ep_first, ep_first + n_local) of the layer's
+    // cfg.n_experts (all of them unless prepared as an expert-parallel shard)
+    int ep_first;
+    int n_local;
     int last_launches;
     // prepared weights (device)
-    int8_t* w_gu;     // [E][2f][d]: per 128-channel block, 128 gate rows then 128 up rows
-    int8_t* w_dn;     // [E][d][f]
-    float* sw_gate;   // [E][f]
-    float* sw_up;     // [E][f]
-    float* sw_dn;     // [E][d]
+    int8_t* w_gu;     // [n_local][2f][d]: per 128-channel block, 128 gate rows then 128 up rows
+    int8_t* w_dn;     // [n_local][d][f]
+    float* sw_gate;   // [n_local][f]
+    float* sw_up;     // [n_local][f]
+    float* sw_dn;     // [n_local][d]
     float* inv_s;     // [d]
     float* w_router;  // [d][E]
     // certified tensor-core router (bf16 X): W_g split into bf16 hi + lo rows
@@ -69,7 +73,21 @@ struct WsLayout {
     int fused_words;             // their number (0: no fused launch)
     size_t total;
 };
-WsLayout ws_layout(const moe_w8a8_weights* w, int T);
+// Which calls use the layout: the whole forward; the routing side of the
+// expert-parallel layer (dispatch and combine: routing state, token codes,
+// no expert buffers); or its expert side (received rows, no routing).
+enum WsPart { WS_FORWARD, WS_ROUTE, WS_EXPERTS };
+WsLayout ws_layout(const moe_w8a8_weights* w, int T, WsPart part = WS_FORWARD);
+
+// Expert-parallel row: d code bytes, then this trailer.
+struct EpTrailer {
+    float sx;        // the token's activation scale
+    float w;         // the slot's gate weight
+    int32_t expert;  // global expert
+    int32_t ts;      // t * k + slot on the sending rank
+};
+constexpr int kEpTrailerBytes = 16;
+static_assert(sizeof(EpTrailer) == kEpTrailerBytes, "trailer layout");
 
 // meta[] words written by the permute scatter kernel
 enum { META_R = 0, META_NACTIVE = 1, META_NTILES = 2, META_WORDS = 8 };
@@ -101,10 +119,23 @@ cudaError_t launch_route_small(const float* logits, const float* bias, int T, in
                                int renorm, int cap, int32_t* idx, float* wts, float* logits_out,
                                int32_t* offsets, int32_t* row2ts, int32_t* ts2row, int32_t* meta,
                                int32_t* active, int32_t* tiles, int32_t* zero_words, int n_zero, cudaStream_t s);
-// act_clip > 0 caps each token's range (saturating clip), 0 = off.
+// act_clip > 0 caps each token's range (saturating clip), 0 = off.  Codes of
+// each kept (t, slot) go to row ts2row of aq (row stride aq_ld bytes; aq may be
+// null); with wts and idx given, an EpTrailer follows the d codes of each row.
 cudaError_t launch_smooth_quant(const void* x, int in_dtype, const float* inv_s, float act_clip, int T,
                                 int d, int k, const int32_t* ts2row, int8_t* xq, float* sx, int8_t* aq,
-                                int fmt, cudaStream_t s);
+                                int64_t aq_ld, const float* wts, const int32_t* idx, int fmt, cudaStream_t s);
+// Expert-parallel receive side.  Local expert of each received row (its
+// trailer's expert - ep_first); an expert outside [0, n_local) is recorded in
+// status (MOE_ERR_INVALID_ARG, site kSiteEpExpert) and the row runs through
+// local expert 0.
+constexpr int kSiteEpExpert = 14;
+cudaError_t launch_ep_read_experts(const uint8_t* recv, int R, int64_t row_bytes, int d, int ep_first,
+                                   int n_local, int32_t* idx, int32_t* status, cudaStream_t s);
+// Codes of received row r to row ts2row[r] of dst (row r when ts2row is
+// null), its scale and gate weight to sx[r] and wts[r].
+cudaError_t launch_ep_gather(const uint8_t* recv, int R, int64_t row_bytes, int d, const int32_t* ts2row,
+                             int8_t* dst, float* sx, float* wts, cudaStream_t s);
 // out[r][j] = |fp32(x[r][j] * inv_s[j])| (calibration of the activation clip)
 cudaError_t launch_scaled_abs(const void* x, int64_t rows, int d, int dtype, const float* inv_s, float* out,
                               cudaStream_t s);

@@ -783,7 +783,7 @@ template <int kSqMaxGroups, int FMT>   // groups of 8 channels per thread: d <= 
 __global__ void __launch_bounds__(kSqThreads) smooth_quant_kernel(
     const void* __restrict__ x, int in_dtype, const float* __restrict__ inv_s, float act_clip, int T, int d,
     int k, const int32_t* __restrict__ ts2row, int8_t* __restrict__ xq, float* __restrict__ sx,
-    int8_t* __restrict__ aq) {
+    int8_t* __restrict__ aq, int64_t aq_ld, const float* __restrict__ wts, const int32_t* __restrict__ idx) {
     // X is an input of the forward and xq / sx are read only by later kernels of
     // this forward: when this kernel starts (its predecessor has passed its own
     // wait) every kernel of the previous forward has finished, so the codes are
@@ -846,7 +846,59 @@ __global__ void __launch_bounds__(kSqThreads) smooth_quant_kernel(
         if (g >= ng) continue;
 #pragma unroll
         for (int sl = 0; sl < kMaxK; ++sl)
-            if (rows[sl] >= 0) *reinterpret_cast<uint2*>(aq + (int64_t)rows[sl] * d + g * 8) = packed[gi];
+            if (rows[sl] >= 0) *reinterpret_cast<uint2*>(aq + (int64_t)rows[sl] * aq_ld + g * 8) = packed[gi];
+    }
+    if (wts && tid < k) {   // expert-parallel send rows: the trailer after the codes
+        const int64_t ts = (int64_t)t * k + tid;
+        const int row = ts2row[ts];
+        if (row >= 0)
+            *reinterpret_cast<int4*>(aq + (int64_t)row * aq_ld + d) =
+                make_int4(__float_as_int(s), __float_as_int(wts[ts]), idx[ts], (int)ts);
+    }
+}
+
+// Expert-parallel receive side: the local expert of each received row.
+__global__ void ep_read_experts_kernel(const uint8_t* __restrict__ recv, int R, int64_t row_bytes, int d,
+                                       int ep_first, int n_local, int32_t* __restrict__ idx,
+                                       int32_t* __restrict__ status) {
+    pdl_wait();
+    pdl_trigger();
+    const int r = blockIdx.x * blockDim.x + threadIdx.x;
+    if (r >= R) return;
+    const EpTrailer* tr = reinterpret_cast<const EpTrailer*>(recv + (int64_t)r * row_bytes + d);
+    const int e = tr->expert - ep_first;
+    if (e < 0 || e >= n_local) {
+        if (atomicCAS(status, 0, (int32_t)MOE_ERR_INVALID_ARG) == 0) {
+            status[1] = kSiteEpExpert;
+            status[2] = r;
+            status[3] = tr->expert;
+        }
+        idx[r] = 0;
+        return;
+    }
+    idx[r] = e;
+}
+
+// Codes of each received row to its sorted row (or row r), scale and gate
+// weight to sx[r], wts[r]: one warp per row, 16-byte copies.
+constexpr int kEpGatherWarps = 8;
+__global__ void __launch_bounds__(kEpGatherWarps * 32) ep_gather_kernel(
+    const uint8_t* __restrict__ recv, int R, int64_t row_bytes, int d, const int32_t* __restrict__ ts2row,
+    int8_t* __restrict__ dst, float* __restrict__ sx, float* __restrict__ wts) {
+    pdl_wait();
+    pdl_trigger();
+    const int lane = threadIdx.x & 31;
+    const int r = blockIdx.x * kEpGatherWarps + (threadIdx.x >> 5);
+    if (r >= R) return;
+    const uint8_t* src = recv + (int64_t)r * row_bytes;
+    const int64_t drow = ts2row ? ts2row[r] : r;
+    int8_t* out = dst + drow * d;
+    for (int j = lane * 16; j < d; j += 32 * 16)
+        *reinterpret_cast<int4*>(out + j) = *reinterpret_cast<const int4*>(src + j);
+    if (lane == 0) {
+        const EpTrailer* tr = reinterpret_cast<const EpTrailer*>(src + d);
+        sx[r] = tr->sx;
+        wts[r] = tr->w;
     }
 }
 
@@ -946,7 +998,7 @@ cudaError_t launch_route_small(const float* logits, const float* bias, int T, in
 
 cudaError_t launch_smooth_quant(const void* x, int in_dtype, const float* inv_s, float act_clip, int T,
                                 int d, int k, const int32_t* ts2row, int8_t* xq, float* sx, int8_t* aq,
-                                int fmt, cudaStream_t s) {
+                                int64_t aq_ld, const float* wts, const int32_t* idx, int fmt, cudaStream_t s) {
     const int groups = (d / 8 + kSqThreads - 1) / kSqThreads;
     auto kern = fmt == FMT_E4M3
                     ? (groups <= 4 ? smooth_quant_kernel<4, FMT_E4M3>
@@ -954,7 +1006,19 @@ cudaError_t launch_smooth_quant(const void* x, int in_dtype, const float* inv_s,
                     : (groups <= 4 ? smooth_quant_kernel<4, FMT_INT8>
                                    : groups <= 8 ? smooth_quant_kernel<8, FMT_INT8> : smooth_quant_kernel<16, FMT_INT8>);
     return launch_pdl(kern, dim3(T), dim3(kSqThreads), 0, s, x, in_dtype, inv_s, act_clip, T, d, k, ts2row, xq,
-                      sx, aq);
+                      sx, aq, aq_ld, wts, idx);
+}
+
+cudaError_t launch_ep_read_experts(const uint8_t* recv, int R, int64_t row_bytes, int d, int ep_first,
+                                   int n_local, int32_t* idx, int32_t* status, cudaStream_t s) {
+    return launch_pdl(ep_read_experts_kernel, dim3((R + 255) / 256), dim3(256), 0, s, recv, R, row_bytes, d,
+                      ep_first, n_local, idx, status);
+}
+
+cudaError_t launch_ep_gather(const uint8_t* recv, int R, int64_t row_bytes, int d, const int32_t* ts2row,
+                             int8_t* dst, float* sx, float* wts, cudaStream_t s) {
+    return launch_pdl(ep_gather_kernel, dim3((R + kEpGatherWarps - 1) / kEpGatherWarps),
+                      dim3(kEpGatherWarps * 32), 0, s, recv, R, row_bytes, d, ts2row, dst, sx, wts);
 }
 
 }  // namespace moe

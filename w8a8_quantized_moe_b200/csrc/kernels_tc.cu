@@ -1139,7 +1139,7 @@ cudaError_t launch(const CUtensorMap& ta, const CUtensorMap& tb, const TcParams&
 
 bool tc_make_weight_maps(moe_w8a8_weights* w) {
     const moe_w8a8_config& c = w->cfg;
-    const uint64_t E = c.n_experts, d = c.d, f = c.f;
+    const uint64_t E = w->n_local, d = c.d, f = c.f;   // the experts this handle holds
     return make_map(&w->tm_w_gu, w->w_gu, d, E * 2 * f, BN) && make_map(&w->tm_w_dn, w->w_dn, f, E * d, BN);
 }
 

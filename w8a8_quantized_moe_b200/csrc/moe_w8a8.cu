@@ -108,7 +108,7 @@ void free_handle(moe_w8a8_weights* w) {
 
 namespace moe {
 
-WsLayout ws_layout(const moe_w8a8_weights* w, int T) {
+WsLayout ws_layout(const moe_w8a8_weights* w, int T, WsPart part) {
     const moe_w8a8_config& c = w->cfg;
     const int E = c.n_experts, k = c.top_k, d = c.d, f = c.f;
     const size_t tk = (size_t)T * k;
@@ -116,15 +116,16 @@ WsLayout ws_layout(const moe_w8a8_weights* w, int T) {
     const size_t nblk = (tk + kPermChunk - 1) / kPermChunk;
     const size_t max_tiles = (tk + kTileM - 1) / kTileM + E;
     const bool stream = choose_path(w, T) == MOE_PATH_STREAM;
+    const bool fwd = part == WS_FORWARD, route = part == WS_ROUTE, experts = part == WS_EXPERTS;
     WsLayout L{};
     size_t p = 0;
     auto take = [&](size_t bytes) { size_t at = p; p = align_up(p + bytes); return at; };
-    L.x_stage = take((size_t)T * d * in_b);
-    L.y_stage = take((size_t)T * d * out_b);
-    L.logits_stage = take((size_t)T * E * 4);
-    L.bias_stage = take((size_t)E * 4);
-    L.logits = take((size_t)T * E * 4);
-    L.logits_sel = take(router_tc_ok(w, T) ? (size_t)T * E * 4 : 0);
+    L.x_stage = take(fwd ? (size_t)T * d * in_b : 0);
+    L.y_stage = take(fwd ? (size_t)T * d * out_b : 0);
+    L.logits_stage = take(fwd ? (size_t)T * E * 4 : 0);
+    L.bias_stage = take(fwd ? (size_t)E * 4 : 0);
+    L.logits = take(experts ? 0 : (size_t)T * E * 4);
+    L.logits_sel = take(!experts && router_tc_ok(w, T) ? (size_t)T * E * 4 : 0);
     L.topk_idx = take(tk * 4);
     L.topk_w = take(tk * 4);
     L.hist = take(nblk * E * 4);
@@ -134,16 +135,17 @@ WsLayout ws_layout(const moe_w8a8_weights* w, int T) {
     L.tiles = take(max_tiles * 8);
     L.row2ts = take(tk * 4);
     L.ts2row = take(tk * 4);
-    L.xq = take((size_t)T * d);
+    L.xq = take(experts && !stream ? 0 : (size_t)T * d);
     L.sx = take((size_t)T * 4);
-    L.aq = take(stream ? 0 : tk * d);
-    L.acc1 = take(stream ? tk * 2 * f * 4 : 0);
-    L.hq = take(tk * f);
-    L.sh = take(tk * 4);
-    L.o = take(tk * d * 4);
-    L.h32 = take(stream ? 0 : tk * f * 4);
-    L.pamax = take(stream ? 0 : tk * (f / 64) * 4);
-    const bool fused = !stream && fused_ok(w, T);
+    const bool ex = !route;   // expert buffers
+    L.aq = take(ex && !stream ? tk * d : 0);
+    L.acc1 = take(ex && stream ? tk * 2 * f * 4 : 0);
+    L.hq = take(ex ? tk * f : 0);
+    L.sh = take(ex ? tk * 4 : 0);
+    L.o = take(ex ? tk * d * 4 : 0);
+    L.h32 = take(ex && !stream ? tk * f * 4 : 0);
+    L.pamax = take(ex && !stream ? tk * (f / 64) * 4 : 0);
+    const bool fused = ex && !stream && fused_ok(w, T);
     L.fused_sync = take(fused ? fused_sync_words(max_tiles) * 4 : 0);
     L.fused_words = fused ? (int)fused_sync_words(max_tiles) : 0;
     L.total = p;
@@ -244,20 +246,31 @@ moe_status moe_w8a8_calibrate_absmax(const void* x, int64_t rows, int32_t d, int
     return MOE_OK;
 }
 
-moe_status moe_w8a8_prepare(const moe_w8a8_config* cfg, const float* w_gate, const float* w_up,
-                            const float* w_down, const float* w_router, const float* act_absmax,
-                            moe_stream_t stream, moe_w8a8_weights** out) {
+}  // extern "C"
+
+namespace {
+
+// Prepare experts [e_first, e_first + n_local) of the layer (all of them for
+// the single-GPU handle).  gateup_absmax: the layer's aw (max over ALL experts)
+// on the device, or null to take it from the given experts.
+moe_status prepare_impl(const moe_w8a8_config* cfg, int e_first, int n_local, const float* w_gate,
+                        const float* w_up, const float* w_down, const float* w_router, const float* act_absmax,
+                        const float* gateup_absmax, moe_stream_t stream, moe_w8a8_weights** out) {
     if (!out) return MOE_ERR_INVALID_ARG;
     *out = nullptr;
     moe_status st = check_config(cfg);
     if (st != MOE_OK) return st;
     if (!w_gate || !w_up || !w_down || !w_router || !act_absmax) return MOE_ERR_INVALID_ARG;
     const moe_w8a8_config c = *cfg;
-    const int E = c.n_experts, d = c.d, f = c.f;
+    if (e_first < 0 || n_local <= 0 || e_first + n_local > c.n_experts) return MOE_ERR_INVALID_ARG;
+    const int E = n_local, d = c.d, f = c.f;   // expert arrays hold the n_local experts
+    const int E_layer = c.n_experts;           // the router scores all of the layer's experts
     cudaStream_t s = (cudaStream_t)stream;
 
     moe_w8a8_weights* w = new moe_w8a8_weights();
     w->cfg = c;
+    w->ep_first = e_first;
+    w->n_local = n_local;
     w->path = MOE_PATH_AUTO;
     w->stream_max_rows = 32;   // measured crossover: streaming wins up to T*k = 32 rows
     if (cudaGetDevice(&w->device) != cudaSuccess ||
@@ -271,7 +284,7 @@ moe_status moe_w8a8_prepare(const moe_w8a8_config* cfg, const float* w_gate, con
               cudaMalloc(&w->sw_up, (size_t)E * f * 4) == cudaSuccess &&
               cudaMalloc(&w->sw_dn, (size_t)E * d * 4) == cudaSuccess &&
               cudaMalloc(&w->inv_s, (size_t)d * 4) == cudaSuccess &&
-              cudaMalloc(&w->w_router, (size_t)d * E * 4) == cudaSuccess &&
+              cudaMalloc(&w->w_router, (size_t)d * E_layer * 4) == cudaSuccess &&
               cudaMalloc(&w->status, 64) == cudaSuccess;
     w->s_host = (float*)std::malloc((size_t)d * 4);
     float* tmp = nullptr;   // aw [d] then s [d] on the device
@@ -289,12 +302,13 @@ moe_status moe_w8a8_prepare(const moe_w8a8_config* cfg, const float* w_gate, con
     };
     float* aw_dev = tmp;
     float* s_dev = tmp + d;
-    if (cudaMemsetAsync(w->status, 0, 64, s) != cudaSuccess ||
-        cudaMemsetAsync(aw_dev, 0, (size_t)d * 4, s) != cudaSuccess ||
-        launch_gateup_input_absmax(w_gate, w_up, E, d, f, aw_dev, s) != cudaSuccess)
+    if (cudaMemsetAsync(w->status, 0, 64, s) != cudaSuccess) return fail(MOE_ERR_CUDA);
+    if (!gateup_absmax && (cudaMemsetAsync(aw_dev, 0, (size_t)d * 4, s) != cudaSuccess ||
+                           launch_gateup_input_absmax(w_gate, w_up, E, d, f, aw_dev, s) != cudaSuccess))
         return fail(MOE_ERR_CUDA);
     std::vector<float> aw(d), ax(d), inv(d);
-    if (cudaMemcpyAsync(aw.data(), aw_dev, (size_t)d * 4, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+    if (cudaMemcpyAsync(aw.data(), gateup_absmax ? gateup_absmax : aw_dev, (size_t)d * 4, cudaMemcpyDeviceToHost,
+                        s) != cudaSuccess ||
         cudaMemcpyAsync(ax.data(), act_absmax, (size_t)d * 4, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
         cudaStreamSynchronize(s) != cudaSuccess)
         return fail(MOE_ERR_CUDA);
@@ -319,7 +333,7 @@ moe_status moe_w8a8_prepare(const moe_w8a8_config* cfg, const float* w_gate, con
                                  kGuBlock, w->sw_up, fmt, s) != cudaSuccess ||
         launch_quantize_channels(w_down, nullptr, E, f, d, w->w_dn, d, d, d, 0, w->sw_dn, fmt, s) !=
             cudaSuccess ||
-        cudaMemcpyAsync(w->w_router, w_router, (size_t)d * E * 4, cudaMemcpyDeviceToDevice, s) !=
+        cudaMemcpyAsync(w->w_router, w_router, (size_t)d * E_layer * 4, cudaMemcpyDeviceToDevice, s) !=
             cudaSuccess ||
         cudaStreamSynchronize(s) != cudaSuccess)
         return fail(MOE_ERR_CUDA);
@@ -330,168 +344,280 @@ moe_status moe_w8a8_prepare(const moe_w8a8_config* cfg, const float* w_gate, con
     return MOE_OK;
 }
 
+}  // namespace
+
+extern "C" {
+
+moe_status moe_w8a8_prepare(const moe_w8a8_config* cfg, const float* w_gate, const float* w_up,
+                            const float* w_down, const float* w_router, const float* act_absmax,
+                            moe_stream_t stream, moe_w8a8_weights** out) {
+    if (!cfg) {
+        if (out) *out = nullptr;
+        return MOE_ERR_INVALID_ARG;
+    }
+    return prepare_impl(cfg, 0, cfg->n_experts, w_gate, w_up, w_down, w_router, act_absmax, nullptr, stream, out);
+}
 
 size_t moe_w8a8_workspace_size(const moe_w8a8_weights* w, int32_t max_tokens) {
     if (!w || max_tokens < 0) return 0;
     return ws_layout(w, max_tokens).total;
 }
 
-static moe_status forward_impl(const moe_w8a8_weights* w, const void* x, int T, const float* bias,
-                               const float* given_logits, void* y, char* ws,
-                               const moe_w8a8_debug* dbg, cudaStream_t s) {
-    const moe_w8a8_config& c = w->cfg;
-    const int E = c.n_experts, k = c.top_k, d = c.d, f = c.f;
-    const WsLayout L = ws_layout(w, T);
-    const int path = choose_path(w, T);
+}  // extern "C"
+
+namespace {
+
+// One call's launch context: the handle whose cfg describes the call (for the
+// expert side of the expert-parallel layer a view of it), the workspace and its
+// layout, the debug buffers and the per-stage profiling marks.
+struct Run {
+    const moe_w8a8_weights* w;
+    WsLayout L;
+    char* ws;
+    const moe_w8a8_debug* dbg;
+    cudaStream_t s;
+    bool prof;
     int launches = 0;
-    auto P = [&](size_t off) { return (void*)(ws + off); };
-    float* logits = (float*)P(L.logits);
-    int32_t* idx = (int32_t*)P(L.topk_idx);
-    float* wts = (float*)P(L.topk_w);
-    int32_t* offsets = (int32_t*)P(L.offsets);
-    int32_t* meta = (int32_t*)P(L.meta);
-    int32_t* active = (int32_t*)P(L.active);
-    int32_t* tiles = (int32_t*)P(L.tiles);
-    int32_t* row2ts = (int32_t*)P(L.row2ts);
-    int32_t* ts2row = (int32_t*)P(L.ts2row);
-    int8_t* xq = (int8_t*)P(L.xq);
-    float* sx = (float*)P(L.sx);
-    int8_t* hq = (int8_t*)P(L.hq);
-    float* sh = (float*)P(L.sh);
-    float* o = (float*)P(L.o);
-    const size_t tk = (size_t)T * k;
-    moe_w8a8_weights* mw = const_cast<moe_w8a8_weights*>(w);
-    const bool prof = w->prof_events && w->prof_n < w->prof_max;
-    auto mark = [&](int stage, int edge) {
+
+    Run(const moe_w8a8_weights* w_, const WsLayout& L_, char* ws_, const moe_w8a8_debug* dbg_, cudaStream_t s_)
+        : w(w_), L(L_), ws(ws_), dbg(dbg_), s(s_), prof(w_->prof_events && w_->prof_n < w_->prof_max) {}
+    template <class V>
+    V* at(size_t off) const { return reinterpret_cast<V*>(ws + off); }
+    void mark(int stage, int edge) const {
         if (prof) cudaEventRecord(w->prof_events[(w->prof_n * MOE_N_STAGES + stage) * 2 + edge], s);
-    };
-    auto empty_stage = [&](int stage) { mark(stage, 0); mark(stage, 1); };
+    }
+    void empty_stage(int stage) const { mark(stage, 0); mark(stage, 1); }
+};
+
+// Router, top-k and the expert-major permutation (with capacity) of T tokens
+// over the layer's E experts.
+moe_status route_stage(Run& r, const void* x, int T, const float* bias, const float* given_logits, int path) {
+    const moe_w8a8_weights* w = r.w;
+    const moe_w8a8_config& c = w->cfg;
+    const int E = c.n_experts, k = c.top_k, d = c.d;
+    const WsLayout& L = r.L;
+    cudaStream_t s = r.s;
+    float* logits = r.at<float>(L.logits);
+    int32_t* idx = r.at<int32_t>(L.topk_idx);
+    float* wts = r.at<float>(L.topk_w);
+    int32_t* offsets = r.at<int32_t>(L.offsets);
+    int32_t* meta = r.at<int32_t>(L.meta);
+    int32_t* active = r.at<int32_t>(L.active);
+    int32_t* tiles = r.at<int32_t>(L.tiles);
+    int32_t* row2ts = r.at<int32_t>(L.row2ts);
+    int32_t* ts2row = r.at<int32_t>(L.ts2row);
+    float* dbg_logits = r.dbg ? r.dbg->logits : nullptr;
 
     const float* lsrc = given_logits;
     const bool certified = !lsrc && router_tc_ok(w, T) && ((uintptr_t)x & 15) == 0;
     if (certified) {
         // approximate logits on the tensor cores, then per token the candidates'
         // logits in the stated order, top-k and gate weights
-        mark(MOE_STAGE_ROUTER, 0);
+        r.mark(MOE_STAGE_ROUTER, 0);
         CUDA_TRY(launch_router_tc(w, x, T, logits, s));
-        mark(MOE_STAGE_ROUTER, 1);
-        mark(MOE_STAGE_TOPK, 0);
-        CUDA_TRY(launch_router_select(w, x, T, logits, bias, (float*)P(L.logits_sel), idx, wts,
-                                      dbg ? dbg->logits : nullptr, s));
-        mark(MOE_STAGE_TOPK, 1);
-        launches += 2;
+        r.mark(MOE_STAGE_ROUTER, 1);
+        r.mark(MOE_STAGE_TOPK, 0);
+        CUDA_TRY(launch_router_select(w, x, T, logits, bias, r.at<float>(L.logits_sel), idx, wts, dbg_logits, s));
+        r.mark(MOE_STAGE_TOPK, 1);
+        r.launches += 2;
     } else if (!lsrc) {
-        mark(MOE_STAGE_ROUTER, 0);
+        r.mark(MOE_STAGE_ROUTER, 0);
         CUDA_TRY(launch_router_logits(x, c.in_dtype, w->w_router, T, d, E, logits, s));
-        mark(MOE_STAGE_ROUTER, 1);
-        ++launches;
+        r.mark(MOE_STAGE_ROUTER, 1);
+        ++r.launches;
         lsrc = logits;
     } else {
-        empty_stage(MOE_STAGE_ROUTER);
+        r.empty_stage(MOE_STAGE_ROUTER);
     }
     if (certified) {
-        mark(MOE_STAGE_PERMUTE, 0);
-        CUDA_TRY(launch_permute(idx, T, k, E, capacity_of(c, T), (int32_t*)P(L.hist), offsets, row2ts,
-                                ts2row, meta, active, tiles, s));
-        mark(MOE_STAGE_PERMUTE, 1);
-        launches += 2;
+        r.mark(MOE_STAGE_PERMUTE, 0);
+        CUDA_TRY(launch_permute(idx, T, k, E, capacity_of(c, T), r.at<int32_t>(L.hist), offsets, row2ts, ts2row,
+                                meta, active, tiles, s));
+        r.mark(MOE_STAGE_PERMUTE, 1);
+        r.launches += 2;
     } else if (route_small_ok(T, k)) {
         // top-k, histogram, scan and scatter in one block
-        mark(MOE_STAGE_TOPK, 0);
+        r.mark(MOE_STAGE_TOPK, 0);
         const bool fused = path == MOE_PATH_TENSOR && L.fused_words > 0;
-        CUDA_TRY(launch_route_small(lsrc, bias, T, E, k, c.renormalize, capacity_of(c, T), idx, wts,
-                                    dbg ? dbg->logits : nullptr, offsets, row2ts, ts2row, meta,
-                                    active, tiles, fused ? (int32_t*)P(L.fused_sync) : nullptr,
-                                    fused ? L.fused_words : 0, s));
-        mark(MOE_STAGE_TOPK, 1);
-        empty_stage(MOE_STAGE_PERMUTE);
-        ++launches;
+        CUDA_TRY(launch_route_small(lsrc, bias, T, E, k, c.renormalize, capacity_of(c, T), idx, wts, dbg_logits,
+                                    offsets, row2ts, ts2row, meta, active, tiles,
+                                    fused ? r.at<int32_t>(L.fused_sync) : nullptr, fused ? L.fused_words : 0, s));
+        r.mark(MOE_STAGE_TOPK, 1);
+        r.empty_stage(MOE_STAGE_PERMUTE);
+        ++r.launches;
     } else {
-        mark(MOE_STAGE_TOPK, 0);
-        CUDA_TRY(launch_topk(lsrc, bias, T, E, k, c.renormalize, idx, wts, dbg ? dbg->logits : nullptr, s));
-        mark(MOE_STAGE_TOPK, 1);
-        ++launches;
-        mark(MOE_STAGE_PERMUTE, 0);
-        CUDA_TRY(launch_permute(idx, T, k, E, capacity_of(c, T), (int32_t*)P(L.hist), offsets, row2ts,
-                                ts2row, meta, active, tiles, s));
-        mark(MOE_STAGE_PERMUTE, 1);
-        launches += 2;
+        r.mark(MOE_STAGE_TOPK, 0);
+        CUDA_TRY(launch_topk(lsrc, bias, T, E, k, c.renormalize, idx, wts, dbg_logits, s));
+        r.mark(MOE_STAGE_TOPK, 1);
+        ++r.launches;
+        r.mark(MOE_STAGE_PERMUTE, 0);
+        CUDA_TRY(launch_permute(idx, T, k, E, capacity_of(c, T), r.at<int32_t>(L.hist), offsets, row2ts, ts2row,
+                                meta, active, tiles, s));
+        r.mark(MOE_STAGE_PERMUTE, 1);
+        r.launches += 2;
     }
-    if (path == MOE_PATH_STREAM) {
-        mark(MOE_STAGE_QUANT, 0);
-        CUDA_TRY(launch_smooth_quant(x, c.in_dtype, w->inv_s, w->act_clip, T, d, k, ts2row, xq, sx, nullptr,
-                                     MOE_FMT_INT8, s));
-        mark(MOE_STAGE_QUANT, 1);
-        int32_t* acc1 = (int32_t*)P(L.acc1);
-        mark(MOE_STAGE_GEMM1, 0);
-        CUDA_TRY(launch_stream_gateup(w, T, xq, row2ts, offsets, active, meta, acc1, s));
-        mark(MOE_STAGE_GEMM1, 1);
-        mark(MOE_STAGE_REQUANT, 0);
-        CUDA_TRY(launch_swiglu_requant(w, acc1, row2ts, idx, sx, meta, (int)tk, hq, sh, s));
-        mark(MOE_STAGE_REQUANT, 1);
-        mark(MOE_STAGE_GEMM2, 0);
-        CUDA_TRY(launch_stream_down(w, T, hq, sh, row2ts, wts, offsets, active, meta, o,
-                                    dbg ? dbg->acc2 : nullptr, s));
-        mark(MOE_STAGE_GEMM2, 1);
-        launches += 4;
-        if (dbg && dbg->acc1)
-            CUDA_TRY(cudaMemcpyAsync(dbg->acc1, acc1, tk * 2 * f * 4, cudaMemcpyDeviceToDevice, s));
-    } else {
-        int8_t* aq = (int8_t*)P(L.aq);
-        mark(MOE_STAGE_QUANT, 0);
-        CUDA_TRY(launch_smooth_quant(x, c.in_dtype, w->inv_s, w->act_clip, T, d, k, ts2row, xq, sx, aq,
-                                     c.expert_format, s));
-        mark(MOE_STAGE_QUANT, 1);
-        if (L.fused_words > 0) {
-            // few rows per expert: GEMM1, requantisation and GEMM2 in one launch
-            // (its time is reported as the GEMM1 stage)
-            mark(MOE_STAGE_GEMM1, 0);
-            CUDA_TRY(launch_tc_ffn_fused(w, T, aq, meta, tiles, offsets, row2ts, sx, wts, (float*)P(L.h32),
-                                         (float*)P(L.pamax), hq, sh, o, dbg ? dbg->acc1 : nullptr,
-                                         dbg ? dbg->acc2 : nullptr, (int32_t*)P(L.fused_sync), s));
-            mark(MOE_STAGE_GEMM1, 1);
-            empty_stage(MOE_STAGE_REQUANT);
-            empty_stage(MOE_STAGE_GEMM2);
-            launches += 2;
-        } else {
-            mark(MOE_STAGE_GEMM1, 0);
-            CUDA_TRY(launch_tc_gemm1(w, T, aq, meta, tiles, offsets, row2ts, sx, (float*)P(L.h32),
-                                     (float*)P(L.pamax), dbg ? dbg->acc1 : nullptr, s));
-            mark(MOE_STAGE_GEMM1, 1);
-            mark(MOE_STAGE_REQUANT, 0);
-            CUDA_TRY(launch_requant((float*)P(L.h32), (float*)P(L.pamax), f, meta, (int)tk, hq, sh,
-                                    c.expert_format, s));
-            mark(MOE_STAGE_REQUANT, 1);
-            mark(MOE_STAGE_GEMM2, 0);
-            CUDA_TRY(launch_tc_gemm2(w, T, hq, sh, meta, tiles, offsets, row2ts, wts, o,
-                                     dbg ? dbg->acc2 : nullptr, s));
-            mark(MOE_STAGE_GEMM2, 1);
-            launches += 4;
-        }
-    }
-    mark(MOE_STAGE_COMBINE, 0);
-    CUDA_TRY(launch_combine(o, ts2row, T, k, d, c.out_dtype, y, s));
-    mark(MOE_STAGE_COMBINE, 1);
-    ++launches;
-    if (prof) ++mw->prof_n;
-    if (dbg) {
-        auto cp = [&](void* dst, const void* src, size_t bytes) {
-            return dst ? cudaMemcpyAsync(dst, src, bytes, cudaMemcpyDeviceToDevice, s) : cudaSuccess;
-        };
-        CUDA_TRY(cp(dbg->topk_idx, idx, tk * 4));
-        CUDA_TRY(cp(dbg->topk_w, wts, tk * 4));
-        CUDA_TRY(cp(dbg->offsets, offsets, (size_t)(E + 1) * 4));
-        CUDA_TRY(cp(dbg->row2ts, row2ts, tk * 4));
-        CUDA_TRY(cp(dbg->ts2row, ts2row, tk * 4));
-        CUDA_TRY(cp(dbg->xq, xq, (size_t)T * d));
-        CUDA_TRY(cp(dbg->sx, sx, (size_t)T * 4));
-        CUDA_TRY(cp(dbg->hq, hq, tk * f));
-        CUDA_TRY(cp(dbg->sh, sh, tk * 4));
-        CUDA_TRY(cp(dbg->o, o, tk * d * 4));
-    }
-    mw->last_launches = launches;
     return MOE_OK;
 }
+
+// Smoothing and per-token quantisation; the codes of each kept (t, slot) go
+// to its sorted row of aq (row stride aq_ld), followed by the expert-parallel
+// trailer when `trailer` is set.
+moe_status quant_stage(Run& r, const void* x, int T, int8_t* aq, int64_t aq_ld, bool trailer, int fmt) {
+    const moe_w8a8_weights* w = r.w;
+    const moe_w8a8_config& c = w->cfg;
+    const WsLayout& L = r.L;
+    r.mark(MOE_STAGE_QUANT, 0);
+    CUDA_TRY(launch_smooth_quant(x, c.in_dtype, w->inv_s, w->act_clip, T, c.d, c.top_k, r.at<int32_t>(L.ts2row),
+                                 r.at<int8_t>(L.xq), r.at<float>(L.sx), aq, aq_ld,
+                                 trailer ? r.at<float>(L.topk_w) : nullptr,
+                                 trailer ? r.at<int32_t>(L.topk_idx) : nullptr, fmt, r.s));
+    r.mark(MOE_STAGE_QUANT, 1);
+    ++r.launches;
+    return MOE_OK;
+}
+
+// The experts of T*k sorted rows (codes in xq by token for the streaming path,
+// in aq by row for the tensor path; sx, topk_w, topk_idx by token / (t, slot))
+// to the per-row outputs O.
+moe_status expert_stage(Run& r, int T, int path) {
+    const moe_w8a8_weights* w = r.w;
+    const moe_w8a8_config& c = w->cfg;
+    const int k = c.top_k, f = c.f;
+    const WsLayout& L = r.L;
+    cudaStream_t s = r.s;
+    const moe_w8a8_debug* dbg = r.dbg;
+    const size_t tk = (size_t)T * k;
+    int32_t* idx = r.at<int32_t>(L.topk_idx);
+    float* wts = r.at<float>(L.topk_w);
+    int32_t* offsets = r.at<int32_t>(L.offsets);
+    int32_t* meta = r.at<int32_t>(L.meta);
+    int32_t* active = r.at<int32_t>(L.active);
+    int32_t* tiles = r.at<int32_t>(L.tiles);
+    int32_t* row2ts = r.at<int32_t>(L.row2ts);
+    float* sx = r.at<float>(L.sx);
+    int8_t* hq = r.at<int8_t>(L.hq);
+    float* sh = r.at<float>(L.sh);
+    float* o = r.at<float>(L.o);
+    if (path == MOE_PATH_STREAM) {
+        int32_t* acc1 = r.at<int32_t>(L.acc1);
+        r.mark(MOE_STAGE_GEMM1, 0);
+        CUDA_TRY(launch_stream_gateup(w, T, r.at<int8_t>(L.xq), row2ts, offsets, active, meta, acc1, s));
+        r.mark(MOE_STAGE_GEMM1, 1);
+        r.mark(MOE_STAGE_REQUANT, 0);
+        CUDA_TRY(launch_swiglu_requant(w, acc1, row2ts, idx, sx, meta, (int)tk, hq, sh, s));
+        r.mark(MOE_STAGE_REQUANT, 1);
+        r.mark(MOE_STAGE_GEMM2, 0);
+        CUDA_TRY(launch_stream_down(w, T, hq, sh, row2ts, wts, offsets, active, meta, o,
+                                    dbg ? dbg->acc2 : nullptr, s));
+        r.mark(MOE_STAGE_GEMM2, 1);
+        r.launches += 3;
+        if (dbg && dbg->acc1)
+            CUDA_TRY(cudaMemcpyAsync(dbg->acc1, acc1, tk * 2 * f * 4, cudaMemcpyDeviceToDevice, s));
+        return MOE_OK;
+    }
+    int8_t* aq = r.at<int8_t>(L.aq);
+    if (L.fused_words > 0) {
+        // few rows per expert: GEMM1, requantisation and GEMM2 in one launch
+        // (its time is reported as the GEMM1 stage)
+        r.mark(MOE_STAGE_GEMM1, 0);
+        CUDA_TRY(launch_tc_ffn_fused(w, T, aq, meta, tiles, offsets, row2ts, sx, wts, r.at<float>(L.h32),
+                                     r.at<float>(L.pamax), hq, sh, o, dbg ? dbg->acc1 : nullptr,
+                                     dbg ? dbg->acc2 : nullptr, r.at<int32_t>(L.fused_sync), s));
+        r.mark(MOE_STAGE_GEMM1, 1);
+        r.empty_stage(MOE_STAGE_REQUANT);
+        r.empty_stage(MOE_STAGE_GEMM2);
+        r.launches += 1;
+        return MOE_OK;
+    }
+    r.mark(MOE_STAGE_GEMM1, 0);
+    CUDA_TRY(launch_tc_gemm1(w, T, aq, meta, tiles, offsets, row2ts, sx, r.at<float>(L.h32), r.at<float>(L.pamax),
+                             dbg ? dbg->acc1 : nullptr, s));
+    r.mark(MOE_STAGE_GEMM1, 1);
+    r.mark(MOE_STAGE_REQUANT, 0);
+    CUDA_TRY(launch_requant(r.at<float>(L.h32), r.at<float>(L.pamax), f, meta, (int)tk, hq, sh, c.expert_format, s));
+    r.mark(MOE_STAGE_REQUANT, 1);
+    r.mark(MOE_STAGE_GEMM2, 0);
+    CUDA_TRY(launch_tc_gemm2(w, T, hq, sh, meta, tiles, offsets, row2ts, wts, o, dbg ? dbg->acc2 : nullptr, s));
+    r.mark(MOE_STAGE_GEMM2, 1);
+    r.launches += 3;
+    return MOE_OK;
+}
+
+// Copies of the intermediates a debug struct asks for (T tokens, k slots,
+// E experts in the offsets array; token codes and expert buffers if present).
+moe_status debug_stage(Run& r, int T, int k, int E, bool token_codes, bool expert_bufs) {
+    const moe_w8a8_debug* dbg = r.dbg;
+    if (!dbg) return MOE_OK;
+    const WsLayout& L = r.L;
+    const size_t tk = (size_t)T * k;
+    const int d = r.w->cfg.d, f = r.w->cfg.f;
+    auto cp = [&](void* dst, size_t off, size_t bytes) {
+        return dst ? cudaMemcpyAsync(dst, r.ws + off, bytes, cudaMemcpyDeviceToDevice, r.s) : cudaSuccess;
+    };
+    CUDA_TRY(cp(dbg->topk_idx, L.topk_idx, tk * 4));
+    CUDA_TRY(cp(dbg->topk_w, L.topk_w, tk * 4));
+    CUDA_TRY(cp(dbg->offsets, L.offsets, (size_t)(E + 1) * 4));
+    CUDA_TRY(cp(dbg->row2ts, L.row2ts, tk * 4));
+    CUDA_TRY(cp(dbg->ts2row, L.ts2row, tk * 4));
+    if (token_codes) CUDA_TRY(cp(dbg->xq, L.xq, (size_t)T * d));
+    CUDA_TRY(cp(dbg->sx, L.sx, (size_t)T * 4));
+    if (expert_bufs) {
+        CUDA_TRY(cp(dbg->hq, L.hq, tk * f));
+        CUDA_TRY(cp(dbg->sh, L.sh, tk * 4));
+        CUDA_TRY(cp(dbg->o, L.o, tk * d * 4));
+    }
+    return MOE_OK;
+}
+
+#define MOE_TRY(expr)                          \
+    do {                                       \
+        moe_status st_ = (expr);               \
+        if (st_ != MOE_OK) return st_;         \
+    } while (0)
+
+moe_status forward_impl(const moe_w8a8_weights* w, const void* x, int T, const float* bias,
+                        const float* given_logits, void* y, char* ws, const moe_w8a8_debug* dbg, cudaStream_t s) {
+    const moe_w8a8_config& c = w->cfg;
+    const int path = choose_path(w, T);
+    Run r(w, ws_layout(w, T), ws, dbg, s);
+    MOE_TRY(route_stage(r, x, T, bias, given_logits, path));
+    if (path == MOE_PATH_STREAM)
+        MOE_TRY(quant_stage(r, x, T, nullptr, c.d, false, MOE_FMT_INT8));
+    else
+        MOE_TRY(quant_stage(r, x, T, r.at<int8_t>(r.L.aq), c.d, false, c.expert_format));
+    MOE_TRY(expert_stage(r, T, path));
+    r.mark(MOE_STAGE_COMBINE, 0);
+    CUDA_TRY(launch_combine(r.at<float>(r.L.o), r.at<int32_t>(r.L.ts2row), T, c.top_k, c.d, c.out_dtype, y, s));
+    r.mark(MOE_STAGE_COMBINE, 1);
+    ++r.launches;
+    moe_w8a8_weights* mw = const_cast<moe_w8a8_weights*>(w);
+    if (r.prof) ++mw->prof_n;
+    MOE_TRY(debug_stage(r, T, c.top_k, c.n_experts, true, true));
+    mw->last_launches = r.launches;
+    return MOE_OK;
+}
+
+// The handle holds every expert of the layer (not an expert-parallel shard).
+bool holds_all_experts(const moe_w8a8_weights* w) { return w->ep_first == 0 && w->n_local == w->cfg.n_experts; }
+
+// The expert side of the expert-parallel layer: the held experts as a layer of
+// n_local experts with one slot per row, no capacity, no router and no
+// profiling (the kernels index scales and gate weights by row).
+moe_w8a8_weights expert_view(const moe_w8a8_weights* w) {
+    moe_w8a8_weights v = *w;
+    v.cfg.n_experts = w->n_local;
+    v.cfg.top_k = 1;
+    v.cfg.capacity_factor = 0.0f;
+    v.ep_first = 0;
+    v.rt_epad = 0;
+    v.prof_events = nullptr;
+    v.prof_max = v.prof_n = 0;
+    return v;
+}
+
+}  // namespace
+
+extern "C" {
 
 moe_status moe_w8a8_forward(const moe_w8a8_weights* w, const void* x, int32_t T,
                             const float* router_bias, const float* router_logits, void* y,
@@ -499,7 +625,7 @@ moe_status moe_w8a8_forward(const moe_w8a8_weights* w, const void* x, int32_t T,
                             moe_stream_t stream) {
     if (!w || T < 0) return MOE_ERR_INVALID_ARG;
     if (T == 0) return MOE_OK;
-    if (!x || !y || !workspace) return MOE_ERR_INVALID_ARG;
+    if (!x || !y || !workspace || !holds_all_experts(w)) return MOE_ERR_INVALID_ARG;
     if ((uintptr_t)workspace % kAlign) return MOE_ERR_INVALID_ARG;
     if (!path_ok(w, T)) return MOE_ERR_UNSUPPORTED_SHAPE;
     if (workspace_bytes < ws_layout(w, T).total) return MOE_ERR_WORKSPACE_TOO_SMALL;
@@ -513,7 +639,7 @@ moe_status moe_w8a8_forward_host(const moe_w8a8_weights* w, const void* x_host, 
                                  moe_stream_t stream) {
     if (!w || T < 0) return MOE_ERR_INVALID_ARG;
     if (T == 0) return MOE_OK;
-    if (!x_host || !y_host || !workspace) return MOE_ERR_INVALID_ARG;
+    if (!x_host || !y_host || !workspace || !holds_all_experts(w)) return MOE_ERR_INVALID_ARG;
     if ((uintptr_t)workspace % kAlign) return MOE_ERR_INVALID_ARG;
     if (!path_ok(w, T)) return MOE_ERR_UNSUPPORTED_SHAPE;
     const WsLayout L = ws_layout(w, T);
@@ -595,7 +721,7 @@ moe_status moe_w8a8_export_weights(const moe_w8a8_weights* w, int8_t* wq_gate, i
                                    float* inv_s, moe_stream_t stream) {
     if (!w) return MOE_ERR_INVALID_ARG;
     const moe_w8a8_config& c = w->cfg;
-    const int E = c.n_experts, d = c.d, f = c.f;
+    const int E = w->n_local, d = c.d, f = c.f;
     cudaStream_t s = (cudaStream_t)stream;
     if (wq_gate || wq_up) CUDA_TRY(launch_export_gateup(w->w_gu, E, d, f, wq_gate, wq_up, s));
     auto cp = [&](void* dst, const void* src, size_t bytes) {
@@ -617,7 +743,7 @@ moe_status moe_w8a8_check_status(const moe_w8a8_weights* w, moe_stream_t stream)
     if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
     if (word != 0) {
         if (cudaMemset(w->status, 0, 64) != cudaSuccess) return MOE_ERR_CUDA;
-        return MOE_ERR_TIMEOUT;
+        return word == MOE_ERR_INVALID_ARG ? MOE_ERR_INVALID_ARG : MOE_ERR_TIMEOUT;
     }
     return MOE_OK;
 }
@@ -672,6 +798,122 @@ moe_status moe_w8a8_profile_stop(moe_w8a8_weights* w) {
     return MOE_OK;
 }
 
+// ---------------------------------------------------------------- expert parallelism
+
+int32_t moe_w8a8_ep_row_bytes(const moe_w8a8_weights* w) { return w ? w->cfg.d + kEpTrailerBytes : 0; }
+
+moe_status moe_w8a8_gateup_absmax(const moe_w8a8_config* cfg, int32_t n_local, const float* w_gate,
+                                  const float* w_up, float* aw, moe_stream_t stream) {
+    moe_status st = check_config(cfg);
+    if (st != MOE_OK) return st;
+    if (!w_gate || !w_up || !aw || n_local <= 0 || n_local > cfg->n_experts) return MOE_ERR_INVALID_ARG;
+    cudaStream_t s = (cudaStream_t)stream;
+    CUDA_TRY(cudaMemsetAsync(aw, 0, (size_t)cfg->d * 4, s));
+    CUDA_TRY(launch_gateup_input_absmax(w_gate, w_up, n_local, cfg->d, cfg->f, aw, s));
+    return MOE_OK;
+}
+
+moe_status moe_w8a8_prepare_shard(const moe_w8a8_config* cfg, int32_t expert_first, int32_t n_local,
+                                  const float* w_gate, const float* w_up, const float* w_down,
+                                  const float* w_router, const float* act_absmax, const float* gateup_absmax,
+                                  moe_stream_t stream, moe_w8a8_weights** out) {
+    if (out) *out = nullptr;
+    if (!cfg || !out || !gateup_absmax) return MOE_ERR_INVALID_ARG;
+    return prepare_impl(cfg, expert_first, n_local, w_gate, w_up, w_down, w_router, act_absmax, gateup_absmax,
+                        stream, out);
+}
+
+size_t moe_w8a8_ep_dispatch_workspace_size(const moe_w8a8_weights* w, int32_t max_tokens) {
+    if (!w || max_tokens < 0) return 0;
+    return ws_layout(w, max_tokens, WS_ROUTE).total;
+}
+
+size_t moe_w8a8_ep_experts_workspace_size(const moe_w8a8_weights* w, int32_t rows) {
+    if (!w || rows < 0) return 0;
+    const moe_w8a8_weights v = expert_view(w);
+    return ws_layout(&v, rows, WS_EXPERTS).total;
+}
+
+moe_status moe_w8a8_ep_dispatch(const moe_w8a8_weights* w, const void* x, int32_t T, const float* router_bias,
+                                const float* router_logits, void* send, int32_t* expert_offsets, void* workspace,
+                                size_t workspace_bytes, const moe_w8a8_debug* dbg, moe_stream_t stream) {
+    if (!w || T < 0 || !expert_offsets) return MOE_ERR_INVALID_ARG;
+    const moe_w8a8_config& c = w->cfg;
+    cudaStream_t s = (cudaStream_t)stream;
+    if (T == 0) {
+        CUDA_TRY(cudaMemsetAsync(expert_offsets, 0, (size_t)(c.n_experts + 1) * 4, s));
+        return MOE_OK;
+    }
+    if (!x || !send || !workspace) return MOE_ERR_INVALID_ARG;
+    if ((uintptr_t)workspace % kAlign || (uintptr_t)send % 16) return MOE_ERR_INVALID_ARG;
+    const WsLayout L = ws_layout(w, T, WS_ROUTE);
+    if (workspace_bytes < L.total) return MOE_ERR_WORKSPACE_TOO_SMALL;
+    Run r(w, L, (char*)workspace, dbg, s);
+    r.prof = false;
+    MOE_TRY(route_stage(r, x, T, router_bias, router_logits, choose_path(w, T)));
+    MOE_TRY(quant_stage(r, x, T, (int8_t*)send, (int64_t)c.d + kEpTrailerBytes, true, c.expert_format));
+    CUDA_TRY(cudaMemcpyAsync(expert_offsets, r.at<int32_t>(L.offsets), (size_t)(c.n_experts + 1) * 4,
+                             cudaMemcpyDeviceToDevice, s));
+    MOE_TRY(debug_stage(r, T, c.top_k, c.n_experts, true, false));
+    const_cast<moe_w8a8_weights*>(w)->last_launches = r.launches;
+    return MOE_OK;
+}
+
+moe_status moe_w8a8_ep_experts(const moe_w8a8_weights* w, const void* recv, int32_t R, float* o_rows,
+                               void* workspace, size_t workspace_bytes, const moe_w8a8_debug* dbg,
+                               moe_stream_t stream) {
+    if (!w || R < 0) return MOE_ERR_INVALID_ARG;
+    if (R == 0) return MOE_OK;
+    if (!recv || !o_rows || !workspace) return MOE_ERR_INVALID_ARG;
+    if ((uintptr_t)workspace % kAlign || (uintptr_t)recv % 16 || (uintptr_t)o_rows % 16) return MOE_ERR_INVALID_ARG;
+    const moe_w8a8_weights v = expert_view(w);
+    if (!path_ok(&v, R)) return MOE_ERR_UNSUPPORTED_SHAPE;
+    const int path = choose_path(&v, R);
+    const WsLayout L = ws_layout(&v, R, WS_EXPERTS);
+    if (workspace_bytes < L.total) return MOE_ERR_WORKSPACE_TOO_SMALL;
+    cudaStream_t s = (cudaStream_t)stream;
+    Run r(&v, L, (char*)workspace, dbg, s);
+    r.prof = false;
+    const int d = v.cfg.d;
+    const int64_t rb = (int64_t)d + kEpTrailerBytes;
+    const uint8_t* rows = (const uint8_t*)recv;
+    int32_t* idx = r.at<int32_t>(L.topk_idx);
+    int32_t* ts2row = r.at<int32_t>(L.ts2row);
+    if (L.fused_words > 0) CUDA_TRY(cudaMemsetAsync(r.at<int32_t>(L.fused_sync), 0, (size_t)L.fused_words * 4, s));
+    // each received row is one (token, slot) pair with k = 1 of the local experts
+    CUDA_TRY(launch_ep_read_experts(rows, R, rb, d, w->ep_first, w->n_local, idx, w->status, s));
+    CUDA_TRY(launch_permute(idx, R, 1, v.cfg.n_experts, -1, r.at<int32_t>(L.hist), r.at<int32_t>(L.offsets),
+                            r.at<int32_t>(L.row2ts), ts2row, r.at<int32_t>(L.meta), r.at<int32_t>(L.active),
+                            r.at<int32_t>(L.tiles), s));
+    const bool stream_path = path == MOE_PATH_STREAM;
+    CUDA_TRY(launch_ep_gather(rows, R, rb, d, stream_path ? nullptr : ts2row,
+                              stream_path ? r.at<int8_t>(L.xq) : r.at<int8_t>(L.aq), r.at<float>(L.sx),
+                              r.at<float>(L.topk_w), s));
+    r.launches += 4;
+    MOE_TRY(expert_stage(r, R, path));
+    // un-sort: O of received row r to o_rows[r] (k = 1)
+    CUDA_TRY(launch_combine(r.at<float>(L.o), ts2row, R, 1, d, MOE_F32, o_rows, s));
+    ++r.launches;
+    MOE_TRY(debug_stage(r, R, 1, v.cfg.n_experts, false, true));
+    const_cast<moe_w8a8_weights*>(w)->last_launches = r.launches;
+    return MOE_OK;
+}
+
+moe_status moe_w8a8_ep_combine(const moe_w8a8_weights* w, const float* o_rows, int32_t T, void* y,
+                               const void* workspace, size_t workspace_bytes, moe_stream_t stream) {
+    if (!w || T < 0) return MOE_ERR_INVALID_ARG;
+    if (T == 0) return MOE_OK;
+    if (!y || !workspace) return MOE_ERR_INVALID_ARG;
+    if ((uintptr_t)workspace % kAlign || (uintptr_t)o_rows % 16) return MOE_ERR_INVALID_ARG;
+    const moe_w8a8_config& c = w->cfg;
+    const WsLayout L = ws_layout(w, T, WS_ROUTE);
+    if (workspace_bytes < L.total) return MOE_ERR_WORKSPACE_TOO_SMALL;
+    const int32_t* ts2row = (const int32_t*)((const char*)workspace + L.ts2row);
+    CUDA_TRY(launch_combine(o_rows, ts2row, T, c.top_k, c.d, c.out_dtype, y, (cudaStream_t)stream));
+    const_cast<moe_w8a8_weights*>(w)->last_launches = 1;
+    return MOE_OK;
+}
+
 const char* moe_w8a8_stage_name(int32_t stage) {
     static const char* names[MOE_N_STAGES] = {"router", "topk", "permute", "quant",
                                               "gemm1", "requant", "gemm2", "combine"};
@@ -718,7 +960,7 @@ extern "C" moe_status moe_w8a8_forward_noalloc(const moe_w8a8_weights* w, const 
                                                moe_stream_t stream) {
     if (!w || T < 0) return MOE_ERR_INVALID_ARG;
     if (T == 0) return MOE_OK;
-    if (!x || !y) return MOE_ERR_INVALID_ARG;
+    if (!x || !y || !holds_all_experts(w)) return MOE_ERR_INVALID_ARG;
     if (!path_ok(w, T)) return MOE_ERR_UNSUPPORTED_SHAPE;
     if (ws_layout(w, T).total > (size_t)MOE_NOALLOC_SCRATCH_BYTES) return MOE_ERR_WORKSPACE_TOO_SMALL;
     void* scratch = noalloc_scratch_for_current_device();

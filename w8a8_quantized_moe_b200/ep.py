@@ -1,0 +1,144 @@
+"""Expert-parallel W8A8 MoE layer: one rank per GPU over ``torch.distributed``.
+
+"Day0 adaptation of ultra-large model inference" (ruibaoantu.com), section 3:
+the experts are spread over the GPUs and each layer moves its tokens with one
+All-to-All each way; section 4: gate -> sort -> All-to-All -> grouped GEMM ->
+reverse All-to-All -> un-sort -> weighted sum.
+
+Rank g holds a contiguous range of the E experts.  Each rank routes and
+quantises its own tokens (``moe_w8a8_ep_dispatch``), sends every kept
+(token, slot) row to the rank that holds its expert, runs its experts on the
+rows it receives (``moe_w8a8_ep_experts``), returns each output row to its
+sender, and sums its tokens' slots in slot order (``moe_w8a8_ep_combine``).
+Every rank's output equals the single-GPU layer on that rank's tokens.
+
+The exchange is ``all_to_all_single`` of the process group (NCCL over
+NVLink/NVSwitch on GPUs, gloo on CPU for the tests).  Its split sizes follow
+the routing, so the host reads the E + 1 row offsets of each layer and then
+one count per peer.  All arithmetic of the layer runs in the library's
+kernels; this module moves buffers and picks split sizes.
+"""
+from __future__ import annotations
+
+import torch
+import torch.distributed as dist
+
+import w8a8_quantized_moe_b200 as M
+
+
+def equal_expert_ranges(n_experts: int, world: int) -> list[tuple[int, int]]:
+    """(first expert, count) per rank: world equal contiguous ranges."""
+    if world <= 0 or n_experts % world:
+        raise ValueError(f"{n_experts} experts do not split evenly over {world} ranks")
+    n = n_experts // world
+    return [(g * n, n) for g in range(world)]
+
+
+def prepare_expert_shard(cfg: M.moe_w8a8_config, expert_first: int, w_gate, w_up, w_down, w_router,
+                         act_absmax, group=None, stream=None) -> M.Weights:
+    """Prepare this rank's experts.  The smoothing statistic aw is the maximum
+    over ALL experts of the layer, so the per-rank maxima are all-reduced
+    before the scales are formed; every rank then holds the same s."""
+    aw = torch.empty(cfg.d, dtype=torch.float32, device=w_gate.device)
+    M.moe_w8a8_gateup_absmax(cfg, w_gate, w_up, aw, stream)
+    if dist.is_initialized() and dist.get_world_size(group) > 1:
+        dist.all_reduce(aw, op=dist.ReduceOp.MAX, group=group)
+    return M.moe_w8a8_prepare_shard(cfg, expert_first, w_gate, w_up, w_down, w_router, act_absmax, aw, stream)
+
+
+class LibraryStages:
+    """The three compute steps of one rank, on the library's kernels.  They run
+    on torch's current stream, the stream the collectives are ordered with."""
+
+    def __init__(self, w: M.Weights):
+        c = w.cfg
+        self.w = w
+        self.d, self.k, self.E = c.d, c.top_k, c.n_experts
+        self.row_bytes = M.moe_w8a8_ep_row_bytes(w)
+        self.device = torch.device("cuda", torch.cuda.current_device())
+        self.out_dtype = torch.bfloat16 if c.out_dtype == M.MOE_BF16 else torch.float32
+
+    def dispatch_workspace(self, T: int) -> int:
+        return M.moe_w8a8_ep_dispatch_workspace_size(self.w, T)
+
+    def experts_workspace(self, R: int) -> int:
+        return M.moe_w8a8_ep_experts_workspace_size(self.w, R)
+
+    def dispatch(self, x, T, router_bias, router_logits, send, offsets, ws):
+        M.moe_w8a8_ep_dispatch(self.w, x, T, router_bias, router_logits, send, offsets, ws)
+
+    def experts(self, recv, R, o_rows, ws):
+        M.moe_w8a8_ep_experts(self.w, recv, R, o_rows, ws)
+
+    def combine(self, o_rows, T, y, ws):
+        M.moe_w8a8_ep_combine(self.w, o_rows, T, y, ws)
+
+
+class ExpertParallelMoE:
+    """One rank of the expert-parallel layer.
+
+    stages  the compute steps (``LibraryStages`` on a GPU)
+    ranges  (first expert, count) of every rank, contiguous and ascending;
+            equal ranges by default
+    """
+
+    def __init__(self, stages, group=None, ranges=None):
+        self.stages = stages
+        self.group = group
+        self.rank = dist.get_rank(group)
+        self.world = dist.get_world_size(group)
+        self.ranges = equal_expert_ranges(stages.E, self.world) if ranges is None else list(ranges)
+        if len(self.ranges) != self.world:
+            raise ValueError("one expert range per rank")
+        nxt = 0
+        for first, n in self.ranges:
+            if first != nxt or n <= 0:
+                raise ValueError("expert ranges must be contiguous, ascending and cover every expert")
+            nxt = first + n
+        if nxt != stages.E:
+            raise ValueError("expert ranges must cover every expert")
+        self._bufs: dict[str, torch.Tensor] = {}
+        self.last_rows = (0, 0)   # rows sent, rows received by the last forward
+
+    def _buf(self, name: str, n: int, dtype) -> torch.Tensor:
+        """A cached flat buffer of at least n elements (grown on demand)."""
+        b = self._bufs.get(name)
+        if b is None or b.numel() < n or b.dtype != dtype:
+            b = torch.empty(max(n, 1), dtype=dtype, device=self.stages.device)
+            self._bufs[name] = b
+        return b[:n]
+
+    def forward(self, x, T: int, router_bias=None, router_logits=None, y=None):
+        st = self.stages
+        k, E, d, rb = st.k, st.E, st.d, st.row_bytes
+        send = self._buf("send", T * k * rb, torch.uint8)
+        offsets = self._buf("offsets", E + 1, torch.int32)
+        ws_route = self._buf("ws_route", st.dispatch_workspace(T), torch.uint8)
+        st.dispatch(x, T, router_bias, router_logits, send, offsets, ws_route)
+
+        # rows per destination: the rows of its experts, contiguous in `send`
+        offs = offsets.cpu().tolist()
+        send_rows = [offs[first + n] - offs[first] for first, n in self.ranges]
+        R_send = offs[E]
+        cnt_send = torch.tensor(send_rows, dtype=torch.int64, device=st.device)
+        cnt_recv = torch.empty_like(cnt_send)
+        dist.all_to_all_single(cnt_recv, cnt_send, group=self.group)
+        recv_rows = cnt_recv.cpu().tolist()
+        R_recv = sum(recv_rows)
+
+        recv = self._buf("recv", R_recv * rb, torch.uint8)
+        dist.all_to_all_single(recv, send[:R_send * rb], [r * rb for r in recv_rows],
+                               [s * rb for s in send_rows], group=self.group)
+        o_recv = self._buf("o_recv", R_recv * d, torch.float32)
+        ws_exp = self._buf("ws_experts", st.experts_workspace(R_recv), torch.uint8)
+        st.experts(recv, R_recv, o_recv.view(R_recv, d), ws_exp)
+
+        # every output row back to the rank and position it came from
+        o_back = self._buf("o_back", R_send * d, torch.float32)
+        dist.all_to_all_single(o_back, o_recv, [s * d for s in send_rows], [r * d for r in recv_rows],
+                               group=self.group)
+        if y is None:
+            y = torch.empty((T, d), dtype=st.out_dtype, device=st.device)
+        st.combine(o_back.view(R_send, d), T, y, ws_route)
+        self.last_rows = (R_send, R_recv)
+        return y
