@@ -11,6 +11,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
 #include <utility>
 
 namespace moe {
@@ -181,6 +182,21 @@ __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;"
 __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
 }  // namespace moe
+
+// Host: raise `kernel`'s dynamic shared-memory limit to `bytes` on the current
+// device, once per device (function attributes belong to each device's
+// context; `done` holds one bit per device that has it).
+template <typename... KArgs>
+inline cudaError_t smem_attr_once(void (*kernel)(KArgs...), size_t bytes, std::atomic<uint64_t>& done) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const uint64_t bit = dev >= 0 && dev < 64 ? (uint64_t)1 << dev : 0;
+    if (bit && (done.load(std::memory_order_acquire) & bit)) return cudaSuccess;
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    if (e == cudaSuccess) done.fetch_or(bit, std::memory_order_acq_rel);
+    return e;
+}
 
 // Host: launch `kernel` on `s` with programmatic stream serialization allowed,
 // so that it may start while the previous kernel on the stream finishes.

@@ -908,25 +908,18 @@ cudaError_t launch_router_logits(const void* x, int in_dtype, const float* wr, i
                                  float* logits, cudaStream_t s) {
     dim3 grid((T + kRtT - 1) / kRtT, (E + kRtE - 1) / kRtE);
     if (in_dtype == MOE_BF16 && E % kRtE == 0 && d % kRwKC == 0 && (reinterpret_cast<uintptr_t>(x) & 15) == 0) {
-        static bool wide_attr = false;
-        if (!wide_attr) {
-            cudaError_t e = cudaFuncSetAttribute(router_logits_wide_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                 (int)sizeof(RouterWideSmem));
-            if (e != cudaSuccess) return e;
-            wide_attr = true;
-        }
+        static std::atomic<uint64_t> wide_attr{0};
+        cudaError_t e = smem_attr_once(router_logits_wide_kernel, sizeof(RouterWideSmem), wide_attr);
+        if (e != cudaSuccess) return e;
         return launch_pdl(router_logits_wide_kernel, grid, dim3(kRwThreads), sizeof(RouterWideSmem), s,
                           reinterpret_cast<const uint16_t*>(x), wr, T, d, E, logits);
     }
     if (E % 4 == 0 && E >= 4) {
-        static bool attr = false;
-        if (!attr) {
-            cudaFuncSetAttribute(router_logits_async_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)sizeof(RouterAsyncSmem<2>));
-            cudaFuncSetAttribute(router_logits_async_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)sizeof(RouterAsyncSmem<4>));
-            attr = true;
-        }
+        static std::atomic<uint64_t> attr2{0}, attr4{0};
+        cudaError_t e = in_dtype == MOE_BF16
+                            ? smem_attr_once(router_logits_async_kernel<2>, sizeof(RouterAsyncSmem<2>), attr2)
+                            : smem_attr_once(router_logits_async_kernel<4>, sizeof(RouterAsyncSmem<4>), attr4);
+        if (e != cudaSuccess) return e;
         if (in_dtype == MOE_BF16)
             return launch_pdl(router_logits_async_kernel<2>, grid, dim3(kRtThreads), sizeof(RouterAsyncSmem<2>), s,
                               x, wr, T, d, E, logits);
@@ -948,13 +941,10 @@ cudaError_t launch_router_select(const moe_w8a8_weights* w, const void* x, int T
     const double c_err = std::ldexp(1.0, -16) + (d / 32 + 6) * std::ldexp(1.0, -24) +
                          (2.0 * (d / 16) + 2.0) * std::ldexp(1.0, -21);
     const size_t smem = (size_t)kSelWarps * d * 2 + (size_t)kSelWarps * kMaxE * 4;
-    static bool attr = false;
-    if (!attr) {
-        cudaError_t e = cudaFuncSetAttribute(router_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)((size_t)kSelWarps * 16384 * 2 + (size_t)kSelWarps * kMaxE * 4));
-        if (e != cudaSuccess) return e;
-        attr = true;
-    }
+    static std::atomic<uint64_t> attr{0};
+    cudaError_t e = smem_attr_once(router_select_kernel, (size_t)kSelWarps * 16384 * 2 + (size_t)kSelWarps * kMaxE * 4,
+                                   attr);
+    if (e != cudaSuccess) return e;
     return launch_pdl(router_select_kernel, dim3((T + kSelWarps - 1) / kSelWarps), dim3(kSelWarps * 32), smem, s,
                       reinterpret_cast<const uint16_t*>(x), approx, bias, w->rt_wt, w->rt_wmax, T, d,
                       w->cfg.n_experts, w->cfg.top_k, (float)c_err, sel, idx, wts, logits_out);
@@ -984,13 +974,9 @@ cudaError_t launch_route_small(const float* logits, const float* bias, int T, in
                                int32_t* offsets, int32_t* row2ts, int32_t* ts2row, int32_t* meta,
                                int32_t* active, int32_t* tiles, int32_t* zero_words, int n_zero,
                                cudaStream_t s) {
-    static bool attr = false;
-    if (!attr) {
-        cudaError_t e = cudaFuncSetAttribute(route_small_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)sizeof(RouteSmallSmem));
-        if (e != cudaSuccess) return e;
-        attr = true;
-    }
+    static std::atomic<uint64_t> attr{0};
+    cudaError_t e = smem_attr_once(route_small_kernel, sizeof(RouteSmallSmem), attr);
+    if (e != cudaSuccess) return e;
     return launch_pdl(route_small_kernel, dim3(1), dim3(kRouteSmallThreads), sizeof(RouteSmallSmem), s, logits,
                       bias, T, E, k, renorm, cap, idx, wts, logits_out, offsets, row2ts, ts2row, meta,
                       active, tiles, zero_words, n_zero);

@@ -265,12 +265,9 @@ cudaError_t launch_stream_gateup(const moe_w8a8_weights* w, int T, const int8_t*
                                  cudaStream_t s) {
     const int d = w->cfg.d, f = w->cfg.f;
     const size_t smem = (size_t)kStRows * d;
-    static bool attr = false;
-    if (!attr) {
-        cudaFuncSetAttribute(stream_gateup_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 100 * 1024);
-        cudaFuncSetAttribute(stream_down_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 100 * 1024);
-        attr = true;
-    }
+    static std::atomic<uint64_t> attr{0};
+    cudaError_t e = smem_attr_once(stream_gateup_kernel, 100 * 1024, attr);
+    if (e != cudaSuccess) return e;
     const int grid = stream_grid(w, w->cfg.n_experts * (2 * f / kGuUnit));
     (void)T;
     return launch_pdl(stream_gateup_kernel, dim3(grid), dim3(kStThreads), smem, s, w->w_gu, d, f,
@@ -282,11 +279,9 @@ cudaError_t launch_swiglu_requant(const moe_w8a8_weights* w, const int32_t* acc1
                                   const int32_t* meta, int max_rows, int8_t* hq, float* sh,
                                   cudaStream_t s) {
     const int f = w->cfg.f;
-    static bool attr = false;
-    if (!attr) {
-        cudaFuncSetAttribute(swiglu_requant_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 100 * 1024);
-        attr = true;
-    }
+    static std::atomic<uint64_t> attr{0};
+    cudaError_t e = smem_attr_once(swiglu_requant_kernel, 100 * 1024, attr);
+    if (e != cudaSuccess) return e;
     return launch_pdl(swiglu_requant_kernel, dim3(max_rows), dim3(kSwThreads), (size_t)f * 4, s, acc1, f,
                       w->cfg.top_k, row2ts, topk_idx, sx, w->sw_gate, w->sw_up, meta, hq, sh);
 }
@@ -299,6 +294,9 @@ cudaError_t launch_stream_down(const moe_w8a8_weights* w, int T, const int8_t* h
     const size_t smem = (size_t)kStRows * f;
     const int grid = stream_grid(w, w->cfg.n_experts * (d / kDnUnit));
     (void)T;
+    static std::atomic<uint64_t> attr{0};
+    cudaError_t e = smem_attr_once(stream_down_kernel, 100 * 1024, attr);
+    if (e != cudaSuccess) return e;
     return launch_pdl(stream_down_kernel, dim3(grid), dim3(kStThreads), smem, s, w->w_dn, d, f, hq, sh,
                       row2ts, topk_w, w->sw_dn, offsets, active, meta, o, acc2_dbg);
 }

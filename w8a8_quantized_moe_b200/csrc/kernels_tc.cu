@@ -1105,13 +1105,9 @@ template <int EPAD>
 cudaError_t launch_router_tc_pad(const CUtensorMap& mx, const moe_w8a8_weights* w, int T, float* approx,
                                  cudaStream_t s) {
     using C = RcCfg<EPAD>;
-    static bool attr = false;
-    if (!attr) {
-        cudaError_t e = cudaFuncSetAttribute(router_tc_kernel<EPAD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)C::kSmem);
-        if (e != cudaSuccess) return e;
-        attr = true;
-    }
+    static std::atomic<uint64_t> attr{0};
+    cudaError_t e = smem_attr_once(router_tc_kernel<EPAD>, C::kSmem, attr);
+    if (e != cudaSuccess) return e;
     return launch_pdl(router_tc_kernel<EPAD>, dim3((T + BM - 1) / BM), dim3(kRcThreads), C::kSmem, s, mx,
                       w->tm_rt_hi, w->tm_rt_lo, T, w->cfg.d, w->cfg.n_experts, approx, w->status);
 }
@@ -1119,13 +1115,9 @@ cudaError_t launch_router_tc_pad(const CUtensorMap& mx, const moe_w8a8_weights* 
 template <int EPI, int FMT>
 cudaError_t launch_fmt(const CUtensorMap& ta, const CUtensorMap& tb, const TcParams& p, int grid,
                        cudaStream_t s) {
-    static bool attr = false;
-    if (!attr) {
-        cudaError_t e = cudaFuncSetAttribute(tc_gemm_kernel<EPI, FMT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)kSmemBytes);
-        if (e != cudaSuccess) return e;
-        attr = true;
-    }
+    static std::atomic<uint64_t> attr{0};
+    cudaError_t e = smem_attr_once(tc_gemm_kernel<EPI, FMT>, kSmemBytes, attr);
+    if (e != cudaSuccess) return e;
     return launch_pdl(tc_gemm_kernel<EPI, FMT>, dim3(grid), dim3(kThreads), kSmemBytes, s, ta, tb, p);
 }
 
@@ -1147,13 +1139,9 @@ template <int FMT>
 cudaError_t launch_fused_fmt(const CUtensorMap& a1, const CUtensorMap& b1, const CUtensorMap& a2,
                              const CUtensorMap& b2, const TcParams& p1, const TcParams& p2, const FusedExtra& fx,
                              int grid, cudaStream_t s) {
-    static bool attr = false;
-    if (!attr) {
-        cudaError_t e = cudaFuncSetAttribute(tc_ffn_fused_kernel<FMT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)kFusedSmemBytes);
-        if (e != cudaSuccess) return e;
-        attr = true;
-    }
+    static std::atomic<uint64_t> attr{0};
+    cudaError_t e = smem_attr_once(tc_ffn_fused_kernel<FMT>, kFusedSmemBytes, attr);
+    if (e != cudaSuccess) return e;
     return launch_pdl(tc_ffn_fused_kernel<FMT>, dim3(grid), dim3(kFusedThreads), kFusedSmemBytes, s, a1, b1, a2,
                       b2, p1, p2, fx);
 }
