@@ -35,6 +35,10 @@
  *     smoothing statistics on the host) and moe_w8a8_check_status.
  *   - Arguments are validated before anything is enqueued; on an error the
  *     call returns a status and enqueues nothing.  No call throws or exits.
+ *   - Calls that run the layer on a handle (forward, forward_host,
+ *     forward_noalloc and the moe_w8a8_ep_* steps) need the handle's device
+ *     to be current (the one current at prepare); otherwise they return
+ *     MOE_ERR_INVALID_ARG.
  *   - Shapes: d and f multiples of 128, 1 <= top_k <= min(8, n_experts),
  *     n_experts <= 256, T >= 0 (T = 0 is a no-op).  Other shapes return
  *     MOE_ERR_UNSUPPORTED_SHAPE.

@@ -600,6 +600,12 @@ moe_status forward_impl(const moe_w8a8_weights* w, const void* x, int T, const f
 // The handle holds every expert of the layer (not an expert-parallel shard).
 bool holds_all_experts(const moe_w8a8_weights* w) { return w->ep_first == 0 && w->n_local == w->cfg.n_experts; }
 
+// The current device is the one the handle's weights live on.
+bool on_handle_device(const moe_w8a8_weights* w) {
+    int dev = -1;
+    return cudaGetDevice(&dev) == cudaSuccess && dev == w->device;
+}
+
 // The expert side of the expert-parallel layer: the held experts as a layer of
 // n_local experts with one slot per row, no capacity, no router and no
 // profiling (the kernels index scales and gate weights by row).
@@ -625,7 +631,7 @@ moe_status moe_w8a8_forward(const moe_w8a8_weights* w, const void* x, int32_t T,
                             moe_stream_t stream) {
     if (!w || T < 0) return MOE_ERR_INVALID_ARG;
     if (T == 0) return MOE_OK;
-    if (!x || !y || !workspace || !holds_all_experts(w)) return MOE_ERR_INVALID_ARG;
+    if (!x || !y || !workspace || !holds_all_experts(w) || !on_handle_device(w)) return MOE_ERR_INVALID_ARG;
     if ((uintptr_t)workspace % kAlign) return MOE_ERR_INVALID_ARG;
     if (!path_ok(w, T)) return MOE_ERR_UNSUPPORTED_SHAPE;
     if (workspace_bytes < ws_layout(w, T).total) return MOE_ERR_WORKSPACE_TOO_SMALL;
@@ -639,7 +645,7 @@ moe_status moe_w8a8_forward_host(const moe_w8a8_weights* w, const void* x_host, 
                                  moe_stream_t stream) {
     if (!w || T < 0) return MOE_ERR_INVALID_ARG;
     if (T == 0) return MOE_OK;
-    if (!x_host || !y_host || !workspace || !holds_all_experts(w)) return MOE_ERR_INVALID_ARG;
+    if (!x_host || !y_host || !workspace || !holds_all_experts(w) || !on_handle_device(w)) return MOE_ERR_INVALID_ARG;
     if ((uintptr_t)workspace % kAlign) return MOE_ERR_INVALID_ARG;
     if (!path_ok(w, T)) return MOE_ERR_UNSUPPORTED_SHAPE;
     const WsLayout L = ws_layout(w, T);
@@ -844,7 +850,7 @@ moe_status moe_w8a8_ep_dispatch(const moe_w8a8_weights* w, const void* x, int32_
         CUDA_TRY(cudaMemsetAsync(expert_offsets, 0, (size_t)(c.n_experts + 1) * 4, s));
         return MOE_OK;
     }
-    if (!x || !send || !workspace) return MOE_ERR_INVALID_ARG;
+    if (!x || !send || !workspace || !on_handle_device(w)) return MOE_ERR_INVALID_ARG;
     if ((uintptr_t)workspace % kAlign || (uintptr_t)send % 16) return MOE_ERR_INVALID_ARG;
     const WsLayout L = ws_layout(w, T, WS_ROUTE);
     if (workspace_bytes < L.total) return MOE_ERR_WORKSPACE_TOO_SMALL;
@@ -864,7 +870,7 @@ moe_status moe_w8a8_ep_experts(const moe_w8a8_weights* w, const void* recv, int3
                                moe_stream_t stream) {
     if (!w || R < 0) return MOE_ERR_INVALID_ARG;
     if (R == 0) return MOE_OK;
-    if (!recv || !o_rows || !workspace) return MOE_ERR_INVALID_ARG;
+    if (!recv || !o_rows || !workspace || !on_handle_device(w)) return MOE_ERR_INVALID_ARG;
     if ((uintptr_t)workspace % kAlign || (uintptr_t)recv % 16 || (uintptr_t)o_rows % 16) return MOE_ERR_INVALID_ARG;
     const moe_w8a8_weights v = expert_view(w);
     if (!path_ok(&v, R)) return MOE_ERR_UNSUPPORTED_SHAPE;
@@ -903,7 +909,7 @@ moe_status moe_w8a8_ep_combine(const moe_w8a8_weights* w, const float* o_rows, i
                                const void* workspace, size_t workspace_bytes, moe_stream_t stream) {
     if (!w || T < 0) return MOE_ERR_INVALID_ARG;
     if (T == 0) return MOE_OK;
-    if (!y || !workspace) return MOE_ERR_INVALID_ARG;
+    if (!y || !workspace || !on_handle_device(w)) return MOE_ERR_INVALID_ARG;
     if ((uintptr_t)workspace % kAlign || (uintptr_t)o_rows % 16) return MOE_ERR_INVALID_ARG;
     const moe_w8a8_config& c = w->cfg;
     const WsLayout L = ws_layout(w, T, WS_ROUTE);
@@ -960,7 +966,7 @@ extern "C" moe_status moe_w8a8_forward_noalloc(const moe_w8a8_weights* w, const 
                                                moe_stream_t stream) {
     if (!w || T < 0) return MOE_ERR_INVALID_ARG;
     if (T == 0) return MOE_OK;
-    if (!x || !y || !holds_all_experts(w)) return MOE_ERR_INVALID_ARG;
+    if (!x || !y || !holds_all_experts(w) || !on_handle_device(w)) return MOE_ERR_INVALID_ARG;
     if (!path_ok(w, T)) return MOE_ERR_UNSUPPORTED_SHAPE;
     if (ws_layout(w, T).total > (size_t)MOE_NOALLOC_SCRATCH_BYTES) return MOE_ERR_WORKSPACE_TOO_SMALL;
     void* scratch = noalloc_scratch_for_current_device();
