@@ -8,10 +8,13 @@ INT8 weights are made once, untimed (the offline preparation step).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload decode|prefill|tiny|large]
     python bench.py --impl reference ...   # the CPU oracle as the reference arm
+    python bench.py --ep [--gpus N] ...    # the expert-parallel layer
 
 Multi-GPU runs (torchrun, one process per GPU) are independent replicas of
 the layer on different token batches; value = all ranks' tokens / the
-slowest rank's device time.
+slowest rank's device time.  With --ep the ranks instead split the experts
+(E/N each), every rank routes its own batch, and rows cross between ranks
+with one All-to-All each way per layer (on one GPU: a one-rank NCCL group).
 """
 from __future__ import annotations
 
@@ -67,6 +70,8 @@ def parse():
     p.add_argument("--act-clip", type=float, default=0.0, metavar="PERCENT",
                    help="saturating activation clip at this percentile of the smoothed calibration "
                         "activations (0: off)")
+    p.add_argument("--ep", action="store_true",
+                   help="time the expert-parallel layer (experts split over the ranks) instead")
     p.add_argument("--no-prefill", action="store_true",
                    help="skip the extra prefill-layer measurement of the decode run")
     return p.parse_args()
@@ -593,12 +598,129 @@ def run_ours(args, world, rank, local):
     print(json.dumps(line), flush=True)
 
 
+def run_ep(args, world, rank, local):
+    """The expert-parallel layer: rank g holds experts [g E/N, (g+1) E/N) (only
+    those are generated and prepared), routes its own batch of T tokens, and
+    exchanges rows with the other ranks (one All-to-All each way).  Times K
+    layer steps with CUDA events on the current stream (the host's reads of
+    the row counts are inside the timed region); max over ranks.  On one rank
+    it also times the single-GPU forward on the same handle."""
+    import datetime
+    import socket
+
+    import torch
+    import torch.distributed as dist
+
+    import w8a8_quantized_moe_b200 as M
+    from w8a8_quantized_moe_b200 import build as B
+    from w8a8_quantized_moe_b200.ep import ExpertParallelMoE, LibraryStages, equal_expert_ranges, \
+        prepare_expert_shard
+
+    if not os.path.exists(M.LIB_PATH):
+        B.build()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    own_group = world == 1
+    if own_group:
+        with socket.socket() as sock:
+            sock.bind(("127.0.0.1", 0))
+            port = sock.getsockname()[1]
+        os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+        dist.init_process_group("nccl", rank=0, world_size=1, timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+    try:
+        wl = replica_workload(synth.WORKLOADS[args.workload], rank)
+        first, n = equal_expert_ranges(wl.E, world)[rank]
+        per = wl.d * wl.f
+        wg = torch.empty((n, wl.d, wl.f), dtype=torch.float32, device=dev)
+        wu = torch.empty((n, wl.d, wl.f), dtype=torch.float32, device=dev)
+        wd = torch.empty((n, wl.f, wl.d), dtype=torch.float32, device=dev)
+        for i in range(n):
+            e = first + i
+            for dst, tid, shape in ((wg, synth.TID_W_GATE, (wl.d, wl.f)), (wu, synth.TID_W_UP, (wl.d, wl.f)),
+                                    (wd, synth.TID_W_DOWN, (wl.f, wl.d))):
+                dst[i].copy_(torch.from_numpy(synth.normal(wl.weight_seed, tid, shape, std=wl.weight_std,
+                                                           start=e * per)))
+        calib_x, _ = synth.activations(wl.weight_seed + synth.CALIB_SEED_OFFSET, synth.CALIB_TOKENS, wl.d,
+                                       wl.outlier_channels(), wl.outlier_factor, wl.in_bf16)
+        if wl.in_bf16:
+            cal = torch.from_numpy(synth.f32_to_bf16_bits(calib_x).view(np.int16)).view(torch.bfloat16).to(dev)
+        else:
+            cal = torch.from_numpy(calib_x).to(dev)
+        ax = torch.zeros(wl.d, dtype=torch.float32, device=dev)
+        M.moe_w8a8_calibrate_absmax(cal, ax)
+        data = synth.make_data(wl)
+        wr = torch.from_numpy(data.w_router).to(dev)
+        cfg = M.make_config(wl.d, wl.f, wl.E, wl.k, wl.alpha, wl.capacity_factor, True,
+                            M.MOE_BF16 if wl.in_bf16 else M.MOE_F32, M.MOE_BF16 if wl.in_bf16 else M.MOE_F32,
+                            M.MOE_FMT_E4M3 if args.format == "e4m3" else M.MOE_FMT_INT8)
+        W = prepare_expert_shard(cfg, first, wg, wu, wd, wr, ax)
+        del wg, wu, wd, cal
+        torch.cuda.empty_cache()
+        layer = ExpertParallelMoE(LibraryStages(W))
+        T = wl.T
+        x = torch.from_numpy(data.x_bits.view(np.int16)).view(torch.bfloat16).to(dev) if wl.in_bf16 \
+            else torch.from_numpy(data.x).to(dev)
+        logits = torch.from_numpy(data.router_logits).to(dev) if data.router_logits is not None else None
+        bias = torch.from_numpy(data.router_bias).to(dev) if data.router_bias is not None else None
+        y = torch.empty((T, wl.d), dtype=torch.bfloat16 if wl.in_bf16 else torch.float32, device=dev)
+        stream = torch.cuda.current_stream(dev)
+
+        def timed(step):
+            for _ in range(args.warmup):
+                step()
+            torch.cuda.synchronize(dev)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            barrier(world)
+            torch.cuda.synchronize(dev)
+            e0.record(stream)
+            for _ in range(args.steps):
+                step()
+            e1.record(stream)
+            torch.cuda.synchronize(dev)
+            barrier(world)
+            return e0.elapsed_time(e1) / args.steps
+
+        clocks = ClockSampler(local)
+        clocks.start()
+        ms_ep = max_over_ranks(timed(lambda: layer.forward(x, T, bias, logits, y)), world)
+        clocks.stop()
+        M.moe_w8a8_check_status(W)
+        sent, received = layer.last_rows
+        ms_fwd = None
+        if world == 1:
+            ws = torch.empty(M.moe_w8a8_workspace_size(W, T), dtype=torch.uint8, device=dev)
+            yf = torch.empty_like(y)
+            ms_fwd = timed(lambda: M.moe_w8a8_forward(W, x, T, bias, logits, yf, ws))
+            torch.cuda.synchronize(dev)
+            assert torch.equal(y, yf), "expert-parallel output differs from the forward"
+        if rank == 0:
+            line = {"metric": "expert-parallel W8A8 MoE layer tokens/s", "value": world * T / ms_ep * 1e3,
+                    "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+                    "ms_per_step": ms_ep, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                    "dtype": "e4m3" if args.format == "e4m3" else "int8", "data": "synthetic",
+                    "config": {"workload": describe(wl) + f"; expert-parallel over {world} rank(s), "
+                                                          f"{n} experts per rank, {T} tokens per rank",
+                               "parallelism": f"ep{world}", "experts_per_rank": n,
+                               "rank0_rows_sent": sent, "rank0_rows_received": received,
+                               "exchange": "torch.distributed all_to_all_single (NCCL), host reads the "
+                                           "row counts each step",
+                               "l2": "weights larger than L2; no flush"},
+                    "single_gpu_forward_ms": ms_fwd, "clocks": clocks.summary()}
+            print(json.dumps(line), flush=True)
+    finally:
+        if own_group:
+            dist.destroy_process_group()
+
+
 def main():
     args = parse()
     world, rank, local = dist_setup(args)
     try:
         if args.impl == "reference":
             run_reference(args, world, rank)
+        elif args.ep:
+            run_ep(args, world, rank, local)
         else:
             run_ours(args, world, rank, local)
     finally:
