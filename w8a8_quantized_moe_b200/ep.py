@@ -35,15 +35,16 @@ def equal_expert_ranges(n_experts: int, world: int) -> list[tuple[int, int]]:
 
 
 def prepare_expert_shard(cfg: M.moe_w8a8_config, expert_first: int, w_gate, w_up, w_down, w_router,
-                         act_absmax, group=None, stream=None) -> M.Weights:
+                         act_absmax, group=None) -> M.Weights:
     """Prepare this rank's experts.  The smoothing statistic aw is the maximum
     over ALL experts of the layer, so the per-rank maxima are all-reduced
-    before the scales are formed; every rank then holds the same s."""
+    before the scales are formed; every rank then holds the same s.  Runs on
+    torch's current stream, the stream the all-reduce is ordered with."""
     aw = torch.empty(cfg.d, dtype=torch.float32, device=w_gate.device)
-    M.moe_w8a8_gateup_absmax(cfg, w_gate, w_up, aw, stream)
+    M.moe_w8a8_gateup_absmax(cfg, w_gate, w_up, aw)
     if dist.is_initialized() and dist.get_world_size(group) > 1:
         dist.all_reduce(aw, op=dist.ReduceOp.MAX, group=group)
-    return M.moe_w8a8_prepare_shard(cfg, expert_first, w_gate, w_up, w_down, w_router, act_absmax, aw, stream)
+    return M.moe_w8a8_prepare_shard(cfg, expert_first, w_gate, w_up, w_down, w_router, act_absmax, aw)
 
 
 class LibraryStages:
