@@ -54,3 +54,24 @@ def test_two_gloo_ranks(tmp_path):
     assert r[0]["wseed"] == r[1]["wseed"]                     # same layer weights
     assert r[0]["seed"] != r[1]["seed"]                       # a different batch per replica
     assert r[1]["ref"] is None                                # only rank 0 runs the reference arm
+
+
+def test_threaded_oracle_step_equals_the_serial_oracle():
+    """The all-cores CPU baseline runs the unchanged oracle on token subsets in
+    threads; its output must be the serial oracle's, bit for bit."""
+    sys.path.insert(0, ROOT)
+    import numpy as np
+
+    import bench
+    import oracle
+    import synth
+    wl = synth.WORKLOADS["tiny"]
+    wts = synth.make_weights(wl)
+    prep = oracle.prepare(wts.w_gate, wts.w_up, wts.w_down, wts.calib_x, wl.alpha)
+    data = synth.make_data(wl)
+    rt = oracle.route(data.x, wl.k, wl.E, w_router=data.w_router, logits=data.router_logits,
+                      bias=data.router_bias, capacity_factor=wl.capacity_factor)
+    y_ref, _ = oracle.moe_tokens(data.x, prep, rt, out_bf16=wl.in_bf16, debug=False)
+    for threads in (1, 3, 8):
+        _, y = bench.oracle_step_threads(wl, prep, data, threads)
+        assert np.array_equal(y, y_ref), threads
