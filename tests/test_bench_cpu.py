@@ -1,0 +1,46 @@
+"""The bench's algorithmic byte / op model (the numerators of the roofline
+fractions), checked against figures worked out by hand from the layer's shapes:
+an active expert carries 3 d f INT8 weight bytes and (2f + d) fp32 scales, a
+token d input and d output elements, and a kept row 2 * 3 d f INT8 ops."""
+import os
+import sys
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _bench():
+    sys.path.insert(0, ROOT)
+    import bench
+    import synth
+    return bench, synth
+
+
+def test_decode_layer_bytes_and_ops():
+    bench, synth = _bench()
+    wl = synth.WORKLOADS["decode"]          # T=32, d=4096, E=64, k=4, f=1536, bf16, given logits
+    a = bench.algorithmic(wl, n_active=56, R=128, tensor=True)
+    # 56 * 3 * 4096 * 1536 weight bytes          = 1,056,964,608
+    # 56 * (2 * 1536 + 4096) * 4 scale bytes     =     1,605,632
+    # 32 tokens * 4096 * 2 bytes, in and out     =       524,288
+    # given router logits 32 * 64 * 4            =         8,192
+    assert a["layer_bytes"] == 1_059_102_720
+    assert a["int8_ops"] == 4_831_838_208     # 2 * 128 * 3 * 4096 * 1536
+    # the fused launch reads both GEMMs' weights once: at least the weight bytes
+    assert a["fused_bytes"] >= 1_056_964_608
+
+
+def test_prefill_ops():
+    bench, synth = _bench()
+    wl = synth.WORKLOADS["prefill"]         # T=16384, top-4: 65,536 rows
+    a = bench.algorithmic(wl, n_active=64, R=65536, tensor=True)
+    assert a["int8_ops"] == 2_473_901_162_496
+    # GEMM1 is two thirds of the ops: 2 * 65536 * 3072 * 4096
+    assert 2 * 65536 * 2 * 1536 * 4096 == 1_649_267_441_664
+
+
+def test_layer_bytes_count_only_active_experts():
+    bench, synth = _bench()
+    wl = synth.WORKLOADS["decode"]
+    a40 = bench.algorithmic(wl, n_active=40, R=128)
+    a41 = bench.algorithmic(wl, n_active=41, R=128)
+    assert a41["layer_bytes"] - a40["layer_bytes"] == 3 * 4096 * 1536 + (2 * 1536 + 4096) * 4
