@@ -117,10 +117,19 @@ def _rank_main(rank, world, port, out_dir, case):
         T = case.get("T", [wl.T] * world)[rank]
         wts = synth.make_weights(wl)
         prep = oracle.prepare(wts.w_gate, wts.w_up, wts.w_down, wts.calib_x, wl.alpha)
-        first, n = equal_expert_ranges(wl.E, world)[rank]
+        ranges = case.get("ranges") or equal_expert_ranges(wl.E, world)
+        first, n = ranges[rank]
         stages = OracleStages(wl, prep, first, n)
-        layer = ExpertParallelMoE(stages)
-        out = {"rows": None, "equal": True, "T": T}
+        layer = ExpertParallelMoE(stages, ranges=ranges)
+        bad = []
+        for r in ([(0, wl.E)], [(1, wl.E - 1)] + [(0, 1)] * (world - 1),
+                  [(0, 2), (3, wl.E - 3)] + [(wl.E, 0)] * (world - 2)):
+            try:
+                ExpertParallelMoE(stages, ranges=r)
+                bad.append(r)
+            except ValueError:
+                pass
+        out = {"rows": None, "equal": True, "T": T, "accepted_bad_ranges": len(bad)}
         for step in range(2):   # two layers' worth of traffic through the same buffers
             wl_r = dataclasses.replace(wl, T=max(T, 1), data_seed=wl.data_seed + 37 * rank + 1000 * step)
             data = synth.make_data(wl_r)
@@ -172,6 +181,14 @@ def test_ep_rank_without_tokens(tmp_path):
     r = _run(tmp_path, 2, {"T": [64, 0]})
     assert r[0]["equal"] and r[1]["T"] == 0
     assert r[1]["rows"][0] == 0 and r[1]["rows"][1] > 0
+
+
+def test_ep_uneven_expert_ranges(tmp_path):
+    # 3 experts on rank 0, 5 on rank 1; malformed range lists are refused
+    r = _run(tmp_path, 2, {"ranges": [(0, 3), (3, 5)]})
+    assert all(x["equal"] for x in r)
+    assert r[0]["range"] == [0, 3] and r[1]["range"] == [3, 5]
+    assert all(x["accepted_bad_ranges"] == 0 for x in r)
 
 
 def test_expert_ranges_host_checks():
