@@ -183,6 +183,14 @@ def test_ep_rank_without_tokens(tmp_path):
     assert r[1]["rows"][0] == 0 and r[1]["rows"][1] > 0
 
 
+def test_ep_eight_ranks_one_expert_each(tmp_path):
+    # one expert per rank and a skewed router: many peer pairs exchange no rows
+    r = _run(tmp_path, 8, {"wl": {"zipf_s": 2.0}, "T": [16] * 8})
+    assert all(x["equal"] for x in r)
+    assert sum(x["rows"][0] for x in r) == sum(x["rows"][1] for x in r) == 8 * 16 * 2
+    assert min(x["rows"][1] for x in r) < 16 < max(x["rows"][1] for x in r)
+
+
 def test_ep_uneven_expert_ranges(tmp_path):
     # 3 experts on rank 0, 5 on rank 1; malformed range lists are refused
     r = _run(tmp_path, 2, {"ranges": [(0, 3), (3, 5)]})
