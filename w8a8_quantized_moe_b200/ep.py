@@ -14,9 +14,10 @@ Every rank's output equals the single-GPU layer on that rank's tokens.
 
 The exchange is ``all_to_all_single`` of the process group (NCCL over
 NVLink/NVSwitch on GPUs, gloo on CPU for the tests).  Its split sizes follow
-the routing, so the host reads the E + 1 row offsets of each layer and then
-one count per peer.  All arithmetic of the layer runs in the library's
-kernels; this module moves buffers and picks split sizes.
+the routing: the per-peer row counts are formed on the device from the row
+offsets, exchanged, and read by the host together, once per layer.  All
+arithmetic of the layer runs in the library's kernels; this module moves
+buffers and picks split sizes.
 """
 from __future__ import annotations
 
@@ -100,6 +101,9 @@ class ExpertParallelMoE:
             raise ValueError("expert ranges must cover every expert")
         self._bufs: dict[str, torch.Tensor] = {}
         self.last_rows = (0, 0)   # rows sent, rows received by the last forward
+        # row-offset indices of each destination's first expert and one past its last
+        self._lo = torch.tensor([first for first, _ in self.ranges], dtype=torch.long, device=stages.device)
+        self._hi = torch.tensor([first + n for first, n in self.ranges], dtype=torch.long, device=stages.device)
 
     def _buf(self, name: str, n: int, dtype) -> torch.Tensor:
         """A cached flat buffer of at least n elements (grown on demand)."""
@@ -117,15 +121,14 @@ class ExpertParallelMoE:
         ws_route = self._buf("ws_route", st.dispatch_workspace(T), torch.uint8)
         st.dispatch(x, T, router_bias, router_logits, send, offsets, ws_route)
 
-        # rows per destination: the rows of its experts, contiguous in `send`
-        offs = offsets.cpu().tolist()
-        send_rows = [offs[first + n] - offs[first] for first, n in self.ranges]
-        R_send = offs[E]
-        cnt_send = torch.tensor(send_rows, dtype=torch.int64, device=st.device)
+        # rows per destination (the rows of its experts, contiguous in `send`),
+        # exchanged on the device; the host reads sent and received counts at once
+        cnt_send = (offsets[self._hi] - offsets[self._lo]).to(torch.int64)
         cnt_recv = torch.empty_like(cnt_send)
         dist.all_to_all_single(cnt_recv, cnt_send, group=self.group)
-        recv_rows = cnt_recv.cpu().tolist()
-        R_recv = sum(recv_rows)
+        counts = torch.cat([cnt_send, cnt_recv]).cpu().tolist()
+        send_rows, recv_rows = counts[:self.world], counts[self.world:]
+        R_send, R_recv = sum(send_rows), sum(recv_rows)
 
         recv = self._buf("recv", R_recv * rb, torch.uint8)
         dist.all_to_all_single(recv, send[:R_send * rb], [r * rb for r in recv_rows],
