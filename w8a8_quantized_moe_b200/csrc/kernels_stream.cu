@@ -17,7 +17,8 @@ namespace {
 constexpr int kStThreads = 256;
 constexpr int kStWarps = kStThreads / 32;
 constexpr int kStRows = 8;       // rows of one expert processed per pass over its weights
-constexpr int kStSegMax = 16;    // 512-byte K segments held in flight per channel (K <= 8192)
+constexpr int kStSegMax = 16;    // 512-byte K segments held in flight per channel per pass
+constexpr int kStMaxK = 16384;   // largest d and f a layer may have: the staged rows take kStRows x K bytes
 
 // acc[r][c] = sum_k A[r][k] * W[ch_c][k] for the nr rows staged in smem (row
 // stride K) and CH consecutive weight rows starting at wrow (stride K).
@@ -266,7 +267,7 @@ cudaError_t launch_stream_gateup(const moe_w8a8_weights* w, int T, const int8_t*
     const int d = w->cfg.d, f = w->cfg.f;
     const size_t smem = (size_t)kStRows * d;
     static std::atomic<uint64_t> attr{0};
-    cudaError_t e = smem_attr_once(stream_gateup_kernel, 100 * 1024, attr);
+    cudaError_t e = smem_attr_once(stream_gateup_kernel, (size_t)kStRows * kStMaxK, attr);
     if (e != cudaSuccess) return e;
     const int grid = stream_grid(w, w->cfg.n_experts * (2 * f / kGuUnit));
     (void)T;
@@ -295,7 +296,7 @@ cudaError_t launch_stream_down(const moe_w8a8_weights* w, int T, const int8_t* h
     const int grid = stream_grid(w, w->cfg.n_experts * (d / kDnUnit));
     (void)T;
     static std::atomic<uint64_t> attr{0};
-    cudaError_t e = smem_attr_once(stream_down_kernel, 100 * 1024, attr);
+    cudaError_t e = smem_attr_once(stream_down_kernel, (size_t)kStRows * kStMaxK, attr);
     if (e != cudaSuccess) return e;
     return launch_pdl(stream_down_kernel, dim3(grid), dim3(kStThreads), smem, s, w->w_dn, d, f, hq, sh,
                       row2ts, topk_w, w->sw_dn, offsets, active, meta, o, acc2_dbg);
