@@ -29,6 +29,24 @@ def test_header_declares_the_binding_exports(M):
     assert declared_functions() == sorted(M.EXPORTS)
 
 
+def declared_arg_counts():
+    """Parameter count of every function the header declares."""
+    text = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    out = {}
+    for m in re.finditer(r"\b(moe_\w+)\s*\(([^;{]*?)\)\s*;", text, flags=re.S):
+        params = m.group(2).strip()
+        out[m.group(1)] = 0 if params in ("", "void") else params.count(",") + 1
+    return out
+
+
+def test_binding_signatures_match_the_header(M):
+    lib = M.lib()
+    counts = declared_arg_counts()
+    assert sorted(counts) == declared_functions()
+    for name, n in counts.items():
+        assert len(getattr(lib, name).argtypes) == n, name
+
+
 def test_every_declared_symbol_is_exported(M):
     lib = M.lib()
     for name in declared_functions():
