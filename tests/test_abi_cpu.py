@@ -45,6 +45,13 @@ def test_binding_signatures_match_the_header(M):
     assert sorted(counts) == declared_functions()
     for name, n in counts.items():
         assert len(getattr(lib, name).argtypes) == n, name
+    text = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    kinds = {"size_t": ctypes.c_size_t, "int32_t": ctypes.c_int32, "moe_status": ctypes.c_int32,
+             "const char*": ctypes.c_char_p, "void": None}
+    for m in re.finditer(r"^\s*([A-Za-z_][\w\s\*]*?)\s*\b(moe_\w+)\s*\(", text, flags=re.M):
+        ret = " ".join(m.group(1).replace("*", " * ").split()).replace(" *", "*")
+        assert ret in kinds, (m.group(2), ret)
+        assert getattr(lib, m.group(2)).restype is kinds[ret], m.group(2)
 
 
 def test_every_declared_symbol_is_exported(M):
