@@ -85,7 +85,8 @@ void oracle_expf_array(const float* x, int64_t n, float* y) {
 /* Symmetric INT8 quantisation of one vector (per output channel for        */
 /* weights, per token for activations): [MiniMax-M3 W8A8 on K100AI] s1.2,   */
 /* s3.2.  scale = amax / 127 (fp32 division); q = rint(v / scale) with      */
-/* ties to even, clamped to [-127, 127]; amax == 0 gives scale 0, q = 0.    */
+/* ties to even, clamped to [-127, 127].  A scale that is 0 in fp32 (amax   */
+/* == 0, or amax so small that amax / 127 underflows) gives q = 0.          */
 /* ------------------------------------------------------------------------ */
 
 static inline int8_t quant_one(float v, float scale) {
@@ -103,11 +104,11 @@ static float quant_vector_clip(const float* v, int64_t n, int64_t stride, int8_t
     float amax = 0.0f;
     for (int64_t i = 0; i < n; ++i) amax = fmaxf(amax, fabsf(v[i * stride]));
     if (clip > 0.0f && amax > clip) amax = clip;
-    if (amax == 0.0f) {
+    const float scale = amax / 127.0f;
+    if (scale == 0.0f) {
         memset(q, 0, (size_t)n);
         return 0.0f;
     }
-    float scale = amax / 127.0f;
     for (int64_t i = 0; i < n; ++i) q[i] = quant_one(v[i * stride], scale);
     return scale;
 }
@@ -551,17 +552,17 @@ void oracle_e4m3_decode_array(const uint8_t* q, int64_t n, float* v) {
 }
 
 /* Scaled E4M3 quantisation of one vector (the FP8 counterpart of the INT8   */
-/* rule): scale = amax / 448 (fp32 division), q = e4m3(v / scale); amax == 0 */
-/* gives scale 0 and codes 0; clip > 0 caps amax as in the INT8 rule.        */
+/* rule): scale = amax / 448 (fp32 division), q = e4m3(v / scale); a scale  */
+/* that is 0 in fp32 gives codes 0; clip > 0 caps amax as in the INT8 rule.  */
 static float quant_vector_fp8(const float* v, int64_t n, int64_t stride, uint8_t* q, float clip) {
     float amax = 0.0f;
     for (int64_t i = 0; i < n; ++i) amax = fmaxf(amax, fabsf(v[i * stride]));
     if (clip > 0.0f && amax > clip) amax = clip;
-    if (amax == 0.0f) {
+    const float scale = amax / 448.0f;
+    if (scale == 0.0f) {   /* amax == 0, or amax / 448 underflows: codes 0 */
         memset(q, 0, (size_t)n);
         return 0.0f;
     }
-    const float scale = amax / 448.0f;
     for (int64_t i = 0; i < n; ++i) q[i] = oracle_e4m3_encode(v[i * stride] / scale);
     return scale;
 }

@@ -73,6 +73,29 @@ def test_quant_error_bound_and_full_range():
     assert q[9, 5] == -127 and np.count_nonzero(q[9]) == 1
 
 
+def test_quant_tiny_rows_scale_underflow_and_subnormal_scales():
+    # amax / 127 underflows to 0 in fp32: scale 0 and codes 0 (like an all-zero row)
+    tiny = np.array([1e-44, -3e-45, 0.0, 7e-45], np.float32)
+    assert np.float32(np.abs(tiny).max()) / np.float32(127.0) == 0.0
+    q, s = oracle.quantize_rows(tiny[None, :])
+    assert s[0] == 0.0 and not q.any()
+    qf, sf = oracle.quantize_rows_fp8(tiny[None, :])
+    assert sf[0] == 0.0 and not qf.any()
+    # a subnormal but non-zero scale still rounds to nearest: |v - q s| <= s/2
+    for amax in (1e-37, 3e-39, 1e-40, 2e-42):
+        v = (synth.normal(40, 1, (1, 300), std=1.0) * np.float32(amax / 4)).astype(np.float32)
+        v[0, 0] = np.float32(amax)
+        q, s = oracle.quantize_rows(v)
+        sc = float(s[0])
+        assert 0.0 < sc < 1.2e-38
+        vv = v[0].astype(np.float64)
+        inside = np.abs(vv / sc) <= 127.0
+        err = np.abs(vv - q[0].astype(np.float64) * sc)
+        assert np.all(err[inside] <= sc * (0.5 + 2.0 ** -20)), amax
+        assert np.all(np.abs(q[0][~inside]) == 127)
+        assert np.all(np.sign(q[0]) == np.sign(np.where(np.abs(vv) >= sc / 2, vv, 0.0)))
+
+
 # ----------------------------------------------------------------------------- activation clip
 
 def test_clip_at_or_above_the_range_changes_nothing():

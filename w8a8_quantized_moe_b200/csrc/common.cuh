@@ -74,8 +74,11 @@ __device__ __forceinline__ int quant_code(float v, float s) {
 // standard rounding-error bound, i.e. below 2.3e-5 for |v / s| <= 128.  So
 // unless t lies within 3e-5 of a half-integer, t and the IEEE quotient round
 // to the same integer; near a half-integer the IEEE quotient is formed.  The
-// result is identical to quant_code(v, s).  `r` must be fp32(1 / s), s > 0.
+// result is identical to quant_code(v, s).  `r` must be fp32(1 / s), s > 0;
+// when 1/s overflows (s below 2^-128, a row whose largest value is under
+// about 3.7e-37) the bound does not hold and the quotient is formed.
 __device__ __forceinline__ int quant_code_fast(float v, float s, float r) {
+    if (isinf(r)) return quant_code(v, s);
     const float t = __fmul_rn(v, r);
     const float n = rintf(t);
     const float dist = fabsf(fabsf(__fsub_rn(t, n)) - 0.5f);
