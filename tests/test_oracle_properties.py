@@ -75,12 +75,41 @@ def test_quantised_rows_round_to_nearest(data):
     vals = data.draw(st.lists(st.floats(-1.0, 1.0, width=32), min_size=n, max_size=n))
     v = (np.array(vals, np.float32) * np.float32(mag)).astype(np.float32)
     q, s = oracle.quantize_rows(v[None, :])
-    amax = float(np.abs(v).max())
-    if amax == 0.0:
+    amax = np.float32(np.abs(v).max())
+    if amax / np.float32(127.0) == 0.0:          # zero row, or a scale that underflows
         assert s[0] == 0.0 and not q.any()
         return
     sc = float(s[0])
-    err = np.abs(v.astype(np.float64) - q[0].astype(np.float64) * sc)
-    assert np.all(err <= sc * (0.5 + 1e-5))
-    assert np.abs(q[0]).max() == 127
+    vv = v.astype(np.float64)
+    inside = np.abs(vv / sc) <= 127.0        # a subnormal scale can sit well below amax / 127
+    err = np.abs(vv - q[0].astype(np.float64) * sc)
+    assert np.all(err[inside] <= sc * (0.5 + 1e-5))
+    assert np.all(q[0][~inside] == np.where(vv[~inside] > 0, 127, -127))
+    if sc >= 2.0 ** -126:                    # a normal scale: the largest value gets the full range
+        assert np.abs(q[0]).max() == 127
     assert np.all((q[0] == 0) | (np.sign(q[0]) == np.sign(v)))
+
+
+@SETTINGS
+@given(st.data())
+def test_fp8_quantised_rows_round_to_nearest(data):
+    n = data.draw(st.integers(1, 48), label="n")
+    mag = data.draw(st.sampled_from([1e-30, 1e-3, 1.0, 1e3, 1e30]), label="magnitude")
+    vals = data.draw(st.lists(st.floats(-1.0, 1.0, width=32), min_size=n, max_size=n))
+    v = (np.array(vals, np.float32) * np.float32(mag)).astype(np.float32)
+    q, s = oracle.quantize_rows_fp8(v[None, :])
+    if np.float32(np.abs(v).max()) / np.float32(448.0) == 0.0:   # zero row, or a scale that underflows
+        assert s[0] == 0.0 and not q.any()
+        return
+    sc = float(s[0])
+    if sc >= 2.0 ** -126:                               # a normal scale: the largest value maps to +-448
+        assert (q[0] & 0x7f).max() == 0x7e
+    t = v.astype(np.float64) / sc
+    dq = oracle.e4m3_decode(q[0]).astype(np.float64)
+    inside = np.abs(t) <= 448.0
+    # half an E4M3 step of the value's binade (2^-3 of the binade for normals, 2^-9 below 2^-6)
+    step = np.where(np.abs(t) >= 2.0 ** -6, 2.0 ** (np.floor(np.log2(np.maximum(np.abs(t), 1e-30))) - 3),
+                    2.0 ** -9)
+    assert np.all((np.abs(t - dq) <= step / 2 * (1 + 1e-6) + 1e-7 * np.abs(t))[inside])
+    assert np.all(np.abs(dq[~inside]) == 448.0)
+    assert np.all((dq == 0) | (np.sign(dq) == np.sign(v)))
