@@ -92,7 +92,7 @@ typedef struct {
     int32_t n_experts;        /* E                                                            */
     int32_t top_k;            /* k                                                            */
     float alpha;              /* SmoothQuant migration strength, in [0, 1] (pages use 0.6)     */
-    float capacity_factor;    /* <= 0: no capacity; else C = ceil(cf * T * k / E) per expert  */
+    float capacity_factor;    /* finite; <= 0: no capacity; else C = min(ceil(cf T k / E), T k) */
     int32_t renormalize;      /* 1: softmax over the k selected logits; 0: over all E          */
     int32_t in_dtype;         /* MOE_F32 or MOE_BF16: X                                       */
     int32_t out_dtype;        /* MOE_F32 or MOE_BF16: Y                                       */
@@ -155,11 +155,18 @@ size_t moe_w8a8_workspace_size(const moe_w8a8_weights* w, int32_t max_tokens);
 
 /*
  * Run the layer on T tokens.
- *   x              device [T][d], cfg.in_dtype
- *   router_bias    device fp32 [E] added to every token's logits, or NULL
- *   router_logits  device fp32 [T][E] used instead of X W_router, or NULL
- *   y              device [T][d], cfg.out_dtype
+ *   x              device [T][d], cfg.in_dtype, 16-byte aligned
+ *   router_bias    device fp32 [E] added to every token's logits, or NULL;
+ *                  16-byte aligned
+ *   router_logits  device fp32 [T][E] used instead of X W_router, or NULL;
+ *                  16-byte aligned
+ *   y              device [T][d], cfg.out_dtype, 16-byte aligned
  *   workspace      device, >= moe_w8a8_workspace_size(w, T) bytes, 256-byte aligned
+ * The kernels read and write x, y, router_bias and router_logits with
+ * 16-byte vector accesses: a NULL or misaligned pointer (NULL is allowed for
+ * the two optional ones) returns MOE_ERR_INVALID_ARG before the handle is
+ * read and before anything is enqueued.  The buffers must hold the sizes
+ * above; the library cannot check that (the Python binding does).
  *   dbg            NULL, or device pointers receiving intermediates
  * Allocates nothing; all scratch lives in the caller's workspace.  Calls
  * that share a workspace must not overlap on the device.
@@ -443,9 +450,12 @@ moe_status moe_w8a8_ep_experts(const moe_w8a8_weights* w, const void* recv, int3
                                moe_stream_t stream);
 
 /*
- * Step 5: y [T][d] (cfg.out_dtype) from the returned rows o_rows (device fp32
- * [R][d], in the row order of `send`; may be NULL when R = 0) and the
- * workspace of the matching moe_w8a8_ep_dispatch with the same T.
+ * Step 5: y [T][d] (cfg.out_dtype, device, 16-byte aligned) from the returned
+ * rows o_rows (device fp32 [R][d], in the row order of `send`, 16-byte
+ * aligned and never NULL, also when R = 0: pass any valid device address
+ * then, it is not read) and the workspace of the matching
+ * moe_w8a8_ep_dispatch with the same T.  A NULL or misaligned pointer returns
+ * MOE_ERR_INVALID_ARG before anything is enqueued.
  */
 moe_status moe_w8a8_ep_combine(const moe_w8a8_weights* w, const float* o_rows, int32_t T, void* y,
                                const void* workspace, size_t workspace_bytes, moe_stream_t stream);

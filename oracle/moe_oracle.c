@@ -269,10 +269,16 @@ void oracle_topk_softmax(const float* logits, const float* bias, int64_t T, int3
 /* section 2 item 2: capacity factor, overflow dropped).                    */
 /* ------------------------------------------------------------------------ */
 
-/* C = ceil(cf * T * k / E) in fp64 (READING); cf <= 0 means no limit (-1). */
+/* C = ceil(cf * T * k / E) in fp64 (READING); cf <= 0 means no limit (-1).
+ * No expert can receive more than T * k arrivals, so C is clamped to T * k
+ * before the integer conversion: the kept set is the same, and a huge or
+ * infinite cf no longer overflows the conversion. */
 int32_t oracle_capacity(float cf, int64_t T, int32_t k, int32_t E) {
     if (!(cf > 0.0f)) return -1;
-    return (int32_t)ceil((double)cf * (double)(T * k) / (double)E);
+    const double tk = (double)(T * k);
+    double c = ceil((double)cf * tk / (double)E);
+    if (!(c <= tk)) c = tk;
+    return (int32_t)c;
 }
 
 /* Rows are the kept (t, slot) pairs ordered by expert, then by token.  The

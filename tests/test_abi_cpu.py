@@ -142,6 +142,67 @@ def test_expert_parallel_host_side_checks(M):
     assert L.moe_w8a8_ep_combine(None, z, 32, z, z, 1 << 20, None) == M.MOE_ERR_INVALID_ARG
 
 
+def test_pointer_checks_come_before_the_handle(M):
+    """Null and misaligned device pointers are refused with
+    MOE_ERR_INVALID_ARG before the handle is looked at (so nothing is
+    enqueued).  The handle here is a zeroed host buffer that is never read:
+    the pointer checks fail first.  x, y, router_bias and router_logits are
+    read with 16-byte vector accesses, so each must be 16-byte aligned."""
+    L = M.lib()
+    fake = ctypes.create_string_buffer(4096)
+    h = ctypes.c_void_p(ctypes.addressof(fake))
+    ok, odd = ctypes.c_void_p(1 << 20), ctypes.c_void_p((1 << 20) + 8)
+    ws = ctypes.c_void_p(1 << 24)
+    bad = M.MOE_ERR_INVALID_ARG
+    fwd = L.moe_w8a8_forward
+    assert fwd(h, odd, 32, None, None, ok, ws, 1 << 30, None, None) == bad           # x
+    assert fwd(h, ok, 32, None, None, odd, ws, 1 << 30, None, None) == bad           # y
+    assert fwd(h, ok, 32, odd, None, ok, ws, 1 << 30, None, None) == bad             # router_bias
+    assert fwd(h, ok, 32, None, odd, ok, ws, 1 << 30, None, None) == bad             # router_logits
+    assert fwd(h, ok, 32, None, None, ok, ctypes.c_void_p((1 << 24) + 16), 1 << 30, None, None) == bad
+    assert fwd(h, None, 32, None, None, ok, ws, 1 << 30, None, None) == bad
+    assert L.moe_w8a8_forward_noalloc(h, odd, 32, None, None, ok, None) == bad
+    assert L.moe_w8a8_forward_noalloc(h, ok, 32, None, odd, ok, None) == bad
+    assert L.moe_w8a8_ep_dispatch(h, odd, 32, None, None, ok, ok, ws, 1 << 30, None, None) == bad
+    assert L.moe_w8a8_ep_dispatch(h, ok, 32, odd, None, ok, ok, ws, 1 << 30, None, None) == bad
+    assert L.moe_w8a8_ep_experts(h, ok, 32, odd, ws, 1 << 30, None, None) == bad
+    # the combine reads o_rows for every kept slot: NULL or misaligned is refused
+    assert L.moe_w8a8_ep_combine(h, None, 32, ok, ws, 1 << 30, None) == bad
+    assert L.moe_w8a8_ep_combine(h, odd, 32, ok, ws, 1 << 30, None) == bad
+    assert L.moe_w8a8_ep_combine(h, ok, 32, odd, ws, 1 << 30, None) == bad
+
+
+def test_capacity_factor_must_be_finite(M):
+    L = M.lib()
+    out = ctypes.c_void_p()
+    z = ctypes.c_void_p(16)
+    for cf in (float("inf"), float("-inf"), float("nan")):
+        c = M.make_config(4096, 1536, 64, 4, capacity_factor=cf)
+        assert L.moe_w8a8_prepare(ctypes.byref(c), z, z, z, z, z, None, ctypes.byref(out)) == \
+            M.MOE_ERR_INVALID_ARG, cf
+
+
+def test_binding_refuses_tensors_shorter_than_the_call(M):
+    """The binding checks element counts before it hands pointers over, so a
+    short tensor is an error, not an out-of-bounds device access."""
+    import torch
+    w = M.Weights(None, M.make_config(256, 512, 8, 2, in_dtype=M.MOE_F32, out_dtype=M.MOE_F32))
+    T, d, E = 16, 256, 8
+    x, y = torch.zeros(T * d), torch.zeros(T * d)
+    ws = torch.zeros(16, dtype=torch.uint8)
+    for args, name in [((torch.zeros(T * d - 1), T, None, None, y, ws), "x"),
+                       ((x, T, None, None, torch.zeros(T * d - 4), ws), "y"),
+                       ((x, T, None, torch.zeros(T * E - 1), y, ws), "router_logits"),
+                       ((x, T, torch.zeros(E - 1), None, y, ws), "router_bias")]:
+        with pytest.raises(ValueError, match=name):
+            M.moe_w8a8_forward(w, *args)
+    with pytest.raises(ValueError, match="x"):
+        M.moe_w8a8_forward_noalloc(w, torch.zeros(5), T, None, None, y)
+    import numpy as np
+    with pytest.raises(ValueError, match="y_host"):
+        M.moe_w8a8_forward_host(w, np.zeros(T * d, np.float32), T, None, None, np.zeros(3, np.float32), ws)
+
+
 def test_product_path_does_not_touch_the_oracle():
     """The library sources and the binding never name the oracle."""
     pkg = os.path.join(ROOT, "w8a8_quantized_moe_b200")

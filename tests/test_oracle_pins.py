@@ -174,6 +174,52 @@ def test_smoothing_closed_forms():
     assert np.allclose(s.astype(np.float64) * inv, 1.0, atol=2 * U32)
 
 
+def test_channel_absmax_is_the_column_max_of_abs():
+    """Calibration statistic ("MiniMax-M3 W8A8 on K100AI" s3.2): per input
+    channel, max |x| over the calibration rows; checked against numpy's
+    column maximum on a non-square matrix with a negative-only column, a zero
+    column and a planted outlier, so a wrong axis or a dropped abs fails."""
+    x = synth.normal(21, 1, (37, 48))
+    x[:, 5] = -np.abs(x[:, 5]) - 1.0
+    x[:, 7] = 0.0
+    x[30, 9] = -1e30
+    x[0, 47] = 3e-39                          # subnormal, the column's only nonzero
+    x[1:, 47] = 0.0
+    ref = np.abs(x).max(axis=0)
+    assert np.array_equal(oracle.channel_absmax(x), ref)
+    assert oracle.channel_absmax(x)[9] == np.float32(1e30)
+    assert np.array_equal(oracle.channel_absmax(x[:1]), np.abs(x[0]))
+    assert not oracle.channel_absmax(np.zeros((0, 8), np.float32)).any()
+
+
+def test_gateup_input_absmax_is_the_max_over_experts_and_outputs():
+    """Smoothing weight statistic ("MiniMax-M3 W8A8 on K100AI" s6.1, with the
+    one-s-per-layer reading): aw_j = max over every expert e and output n of
+    |W_gate[e][j][n]| and |W_up[e][j][n]|.  Brute force over (e, n), with each
+    row's maximum planted in a different expert, projection, column and sign;
+    accumulation over expert chunks equals the one-shot result."""
+    E, d, f = 5, 24, 40
+    wg = synth.normal(22, 1, (E, d, f), std=0.02)
+    wu = synth.normal(22, 2, (E, d, f), std=0.02)
+    for j in range(d):
+        tgt = wg if j % 2 else wu
+        tgt[(3 * j) % E, j, (7 * j) % f] = (-1.0 if j % 3 else 1.0) * (0.5 + j / 100.0)
+    brute = np.zeros(d, np.float32)
+    for e in range(E):
+        for j in range(d):
+            for n in range(f):
+                brute[j] = max(brute[j], abs(wg[e, j, n]), abs(wu[e, j, n]))
+    assert np.array_equal(oracle.gateup_input_absmax(wg, wu), brute)
+    aw = np.zeros(d, np.float32)
+    for lo, hi in ((0, 2), (2, 3), (3, 5)):
+        oracle.gateup_input_absmax(wg[lo:hi], wu[lo:hi], aw)
+    assert np.array_equal(aw, brute)
+    # every expert and both projections take part: leaving any out changes aw
+    assert not np.array_equal(oracle.gateup_input_absmax(wg[:E - 1], wu[:E - 1]), brute)
+    assert not np.array_equal(oracle.gateup_input_absmax(wg, np.zeros_like(wu)), brute)
+    assert not np.array_equal(oracle.gateup_input_absmax(np.zeros_like(wg), wu), brute)
+
+
 def test_weight_quant_is_per_output_channel_of_smoothed_weights():
     d, f = 32, 24
     w = synth.normal(14, 3, (d, f), std=0.02)
@@ -338,6 +384,24 @@ def test_capacity_drops_in_token_order():
     assert np.array_equal(row2ts[ts2row[kept]], np.flatnonzero(kept.reshape(-1)))
     assert oracle.capacity(0.0, T, k, E) == -1
     assert oracle.capacity(1.25, 4096, 8, 256) == 160
+
+
+def test_capacity_is_clamped_to_the_row_count():
+    """No expert can receive more than T k arrivals, so a capacity factor that
+    large keeps everything: the capacity is clamped to T k (also for an
+    infinite factor) and the permutation equals the one without a limit."""
+    T, k, E = 50, 2, 4
+    assert oracle.capacity(1e30, T, k, E) == T * k
+    assert oracle.capacity(float("inf"), T, k, E) == T * k
+    assert oracle.capacity(float(E), T, k, E) == T * k
+    assert oracle.capacity(1.0, T, k, E) == math.ceil(T * k / E)
+    keys = synth.bits(19, 1, T * k)
+    idx = np.array([[int(keys[t * k]) % E, (int(keys[t * k]) % E + 1 + int(keys[t * k + 1]) % (E - 1)) % E]
+                    for t in range(T)], np.int32)
+    capped = oracle.permute(idx, E, oracle.capacity(1e30, T, k, E))
+    free = oracle.permute(idx, E, -1)
+    for a, b in zip(capped, free):
+        assert np.array_equal(a, b)
 
 
 # ----------------------------------------------------------------------------- GEMM
@@ -611,3 +675,55 @@ def test_fp8_whole_layer_closed_form_exact_codes():
             assert np.all(np.abs(dq - q) <= step / 2 * (1 + 1e-4) + 1e-6 * np.abs(q))
             acc2 = wd[e].T @ dq                                      # exact: products fit fp64
             assert np.array_equal(dbg["acc2"][t, s], acc2.astype(np.float32))
+
+
+# ----------------------------------------------------------------------------- bf16 output cast
+
+def _bf16_rne_by_distance(v32):
+    """Round-to-nearest-even to bf16 written from the definition: the two bf16
+    neighbours of |v| (its truncation and the next bf16 above it; above the
+    largest finite bf16 the next is 2^128, i.e. infinity) are compared by
+    exact distance in fp64, a tie goes to the neighbour whose last significand
+    bit is 0, and the sign is put back."""
+    bits = v32.view(np.uint32).astype(np.uint64)
+    lo_bits = bits & 0x7FFF0000
+    hi_bits = lo_bits + 0x10000
+    lo = lo_bits.astype(np.uint32).view(np.float32).astype(np.float64)
+    hi = np.where(hi_bits >= 0x7F800000, 2.0 ** 128,
+                  np.minimum(hi_bits, 0x7F7F0000).astype(np.uint32).view(np.float32).astype(np.float64))
+    x = np.abs(v32.astype(np.float64))
+    d_lo, d_hi = x - lo, hi - x
+    lo_even = ((lo_bits >> 16) & 1) == 0
+    out = np.where((d_hi < d_lo) | ((d_hi == d_lo) & ~lo_even), hi_bits, lo_bits)
+    return (out | (bits & 0x80000000)).astype(np.uint32)
+
+
+def test_round_bf16_is_round_to_nearest_even():
+    """The final bf16 cast of every bf16 layer: equal, bit for bit, to the
+    definition above and to torch's fp32 -> bf16 conversion, on every tie
+    pattern (even and odd last kept bit, carries into the exponent, the
+    largest finite bf16 and the overflow to infinity), on subnormals and on
+    10^6 random finite fp32 values."""
+    import torch
+    pat = []
+    for exp_bits in (0x00, 0x01, 0x3F, 0x7E, 0x80, 0xFE):
+        for m7 in (0x00, 0x01, 0x3E, 0x7E, 0x7F):
+            for low in (0x0000, 0x0001, 0x7FFF, 0x8000, 0x8001, 0xFFFF):
+                for sign in (0, 1):
+                    pat.append((sign << 31) | (exp_bits << 23) | (m7 << 16) | low)
+    keys = synth.bits(23, 1, 1_000_000).astype(np.uint64)
+    rnd = (keys & 0xFFFFFFFF).astype(np.uint32)
+    rnd = rnd[((rnd >> 23) & 0xFF) != 0xFF]                  # finite values only
+    near_max = (0x7F7F0000 + (keys[:4096] & 0xFFFF)).astype(np.uint32)
+    v = np.concatenate([np.array(pat, np.uint32), rnd, near_max]).view(np.float32)
+    got = oracle.round_bf16(v).view(np.uint32)
+    assert np.array_equal(got, _bf16_rne_by_distance(v))
+    lib = torch.from_numpy(v.copy()).to(torch.bfloat16).to(torch.float32).numpy().view(np.uint32)
+    assert np.array_equal(got, lib)
+    # hand-worked cases: ties to even, carry into the exponent, overflow
+    one = np.float32(1.0).view(np.uint32)
+    cases = {one | 0x8000: one, (one | 0x10000) | 0x8000: one + 0x20000,
+             0x3F7F8000: 0x3F800000, 0x7F7F7FFF: 0x7F7F0000, 0x7F7F8000: 0x7F800000,
+             0x00008000: 0x00000000, 0x00018000: 0x00020000}
+    for src, dst in cases.items():
+        assert oracle.round_bf16(np.array([src], np.uint32).view(np.float32)).view(np.uint32)[0] == dst, hex(src)

@@ -147,6 +147,24 @@ def _dev_ptr(t, dtype=None, name="tensor", allow_none=False):
     return ctypes.c_void_p(t.data_ptr())
 
 
+def _need(t, n: int, name: str):
+    """A tensor passed for n elements must hold at least n of them (the
+    library indexes it up to there)."""
+    if t is None:
+        return
+    count = int(t.size) if not callable(getattr(t, "size", None)) else t.numel()   # numpy or torch
+    if count < n:
+        raise ValueError(f"{name} holds {count} elements, the call reads or writes {n}")
+
+
+def _layer_io(w, x, T: int, router_bias, router_logits, y, suffix: str = ""):
+    c = w.cfg
+    _need(x, T * c.d, "x" + suffix)
+    _need(y, T * c.d, "y" + suffix)
+    _need(router_logits, T * c.n_experts, "router_logits" + suffix)
+    _need(router_bias, c.n_experts, "router_bias" + suffix)
+
+
 def _host_ptr(a, name="array", allow_none=False):
     if a is None:
         if allow_none:
@@ -252,6 +270,7 @@ def _debug_struct(dbg: dict | None):
 def moe_w8a8_forward(w: Weights, x, T: int, router_bias, router_logits, y, workspace,
                      dbg: dict | None = None, stream=None):
     torch = _torch()
+    _layer_io(w, x, T, router_bias, router_logits, y)
     _s, dptr = _debug_struct(dbg)
     _check(lib().moe_w8a8_forward(
         w.handle, _dev_ptr(x, _act_dtype(w.cfg.in_dtype), "x"), int(T),
@@ -263,6 +282,7 @@ def moe_w8a8_forward(w: Weights, x, T: int, router_bias, router_logits, y, works
 
 def moe_w8a8_forward_host(w: Weights, x_host, T: int, router_bias_host, router_logits_host,
                           y_host, workspace, stream=None):
+    _layer_io(w, x_host, T, router_bias_host, router_logits_host, y_host, "_host")
     _check(lib().moe_w8a8_forward_host(
         w.handle, _host_ptr(x_host, "x_host"), int(T),
         _host_ptr(router_bias_host, "router_bias_host", True),
@@ -358,6 +378,7 @@ def moe_w8a8_forward_noalloc(w: Weights, x, T: int, router_bias, router_logits, 
     """Forward for callers that cannot allocate: scratch comes from the
     library's fixed device array (see the header); no workspace argument."""
     torch = _torch()
+    _layer_io(w, x, T, router_bias, router_logits, y)
     _check(lib().moe_w8a8_forward_noalloc(
         w.handle, _dev_ptr(x, _act_dtype(w.cfg.in_dtype), "x"), int(T),
         _dev_ptr(router_bias, torch.float32, "router_bias", True),
@@ -418,6 +439,12 @@ def moe_w8a8_ep_experts_workspace_size(w: Weights, rows: int) -> int:
 def moe_w8a8_ep_dispatch(w: Weights, x, T: int, router_bias, router_logits, send, expert_offsets, workspace,
                          dbg: dict | None = None, stream=None):
     torch = _torch()
+    c = w.cfg
+    _need(x, T * c.d, "x")
+    _need(router_logits, T * c.n_experts, "router_logits")
+    _need(router_bias, c.n_experts, "router_bias")
+    _need(send, T * c.top_k * moe_w8a8_ep_row_bytes(w), "send")
+    _need(expert_offsets, c.n_experts + 1, "expert_offsets")
     _s, dptr = _debug_struct(dbg)
     _check(lib().moe_w8a8_ep_dispatch(
         w.handle, _dev_ptr(x, _act_dtype(w.cfg.in_dtype), "x", T == 0), int(T),
@@ -432,6 +459,8 @@ def moe_w8a8_ep_experts(w: Weights, recv, R: int, o_rows, workspace, dbg: dict |
     torch = _torch()
     if R == 0:
         return
+    _need(recv, R * moe_w8a8_ep_row_bytes(w), "recv")
+    _need(o_rows, R * w.cfg.d, "o_rows")
     _s, dptr = _debug_struct(dbg)
     _check(lib().moe_w8a8_ep_experts(
         w.handle, _dev_ptr(recv, torch.uint8, "recv"), int(R), _dev_ptr(o_rows, torch.float32, "o_rows"),
@@ -442,7 +471,10 @@ def moe_w8a8_ep_combine(w: Weights, o_rows, T: int, y, workspace, stream=None):
     torch = _torch()
     if T == 0:
         return
-    o_ptr = None if o_rows is None or o_rows.numel() == 0 else _dev_ptr(o_rows, torch.float32, "o_rows")
+    _need(y, T * w.cfg.d, "y")
+    # o_rows may hold no rows (every slot dropped), but its pointer must be a
+    # real device address: the library refuses NULL
+    o_ptr = ctypes.c_void_p(o_rows.data_ptr()) if o_rows is not None and o_rows.is_cuda else None
     _check(lib().moe_w8a8_ep_combine(
         w.handle, o_ptr, int(T), _dev_ptr(y, _act_dtype(w.cfg.out_dtype), "y"),
         _dev_ptr(workspace, name="workspace"), _nbytes(workspace), _stream(stream)), "moe_w8a8_ep_combine")

@@ -26,7 +26,7 @@ moe_status check_config(const moe_w8a8_config* c) {
     if (c->out_dtype != MOE_F32 && c->out_dtype != MOE_BF16) return MOE_ERR_INVALID_ARG;
     if (c->renormalize != 0 && c->renormalize != 1) return MOE_ERR_INVALID_ARG;
     if (c->expert_format != MOE_FMT_INT8 && c->expert_format != MOE_FMT_E4M3) return MOE_ERR_INVALID_ARG;
-    if (std::isnan(c->capacity_factor)) return MOE_ERR_INVALID_ARG;
+    if (!std::isfinite(c->capacity_factor)) return MOE_ERR_INVALID_ARG;
     if (c->d <= 0 || c->f <= 0 || c->n_experts <= 0 || c->top_k <= 0) return MOE_ERR_UNSUPPORTED_SHAPE;
     if (c->d % 128 || c->f % 128) return MOE_ERR_UNSUPPORTED_SHAPE;
     if (c->d > 16384 || c->f > 16384) return MOE_ERR_UNSUPPORTED_SHAPE;
@@ -34,11 +34,18 @@ moe_status check_config(const moe_w8a8_config* c) {
     return MOE_OK;
 }
 
-// Capacity per expert: ceil(cf * T * k / E) in fp64, -1 for none.
+// Capacity per expert: ceil(cf * T * k / E) in fp64, -1 for none.  Clamped to
+// T * k before the conversion (no expert can receive more rows than that, so
+// the clamp changes nothing but keeps the conversion defined for large cf).
 int capacity_of(const moe_w8a8_config& c, int T) {
     if (!(c.capacity_factor > 0.0f)) return -1;
-    return (int)std::ceil((double)c.capacity_factor * (double)((int64_t)T * c.top_k) / (double)c.n_experts);
+    const double tk = (double)((int64_t)T * c.top_k);
+    const double cap = std::ceil((double)c.capacity_factor * tk / (double)c.n_experts);
+    return (int)std::min(cap, tk);
 }
+
+// A device pointer the kernels read or write with 16-byte vector accesses.
+bool misaligned16(const void* p) { return ((uintptr_t)p & 15) != 0; }
 
 bool tensor_ok(const moe_w8a8_weights* w) { return w->tmaps_ok && tc_supported(w->cfg); }
 
@@ -409,7 +416,7 @@ moe_status route_stage(Run& r, const void* x, int T, const float* bias, const fl
     float* dbg_logits = r.dbg ? r.dbg->logits : nullptr;
 
     const float* lsrc = given_logits;
-    const bool certified = !lsrc && router_tc_ok(w, T) && ((uintptr_t)x & 15) == 0;
+    const bool certified = !lsrc && router_tc_ok(w, T);
     if (certified) {
         // approximate logits on the tensor cores, then per token the candidates'
         // logits in the stated order, top-k and gate weights
@@ -631,8 +638,11 @@ moe_status moe_w8a8_forward(const moe_w8a8_weights* w, const void* x, int32_t T,
                             moe_stream_t stream) {
     if (!w || T < 0) return MOE_ERR_INVALID_ARG;
     if (T == 0) return MOE_OK;
-    if (!x || !y || !workspace || !holds_all_experts(w) || !on_handle_device(w)) return MOE_ERR_INVALID_ARG;
-    if ((uintptr_t)workspace % kAlign) return MOE_ERR_INVALID_ARG;
+    if (!x || !y || !workspace) return MOE_ERR_INVALID_ARG;
+    if ((uintptr_t)workspace % kAlign || misaligned16(x) || misaligned16(y) || misaligned16(router_bias) ||
+        misaligned16(router_logits))
+        return MOE_ERR_INVALID_ARG;
+    if (!holds_all_experts(w) || !on_handle_device(w)) return MOE_ERR_INVALID_ARG;
     if (!path_ok(w, T)) return MOE_ERR_UNSUPPORTED_SHAPE;
     if (workspace_bytes < ws_layout(w, T).total) return MOE_ERR_WORKSPACE_TOO_SMALL;
     return forward_impl(w, x, T, router_bias, router_logits, y, (char*)workspace, dbg,
@@ -645,8 +655,9 @@ moe_status moe_w8a8_forward_host(const moe_w8a8_weights* w, const void* x_host, 
                                  moe_stream_t stream) {
     if (!w || T < 0) return MOE_ERR_INVALID_ARG;
     if (T == 0) return MOE_OK;
-    if (!x_host || !y_host || !workspace || !holds_all_experts(w) || !on_handle_device(w)) return MOE_ERR_INVALID_ARG;
+    if (!x_host || !y_host || !workspace) return MOE_ERR_INVALID_ARG;
     if ((uintptr_t)workspace % kAlign) return MOE_ERR_INVALID_ARG;
+    if (!holds_all_experts(w) || !on_handle_device(w)) return MOE_ERR_INVALID_ARG;
     if (!path_ok(w, T)) return MOE_ERR_UNSUPPORTED_SHAPE;
     const WsLayout L = ws_layout(w, T);
     if (workspace_bytes < L.total) return MOE_ERR_WORKSPACE_TOO_SMALL;
@@ -850,8 +861,11 @@ moe_status moe_w8a8_ep_dispatch(const moe_w8a8_weights* w, const void* x, int32_
         CUDA_TRY(cudaMemsetAsync(expert_offsets, 0, (size_t)(c.n_experts + 1) * 4, s));
         return MOE_OK;
     }
-    if (!x || !send || !workspace || !on_handle_device(w)) return MOE_ERR_INVALID_ARG;
-    if ((uintptr_t)workspace % kAlign || (uintptr_t)send % 16) return MOE_ERR_INVALID_ARG;
+    if (!x || !send || !workspace) return MOE_ERR_INVALID_ARG;
+    if ((uintptr_t)workspace % kAlign || misaligned16(send) || misaligned16(x) || misaligned16(router_bias) ||
+        misaligned16(router_logits))
+        return MOE_ERR_INVALID_ARG;
+    if (!on_handle_device(w)) return MOE_ERR_INVALID_ARG;
     const WsLayout L = ws_layout(w, T, WS_ROUTE);
     if (workspace_bytes < L.total) return MOE_ERR_WORKSPACE_TOO_SMALL;
     Run r(w, L, (char*)workspace, dbg, s);
@@ -870,8 +884,9 @@ moe_status moe_w8a8_ep_experts(const moe_w8a8_weights* w, const void* recv, int3
                                moe_stream_t stream) {
     if (!w || R < 0) return MOE_ERR_INVALID_ARG;
     if (R == 0) return MOE_OK;
-    if (!recv || !o_rows || !workspace || !on_handle_device(w)) return MOE_ERR_INVALID_ARG;
-    if ((uintptr_t)workspace % kAlign || (uintptr_t)recv % 16 || (uintptr_t)o_rows % 16) return MOE_ERR_INVALID_ARG;
+    if (!recv || !o_rows || !workspace) return MOE_ERR_INVALID_ARG;
+    if ((uintptr_t)workspace % kAlign || misaligned16(recv) || misaligned16(o_rows)) return MOE_ERR_INVALID_ARG;
+    if (!on_handle_device(w)) return MOE_ERR_INVALID_ARG;
     const moe_w8a8_weights v = expert_view(w);
     if (!path_ok(&v, R)) return MOE_ERR_UNSUPPORTED_SHAPE;
     const int path = choose_path(&v, R);
@@ -909,8 +924,9 @@ moe_status moe_w8a8_ep_combine(const moe_w8a8_weights* w, const float* o_rows, i
                                const void* workspace, size_t workspace_bytes, moe_stream_t stream) {
     if (!w || T < 0) return MOE_ERR_INVALID_ARG;
     if (T == 0) return MOE_OK;
-    if (!y || !workspace || !on_handle_device(w)) return MOE_ERR_INVALID_ARG;
-    if ((uintptr_t)workspace % kAlign || (uintptr_t)o_rows % 16) return MOE_ERR_INVALID_ARG;
+    if (!y || !o_rows || !workspace) return MOE_ERR_INVALID_ARG;
+    if ((uintptr_t)workspace % kAlign || misaligned16(o_rows) || misaligned16(y)) return MOE_ERR_INVALID_ARG;
+    if (!on_handle_device(w)) return MOE_ERR_INVALID_ARG;
     const moe_w8a8_config& c = w->cfg;
     const WsLayout L = ws_layout(w, T, WS_ROUTE);
     if (workspace_bytes < L.total) return MOE_ERR_WORKSPACE_TOO_SMALL;
@@ -966,7 +982,10 @@ extern "C" moe_status moe_w8a8_forward_noalloc(const moe_w8a8_weights* w, const 
                                                moe_stream_t stream) {
     if (!w || T < 0) return MOE_ERR_INVALID_ARG;
     if (T == 0) return MOE_OK;
-    if (!x || !y || !holds_all_experts(w) || !on_handle_device(w)) return MOE_ERR_INVALID_ARG;
+    if (!x || !y) return MOE_ERR_INVALID_ARG;
+    if (misaligned16(x) || misaligned16(y) || misaligned16(router_bias) || misaligned16(router_logits))
+        return MOE_ERR_INVALID_ARG;
+    if (!holds_all_experts(w) || !on_handle_device(w)) return MOE_ERR_INVALID_ARG;
     if (!path_ok(w, T)) return MOE_ERR_UNSUPPORTED_SHAPE;
     if (ws_layout(w, T).total > (size_t)MOE_NOALLOC_SCRATCH_BYTES) return MOE_ERR_WORKSPACE_TOO_SMALL;
     void* scratch = noalloc_scratch_for_current_device();
