@@ -74,6 +74,9 @@ def parse():
                    help="time the expert-parallel layer (experts split over the ranks) instead")
     p.add_argument("--no-prefill", action="store_true",
                    help="skip the extra prefill-layer measurement of the decode run")
+    p.add_argument("--no-tensor-peak", action="store_true",
+                   help="skip the 8-bit tensor-core rate loop (the tensor-bound roofline then divides by "
+                        "2 x the bf16 peak)")
     return p.parse_args()
 
 
@@ -153,6 +156,42 @@ class ClockSampler:
         return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
                 "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
                 "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------------ measured 8-bit tensor peak
+
+NOMINAL_INT8_TOPS = 4500.0   # NVIDIA's dense INT8 / FP8 figure for B200 (context only)
+
+
+def measure_tensor_peak(local: int, fmt: int) -> dict:
+    """The dense 8-bit tensor-core rate of this GPU with the library's own
+    tcgen05 MMA loop (operands resident in shared memory, one block per SM):
+    a burst (~20 ms, the rate a kernel timed alone sees) and a sustained run
+    (~0.5-1 s, under the power cap), each with the SM clocks sampled during
+    it."""
+    import torch
+
+    import w8a8_quantized_moe_b200 as M
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream(dev)
+    M.moe_w8a8_tensor_peak_loop(fmt, 1 << 14)
+    torch.cuda.synchronize(dev)
+    out = {}
+    for name, n in (("burst", 1 << 18), ("sustained", 1 << 23)):
+        clocks = ClockSampler(local)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        clocks.start()
+        e0.record(stream)
+        ops = M.moe_w8a8_tensor_peak_loop(fmt, n)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        clocks.stop()
+        ms = e0.elapsed_time(e1)
+        out[name] = {"tops": ops / (ms / 1e3) / 1e12, "ms": ms, "mma_per_sm": n, "clocks": clocks.summary()}
+    out["kernel"] = "tc_peak_kernel (tcgen05.mma %s, M=128 N=256 K=32, operands in shared memory)" % (
+        "kind::f8f6f4 E4M3" if fmt == 1 else "kind::i8")
+    out["nominal_tops"] = NOMINAL_INT8_TOPS
+    return out
 
 
 # ------------------------------------------------------------------ byte / op model
@@ -297,7 +336,8 @@ def run_reference(args, world, rank):
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": 1e3 * secs / args.steps, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "e4m3" if args.format == "e4m3" else "int8", "data": "synthetic",
-            "config": {"workload": describe(wl), "parallelism": "single CPU thread"},
+            "config": {"workload": describe(wl), "T": wl.T, "d": wl.d, "E": wl.E, "k": wl.k, "f": wl.f,
+                       "alpha": wl.alpha, "parallelism": "single CPU thread"},
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
@@ -442,7 +482,14 @@ def measure(args, wl, world, rank, local, e2e_on=True, wts=None):
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(yh.numel() * yh.element_size())}
 
     peaks, peak_src = load_peaks()
-    int8_peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]) * INT8_PER_BF16
+    tpk = getattr(args, "tensor_peak", None)
+    if tpk:
+        int8_peak = tpk["burst"]["tops"]
+        int8_src = (f"burst rate of the library's own tcgen05 8-bit MMA loop on this GPU "
+                    f"({tpk['burst']['ms']:.1f} ms); sustained {tpk['sustained']['tops']:.0f} TOPS")
+    else:
+        int8_peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]) * INT8_PER_BF16
+        int8_src = f"2 x bf16_tflops_sustained of {peak_src} (INT8 dense = 2 x bf16, nominal)"
     roof = None
     if stages:
         dom = max(("gemm1", "gemm2"), key=lambda k: stages[k])
@@ -459,9 +506,11 @@ def measure(args, wl, world, rank, local, e2e_on=True, wts=None):
             roof = {"bound": "tensor", "kernel": f"{dom} ({kernel})", "achieved": achieved,
                     "peak": int8_peak, "unit": "TFLOP/s", "frac": achieved / int8_peak,
                     "traffic": TRAFFIC.get((wl.name, wl.T, kernel)),
-                    "peak_source": f"2 x bf16_tflops_sustained of {peak_src} (INT8 dense = 2 x bf16, nominal)",
+                    "peak_source": int8_src,
                     "int8_ops_per_launch": ops, "launch_ms": dom_ms,
-                    "frac_of_nominal_4500": achieved / 4500.0}
+                    "frac_of_nominal_4500": achieved / NOMINAL_INT8_TOPS}
+            if tpk:
+                roof["frac_of_sustained"] = achieved / tpk["sustained"]["tops"]
         else:
             achieved = nbytes / (dom_ms / 1e3) / 1e9
             roof = {"bound": "hbm", "kernel": f"{dom} ({kernel})", "achieved": achieved,
@@ -483,7 +532,9 @@ def measure(args, wl, world, rank, local, e2e_on=True, wts=None):
                    "parallelism": "replicas" if world > 1 else "single GPU",
                    "layer_bytes_per_step": alg["layer_bytes"], "layer_gbs": layer_gbs,
                    "layer_hbm_frac": layer_gbs / peaks["hbm_gbs"],
-                   "int8_ops_per_step": alg["int8_ops"], "layer_int8_tops": layer_tops},
+                   "int8_ops_per_step": alg["int8_ops"], "layer_int8_tops": layer_tops,
+                   "layer_int8_frac": layer_tops / int8_peak,
+                   "layer_int8_frac_of_nominal_4500": layer_tops / NOMINAL_INT8_TOPS},
         "roofline": roof, "stages_ms": stages, "e2e": e2e, "gpu_launches": launches,
         "clocks": clocks.summary(),
     }
@@ -503,7 +554,8 @@ def run_sweep(args, local):
 
     dev = torch.device("cuda", local)
     peaks, peak_src = load_peaks()
-    int8_peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]) * INT8_PER_BF16
+    tpk = measure_tensor_peak(local, 0)
+    int8_peak = tpk["burst"]["tops"]
     points = synth.sweep_workloads()
     base = synth.WORKLOADS["decode"]
     wts = synth.make_weights(base)
@@ -558,7 +610,8 @@ def run_sweep(args, local):
                               "tokens_per_s": T / step_s, "ms_per_step": step_s * 1e3,
                               "active_experts": n_active, "rows": R, "bound": bound,
                               "roofline_frac": max(t_hbm, t_tc) / step_s,
-                              "peak_source": f"{peak_src} (hbm_gbs, 2 x bf16_tflops_sustained)"}),
+                              "peak_source": f"hbm_gbs of {peak_src}; 8-bit tensor burst rate of the "
+                                             f"library's MMA loop on this GPU ({int8_peak:.0f} TOPS)"}),
                   flush=True)
             del ws
         M.moe_w8a8_set_path(W, M.MOE_PATH_AUTO)
@@ -582,6 +635,8 @@ def run_ours(args, world, rank, local):
     if args.tokens > 0:
         base = dataclasses.replace(base, T=args.tokens)
     wl = replica_workload(base, rank)
+    args.tensor_peak = measure_tensor_peak(local, 1 if args.format == "e4m3" else 0) \
+        if not args.no_tensor_peak else None
     res, wts, W = measure(args, wl, world, rank, local)
     del W
 
@@ -634,6 +689,8 @@ def run_ours(args, world, rank, local):
             "clocks": res["clocks"], "cpu_baseline": cpu}
     if extra is not None:
         line["prefill"] = extra
+    if args.tensor_peak:
+        line["tensor_peak"] = args.tensor_peak
     print(json.dumps(line), flush=True)
 
 

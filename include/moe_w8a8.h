@@ -230,6 +230,22 @@ moe_status moe_w8a8_forward_noalloc(const moe_w8a8_weights* w, const void* x, in
                                     const float* router_bias, const float* router_logits,
                                     void* y, moe_stream_t stream);
 
+/*
+ * Measurement aid (no counterpart on the pages): the dense 8-bit tensor-core
+ * rate this library's own MMA reaches on the current device, the denominator
+ * of the tensor-bound roofline.  Enqueues one launch of one thread block per
+ * SM; each issues mma_per_sm tcgen05 MMAs of M=128 x N=256 x K=32 (kind::i8
+ * for MOE_FMT_INT8, kind::f8f6f4 E4M3 for MOE_FMT_E4M3) back to back on
+ * operands held in shared memory (pseudo-random codes), with no data
+ * movement.  *ops_out receives the launch's operation count (2 x M x N x K x
+ * MMAs x SMs); the caller times the launch (events on `stream`).
+ * 0 < mma_per_sm <= MOE_PEAK_MAX_MMA (about a second of work), else
+ * MOE_ERR_INVALID_ARG.  Allocates nothing.
+ */
+#define MOE_PEAK_MAX_MMA (1LL << 24)
+moe_status moe_w8a8_tensor_peak_loop(int32_t expert_format, int64_t mma_per_sm, double* ops_out,
+                                     moe_stream_t stream);
+
 /* Select the expert GEMM path (MOE_PATH_*). */
 moe_status moe_w8a8_set_path(moe_w8a8_weights* w, int32_t path);
 

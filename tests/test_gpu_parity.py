@@ -124,7 +124,7 @@ def test_capacity_drops_overflow_in_token_order(M):
     assert (rt.ts2row < 0).sum() > 0
 
 
-def test_zipf_bias_and_no_renormalise_paths_match(M):
+def test_zipf_bias_stream_path(M):
     wl = dataclasses.replace(synth.WORKLOADS["tiny"], T=48, data_seed=12, zipf_s=1.1)
     run_case(M, wl, path=M.MOE_PATH_STREAM)
 

@@ -27,14 +27,10 @@ def M():
     return mod
 
 
-@pytest.mark.parametrize("name", ["tiny", "decode"])
-def test_noalloc_forward_matches_workspace_forward(M, name):
+def _check_against_workspace_forward(M, W, wl, data, T):
+    """moe_w8a8_forward_noalloc, twice in a row, against moe_w8a8_forward on
+    the same inputs."""
     import torch
-    wl = synth.WORKLOADS[name]
-    wts = synth.make_weights(wl)
-    data = synth.make_data(wl)
-    W = H.gpu_prepare(wl, wts)
-    T = wl.T
     x = H.x_tensor(wl, data)
     bias = H.to_dev(data.router_bias) if data.router_bias is not None else None
     logits = H.to_dev(data.router_logits) if data.router_logits is not None else None
@@ -53,6 +49,43 @@ def test_noalloc_forward_matches_workspace_forward(M, name):
         got = y.float().cpu().numpy()
         assert H.max_rel_err(got, ref) <= H.TOL[wl.in_bf16]
         assert np.array_equal(got, ref)
+
+
+@pytest.fixture(scope="module")
+def decode_handle(M):
+    wl = synth.WORKLOADS["decode"]
+    return wl, H.gpu_prepare(wl, synth.make_weights(wl))
+
+
+@pytest.mark.parametrize("path", ["auto", "stream", "tensor"])
+def test_noalloc_forward_matches_workspace_forward_tiny(M, path):
+    """The tiny layer on each expert path: the streaming path's scratch
+    layout (INT32 accumulators, token codes) and the tensor path's (sorted
+    rows, h, fused-launch counters) both live in the shared array."""
+    wl = synth.WORKLOADS["tiny"]
+    W = H.gpu_prepare(wl, synth.make_weights(wl))
+    M.moe_w8a8_set_path(W, {"auto": M.MOE_PATH_AUTO, "stream": M.MOE_PATH_STREAM,
+                            "tensor": M.MOE_PATH_TENSOR}[path])
+    _check_against_workspace_forward(M, W, wl, synth.make_data(wl), wl.T)
+
+
+def test_noalloc_forward_matches_workspace_forward_decode(M, decode_handle):
+    wl, W = decode_handle
+    _check_against_workspace_forward(M, W, wl, synth.make_data(wl), wl.T)
+
+
+def test_noalloc_largest_decode_batch_and_the_first_refused(M, decode_handle):
+    """The decode layer's largest batch that fits the array (62 tokens) runs
+    and matches; 63 tokens do not fit and are refused before anything runs."""
+    import torch
+    wl, W = decode_handle
+    assert M.moe_w8a8_workspace_size(W, 62) <= M.MOE_NOALLOC_SCRATCH_BYTES < M.moe_w8a8_workspace_size(W, 63)
+    _check_against_workspace_forward(M, W, wl, synth.make_data(wl, T=62), 62)
+    data = synth.make_data(wl, T=63)
+    y = torch.zeros((63, wl.d), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(M.MoeError) as e:
+        M.moe_w8a8_forward_noalloc(W, H.x_tensor(wl, data), 63, None, H.to_dev(data.router_logits), y)
+    assert e.value.status == M.MOE_ERR_WORKSPACE_TOO_SMALL
 
 
 def test_noalloc_refuses_token_counts_beyond_the_scratch(M):

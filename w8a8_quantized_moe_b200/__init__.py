@@ -44,9 +44,11 @@ EXPORTS = (
     "moe_w8a8_ep_row_bytes", "moe_w8a8_gateup_absmax", "moe_w8a8_prepare_shard",
     "moe_w8a8_ep_dispatch_workspace_size", "moe_w8a8_ep_experts_workspace_size",
     "moe_w8a8_ep_dispatch", "moe_w8a8_ep_experts", "moe_w8a8_ep_combine",
+    "moe_w8a8_tensor_peak_loop",
 )
 
 MOE_NOALLOC_SCRATCH_BYTES = 8 << 20
+MOE_PEAK_MAX_MMA = 1 << 24
 
 MOE_N_STAGES = 8
 
@@ -116,6 +118,7 @@ def lib():
             "moe_w8a8_ep_dispatch": ([vp, vp, i32, vp, vp, vp, vp, vp, sz, vp, vp], i32),
             "moe_w8a8_ep_experts": ([vp, vp, i32, vp, vp, sz, vp, vp], i32),
             "moe_w8a8_ep_combine": ([vp, vp, i32, vp, vp, sz, vp], i32),
+            "moe_w8a8_tensor_peak_loop": ([i32, i64, ctypes.POINTER(ctypes.c_double), vp], i32),
         }
         for name, (args, res) in sig.items():
             fn = getattr(L, name)
@@ -478,3 +481,14 @@ def moe_w8a8_ep_combine(w: Weights, o_rows, T: int, y, workspace, stream=None):
     _check(lib().moe_w8a8_ep_combine(
         w.handle, o_ptr, int(T), _dev_ptr(y, _act_dtype(w.cfg.out_dtype), "y"),
         _dev_ptr(workspace, name="workspace"), _nbytes(workspace), _stream(stream)), "moe_w8a8_ep_combine")
+
+
+# ------------------------------------------------------------------ measurement aid
+
+def moe_w8a8_tensor_peak_loop(expert_format: int, mma_per_sm: int, stream=None) -> float:
+    """Enqueue the tensor-core rate loop; returns its operation count (the
+    caller times the launch)."""
+    ops = ctypes.c_double(0.0)
+    _check(lib().moe_w8a8_tensor_peak_loop(int(expert_format), int(mma_per_sm), ctypes.byref(ops),
+                                           _stream(stream)), "moe_w8a8_tensor_peak_loop")
+    return float(ops.value)

@@ -165,6 +165,9 @@ cudaError_t launch_router_select(const moe_w8a8_weights* w, const void* x, int T
                                  cudaStream_t s);
 constexpr int kRouterTcMinTokens = 1024;   // the certified router runs from this many tokens up
 bool tc_supported(const moe_w8a8_config& c);
+// n_mma back-to-back M=128 N=256 K=32 8-bit MMAs per CTA on `grid` CTAs
+// (operands resident in shared memory): the tensor pipe's own rate.
+cudaError_t launch_tc_peak(int fmt, int64_t n_mma, int grid, cudaStream_t s);
 cudaError_t launch_tc_gemm1(const moe_w8a8_weights* w, int T, const int8_t* aq, const int32_t* meta,
                             const int32_t* tiles, const int32_t* offsets, const int32_t* row2ts,
                             const float* sx, float* h32, float* pamax, int32_t* acc_dbg,

@@ -1054,6 +1054,69 @@ __global__ void __launch_bounds__(kRcThreads, 1)
     }
 }
 
+// ------------------------------------------------------------------ tensor-core rate
+
+// The dense 8-bit tensor-core rate of this GPU as this library's own MMAs
+// reach it: one CTA per SM; the A (128 x 128 B) and B (256 x 128 B) tiles of
+// one k-block of the grouped GEMMs, filled once with pseudo-random codes (the
+// switching activity, hence the power draw and the clock, of real operands),
+// stay in shared memory; one thread issues n_mma M=128 x N=256 x K=32 MMAs
+// back to back, stepping through the k-block's four K slices as the GEMMs do,
+// into one 256-column TMEM accumulator (restarted every 1024 MMAs so the
+// sums stay bounded).  No copies, no epilogue: the loop is the tensor pipe
+// alone.  The final commit is waited for (bounded) before TMEM is freed.
+constexpr int kPeakThreads = 128;
+constexpr size_t kPeakSmem = (size_t)kABytes + kBBytes + 1024 + 256;
+constexpr uint64_t kPeakDrainNs = 10000000000ull;   // 10 s
+
+template <int FMT>
+__global__ void __launch_bounds__(kPeakThreads, 1) tc_peak_kernel(int64_t n_mma) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    Ctl* ctl = reinterpret_cast<Ctl*>(smem + kABytes + kBBytes);
+    const int warp = threadIdx.x >> 5;
+    // pseudo-random codes; E4M3 codes keep exponent field < 15 (finite, no NaN)
+    uint32_t* w32 = reinterpret_cast<uint32_t*>(smem);
+    for (int i = threadIdx.x; i < (kABytes + kBBytes) / 4; i += blockDim.x) {
+        uint32_t h = (uint32_t)i * 0x9E3779B1u + blockIdx.x * 0x85EBCA77u;
+        h ^= h >> 15;
+        h *= 0x2C1B3C6Du;
+        h ^= h >> 13;
+        w32[i] = FMT == FMT_E4M3 ? (h & 0xB7B7B7B7u) : h;
+    }
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    if (threadIdx.x == 0) {
+        mbar_init(&ctl->drain, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 0) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         smem_u32(&ctl->tmem_base)),
+                     "r"((uint32_t)BN));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = ctl->tmem_base;
+    if (threadIdx.x == 0) {
+        const uint32_t a_addr = smem_u32(smem), b_addr = a_addr + kABytes;
+        for (int64_t i = 0; i < n_mma; ++i) {
+            const int kk = (int)(i & 3);
+            mma_8bit<FMT>(tmem, desc_sw128(a_addr + kk * 32), desc_sw128(b_addr + kk * 32), (i & 1023) ? 1u : 0u);
+        }
+        mma_commit(&ctl->drain);
+        const uint64_t t0 = global_timer();
+        while (!mbar_try_wait(&ctl->drain, 0) && global_timer() - t0 < kPeakDrainNs) {}
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"((uint32_t)BN));
+    }
+}
+
 // ------------------------------------------------------------------ host side
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -1205,6 +1268,18 @@ cudaError_t launch_router_tc(const moe_w8a8_weights* w, const void* x, int T, fl
         case 256: return launch_router_tc_pad<256>(mx, w, T, approx, s);
     }
     return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_tc_peak(int fmt, int64_t n_mma, int grid, cudaStream_t s) {
+    static std::atomic<uint64_t> a8{0}, af8{0};
+    if (fmt == FMT_E4M3) {
+        cudaError_t e = smem_attr_once(tc_peak_kernel<FMT_E4M3>, kPeakSmem, af8);
+        if (e != cudaSuccess) return e;
+        return launch_pdl(tc_peak_kernel<FMT_E4M3>, dim3(grid), dim3(kPeakThreads), kPeakSmem, s, n_mma);
+    }
+    cudaError_t e = smem_attr_once(tc_peak_kernel<FMT_INT8>, kPeakSmem, a8);
+    if (e != cudaSuccess) return e;
+    return launch_pdl(tc_peak_kernel<FMT_INT8>, dim3(grid), dim3(kPeakThreads), kPeakSmem, s, n_mma);
 }
 
 bool tc_supported(const moe_w8a8_config& c) { return c.d % BN == 0 && c.f % BK == 0 && c.d % BK == 0; }

@@ -936,6 +936,21 @@ moe_status moe_w8a8_ep_combine(const moe_w8a8_weights* w, const float* o_rows, i
     return MOE_OK;
 }
 
+moe_status moe_w8a8_tensor_peak_loop(int32_t expert_format, int64_t mma_per_sm, double* ops_out,
+                                     moe_stream_t stream) {
+    if (!ops_out) return MOE_ERR_INVALID_ARG;
+    *ops_out = 0.0;
+    if (expert_format != MOE_FMT_INT8 && expert_format != MOE_FMT_E4M3) return MOE_ERR_INVALID_ARG;
+    if (mma_per_sm <= 0 || mma_per_sm > MOE_PEAK_MAX_MMA) return MOE_ERR_INVALID_ARG;
+    int dev = -1, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    CUDA_TRY(launch_tc_peak(expert_format, mma_per_sm, sms, (cudaStream_t)stream));
+    *ops_out = (double)sms * (double)mma_per_sm * 2.0 * 128.0 * 256.0 * 32.0;
+    return MOE_OK;
+}
+
 const char* moe_w8a8_stage_name(int32_t stage) {
     static const char* names[MOE_N_STAGES] = {"router", "topk", "permute", "quant",
                                               "gemm1", "requant", "gemm2", "combine"};
