@@ -305,14 +305,45 @@ moe_status moe_w8a8_check_status(const moe_w8a8_weights* w, moe_stream_t stream)
 /*
  * Diagnostics after MOE_ERR_TIMEOUT: synchronise `stream` and copy the
  * handle's status words to words_host[0..n) (n <= 16): word 0 is the status
- * code, words 1-4 say where the first bounded wait gave up (site: 1 producer
- * stage-free, 2 MMA accumulator-free, 3 MMA stage-full, 4 epilogue
- * accumulator-full; then block index, tile, and the awaited phase parity;
- * site 14: a received expert-parallel row names an expert outside the
- * handle's range, then the row index and the expert).  Does not clear them.
+ * code, words 1-4 say where the first bounded wait gave up: word 1 the site,
+ * word 2 the thread block, words 3-4 site-specific.  Sites of the tensor-core
+ * expert kernels: 1 producer waiting for a free stage, 2 MMA issuer waiting
+ * for a free accumulator, 3 MMA issuer waiting for a full stage, 4 epilogue
+ * waiting for a full accumulator (words 3-4: tile, awaited phase parity);
+ * of the fused expert launch also 6 a down-projection producer waiting for
+ * an m-tile's h codes (words 3-4: tile, m-tile), 7 a requantisation warp
+ * waiting for a queue slot (word 3: slot), 8-10 the producer, MMA issuer and
+ * epilogue waiting on the block's tile ring; 11-13 the certified router's
+ * producer, MMA issuer and epilogue.  Site 14 (with MOE_ERR_INVALID_ARG): a
+ * received expert-parallel row names an expert outside the handle's range
+ * (words 2-3: row index, expert).  Does not clear them.
  */
 moe_status moe_w8a8_status_words(const moe_w8a8_weights* w, int32_t* words_host, int32_t n,
                                  moe_stream_t stream);
+
+/*
+ * Bound on each wait of one thread block for results of another block (the
+ * fused expert launch: a down-projection tile waiting for its rows' h codes,
+ * a requantisation warp waiting for a finished m-tile), in nanoseconds, from
+ * 1 ms to 60 s; default 2 s.  When such a wait runs out the launch records
+ * MOE_ERR_TIMEOUT and the place (moe_w8a8_status_words), every block of it
+ * stops issuing work, waits (bounded) for its copies and MMAs in flight,
+ * frees its tensor memory and returns, so the GPU context stays usable;
+ * moe_w8a8_check_status reports it.  Waits on a block's own copies and MMAs
+ * keep a fixed 2 s bound.  (No counterpart on the pages, whose watchdog is a
+ * host-side check; "One night of MoE inference optimisation", s6.4.)
+ */
+moe_status moe_w8a8_set_wait_budget(moe_w8a8_weights* w, int64_t ns);
+
+/*
+ * Testing aid for the failure path above, off by default: with m_tile >= 0
+ * every later fused expert launch of this handle computes as usual but never
+ * releases the h codes of that 128-row tile (one expert's rows), so the
+ * down-projection tiles that need them wait until the budget runs out and the
+ * launch ends with MOE_ERR_TIMEOUT; the output of such a call is undefined.
+ * m_tile = -1 turns it off.  Launches that are not the fused one ignore it.
+ */
+moe_status moe_w8a8_test_withhold_release(moe_w8a8_weights* w, int32_t m_tile);
 
 /* Free the handle and its device memory (NULL is a no-op).  The caller makes
  * sure no enqueued forward still uses it. */

@@ -205,3 +205,57 @@ def test_expert_ranges_host_checks():
     assert equal_expert_ranges(64, 8) == [(8 * g, 8) for g in range(8)]
     with pytest.raises(ValueError):
         equal_expert_ranges(10, 4)
+
+
+def _leave_main(rank, world, port, out_dir):
+    """Rank 1 leaves between two layer steps (after its first step completes,
+    with nothing in flight); rank 0 starts the next step, and its first
+    exchange must end with an error within the process group's timeout
+    instead of waiting for good."""
+    sys.path.insert(0, ROOT)
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    import datetime
+    import json
+    import time
+
+    import torch.distributed as dist
+
+    import oracle
+    import synth
+    from w8a8_quantized_moe_b200.ep import ExpertParallelMoE, equal_expert_ranges
+
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=5))
+    wl = synth.WORKLOADS["tiny"]
+    wts = synth.make_weights(wl)
+    prep = oracle.prepare(wts.w_gate, wts.w_up, wts.w_down, wts.calib_x, wl.alpha)
+    first, n = equal_expert_ranges(wl.E, world)[rank]
+    layer = ExpertParallelMoE(OracleStages(wl, prep, first, n))
+    out = {"first_step": False, "error": None, "seconds": None}
+    data = synth.make_data(dataclasses.replace(wl, data_seed=wl.data_seed + 37 * rank))
+    layer.forward(data, wl.T)
+    out["first_step"] = True
+    dist.barrier()
+    if rank == 1:
+        with open(os.path.join(out_dir, f"r{rank}.json"), "w") as fh:
+            json.dump(out, fh)
+        os._exit(0)          # leaves between steps: no collective of its own in flight
+    time.sleep(0.5)
+    t0 = time.time()
+    try:
+        layer.forward(data, wl.T)
+    except Exception as exc:   # the exchange with the departed rank fails
+        out["error"] = type(exc).__name__ + ": " + str(exc).splitlines()[0][:200]
+    out["seconds"] = time.time() - t0
+    with open(os.path.join(out_dir, f"r{rank}.json"), "w") as fh:
+        json.dump(out, fh)
+    os._exit(0)
+
+
+def test_ep_rank_leaving_between_steps_is_an_error_not_a_hang(tmp_path):
+    import json
+    mp.start_processes(_leave_main, args=(2, _free_port(), str(tmp_path)), nprocs=2, start_method="spawn",
+                       join=True)
+    r0, r1 = (json.load(open(tmp_path / f"r{i}.json")) for i in range(2))
+    assert r0["first_step"] and r1["first_step"]
+    assert r0["error"] is not None
+    assert r0["seconds"] < 30.0     # the group timeout is 5 s; the peer's closed socket may end it sooner

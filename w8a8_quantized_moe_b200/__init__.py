@@ -44,7 +44,7 @@ EXPORTS = (
     "moe_w8a8_ep_row_bytes", "moe_w8a8_gateup_absmax", "moe_w8a8_prepare_shard",
     "moe_w8a8_ep_dispatch_workspace_size", "moe_w8a8_ep_experts_workspace_size",
     "moe_w8a8_ep_dispatch", "moe_w8a8_ep_experts", "moe_w8a8_ep_combine",
-    "moe_w8a8_tensor_peak_loop",
+    "moe_w8a8_tensor_peak_loop", "moe_w8a8_set_wait_budget", "moe_w8a8_test_withhold_release",
 )
 
 MOE_NOALLOC_SCRATCH_BYTES = 8 << 20
@@ -119,6 +119,8 @@ def lib():
             "moe_w8a8_ep_experts": ([vp, vp, i32, vp, vp, sz, vp, vp], i32),
             "moe_w8a8_ep_combine": ([vp, vp, i32, vp, vp, sz, vp], i32),
             "moe_w8a8_tensor_peak_loop": ([i32, i64, ctypes.POINTER(ctypes.c_double), vp], i32),
+            "moe_w8a8_set_wait_budget": ([vp, i64], i32),
+            "moe_w8a8_test_withhold_release": ([vp, i32], i32),
         }
         for name, (args, res) in sig.items():
             fn = getattr(L, name)
@@ -387,6 +389,14 @@ def moe_w8a8_forward_noalloc(w: Weights, x, T: int, router_bias, router_logits, 
         _dev_ptr(router_bias, torch.float32, "router_bias", True),
         _dev_ptr(router_logits, torch.float32, "router_logits", True),
         _dev_ptr(y, _act_dtype(w.cfg.out_dtype), "y"), _stream(stream)), "moe_w8a8_forward_noalloc")
+
+
+def moe_w8a8_set_wait_budget(w: Weights, ns: int):
+    _check(lib().moe_w8a8_set_wait_budget(w.handle, int(ns)), "moe_w8a8_set_wait_budget")
+
+
+def moe_w8a8_test_withhold_release(w: Weights, m_tile: int):
+    _check(lib().moe_w8a8_test_withhold_release(w.handle, int(m_tile)), "moe_w8a8_test_withhold_release")
 
 
 def moe_w8a8_status_words(w: Weights, n: int = 5, stream=None):

@@ -40,6 +40,8 @@ struct moe_w8a8_weights {
     int rt_epad;      // 0: no tensor-core router for this handle
     float* s_host;    // [d] (host)
     int32_t* status;  // device status word
+    uint64_t wait_budget_ns;   // bound on a block's wait for another block's results
+    int test_skip_ready;       // testing aid: fused launch withholds this m-tile's ready flag (-1: none)
     // tensor maps of the weights for the tensor-core path (built at prepare)
     CUtensorMap tm_w_gu;
     CUtensorMap tm_w_dn;

@@ -572,6 +572,8 @@ struct FusedExtra {
     int32_t* next;    // next tile to take (dynamic schedule)
     int8_t* hq;       // [rows][f] h codes
     float* sh;        // [rows] h scales
+    uint64_t budget_ns;   // bound on each wait for another block's results (ready flags, queue)
+    int skip_ready;       // testing aid: the m-tile whose ready flag is never released (-1: none)
 };                    // (count, ready, queue, qtail, qhead, next zeroed before the launch)
 
 constexpr int kFusedThreads = kThreads + 32;   // + one requantisation warp (warp 10)
@@ -604,7 +606,7 @@ constexpr size_t kFusedSmemBytes = kSmemBytes + kEpiStageBytes + 256;
 // warps of many CTAs and never delays an epilogue (when the epilogue warp that
 // completed an m-tile requantised it itself, it fell behind, became the last
 // arrival again, and the delays piled up).  The producer of a GEMM2 tile waits
-// for ready[m] (bounded) before loading its h codes.  GEMM1 tiles are all taken
+// for ready[m] (bounded by the handle's wait budget) before loading its h codes.  GEMM1 tiles are all taken
 // before any GEMM2 tile, GEMM1 tiles wait on nothing, and the requant warps
 // wait only on GEMM1 tiles, so the waits always end.  Arithmetic per element
 // is that of the two separate kernels and requant_kernel, so the results are
@@ -699,7 +701,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
                     const uint64_t t0 = global_timer();
                     while (ld_acquire(fx.ready + mt) == 0) {
                         if (*abort) { ok = false; break; }
-                        if (global_timer() - t0 > kWaitBudgetNs) {
+                        if (global_timer() - t0 > fx.budget_ns) {
                             *abort = 1;
                             report_timeout(p.status, 6, t, mt);
                             ok = false;
@@ -779,7 +781,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
                 const uint64_t t0 = global_timer();
                 while ((v = ld_acquire(fx.queue + i)) == 0) {
                     if (*abort) break;
-                    if (global_timer() - t0 > kWaitBudgetNs) {
+                    if (global_timer() - t0 > fx.budget_ns) {
                         *abort = 1;
                         report_timeout(p1.status, 7, i, 0);
                         break;
@@ -797,7 +799,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
             fence_proxy_async_global();
             __threadfence();
             __syncwarp();
-            if (lane == 0) st_release(fx.ready + mt, 1);
+            if (lane == 0 && mt != fx.skip_ready) st_release(fx.ready + mt, 1);
         }
     } else {
         // ---------------- epilogue warps
@@ -1247,7 +1249,8 @@ cudaError_t launch_tc_ffn_fused(const moe_w8a8_weights* w, int T, const int8_t* 
     p2.acc_dbg = acc2_dbg;
     const int max_mt = (rows + BM - 1) / BM + c.n_experts;
     const FusedExtra fx{sync_words, sync_words + max_mt, sync_words + 2 * max_mt, sync_words + 3 * max_mt,
-                        sync_words + 3 * max_mt + 1, sync_words + 3 * max_mt + 2, hq, sh};
+                        sync_words + 3 * max_mt + 1, sync_words + 3 * max_mt + 2, hq, sh,
+                        w->wait_budget_ns, w->test_skip_ready};
     const int grid = max(1, min(w->num_sms, max_mt * (p1.n_tiles_n + p2.n_tiles_n)));
     if (c.expert_format == FMT_E4M3)
         return launch_fused_fmt<FMT_E4M3>(a1, w->tm_w_gu, a2, w->tm_w_dn, p1, p2, fx, grid, s);

@@ -280,6 +280,8 @@ moe_status prepare_impl(const moe_w8a8_config* cfg, int e_first, int n_local, co
     w->n_local = n_local;
     w->path = MOE_PATH_AUTO;
     w->stream_max_rows = 32;   // measured crossover: streaming wins up to T*k = 32 rows
+    w->wait_budget_ns = 2000000000ull;
+    w->test_skip_ready = -1;
     if (cudaGetDevice(&w->device) != cudaSuccess ||
         cudaDeviceGetAttribute(&w->num_sms, cudaDevAttrMultiProcessorCount, w->device) != cudaSuccess) {
         free_handle(w);
@@ -693,6 +695,18 @@ moe_status moe_w8a8_set_path(moe_w8a8_weights* w, int32_t path) {
 moe_status moe_w8a8_set_stream_threshold(moe_w8a8_weights* w, int32_t max_rows) {
     if (!w || max_rows < 0) return MOE_ERR_INVALID_ARG;
     w->stream_max_rows = max_rows;
+    return MOE_OK;
+}
+
+moe_status moe_w8a8_set_wait_budget(moe_w8a8_weights* w, int64_t ns) {
+    if (!w || ns < 1000000 || ns > 60000000000ll) return MOE_ERR_INVALID_ARG;
+    w->wait_budget_ns = (uint64_t)ns;
+    return MOE_OK;
+}
+
+moe_status moe_w8a8_test_withhold_release(moe_w8a8_weights* w, int32_t m_tile) {
+    if (!w || m_tile < -1) return MOE_ERR_INVALID_ARG;
+    w->test_skip_ready = m_tile;
     return MOE_OK;
 }
 
