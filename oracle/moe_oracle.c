@@ -433,6 +433,11 @@ float oracle_round_bf16(float v) {
  * out_bf16), and per (i, slot): acc1 [i][s][2f] (gate | up), hq [i][s][f],
  * sh [i][s], acc2 [i][s][d], o [i][s][d].  Any debug output may be NULL.
  * Also xq [i][d], sx [i].
+ * READING ([Day0 adaptation] section 4 un-sorts the expert outputs and then
+ * forms the weighted sum, without fixing the precision of the per-slot rows
+ * in between): for a bf16-output layer each per-slot row o is stored in the
+ * layer's output precision, bf16 (nearest even), before the slot-order sum;
+ * an fp32-output layer keeps it in fp32.
  */
 void oracle_moe_tokens(const float* x, int32_t d, int32_t f, int32_t E, int32_t k,
                        const int8_t* wq_gate, const int8_t* wq_up, const float* sw_gate,
@@ -471,6 +476,8 @@ void oracle_moe_tokens(const float* x, int32_t d, int32_t f, int32_t E, int32_t 
                                   f, NULL, hq, &sh);
             oracle_gemm_i8(hq, wq_down + (int64_t)e * d * f, 1, d, f, acc2);
             oracle_down_epilogue(acc2, sh, sw_down + (int64_t)e * d, w[ts], d, o);
+            if (out_bf16)
+                for (int32_t n = 0; n < d; ++n) o[n] = oracle_round_bf16(o[n]);
             for (int32_t n = 0; n < d; ++n) yt[n] = yt[n] + o[n];
             if (acc1_out) {
                 memcpy(acc1_out + dbg * 2 * f, acc_g, sizeof(int32_t) * (size_t)f);
@@ -675,6 +682,8 @@ void oracle_moe_tokens_fp8(const float* x, int32_t d, int32_t f, int32_t E, int3
                                       NULL, hq, &sh);
             oracle_gemm_fp8(hq, wq_down + (int64_t)e * d * f, 1, d, f, acc2);
             for (int32_t n = 0; n < d; ++n) o[n] = ((acc2[n] * sh) * sw_down[(int64_t)e * d + n]) * w[ts];
+            if (out_bf16)   /* per-slot rows in the output precision, as for INT8 experts */
+                for (int32_t n = 0; n < d; ++n) o[n] = oracle_round_bf16(o[n]);
             for (int32_t n = 0; n < d; ++n) yt[n] = yt[n] + o[n];
             if (acc1_out) {
                 memcpy(acc1_out + dbg * 2 * f, acc_g, sizeof(float) * (size_t)f);

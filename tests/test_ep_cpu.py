@@ -86,7 +86,10 @@ class OracleStages:
             acc_u = oracle.gemm_i8(codes[None], p.wq_up[e])[0]
             _h, hq, sh = oracle.swiglu_requant(acc_g, acc_u, float(sx), p.sw_gate[e], p.sw_up[e])
             acc2 = oracle.gemm_i8(hq[None], p.wq_down[e])[0]
-            o_rows[r] = torch.from_numpy(oracle.down_epilogue(acc2, sh, p.sw_down[e], float(w)))
+            o = oracle.down_epilogue(acc2, sh, p.sw_down[e], float(w))
+            if self.wl.in_bf16:          # per-slot rows in the layer's output precision
+                o = oracle.round_bf16(o)
+            o_rows[r] = torch.from_numpy(o)
 
     def combine(self, o_rows, T, y, ws):
         import torch

@@ -5,6 +5,7 @@ Each test names the part of the layer it pins.  A plausible mistake in the
 oracle (a dropped term, a wrong sign or index, a transposed operand, a wrong
 tie rule) fails at least one of them.
 """
+import dataclasses
 import itertools
 import math
 
@@ -727,3 +728,35 @@ def test_round_bf16_is_round_to_nearest_even():
              0x00008000: 0x00000000, 0x00018000: 0x00020000}
     for src, dst in cases.items():
         assert oracle.round_bf16(np.array([src], np.uint32).view(np.float32)).view(np.uint32)[0] == dst, hex(src)
+
+
+def test_bf16_layer_rounds_each_slot_row_then_sums_in_slot_order():
+    """For a bf16-output layer the oracle stores each per-slot expert output
+    row in bf16 and sums the rows in slot order in fp32 before the final bf16
+    cast; for an fp32-output layer the rows stay fp32.  Rebuilt here from the
+    oracle's own accumulators with torch's bf16 conversion and numpy sums."""
+    import torch
+    wl = dataclasses.replace(synth.WORKLOADS["tiny"], T=12, data_seed=24)
+    wts = synth.make_weights(wl)
+    data = synth.make_data(wl)
+    prep = oracle.prepare(wts.w_gate, wts.w_up, wts.w_down, wts.calib_x, wl.alpha)
+    rt = oracle.route(data.x, wl.k, wl.E, w_router=data.w_router)
+
+    def bf16(a):
+        return torch.from_numpy(np.ascontiguousarray(a, np.float32)).to(torch.bfloat16).to(torch.float32).numpy()
+
+    for out_bf16 in (False, True):
+        y, dbg = oracle.moe_tokens(data.x, prep, rt, out_bf16=out_bf16)
+        want = np.zeros_like(y)
+        for t in range(wl.T):
+            for s_ in range(wl.k):
+                e = rt.idx[t, s_]
+                o = oracle.down_epilogue(dbg["acc2"][t, s_], float(dbg["sh"][t, s_]), prep.sw_down[e],
+                                         float(rt.w[t, s_]))
+                if out_bf16:
+                    o = bf16(o)
+                assert np.array_equal(dbg["o"][t, s_], o)
+                want[t] = (want[t] + o).astype(np.float32)
+        if out_bf16:
+            want = bf16(want)
+        assert np.array_equal(y, want)
