@@ -43,7 +43,7 @@ TRAFFIC = {
     ("decode", 32, "tc_ffn_fused_kernel"): 1060.720e6 + 6.530304e6,
 }
 
-FUSED_MAX_ROWS = 512   # T*k at or below which the tensor path runs GEMM1 + requant + GEMM2 as one launch
+FUSED_MAX_ROWS = 512   # the library's default: T*k up to which GEMM1 + requant + GEMM2 are one launch
 
 
 def parse():
@@ -74,6 +74,9 @@ def parse():
                    help="time the expert-parallel layer (experts split over the ranks) instead")
     p.add_argument("--no-prefill", action="store_true",
                    help="skip the extra prefill-layer measurement of the decode run")
+    p.add_argument("--fused-max-rows", type=int, default=-1,
+                   help="rows (T*k) up to which the tensor path runs GEMM1 + requant + GEMM2 as one launch "
+                        "(-1: the library's default)")
     p.add_argument("--no-tensor-peak", action="store_true",
                    help="skip the 8-bit tensor-core rate loop (the tensor-bound roofline then divides by "
                         "2 x the bf16 peak)")
@@ -202,8 +205,8 @@ def algorithmic(wl: synth.Workload, n_active: int, R: int, tensor: bool = False)
     intermediates excluded.  Per GEMM launch: the weights of the active experts
     plus that launch's own inputs and outputs (streaming path: A rows and the
     INT32 accumulators; tensor path: sorted A rows, fp32 h + partial maxima for
-    GEMM1, h codes and fp32 expert outputs for GEMM2; the fused launch of few-row
-    batches: the sum of the two)."""
+    GEMM1, h codes and the per-slot output rows (in the output dtype) for GEMM2;
+    the fused launch: the sum of the two)."""
     in_b = 2 if wl.in_bf16 else 4
     w_bytes = n_active * 3 * wl.d * wl.f
     scales = n_active * (2 * wl.f + wl.d) * 4
@@ -213,7 +216,7 @@ def algorithmic(wl: synth.Workload, n_active: int, R: int, tensor: bool = False)
         gemm1 = n_active * 2 * wl.f * wl.d + R * wl.d + R * wl.f * 4 + R * (wl.f // 64) * 4
     else:
         gemm1 = n_active * 2 * wl.f * wl.d + wl.T * wl.d + R * 2 * wl.f * 4
-    gemm2 = n_active * wl.d * wl.f + R * wl.f + R * wl.d * 4 + n_active * wl.d * 4
+    gemm2 = n_active * wl.d * wl.f + R * wl.f + R * wl.d * in_b + n_active * wl.d * 4   # O rows: output dtype
     ops = 2 * R * 3 * wl.d * wl.f
     # the fused launch (GEMM1 + requantisation + GEMM2): both GEMMs' bytes
     return dict(layer_bytes=layer, gemm1_bytes=gemm1, gemm2_bytes=gemm2, fused_bytes=gemm1 + gemm2,
@@ -394,6 +397,8 @@ def measure(args, wl, world, rank, local, e2e_on=True, wts=None):
     W = M.moe_w8a8_prepare(cfg, wg, wu, wd, wr, ax)
     M.moe_w8a8_set_path(W, {"auto": M.MOE_PATH_AUTO, "stream": M.MOE_PATH_STREAM,
                             "tensor": M.MOE_PATH_TENSOR}[args.path])
+    if getattr(args, "fused_max_rows", -1) >= 0:
+        M.moe_w8a8_set_fused_threshold(W, args.fused_max_rows)
     clip = 0.0
     if getattr(args, "act_clip", 0.0) > 0.0:
         clip = M.moe_w8a8_calibrate_act_clip(W, cal, args.act_clip)
@@ -415,7 +420,8 @@ def measure(args, wl, world, rank, local, e2e_on=True, wts=None):
     counts = np.diff(offs.cpu().numpy())
     n_active, R = int((counts > 0).sum()), int(counts.sum())
     tensor = args.path == "tensor" or (args.path == "auto" and (fp8 or T * wl.k > 32))
-    fused = tensor and T * wl.k <= FUSED_MAX_ROWS
+    fmax = args.fused_max_rows if getattr(args, "fused_max_rows", -1) >= 0 else FUSED_MAX_ROWS
+    fused = tensor and T * wl.k <= fmax
     alg = algorithmic(wl, n_active, R, tensor)
 
     stream = torch.cuda.current_stream(dev)

@@ -118,7 +118,9 @@ typedef struct {
     int8_t* hq;          /* [T*k][f]  INT8 h                                           */
     float* sh;           /* [T*k]     per-row h scales                                 */
     int32_t* acc2;       /* [T*k][d]  down-projection INT32 accumulators               */
-    float* o;            /* [T*k][d]  weighted expert outputs, fp32                    */
+    void* o;             /* [T*k][d]  weighted expert outputs (the per-slot rows the
+                                          combine sums), in the output precision:
+                                          bf16 for MOE_BF16 output, else fp32          */
 } moe_w8a8_debug;
 
 /*
@@ -251,6 +253,16 @@ moe_status moe_w8a8_set_path(moe_w8a8_weights* w, int32_t path);
 
 /* Row count at or below which MOE_PATH_AUTO uses the streaming path. */
 moe_status moe_w8a8_set_stream_threshold(moe_w8a8_weights* w, int32_t max_rows);
+
+/*
+ * Row count (T * k) at or below which the tensor-core path runs GEMM1, the
+ * requantisation of h and GEMM2 as one persistent launch with per-expert
+ * dependencies between its thread blocks (above it: three launches).  The
+ * results are identical either way; max_rows >= 0.  Changing it can change
+ * moe_w8a8_workspace_size (the fused launch keeps a few counters per 128-row
+ * tile in the workspace).
+ */
+moe_status moe_w8a8_set_fused_threshold(moe_w8a8_weights* w, int64_t max_rows);
 
 /*
  * Saturating activation clip (mhpq.cn page s6.4, the third defence against

@@ -115,13 +115,13 @@ def gpu_forward(W, wl: synth.Workload, data: synth.LayerData, debug=True, path=N
                    hq=torch.empty((tk, wl.f), dtype=torch.int8, device=dev),
                    sh=torch.empty(tk, dtype=torch.float32, device=dev),
                    acc2=torch.zeros((tk, wl.d), dtype=torch.int32, device=dev),
-                   o=torch.empty((tk, wl.d), dtype=torch.float32, device=dev))
+                   o=torch.empty((tk, wl.d), dtype=odt, device=dev))   # per-slot rows: output precision
         dbg = {k: v for k, v in dbg.items() if k in fields}
     M.moe_w8a8_forward(W, x, T, bias, logits, y, ws, dbg)
     M.moe_w8a8_check_status(W)
     out = {}
     if dbg:
-        out = {k: v.cpu().numpy() for k, v in dbg.items()}
+        out = {k: (v.float() if v.dtype == torch.bfloat16 else v).cpu().numpy() for k, v in dbg.items()}
     return y.float().cpu().numpy(), out
 
 

@@ -44,3 +44,11 @@ def test_layer_bytes_count_only_active_experts():
     a40 = bench.algorithmic(wl, n_active=40, R=128)
     a41 = bench.algorithmic(wl, n_active=41, R=128)
     assert a41["layer_bytes"] - a40["layer_bytes"] == 3 * 4096 * 1536 + (2 * 1536 + 4096) * 4
+
+
+def test_gemm2_bytes_count_per_slot_rows_in_the_output_dtype():
+    bench, synth = _bench()
+    wl = synth.WORKLOADS["decode"]           # bf16 output: 2-byte per-slot rows
+    a = bench.algorithmic(wl, n_active=56, R=128, tensor=True)
+    # 56 * 4096 * 1536 weights + 128 * 1536 h codes + 128 * 4096 * 2 rows + 56 * 4096 * 4 scales
+    assert a["gemm2_bytes"] == 352_321_536 + 196_608 + 1_048_576 + 917_504

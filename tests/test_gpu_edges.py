@@ -249,3 +249,36 @@ def test_smallest_hidden_and_ffn_sizes(M):
         assert e.value.status == M.MOE_ERR_UNSUPPORTED_SHAPE
     finally:
         M.moe_w8a8_set_path(W, M.MOE_PATH_AUTO)
+
+
+# ----------------------------------------------------------------- the fused expert launch behind the large-batch front end
+
+def test_fused_launch_behind_the_two_kernel_permutation(M):
+    """T k = 2200 > 2048 (warp top-k, histogram and scatter kernels, the scatter
+    clearing the fused launch's counters) with GEMM1, requantisation and GEMM2
+    as one launch; twice in a row, so the second forward relies on the
+    counters being cleared again."""
+    wl = dataclasses.replace(synth.WORKLOADS["tiny"], T=1100, data_seed=74, logits_uniform=True)
+    wts, data, W, prep = layer(wl)
+    M.moe_w8a8_set_fused_threshold(W, 1 << 20)
+    try:
+        for _ in range(2):
+            run(M, wl, W, prep, data, path=M.MOE_PATH_TENSOR, tokens=spread(wl.T, 48))
+    finally:
+        M.moe_w8a8_set_fused_threshold(W, 512)
+
+
+def test_fused_launch_behind_the_certified_router(M, sweep_layer):
+    """The decode layer's shape at T = 2048 with computed bf16 logits (the
+    certified tensor-core router, then the two-kernel permutation) and the
+    fused expert launch over its 8192 rows."""
+    w_router, get = sweep_layer
+    wl = next(p for p in synth.sweep_workloads() if p.T == 2048 and p.zipf_s == 0 and p.alpha == 0.5)
+    W, prep = get(0.5)
+    data = synth.make_data(wl)
+    data.w_router = w_router
+    M.moe_w8a8_set_fused_threshold(W, 1 << 20)
+    try:
+        run(M, wl, W, prep, data, tokens=spread(wl.T, 16), fields=H.DBG_SMALL + ("acc1", "acc2", "o"))
+    finally:
+        M.moe_w8a8_set_fused_threshold(W, 512)

@@ -114,6 +114,8 @@ def compare_fp8(wl, prep, rt, dbg, y, y_ref, odbg, tokens, bias=None):
             # the down epilogue and combine, from the GPU's own h codes and exact sums
             acc2_x = (_dec(prep.wq_down[e]) @ _dec(hq)).astype(np.float32)
             o = ((acc2_x * np.float32(sh)) * prep.sw_down[e]) * np.float32(rt.w[t, s])
+            if wl.in_bf16:       # per-slot rows in the layer's output precision
+                o = _bf16_round(o)
             y_mid[i] = y_mid[i] + o
     if wl.in_bf16:
         y_mid = _bf16_round(y_mid)

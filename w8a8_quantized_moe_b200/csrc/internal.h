@@ -42,6 +42,7 @@ struct moe_w8a8_weights {
     int32_t* status;  // device status word
     uint64_t wait_budget_ns;   // bound on a block's wait for another block's results
     int test_skip_ready;       // testing aid: fused launch withholds this m-tile's ready flag (-1: none)
+    int64_t fused_max_rows;    // tensor path: T*k at or below which GEMM1, requant and GEMM2 are one launch
     // tensor maps of the weights for the tensor-core path (built at prepare)
     CUtensorMap tm_w_gu;
     CUtensorMap tm_w_dn;
@@ -113,9 +114,12 @@ cudaError_t launch_router_logits(const void* x, int in_dtype, const float* wr, i
                                  float* logits, cudaStream_t s);
 cudaError_t launch_topk(const float* logits, const float* bias, int T, int E, int k, int renorm,
                         int32_t* idx, float* wts, float* logits_out, cudaStream_t s);
+// zero_words[0, n_zero): counters a later kernel of the forward starts from
+// zero (the fused expert launch); block 0 of the scatter clears them.
 cudaError_t launch_permute(const int32_t* idx, int T, int k, int E, int cap, int32_t* hist,
                            int32_t* offsets, int32_t* row2ts, int32_t* ts2row, int32_t* meta,
-                           int32_t* active, int32_t* tiles, cudaStream_t s);
+                           int32_t* active, int32_t* tiles, cudaStream_t s, int32_t* zero_words = nullptr,
+                           int n_zero = 0);
 bool route_small_ok(int T, int k);
 cudaError_t launch_route_small(const float* logits, const float* bias, int T, int E, int k,
                                int renorm, int cap, int32_t* idx, float* wts, float* logits_out,
@@ -153,7 +157,7 @@ cudaError_t launch_swiglu_requant(const moe_w8a8_weights* w, const int32_t* acc1
 cudaError_t launch_stream_down(const moe_w8a8_weights* w, int T, const int8_t* hq,
                                const float* sh, const int32_t* row2ts, const float* topk_w,
                                const int32_t* offsets, const int32_t* active, const int32_t* meta,
-                               float* o, int32_t* acc2_dbg, cudaStream_t s);
+                               void* o, int32_t* acc2_dbg, cudaStream_t s);
 // tensor-core path (kernels_tc.cu)
 bool tc_make_weight_maps(moe_w8a8_weights* w);
 // Certified tensor-core router: approximate logits l~ [T][E] from bf16 X (this
@@ -178,7 +182,7 @@ cudaError_t launch_requant(const float* h32, const float* pamax, int f, const in
                            int max_rows, int8_t* hq, float* sh, int fmt, cudaStream_t s);
 cudaError_t launch_tc_gemm2(const moe_w8a8_weights* w, int T, const int8_t* hq, const float* sh,
                             const int32_t* meta, const int32_t* tiles, const int32_t* offsets,
-                            const int32_t* row2ts, const float* topk_w, float* o, int32_t* acc_dbg,
+                            const int32_t* row2ts, const float* topk_w, void* o, int32_t* acc_dbg,
                             cudaStream_t s);
 
 // GEMM1 + requantisation of h + GEMM2 in one persistent launch (few rows per
@@ -186,12 +190,16 @@ cudaError_t launch_tc_gemm2(const moe_w8a8_weights* w, int T, const int8_t* hq, 
 cudaError_t launch_tc_ffn_fused(const moe_w8a8_weights* w, int T, const int8_t* aq, const int32_t* meta,
                                 const int32_t* tiles, const int32_t* offsets, const int32_t* row2ts,
                                 const float* sx, const float* topk_w, float* h32, float* pamax, int8_t* hq,
-                                float* sh, float* o, int32_t* acc1_dbg, int32_t* acc2_dbg, int32_t* sync_words,
+                                float* sh, void* o, int32_t* acc1_dbg, int32_t* acc2_dbg, int32_t* sync_words,
                                 cudaStream_t s);
 inline size_t fused_sync_words(size_t max_mtiles) { return 3 * max_mtiles + 3; }
-constexpr int kFusedMaxRows = 512;   // T*k at or below which the tensor path runs the fused launch
+constexpr int kFusedMaxRows = 512;   // default: T*k at or below which the tensor path runs the fused launch
 
-cudaError_t launch_combine(const float* o, const int32_t* ts2row, int T, int k, int d,
+// The per-slot rows o (sorted, [rows][d]) are fp32, or bf16 when o_bf16; the
+// expert FFN writes them in the layer's output precision.
+cudaError_t launch_combine(const void* o, int o_bf16, const int32_t* ts2row, int T, int k, int d,
                            int out_dtype, void* y, cudaStream_t s);
+// Bytes of one per-slot output value: the layer's output precision.
+inline size_t o_bytes(const moe_w8a8_config& c) { return c.out_dtype == MOE_BF16 ? 2 : 4; }
 
 }  // namespace moe

@@ -686,9 +686,12 @@ __global__ void __launch_bounds__(kPermThreads) perm_scatter_kernel(
     const int32_t* __restrict__ idx, int n, int E, int cap, int nblk,
     const int32_t* __restrict__ hist, int32_t* __restrict__ offsets, int32_t* __restrict__ row2ts,
     int32_t* __restrict__ ts2row, int32_t* __restrict__ meta, int32_t* __restrict__ active,
-    int32_t* __restrict__ tiles) {
+    int32_t* __restrict__ tiles, int32_t* __restrict__ zero_words, int n_zero) {
     pdl_wait();
     pdl_trigger();
+    // counters a later kernel of this forward starts from zero (the fused expert launch)
+    if (blockIdx.x == 0)
+        for (int i = threadIdx.x; i < n_zero; i += blockDim.x) zero_words[i] = 0;
 
     __shared__ int pre[kMaxE], off[kMaxE + 1], running[kMaxE], kept[kMaxE];
     __shared__ int wcnt[kPermThreads / 32][kMaxE];
@@ -958,13 +961,13 @@ cudaError_t launch_topk(const float* logits, const float* bias, int T, int E, in
 
 cudaError_t launch_permute(const int32_t* idx, int T, int k, int E, int cap, int32_t* hist,
                            int32_t* offsets, int32_t* row2ts, int32_t* ts2row, int32_t* meta,
-                           int32_t* active, int32_t* tiles, cudaStream_t s) {
+                           int32_t* active, int32_t* tiles, cudaStream_t s, int32_t* zero_words, int n_zero) {
     const int n = T * k;
     const int nblk = (n + kPermChunk - 1) / kPermChunk;
     cudaError_t err = launch_pdl(perm_hist_kernel, dim3(nblk), dim3(256), 0, s, idx, n, E, hist);
     if (err != cudaSuccess) return err;
     return launch_pdl(perm_scatter_kernel, dim3(nblk), dim3(kPermThreads), 0, s, idx, n, E, cap, nblk, hist,
-                      offsets, row2ts, ts2row, meta, active, tiles);
+                      offsets, row2ts, ts2row, meta, active, tiles, zero_words, n_zero);
 }
 
 bool route_small_ok(int T, int k) { return (int64_t)T * k <= kRouteSmallMax; }

@@ -184,7 +184,7 @@ __global__ void __launch_bounds__(kStThreads) stream_down_kernel(
     const float* __restrict__ sh, const int32_t* __restrict__ row2ts,
     const float* __restrict__ topk_w, const float* __restrict__ sw_dn,
     const int32_t* __restrict__ offsets, const int32_t* __restrict__ active,
-    const int32_t* __restrict__ meta, float* __restrict__ o, int32_t* __restrict__ acc2_dbg) {    pdl_wait();
+    const int32_t* __restrict__ meta, void* __restrict__ o, int o_bf16, int32_t* __restrict__ acc2_dbg) {    pdl_wait();
     pdl_trigger();
 
     extern __shared__ __align__(16) int8_t As[];   // [kStRows][f]
@@ -217,7 +217,10 @@ __global__ void __launch_bounds__(kStThreads) stream_down_kernel(
                         const float v = __fmul_rn(__fmul_rn(__fmul_rn(__int2float_rn(acc[r][c]), sh[row]),
                                                             sw_dn[(int64_t)e * d + n]),
                                                   topk_w[row2ts[row]]);
-                        o[(int64_t)row * d + n] = v;
+                        if (o_bf16)
+                            reinterpret_cast<uint16_t*>(o)[(int64_t)row * d + n] = f32_to_bf16_bits(v);
+                        else
+                            reinterpret_cast<float*>(o)[(int64_t)row * d + n] = v;
                         if (acc2_dbg) acc2_dbg[(int64_t)row * d + n] = acc[r][c];
                     }
                 }
@@ -227,8 +230,10 @@ __global__ void __launch_bounds__(kStThreads) stream_down_kernel(
 }
 
 // Un-sort + weighted sum: y[t] = ((0 + o_slot0) + o_slot1) + ... over the kept
-// slots, in slot order, then cast to the output dtype.
-__global__ void combine_kernel(const float* __restrict__ o, const int32_t* __restrict__ ts2row,
+// slots, in slot order, then cast to the output dtype.  O16: the per-slot rows
+// are bf16 (bf16-output layers), else fp32.
+template <bool O16>
+__global__ void combine_kernel(const void* __restrict__ o, const int32_t* __restrict__ ts2row,
                                int k, int d, int out_dtype, void* __restrict__ y) {    pdl_wait();
     pdl_trigger();
 
@@ -239,7 +244,14 @@ __global__ void combine_kernel(const float* __restrict__ o, const int32_t* __res
     for (int s = 0; s < k; ++s) {
         const int row = ts2row[(int64_t)t * k + s];
         if (row < 0) continue;
-        const float4 v = reinterpret_cast<const float4*>(o + (int64_t)row * d)[n4];
+        float4 v;
+        if (O16) {
+            const uint2 b = reinterpret_cast<const uint2*>(reinterpret_cast<const uint16_t*>(o) + (int64_t)row * d)[n4];
+            v = make_float4(__uint_as_float(b.x << 16), __uint_as_float(b.x & 0xFFFF0000u),
+                            __uint_as_float(b.y << 16), __uint_as_float(b.y & 0xFFFF0000u));
+        } else {
+            v = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(o) + (int64_t)row * d)[n4];
+        }
         acc.x = __fadd_rn(acc.x, v.x);
         acc.y = __fadd_rn(acc.y, v.y);
         acc.z = __fadd_rn(acc.z, v.z);
@@ -289,7 +301,7 @@ cudaError_t launch_swiglu_requant(const moe_w8a8_weights* w, const int32_t* acc1
 
 cudaError_t launch_stream_down(const moe_w8a8_weights* w, int T, const int8_t* hq, const float* sh,
                                const int32_t* row2ts, const float* topk_w, const int32_t* offsets,
-                               const int32_t* active, const int32_t* meta, float* o,
+                               const int32_t* active, const int32_t* meta, void* o,
                                int32_t* acc2_dbg, cudaStream_t s) {
     const int d = w->cfg.d, f = w->cfg.f;
     const size_t smem = (size_t)kStRows * f;
@@ -299,13 +311,15 @@ cudaError_t launch_stream_down(const moe_w8a8_weights* w, int T, const int8_t* h
     cudaError_t e = smem_attr_once(stream_down_kernel, (size_t)kStRows * kStMaxK, attr);
     if (e != cudaSuccess) return e;
     return launch_pdl(stream_down_kernel, dim3(grid), dim3(kStThreads), smem, s, w->w_dn, d, f, hq, sh,
-                      row2ts, topk_w, w->sw_dn, offsets, active, meta, o, acc2_dbg);
+                      row2ts, topk_w, w->sw_dn, offsets, active, meta, o, (int)(w->cfg.out_dtype == MOE_BF16),
+                      acc2_dbg);
 }
 
-cudaError_t launch_combine(const float* o, const int32_t* ts2row, int T, int k, int d,
+cudaError_t launch_combine(const void* o, int o_bf16, const int32_t* ts2row, int T, int k, int d,
                            int out_dtype, void* y, cudaStream_t s) {
     dim3 grid(T, (d / 4 + 255) / 256);
-    return launch_pdl(combine_kernel, grid, dim3(256), 0, s, o, ts2row, k, d, out_dtype, y);
+    if (o_bf16) return launch_pdl(combine_kernel<true>, grid, dim3(256), 0, s, o, ts2row, k, d, out_dtype, y);
+    return launch_pdl(combine_kernel<false>, grid, dim3(256), 0, s, o, ts2row, k, d, out_dtype, y);
 }
 
 }  // namespace moe

@@ -84,7 +84,8 @@ struct TcParams {
     const float* sh;          // GEMM2: per-row h scale
     float* h32;               // GEMM1: h [rows][f]
     float* pamax;             // GEMM1: per-row partial max [rows][f/64]
-    float* o;                 // GEMM2: [rows][d]
+    void* o;                  // GEMM2: [rows][d], fp32 or (o_bf16) bf16
+    int o_bf16;               // GEMM2: per-slot rows in bf16 (bf16-output layers)
     int32_t* acc_dbg;         // optional raw accumulators (canonical channel order)
     int32_t* status;
 };
@@ -263,6 +264,34 @@ __device__ __forceinline__ void store_rows32(float* stage, const uint32_t (&v)[3
     }
 }
 
+// Store a warp's 32 rows x 32 values as bf16 (lane l holds row l's fp32
+// values v[0..31], rounded to nearest even here) to rows gbase + l*ld (only
+// the first nvalid rows): one pass through the same 2 KB buffer, 64 bytes per
+// row in four 16-byte chunks swizzled by (row / 2) mod 4, so that the
+// shared-memory writes and reads are conflict-free; four lanes write one
+// row's 64 contiguous bytes.
+__device__ __forceinline__ void store_rows32_bf16(float* stage, const uint32_t (&v)[32], uint16_t* gbase,
+                                                  int64_t ld, int nvalid, int lane) {
+    uint4* st4 = reinterpret_cast<uint4*>(stage);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        uint32_t w[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+            w[q] = (uint32_t)f32_to_bf16_bits(__uint_as_float(v[8 * j + 2 * q])) |
+                   ((uint32_t)f32_to_bf16_bits(__uint_as_float(v[8 * j + 2 * q + 1])) << 16);
+        st4[lane * 4 + (j ^ ((lane >> 1) & 3))] = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+    __syncwarp();
+#pragma unroll
+    for (int it = 0; it < 4; ++it) {
+        const int r = it * 8 + (lane >> 2), c = lane & 3;
+        const uint4 q = st4[r * 4 + (c ^ ((r >> 1) & 3))];
+        if (r < nvalid) reinterpret_cast<uint4*>(gbase + (int64_t)r * ld)[c] = q;
+    }
+    __syncwarp();
+}
+
 // GEMM1 tile: columns 0..127 of the accumulator are gate channels
 // nt*128 + c, columns 128..255 the matching up channels.  Each warp owns 32
 // rows (its TMEM lane quarter) and 64 of the 128 h columns.
@@ -356,7 +385,11 @@ __device__ __forceinline__ void epilogue_down(const TcParams& p, uint32_t taddr,
                 a[j + q] = __float_as_uint(
                     __fmul_rn(__fmul_rn(__fmul_rn(acc_value<FMT>(a[j + q]), shr), sv[q]), wr));
         }
-        store_rows32(stage, a, p.o + (int64_t)wrow0 * d + ch0, d, nvalid, lane);
+        if (p.o_bf16)
+            store_rows32_bf16(stage, a, reinterpret_cast<uint16_t*>(p.o) + (int64_t)wrow0 * d + ch0, d, nvalid,
+                              lane);
+        else
+            store_rows32(stage, a, reinterpret_cast<float*>(p.o) + (int64_t)wrow0 * d + ch0, d, nvalid, lane);
     }
 }
 
@@ -1214,7 +1247,7 @@ cudaError_t launch_fused_fmt(const CUtensorMap& a1, const CUtensorMap& b1, const
 cudaError_t launch_tc_ffn_fused(const moe_w8a8_weights* w, int T, const int8_t* aq, const int32_t* meta,
                                 const int32_t* tiles, const int32_t* offsets, const int32_t* row2ts,
                                 const float* sx, const float* topk_w, float* h32, float* pamax, int8_t* hq,
-                                float* sh, float* o, int32_t* acc1_dbg, int32_t* acc2_dbg, int32_t* sync_words,
+                                float* sh, void* o, int32_t* acc1_dbg, int32_t* acc2_dbg, int32_t* sync_words,
                                 cudaStream_t s) {
     const moe_w8a8_config& c = w->cfg;
     const int rows = T * c.top_k;
@@ -1246,6 +1279,7 @@ cudaError_t launch_tc_ffn_fused(const moe_w8a8_weights* w, int T, const int8_t* 
     p2.sw0 = w->sw_dn;
     p2.sh = sh;
     p2.o = o;
+    p2.o_bf16 = c.out_dtype == MOE_BF16;
     p2.acc_dbg = acc2_dbg;
     const int max_mt = (rows + BM - 1) / BM + c.n_experts;
     const FusedExtra fx{sync_words, sync_words + max_mt, sync_words + 2 * max_mt, sync_words + 3 * max_mt,
@@ -1328,7 +1362,7 @@ cudaError_t launch_tc_gemm1(const moe_w8a8_weights* w, int T, const int8_t* aq, 
 
 cudaError_t launch_tc_gemm2(const moe_w8a8_weights* w, int T, const int8_t* hq, const float* sh,
                             const int32_t* meta, const int32_t* tiles, const int32_t* offsets,
-                            const int32_t* row2ts, const float* topk_w, float* o, int32_t* acc_dbg,
+                            const int32_t* row2ts, const float* topk_w, void* o, int32_t* acc_dbg,
                             cudaStream_t s) {
     const moe_w8a8_config& c = w->cfg;
     CUtensorMap ta;
@@ -1348,6 +1382,7 @@ cudaError_t launch_tc_gemm2(const moe_w8a8_weights* w, int T, const int8_t* hq, 
     p.sw0 = w->sw_dn;
     p.sh = sh;
     p.o = o;
+    p.o_bf16 = c.out_dtype == MOE_BF16;
     p.acc_dbg = acc_dbg;
     p.status = w->status;
     const int max_mt = (rows + BM - 1) / BM + c.n_experts;

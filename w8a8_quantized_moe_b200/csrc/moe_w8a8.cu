@@ -65,8 +65,8 @@ bool path_ok(const moe_w8a8_weights* w, int T) {
 }
 
 // The tensor path runs GEMM1, the requantisation of h and GEMM2 as one
-// launch when there are few rows per expert (and the routing front end is the
-// one-block kernel, which clears the launch's counters).
+// launch up to the handle's row threshold (the routing front end, the
+// one-block kernel or the scatter kernel, clears the launch's counters).
 // The certified tensor-core router serves large batches with computed logits
 // (the one-block routing front end keeps the FMA router).
 bool router_tc_ok(const moe_w8a8_weights* w, int T) {
@@ -74,8 +74,7 @@ bool router_tc_ok(const moe_w8a8_weights* w, int T) {
 }
 
 bool fused_ok(const moe_w8a8_weights* w, int T) {
-    const int64_t tk = (int64_t)T * w->cfg.top_k;
-    return tk <= kFusedMaxRows && route_small_ok(T, w->cfg.top_k);
+    return (int64_t)T * w->cfg.top_k <= w->fused_max_rows;
 }
 
 void prof_free(moe_w8a8_weights* w) {
@@ -149,7 +148,7 @@ WsLayout ws_layout(const moe_w8a8_weights* w, int T, WsPart part) {
     L.acc1 = take(ex && stream ? tk * 2 * f * 4 : 0);
     L.hq = take(ex ? tk * f : 0);
     L.sh = take(ex ? tk * 4 : 0);
-    L.o = take(ex ? tk * d * 4 : 0);
+    L.o = take(ex ? tk * d * o_bytes(c) : 0);
     L.h32 = take(ex && !stream ? tk * f * 4 : 0);
     L.pamax = take(ex && !stream ? tk * (f / 64) * 4 : 0);
     const bool fused = ex && !stream && fused_ok(w, T);
@@ -282,6 +281,7 @@ moe_status prepare_impl(const moe_w8a8_config* cfg, int e_first, int n_local, co
     w->stream_max_rows = 32;   // measured crossover: streaming wins up to T*k = 32 rows
     w->wait_budget_ns = 2000000000ull;
     w->test_skip_ready = -1;
+    w->fused_max_rows = kFusedMaxRows;
     if (cudaGetDevice(&w->device) != cudaSuccess ||
         cudaDeviceGetAttribute(&w->num_sms, cudaDevAttrMultiProcessorCount, w->device) != cudaSuccess) {
         free_handle(w);
@@ -438,19 +438,20 @@ moe_status route_stage(Run& r, const void* x, int T, const float* bias, const fl
     } else {
         r.empty_stage(MOE_STAGE_ROUTER);
     }
+    const bool fused = path == MOE_PATH_TENSOR && L.fused_words > 0;
+    int32_t* zero_words = fused ? r.at<int32_t>(L.fused_sync) : nullptr;
+    const int n_zero = fused ? L.fused_words : 0;
     if (certified) {
         r.mark(MOE_STAGE_PERMUTE, 0);
         CUDA_TRY(launch_permute(idx, T, k, E, capacity_of(c, T), r.at<int32_t>(L.hist), offsets, row2ts, ts2row,
-                                meta, active, tiles, s));
+                                meta, active, tiles, s, zero_words, n_zero));
         r.mark(MOE_STAGE_PERMUTE, 1);
         r.launches += 2;
     } else if (route_small_ok(T, k)) {
         // top-k, histogram, scan and scatter in one block
         r.mark(MOE_STAGE_TOPK, 0);
-        const bool fused = path == MOE_PATH_TENSOR && L.fused_words > 0;
         CUDA_TRY(launch_route_small(lsrc, bias, T, E, k, c.renormalize, capacity_of(c, T), idx, wts, dbg_logits,
-                                    offsets, row2ts, ts2row, meta, active, tiles,
-                                    fused ? r.at<int32_t>(L.fused_sync) : nullptr, fused ? L.fused_words : 0, s));
+                                    offsets, row2ts, ts2row, meta, active, tiles, zero_words, n_zero, s));
         r.mark(MOE_STAGE_TOPK, 1);
         r.empty_stage(MOE_STAGE_PERMUTE);
         ++r.launches;
@@ -461,7 +462,7 @@ moe_status route_stage(Run& r, const void* x, int T, const float* bias, const fl
         ++r.launches;
         r.mark(MOE_STAGE_PERMUTE, 0);
         CUDA_TRY(launch_permute(idx, T, k, E, capacity_of(c, T), r.at<int32_t>(L.hist), offsets, row2ts, ts2row,
-                                meta, active, tiles, s));
+                                meta, active, tiles, s, zero_words, n_zero));
         r.mark(MOE_STAGE_PERMUTE, 1);
         r.launches += 2;
     }
@@ -506,7 +507,7 @@ moe_status expert_stage(Run& r, int T, int path) {
     float* sx = r.at<float>(L.sx);
     int8_t* hq = r.at<int8_t>(L.hq);
     float* sh = r.at<float>(L.sh);
-    float* o = r.at<float>(L.o);
+    void* o = r.at<void>(L.o);
     if (path == MOE_PATH_STREAM) {
         int32_t* acc1 = r.at<int32_t>(L.acc1);
         r.mark(MOE_STAGE_GEMM1, 0);
@@ -573,7 +574,7 @@ moe_status debug_stage(Run& r, int T, int k, int E, bool token_codes, bool exper
     if (expert_bufs) {
         CUDA_TRY(cp(dbg->hq, L.hq, tk * f));
         CUDA_TRY(cp(dbg->sh, L.sh, tk * 4));
-        CUDA_TRY(cp(dbg->o, L.o, tk * d * 4));
+        CUDA_TRY(cp(dbg->o, L.o, tk * d * o_bytes(r.w->cfg)));
     }
     return MOE_OK;
 }
@@ -596,7 +597,8 @@ moe_status forward_impl(const moe_w8a8_weights* w, const void* x, int T, const f
         MOE_TRY(quant_stage(r, x, T, r.at<int8_t>(r.L.aq), c.d, false, c.expert_format));
     MOE_TRY(expert_stage(r, T, path));
     r.mark(MOE_STAGE_COMBINE, 0);
-    CUDA_TRY(launch_combine(r.at<float>(r.L.o), r.at<int32_t>(r.L.ts2row), T, c.top_k, c.d, c.out_dtype, y, s));
+    CUDA_TRY(launch_combine(r.at<void>(r.L.o), c.out_dtype == MOE_BF16, r.at<int32_t>(r.L.ts2row), T, c.top_k, c.d,
+                            c.out_dtype, y, s));
     r.mark(MOE_STAGE_COMBINE, 1);
     ++r.launches;
     moe_w8a8_weights* mw = const_cast<moe_w8a8_weights*>(w);
@@ -695,6 +697,12 @@ moe_status moe_w8a8_set_path(moe_w8a8_weights* w, int32_t path) {
 moe_status moe_w8a8_set_stream_threshold(moe_w8a8_weights* w, int32_t max_rows) {
     if (!w || max_rows < 0) return MOE_ERR_INVALID_ARG;
     w->stream_max_rows = max_rows;
+    return MOE_OK;
+}
+
+moe_status moe_w8a8_set_fused_threshold(moe_w8a8_weights* w, int64_t max_rows) {
+    if (!w || max_rows < 0) return MOE_ERR_INVALID_ARG;
+    w->fused_max_rows = max_rows;
     return MOE_OK;
 }
 
@@ -927,7 +935,7 @@ moe_status moe_w8a8_ep_experts(const moe_w8a8_weights* w, const void* recv, int3
     r.launches += 4;
     MOE_TRY(expert_stage(r, R, path));
     // un-sort: O of received row r to o_rows[r] (k = 1)
-    CUDA_TRY(launch_combine(r.at<float>(L.o), ts2row, R, 1, d, MOE_F32, o_rows, s));
+    CUDA_TRY(launch_combine(r.at<void>(L.o), v.cfg.out_dtype == MOE_BF16, ts2row, R, 1, d, MOE_F32, o_rows, s));
     ++r.launches;
     MOE_TRY(debug_stage(r, R, 1, v.cfg.n_experts, false, true));
     const_cast<moe_w8a8_weights*>(w)->last_launches = r.launches;
@@ -945,7 +953,7 @@ moe_status moe_w8a8_ep_combine(const moe_w8a8_weights* w, const float* o_rows, i
     const WsLayout L = ws_layout(w, T, WS_ROUTE);
     if (workspace_bytes < L.total) return MOE_ERR_WORKSPACE_TOO_SMALL;
     const int32_t* ts2row = (const int32_t*)((const char*)workspace + L.ts2row);
-    CUDA_TRY(launch_combine(o_rows, ts2row, T, c.top_k, c.d, c.out_dtype, y, (cudaStream_t)stream));
+    CUDA_TRY(launch_combine(o_rows, 0, ts2row, T, c.top_k, c.d, c.out_dtype, y, (cudaStream_t)stream));
     const_cast<moe_w8a8_weights*>(w)->last_launches = 1;
     return MOE_OK;
 }
