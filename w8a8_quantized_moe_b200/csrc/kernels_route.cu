@@ -773,8 +773,9 @@ __global__ void __launch_bounds__(kRouteSmallThreads) route_small_kernel(
 // ---------------------------------------------------------------------------
 // Smoothed per-token quantisation: x' = fp32(x * inv_s); sx = amax/127;
 // q = rint(x'/sx) clamped to +-127.  One block per token; each thread owns
-// groups of 8 channels.  Writes xq[t] and, when aq is given, the copy of the
-// token's codes into every kept (t, slot) row of the expert-sorted matrix.
+// groups of 8 channels.  Writes xq[t] (unless xq is null) and, when aq is
+// given, the copy of the token's codes into every kept (t, slot) row of the
+// expert-sorted matrix.
 // ---------------------------------------------------------------------------
 // One block of 128 threads per token: thread i owns channel groups i, i + 128,
 // ... (8 channels each); all of a thread's loads are issued before the block
@@ -836,7 +837,7 @@ __global__ void __launch_bounds__(kSqThreads) smooth_quant_kernel(
 #pragma unroll
         for (int c = 0; c < 8; ++c) q[c] = s > 0.0f ? (int)fmt_code<FMT>(v[gi][c], s, rs) : 0;
         packed[gi] = make_uint2(pack4(q[0], q[1], q[2], q[3]), pack4(q[4], q[5], q[6], q[7]));
-        *reinterpret_cast<uint2*>(xq + (int64_t)t * d + g * 8) = packed[gi];
+        if (xq) *reinterpret_cast<uint2*>(xq + (int64_t)t * d + g * 8) = packed[gi];
     }
     pdl_wait();   // the routing of this forward is complete from here on
     if (!aq) return;

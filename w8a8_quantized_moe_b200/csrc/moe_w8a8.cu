@@ -476,9 +476,12 @@ moe_status quant_stage(Run& r, const void* x, int T, int8_t* aq, int64_t aq_ld, 
     const moe_w8a8_weights* w = r.w;
     const moe_w8a8_config& c = w->cfg;
     const WsLayout& L = r.L;
+    // the per-token codes are read by the streaming path and the debug copy;
+    // the tensor path and the expert-parallel send rows use the sorted copies
+    const bool need_xq = !aq || (r.dbg && r.dbg->xq);
     r.mark(MOE_STAGE_QUANT, 0);
     CUDA_TRY(launch_smooth_quant(x, c.in_dtype, w->inv_s, w->act_clip, T, c.d, c.top_k, r.at<int32_t>(L.ts2row),
-                                 r.at<int8_t>(L.xq), r.at<float>(L.sx), aq, aq_ld,
+                                 need_xq ? r.at<int8_t>(L.xq) : nullptr, r.at<float>(L.sx), aq, aq_ld,
                                  trailer ? r.at<float>(L.topk_w) : nullptr,
                                  trailer ? r.at<int32_t>(L.topk_idx) : nullptr, fmt, r.s));
     r.mark(MOE_STAGE_QUANT, 1);
