@@ -74,6 +74,8 @@ def parse():
                    help="time the expert-parallel layer (experts split over the ranks) instead")
     p.add_argument("--no-prefill", action="store_true",
                    help="skip the extra prefill-layer measurement of the decode run")
+    p.add_argument("--no-large", action="store_true",
+                   help="skip the extra large-sparse-layer measurement of the decode run")
     p.add_argument("--fused-max-rows", type=int, default=-1,
                    help="rows (T*k) up to which the tensor path runs GEMM1 + requant + GEMM2 as one launch "
                         "(-1: the library's default)")
@@ -654,6 +656,18 @@ def run_ours(args, world, rank, local):
         del PW
         torch.cuda.empty_cache()
         extra = {"metric": "prefill layer tokens/s (T=16384)", "unit": "tokens/s", **pres}
+    large = None
+    if args.workload == "decode" and not args.no_large:
+        lw = replica_workload(synth.WORKLOADS["large"], rank)
+        # its fp32 weights (51.5 GB) are generated and uploaded expert by expert, untimed
+        lres, _, LW = measure(args, lw, world, rank, local, e2e_on=False)
+        del LW
+        torch.cuda.empty_cache()
+        large = {"metric": "large sparse layer tokens/s (T=4096, d=8192, E=256, top-8, capacity 1.25)",
+                 "unit": "tokens/s", **lres,
+                 "cpu_baseline": {"value": None, "unit": "tokens/s", "cores": 0, "kind": "oracle",
+                                  "sample": "not run for this layer: its smoothing statistic needs all 256 "
+                                            "experts' fp32 weights on the host"}}
 
     if rank != 0:
         return
@@ -695,6 +709,8 @@ def run_ours(args, world, rank, local):
             "clocks": res["clocks"], "cpu_baseline": cpu}
     if extra is not None:
         line["prefill"] = extra
+    if large is not None:
+        line["large"] = large
     if args.tensor_peak:
         line["tensor_peak"] = args.tensor_peak
     print(json.dumps(line), flush=True)
