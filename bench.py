@@ -79,6 +79,9 @@ def parse():
     p.add_argument("--fused-max-rows", type=int, default=-1,
                    help="rows (T*k) up to which the tensor path runs GEMM1 + requant + GEMM2 as one launch "
                         "(-1: the library's default)")
+    p.add_argument("--cta-pairs", type=int, default=-1, choices=[-1, 0, 1, 2],
+                   help="separate GEMM launches on SM pairs: 0 never, 1 always, 2 by rows per expert "
+                        "(-1: the library's default)")
     p.add_argument("--no-tensor-peak", action="store_true",
                    help="skip the 8-bit tensor-core rate loop (the tensor-bound roofline then divides by "
                         "2 x the bf16 peak)")
@@ -401,6 +404,8 @@ def measure(args, wl, world, rank, local, e2e_on=True, wts=None):
                             "tensor": M.MOE_PATH_TENSOR}[args.path])
     if getattr(args, "fused_max_rows", -1) >= 0:
         M.moe_w8a8_set_fused_threshold(W, args.fused_max_rows)
+    if getattr(args, "cta_pairs", -1) >= 0:
+        M.moe_w8a8_set_cta_pairs(W, args.cta_pairs)
     clip = 0.0
     if getattr(args, "act_clip", 0.0) > 0.0:
         clip = M.moe_w8a8_calibrate_act_clip(W, cal, args.act_clip)

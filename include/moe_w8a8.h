@@ -265,6 +265,17 @@ moe_status moe_w8a8_set_stream_threshold(moe_w8a8_weights* w, int32_t max_rows);
 moe_status moe_w8a8_set_fused_threshold(moe_w8a8_weights* w, int64_t max_rows);
 
 /*
+ * Whether the tensor-core path's separate GEMM launches run on pairs of SMs:
+ * a cluster of two thread blocks computes 256-row tiles with one
+ * tcgen05.mma.cta_group::2 per K slice, each SM loading half of the tile's
+ * weight columns (less operand traffic per MMA, deeper pipelines) at the cost
+ * of MMA work on the unused rows of each expert's last 256-row tile.
+ * mode 0: never; 1: always; 2 (default): when T * k >= 256 * E, i.e. the rows
+ * per expert fill such tiles on average.  The results are identical.
+ */
+moe_status moe_w8a8_set_cta_pairs(moe_w8a8_weights* w, int32_t mode);
+
+/*
  * Saturating activation clip (mhpq.cn page s6.4, the third defence against
  * activation outliers: cut values at a threshold instead of stretching the
  * scale to the maximum; gtnt.cn page s3.2: the threshold is a percentile of

@@ -282,3 +282,34 @@ def test_fused_launch_behind_the_certified_router(M, sweep_layer):
         run(M, wl, W, prep, data, tokens=spread(wl.T, 16), fields=H.DBG_SMALL + ("acc1", "acc2", "o"))
     finally:
         M.moe_w8a8_set_fused_threshold(W, 512)
+
+
+# ----------------------------------------------------------------- GEMMs on SM pairs (cta_group::2)
+
+@pytest.mark.parametrize("T", [1000, 300])
+def test_pair_gemms_tiny_layer(M, T):
+    """The separate GEMM launches on SM pairs (256-row tiles, one 256-row MMA
+    per K slice over two SMs): T = 1000 gives about 250 rows per expert, so
+    pair tiles end half empty, T = 300 fewer rows than one pair tile per
+    expert.  Accumulators, codes and outputs bit for bit."""
+    wl = dataclasses.replace(synth.WORKLOADS["tiny"], T=T, data_seed=500 + T)
+    wts, data, W, prep = layer(wl)
+    M.moe_w8a8_set_cta_pairs(W, 1)
+    M.moe_w8a8_set_fused_threshold(W, 0)
+    run(M, wl, W, prep, data, path=M.MOE_PATH_TENSOR, tokens=spread(wl.T, 64))
+
+
+def test_pair_gemms_decode_shape_certified_router(M, sweep_layer):
+    """The decode layer's shape at T = 4096 (the certified router; 256 rows per
+    expert on average) with the GEMMs on SM pairs."""
+    w_router, get = sweep_layer
+    base = next(p for p in synth.sweep_workloads() if p.T == 2048 and p.zipf_s == 0 and p.alpha == 0.5)
+    wl = dataclasses.replace(base, T=4096, data_seed=77)
+    W, prep = get(0.5)
+    data = synth.make_data(wl)
+    data.w_router = w_router
+    M.moe_w8a8_set_cta_pairs(W, 1)
+    try:
+        run(M, wl, W, prep, data, tokens=spread(wl.T, 16), fields=H.DBG_SMALL + ("acc1", "acc2", "o"))
+    finally:
+        M.moe_w8a8_set_cta_pairs(W, 2)

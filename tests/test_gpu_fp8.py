@@ -184,3 +184,14 @@ def test_fp8_refuses_the_streaming_path(M, decode_fp8):
         assert e.value.status == M.MOE_ERR_UNSUPPORTED_SHAPE
     finally:
         M.moe_w8a8_set_path(W, M.MOE_PATH_AUTO)
+
+
+def test_fp8_pair_gemms(M):
+    """FP8 experts with the separate GEMM launches on SM pairs
+    (tcgen05.mma.cta_group::2.kind::f8f6f4)."""
+    wl = dataclasses.replace(synth.WORKLOADS["tiny"], T=600, data_seed=610)
+    wts = synth.make_weights(wl)
+    W = H.gpu_prepare(wl, wts, fmt=M.MOE_FMT_E4M3)
+    M.moe_w8a8_set_cta_pairs(W, 1)
+    M.moe_w8a8_set_fused_threshold(W, 0)
+    run_fp8(M, wl, wts=wts, W=W)

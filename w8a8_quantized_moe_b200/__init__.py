@@ -45,7 +45,7 @@ EXPORTS = (
     "moe_w8a8_ep_dispatch_workspace_size", "moe_w8a8_ep_experts_workspace_size",
     "moe_w8a8_ep_dispatch", "moe_w8a8_ep_experts", "moe_w8a8_ep_combine",
     "moe_w8a8_tensor_peak_loop", "moe_w8a8_set_wait_budget", "moe_w8a8_test_withhold_release",
-    "moe_w8a8_set_fused_threshold",
+    "moe_w8a8_set_fused_threshold", "moe_w8a8_set_cta_pairs",
 )
 
 MOE_NOALLOC_SCRATCH_BYTES = 8 << 20
@@ -122,6 +122,7 @@ def lib():
             "moe_w8a8_tensor_peak_loop": ([i32, i64, ctypes.POINTER(ctypes.c_double), vp], i32),
             "moe_w8a8_set_wait_budget": ([vp, i64], i32),
             "moe_w8a8_set_fused_threshold": ([vp, i64], i32),
+            "moe_w8a8_set_cta_pairs": ([vp, i32], i32),
             "moe_w8a8_test_withhold_release": ([vp, i32], i32),
         }
         for name, (args, res) in sig.items():
@@ -309,6 +310,10 @@ def moe_w8a8_set_stream_threshold(w: Weights, max_rows: int):
 
 def moe_w8a8_set_fused_threshold(w: Weights, max_rows: int):
     _check(lib().moe_w8a8_set_fused_threshold(w.handle, int(max_rows)), "moe_w8a8_set_fused_threshold")
+
+
+def moe_w8a8_set_cta_pairs(w: Weights, mode: int):
+    _check(lib().moe_w8a8_set_cta_pairs(w.handle, int(mode)), "moe_w8a8_set_cta_pairs")
 
 
 def moe_w8a8_set_act_clip(w: Weights, clip: float):

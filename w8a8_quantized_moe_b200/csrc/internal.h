@@ -46,6 +46,9 @@ struct moe_w8a8_weights {
     // tensor maps of the weights for the tensor-core path (built at prepare)
     CUtensorMap tm_w_gu;
     CUtensorMap tm_w_dn;
+    CUtensorMap tm_w_gu_half;  // the same weights in 128-row boxes (one CTA of a pair loads half a tile)
+    CUtensorMap tm_w_dn_half;
+    int cta_pairs;             // separate GEMM launches on SM pairs: 0 never, 1 always, 2 by rows per expert
     bool tmaps_ok;
     CUtensorMap tm_rt_hi;
     CUtensorMap tm_rt_lo;
@@ -67,7 +70,7 @@ struct WsLayout {
     size_t x_stage, y_stage, logits_stage, bias_stage;   // forward_host staging
     size_t logits, topk_idx, topk_w;
     size_t logits_sel;           // certified router: exact-or--inf logits [T][E]
-    size_t hist, offsets, meta, active, tiles;
+    size_t hist, offsets, meta, active, tiles, pairs;
     size_t row2ts, ts2row;
     size_t xq, sx, aq;
     size_t acc1, hq, sh, o;
@@ -93,8 +96,9 @@ constexpr int kEpTrailerBytes = 16;
 static_assert(sizeof(EpTrailer) == kEpTrailerBytes, "trailer layout");
 
 // meta[] words written by the permute scatter kernel
-enum { META_R = 0, META_NACTIVE = 1, META_NTILES = 2, META_WORDS = 8 };
+enum { META_R = 0, META_NACTIVE = 1, META_NTILES = 2, META_NPAIRS = 3, META_WORDS = 8 };
 constexpr int kTileM = 128;   // rows per tensor-core tile
+constexpr int kPairM = 256;   // rows per tile of a CTA pair (two SMs, one 256-row MMA)
 
 // ------------------------------------------------------------------ kernels
 cudaError_t launch_calib_absmax(const void* x, int64_t rows, int d, int dtype, float* absmax,
@@ -118,13 +122,14 @@ cudaError_t launch_topk(const float* logits, const float* bias, int T, int E, in
 // zero (the fused expert launch); block 0 of the scatter clears them.
 cudaError_t launch_permute(const int32_t* idx, int T, int k, int E, int cap, int32_t* hist,
                            int32_t* offsets, int32_t* row2ts, int32_t* ts2row, int32_t* meta,
-                           int32_t* active, int32_t* tiles, cudaStream_t s, int32_t* zero_words = nullptr,
-                           int n_zero = 0);
+                           int32_t* active, int32_t* tiles, int32_t* pairs, cudaStream_t s,
+                           int32_t* zero_words = nullptr, int n_zero = 0);
 bool route_small_ok(int T, int k);
 cudaError_t launch_route_small(const float* logits, const float* bias, int T, int E, int k,
                                int renorm, int cap, int32_t* idx, float* wts, float* logits_out,
                                int32_t* offsets, int32_t* row2ts, int32_t* ts2row, int32_t* meta,
-                               int32_t* active, int32_t* tiles, int32_t* zero_words, int n_zero, cudaStream_t s);
+                               int32_t* active, int32_t* tiles, int32_t* pairs, int32_t* zero_words, int n_zero,
+                               cudaStream_t s);
 // act_clip > 0 caps each token's range (saturating clip), 0 = off.  Codes of
 // each kept (t, slot) go to row ts2row of aq (row stride aq_ld bytes; aq may be
 // null); with wts and idx given, an EpTrailer follows the d codes of each row.
@@ -174,16 +179,17 @@ bool tc_supported(const moe_w8a8_config& c);
 // n_mma back-to-back M=128 N=256 K=32 8-bit MMAs per CTA on `grid` CTAs
 // (operands resident in shared memory): the tensor pipe's own rate.
 cudaError_t launch_tc_peak(int fmt, int64_t n_mma, int grid, cudaStream_t s);
+// pairs != null: run on SM pairs (cta_group::2 MMA, 256-row pair tiles).
 cudaError_t launch_tc_gemm1(const moe_w8a8_weights* w, int T, const int8_t* aq, const int32_t* meta,
-                            const int32_t* tiles, const int32_t* offsets, const int32_t* row2ts,
-                            const float* sx, float* h32, float* pamax, int32_t* acc_dbg,
+                            const int32_t* tiles, const int32_t* pairs, const int32_t* offsets,
+                            const int32_t* row2ts, const float* sx, float* h32, float* pamax, int32_t* acc_dbg,
                             cudaStream_t s);
 cudaError_t launch_requant(const float* h32, const float* pamax, int f, const int32_t* meta,
                            int max_rows, int8_t* hq, float* sh, int fmt, cudaStream_t s);
 cudaError_t launch_tc_gemm2(const moe_w8a8_weights* w, int T, const int8_t* hq, const float* sh,
-                            const int32_t* meta, const int32_t* tiles, const int32_t* offsets,
-                            const int32_t* row2ts, const float* topk_w, void* o, int32_t* acc_dbg,
-                            cudaStream_t s);
+                            const int32_t* meta, const int32_t* tiles, const int32_t* pairs,
+                            const int32_t* offsets, const int32_t* row2ts, const float* topk_w, void* o,
+                            int32_t* acc_dbg, cudaStream_t s);
 
 // GEMM1 + requantisation of h + GEMM2 in one persistent launch (few rows per
 // expert).  sync_words: fused_sync_words(max m-tiles) words, zeroed before the launch.

@@ -583,28 +583,32 @@ __global__ void __launch_bounds__(kSelWarps * 32) router_select_kernel(
 // ---------------------------------------------------------------------------
 
 // Expert offsets (exclusive scan of kept counts) and the lists the expert
-// kernels read: active experts and 128-row tiles.  Run by one full warp: lane
-// l owns experts [l*per, l*per + per), three exclusive warp scans place its
-// offsets, active entries and tiles.
+// kernels read: active experts, 128-row tiles and 256-row pair tiles (for the
+// kernels that run one 256-row MMA on a pair of SMs).  Run by one full warp:
+// lane l owns experts [l*per, l*per + per), exclusive warp scans place its
+// offsets, active entries, tiles and pair tiles.
 __device__ void write_offsets_and_lists(const int* kept, int E, int* off, int32_t* offsets,
-                                        int32_t* meta, int32_t* active, int32_t* tiles, int lane) {
+                                        int32_t* meta, int32_t* active, int32_t* tiles, int32_t* pairs,
+                                        int lane) {
     const int per = (E + 31) / 32;
     const int e0 = min(E, lane * per), e1 = min(E, e0 + per);
-    int rows = 0, nact = 0, ntl = 0;
+    int rows = 0, nact = 0, ntl = 0, npr = 0;
     for (int e = e0; e < e1; ++e) {
         rows += kept[e];
         nact += kept[e] > 0;
         ntl += (kept[e] + kTileM - 1) / kTileM;
+        npr += (kept[e] + kPairM - 1) / kPairM;
     }
-    int xr = rows, xa = nact, xt = ntl;   // inclusive scans
+    int xr = rows, xa = nact, xt = ntl, xp = npr;   // inclusive scans
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
         const int a = __shfl_up_sync(0xffffffffu, xr, o);
         const int b = __shfl_up_sync(0xffffffffu, xa, o);
         const int c = __shfl_up_sync(0xffffffffu, xt, o);
-        if (lane >= o) { xr += a; xa += b; xt += c; }
+        const int d = __shfl_up_sync(0xffffffffu, xp, o);
+        if (lane >= o) { xr += a; xa += b; xt += c; xp += d; }
     }
-    int r = xr - rows, na = xa - nact, nt = xt - ntl;
+    int r = xr - rows, na = xa - nact, nt = xt - ntl, np = xp - npr;
     for (int e = e0; e < e1; ++e) {
         off[e] = r;
         offsets[e] = r;
@@ -614,6 +618,11 @@ __device__ void write_offsets_and_lists(const int* kept, int E, int* off, int32_
             tiles[2 * nt + 1] = r + m * kTileM;
             ++nt;
         }
+        for (int m = 0; m * kPairM < kept[e]; ++m) {
+            pairs[2 * np] = e;
+            pairs[2 * np + 1] = r + m * kPairM;
+            ++np;
+        }
         r += kept[e];
     }
     if (lane == 31) {
@@ -622,6 +631,7 @@ __device__ void write_offsets_and_lists(const int* kept, int E, int* off, int32_
         meta[META_R] = xr;
         meta[META_NACTIVE] = xa;
         meta[META_NTILES] = xt;
+        meta[META_NPAIRS] = xp;
     }
 }
 
@@ -686,7 +696,7 @@ __global__ void __launch_bounds__(kPermThreads) perm_scatter_kernel(
     const int32_t* __restrict__ idx, int n, int E, int cap, int nblk,
     const int32_t* __restrict__ hist, int32_t* __restrict__ offsets, int32_t* __restrict__ row2ts,
     int32_t* __restrict__ ts2row, int32_t* __restrict__ meta, int32_t* __restrict__ active,
-    int32_t* __restrict__ tiles, int32_t* __restrict__ zero_words, int n_zero) {
+    int32_t* __restrict__ tiles, int32_t* __restrict__ pairs, int32_t* __restrict__ zero_words, int n_zero) {
     pdl_wait();
     pdl_trigger();
     // counters a later kernel of this forward starts from zero (the fused expert launch)
@@ -710,7 +720,7 @@ __global__ void __launch_bounds__(kPermThreads) perm_scatter_kernel(
     __syncthreads();
     if (tid < 32) {
         if (blockIdx.x == 0) {
-            write_offsets_and_lists(kept, E, off, offsets, meta, active, tiles, tid);
+            write_offsets_and_lists(kept, E, off, offsets, meta, active, tiles, pairs, tid);
         } else if (tid == 0) {
             int acc = 0;
             for (int e = 0; e < E; ++e) { off[e] = acc; acc += kept[e]; }
@@ -742,7 +752,7 @@ __global__ void __launch_bounds__(kRouteSmallThreads) route_small_kernel(
     int renorm, int cap, int32_t* __restrict__ idx, float* __restrict__ wts,
     float* __restrict__ logits_out, int32_t* __restrict__ offsets, int32_t* __restrict__ row2ts,
     int32_t* __restrict__ ts2row, int32_t* __restrict__ meta, int32_t* __restrict__ active,
-    int32_t* __restrict__ tiles, int32_t* __restrict__ zero_words, int n_zero) {
+    int32_t* __restrict__ tiles, int32_t* __restrict__ pairs, int32_t* __restrict__ zero_words, int n_zero) {
     pdl_wait();
     pdl_trigger();
     // counters a later kernel of this forward starts from zero (the fused expert launch)
@@ -765,7 +775,7 @@ __global__ void __launch_bounds__(kRouteSmallThreads) route_small_kernel(
     if (cap >= 0)
         for (int e = tid; e < E; e += blockDim.x) sm.kept[e] = min(sm.kept[e], cap);
     __syncthreads();
-    if (tid < 32) write_offsets_and_lists(sm.kept, E, sm.off, offsets, meta, active, tiles, tid);
+    if (tid < 32) write_offsets_and_lists(sm.kept, E, sm.off, offsets, meta, active, tiles, pairs, tid);
     __syncthreads();
     scatter_entries(sm.idx, 0, n, E, cap, sm.pre, sm.off, sm.running, sm.u.wcnt, row2ts, ts2row);
 }
@@ -962,13 +972,14 @@ cudaError_t launch_topk(const float* logits, const float* bias, int T, int E, in
 
 cudaError_t launch_permute(const int32_t* idx, int T, int k, int E, int cap, int32_t* hist,
                            int32_t* offsets, int32_t* row2ts, int32_t* ts2row, int32_t* meta,
-                           int32_t* active, int32_t* tiles, cudaStream_t s, int32_t* zero_words, int n_zero) {
+                           int32_t* active, int32_t* tiles, int32_t* pairs, cudaStream_t s, int32_t* zero_words,
+                           int n_zero) {
     const int n = T * k;
     const int nblk = (n + kPermChunk - 1) / kPermChunk;
     cudaError_t err = launch_pdl(perm_hist_kernel, dim3(nblk), dim3(256), 0, s, idx, n, E, hist);
     if (err != cudaSuccess) return err;
     return launch_pdl(perm_scatter_kernel, dim3(nblk), dim3(kPermThreads), 0, s, idx, n, E, cap, nblk, hist,
-                      offsets, row2ts, ts2row, meta, active, tiles, zero_words, n_zero);
+                      offsets, row2ts, ts2row, meta, active, tiles, pairs, zero_words, n_zero);
 }
 
 bool route_small_ok(int T, int k) { return (int64_t)T * k <= kRouteSmallMax; }
@@ -976,14 +987,14 @@ bool route_small_ok(int T, int k) { return (int64_t)T * k <= kRouteSmallMax; }
 cudaError_t launch_route_small(const float* logits, const float* bias, int T, int E, int k,
                                int renorm, int cap, int32_t* idx, float* wts, float* logits_out,
                                int32_t* offsets, int32_t* row2ts, int32_t* ts2row, int32_t* meta,
-                               int32_t* active, int32_t* tiles, int32_t* zero_words, int n_zero,
+                               int32_t* active, int32_t* tiles, int32_t* pairs, int32_t* zero_words, int n_zero,
                                cudaStream_t s) {
     static std::atomic<uint64_t> attr{0};
     cudaError_t e = smem_attr_once(route_small_kernel, sizeof(RouteSmallSmem), attr);
     if (e != cudaSuccess) return e;
     return launch_pdl(route_small_kernel, dim3(1), dim3(kRouteSmallThreads), sizeof(RouteSmallSmem), s, logits,
                       bias, T, E, k, renorm, cap, idx, wts, logits_out, offsets, row2ts, ts2row, meta,
-                      active, tiles, zero_words, n_zero);
+                      active, tiles, pairs, zero_words, n_zero);
 }
 
 cudaError_t launch_smooth_quant(const void* x, int in_dtype, const float* inv_s, float act_clip, int T,

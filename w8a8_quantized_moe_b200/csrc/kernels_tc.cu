@@ -75,6 +75,7 @@ struct TcParams {
     int N, K, n_tiles_n, f, k;
     const int32_t* meta;
     const int32_t* tiles;     // [m-tile][2] = (expert, first row)
+    const int32_t* pairs;     // [pair tile][2] = (expert, first of 256 rows), for CTA pairs
     const int32_t* offsets;   // [E+1]
     const int32_t* row2ts;
     const float* topk_w;
@@ -295,10 +296,24 @@ __device__ __forceinline__ void store_rows32_bf16(float* stage, const uint32_t (
 // GEMM1 tile: columns 0..127 of the accumulator are gate channels
 // nt*128 + c, columns 128..255 the matching up channels.  Each warp owns 32
 // rows (its TMEM lane quarter) and 64 of the 128 h columns.
-template <int FMT>
+// Release of an accumulator buffer by one epilogue warp: a local arrive, or,
+// for a CTA pair, an arrive on the pair leader's barrier (same offset in the
+// leader's shared memory), which counts the warps of both CTAs.
+template <bool PAIR>
+__device__ __forceinline__ void release_acc(uint64_t* bar) {
+    if (PAIR) {
+        uint32_t remote;
+        asm volatile("mapa.shared::cluster.u32 %0, %1, 0;" : "=r"(remote) : "r"(smem_u32(bar)));
+        asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(remote) : "memory");
+    } else {
+        mbar_arrive(bar);
+    }
+}
+
+template <int FMT, bool PAIR = false>
 __device__ __forceinline__ void epilogue_swiglu(const TcParams& p, uint32_t taddr, int half, int e,
                                                 int nt, int wrow0, int nvalid, float* stage,
-                                                Ctl* ctl, int buf, int lane) {
+                                                uint64_t* acc_empty, int lane) {
     const int f = p.f;
     const bool valid = lane < nvalid;
     const int grow = wrow0 + lane;
@@ -315,7 +330,7 @@ __device__ __forceinline__ void epilogue_swiglu(const TcParams& p, uint32_t tadd
         if (c == 1) {
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&ctl->acc_empty[buf]);
+            if (lane == 0) release_acc<PAIR>(acc_empty);
         }
         const int ch0 = nt * 128 + col0;
         const float* swg = p.sw0 + (int64_t)e * f + ch0;
@@ -347,10 +362,10 @@ __device__ __forceinline__ void epilogue_swiglu(const TcParams& p, uint32_t tadd
     if (valid) p.pamax[(int64_t)grow * (f / 64) + nt * 2 + half] = amax;
 }
 
-template <int FMT>
+template <int FMT, bool PAIR = false>
 __device__ __forceinline__ void epilogue_down(const TcParams& p, uint32_t taddr, int half, int e,
-                                              int nt, int wrow0, int nvalid, float* stage, Ctl* ctl,
-                                              int buf, int lane) {
+                                              int nt, int wrow0, int nvalid, float* stage, uint64_t* acc_empty,
+                                              int lane) {
     const int d = p.N;
     const bool valid = lane < nvalid;
     const int grow = wrow0 + lane;
@@ -368,7 +383,7 @@ __device__ __forceinline__ void epilogue_down(const TcParams& p, uint32_t taddr,
         if (c == 3) {
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&ctl->acc_empty[buf]);
+            if (lane == 0) release_acc<PAIR>(acc_empty);
         }
         const int ch0 = nt * BN + col0;
         const float* sw = p.sw0 + (int64_t)e * d + ch0;
@@ -516,9 +531,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int nvalid = max(0, min(32, nrows - quad * 32));
             const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(buf * BN);
             if (EPI == EPI_SWIGLU)
-                epilogue_swiglu<FMT>(p, taddr, half, e, nt, wrow0, nvalid, stage, ctl, buf, lane);
+                epilogue_swiglu<FMT>(p, taddr, half, e, nt, wrow0, nvalid, stage, &ctl->acc_empty[buf], lane);
             else
-                epilogue_down<FMT>(p, taddr, half, e, nt, wrow0, nvalid, stage, ctl, buf, lane);
+                epilogue_down<FMT>(p, taddr, half, e, nt, wrow0, nvalid, stage, &ctl->acc_empty[buf], lane);
             buf ^= 1;
             if (buf == 0) aph ^= 1;
         }
@@ -529,6 +544,293 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == 1) {
         tc_fence_after();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols));
+    }
+}
+
+// ------------------------------------------------------------------ CTA-pair grouped GEMM
+
+// The same grouped GEMM on pairs of SMs: a cluster of two CTAs computes a
+// 256-row x 256-column tile with one tcgen05.mma.cta_group::2 per K slice
+// (M = 256: CTA r holds rows 128 r .. 128 r + 127 of A and columns
+// 128 r .. 128 r + 127 of B in its shared memory, and its 128 rows of the
+// accumulator in its tensor memory).  Each SM so loads half of the tile's
+// weight columns and all of its own rows: 32 KB per 128-byte K block instead
+// of 48 KB for the same MMA work, and six stages fit where four did.
+// Tiles are the pair tiles of the routing metadata (256 rows of one expert;
+// the second CTA's rows may be past the expert's last row, then they are
+// computed and not stored).
+//   warp 0 (both CTAs)   TMA producer for its own A rows and B columns; the
+//                        loads signal the leader CTA's stage barrier, whose
+//                        expected byte count covers both CTAs' loads
+//   warp 1 (leader)      MMA issuer; each K block's commit is multicast to the
+//                        stage-free barriers of both CTAs, each tile's to
+//                        both CTAs' accumulator-full barriers
+//   warps 2..9 (both)    epilogue on the CTA's own 128 rows; every warp
+//                        releases the accumulator on the leader's barrier
+//                        (16 arrivals per phase)
+// Both CTAs allocate and free the tensor memory together (cta_group::2); a
+// cluster barrier after set-up and before the free keeps either CTA from
+// touching the other's barriers or memory while it does not exist.
+constexpr int kStagesP = 6;
+constexpr int kABytesP = BM * BK;             // 16 KB: this CTA's rows of A
+constexpr int kBBytesP = (BN / 2) * BK;       // 16 KB: this CTA's half of the B columns
+constexpr int kStageBytesP = kABytesP + kBBytesP;
+constexpr size_t kSmemBytesP =
+    (size_t)kStagesP * kStageBytesP + (size_t)kEpiWarps * kEpiStageBytes + 1024 + 256;
+
+struct CtlP {
+    uint64_t full[kStagesP];
+    uint64_t empty[kStagesP];
+    uint64_t acc_full[2];
+    uint64_t acc_empty[2];
+    uint64_t drain;
+    uint32_t tmem_base;
+    int abort;
+};
+
+// Instruction descriptor of the pair MMA: as idesc(), with M = 256.
+template <int FMT>
+__host__ __device__ constexpr uint32_t idesc_pair() {
+    return (FMT == FMT_E4M3 ? (1u << 4) : ((2u << 4) | (1u << 7) | (1u << 10))) | ((uint32_t)(BN >> 3) << 17) |
+           ((uint32_t)((2 * BM) >> 4) << 24);
+}
+
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ uint32_t cluster_index() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%clusterid.x;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ uint32_t cluster_count() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%nclusterid.x;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// The address of this CTA's shared variable in the leader's (rank 0) shared memory.
+__device__ __forceinline__ uint32_t leader_addr(const void* p) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, 0;" : "=r"(r) : "r"(smem_u32(p)));
+    return r;
+}
+
+// TMA load into this CTA's shared memory whose completion is counted on a
+// barrier of the pair (here: the leader's stage barrier).  No multicast.
+__device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* map, uint32_t bar, int x, int y) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], "
+        "[%2];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y)
+        : "memory");
+}
+
+template <int FMT>
+__device__ __forceinline__ void mma_8bit_pair(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t accum) {
+    if (FMT == FMT_E4M3)
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "setp.ne.b32 p, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(tmem_d),
+            "l"(adesc), "l"(bdesc), "r"(idesc_pair<FMT>()), "r"(accum));
+    else
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "setp.ne.b32 p, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::2.kind::i8 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(tmem_d),
+            "l"(adesc), "l"(bdesc), "r"(idesc_pair<FMT>()), "r"(accum));
+}
+
+// Arrive, when the pair MMAs issued so far are done, on `bar` in each CTA of
+// `mask` (same shared-memory offset in each).
+__device__ __forceinline__ void mma_commit_pair(uint64_t* bar, uint16_t mask) {
+    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+                     smem_u32(bar)),
+                 "h"(mask)
+                 : "memory");
+}
+
+// try_wait with cluster-scope acquire: for barriers the other CTA arrives on.
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+__device__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, volatile int* abort, int32_t* status, int site,
+                                  int iter) {
+    if (mbar_try_wait_cluster(bar, parity)) return true;
+    const uint64_t t0 = global_timer();
+    while (true) {
+        if (mbar_try_wait_cluster(bar, parity)) return true;
+        if (*abort) return false;
+        if (global_timer() - t0 > kWaitBudgetNs) {
+            *abort = 1;
+            report_timeout(status, site, iter, (int)parity);
+            return false;
+        }
+    }
+}
+
+template <int EPI, int FMT>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+    tc_pair_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
+                        const TcParams p) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    float* epi_stage = reinterpret_cast<float*>(smem + kStagesP * kStageBytesP);
+    CtlP* ctl = reinterpret_cast<CtlP*>(smem + kStagesP * kStageBytesP + kEpiWarps * kEpiStageBytes);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int rank = (int)cluster_ctarank();
+    const bool leader = rank == 0;
+    const int nkb = p.K / BK;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStagesP; ++s) {
+            mbar_init(&ctl->full[s], 1);
+            mbar_init(&ctl->empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&ctl->acc_full[b], 1);
+            mbar_init(&ctl->acc_empty[b], 2 * kEpiWarps);
+        }
+        mbar_init(&ctl->drain, 1);
+        ctl->abort = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         smem_u32(&ctl->tmem_base)),
+                     "r"(kTmemCols));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;");
+    }
+    tc_fence_before();
+    cluster_sync_all();
+    tc_fence_after();
+    const uint32_t tmem = ctl->tmem_base;
+    volatile int* abort = &ctl->abort;
+    pdl_wait();
+    pdl_trigger();
+    const int num_tiles = p.meta[META_NPAIRS] * p.n_tiles_n;
+    const int cid = (int)cluster_index(), ncl = (int)cluster_count();
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // ---------------- TMA producer (both CTAs): own rows of A, own half of B
+            int s = 0;
+            uint32_t ph = 0;
+            uint32_t issued_par[kStagesP];
+            bool issued[kStagesP];
+            for (int i = 0; i < kStagesP; ++i) issued[i] = false;
+            bool ok = true;
+            for (int t = cid; t < num_tiles && ok; t += ncl) {
+                const int mt = t / p.n_tiles_n, nt = t % p.n_tiles_n;
+                const int e = p.pairs[2 * mt], row0 = p.pairs[2 * mt + 1] + rank * BM;
+                const int brow = e * p.N + nt * BN + rank * (BN / 2);
+                for (int kb = 0; kb < nkb; ++kb) {
+                    if (!mbar_wait(&ctl->empty[s], ph ^ 1, abort, p.status, 1, t)) { ok = false; break; }
+                    if (leader) mbar_arrive_expect_tx(&ctl->full[s], 2 * kStageBytesP);
+                    const uint32_t bar = leader_addr(&ctl->full[s]);
+                    uint8_t* sa = smem + s * kStageBytesP;
+                    tma_load_2d_pair(sa, &tm_a, bar, kb * BK, row0);
+                    tma_load_2d_pair(sa + kABytesP, &tm_b, bar, kb * BK, brow);
+                    issued[s] = true;
+                    issued_par[s] = ph;
+                    if (++s == kStagesP) { s = 0; ph ^= 1; }
+                }
+            }
+            if (leader) {
+                // the leader's stage barriers count both CTAs' bytes: wait for the
+                // copies of every stage it issued to land (bounded)
+                for (int i = 0; i < kStagesP; ++i) {
+                    if (!issued[i]) continue;
+                    const uint64_t t0 = global_timer();
+                    while (!mbar_try_wait(&ctl->full[i], issued_par[i]) && global_timer() - t0 < kWaitBudgetNs) {}
+                }
+            }
+            if (!ok) {
+                // after a timeout, copies this CTA issued may still be in flight and
+                // their completion is counted only on the other CTA's barrier: give
+                // them time to land before the CTA can exit (bounded)
+                const uint64_t t0 = global_timer();
+                while (global_timer() - t0 < 200000ull) {}
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0 && leader) {
+            // ---------------- MMA issuer (leader CTA only)
+            int s = 0, buf = 0;
+            uint32_t ph = 0, aph = 0;
+            bool ok = true;
+            for (int t = cid; t < num_tiles && ok; t += ncl) {
+                if (!mbar_wait_cluster(&ctl->acc_empty[buf], aph ^ 1, abort, p.status, 2, t)) break;
+                tc_fence_after();
+                const uint32_t d_tmem = tmem + (uint32_t)(buf * BN);
+                for (int kb = 0; kb < nkb; ++kb) {
+                    if (!mbar_wait(&ctl->full[s], ph, abort, p.status, 3, t)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t a_addr = smem_u32(smem + s * kStageBytesP);
+                    const uint32_t b_addr = a_addr + kABytesP;
+#pragma unroll
+                    for (int kk = 0; kk < BK / 32; ++kk)
+                        mma_8bit_pair<FMT>(d_tmem, desc_sw128(a_addr + kk * 32), desc_sw128(b_addr + kk * 32),
+                                           (kb | kk) != 0 ? 1u : 0u);
+                    mma_commit_pair(&ctl->empty[s], 0x3);
+                    if (++s == kStagesP) { s = 0; ph ^= 1; }
+                }
+                if (!ok) break;
+                mma_commit_pair(&ctl->acc_full[buf], 0x3);
+                buf ^= 1;
+                if (buf == 0) aph ^= 1;
+            }
+            // all MMAs issued by this thread complete before the tensor memory is freed (bounded)
+            mma_commit_pair(&ctl->drain, 0x1);
+            const uint64_t t0 = global_timer();
+            while (!mbar_try_wait(&ctl->drain, 0) && global_timer() - t0 < kWaitBudgetNs) {}
+        }
+    } else {
+        // ---------------- epilogue warps (both CTAs): this CTA's 128 rows of the tile
+        const int ew = warp - 2;
+        const int quad = warp & 3;
+        const int half = ew >> 2;
+        float* stage = epi_stage + ew * (kEpiStageBytes / 4);
+        int buf = 0;
+        uint32_t aph = 0;
+        for (int t = cid; t < num_tiles; t += ncl) {
+            if (!mbar_wait(&ctl->acc_full[buf], aph, abort, p.status, 4, t)) break;
+            tc_fence_after();
+            const int mt = t / p.n_tiles_n, nt = t % p.n_tiles_n;
+            const int e = p.pairs[2 * mt], row0 = p.pairs[2 * mt + 1] + rank * BM;
+            const int nrows = min(BM, p.offsets[e + 1] - row0);
+            const int wrow0 = row0 + quad * 32;
+            const int nvalid = max(0, min(32, nrows - quad * 32));
+            const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(buf * BN);
+            if (EPI == EPI_SWIGLU)
+                epilogue_swiglu<FMT, true>(p, taddr, half, e, nt, wrow0, nvalid, stage, &ctl->acc_empty[buf], lane);
+            else
+                epilogue_down<FMT, true>(p, taddr, half, e, nt, wrow0, nvalid, stage, &ctl->acc_empty[buf], lane);
+            buf ^= 1;
+            if (buf == 0) aph ^= 1;
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync_all();
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols));
     }
 }
 
@@ -863,7 +1165,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
             const int nvalid = max(0, min(32, nrows - quad * 32));
             const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(buf * BN);
             if (g1) {
-                epilogue_swiglu<FMT>(p1, taddr, half, e, nt, wrow0, nvalid, stage, ctl, buf, lane);
+                epilogue_swiglu<FMT>(p1, taddr, half, e, nt, wrow0, nvalid, stage, &ctl->acc_empty[buf], lane);
                 // this warp's share of the tile is stored: count it; the last arrival requantises
                 __threadfence();
                 __syncwarp();
@@ -877,7 +1179,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
                 }
             } else {
                 (void)ld_acquire(fx.ready + mt);   // the h scales this epilogue reads were released there
-                epilogue_down<FMT>(p2, taddr, half, e, nt, wrow0, nvalid, stage, ctl, buf, lane);
+                epilogue_down<FMT>(p2, taddr, half, e, nt, wrow0, nvalid, stage, &ctl->acc_empty[buf], lane);
             }
             buf ^= 1;
             if (buf == 0) aph ^= 1;
@@ -1225,12 +1527,57 @@ cudaError_t launch(const CUtensorMap& ta, const CUtensorMap& tb, const TcParams&
     return fmt == FMT_E4M3 ? launch_fmt<EPI, FMT_E4M3>(ta, tb, p, grid, s) : launch_fmt<EPI, FMT_INT8>(ta, tb, p, grid, s);
 }
 
+// The pair kernel on as many SM pairs as can be resident at once (one pair
+// per cluster of two CTAs; persistent), at most one per pair tile x column tile.
+template <int EPI, int FMT>
+cudaError_t launch_pair_fmt(const CUtensorMap& ta, const CUtensorMap& tb, const TcParams& p, int max_units,
+                            cudaStream_t s) {
+    static std::atomic<uint64_t> attr{0};
+    static int clusters[64] = {};
+    auto kern = tc_pair_gemm_kernel<EPI, FMT>;
+    cudaError_t e = smem_attr_once(kern, kSmemBytesP, attr);
+    if (e != cudaSuccess) return e;
+    int dev = 0;
+    e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    int& nc = clusters[dev & 63];
+    if (nc == 0) {
+        cudaLaunchConfig_t q = {};
+        q.gridDim = dim3(2);
+        q.blockDim = dim3(kThreads);
+        q.dynamicSmemBytes = kSmemBytesP;
+        cudaLaunchAttribute a[1];
+        a[0].id = cudaLaunchAttributeClusterDimension;
+        a[0].val.clusterDim.x = 2;
+        a[0].val.clusterDim.y = 1;
+        a[0].val.clusterDim.z = 1;
+        q.attrs = a;
+        q.numAttrs = 1;
+        int n = 0;
+        e = cudaOccupancyMaxActiveClusters(&n, (const void*)kern, &q);
+        if (e != cudaSuccess) return e;
+        if (n <= 0) return cudaErrorInvalidConfiguration;
+        nc = n;
+    }
+    const int grid = 2 * std::max(1, std::min(nc, max_units));
+    return launch_pdl(kern, dim3(grid), dim3(kThreads), kSmemBytesP, s, ta, tb, p);
+}
+
+template <int EPI>
+cudaError_t launch_pair(const CUtensorMap& ta, const CUtensorMap& tb, const TcParams& p, int max_units, int fmt,
+                        cudaStream_t s) {
+    return fmt == FMT_E4M3 ? launch_pair_fmt<EPI, FMT_E4M3>(ta, tb, p, max_units, s)
+                           : launch_pair_fmt<EPI, FMT_INT8>(ta, tb, p, max_units, s);
+}
+
 }  // namespace
 
 bool tc_make_weight_maps(moe_w8a8_weights* w) {
     const moe_w8a8_config& c = w->cfg;
     const uint64_t E = w->n_local, d = c.d, f = c.f;   // the experts this handle holds
-    return make_map(&w->tm_w_gu, w->w_gu, d, E * 2 * f, BN) && make_map(&w->tm_w_dn, w->w_dn, f, E * d, BN);
+    return make_map(&w->tm_w_gu, w->w_gu, d, E * 2 * f, BN) && make_map(&w->tm_w_dn, w->w_dn, f, E * d, BN) &&
+           make_map(&w->tm_w_gu_half, w->w_gu, d, E * 2 * f, BN / 2) &&
+           make_map(&w->tm_w_dn_half, w->w_dn, f, E * d, BN / 2);
 }
 
 template <int FMT>
@@ -1331,8 +1678,8 @@ cudaError_t launch_requant(const float* h32, const float* pamax, int f, const in
 }
 
 cudaError_t launch_tc_gemm1(const moe_w8a8_weights* w, int T, const int8_t* aq, const int32_t* meta,
-                            const int32_t* tiles, const int32_t* offsets, const int32_t* row2ts,
-                            const float* sx, float* h32, float* pamax, int32_t* acc_dbg,
+                            const int32_t* tiles, const int32_t* pairs, const int32_t* offsets,
+                            const int32_t* row2ts, const float* sx, float* h32, float* pamax, int32_t* acc_dbg,
                             cudaStream_t s) {
     const moe_w8a8_config& c = w->cfg;
     CUtensorMap ta;
@@ -1355,15 +1702,20 @@ cudaError_t launch_tc_gemm1(const moe_w8a8_weights* w, int T, const int8_t* aq, 
     p.pamax = pamax;
     p.acc_dbg = acc_dbg;
     p.status = w->status;
+    p.pairs = pairs;
+    if (pairs) {
+        const int max_pt = (rows + 2 * BM - 1) / (2 * BM) + w->n_local;
+        return launch_pair<EPI_SWIGLU>(ta, w->tm_w_gu_half, p, max_pt * p.n_tiles_n, c.expert_format, s);
+    }
     const int max_mt = (rows + BM - 1) / BM + c.n_experts;
     const int grid = max(1, min(w->num_sms, max_mt * p.n_tiles_n));
     return launch<EPI_SWIGLU>(ta, w->tm_w_gu, p, grid, c.expert_format, s);
 }
 
 cudaError_t launch_tc_gemm2(const moe_w8a8_weights* w, int T, const int8_t* hq, const float* sh,
-                            const int32_t* meta, const int32_t* tiles, const int32_t* offsets,
-                            const int32_t* row2ts, const float* topk_w, void* o, int32_t* acc_dbg,
-                            cudaStream_t s) {
+                            const int32_t* meta, const int32_t* tiles, const int32_t* pairs,
+                            const int32_t* offsets, const int32_t* row2ts, const float* topk_w, void* o,
+                            int32_t* acc_dbg, cudaStream_t s) {
     const moe_w8a8_config& c = w->cfg;
     CUtensorMap ta;
     const int rows = T * c.top_k;
@@ -1385,6 +1737,11 @@ cudaError_t launch_tc_gemm2(const moe_w8a8_weights* w, int T, const int8_t* hq, 
     p.o_bf16 = c.out_dtype == MOE_BF16;
     p.acc_dbg = acc_dbg;
     p.status = w->status;
+    p.pairs = pairs;
+    if (pairs) {
+        const int max_pt = (rows + 2 * BM - 1) / (2 * BM) + w->n_local;
+        return launch_pair<EPI_DOWN>(ta, w->tm_w_dn_half, p, max_pt * p.n_tiles_n, c.expert_format, s);
+    }
     const int max_mt = (rows + BM - 1) / BM + c.n_experts;
     const int grid = max(1, min(w->num_sms, max_mt * p.n_tiles_n));
     return launch<EPI_DOWN>(ta, w->tm_w_dn, p, grid, c.expert_format, s);

@@ -139,6 +139,7 @@ WsLayout ws_layout(const moe_w8a8_weights* w, int T, WsPart part) {
     L.meta = take(META_WORDS * 4);
     L.active = take((size_t)E * 4);
     L.tiles = take(max_tiles * 8);
+    L.pairs = take(((tk + kPairM - 1) / kPairM + E) * 8);
     L.row2ts = take(tk * 4);
     L.ts2row = take(tk * 4);
     L.xq = take(experts && !stream ? 0 : (size_t)T * d);
@@ -282,6 +283,7 @@ moe_status prepare_impl(const moe_w8a8_config* cfg, int e_first, int n_local, co
     w->wait_budget_ns = 2000000000ull;
     w->test_skip_ready = -1;
     w->fused_max_rows = kFusedMaxRows;
+    w->cta_pairs = 2;
     if (cudaGetDevice(&w->device) != cudaSuccess ||
         cudaDeviceGetAttribute(&w->num_sms, cudaDevAttrMultiProcessorCount, w->device) != cudaSuccess) {
         free_handle(w);
@@ -444,14 +446,15 @@ moe_status route_stage(Run& r, const void* x, int T, const float* bias, const fl
     if (certified) {
         r.mark(MOE_STAGE_PERMUTE, 0);
         CUDA_TRY(launch_permute(idx, T, k, E, capacity_of(c, T), r.at<int32_t>(L.hist), offsets, row2ts, ts2row,
-                                meta, active, tiles, s, zero_words, n_zero));
+                                meta, active, tiles, r.at<int32_t>(L.pairs), s, zero_words, n_zero));
         r.mark(MOE_STAGE_PERMUTE, 1);
         r.launches += 2;
     } else if (route_small_ok(T, k)) {
         // top-k, histogram, scan and scatter in one block
         r.mark(MOE_STAGE_TOPK, 0);
         CUDA_TRY(launch_route_small(lsrc, bias, T, E, k, c.renormalize, capacity_of(c, T), idx, wts, dbg_logits,
-                                    offsets, row2ts, ts2row, meta, active, tiles, zero_words, n_zero, s));
+                                    offsets, row2ts, ts2row, meta, active, tiles, r.at<int32_t>(L.pairs), zero_words,
+                                    n_zero, s));
         r.mark(MOE_STAGE_TOPK, 1);
         r.empty_stage(MOE_STAGE_PERMUTE);
         ++r.launches;
@@ -462,7 +465,7 @@ moe_status route_stage(Run& r, const void* x, int T, const float* bias, const fl
         ++r.launches;
         r.mark(MOE_STAGE_PERMUTE, 0);
         CUDA_TRY(launch_permute(idx, T, k, E, capacity_of(c, T), r.at<int32_t>(L.hist), offsets, row2ts, ts2row,
-                                meta, active, tiles, s, zero_words, n_zero));
+                                meta, active, tiles, r.at<int32_t>(L.pairs), s, zero_words, n_zero));
         r.mark(MOE_STAGE_PERMUTE, 1);
         r.launches += 2;
     }
@@ -543,14 +546,20 @@ moe_status expert_stage(Run& r, int T, int path) {
         return MOE_OK;
     }
     r.mark(MOE_STAGE_GEMM1, 0);
-    CUDA_TRY(launch_tc_gemm1(w, T, aq, meta, tiles, offsets, row2ts, sx, r.at<float>(L.h32), r.at<float>(L.pamax),
+    // SM pairs (256-row tiles) when asked to, or by default when the rows per
+    // expert fill such tiles on average (a pair tile's second half is wasted
+    // MMA work on an expert's last rows)
+    const bool pair = w->cta_pairs == 1 || (w->cta_pairs == 2 && tk >= (size_t)kPairM * w->cfg.n_experts);
+    const int32_t* pairs = pair ? r.at<int32_t>(L.pairs) : nullptr;
+    CUDA_TRY(launch_tc_gemm1(w, T, aq, meta, tiles, pairs, offsets, row2ts, sx, r.at<float>(L.h32), r.at<float>(L.pamax),
                              dbg ? dbg->acc1 : nullptr, s));
     r.mark(MOE_STAGE_GEMM1, 1);
     r.mark(MOE_STAGE_REQUANT, 0);
     CUDA_TRY(launch_requant(r.at<float>(L.h32), r.at<float>(L.pamax), f, meta, (int)tk, hq, sh, c.expert_format, s));
     r.mark(MOE_STAGE_REQUANT, 1);
     r.mark(MOE_STAGE_GEMM2, 0);
-    CUDA_TRY(launch_tc_gemm2(w, T, hq, sh, meta, tiles, offsets, row2ts, wts, o, dbg ? dbg->acc2 : nullptr, s));
+    CUDA_TRY(launch_tc_gemm2(w, T, hq, sh, meta, tiles, pairs, offsets, row2ts, wts, o, dbg ? dbg->acc2 : nullptr,
+                             s));
     r.mark(MOE_STAGE_GEMM2, 1);
     r.launches += 3;
     return MOE_OK;
@@ -700,6 +709,12 @@ moe_status moe_w8a8_set_path(moe_w8a8_weights* w, int32_t path) {
 moe_status moe_w8a8_set_stream_threshold(moe_w8a8_weights* w, int32_t max_rows) {
     if (!w || max_rows < 0) return MOE_ERR_INVALID_ARG;
     w->stream_max_rows = max_rows;
+    return MOE_OK;
+}
+
+moe_status moe_w8a8_set_cta_pairs(moe_w8a8_weights* w, int32_t mode) {
+    if (!w || mode < 0 || mode > 2) return MOE_ERR_INVALID_ARG;
+    w->cta_pairs = mode;
     return MOE_OK;
 }
 
@@ -930,7 +945,7 @@ moe_status moe_w8a8_ep_experts(const moe_w8a8_weights* w, const void* recv, int3
     CUDA_TRY(launch_ep_read_experts(rows, R, rb, d, w->ep_first, w->n_local, idx, w->status, s));
     CUDA_TRY(launch_permute(idx, R, 1, v.cfg.n_experts, -1, r.at<int32_t>(L.hist), r.at<int32_t>(L.offsets),
                             r.at<int32_t>(L.row2ts), ts2row, r.at<int32_t>(L.meta), r.at<int32_t>(L.active),
-                            r.at<int32_t>(L.tiles), s));
+                            r.at<int32_t>(L.tiles), r.at<int32_t>(L.pairs), s));
     const bool stream_path = path == MOE_PATH_STREAM;
     CUDA_TRY(launch_ep_gather(rows, R, rb, d, stream_path ? nullptr : ts2row,
                               stream_path ? r.at<int8_t>(L.xq) : r.at<int8_t>(L.aq), r.at<float>(L.sx),
