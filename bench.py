@@ -38,10 +38,85 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 INT8_PER_BF16 = 2.0   # nominal dense ratio (4.5 POPS int8 / 2.25 PFLOPS bf16)
 
 # DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum) of the dominant
-# kernel, from one ncu capture of the current kernel source (see profiles/).
-TRAFFIC = {
-    ("decode", 32, "tc_ffn_fused_kernel"): 1060.720e6 + 6.530304e6,
-}
+# kernels, recorded from ncu captures into profiles/dram_traffic.md (--record-traffic) with a
+# hash of the CUDA sources; a figure whose hash no longer matches the sources is not used.
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "dram_traffic.md")
+
+
+def sources_hash() -> str:
+    """First 16 hex digits of a SHA-256 over the library's CUDA sources and headers."""
+    import glob
+    import hashlib
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "w8a8_quantized_moe_b200", "csrc")
+    for fn in sorted(glob.glob(os.path.join(csrc, "*.cu")) + glob.glob(os.path.join(csrc, "*.cuh")) +
+                     glob.glob(os.path.join(csrc, "*.h"))):
+        h.update(os.path.basename(fn).encode())
+        with open(fn, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def load_traffic() -> dict:
+    """{(workload, T, kernel): bytes per launch} for the current sources."""
+    out = {}
+    if not os.path.exists(TRAFFIC_FILE):
+        return out
+    cur = sources_hash()
+    for line in open(TRAFFIC_FILE):
+        cells = [c.strip() for c in line.strip().strip("|").split("|")]
+        if len(cells) != 8 or not cells[1].isdigit():
+            continue
+        wl, T, kernel, launches, rd, wr, per_launch, sha = cells
+        if sha == cur:
+            out[(wl, int(T), kernel)] = float(per_launch)
+    return out
+
+
+def record_traffic(csv_path: str, workload: str, T: int, scale: float = 1.0):
+    """Parse an ncu CSV (--metrics dram__bytes_read.sum,dram__bytes_write.sum --csv) and
+    write the per-launch DRAM bytes of each kernel to profiles/dram_traffic.md (mean over
+    its captured launches, times `scale` when a smaller case stands in for the workload),
+    replacing the rows of this workload and T."""
+    import csv
+    import re
+    unit = {"byte": 1.0, "Kbyte": 1e3, "Mbyte": 1e6, "Gbyte": 1e9, "Tbyte": 1e12}
+    per = {}
+    with open(csv_path) as fh:
+        rows = [r for r in csv.reader(l for l in fh if l.startswith('"'))]
+    hdr = rows[0]
+    col = {n: hdr.index(n) for n in ("ID", "Kernel Name", "Metric Name", "Metric Unit", "Metric Value")}
+    for r in rows[1:]:
+        raw = re.sub(r"\(anonymous namespace\)::", "", r[col["Kernel Name"]]).split("(")[0].split("<")[0]
+        name = raw.split("::")[-1].split()[-1]
+        m = r[col["Metric Name"]]
+        if m not in ("dram__bytes_read.sum", "dram__bytes_write.sum"):
+            continue
+        v = float(r[col["Metric Value"]].replace(",", "")) * unit.get(r[col["Metric Unit"]], 1.0)
+        d = per.setdefault(name, {}).setdefault(r[col["ID"]], {})
+        d[m] = v
+    keep = []
+    if os.path.exists(TRAFFIC_FILE):
+        for line in open(TRAFFIC_FILE):
+            cells = [c.strip() for c in line.strip().strip("|").split("|")]
+            if len(cells) == 8 and cells[1].isdigit() and (cells[0], int(cells[1])) == (workload, T):
+                continue
+            keep.append(line.rstrip("\n"))
+    if not keep:
+        keep = ["# DRAM traffic per launch of the dominant kernels (ncu)", "",
+                "Written by `python bench.py --record-traffic <ncu csv> --workload <w> [--tokens T]` from",
+                "`ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum --clock-control none --csv` of the",
+                "same bench command; bench.py uses a row only while the sources hash still matches.", "",
+                "| workload | T | kernel | launches | read bytes | write bytes | bytes per launch | sources |",
+                "|---|---|---|---|---|---|---|---|"]
+    sha = sources_hash()
+    for name, launches in sorted(per.items()):
+        rd = sum(x.get("dram__bytes_read.sum", 0.0) for x in launches.values()) / len(launches)
+        wr = sum(x.get("dram__bytes_write.sum", 0.0) for x in launches.values()) / len(launches)
+        keep.append(f"| {workload} | {T} | {name} | {len(launches)} | {rd * scale:.0f} | {wr * scale:.0f} | "
+                    f"{(rd + wr) * scale:.0f} | {sha} |")
+    with open(TRAFFIC_FILE, "w") as fh:
+        fh.write("\n".join(keep) + "\n")
 
 FUSED_MAX_ROWS = 512   # the library's default: T*k up to which GEMM1 + requant + GEMM2 are one launch
 
@@ -74,6 +149,11 @@ def parse():
                    help="time the expert-parallel layer (experts split over the ranks) instead")
     p.add_argument("--no-prefill", action="store_true",
                    help="skip the extra prefill-layer measurement of the decode run")
+    p.add_argument("--record-traffic", metavar="NCU_CSV", default="",
+                   help="write the per-launch DRAM bytes of an ncu CSV (dram__bytes_read.sum, "
+                        "dram__bytes_write.sum) for --workload / --tokens to profiles/dram_traffic.md and exit")
+    p.add_argument("--traffic-scale", type=float, default=1.0,
+                   help="with --record-traffic: factor from the captured case to the workload's launch")
     p.add_argument("--no-large", action="store_true",
                    help="skip the extra large-sparse-layer measurement of the decode run")
     p.add_argument("--fused-max-rows", type=int, default=-1,
@@ -518,7 +598,7 @@ def measure(args, wl, world, rank, local, e2e_on=True, wts=None):
             achieved = ops / (dom_ms / 1e3) / 1e12
             roof = {"bound": "tensor", "kernel": f"{dom} ({kernel})", "achieved": achieved,
                     "peak": int8_peak, "unit": "TFLOP/s", "frac": achieved / int8_peak,
-                    "traffic": TRAFFIC.get((wl.name, wl.T, kernel)),
+                    "traffic": load_traffic().get((wl.name, wl.T, kernel)),
                     "peak_source": int8_src,
                     "int8_ops_per_launch": ops, "launch_ms": dom_ms,
                     "frac_of_nominal_4500": achieved / NOMINAL_INT8_TOPS}
@@ -528,7 +608,7 @@ def measure(args, wl, world, rank, local, e2e_on=True, wts=None):
             achieved = nbytes / (dom_ms / 1e3) / 1e9
             roof = {"bound": "hbm", "kernel": f"{dom} ({kernel})", "achieved": achieved,
                     "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
-                    "traffic": TRAFFIC.get((wl.name, wl.T, kernel)),
+                    "traffic": load_traffic().get((wl.name, wl.T, kernel)),
                     "peak_source": f"hbm_gbs of {peak_src}",
                     "algorithmic_bytes_per_launch": nbytes, "launch_ms": dom_ms}
     step_s = ms_total / K / 1e3
@@ -838,6 +918,10 @@ def run_ep(args, world, rank, local):
 
 def main():
     args = parse()
+    if args.record_traffic:
+        wl = synth.WORKLOADS[args.workload]
+        record_traffic(args.record_traffic, args.workload, args.tokens or wl.T, args.traffic_scale)
+        return
     world, rank, local = dist_setup(args)
     try:
         if args.impl == "reference":

@@ -52,3 +52,26 @@ def test_gemm2_bytes_count_per_slot_rows_in_the_output_dtype():
     a = bench.algorithmic(wl, n_active=56, R=128, tensor=True)
     # 56 * 4096 * 1536 weights + 128 * 1536 h codes + 128 * 4096 * 2 rows + 56 * 4096 * 4 scales
     assert a["gemm2_bytes"] == 352_321_536 + 196_608 + 1_048_576 + 917_504
+
+
+def test_traffic_record_and_lookup(tmp_path, monkeypatch):
+    """An ncu CSV's per-kernel DRAM bytes become a table row stamped with the
+    sources hash; the lookup uses it only while the hash matches."""
+    bench, synth = _bench()
+    monkeypatch.setattr(bench, "TRAFFIC_FILE", str(tmp_path / "dram_traffic.md"))
+    hdr = ('"ID","Process ID","Process Name","Host Name","Kernel Name","Context","Stream","Block Size",'
+           '"Grid Size","Device","CC","Section Name","Metric Name","Metric Unit","Metric Value"\n')
+    rows = []
+    for i, (rd, wr) in enumerate([(1000.0, 10.0), (1002.0, 12.0)]):
+        for m, v in (("dram__bytes_read.sum", rd), ("dram__bytes_write.sum", wr)):
+            rows.append(f'"{i}","1","python","h","void moe::(anonymous namespace)::tc_ffn_fused_kernel<0>'
+                        f'(CUtensorMap_st, TcParams)","1","7","(352, 1, 1)","(148, 1, 1)","0","10.0",'
+                        f'"Command line profiler metrics","{m}","Mbyte","{v}"\n')
+    csv_path = tmp_path / "l.csv"
+    csv_path.write_text("==PROF== noise\n" + hdr + "".join(rows))
+    bench.record_traffic(str(csv_path), "decode", 32)
+    t = bench.load_traffic()
+    assert abs(t[("decode", 32, "tc_ffn_fused_kernel")] - 1012e6) < 1.0
+    # a different sources hash: the row is ignored
+    monkeypatch.setattr(bench, "sources_hash", lambda: "0" * 16)
+    assert bench.load_traffic() == {}
