@@ -313,3 +313,24 @@ def test_pair_gemms_decode_shape_certified_router(M, sweep_layer):
         run(M, wl, W, prep, data, tokens=spread(wl.T, 16), fields=H.DBG_SMALL + ("acc1", "acc2", "o"))
     finally:
         M.moe_w8a8_set_cta_pairs(W, 2)
+
+
+def test_large_batch_quantiser_with_activation_clip(M):
+    """From 1024 tokens on the tensor path the quantisation runs one warp per
+    token on bulk-copied X rows; with a saturating clip at the 99.9th
+    percentile of the calibration activations every stage still matches."""
+    import torch
+    wl = dataclasses.replace(synth.WORKLOADS["tiny"], T=1100, data_seed=75, logits_uniform=True)
+    wts, data, W, prep = layer(wl)
+    cal = H.to_dev(wts.calib_x)
+    clip = M.moe_w8a8_calibrate_act_clip(W, cal, 99.9)
+    assert clip == oracle.act_clip_percentile(wts.calib_x, prep.inv_s, 99.9)
+    M.moe_w8a8_set_act_clip(W, clip)
+    rt = H.oracle_route(wl, data)
+    y, dbg = H.gpu_forward(W, wl, data, path=M.MOE_PATH_TENSOR)
+    toks = spread(wl.T, 48)
+    y_ref, odbg = oracle.moe_tokens(data.x, prep, rt, tokens=toks, out_bf16=wl.in_bf16, act_clip=clip)
+    H.compare_stages(wl, rt, dbg, y, y_ref, odbg, toks)
+    assert np.array_equal(y[toks], y_ref)
+    assert (dbg["sx"] == np.float32(clip) / np.float32(127.0)).sum() > 0
+    del torch

@@ -189,7 +189,7 @@ def test_fp8_refuses_the_streaming_path(M, decode_fp8):
 def test_fp8_pair_gemms(M):
     """FP8 experts with the separate GEMM launches on SM pairs
     (tcgen05.mma.cta_group::2.kind::f8f6f4)."""
-    wl = dataclasses.replace(synth.WORKLOADS["tiny"], T=600, data_seed=610)
+    wl = dataclasses.replace(synth.WORKLOADS["tiny"], T=1200, data_seed=610)   # also the large-batch quantiser
     wts = synth.make_weights(wl)
     W = H.gpu_prepare(wl, wts, fmt=M.MOE_FMT_E4M3)
     M.moe_w8a8_set_cta_pairs(W, 1)
