@@ -231,38 +231,58 @@ __global__ void __launch_bounds__(kStThreads) stream_down_kernel(
 
 // Un-sort + weighted sum: y[t] = ((0 + o_slot0) + o_slot1) + ... over the kept
 // slots, in slot order, then cast to the output dtype.  O16: the per-slot rows
-// are bf16 (bf16-output layers), else fp32.
+// are bf16 (bf16-output layers), else fp32.  A thread owns 8 channels of one
+// token: the token's row indices first, then all kept slots' loads (16 bytes
+// each for bf16 rows) in flight together, then the sum in slot order.
 template <bool O16>
 __global__ void combine_kernel(const void* __restrict__ o, const int32_t* __restrict__ ts2row,
-                               int k, int d, int out_dtype, void* __restrict__ y) {    pdl_wait();
+                               int k, int d, int out_dtype, void* __restrict__ y) {
+    pdl_wait();
     pdl_trigger();
 
     const int t = blockIdx.x;
-    const int n4 = blockIdx.y * blockDim.x + threadIdx.x;
-    if (n4 * 4 >= d) return;
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int s = 0; s < k; ++s) {
-        const int row = ts2row[(int64_t)t * k + s];
-        if (row < 0) continue;
-        float4 v;
+    const int n8 = blockIdx.y * blockDim.x + threadIdx.x;
+    if (n8 * 8 >= d) return;
+    int rows[kMaxK];
+#pragma unroll
+    for (int s = 0; s < kMaxK; ++s) rows[s] = s < k ? ts2row[(int64_t)t * k + s] : -1;
+    float v[kMaxK][8];
+#pragma unroll
+    for (int s = 0; s < kMaxK; ++s) {
+        if (rows[s] < 0) continue;
         if (O16) {
-            const uint2 b = reinterpret_cast<const uint2*>(reinterpret_cast<const uint16_t*>(o) + (int64_t)row * d)[n4];
-            v = make_float4(__uint_as_float(b.x << 16), __uint_as_float(b.x & 0xFFFF0000u),
-                            __uint_as_float(b.y << 16), __uint_as_float(b.y & 0xFFFF0000u));
+            const uint4 b =
+                reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(o) + (int64_t)rows[s] * d)[n8];
+            const uint32_t w[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                v[s][2 * i] = __uint_as_float(w[i] << 16);
+                v[s][2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+            }
         } else {
-            v = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(o) + (int64_t)row * d)[n4];
+            const float4* src = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(o) + (int64_t)rows[s] * d);
+            const float4 a = src[2 * n8], b = src[2 * n8 + 1];
+            v[s][0] = a.x; v[s][1] = a.y; v[s][2] = a.z; v[s][3] = a.w;
+            v[s][4] = b.x; v[s][5] = b.y; v[s][6] = b.z; v[s][7] = b.w;
         }
-        acc.x = __fadd_rn(acc.x, v.x);
-        acc.y = __fadd_rn(acc.y, v.y);
-        acc.z = __fadd_rn(acc.z, v.z);
-        acc.w = __fadd_rn(acc.w, v.w);
+    }
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int s = 0; s < kMaxK; ++s) {
+        if (rows[s] < 0) continue;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) acc[c] = __fadd_rn(acc[c], v[s][c]);
     }
     if (out_dtype == MOE_BF16) {
-        const uint2 p = make_uint2((uint32_t)f32_to_bf16_bits(acc.x) | ((uint32_t)f32_to_bf16_bits(acc.y) << 16),
-                                   (uint32_t)f32_to_bf16_bits(acc.z) | ((uint32_t)f32_to_bf16_bits(acc.w) << 16));
-        reinterpret_cast<uint2*>(reinterpret_cast<uint16_t*>(y) + (int64_t)t * d)[n4] = p;
+        uint32_t p[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            p[i] = (uint32_t)f32_to_bf16_bits(acc[2 * i]) | ((uint32_t)f32_to_bf16_bits(acc[2 * i + 1]) << 16);
+        reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(y) + (int64_t)t * d)[n8] = make_uint4(p[0], p[1], p[2], p[3]);
     } else {
-        reinterpret_cast<float4*>(reinterpret_cast<float*>(y) + (int64_t)t * d)[n4] = acc;
+        float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(y) + (int64_t)t * d);
+        dst[2 * n8] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+        dst[2 * n8 + 1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
     }
 }
 
@@ -317,7 +337,7 @@ cudaError_t launch_stream_down(const moe_w8a8_weights* w, int T, const int8_t* h
 
 cudaError_t launch_combine(const void* o, int o_bf16, const int32_t* ts2row, int T, int k, int d,
                            int out_dtype, void* y, cudaStream_t s) {
-    dim3 grid(T, (d / 4 + 255) / 256);
+    dim3 grid(T, (d / 8 + 255) / 256);
     if (o_bf16) return launch_pdl(combine_kernel<true>, grid, dim3(256), 0, s, o, ts2row, k, d, out_dtype, y);
     return launch_pdl(combine_kernel<false>, grid, dim3(256), 0, s, o, ts2row, k, d, out_dtype, y);
 }
