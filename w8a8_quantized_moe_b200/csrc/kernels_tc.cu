@@ -1197,18 +1197,20 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
 // ------------------------------------------------------------------ requantisation of h
 
 // One warp per sorted row: sh = max over the row's partial maxima / 127 and
-// codes rint(h / sh), ties to even, clamped to +-127 (sh = 0 gives 0).  The h
-// loads of a batch (up to 8 x 16 bytes per lane) are issued together with the
-// partial-maximum loads, before the reduction.
+// codes rint(h / sh), ties to even, clamped to +-127 (sh = 0 gives 0).  The
+// scale comes from the partial maxima, not from h, so a row's h loads (up to
+// kRqBatch x 16 bytes per lane) and its partial-maximum loads are issued
+// together: one memory round trip per row for f <= 2048.
 constexpr int kRqThreads = 256;
-constexpr int kRqBatch = 8;
+constexpr int kRqBatch = 16;
 
 template <int FMT>
 __global__ void __launch_bounds__(kRqThreads) requant_kernel(const float* __restrict__ h32,
                                                              const float* __restrict__ pamax, int f,
                                                              const int32_t* __restrict__ meta,
                                                              int8_t* __restrict__ hq,
-                                                             float* __restrict__ sh) {    pdl_wait();
+                                                             float* __restrict__ sh) {
+    pdl_wait();
     pdl_trigger();
 
     const int lane = threadIdx.x & 31;
