@@ -218,7 +218,7 @@ moe_status moe_w8a8_forward_host(const moe_w8a8_weights* w, const void* x_host, 
  * T is limited by the array: a call whose moe_w8a8_workspace_size(w, T)
  * exceeds MOE_NOALLOC_SCRATCH_BYTES returns MOE_ERR_WORKSPACE_TOO_SMALL and
  * enqueues nothing (for the d=4096, E=64, top-4, f=1536 decode layer that is
- * T up to 62 tokens).
+ * T up to 82 tokens).
  * The first call on a device looks up the array's device address with that
  * device current (cudaGetSymbolAddress) and caches it; make that first call
  * before any stream capture.  Every call on a device shares the one array,

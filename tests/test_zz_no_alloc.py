@@ -75,16 +75,21 @@ def test_noalloc_forward_matches_workspace_forward_decode(M, decode_handle):
 
 
 def test_noalloc_largest_decode_batch_and_the_first_refused(M, decode_handle):
-    """The decode layer's largest batch that fits the array (62 tokens) runs
-    and matches; 63 tokens do not fit and are refused before anything runs."""
+    """The decode layer's largest batch that fits the array (82 tokens, as the
+    header states) runs and matches; one more token does not fit and is
+    refused before anything runs."""
     import torch
     wl, W = decode_handle
-    assert M.moe_w8a8_workspace_size(W, 62) <= M.MOE_NOALLOC_SCRATCH_BYTES < M.moe_w8a8_workspace_size(W, 63)
-    _check_against_workspace_forward(M, W, wl, synth.make_data(wl, T=62), 62)
-    data = synth.make_data(wl, T=63)
-    y = torch.zeros((63, wl.d), dtype=torch.bfloat16, device="cuda")
+    t_max = 1
+    while M.moe_w8a8_workspace_size(W, t_max + 1) <= M.MOE_NOALLOC_SCRATCH_BYTES:
+        t_max += 1
+    assert t_max == 82, f"the header states 82 tokens for this layer; the array now fits {t_max}"
+    _check_against_workspace_forward(M, W, wl, synth.make_data(wl, T=t_max), t_max)
+    T = t_max + 1
+    data = synth.make_data(wl, T=T)
+    y = torch.zeros((T, wl.d), dtype=torch.bfloat16, device="cuda")
     with pytest.raises(M.MoeError) as e:
-        M.moe_w8a8_forward_noalloc(W, H.x_tensor(wl, data), 63, None, H.to_dev(data.router_logits), y)
+        M.moe_w8a8_forward_noalloc(W, H.x_tensor(wl, data), T, None, H.to_dev(data.router_logits), y)
     assert e.value.status == M.MOE_ERR_WORKSPACE_TOO_SMALL
 
 

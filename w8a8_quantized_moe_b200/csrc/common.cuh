@@ -177,13 +177,6 @@ __device__ __forceinline__ void load8_act(const void* x, int64_t idx, int in_dty
     }
 }
 
-// The GPU's global nanosecond timer (bounds on waits).
-__device__ __forceinline__ uint64_t globaltimer_ns() {
-    uint64_t t;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-    return t;
-}
-
 // Programmatic dependent launch: every kernel of a forward lets the next one be
 // scheduled as soon as it starts (trigger) and waits for the previous kernel's
 // results before touching any shared buffer (wait).  Both are no-ops for a

@@ -136,21 +136,12 @@ cudaError_t launch_route_small(const float* logits, const float* bias, int T, in
 cudaError_t launch_smooth_quant(const void* x, int in_dtype, const float* inv_s, float act_clip, int T,
                                 int d, int k, const int32_t* ts2row, int8_t* xq, float* sx, int8_t* aq,
                                 int64_t aq_ld, const float* wts, const int32_t* idx, int fmt, cudaStream_t s);
-// Large batches on the tensor path: one warp per token, X rows staged by bulk
-// copies (no expert-parallel trailer).  _ok: d and the input dtype fit its
-// shared-memory ring.
-bool smooth_quant_rows_ok(int d, int in_dtype);
-cudaError_t launch_smooth_quant_rows(const void* x, int in_dtype, const float* inv_s, float act_clip, int T, int d,
-                                     int k, const int32_t* ts2row, int8_t* xq, float* sx, int8_t* aq, int64_t aq_ld,
-                                     int fmt, int num_sms, int32_t* status, cudaStream_t s);
 // Expert-parallel receive side.  Local expert of each received row (its
 // trailer's expert - ep_first); an expert outside [0, n_local) is recorded in
 // status (MOE_ERR_INVALID_ARG, site kSiteEpExpert) and the row runs through
 // local expert 0.
 constexpr int kSiteEpExpert = 14;
-// Status site of the large-batch quantisation kernel: a bulk copy of an X row
-// did not land within 2 s (words 2-3: block, token).
-constexpr int kSiteQuantCopy = 15;
+
 cudaError_t launch_ep_read_experts(const uint8_t* recv, int R, int64_t row_bytes, int d, int ep_first,
                                    int n_local, int32_t* idx, int32_t* status, cudaStream_t s);
 // Codes of received row r to row ts2row[r] of dst (row r when ts2row is
@@ -185,7 +176,6 @@ cudaError_t launch_router_select(const moe_w8a8_weights* w, const void* x, int T
                                  const float* bias, float* sel, int32_t* idx, float* wts, float* logits_out,
                                  cudaStream_t s);
 constexpr int kRouterTcMinTokens = 1024;   // the certified router runs from this many tokens up
-constexpr int kQuantRowsMinTokens = 1024;   // the warp-per-token quantisation kernel from this many tokens up
 bool tc_supported(const moe_w8a8_config& c);
 // n_mma back-to-back M=128 N=256 K=32 8-bit MMAs per CTA on `grid` CTAs
 // (operands resident in shared memory): the tensor pipe's own rate.

@@ -871,163 +871,6 @@ __global__ void __launch_bounds__(kSqThreads) smooth_quant_kernel(
     }
 }
 
-// Smoothed per-token quantisation for large batches on the tensor-core path
-// (same arithmetic as smooth_quant_kernel).  One warp per token; persistent
-// blocks of kSqrWarps warps.  Each warp streams its tokens' X rows into a
-// ring of `stages` row buffers in shared memory with bulk copies (the next
-// rows are in flight while it quantises the current one), inv_s is staged
-// once per block.  Pass 1 over the staged row: the range max |x inv_s| (warp
-// max); pass 2: the codes, stored to each kept (t, slot) row of the sorted
-// matrix (and to xq[t] when given), 8 bytes per lane per group of 8 channels,
-// so a warp writes 256 contiguous bytes per store instruction.  X is an
-// input: the first copies are issued before the routing wait.  The copies'
-// barriers are waited for with a bound (the status word records a timeout).
-constexpr int kSqrWarps = 8;
-
-__device__ __forceinline__ void bulk_copy_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
-    asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-            (uint32_t)__cvta_generic_to_shared(dst)),
-        "l"(src), "r"(bytes), "r"((uint32_t)__cvta_generic_to_shared(bar))
-        : "memory");
-}
-__device__ __forceinline__ void mbar_init_sq(uint64_t* bar) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"((uint32_t)__cvta_generic_to_shared(bar)));
-}
-__device__ __forceinline__ void mbar_expect_tx_sq(uint64_t* bar, uint32_t bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(
-                     (uint32_t)__cvta_generic_to_shared(bar)),
-                 "r"(bytes)
-                 : "memory");
-}
-__device__ __forceinline__ bool mbar_test_sq(uint64_t* bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}\n"
-        : "=r"(ok)
-        : "r"((uint32_t)__cvta_generic_to_shared(bar)), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-
-// 8 consecutive staged activations (bf16 or fp32) times inv_s, as fp32.
-__device__ __forceinline__ void smoothed8(const uint8_t* row, const float* s_inv, int g, int in_dtype, float v[8]) {
-    if (in_dtype == MOE_BF16) {
-        const uint4 raw = reinterpret_cast<const uint4*>(row)[g];
-        const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            v[2 * i] = __uint_as_float(w[i] << 16);
-            v[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
-        }
-    } else {
-        const float4 a = reinterpret_cast<const float4*>(row)[2 * g];
-        const float4 b = reinterpret_cast<const float4*>(row)[2 * g + 1];
-        v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
-        v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
-    }
-    const float4 s0 = reinterpret_cast<const float4*>(s_inv)[2 * g];
-    const float4 s1 = reinterpret_cast<const float4*>(s_inv)[2 * g + 1];
-    const float sv[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
-#pragma unroll
-    for (int c = 0; c < 8; ++c) v[c] = __fmul_rn(v[c], sv[c]);
-}
-
-template <int FMT>
-__global__ void __launch_bounds__(kSqrWarps * 32, 1) smooth_quant_rows_kernel(
-    const void* __restrict__ x, int in_dtype, const float* __restrict__ inv_s, float act_clip, int T, int d,
-    int k, int stages, const int32_t* __restrict__ ts2row, int8_t* __restrict__ xq, float* __restrict__ sx,
-    int8_t* __restrict__ aq, int64_t aq_ld, int32_t* __restrict__ status) {
-    extern __shared__ __align__(16) uint8_t smem_raw[];
-    float* s_inv = reinterpret_cast<float*>(smem_raw);
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem_raw + (size_t)d * 4);
-    const uint32_t row_bytes = (uint32_t)d * (in_dtype == MOE_BF16 ? 2u : 4u);
-    uint8_t* rows = smem_raw + (size_t)d * 4 + 128 * ((kSqrWarps * stages * 8 + 127) / 128);
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    uint64_t* wbar = bars + warp * stages;
-    uint8_t* wrows = rows + (size_t)warp * stages * row_bytes;
-    const int gw = blockIdx.x * kSqrWarps + warp, nw = gridDim.x * kSqrWarps;
-    const uint8_t* xb = reinterpret_cast<const uint8_t*>(x);
-
-    if (lane == 0) {
-        for (int st = 0; st < stages; ++st) mbar_init_sq(&wbar[st]);
-        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-        for (int st = 0; st < stages; ++st) {
-            const int t = gw + st * nw;
-            if (t < T) {
-                mbar_expect_tx_sq(&wbar[st], row_bytes);
-                bulk_copy_g2s(wrows + (size_t)st * row_bytes, xb + (size_t)t * row_bytes, row_bytes, &wbar[st]);
-            }
-        }
-    }
-    for (int i = threadIdx.x; i < d / 4; i += blockDim.x)
-        reinterpret_cast<float4*>(s_inv)[i] = reinterpret_cast<const float4*>(inv_s)[i];
-    __syncthreads();
-    pdl_wait();   // the routing of this forward (ts2row) is complete from here on
-    pdl_trigger();
-
-    const int ng = d / 8;
-    int st = 0;
-    uint32_t ph = 0;
-    for (int t = gw; t < T; t += nw) {
-        if (!mbar_test_sq(&wbar[st], ph)) {
-            const uint64_t t0 = globaltimer_ns();
-            while (!mbar_test_sq(&wbar[st], ph)) {
-                if (globaltimer_ns() - t0 > 2000000000ull) {
-                    if (lane == 0 && atomicCAS(status, 0, (int32_t)MOE_ERR_TIMEOUT) == 0) {
-                        status[1] = kSiteQuantCopy;
-                        status[2] = (int32_t)blockIdx.x;
-                        status[3] = t;
-                    }
-                    return;
-                }
-            }
-        }
-        const uint8_t* row = wrows + (size_t)st * row_bytes;
-        float m = 0.0f;
-        for (int g = lane; g < ng; g += 32) {
-            float v[8];
-            smoothed8(row, s_inv, g, in_dtype, v);
-#pragma unroll
-            for (int c = 0; c < 8; ++c) m = fmaxf(m, fabsf(v[c]));
-        }
-        m = warp_max(m);
-        if (act_clip > 0.0f) m = fminf(m, act_clip);   // saturating clip: values beyond it go to +-127
-        const float s = m > 0.0f ? __fdiv_rn(m, fmt_qmax<FMT>()) : 0.0f;
-        const float rs = s > 0.0f ? __frcp_rn(s) : 0.0f;
-        if (lane == 0) sx[t] = s;
-        int myrow = lane < k ? ts2row[(int64_t)t * k + lane] : -1;
-        int rws[kMaxK];
-#pragma unroll
-        for (int sl = 0; sl < kMaxK; ++sl) rws[sl] = __shfl_sync(0xffffffffu, myrow, sl);
-        for (int g = lane; g < ng; g += 32) {
-            float v[8];
-            smoothed8(row, s_inv, g, in_dtype, v);
-            int q[8];
-#pragma unroll
-            for (int c = 0; c < 8; ++c) q[c] = s > 0.0f ? (int)fmt_code<FMT>(v[c], s, rs) : 0;
-            const uint2 packed = make_uint2(pack4(q[0], q[1], q[2], q[3]), pack4(q[4], q[5], q[6], q[7]));
-            if (xq) *reinterpret_cast<uint2*>(xq + (int64_t)t * d + g * 8) = packed;
-#pragma unroll
-            for (int sl = 0; sl < kMaxK; ++sl)
-                if (rws[sl] >= 0) *reinterpret_cast<uint2*>(aq + (int64_t)rws[sl] * aq_ld + g * 8) = packed;
-        }
-        // every lane has read this buffer: refill it with the warp's token `stages` turns ahead
-        __syncwarp();
-        if (lane == 0) {
-            const int t2 = t + stages * nw;
-            if (t2 < T) {
-                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-                mbar_expect_tx_sq(&wbar[st], row_bytes);
-                bulk_copy_g2s(wrows + (size_t)st * row_bytes, xb + (size_t)t2 * row_bytes, row_bytes, &wbar[st]);
-            }
-        }
-        if (++st == stages) { st = 0; ph ^= 1; }
-    }
-}
-
 // Expert-parallel receive side: the local expert of each received row.
 __global__ void ep_read_experts_kernel(const uint8_t* __restrict__ recv, int R, int64_t row_bytes, int d,
                                        int ep_first, int n_local, int32_t* __restrict__ idx,
@@ -1165,36 +1008,6 @@ cudaError_t launch_smooth_quant(const void* x, int in_dtype, const float* inv_s,
                                    : groups <= 8 ? smooth_quant_kernel<8, FMT_INT8> : smooth_quant_kernel<16, FMT_INT8>);
     return launch_pdl(kern, dim3(T), dim3(kSqThreads), 0, s, x, in_dtype, inv_s, act_clip, T, d, k, ts2row, xq,
                       sx, aq, aq_ld, wts, idx);
-}
-
-// Shared memory of smooth_quant_rows_kernel for `stages` row buffers per warp.
-static size_t sq_rows_smem(int d, int in_dtype, int stages) {
-    const size_t row_bytes = (size_t)d * (in_dtype == MOE_BF16 ? 2 : 4);
-    return (size_t)d * 4 + 128 * ((kSqrWarps * stages * 8 + 127) / 128) + (size_t)kSqrWarps * stages * row_bytes;
-}
-
-constexpr size_t kSqrSmemMax = 224 * 1024;
-
-bool smooth_quant_rows_ok(int d, int in_dtype) { return sq_rows_smem(d, in_dtype, 1) <= kSqrSmemMax; }
-
-cudaError_t launch_smooth_quant_rows(const void* x, int in_dtype, const float* inv_s, float act_clip, int T, int d,
-                                     int k, const int32_t* ts2row, int8_t* xq, float* sx, int8_t* aq, int64_t aq_ld,
-                                     int fmt, int num_sms, int32_t* status, cudaStream_t s) {
-    int stages = 3;
-    while (stages > 1 && sq_rows_smem(d, in_dtype, stages) > kSqrSmemMax) --stages;
-    const size_t smem = sq_rows_smem(d, in_dtype, stages);
-    static std::atomic<uint64_t> a8{0}, af8{0};
-    const int grid = std::max(1, std::min(num_sms, (T + kSqrWarps - 1) / kSqrWarps));
-    if (fmt == FMT_E4M3) {
-        cudaError_t e = smem_attr_once(smooth_quant_rows_kernel<FMT_E4M3>, kSqrSmemMax, af8);
-        if (e != cudaSuccess) return e;
-        return launch_pdl(smooth_quant_rows_kernel<FMT_E4M3>, dim3(grid), dim3(kSqrWarps * 32), smem, s, x, in_dtype,
-                          inv_s, act_clip, T, d, k, stages, ts2row, xq, sx, aq, aq_ld, status);
-    }
-    cudaError_t e = smem_attr_once(smooth_quant_rows_kernel<FMT_INT8>, kSqrSmemMax, a8);
-    if (e != cudaSuccess) return e;
-    return launch_pdl(smooth_quant_rows_kernel<FMT_INT8>, dim3(grid), dim3(kSqrWarps * 32), smem, s, x, in_dtype,
-                      inv_s, act_clip, T, d, k, stages, ts2row, xq, sx, aq, aq_ld, status);
 }
 
 cudaError_t launch_ep_read_experts(const uint8_t* recv, int R, int64_t row_bytes, int d, int ep_first,

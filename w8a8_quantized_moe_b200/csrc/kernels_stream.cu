@@ -246,32 +246,41 @@ __global__ void combine_kernel(const void* __restrict__ o, const int32_t* __rest
     int rows[kMaxK];
 #pragma unroll
     for (int s = 0; s < kMaxK; ++s) rows[s] = s < k ? ts2row[(int64_t)t * k + s] : -1;
-    float v[kMaxK][8];
+    // loads of every kept slot first (raw 16-byte words: few registers, so many
+    // warps per SM), then the sum in slot order
+    uint4 raw[kMaxK][O16 ? 1 : 2];
 #pragma unroll
     for (int s = 0; s < kMaxK; ++s) {
         if (rows[s] < 0) continue;
         if (O16) {
-            const uint4 b =
-                reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(o) + (int64_t)rows[s] * d)[n8];
-            const uint32_t w[4] = {b.x, b.y, b.z, b.w};
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                v[s][2 * i] = __uint_as_float(w[i] << 16);
-                v[s][2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
-            }
+            raw[s][0] = reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(o) + (int64_t)rows[s] * d)[n8];
         } else {
-            const float4* src = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(o) + (int64_t)rows[s] * d);
-            const float4 a = src[2 * n8], b = src[2 * n8 + 1];
-            v[s][0] = a.x; v[s][1] = a.y; v[s][2] = a.z; v[s][3] = a.w;
-            v[s][4] = b.x; v[s][5] = b.y; v[s][6] = b.z; v[s][7] = b.w;
+            const uint4* src = reinterpret_cast<const uint4*>(reinterpret_cast<const float*>(o) + (int64_t)rows[s] * d);
+            raw[s][0] = src[2 * n8];
+            raw[s][O16 ? 0 : 1] = src[2 * n8 + 1];
         }
     }
     float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int s = 0; s < kMaxK; ++s) {
         if (rows[s] < 0) continue;
+        float v[8];
+        if (O16) {
+            const uint32_t w[4] = {raw[s][0].x, raw[s][0].y, raw[s][0].z, raw[s][0].w};
 #pragma unroll
-        for (int c = 0; c < 8; ++c) acc[c] = __fadd_rn(acc[c], v[s][c]);
+            for (int i = 0; i < 4; ++i) {
+                v[2 * i] = __uint_as_float(w[i] << 16);
+                v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+            }
+        } else {
+            const uint32_t w[8] = {raw[s][0].x, raw[s][0].y, raw[s][0].z, raw[s][0].w,
+                                   raw[s][O16 ? 0 : 1].x, raw[s][O16 ? 0 : 1].y, raw[s][O16 ? 0 : 1].z,
+                                   raw[s][O16 ? 0 : 1].w};
+#pragma unroll
+            for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(w[i]);
+        }
+#pragma unroll
+        for (int c = 0; c < 8; ++c) acc[c] = __fadd_rn(acc[c], v[c]);
     }
     if (out_dtype == MOE_BF16) {
         uint32_t p[4];

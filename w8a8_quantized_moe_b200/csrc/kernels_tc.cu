@@ -298,13 +298,16 @@ __device__ __forceinline__ void store_rows32_bf16(float* stage, const uint32_t (
 // rows (its TMEM lane quarter) and 64 of the 128 h columns.
 // Release of an accumulator buffer by one epilogue warp: a local arrive, or,
 // for a CTA pair, an arrive on the pair leader's barrier (same offset in the
-// leader's shared memory), which counts the warps of both CTAs.
+// leader's shared memory), which counts the warps of both CTAs.  Only the
+// warp's tensor-memory reads must precede it (tcgen05.wait::ld and the
+// before-thread-sync fence); the default CTA-scope semantics of the arrive do
+// not make it wait for the warp's outstanding global stores.
 template <bool PAIR>
 __device__ __forceinline__ void release_acc(uint64_t* bar) {
     if (PAIR) {
         uint32_t remote;
         asm volatile("mapa.shared::cluster.u32 %0, %1, 0;" : "=r"(remote) : "r"(smem_u32(bar)));
-        asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(remote) : "memory");
+        asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(remote) : "memory");
     } else {
         mbar_arrive(bar);
     }
@@ -1200,9 +1203,11 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
 // codes rint(h / sh), ties to even, clamped to +-127 (sh = 0 gives 0).  The
 // scale comes from the partial maxima, not from h, so a row's h loads (up to
 // kRqBatch x 16 bytes per lane) and its partial-maximum loads are issued
-// together: one memory round trip per row for f <= 2048.
+// together; further batches follow (f = 1536: 12 x 16 bytes per lane in two
+// batches).  A small batch keeps the registers, and so the warps per SM that
+// hide the per-element arithmetic, in balance with the bytes in flight.
 constexpr int kRqThreads = 256;
-constexpr int kRqBatch = 16;
+constexpr int kRqBatch = 8;
 
 template <int FMT>
 __global__ void __launch_bounds__(kRqThreads) requant_kernel(const float* __restrict__ h32,

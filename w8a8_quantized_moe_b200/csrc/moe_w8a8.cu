@@ -483,15 +483,6 @@ moe_status quant_stage(Run& r, const void* x, int T, int8_t* aq, int64_t aq_ld, 
     // the tensor path and the expert-parallel send rows use the sorted copies
     const bool need_xq = !aq || (r.dbg && r.dbg->xq);
     r.mark(MOE_STAGE_QUANT, 0);
-    if (aq && !trailer && T >= kQuantRowsMinTokens && smooth_quant_rows_ok(c.d, c.in_dtype)) {
-        // large batches on the tensor path: warp per token, bulk-copied X rows
-        CUDA_TRY(launch_smooth_quant_rows(x, c.in_dtype, w->inv_s, w->act_clip, T, c.d, c.top_k,
-                                          r.at<int32_t>(L.ts2row), need_xq ? r.at<int8_t>(L.xq) : nullptr,
-                                          r.at<float>(L.sx), aq, aq_ld, fmt, w->num_sms, w->status, r.s));
-        r.mark(MOE_STAGE_QUANT, 1);
-        ++r.launches;
-        return MOE_OK;
-    }
     CUDA_TRY(launch_smooth_quant(x, c.in_dtype, w->inv_s, w->act_clip, T, c.d, c.top_k, r.at<int32_t>(L.ts2row),
                                  need_xq ? r.at<int8_t>(L.xq) : nullptr, r.at<float>(L.sx), aq, aq_ld,
                                  trailer ? r.at<float>(L.topk_w) : nullptr,
