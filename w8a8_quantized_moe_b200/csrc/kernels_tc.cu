@@ -48,7 +48,8 @@ constexpr int kEpiWarps = 8;
 constexpr int kThreads = 64 + kEpiWarps * 32;     // 320
 constexpr uint32_t kTmemCols = 2 * BN;            // two 256-column accumulators
 constexpr uint64_t kWaitBudgetNs = 2000000000ull; // 2 s per wait
-constexpr int kEpiStageBytes = 16 * 32 * 4;      // 16 rows x 32 fp32 per epilogue warp
+constexpr int kEpiStoreBytes = 16 * 32 * 4;      // 16 rows x 32 fp32 per epilogue warp (store staging)
+constexpr int kEpiStageBytes = kEpiStoreBytes + 512;   // + the tile's 128 column scales
 constexpr size_t kSmemBytes = (size_t)kStages * kStageBytes + (size_t)kEpiWarps * kEpiStageBytes + 1024 + 256;
 
 
@@ -293,9 +294,6 @@ __device__ __forceinline__ void store_rows32_bf16(float* stage, const uint32_t (
     __syncwarp();
 }
 
-// GEMM1 tile: columns 0..127 of the accumulator are gate channels
-// nt*128 + c, columns 128..255 the matching up channels.  Each warp owns 32
-// rows (its TMEM lane quarter) and 64 of the 128 h columns.
 // Release of an accumulator buffer by one epilogue warp: a local arrive, or,
 // for a CTA pair, an arrive on the pair leader's barrier (same offset in the
 // leader's shared memory), which counts the warps of both CTAs.  Only the
@@ -313,15 +311,41 @@ __device__ __forceinline__ void release_acc(uint64_t* bar) {
     }
 }
 
+// The per-tile inputs of an epilogue warp, fetched before it waits for the
+// accumulator so that their memory latency overlaps the tile's MMAs: the
+// scalars of its lane's row (GEMM1: the token's activation scale; GEMM2: the
+// row's h scale and routing weight) into registers, and the 128 column scales
+// of its half tile into its slice `sc` of shared memory (GEMM1: 64 gate then
+// 64 up scales of its 64 h channels; GEMM2: the scales of its 128 output
+// columns), one 16-byte load per lane.
+template <int EPI>
+__device__ __forceinline__ void epi_prefetch(const TcParams& p, int e, int nt, int half, int grow, bool valid,
+                                             float* sc, int lane, float& r0, float& r1) {
+    if (EPI == EPI_SWIGLU) {
+        const float* base = (lane < 16 ? p.sw0 : p.sw1) + (int64_t)e * p.f + nt * 128 + 64 * half;
+        reinterpret_cast<float4*>(sc)[lane] = reinterpret_cast<const float4*>(base)[lane & 15];
+        r0 = valid ? p.sx[p.row2ts[grow] / p.k] : 0.0f;
+        r1 = 0.0f;
+    } else {
+        const float* base = p.sw0 + (int64_t)e * p.N + nt * BN + 128 * half;
+        reinterpret_cast<float4*>(sc)[lane] = reinterpret_cast<const float4*>(base)[lane];
+        r0 = valid ? p.sh[grow] : 0.0f;
+        r1 = valid ? p.topk_w[p.row2ts[grow]] : 0.0f;
+    }
+    __syncwarp();
+}
+
+// GEMM1 tile: columns 0..127 of the accumulator are gate channels
+// nt*128 + c, columns 128..255 the matching up channels.  Each warp owns 32
+// rows (its TMEM lane quarter) and 64 of the 128 h columns.  sc, sxt: from
+// epi_prefetch<EPI_SWIGLU>.
 template <int FMT, bool PAIR = false>
 __device__ __forceinline__ void epilogue_swiglu(const TcParams& p, uint32_t taddr, int half, int e,
-                                                int nt, int wrow0, int nvalid, float* stage,
-                                                uint64_t* acc_empty, int lane) {
+                                                int nt, int wrow0, int nvalid, float* stage, const float* sc,
+                                                float sxt, uint64_t* acc_empty, int lane) {
     const int f = p.f;
     const bool valid = lane < nvalid;
     const int grow = wrow0 + lane;
-    float sxt = 0.0f;
-    if (valid) sxt = p.sx[p.row2ts[grow] / p.k];
     float amax = 0.0f;
 #pragma unroll 1
     for (int c = 0; c < 2; ++c) {
@@ -336,8 +360,8 @@ __device__ __forceinline__ void epilogue_swiglu(const TcParams& p, uint32_t tadd
             if (lane == 0) release_acc<PAIR>(acc_empty);
         }
         const int ch0 = nt * 128 + col0;
-        const float* swg = p.sw0 + (int64_t)e * f + ch0;
-        const float* swu = p.sw1 + (int64_t)e * f + ch0;
+        const float* swg = sc + 32 * c;
+        const float* swu = sc + 64 + 32 * c;
         if (p.acc_dbg && valid) {
             int32_t* dg = p.acc_dbg + (int64_t)grow * 2 * f + ch0;
             for (int j = 0; j < 32; ++j) {
@@ -365,18 +389,15 @@ __device__ __forceinline__ void epilogue_swiglu(const TcParams& p, uint32_t tadd
     if (valid) p.pamax[(int64_t)grow * (f / 64) + nt * 2 + half] = amax;
 }
 
+// GEMM2 tile: each warp owns 32 rows and 128 of the 256 output columns.  sc,
+// shr, wr: from epi_prefetch<EPI_DOWN>.
 template <int FMT, bool PAIR = false>
 __device__ __forceinline__ void epilogue_down(const TcParams& p, uint32_t taddr, int half, int e,
-                                              int nt, int wrow0, int nvalid, float* stage, uint64_t* acc_empty,
-                                              int lane) {
+                                              int nt, int wrow0, int nvalid, float* stage, const float* sc,
+                                              float shr, float wr, uint64_t* acc_empty, int lane) {
     const int d = p.N;
     const bool valid = lane < nvalid;
     const int grow = wrow0 + lane;
-    float shr = 0.0f, wr = 0.0f;
-    if (valid) {
-        shr = p.sh[grow];
-        wr = p.topk_w[p.row2ts[grow]];
-    }
 #pragma unroll 1
     for (int c = 0; c < 4; ++c) {
         const int col0 = 128 * half + 32 * c;
@@ -389,7 +410,7 @@ __device__ __forceinline__ void epilogue_down(const TcParams& p, uint32_t taddr,
             if (lane == 0) release_acc<PAIR>(acc_empty);
         }
         const int ch0 = nt * BN + col0;
-        const float* sw = p.sw0 + (int64_t)e * d + ch0;
+        const float* sw = sc + 32 * c;
         if (p.acc_dbg && valid) {
             int32_t* da = p.acc_dbg + (int64_t)grow * d + ch0;
             for (int j = 0; j < 32; ++j) da[j] = (int32_t)a[j];
@@ -524,19 +545,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         float* stage = epi_stage + ew * (kEpiStageBytes / 4);
         int buf = 0;
         uint32_t aph = 0;
+        float* sc = stage + kEpiStoreBytes / 4;
         for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
-            if (!mbar_wait(&ctl->acc_full[buf], aph, abort, p.status, 4, t)) break;
-            tc_fence_after();
             const int mt = t / p.n_tiles_n, nt = t % p.n_tiles_n;
             const int e = p.tiles[2 * mt], row0 = p.tiles[2 * mt + 1];
             const int nrows = min(BM, p.offsets[e + 1] - row0);
             const int wrow0 = row0 + quad * 32;                      // this warp's 32 rows
             const int nvalid = max(0, min(32, nrows - quad * 32));
+            float r0, r1;
+            epi_prefetch<EPI>(p, e, nt, half, wrow0 + lane, lane < nvalid, sc, lane, r0, r1);
+            if (!mbar_wait(&ctl->acc_full[buf], aph, abort, p.status, 4, t)) break;
+            tc_fence_after();
             const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(buf * BN);
             if (EPI == EPI_SWIGLU)
-                epilogue_swiglu<FMT>(p, taddr, half, e, nt, wrow0, nvalid, stage, &ctl->acc_empty[buf], lane);
+                epilogue_swiglu<FMT>(p, taddr, half, e, nt, wrow0, nvalid, stage, sc, r0, &ctl->acc_empty[buf], lane);
             else
-                epilogue_down<FMT>(p, taddr, half, e, nt, wrow0, nvalid, stage, &ctl->acc_empty[buf], lane);
+                epilogue_down<FMT>(p, taddr, half, e, nt, wrow0, nvalid, stage, sc, r0, r1, &ctl->acc_empty[buf],
+                                   lane);
             buf ^= 1;
             if (buf == 0) aph ^= 1;
         }
@@ -810,19 +835,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         float* stage = epi_stage + ew * (kEpiStageBytes / 4);
         int buf = 0;
         uint32_t aph = 0;
+        float* sc = stage + kEpiStoreBytes / 4;
         for (int t = cid; t < num_tiles; t += ncl) {
-            if (!mbar_wait(&ctl->acc_full[buf], aph, abort, p.status, 4, t)) break;
-            tc_fence_after();
             const int mt = t / p.n_tiles_n, nt = t % p.n_tiles_n;
             const int e = p.pairs[2 * mt], row0 = p.pairs[2 * mt + 1] + rank * BM;
             const int nrows = min(BM, p.offsets[e + 1] - row0);
             const int wrow0 = row0 + quad * 32;
             const int nvalid = max(0, min(32, nrows - quad * 32));
+            float r0, r1;
+            epi_prefetch<EPI>(p, e, nt, half, wrow0 + lane, lane < nvalid, sc, lane, r0, r1);
+            if (!mbar_wait(&ctl->acc_full[buf], aph, abort, p.status, 4, t)) break;
+            tc_fence_after();
             const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(buf * BN);
             if (EPI == EPI_SWIGLU)
-                epilogue_swiglu<FMT, true>(p, taddr, half, e, nt, wrow0, nvalid, stage, &ctl->acc_empty[buf], lane);
+                epilogue_swiglu<FMT, true>(p, taddr, half, e, nt, wrow0, nvalid, stage, sc, r0,
+                                           &ctl->acc_empty[buf], lane);
             else
-                epilogue_down<FMT, true>(p, taddr, half, e, nt, wrow0, nvalid, stage, &ctl->acc_empty[buf], lane);
+                epilogue_down<FMT, true>(p, taddr, half, e, nt, wrow0, nvalid, stage, sc, r0, r1,
+                                         &ctl->acc_empty[buf], lane);
             buf ^= 1;
             if (buf == 0) aph ^= 1;
         }
@@ -1145,6 +1175,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
         const int quad = warp & 3;
         const int half = ew >> 2;
         float* stage = epi_stage + ew * (kEpiStageBytes / 4);
+        float* sc = stage + kEpiStoreBytes / 4;
         int buf = 0;
         uint32_t aph = 0;
         int q = 0;
@@ -1156,8 +1187,6 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
             if (lane == 0) mbar_arrive(&ring->empty[q]);
             if (++q == kTileRing) { q = 0; rph ^= 1; }
             if (t < 0) break;
-            if (!mbar_wait(&ctl->acc_full[buf], aph, abort, p1.status, 4, t)) break;
-            tc_fence_after();
             bool g1;
             int mt, nt;
             decode(t, g1, mt, nt);
@@ -1166,9 +1195,20 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
             const int nrows = min(BM, p.offsets[e + 1] - row0);
             const int wrow0 = row0 + quad * 32;
             const int nvalid = max(0, min(32, nrows - quad * 32));
+            float r0, r1;
+            if (g1) {
+                epi_prefetch<EPI_SWIGLU>(p1, e, nt, half, wrow0 + lane, lane < nvalid, sc, lane, r0, r1);
+            } else {
+                // the h scales this epilogue reads were released with the m-tile's ready flag,
+                // which the tile's producer waited for before loading its h codes
+                (void)ld_acquire(fx.ready + mt);
+                epi_prefetch<EPI_DOWN>(p2, e, nt, half, wrow0 + lane, lane < nvalid, sc, lane, r0, r1);
+            }
+            if (!mbar_wait(&ctl->acc_full[buf], aph, abort, p1.status, 4, t)) break;
+            tc_fence_after();
             const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(buf * BN);
             if (g1) {
-                epilogue_swiglu<FMT>(p1, taddr, half, e, nt, wrow0, nvalid, stage, &ctl->acc_empty[buf], lane);
+                epilogue_swiglu<FMT>(p1, taddr, half, e, nt, wrow0, nvalid, stage, sc, r0, &ctl->acc_empty[buf], lane);
                 // this warp's share of the tile is stored: count it; the last arrival requantises
                 __threadfence();
                 __syncwarp();
@@ -1181,8 +1221,8 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
                     st_release(fx.queue + slot, mt + 1);
                 }
             } else {
-                (void)ld_acquire(fx.ready + mt);   // the h scales this epilogue reads were released there
-                epilogue_down<FMT>(p2, taddr, half, e, nt, wrow0, nvalid, stage, &ctl->acc_empty[buf], lane);
+                epilogue_down<FMT>(p2, taddr, half, e, nt, wrow0, nvalid, stage, sc, r0, r1, &ctl->acc_empty[buf],
+                                   lane);
             }
             buf ^= 1;
             if (buf == 0) aph ^= 1;
