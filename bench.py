@@ -614,6 +614,14 @@ def measure(args, wl, world, rank, local, e2e_on=True, wts=None):
     step_s = ms_total / K / 1e3
     layer_gbs = alg["layer_bytes"] / step_s / 1e9
     layer_tops = alg["int8_ops"] / step_s / 1e12
+    if roof is not None:
+        # the whole layer step against the same bound (roofline.frac is the dominant kernel's)
+        if roof["bound"] == "hbm":
+            roof["layer"] = {"achieved": layer_gbs, "frac": layer_gbs / peaks["hbm_gbs"], "unit": "GB/s",
+                             "algorithmic_bytes_per_step": alg["layer_bytes"]}
+        else:
+            roof["layer"] = {"achieved": layer_tops, "frac": layer_tops / int8_peak, "unit": "TOPS",
+                             "int8_ops_per_step": alg["int8_ops"]}
     out = {
         "value": world * T * K / (ms_total / 1e3), "ms_per_step": ms_total / K,
         "config": {"workload": describe(wl), "T": T, "d": wl.d, "E": wl.E, "k": wl.k, "f": wl.f,
