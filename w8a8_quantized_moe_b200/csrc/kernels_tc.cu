@@ -1199,9 +1199,23 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
             if (g1) {
                 epi_prefetch<EPI_SWIGLU>(p1, e, nt, half, wrow0 + lane, lane < nvalid, sc, lane, r0, r1);
             } else {
-                // the h scales this epilogue reads were released with the m-tile's ready flag,
-                // which the tile's producer waited for before loading its h codes
-                (void)ld_acquire(fx.ready + mt);
+                // the h scales this epilogue reads are released with the m-tile's ready flag:
+                // wait for it (bounded) before fetching them
+                int rdy = 0;
+                if (lane == 0) {
+                    const uint64_t t0 = global_timer();
+                    while ((rdy = ld_acquire(fx.ready + mt)) == 0) {
+                        if (*abort) break;
+                        if (global_timer() - t0 > fx.budget_ns) {
+                            *abort = 1;
+                            report_timeout(p2.status, 16, t, mt);
+                            break;
+                        }
+                    }
+                }
+                rdy = __shfl_sync(0xffffffffu, rdy, 0);
+                if (rdy == 0) break;
+                (void)ld_acquire(fx.ready + mt);   // each lane's own acquire of the released scales
                 epi_prefetch<EPI_DOWN>(p2, e, nt, half, wrow0 + lane, lane < nvalid, sc, lane, r0, r1);
             }
             if (!mbar_wait(&ctl->acc_full[buf], aph, abort, p1.status, 4, t)) break;
