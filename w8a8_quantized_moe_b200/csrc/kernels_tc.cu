@@ -230,6 +230,16 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
         : "r"(taddr));
 }
 
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+          "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+}
+
 __device__ __forceinline__ void tmem_ld_wait() {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
@@ -335,6 +345,26 @@ __device__ __forceinline__ void epi_prefetch(const TcParams& p, int e, int nt, i
     __syncwarp();
 }
 
+// Store a warp's 32 rows x 16 fp32 values (lane l holds row l's v[0..15]) to
+// rows gbase + l*ld (first nvalid rows): 64 bytes per row, staged like
+// store_rows32_bf16 (16-byte chunks swizzled by (row / 2) mod 4), four lanes
+// per row on the global side.
+__device__ __forceinline__ void store_rows16(float* stage, const uint32_t (&v)[16], float* gbase, int64_t ld,
+                                             int nvalid, int lane) {
+    uint4* st4 = reinterpret_cast<uint4*>(stage);
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+        st4[lane * 4 + (j ^ ((lane >> 1) & 3))] = make_uint4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+    __syncwarp();
+#pragma unroll
+    for (int it = 0; it < 4; ++it) {
+        const int r = it * 8 + (lane >> 2), c = lane & 3;
+        const uint4 q = st4[r * 4 + (c ^ ((r >> 1) & 3))];
+        if (r < nvalid) reinterpret_cast<uint4*>(gbase + (int64_t)r * ld)[c] = q;
+    }
+    __syncwarp();
+}
+
 // GEMM1 tile: columns 0..127 of the accumulator are gate channels
 // nt*128 + c, columns 128..255 the matching up channels.  Each warp owns 32
 // rows (its TMEM lane quarter) and 64 of the 128 h columns.  sc, sxt: from
@@ -347,31 +377,40 @@ __device__ __forceinline__ void epilogue_swiglu(const TcParams& p, uint32_t tadd
     const bool valid = lane < nvalid;
     const int grow = wrow0 + lane;
     float amax = 0.0f;
-#pragma unroll 1
-    for (int c = 0; c < 2; ++c) {
-        const int col0 = 64 * half + 32 * c;
-        uint32_t g[32], u[32];
-        tmem_ld32(taddr + col0, g);
-        tmem_ld32(taddr + 128 + col0, u);
+    // four 16-column sub-chunks of gate and up words, double-buffered: sub-chunk
+    // c + 1 is requested right after sub-chunk c has arrived, so its latency
+    // overlaps c's math and stores; the accumulator is released once the last
+    // sub-chunk is in registers
+    uint32_t gb[2][16], ub[2][16];
+    tmem_ld16(taddr + 64 * half, gb[0]);
+    tmem_ld16(taddr + 128 + 64 * half, ub[0]);
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+        const int col0 = 64 * half + 16 * c;
+        uint32_t (&g)[16] = gb[c & 1];
+        uint32_t (&u)[16] = ub[c & 1];
         tmem_ld_wait();
-        if (c == 1) {
+        if (c < 3) {
+            tmem_ld16(taddr + col0 + 16, gb[(c + 1) & 1]);
+            tmem_ld16(taddr + 128 + col0 + 16, ub[(c + 1) & 1]);
+        } else {
             tc_fence_before();
             __syncwarp();
             if (lane == 0) release_acc<PAIR>(acc_empty);
         }
         const int ch0 = nt * 128 + col0;
-        const float* swg = sc + 32 * c;
-        const float* swu = sc + 64 + 32 * c;
+        const float* swg = sc + 16 * c;
+        const float* swu = sc + 64 + 16 * c;
         if (p.acc_dbg && valid) {
             int32_t* dg = p.acc_dbg + (int64_t)grow * 2 * f + ch0;
-            for (int j = 0; j < 32; ++j) {
+            for (int j = 0; j < 16; ++j) {
                 dg[j] = (int32_t)g[j];
                 dg[f + j] = (int32_t)u[j];
             }
         }
-        // h overwrites u in place (each u is dead once its h is formed)
+        uint32_t hv[16];
 #pragma unroll
-        for (int j = 0; j < 32; j += 4) {
+        for (int j = 0; j < 16; j += 4) {
             const float4 sg = *reinterpret_cast<const float4*>(swg + j);
             const float4 su = *reinterpret_cast<const float4*>(swu + j);
             const float sgv[4] = {sg.x, sg.y, sg.z, sg.w}, suv[4] = {su.x, su.y, su.z, su.w};
@@ -381,10 +420,10 @@ __device__ __forceinline__ void epilogue_swiglu(const TcParams& p, uint32_t tadd
                 const float uf = __fmul_rn(__fmul_rn(acc_value<FMT>(u[j + q]), sxt), suv[q]);
                 const float h = __fmul_rn(moe_silu(gf), uf);
                 if (valid) amax = fmaxf(amax, fabsf(h));
-                u[j + q] = __float_as_uint(h);
+                hv[j + q] = __float_as_uint(h);
             }
         }
-        store_rows32(stage, u, p.h32 + (int64_t)wrow0 * f + ch0, f, nvalid, lane);
+        store_rows16(stage, hv, p.h32 + (int64_t)wrow0 * f + ch0, f, nvalid, lane);
     }
     if (valid) p.pamax[(int64_t)grow * (f / 64) + nt * 2 + half] = amax;
 }
@@ -398,13 +437,19 @@ __device__ __forceinline__ void epilogue_down(const TcParams& p, uint32_t taddr,
     const int d = p.N;
     const bool valid = lane < nvalid;
     const int grow = wrow0 + lane;
-#pragma unroll 1
+    // two register sets: chunk c + 1's accumulator words are requested right
+    // after chunk c's have arrived, so their latency overlaps chunk c's math
+    // and stores
+    uint32_t buf2[2][32];
+    tmem_ld32(taddr + 128 * half, buf2[0]);
+#pragma unroll
     for (int c = 0; c < 4; ++c) {
         const int col0 = 128 * half + 32 * c;
-        uint32_t a[32];
-        tmem_ld32(taddr + col0, a);
+        uint32_t (&a)[32] = buf2[c & 1];
         tmem_ld_wait();
-        if (c == 3) {
+        if (c < 3) {
+            tmem_ld32(taddr + col0 + 32, buf2[(c + 1) & 1]);
+        } else {
             tc_fence_before();
             __syncwarp();
             if (lane == 0) release_acc<PAIR>(acc_empty);
