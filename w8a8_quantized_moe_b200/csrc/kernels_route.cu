@@ -447,9 +447,11 @@ __global__ void __launch_bounds__(kSelWarps * 32) router_select_kernel(
     const int t = blockIdx.x * kSelWarps + warp;
     if (t >= T) return;
     {
-        const int4* src = reinterpret_cast<const int4*>(x + (int64_t)t * d);
-        int4* dst = reinterpret_cast<int4*>(xs);
-        for (int i = lane; i < d / 8; i += 32) dst[i] = src[i];
+        // the token's X row into shared memory: every 16-byte piece in flight at once
+        const uint16_t* src = x + (int64_t)t * d;
+        for (int i = lane; i < d / 8; i += 32) cp_async16(xs + 8 * i, src + 8 * i, 16);
+        cp_async_commit();
+        cp_async_wait<0>();
         __syncwarp();
     }
     const int nj = d / 128;   // 16-byte steps per lane
