@@ -88,6 +88,8 @@ struct TcParams {
     float* pamax;             // GEMM1: per-row partial max [rows][f/64]
     void* o;                  // GEMM2: [rows][d], fp32 or (o_bf16) bf16
     int o_bf16;               // GEMM2: per-slot rows in bf16 (bf16-output layers)
+    int tma_c;                // the kernel's output map (tm_c) serves bulk tensor stores of full 32-row
+                              // chunks (64-byte rows: GEMM1 16 fp32 h values, GEMM2 32 bf16 values)
     int32_t* acc_dbg;         // optional raw accumulators (canonical channel order)
     int32_t* status;
 };
@@ -167,6 +169,21 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, u
         "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y)
         : "memory");
 }
+
+// TMA store of a staged box from this CTA's shared memory (bulk async group);
+// the staged data must have been made visible to the async proxy
+// (fence.proxy.async.shared::cta by the writing threads) first.
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void* src, int x, int y) {
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(smem_u32(src)), "r"(x), "r"(y)
+                 : "memory");
+    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// The previous bulk stores of this thread have finished reading shared memory.
+__device__ __forceinline__ void tma_store_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// The previous bulk stores of this thread are complete.
+__device__ __forceinline__ void tma_store_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 // Shared-memory matrix descriptor, K-major, 128-byte swizzle: 8-row atoms of
 // 1024 bytes (stride byte offset 1024); leading byte offset unused for this
@@ -276,34 +293,6 @@ __device__ __forceinline__ void store_rows32(float* stage, const uint32_t (&v)[3
     }
 }
 
-// Store a warp's 32 rows x 32 values as bf16 (lane l holds row l's fp32
-// values v[0..31], rounded to nearest even here) to rows gbase + l*ld (only
-// the first nvalid rows): one pass through the same 2 KB buffer, 64 bytes per
-// row in four 16-byte chunks swizzled by (row / 2) mod 4, so that the
-// shared-memory writes and reads are conflict-free; four lanes write one
-// row's 64 contiguous bytes.
-__device__ __forceinline__ void store_rows32_bf16(float* stage, const uint32_t (&v)[32], uint16_t* gbase,
-                                                  int64_t ld, int nvalid, int lane) {
-    uint4* st4 = reinterpret_cast<uint4*>(stage);
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        uint32_t w[4];
-#pragma unroll
-        for (int q = 0; q < 4; ++q)
-            w[q] = (uint32_t)f32_to_bf16_bits(__uint_as_float(v[8 * j + 2 * q])) |
-                   ((uint32_t)f32_to_bf16_bits(__uint_as_float(v[8 * j + 2 * q + 1])) << 16);
-        st4[lane * 4 + (j ^ ((lane >> 1) & 3))] = make_uint4(w[0], w[1], w[2], w[3]);
-    }
-    __syncwarp();
-#pragma unroll
-    for (int it = 0; it < 4; ++it) {
-        const int r = it * 8 + (lane >> 2), c = lane & 3;
-        const uint4 q = st4[r * 4 + (c ^ ((r >> 1) & 3))];
-        if (r < nvalid) reinterpret_cast<uint4*>(gbase + (int64_t)r * ld)[c] = q;
-    }
-    __syncwarp();
-}
-
 // Release of an accumulator buffer by one epilogue warp: a local arrive, or,
 // for a CTA pair, an arrive on the pair leader's barrier (same offset in the
 // leader's shared memory), which counts the warps of both CTAs.  Only the
@@ -345,22 +334,35 @@ __device__ __forceinline__ void epi_prefetch(const TcParams& p, int e, int nt, i
     __syncwarp();
 }
 
-// Store a warp's 32 rows x 16 fp32 values (lane l holds row l's v[0..15]) to
-// rows gbase + l*ld (first nvalid rows): 64 bytes per row, staged like
-// store_rows32_bf16 (16-byte chunks swizzled by (row / 2) mod 4), four lanes
-// per row on the global side.
-__device__ __forceinline__ void store_rows16(float* stage, const uint32_t (&v)[16], float* gbase, int64_t ld,
-                                             int nvalid, int lane) {
+// Store a warp's 32 rows x 64 bytes (lane l holds row l's 16 words w[0..15])
+// to the rows [row0, row0 + 32) at column x of a tensor whose map `tmc` has a
+// 32-row x 64-byte box with 64-byte swizzle: the rows are staged in that
+// layout (16-byte chunks XOR (row / 2) mod 4, the same layout the plain path
+// uses) and one lane issues a bulk tensor store, which writes the box
+// asynchronously.  When fewer than 32 rows are valid (an expert's last
+// rows: the box would overwrite the next expert's) or there is no map, the
+// plain stores write the first nvalid rows to gbase.  `stage` is 512-byte
+// aligned; before it is rewritten the previous bulk store must have read it.
+__device__ __forceinline__ void store_rows_64b(float* stage, const uint32_t (&v)[16], const CUtensorMap* tmc,
+                                               int x, int row0, void* gbase, int64_t ld_bytes, int nvalid, int lane) {
     uint4* st4 = reinterpret_cast<uint4*>(stage);
+    if (lane == 0) tma_store_wait_read();
+    __syncwarp();
 #pragma unroll
     for (int j = 0; j < 4; ++j)
         st4[lane * 4 + (j ^ ((lane >> 1) & 3))] = make_uint4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+    if (tmc && nvalid == 32) {
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        __syncwarp();
+        if (lane == 0) tma_store_2d(tmc, stage, x, row0);
+        return;
+    }
     __syncwarp();
 #pragma unroll
     for (int it = 0; it < 4; ++it) {
         const int r = it * 8 + (lane >> 2), c = lane & 3;
         const uint4 q = st4[r * 4 + (c ^ ((r >> 1) & 3))];
-        if (r < nvalid) reinterpret_cast<uint4*>(gbase + (int64_t)r * ld)[c] = q;
+        if (r < nvalid) reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(gbase) + (int64_t)r * ld_bytes)[c] = q;
     }
     __syncwarp();
 }
@@ -372,7 +374,7 @@ __device__ __forceinline__ void store_rows16(float* stage, const uint32_t (&v)[1
 template <int FMT, bool PAIR = false>
 __device__ __forceinline__ void epilogue_swiglu(const TcParams& p, uint32_t taddr, int half, int e,
                                                 int nt, int wrow0, int nvalid, float* stage, const float* sc,
-                                                float sxt, uint64_t* acc_empty, int lane) {
+                                                float sxt, uint64_t* acc_empty, const CUtensorMap* tmc, int lane) {
     const int f = p.f;
     const bool valid = lane < nvalid;
     const int grow = wrow0 + lane;
@@ -423,7 +425,7 @@ __device__ __forceinline__ void epilogue_swiglu(const TcParams& p, uint32_t tadd
                 hv[j + q] = __float_as_uint(h);
             }
         }
-        store_rows16(stage, hv, p.h32 + (int64_t)wrow0 * f + ch0, f, nvalid, lane);
+        store_rows_64b(stage, hv, tmc, ch0, wrow0, p.h32 + (int64_t)wrow0 * f + ch0, (int64_t)f * 4, nvalid, lane);
     }
     if (valid) p.pamax[(int64_t)grow * (f / 64) + nt * 2 + half] = amax;
 }
@@ -433,7 +435,8 @@ __device__ __forceinline__ void epilogue_swiglu(const TcParams& p, uint32_t tadd
 template <int FMT, bool PAIR = false>
 __device__ __forceinline__ void epilogue_down(const TcParams& p, uint32_t taddr, int half, int e,
                                               int nt, int wrow0, int nvalid, float* stage, const float* sc,
-                                              float shr, float wr, uint64_t* acc_empty, int lane) {
+                                              float shr, float wr, uint64_t* acc_empty, const CUtensorMap* tmc,
+                                              int lane) {
     const int d = p.N;
     const bool valid = lane < nvalid;
     const int grow = wrow0 + lane;
@@ -469,10 +472,15 @@ __device__ __forceinline__ void epilogue_down(const TcParams& p, uint32_t taddr,
                 a[j + q] = __float_as_uint(
                     __fmul_rn(__fmul_rn(__fmul_rn(acc_value<FMT>(a[j + q]), shr), sv[q]), wr));
         }
-        if (p.o_bf16)
-            store_rows32_bf16(stage, a, reinterpret_cast<uint16_t*>(p.o) + (int64_t)wrow0 * d + ch0, d, nvalid,
-                              lane);
-        else
+        if (p.o_bf16) {
+            uint32_t w[16];
+#pragma unroll
+            for (int q = 0; q < 16; ++q)
+                w[q] = (uint32_t)f32_to_bf16_bits(__uint_as_float(a[2 * q])) |
+                       ((uint32_t)f32_to_bf16_bits(__uint_as_float(a[2 * q + 1])) << 16);
+            store_rows_64b(stage, w, tmc, ch0, wrow0, reinterpret_cast<uint16_t*>(p.o) + (int64_t)wrow0 * d + ch0,
+                           (int64_t)d * 2, nvalid, lane);
+        } else
             store_rows32(stage, a, reinterpret_cast<float*>(p.o) + (int64_t)wrow0 * d + ch0, d, nvalid, lane);
     }
 }
@@ -482,7 +490,7 @@ __device__ __forceinline__ void epilogue_down(const TcParams& p, uint32_t taddr,
 template <int EPI, int FMT>
 __global__ void __launch_bounds__(kThreads, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
-                   const TcParams p) {
+                   const __grid_constant__ CUtensorMap tm_c, const TcParams p) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
     float* epi_stage = reinterpret_cast<float*>(smem + kStages * kStageBytes);
@@ -603,13 +611,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_after();
             const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(buf * BN);
             if (EPI == EPI_SWIGLU)
-                epilogue_swiglu<FMT>(p, taddr, half, e, nt, wrow0, nvalid, stage, sc, r0, &ctl->acc_empty[buf], lane);
+                epilogue_swiglu<FMT>(p, taddr, half, e, nt, wrow0, nvalid, stage, sc, r0, &ctl->acc_empty[buf],
+                                     p.tma_c ? &tm_c : nullptr, lane);
             else
                 epilogue_down<FMT>(p, taddr, half, e, nt, wrow0, nvalid, stage, sc, r0, r1, &ctl->acc_empty[buf],
-                                   lane);
+                                   p.tma_c ? &tm_c : nullptr, lane);
             buf ^= 1;
             if (buf == 0) aph ^= 1;
         }
+        if (lane == 0) tma_store_wait_all();     // this warp's bulk stores have landed
     }
 
     tc_fence_before();
@@ -759,7 +769,7 @@ __device__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, volatile int* 
 template <int EPI, int FMT>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     tc_pair_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
-                        const TcParams p) {
+                        const __grid_constant__ CUtensorMap tm_c, const TcParams p) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
     float* epi_stage = reinterpret_cast<float*>(smem + kStagesP * kStageBytesP);
@@ -894,13 +904,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(buf * BN);
             if (EPI == EPI_SWIGLU)
                 epilogue_swiglu<FMT, true>(p, taddr, half, e, nt, wrow0, nvalid, stage, sc, r0,
-                                           &ctl->acc_empty[buf], lane);
+                                           &ctl->acc_empty[buf], p.tma_c ? &tm_c : nullptr, lane);
             else
                 epilogue_down<FMT, true>(p, taddr, half, e, nt, wrow0, nvalid, stage, sc, r0, r1,
-                                         &ctl->acc_empty[buf], lane);
+                                         &ctl->acc_empty[buf], p.tma_c ? &tm_c : nullptr, lane);
             buf ^= 1;
             if (buf == 0) aph ^= 1;
         }
+        if (lane == 0) tma_store_wait_all();
     }
 
     tc_fence_before();
@@ -1267,7 +1278,8 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
             tc_fence_after();
             const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(buf * BN);
             if (g1) {
-                epilogue_swiglu<FMT>(p1, taddr, half, e, nt, wrow0, nvalid, stage, sc, r0, &ctl->acc_empty[buf], lane);
+                epilogue_swiglu<FMT>(p1, taddr, half, e, nt, wrow0, nvalid, stage, sc, r0, &ctl->acc_empty[buf], nullptr,
+                                     lane);
                 // this warp's share of the tile is stored: count it; the last arrival requantises
                 __threadfence();
                 __syncwarp();
@@ -1281,7 +1293,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
                 }
             } else {
                 epilogue_down<FMT>(p2, taddr, half, e, nt, wrow0, nvalid, stage, sc, r0, r1, &ctl->acc_empty[buf],
-                                   lane);
+                                   nullptr, lane);
             }
             buf ^= 1;
             if (buf == 0) aph ^= 1;
@@ -1607,6 +1619,22 @@ bool make_map_bf16(CUtensorMap* m, const void* base, uint64_t K, uint64_t rows, 
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 2-D map over a row-major [rows][cols] fp32 or bf16 output whose box is 32
+// rows x 64 bytes (16 fp32 or 32 bf16 values) with 64-byte swizzle: the
+// layout the epilogue warps stage a chunk of their 32 rows in.
+bool make_out_map(CUtensorMap* m, void* base, uint64_t cols, uint64_t rows, bool bf16) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const uint64_t esz = bf16 ? 2 : 4;
+    const cuuint64_t dims[2] = {cols, rows};
+    const cuuint64_t strides[1] = {cols * esz};
+    const cuuint32_t box[2] = {(cuuint32_t)(64 / esz), 32};
+    const cuuint32_t estr[2] = {1, 1};
+    return fn(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, base, dims, strides,
+              box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <int EPAD>
 cudaError_t launch_router_tc_pad(const CUtensorMap& mx, const moe_w8a8_weights* w, int T, float* approx,
                                  cudaStream_t s) {
@@ -1619,25 +1647,26 @@ cudaError_t launch_router_tc_pad(const CUtensorMap& mx, const moe_w8a8_weights* 
 }
 
 template <int EPI, int FMT>
-cudaError_t launch_fmt(const CUtensorMap& ta, const CUtensorMap& tb, const TcParams& p, int grid,
-                       cudaStream_t s) {
+cudaError_t launch_fmt(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tc, const TcParams& p,
+                       int grid, cudaStream_t s) {
     static std::atomic<uint64_t> attr{0};
     cudaError_t e = smem_attr_once(tc_gemm_kernel<EPI, FMT>, kSmemBytes, attr);
     if (e != cudaSuccess) return e;
-    return launch_pdl(tc_gemm_kernel<EPI, FMT>, dim3(grid), dim3(kThreads), kSmemBytes, s, ta, tb, p);
+    return launch_pdl(tc_gemm_kernel<EPI, FMT>, dim3(grid), dim3(kThreads), kSmemBytes, s, ta, tb, tc, p);
 }
 
 template <int EPI>
-cudaError_t launch(const CUtensorMap& ta, const CUtensorMap& tb, const TcParams& p, int grid, int fmt,
-                   cudaStream_t s) {
-    return fmt == FMT_E4M3 ? launch_fmt<EPI, FMT_E4M3>(ta, tb, p, grid, s) : launch_fmt<EPI, FMT_INT8>(ta, tb, p, grid, s);
+cudaError_t launch(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tc, const TcParams& p,
+                   int grid, int fmt, cudaStream_t s) {
+    return fmt == FMT_E4M3 ? launch_fmt<EPI, FMT_E4M3>(ta, tb, tc, p, grid, s)
+                           : launch_fmt<EPI, FMT_INT8>(ta, tb, tc, p, grid, s);
 }
 
 // The pair kernel on as many SM pairs as can be resident at once (one pair
 // per cluster of two CTAs; persistent), at most one per pair tile x column tile.
 template <int EPI, int FMT>
-cudaError_t launch_pair_fmt(const CUtensorMap& ta, const CUtensorMap& tb, const TcParams& p, int max_units,
-                            cudaStream_t s) {
+cudaError_t launch_pair_fmt(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tc, const TcParams& p,
+                            int max_units, cudaStream_t s) {
     static std::atomic<uint64_t> attr{0};
     static int clusters[64] = {};
     auto kern = tc_pair_gemm_kernel<EPI, FMT>;
@@ -1666,14 +1695,14 @@ cudaError_t launch_pair_fmt(const CUtensorMap& ta, const CUtensorMap& tb, const 
         nc = n;
     }
     const int grid = 2 * std::max(1, std::min(nc, max_units));
-    return launch_pdl(kern, dim3(grid), dim3(kThreads), kSmemBytesP, s, ta, tb, p);
+    return launch_pdl(kern, dim3(grid), dim3(kThreads), kSmemBytesP, s, ta, tb, tc, p);
 }
 
 template <int EPI>
-cudaError_t launch_pair(const CUtensorMap& ta, const CUtensorMap& tb, const TcParams& p, int max_units, int fmt,
-                        cudaStream_t s) {
-    return fmt == FMT_E4M3 ? launch_pair_fmt<EPI, FMT_E4M3>(ta, tb, p, max_units, s)
-                           : launch_pair_fmt<EPI, FMT_INT8>(ta, tb, p, max_units, s);
+cudaError_t launch_pair(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tc, const TcParams& p,
+                        int max_units, int fmt, cudaStream_t s) {
+    return fmt == FMT_E4M3 ? launch_pair_fmt<EPI, FMT_E4M3>(ta, tb, tc, p, max_units, s)
+                           : launch_pair_fmt<EPI, FMT_INT8>(ta, tb, tc, p, max_units, s);
 }
 
 }  // namespace
@@ -1809,13 +1838,16 @@ cudaError_t launch_tc_gemm1(const moe_w8a8_weights* w, int T, const int8_t* aq, 
     p.acc_dbg = acc_dbg;
     p.status = w->status;
     p.pairs = pairs;
+    CUtensorMap tc;
+    if (!make_out_map(&tc, h32, c.f, rows, false)) return cudaErrorInvalidValue;
+    p.tma_c = 1;
     if (pairs) {
         const int max_pt = (rows + 2 * BM - 1) / (2 * BM) + w->n_local;
-        return launch_pair<EPI_SWIGLU>(ta, w->tm_w_gu_half, p, max_pt * p.n_tiles_n, c.expert_format, s);
+        return launch_pair<EPI_SWIGLU>(ta, w->tm_w_gu_half, tc, p, max_pt * p.n_tiles_n, c.expert_format, s);
     }
     const int max_mt = (rows + BM - 1) / BM + c.n_experts;
     const int grid = max(1, min(w->num_sms, max_mt * p.n_tiles_n));
-    return launch<EPI_SWIGLU>(ta, w->tm_w_gu, p, grid, c.expert_format, s);
+    return launch<EPI_SWIGLU>(ta, w->tm_w_gu, tc, p, grid, c.expert_format, s);
 }
 
 cudaError_t launch_tc_gemm2(const moe_w8a8_weights* w, int T, const int8_t* hq, const float* sh,
@@ -1844,13 +1876,18 @@ cudaError_t launch_tc_gemm2(const moe_w8a8_weights* w, int T, const int8_t* hq, 
     p.acc_dbg = acc_dbg;
     p.status = w->status;
     p.pairs = pairs;
+    // bf16 O rows leave through bulk tensor stores; fp32 rows (128 bytes per
+    // chunk row) keep the plain stores, and the map is then only a placeholder
+    CUtensorMap tc;
+    if (!make_out_map(&tc, o, c.d, rows, true)) return cudaErrorInvalidValue;
+    p.tma_c = p.o_bf16;
     if (pairs) {
         const int max_pt = (rows + 2 * BM - 1) / (2 * BM) + w->n_local;
-        return launch_pair<EPI_DOWN>(ta, w->tm_w_dn_half, p, max_pt * p.n_tiles_n, c.expert_format, s);
+        return launch_pair<EPI_DOWN>(ta, w->tm_w_dn_half, tc, p, max_pt * p.n_tiles_n, c.expert_format, s);
     }
     const int max_mt = (rows + BM - 1) / BM + c.n_experts;
     const int grid = max(1, min(w->num_sms, max_mt * p.n_tiles_n));
-    return launch<EPI_DOWN>(ta, w->tm_w_dn, p, grid, c.expert_format, s);
+    return launch<EPI_DOWN>(ta, w->tm_w_dn, tc, p, grid, c.expert_format, s);
 }
 
 }  // namespace moe
