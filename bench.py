@@ -898,6 +898,13 @@ def run_ep(args, world, rank, local):
         clocks.stop()
         M.moe_w8a8_check_status(W)
         sent, received = layer.last_rows
+        # the fixed-block exchange: equal All-to-All parts, no host read of a count
+        blocked = ExpertParallelMoE(LibraryStages(W), block_tokens=T)
+        yb = torch.empty_like(y)
+        ms_blocked = max_over_ranks(timed(lambda: blocked.forward(x, T, bias, logits, yb)), world)
+        M.moe_w8a8_check_status(W)
+        torch.cuda.synchronize(dev)
+        assert torch.equal(y, yb), "fixed-block exchange output differs from the counted one"
         ms_fwd = None
         if world == 1:
             ws = torch.empty(M.moe_w8a8_workspace_size(W, T), dtype=torch.uint8, device=dev)
@@ -917,7 +924,12 @@ def run_ep(args, world, rank, local):
                                "exchange": "torch.distributed all_to_all_single (NCCL), host reads the "
                                            "row counts each step",
                                "l2": "weights larger than L2; no flush"},
-                    "single_gpu_forward_ms": ms_fwd, "clocks": clocks.summary()}
+                    "single_gpu_forward_ms": ms_fwd, "clocks": clocks.summary(),
+                    "blocked_exchange": {"ms_per_step": ms_blocked, "value": world * T / ms_blocked * 1e3,
+                                         "unit": "tokens/s", "block_tokens": T,
+                                         "exchange": "all_to_all_single of fixed blocks (T k + 1 rows per "
+                                                     "peer, count in a header row read on the device); no "
+                                                     "host read"}}
             print(json.dumps(line), flush=True)
     finally:
         if own_group:

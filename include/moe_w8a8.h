@@ -340,7 +340,9 @@ moe_status moe_w8a8_check_status(const moe_w8a8_weights* w, moe_stream_t stream)
  * waiting for an m-tile's h scales (words 3-4: tile, m-tile); 11-13 the certified router's
  * producer, MMA issuer and epilogue.  Site 14 (with MOE_ERR_INVALID_ARG): a
  * received expert-parallel row names an expert outside the handle's range
- * (words 2-3: row index, expert).  Does not clear them.
+ * (words 2-3: row index, expert); site 15 (with MOE_ERR_INVALID_ARG): a
+ * received fixed block's row count is outside [0, block rows - 1] (words 2-3:
+ * block, count).  Does not clear them.
  */
 moe_status moe_w8a8_status_words(const moe_w8a8_weights* w, int32_t* words_host, int32_t n,
                                  moe_stream_t stream);
@@ -530,6 +532,73 @@ moe_status moe_w8a8_ep_experts(const moe_w8a8_weights* w, const void* recv, int3
  */
 moe_status moe_w8a8_ep_combine(const moe_w8a8_weights* w, const float* o_rows, int32_t T, void* y,
                                const void* workspace, size_t workspace_bytes, moe_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * The same layer with a fixed-block exchange, for decode-sized batches: no
+ * row count ever has to reach the host.  ("Day0 adaptation of ultra-large
+ * model inference", section 3: one All-to-All each way; here both have sizes
+ * known in advance.)  Every rank uses the same block_tokens B >= its T.  Rank
+ * g's block for peer h is moe_w8a8_ep_block_rows(w, B) = B k + 1 rows of
+ * moe_w8a8_ep_row_bytes(w) bytes: a header row, whose first int32 is the
+ * number n of rows for h's experts (the rest of the header zero), then those
+ * n rows in the order of `send`; rows past n are unused and may hold
+ * anything.  One layer on one rank of G:
+ *   1. moe_w8a8_ep_dispatch as above;
+ *   2. moe_w8a8_ep_pack: `send` into G blocks, one per destination;
+ *   3. an All-to-All of equal parts (one block each way per peer);
+ *   4. moe_w8a8_ep_experts_blocked on the G received blocks: the output row
+ *      of every received row at the same position of the output blocks
+ *      (fp32, d per row; headers and unused rows get zeros);
+ *   5. an All-to-All of equal parts back (one output block per peer);
+ *   6. moe_w8a8_ep_combine_blocked: each token's output from the returned
+ *      blocks (the position of each kept slot follows from the dispatch's
+ *      row offsets, kept in its workspace).
+ * rank_first: host int32 [G + 1], rank g holding experts
+ * [rank_first[g], rank_first[g + 1]): rank_first[0] = 0, strictly increasing,
+ * rank_first[G] = E; G from 1 to 64.
+ * ------------------------------------------------------------------------ */
+
+/* Rows per block, B k + 1 (0 on a NULL handle or B < 1). */
+int32_t moe_w8a8_ep_block_rows(const moe_w8a8_weights* w, int32_t block_tokens);
+
+/*
+ * Step 2: blocks, device [G][moe_w8a8_ep_block_rows(w, B)][row bytes],
+ * 16-byte aligned, from `send` and the expert_offsets (device) of the
+ * preceding moe_w8a8_ep_dispatch (whose T must be <= B).  A count above the
+ * block's capacity cannot occur when T <= B; the receiving side reports one
+ * (status word site 15) and reads it as 0.  MOE_ERR_INVALID_ARG for a NULL or
+ * misaligned pointer or bad rank_first.
+ */
+moe_status moe_w8a8_ep_pack(const moe_w8a8_weights* w, const void* send, const int32_t* expert_offsets,
+                            const int32_t* rank_first, int32_t world, int32_t block_tokens, void* blocks,
+                            moe_stream_t stream);
+
+/* Workspace of moe_w8a8_ep_experts_blocked for G blocks of B tokens. */
+size_t moe_w8a8_ep_experts_blocked_workspace_size(const moe_w8a8_weights* w, int32_t world,
+                                                  int32_t block_tokens);
+
+/*
+ * Step 4: the experts this handle holds, on the G received blocks (device,
+ * 16-byte aligned, as written by moe_w8a8_ep_pack on the G ranks in rank
+ * order).  o_blocks: device fp32 [G][block rows][d], 16-byte aligned; the
+ * output row of received row i of block g at row i of output block g.  The
+ * row counts are read on the device.  Errors and dbg as moe_w8a8_ep_experts,
+ * with R = G x block rows and each header and unused row left out.
+ */
+moe_status moe_w8a8_ep_experts_blocked(const moe_w8a8_weights* w, const void* blocks, int32_t world,
+                                       int32_t block_tokens, float* o_blocks, void* workspace,
+                                       size_t workspace_bytes, const moe_w8a8_debug* dbg, moe_stream_t stream);
+
+/*
+ * Step 6: y [T][d] (cfg.out_dtype, device, 16-byte aligned) from the G
+ * returned output blocks (device fp32 [G][block rows][d], 16-byte aligned:
+ * block g from rank g) and the workspace of the matching moe_w8a8_ep_dispatch
+ * with the same T (T <= B).  MOE_ERR_INVALID_ARG for a NULL or misaligned
+ * pointer or bad rank_first, before anything is enqueued.
+ */
+moe_status moe_w8a8_ep_combine_blocked(const moe_w8a8_weights* w, const float* o_blocks, int32_t T,
+                                       const int32_t* rank_first, int32_t world, int32_t block_tokens, void* y,
+                                       const void* workspace, size_t workspace_bytes, moe_stream_t stream);
 
 #ifdef __cplusplus
 }

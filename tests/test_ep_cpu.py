@@ -66,30 +66,81 @@ class OracleStages:
             rows[r, :d] = xq[t].view(np.uint8)
             rows[r, d:d + 8] = np.array([sx[t], rt.w[t, sl]], np.float32).view(np.uint8)
             rows[r, d + 8:] = np.array([rt.idx[t, sl], ts], np.int32).view(np.uint8)
-        send.copy_(torch.from_numpy(rows.reshape(-1)))
+        send[:rows.size].copy_(torch.from_numpy(rows.reshape(-1)))
         offsets.copy_(torch.from_numpy(rt.offsets.astype(np.int32)))
         self.ts2row = rt.ts2row
 
-    def experts(self, recv, R, o_rows, ws):
-        import torch
-
+    def _expert_row(self, row):
         import oracle
         d, p = self.d, self.prep
+        codes = row[:d].view(np.int8)
+        sx, w = row[d:d + 8].view(np.float32)
+        e, _ts = row[d + 8:].view(np.int32)
+        assert self.first <= e < self.first + self.n, f"row for expert {e} on the wrong rank"
+        self.seen_experts.add(int(e))
+        acc_g = oracle.gemm_i8(codes[None], p.wq_gate[e])[0]
+        acc_u = oracle.gemm_i8(codes[None], p.wq_up[e])[0]
+        _h, hq, sh = oracle.swiglu_requant(acc_g, acc_u, float(sx), p.sw_gate[e], p.sw_up[e])
+        acc2 = oracle.gemm_i8(hq[None], p.wq_down[e])[0]
+        o = oracle.down_epilogue(acc2, sh, p.sw_down[e], float(w))
+        if self.wl.in_bf16:          # per-slot rows in the layer's output precision
+            o = oracle.round_bf16(o)
+        return o
+
+    def experts(self, recv, R, o_rows, ws):
+        import torch
         rows = recv.numpy().reshape(R, self.row_bytes)
         for r in range(R):
-            codes = rows[r, :d].view(np.int8)
-            sx, w = rows[r, d:d + 8].view(np.float32)
-            e, _ts = rows[r, d + 8:].view(np.int32)
-            assert self.first <= e < self.first + self.n, f"row for expert {e} on the wrong rank"
-            self.seen_experts.add(int(e))
-            acc_g = oracle.gemm_i8(codes[None], p.wq_gate[e])[0]
-            acc_u = oracle.gemm_i8(codes[None], p.wq_up[e])[0]
-            _h, hq, sh = oracle.swiglu_requant(acc_g, acc_u, float(sx), p.sw_gate[e], p.sw_up[e])
-            acc2 = oracle.gemm_i8(hq[None], p.wq_down[e])[0]
-            o = oracle.down_epilogue(acc2, sh, p.sw_down[e], float(w))
-            if self.wl.in_bf16:          # per-slot rows in the layer's output precision
-                o = oracle.round_bf16(o)
-            o_rows[r] = torch.from_numpy(o)
+            o_rows[r] = torch.from_numpy(self._expert_row(rows[r]))
+
+    # fixed-block exchange: the library's block layout (header row with the
+    # count, then the rows; unused rows filled with junk that must be ignored)
+    def block_rows(self, B):
+        return B * self.k + 1
+
+    def pack(self, send, offsets, rank_first, B, blocks):
+        rb, nb = self.row_bytes, self.block_rows(B)
+        src = send.numpy().reshape(-1, rb)
+        off = offsets.numpy()
+        out = blocks.numpy().reshape(len(rank_first) - 1, nb, rb)
+        out[:] = 0xA5
+        for g in range(len(rank_first) - 1):
+            lo, hi = int(off[rank_first[g]]), int(off[rank_first[g + 1]])
+            out[g, 0] = 0
+            out[g, 0, :4] = np.array([hi - lo], np.int32).view(np.uint8)
+            out[g, 1:1 + hi - lo] = src[lo:hi]
+        self.offsets_host = off.copy()
+
+    def experts_blocked_workspace(self, world, B):
+        return 16
+
+    def experts_blocked(self, blocks, world, B, o_blocks, ws):
+        import torch
+        nb = self.block_rows(B)
+        b = blocks.numpy().reshape(world, nb, self.row_bytes)
+        o = o_blocks.view(world, nb, self.d)
+        o.zero_()
+        for g in range(world):
+            n = int(b[g, 0, :4].view(np.int32)[0])
+            assert 0 <= n <= nb - 1
+            for i in range(1, n + 1):
+                o[g, i] = torch.from_numpy(self._expert_row(b[g, i]))
+            self.blocked_recv = getattr(self, "blocked_recv", 0) + n
+
+    def combine_blocked(self, o_back, T, rank_first, B, y, ws):
+        import torch
+        nb = self.block_rows(B)
+        o = o_back.numpy().reshape(-1, self.d)
+        off = self.offsets_host
+        acc = np.zeros((T, self.d), np.float32)
+        for sl in range(self.k):
+            for t in range(T):
+                r = int(self.ts2row[t, sl])
+                if r < 0:
+                    continue
+                g = max(h for h in range(len(rank_first) - 1) if off[rank_first[h]] <= r)
+                acc[t] = acc[t] + o[g * nb + 1 + r - int(off[rank_first[g]])]
+        y.copy_(torch.from_numpy(acc))
 
     def combine(self, o_rows, T, y, ws):
         import torch
@@ -123,7 +174,7 @@ def _rank_main(rank, world, port, out_dir, case):
         ranges = case.get("ranges") or equal_expert_ranges(wl.E, world)
         first, n = ranges[rank]
         stages = OracleStages(wl, prep, first, n)
-        layer = ExpertParallelMoE(stages, ranges=ranges)
+        layer = ExpertParallelMoE(stages, ranges=ranges, block_tokens=case.get("block_tokens"))
         bad = []
         for r in ([(0, wl.E)], [(1, wl.E - 1)] + [(0, 1)] * (world - 1),
                   [(0, 2), (3, wl.E - 3)] + [(wl.E, 0)] * (world - 2)):
@@ -144,6 +195,7 @@ def _rank_main(rank, world, port, out_dir, case):
                 out["equal"] &= bool(np.array_equal(y, y_ref))
             out["rows"] = list(layer.last_rows)
         out["seen"] = sorted(stages.seen_experts)
+        out["blocked_recv"] = getattr(stages, "blocked_recv", 0)
         out["range"] = [first, n]
         with open(os.path.join(out_dir, f"r{rank}.json"), "w") as fh:
             json.dump(out, fh)
@@ -262,3 +314,28 @@ def test_ep_rank_leaving_between_steps_is_an_error_not_a_hang(tmp_path):
     assert r0["first_step"] and r1["first_step"]
     assert r0["error"] is not None
     assert r0["seconds"] < 30.0     # the group timeout is 5 s; the peer's closed socket may end it sooner
+
+
+def test_ep_blocked_two_ranks(tmp_path):
+    # fixed blocks of 64 tokens (129 rows per peer): no row count reaches the host
+    r = _run(tmp_path, 2, {"block_tokens": 64})
+    assert all(x["equal"] for x in r)
+    assert sum(x["blocked_recv"] for x in r) == 2 * 2 * 64 * 2   # two steps, every slot travels once
+    for x in r:
+        first, n = x["range"]
+        assert x["seen"] and all(first <= e < first + n for e in x["seen"])
+
+
+def test_ep_blocked_skew_capacity_and_short_batches(tmp_path):
+    # blocks larger than the batches (T = 40, 64, 17, 0 under B = 64), Zipf skew
+    # and capacity: unequal counts per peer, empty blocks, an idle sender
+    r = _run(tmp_path, 4, {"wl": {"zipf_s": 1.5, "capacity_factor": 1.0}, "T": [40, 64, 17, 0],
+                           "block_tokens": 64})
+    assert all(x["equal"] for x in r)
+    assert r[3]["T"] == 0 and r[3]["blocked_recv"] > 0
+
+
+def test_ep_blocked_eight_ranks_one_expert_each(tmp_path):
+    r = _run(tmp_path, 8, {"wl": {"zipf_s": 2.0}, "T": [16] * 8, "block_tokens": 16})
+    assert all(x["equal"] for x in r)
+    assert sum(x["blocked_recv"] for x in r) == 2 * 8 * 16 * 2

@@ -139,6 +139,52 @@ def run_emulated(M, L, datas, Ts):
     return ys, count.sum(axis=0)
 
 
+def run_emulated_blocked(M, L, datas, Ts, B):
+    """The fixed-block exchange over G emulated ranks: every block travels
+    whole (the host copies blocks, it never reads a count); returns y per rank
+    and the number of rows each rank's experts saw (from their debug offsets)."""
+    torch = _torch()
+    wl, G = L.wl, L.G
+    k, E, d = wl.k, wl.E, wl.d
+    rb = M.moe_w8a8_ep_row_bytes(L.shards[0])
+    nb = M.moe_w8a8_ep_block_rows(L.shards[0], B)
+    assert nb == B * k + 1
+    rank_first = [first for first, _ in L.ranges] + [E]
+    odt = torch.bfloat16 if wl.in_bf16 else torch.float32
+    blocks, wss = [], []
+    for g in range(G):
+        T = Ts[g]
+        x, logits, bias = _inputs(wl, datas[g])
+        send = torch.empty(B * k * rb, dtype=torch.uint8, device="cuda")
+        off = torch.empty(E + 1, dtype=torch.int32, device="cuda")
+        ws = torch.empty(M.moe_w8a8_ep_dispatch_workspace_size(L.shards[g], B), dtype=torch.uint8, device="cuda")
+        M.moe_w8a8_ep_dispatch(L.shards[g], x[:T], T, bias, logits[:T] if logits is not None else None,
+                               send, off, ws)
+        blk = torch.full((G * nb * rb,), 0x5A, dtype=torch.uint8, device="cuda")   # junk in unused rows
+        M.moe_w8a8_ep_pack(L.shards[g], send, off, rank_first, B, blk)
+        blocks.append(blk.view(G, nb * rb))
+        wss.append(ws)
+    o_blocks, seen = [], []
+    for h in range(G):
+        recv = torch.cat([blocks[g][h] for g in range(G)]).contiguous()   # block h of every source
+        o = torch.full((G * nb, d), float("nan"), dtype=torch.float32, device="cuda")
+        ws = torch.empty(M.moe_w8a8_ep_experts_blocked_workspace_size(L.shards[h], G, B), dtype=torch.uint8,
+                         device="cuda")
+        offs = torch.empty(L.ranges[h][1] + 1, dtype=torch.int32, device="cuda")
+        M.moe_w8a8_ep_experts_blocked(L.shards[h], recv, G, B, o, ws, {"offsets": offs})
+        o_blocks.append(o.view(G, nb * d))
+        seen.append(int(offs[-1].item()))
+    ys = []
+    for g in range(G):
+        o_back = torch.cat([o_blocks[h][g] for h in range(G)]).contiguous()   # block g of every destination
+        y = torch.empty((Ts[g], d), dtype=odt, device="cuda")
+        M.moe_w8a8_ep_combine_blocked(L.shards[g], o_back, Ts[g], rank_first, B, y, wss[g])
+        ys.append(y)
+    for s in L.shards:
+        M.moe_w8a8_check_status(s)
+    return ys, np.array(seen)
+
+
 def full_forward(M, L, data, T):
     torch = _torch()
     wl = L.wl
@@ -151,11 +197,14 @@ def full_forward(M, L, data, T):
     return y
 
 
-def check_layer(M, L, Ts, steps=1):
+def check_layer(M, L, Ts, steps=1, block_tokens=None):
     recv_rows = None
     for step in range(steps):
         datas = [L.rank_data(g, max(Ts[g], 1), step) for g in range(L.G)]
-        ys, recv_rows = run_emulated(M, L, datas, Ts)
+        if block_tokens is None:
+            ys, recv_rows = run_emulated(M, L, datas, Ts)
+        else:
+            ys, recv_rows = run_emulated_blocked(M, L, datas, Ts, block_tokens)
         for g in range(L.G):
             if Ts[g] == 0:
                 continue
@@ -223,6 +272,54 @@ def test_rank_without_tokens_and_separate_expert_launches(M):
     L = Layer(M, synth.WORKLOADS["decode"], 2)
     rows = check_layer(M, L, [512, 0])
     assert rows.sum() == 2048 and rows.min() > 800
+
+
+@pytest.mark.parametrize("G", [2, 4])
+def test_blocked_exchange_decode(M, G):
+    # fixed blocks of 32 tokens (129 rows per peer), each rank's experts take
+    # their row counts from the block headers on the device
+    L = Layer(M, synth.WORKLOADS["decode"], G)
+    rows = check_layer(M, L, [32] * G, steps=2, block_tokens=32)
+    assert rows.sum() == 32 * 4 * G
+
+
+def test_blocked_exchange_short_batches_skew_and_idle_rank(M):
+    # batches at and below the block (T = 20, 7, 0, 32 under B = 32), Zipf
+    # skew and capacity, on the tiny layer (fp32 in and out)
+    wl = dataclasses.replace(synth.WORKLOADS["tiny"], zipf_s=1.5, capacity_factor=1.0)
+    L = Layer(M, wl, 4)
+    check_layer(M, L, [20, 7, 0, 32], block_tokens=32)
+
+
+def test_blocked_exchange_streaming_expert_path(M):
+    # 1 token per rank: 2 x (4 + 1) rows per rank's experts, the streaming path
+    L = Layer(M, synth.WORKLOADS["decode"], 2)
+    check_layer(M, L, [1, 1], block_tokens=1)
+
+
+def test_block_count_out_of_range_is_reported(M):
+    torch = _torch()
+    wl = synth.WORKLOADS["tiny"]
+    L = Layer(M, wl, 2)
+    B = 2
+    nb = M.moe_w8a8_ep_block_rows(L.shards[0], B)
+    rb = wl.d + 16
+    blk = torch.zeros((2, nb, rb), dtype=torch.uint8)
+    blk[1, 0, :4] = torch.from_numpy(np.array([nb], np.int32).view(np.uint8))   # one more than fits
+    o = torch.empty((2 * nb, wl.d), dtype=torch.float32, device="cuda")
+    ws = torch.empty(M.moe_w8a8_ep_experts_blocked_workspace_size(L.shards[0], 2, B), dtype=torch.uint8,
+                     device="cuda")
+    M.moe_w8a8_ep_experts_blocked(L.shards[0], blk.cuda().reshape(-1), 2, B, o, ws)
+    words = M.moe_w8a8_status_words(L.shards[0], 4)
+    with pytest.raises(M.MoeError) as e:
+        M.moe_w8a8_check_status(L.shards[0])
+    assert e.value.status == M.MOE_ERR_INVALID_ARG
+    assert words[1] == 15 and words[2] == 1 and words[3] == nb
+    assert torch.count_nonzero(o).item() == 0     # every row left out: zeros
+    with pytest.raises(M.MoeError):
+        M.moe_w8a8_ep_pack(L.shards[0], torch.empty(64, dtype=torch.uint8, device="cuda"),
+                           torch.zeros(wl.E + 1, dtype=torch.int32, device="cuda"), [0, 3, 2, wl.E], B,
+                           torch.empty(3 * nb * rb, dtype=torch.uint8, device="cuda"))
 
 
 def test_fp8_experts(M):
@@ -303,5 +400,16 @@ def test_driver_on_a_one_rank_nccl_group(M):
             torch.cuda.synchronize()
             assert torch.equal(y, ref)
             assert layer.last_rows == (wl.T * wl.k, wl.T * wl.k)
+        # the fixed-block exchange through the same group: no count reaches the host
+        blocked = ExpertParallelMoE(LibraryStages(shard), block_tokens=wl.T)
+        for step in range(2):
+            data = synth.make_data(dataclasses.replace(wl, data_seed=wl.data_seed + 13 * step))
+            x, logits, bias = _inputs(wl, data)
+            y = blocked.forward(x, wl.T, bias, logits)
+            ref = torch.empty_like(y)
+            ws = torch.empty(M.moe_w8a8_workspace_size(full, wl.T), dtype=torch.uint8, device="cuda")
+            M.moe_w8a8_forward(full, x, wl.T, bias, logits, ref, ws)
+            torch.cuda.synchronize()
+            assert torch.equal(y, ref)
     finally:
         dist.destroy_process_group()

@@ -46,6 +46,8 @@ EXPORTS = (
     "moe_w8a8_ep_dispatch", "moe_w8a8_ep_experts", "moe_w8a8_ep_combine",
     "moe_w8a8_tensor_peak_loop", "moe_w8a8_set_wait_budget", "moe_w8a8_test_withhold_release",
     "moe_w8a8_set_fused_threshold", "moe_w8a8_set_cta_pairs",
+    "moe_w8a8_ep_block_rows", "moe_w8a8_ep_pack", "moe_w8a8_ep_experts_blocked_workspace_size",
+    "moe_w8a8_ep_experts_blocked", "moe_w8a8_ep_combine_blocked",
 )
 
 MOE_NOALLOC_SCRATCH_BYTES = 8 << 20
@@ -124,6 +126,11 @@ def lib():
             "moe_w8a8_set_fused_threshold": ([vp, i64], i32),
             "moe_w8a8_set_cta_pairs": ([vp, i32], i32),
             "moe_w8a8_test_withhold_release": ([vp, i32], i32),
+            "moe_w8a8_ep_block_rows": ([vp, i32], i32),
+            "moe_w8a8_ep_pack": ([vp, vp, vp, vp, i32, i32, vp, vp], i32),
+            "moe_w8a8_ep_experts_blocked_workspace_size": ([vp, i32, i32], sz),
+            "moe_w8a8_ep_experts_blocked": ([vp, vp, i32, i32, vp, vp, sz, vp, vp], i32),
+            "moe_w8a8_ep_combine_blocked": ([vp, vp, i32, vp, i32, i32, vp, vp, sz, vp], i32),
         }
         for name, (args, res) in sig.items():
             fn = getattr(L, name)
@@ -502,6 +509,62 @@ def moe_w8a8_ep_combine(w: Weights, o_rows, T: int, y, workspace, stream=None):
     _check(lib().moe_w8a8_ep_combine(
         w.handle, o_ptr, int(T), _dev_ptr(y, _act_dtype(w.cfg.out_dtype), "y"),
         _dev_ptr(workspace, name="workspace"), _nbytes(workspace), _stream(stream)), "moe_w8a8_ep_combine")
+
+
+# fixed-block exchange (no row count reaches the host)
+
+def moe_w8a8_ep_block_rows(w: Weights, block_tokens: int) -> int:
+    return int(lib().moe_w8a8_ep_block_rows(w.handle, int(block_tokens)))
+
+
+def _rank_first(rank_first):
+    """Host int32 [G + 1] array of the ranks' first experts (kept alive by the caller)."""
+    import numpy as np
+    a = np.ascontiguousarray(np.asarray(rank_first, dtype=np.int32))
+    return a, ctypes.c_void_p(a.ctypes.data), len(a) - 1
+
+
+def moe_w8a8_ep_pack(w: Weights, send, expert_offsets, rank_first, block_tokens: int, blocks, stream=None):
+    torch = _torch()
+    a, ptr, world = _rank_first(rank_first)
+    rb = moe_w8a8_ep_row_bytes(w)
+    _need(expert_offsets, w.cfg.n_experts + 1, "expert_offsets")
+    _need(blocks, world * moe_w8a8_ep_block_rows(w, block_tokens) * rb, "blocks")
+    _check(lib().moe_w8a8_ep_pack(
+        w.handle, _dev_ptr(send, torch.uint8, "send"), _dev_ptr(expert_offsets, torch.int32, "expert_offsets"),
+        ptr, int(world), int(block_tokens), _dev_ptr(blocks, torch.uint8, "blocks"), _stream(stream)),
+        "moe_w8a8_ep_pack")
+
+
+def moe_w8a8_ep_experts_blocked_workspace_size(w: Weights, world: int, block_tokens: int) -> int:
+    return int(lib().moe_w8a8_ep_experts_blocked_workspace_size(w.handle, int(world), int(block_tokens)))
+
+
+def moe_w8a8_ep_experts_blocked(w: Weights, blocks, world: int, block_tokens: int, o_blocks, workspace,
+                                dbg: dict | None = None, stream=None):
+    torch = _torch()
+    rows = int(world) * moe_w8a8_ep_block_rows(w, block_tokens)
+    _need(blocks, rows * moe_w8a8_ep_row_bytes(w), "blocks")
+    _need(o_blocks, rows * w.cfg.d, "o_blocks")
+    _s, dptr = _debug_struct(dbg)
+    _check(lib().moe_w8a8_ep_experts_blocked(
+        w.handle, _dev_ptr(blocks, torch.uint8, "blocks"), int(world), int(block_tokens),
+        _dev_ptr(o_blocks, torch.float32, "o_blocks"), _dev_ptr(workspace, name="workspace"), _nbytes(workspace),
+        dptr, _stream(stream)), "moe_w8a8_ep_experts_blocked")
+
+
+def moe_w8a8_ep_combine_blocked(w: Weights, o_blocks, T: int, rank_first, block_tokens: int, y, workspace,
+                                stream=None):
+    torch = _torch()
+    a, ptr, world = _rank_first(rank_first)
+    if T == 0:
+        return
+    _need(y, T * w.cfg.d, "y")
+    _need(o_blocks, world * moe_w8a8_ep_block_rows(w, block_tokens) * w.cfg.d, "o_blocks")
+    _check(lib().moe_w8a8_ep_combine_blocked(
+        w.handle, _dev_ptr(o_blocks, torch.float32, "o_blocks"), int(T), ptr, int(world), int(block_tokens),
+        _dev_ptr(y, _act_dtype(w.cfg.out_dtype), "y"), _dev_ptr(workspace, name="workspace"), _nbytes(workspace),
+        _stream(stream)), "moe_w8a8_ep_combine_blocked")
 
 
 # ------------------------------------------------------------------ measurement aid

@@ -23,6 +23,15 @@ struct moe_w8a8_weights {
     int last_launches;
     // prepared weights (device)
     int8_t* w_gu;     // [n_local][2f][d]: per 128-channel block, 128 gate rows then 128 up rows
+    // The same INT8 (or E4M3) weights for the separate GEMM launches, tiled:
+    // the 256-row x 128-byte box that one k-block of a tile loads is 32 KB of
+    // contiguous memory ([row tile][k-block][256 rows][128 bytes]).  Measured
+    // on one box: large layer 3.05 -> 2.94 ms (its HBM-bound GEMM1 1.63 -> 1.55
+    // ms), while the fused decode launch was 2-3% faster on the canonical
+    // layout (many CTAs each reading 128 bytes of 256 rows spread the requests
+    // over more DRAM channels), so it keeps that one.
+    int8_t* w_gu_t;
+    int8_t* w_dn_t;
     int8_t* w_dn;     // [n_local][d][f]
     float* sw_gate;   // [n_local][f]
     float* sw_up;     // [n_local][f]
@@ -43,11 +52,13 @@ struct moe_w8a8_weights {
     uint64_t wait_budget_ns;   // bound on a block's wait for another block's results
     int test_skip_ready;       // testing aid: fused launch withholds this m-tile's ready flag (-1: none)
     int64_t fused_max_rows;    // tensor path: T*k at or below which GEMM1, requant and GEMM2 are one launch
-    // tensor maps of the weights for the tensor-core path (built at prepare)
+    // tensor maps of the weights for the tensor-core path (built at prepare):
+    // canonical layout (the fused launch), the tiled copies (the separate GEMM
+    // launches), and the tiled copies in 128-row boxes (one CTA of a pair loads
+    // half a tile)
     CUtensorMap tm_w_gu;
     CUtensorMap tm_w_dn;
-    CUtensorMap tm_w_gu_half;  // the same weights in 128-row boxes (one CTA of a pair loads half a tile)
-    CUtensorMap tm_w_dn_half;
+    CUtensorMap tm_w_gu_t, tm_w_dn_t, tm_w_gu_t_half, tm_w_dn_t_half;
     int cta_pairs;             // separate GEMM launches on SM pairs: 0 never, 1 always, 2 by rows per expert
     bool tmaps_ok;
     CUtensorMap tm_rt_hi;
@@ -120,10 +131,12 @@ cudaError_t launch_topk(const float* logits, const float* bias, int T, int E, in
                         int32_t* idx, float* wts, float* logits_out, cudaStream_t s);
 // zero_words[0, n_zero): counters a later kernel of the forward starts from
 // zero (the fused expert launch); block 0 of the scatter clears them.
+// hist_ready: `hist` ([chunks][E], kPermChunk entries per chunk) was already
+// counted (by the certified router's selection); only the scatter runs.
 cudaError_t launch_permute(const int32_t* idx, int T, int k, int E, int cap, int32_t* hist,
                            int32_t* offsets, int32_t* row2ts, int32_t* ts2row, int32_t* meta,
                            int32_t* active, int32_t* tiles, int32_t* pairs, cudaStream_t s,
-                           int32_t* zero_words = nullptr, int n_zero = 0);
+                           int32_t* zero_words = nullptr, int n_zero = 0, bool hist_ready = false);
 bool route_small_ok(int T, int k);
 cudaError_t launch_route_small(const float* logits, const float* bias, int T, int E, int k,
                                int renorm, int cap, int32_t* idx, float* wts, float* logits_out,
@@ -139,13 +152,29 @@ cudaError_t launch_smooth_quant(const void* x, int in_dtype, const float* inv_s,
 // Expert-parallel receive side.  Local expert of each received row (its
 // trailer's expert - ep_first); an expert outside [0, n_local) is recorded in
 // status (MOE_ERR_INVALID_ARG, site kSiteEpExpert) and the row runs through
-// local expert 0.
+// local expert 0.  With block_rows > 0 the rows are fixed blocks of that many
+// rows, each a header row (row count) and then the rows: headers and rows past
+// the count get idx -1 (left out); a count outside [0, block_rows - 1] is
+// recorded (site kSiteEpBlock) and read as 0.
 constexpr int kSiteEpExpert = 14;
+constexpr int kSiteEpBlock = 15;
 
-cudaError_t launch_ep_read_experts(const uint8_t* recv, int R, int64_t row_bytes, int d, int ep_first,
-                                   int n_local, int32_t* idx, int32_t* status, cudaStream_t s);
+cudaError_t launch_ep_read_experts(const uint8_t* recv, int R, int64_t row_bytes, int d, int block_rows,
+                                   int ep_first, int n_local, int32_t* idx, int32_t* status, cudaStream_t s);
+
+// The expert ranges of the ranks of a fixed-block exchange: rank g holds
+// global experts [first[g], first[g + 1]).
+constexpr int kEpMaxWorld = 64;
+struct EpRanks {
+    int32_t first[kEpMaxWorld + 1];
+};
+// Send rows (expert-major, `offsets` the E + 1 row offsets) into world fixed
+// blocks of block_rows rows: header row with the count, then the rows.
+cudaError_t launch_ep_pack(const uint8_t* send, const int32_t* offsets, const EpRanks& ranks, int world,
+                           int block_rows, int64_t row_bytes, uint8_t* blocks, cudaStream_t s);
 // Codes of received row r to row ts2row[r] of dst (row r when ts2row is
-// null), its scale and gate weight to sx[r] and wts[r].
+// null; nothing when ts2row[r] < 0), its scale and gate weight to sx[r] and
+// wts[r].
 cudaError_t launch_ep_gather(const uint8_t* recv, int R, int64_t row_bytes, int d, const int32_t* ts2row,
                              int8_t* dst, float* sx, float* wts, cudaStream_t s);
 // out[r][j] = |fp32(x[r][j] * inv_s[j])| (calibration of the activation clip)
@@ -166,15 +195,21 @@ cudaError_t launch_stream_down(const moe_w8a8_weights* w, int T, const int8_t* h
                                void* o, int32_t* acc2_dbg, cudaStream_t s);
 // tensor-core path (kernels_tc.cu)
 bool tc_make_weight_maps(moe_w8a8_weights* w);
+// dst = src [rows][K] (rows % 256 == 0, K % 128 == 0) in the tiled layout of w_gu_t.
+cudaError_t launch_tile_weights(const int8_t* src, int64_t rows, int K, int8_t* dst, cudaStream_t s);
 // Certified tensor-core router: approximate logits l~ [T][E] from bf16 X (this
 // file's kernels_tc.cu), then per token the candidate experts within the error
 // bound, their logits in the stated fp32 order, top-k and gate weights
 // (kernels_route.cu).  sel: [T][E] scratch.
 bool router_tc_make_maps(moe_w8a8_weights* w);
-cudaError_t launch_router_tc(const moe_w8a8_weights* w, const void* x, int T, float* approx, cudaStream_t s);
+// Also zeroes zero_words[0, n_zero) (the selection's histogram) before it ends.
+cudaError_t launch_router_tc(const moe_w8a8_weights* w, const void* x, int T, float* approx, int32_t* zero_words,
+                             int n_zero, cudaStream_t s);
+// Also counts the chosen (token, slot) entries per kPermChunk chunk and
+// expert into hist ([chunks][E], zeroed beforehand), for the permutation.
 cudaError_t launch_router_select(const moe_w8a8_weights* w, const void* x, int T, const float* approx,
                                  const float* bias, float* sel, int32_t* idx, float* wts, float* logits_out,
-                                 cudaStream_t s);
+                                 int32_t* hist, cudaStream_t s);
 constexpr int kRouterTcMinTokens = 1024;   // the certified router runs from this many tokens up
 bool tc_supported(const moe_w8a8_config& c);
 // n_mma back-to-back M=128 N=256 K=32 8-bit MMAs per CTA on `grid` CTAs
@@ -206,6 +241,11 @@ constexpr int kFusedMaxRows = 512;   // default: T*k at or below which the tenso
 // expert FFN writes them in the layer's output precision.
 cudaError_t launch_combine(const void* o, int o_bf16, const int32_t* ts2row, int T, int k, int d,
                            int out_dtype, void* y, cudaStream_t s);
+// The combine over fp32 output rows returned in the fixed blocks of an
+// expert-parallel exchange (`offsets` the dispatch's E + 1 row offsets).
+cudaError_t launch_combine_blocked(const float* o_blocks, const int32_t* ts2row, const int32_t* offsets,
+                                   const EpRanks& ranks, int world, int block_rows, int T, int k, int d,
+                                   int out_dtype, void* y, cudaStream_t s);
 // Bytes of one per-slot output value: the layer's output precision.
 inline size_t o_bytes(const moe_w8a8_config& c) { return c.out_dtype == MOE_BF16 ? 2 : 4; }
 

@@ -323,8 +323,9 @@ __device__ __forceinline__ bool better(float v, int i, float v2, int i2) {
 
 // One warp: top-k and gate weights of token t.  lsh: kMaxE floats of shared
 // scratch for this warp (used when the softmax runs over all E experts).
-// When idx_copy is given, the chosen experts are also written there.
-__device__ __forceinline__ void topk_token(const float* __restrict__ logits,
+// When idx_copy is given, the chosen experts are also written there.  Returns
+// the expert of slot `lane` to lanes below k (-1 to the others).
+__device__ __forceinline__ int topk_token(const float* __restrict__ logits,
                                            const float* __restrict__ bias, int t, int E, int k,
                                            int renorm, int32_t* __restrict__ idx,
                                            float* __restrict__ wts, float* __restrict__ logits_out,
@@ -379,6 +380,7 @@ __device__ __forceinline__ void topk_token(const float* __restrict__ logits,
     } else {
         for (int e = 0; e < E; ++e) z = __fadd_rn(z, moe_exp(__fsub_rn(lsh[e], lmax)));
     }
+    int mine = -1;
 #pragma unroll
     for (int s = 0; s < kMaxK; ++s) {
         if (s >= k) break;
@@ -386,8 +388,10 @@ __device__ __forceinline__ void topk_token(const float* __restrict__ logits,
             idx[(int64_t)t * k + s] = sel_i[s];
             wts[(int64_t)t * k + s] = __fdiv_rn(moe_exp(__fsub_rn(sel_v[s], lmax)), z);
             if (idx_copy) idx_copy[t * k + s] = sel_i[s];
+            mine = sel_i[s];
         }
     }
+    return mine;
 }
 
 __global__ void topk_kernel(const float* __restrict__ logits, const float* __restrict__ bias, int T,
@@ -436,7 +440,8 @@ __device__ __forceinline__ float4 ld_lane4(const float* rowbase, int j, int lane
 __global__ void __launch_bounds__(kSelWarps * 32) router_select_kernel(
     const uint16_t* __restrict__ x, const float* __restrict__ approx, const float* __restrict__ bias,
     const float* __restrict__ wt, const float* __restrict__ wmax, int T, int d, int E, int k, float c_err,
-    float* __restrict__ sel, int32_t* __restrict__ idx, float* __restrict__ wts, float* __restrict__ logits_out) {
+    float* __restrict__ sel, int32_t* __restrict__ idx, float* __restrict__ wts, float* __restrict__ logits_out,
+    int32_t* __restrict__ hist) {
     pdl_wait();
     pdl_trigger();
 
@@ -572,7 +577,9 @@ __global__ void __launch_bounds__(kSelWarps * 32) router_select_kernel(
         }
     }
     __syncwarp();
-    topk_token(sel, nullptr, t, E, k, 1, idx, wts, nullptr, lsh, nullptr, lane);
+    const int e = topk_token(sel, nullptr, t, E, k, 1, idx, wts, nullptr, lsh, nullptr, lane);
+    // the permutation's histogram: entry t k + s (expert e of lane s) of chunk (t k + s) / kPermChunk
+    if (lane < k) atomicAdd(&hist[(int64_t)((t * k + lane) / kPermChunk) * E + e], 1);
 }
 
 // ---------------------------------------------------------------------------
@@ -649,12 +656,14 @@ __device__ void scatter_entries(const int32_t* idx, int base, int len, int E, in
         for (int i = tid; i < nw * E; i += blockDim.x) wcnt[i / E][i % E] = 0;
         __syncthreads();
         const int i = base + r0 + tid;
-        const bool valid = r0 + tid < len;
-        const int e = valid ? idx[i] : -1;
+        const bool in = r0 + tid < len;
+        const int e = in ? idx[i] : -1;
+        const bool valid = in && e >= 0;   // e < 0: an entry to leave out (no row)
         const unsigned m = __match_any_sync(0xffffffffu, e);
         const int rank_w = __popc(m & ((1u << lane) - 1u));
         if (valid && rank_w == 0) wcnt[warp][e] = __popc(m);
         __syncthreads();
+        if (in && !valid) ts2row[i] = -1;
         if (valid) {
             int rank = running[e] + rank_w;
             for (int w2 = 0; w2 < warp; ++w2) rank += wcnt[w2][e];
@@ -687,7 +696,10 @@ __global__ void perm_hist_kernel(const int32_t* __restrict__ idx, int n, int E,
     __syncthreads();
     const int base = blockIdx.x * kPermChunk;
     for (int i = threadIdx.x; i < kPermChunk; i += blockDim.x)
-        if (base + i < n) atomicAdd(&cnt[idx[base + i]], 1);
+        if (base + i < n) {
+            const int e = idx[base + i];
+            if (e >= 0) atomicAdd(&cnt[e], 1);   // e < 0: an entry to leave out
+        }
     __syncthreads();
     for (int e = threadIdx.x; e < E; e += blockDim.x) hist[(int64_t)blockIdx.x * E + e] = cnt[e];
 }
@@ -782,6 +794,62 @@ __global__ void __launch_bounds__(kRouteSmallThreads) route_small_kernel(
     scatter_entries(sm.idx, 0, n, E, cap, sm.pre, sm.off, sm.running, sm.u.wcnt, row2ts, ts2row);
 }
 
+// Decode-sized inputs (T <= 32 tokens, T*k <= kRouteTinyMax entries): the same
+// results as route_small_kernel with three block barriers instead of about ten.
+// Warp t does token t's top-k; thread i then finds entry i's rank among the
+// earlier entries of its expert by a plain count over the entries before it
+// (at most kRouteTinyMax - 1 shared-memory reads, broadcast across the warp),
+// warp 0 places the offsets and lists, and each entry is stored at its row.
+constexpr int kRouteTinyMax = 256;
+
+struct RouteTinySmem {
+    int32_t idx[kRouteTinyMax];
+    int kept[kMaxE], off[kMaxE + 1];
+    float lsh[32][kMaxE];
+};
+
+__global__ void __launch_bounds__(1024) route_tiny_kernel(
+    const float* __restrict__ logits, const float* __restrict__ bias, int T, int E, int k,
+    int renorm, int cap, int32_t* __restrict__ idx, float* __restrict__ wts,
+    float* __restrict__ logits_out, int32_t* __restrict__ offsets, int32_t* __restrict__ row2ts,
+    int32_t* __restrict__ ts2row, int32_t* __restrict__ meta, int32_t* __restrict__ active,
+    int32_t* __restrict__ tiles, int32_t* __restrict__ pairs, int32_t* __restrict__ zero_words, int n_zero) {
+    pdl_wait();
+    pdl_trigger();
+    for (int i = threadIdx.x; i < n_zero; i += blockDim.x) zero_words[i] = 0;
+
+    extern __shared__ __align__(16) uint8_t smem_raw[];
+    RouteTinySmem& sm = *reinterpret_cast<RouteTinySmem*>(smem_raw);
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int n = T * k;
+    for (int e = tid; e < E; e += blockDim.x) sm.kept[e] = 0;
+    if (warp < T) topk_token(logits, bias, warp, E, k, renorm, idx, wts, logits_out, sm.lsh[warp], sm.idx, lane);
+    __syncthreads();
+    int e = -1, rank = 0;
+    if (tid < n) {
+        e = sm.idx[tid];
+        for (int j = 0; j < tid; ++j) rank += sm.idx[j] == e;
+        atomicAdd(&sm.kept[e], 1);
+    }
+    __syncthreads();
+    if (warp == 0) {
+        if (cap >= 0)
+            for (int x = lane; x < E; x += 32) sm.kept[x] = min(sm.kept[x], cap);
+        __syncwarp();
+        write_offsets_and_lists(sm.kept, E, sm.off, offsets, meta, active, tiles, pairs, lane);
+    }
+    __syncthreads();
+    if (tid < n) {
+        if (cap < 0 || rank < cap) {
+            const int row = sm.off[e] + rank;
+            ts2row[tid] = row;
+            row2ts[row] = tid;
+        } else {
+            ts2row[tid] = -1;
+        }
+    }
+}
+
 // ---------------------------------------------------------------------------
 // Smoothed per-token quantisation: x' = fp32(x * inv_s); sx = amax/127;
 // q = rint(x'/sx) clamped to +-127.  One block per token; each thread owns
@@ -873,14 +941,33 @@ __global__ void __launch_bounds__(kSqThreads) smooth_quant_kernel(
     }
 }
 
-// Expert-parallel receive side: the local expert of each received row.
+// Expert-parallel receive side: the local expert of each received row.  In
+// fixed blocks (block_rows > 0) row 0 of each block of block_rows rows is the
+// block's header (its first word the number of rows that follow) and rows
+// past that number are left out (idx -1).
 __global__ void ep_read_experts_kernel(const uint8_t* __restrict__ recv, int R, int64_t row_bytes, int d,
-                                       int ep_first, int n_local, int32_t* __restrict__ idx,
+                                       int block_rows, int ep_first, int n_local, int32_t* __restrict__ idx,
                                        int32_t* __restrict__ status) {
     pdl_wait();
     pdl_trigger();
     const int r = blockIdx.x * blockDim.x + threadIdx.x;
     if (r >= R) return;
+    if (block_rows > 0) {
+        const int g = r / block_rows, i = r % block_rows;
+        int count = *reinterpret_cast<const int32_t*>(recv + (int64_t)g * block_rows * row_bytes);
+        if (count < 0 || count > block_rows - 1) {
+            if (i == 0 && atomicCAS(status, 0, (int32_t)MOE_ERR_INVALID_ARG) == 0) {
+                status[1] = kSiteEpBlock;
+                status[2] = g;
+                status[3] = count;
+            }
+            count = 0;
+        }
+        if (i == 0 || i > count) {
+            idx[r] = -1;
+            return;
+        }
+    }
     const EpTrailer* tr = reinterpret_cast<const EpTrailer*>(recv + (int64_t)r * row_bytes + d);
     const int e = tr->expert - ep_first;
     if (e < 0 || e >= n_local) {
@@ -908,6 +995,7 @@ __global__ void __launch_bounds__(kEpGatherWarps * 32) ep_gather_kernel(
     if (r >= R) return;
     const uint8_t* src = recv + (int64_t)r * row_bytes;
     const int64_t drow = ts2row ? ts2row[r] : r;
+    if (drow < 0) return;   // a row left out (a fixed block's header or unused row)
     int8_t* out = dst + drow * d;
     for (int j = lane * 16; j < d; j += 32 * 16)
         *reinterpret_cast<int4*>(out + j) = *reinterpret_cast<const int4*>(src + j);
@@ -916,6 +1004,34 @@ __global__ void __launch_bounds__(kEpGatherWarps * 32) ep_gather_kernel(
         sx[r] = tr->sx;
         wts[r] = tr->w;
     }
+}
+
+// Fixed-block send buffer: block g (of `block_rows` rows) holds a header row
+// (first word: the number of rows for rank g's experts, the rest zero) and
+// then those rows, copied from the expert-major send rows
+// [offsets[first[g]], offsets[first[g + 1]]).  One warp per block row,
+// 16-byte copies; rows past the count are not written.
+__global__ void __launch_bounds__(kEpGatherWarps * 32) ep_pack_kernel(
+    const uint8_t* __restrict__ send, const int32_t* __restrict__ offsets, EpRanks ranks, int block_rows,
+    int64_t row_bytes, uint8_t* __restrict__ blocks) {
+    pdl_wait();
+    pdl_trigger();
+    const int lane = threadIdx.x & 31;
+    const int g = blockIdx.y;
+    const int i = blockIdx.x * kEpGatherWarps + (threadIdx.x >> 5);
+    if (i >= block_rows) return;
+    const int lo = offsets[ranks.first[g]], hi = offsets[ranks.first[g + 1]];
+    uint8_t* dst = blocks + ((int64_t)g * block_rows + i) * row_bytes;
+    if (i == 0) {
+        for (int64_t j = lane * 16; j < row_bytes; j += 32 * 16)
+            *reinterpret_cast<int4*>(dst + j) = make_int4(j == 0 ? hi - lo : 0, 0, 0, 0);
+        return;
+    }
+    const int r = lo + i - 1;
+    if (r >= hi) return;
+    const uint8_t* src = send + (int64_t)r * row_bytes;
+    for (int64_t j = lane * 16; j < row_bytes; j += 32 * 16)
+        *reinterpret_cast<int4*>(dst + j) = *reinterpret_cast<const int4*>(src + j);
 }
 
 }  // namespace
@@ -950,7 +1066,7 @@ cudaError_t launch_router_logits(const void* x, int in_dtype, const float* wr, i
 
 cudaError_t launch_router_select(const moe_w8a8_weights* w, const void* x, int T, const float* approx,
                                  const float* bias, float* sel, int32_t* idx, float* wts, float* logits_out,
-                                 cudaStream_t s) {
+                                 int32_t* hist, cudaStream_t s) {
     const int d = w->cfg.d;
     // bf16 split of W_g (2^-16), the stated order's own rounding ((d/32 + 6) ulps), the
     // tensor cores' accumulation: 2 x (d/16 + 1) MMA steps, 2^-21 of the running sum each
@@ -963,7 +1079,7 @@ cudaError_t launch_router_select(const moe_w8a8_weights* w, const void* x, int T
     if (e != cudaSuccess) return e;
     return launch_pdl(router_select_kernel, dim3((T + kSelWarps - 1) / kSelWarps), dim3(kSelWarps * 32), smem, s,
                       reinterpret_cast<const uint16_t*>(x), approx, bias, w->rt_wt, w->rt_wmax, T, d,
-                      w->cfg.n_experts, w->cfg.top_k, (float)c_err, sel, idx, wts, logits_out);
+                      w->cfg.n_experts, w->cfg.top_k, (float)c_err, sel, idx, wts, logits_out, hist);
 }
 
 cudaError_t launch_topk(const float* logits, const float* bias, int T, int E, int k, int renorm,
@@ -975,11 +1091,13 @@ cudaError_t launch_topk(const float* logits, const float* bias, int T, int E, in
 cudaError_t launch_permute(const int32_t* idx, int T, int k, int E, int cap, int32_t* hist,
                            int32_t* offsets, int32_t* row2ts, int32_t* ts2row, int32_t* meta,
                            int32_t* active, int32_t* tiles, int32_t* pairs, cudaStream_t s, int32_t* zero_words,
-                           int n_zero) {
+                           int n_zero, bool hist_ready) {
     const int n = T * k;
     const int nblk = (n + kPermChunk - 1) / kPermChunk;
-    cudaError_t err = launch_pdl(perm_hist_kernel, dim3(nblk), dim3(256), 0, s, idx, n, E, hist);
-    if (err != cudaSuccess) return err;
+    if (!hist_ready) {
+        cudaError_t err = launch_pdl(perm_hist_kernel, dim3(nblk), dim3(256), 0, s, idx, n, E, hist);
+        if (err != cudaSuccess) return err;
+    }
     return launch_pdl(perm_scatter_kernel, dim3(nblk), dim3(kPermThreads), 0, s, idx, n, E, cap, nblk, hist,
                       offsets, row2ts, ts2row, meta, active, tiles, pairs, zero_words, n_zero);
 }
@@ -991,6 +1109,12 @@ cudaError_t launch_route_small(const float* logits, const float* bias, int T, in
                                int32_t* offsets, int32_t* row2ts, int32_t* ts2row, int32_t* meta,
                                int32_t* active, int32_t* tiles, int32_t* pairs, int32_t* zero_words, int n_zero,
                                cudaStream_t s) {
+    if (T <= 32 && T * k <= kRouteTinyMax) {
+        const int threads = std::max(T * 32, kRouteTinyMax);
+        return launch_pdl(route_tiny_kernel, dim3(1), dim3(threads), sizeof(RouteTinySmem), s, logits, bias, T, E, k,
+                          renorm, cap, idx, wts, logits_out, offsets, row2ts, ts2row, meta, active, tiles, pairs,
+                          zero_words, n_zero);
+    }
     static std::atomic<uint64_t> attr{0};
     cudaError_t e = smem_attr_once(route_small_kernel, sizeof(RouteSmallSmem), attr);
     if (e != cudaSuccess) return e;
@@ -1012,10 +1136,16 @@ cudaError_t launch_smooth_quant(const void* x, int in_dtype, const float* inv_s,
                       sx, aq, aq_ld, wts, idx);
 }
 
-cudaError_t launch_ep_read_experts(const uint8_t* recv, int R, int64_t row_bytes, int d, int ep_first,
-                                   int n_local, int32_t* idx, int32_t* status, cudaStream_t s) {
+cudaError_t launch_ep_read_experts(const uint8_t* recv, int R, int64_t row_bytes, int d, int block_rows,
+                                   int ep_first, int n_local, int32_t* idx, int32_t* status, cudaStream_t s) {
     return launch_pdl(ep_read_experts_kernel, dim3((R + 255) / 256), dim3(256), 0, s, recv, R, row_bytes, d,
-                      ep_first, n_local, idx, status);
+                      block_rows, ep_first, n_local, idx, status);
+}
+
+cudaError_t launch_ep_pack(const uint8_t* send, const int32_t* offsets, const EpRanks& ranks, int world,
+                           int block_rows, int64_t row_bytes, uint8_t* blocks, cudaStream_t s) {
+    return launch_pdl(ep_pack_kernel, dim3((block_rows + kEpGatherWarps - 1) / kEpGatherWarps, world),
+                      dim3(kEpGatherWarps * 32), 0, s, send, offsets, ranks, block_rows, row_bytes, blocks);
 }
 
 cudaError_t launch_ep_gather(const uint8_t* recv, int R, int64_t row_bytes, int d, const int32_t* ts2row,

@@ -234,9 +234,25 @@ __global__ void __launch_bounds__(kStThreads) stream_down_kernel(
 // are bf16 (bf16-output layers), else fp32.  A thread owns 8 channels of one
 // token: the token's row indices first, then all kept slots' loads (16 bytes
 // each for bf16 rows) in flight together, then the sum in slot order.
-template <bool O16>
+// Where a sorted row's output sits in fixed blocks returned by the ranks of
+// an expert-parallel exchange: row r of rank g's experts (rows
+// [offsets[first[g]], offsets[first[g + 1]])) is row 1 + r - offsets[first[g]]
+// of block g (blocks of block_rows rows; row 0 is the header).
+struct BlockMap {
+    const int32_t* offsets;   // null: rows are not blocked
+    EpRanks ranks;
+    int world, block_rows;
+};
+
+__device__ __forceinline__ int block_row(const BlockMap& bm, int r) {
+    int g = 0;
+    while (g + 1 < bm.world && r >= bm.offsets[bm.ranks.first[g + 1]]) ++g;
+    return g * bm.block_rows + 1 + r - bm.offsets[bm.ranks.first[g]];
+}
+
+template <bool O16, bool BLOCKED>
 __global__ void combine_kernel(const void* __restrict__ o, const int32_t* __restrict__ ts2row,
-                               int k, int d, int out_dtype, void* __restrict__ y) {
+                               int k, int d, int out_dtype, void* __restrict__ y, const BlockMap bm) {
     pdl_wait();
     pdl_trigger();
 
@@ -246,6 +262,11 @@ __global__ void combine_kernel(const void* __restrict__ o, const int32_t* __rest
     int rows[kMaxK];
 #pragma unroll
     for (int s = 0; s < kMaxK; ++s) rows[s] = s < k ? ts2row[(int64_t)t * k + s] : -1;
+    if (BLOCKED) {
+#pragma unroll
+        for (int s = 0; s < kMaxK; ++s)
+            if (rows[s] >= 0) rows[s] = block_row(bm, rows[s]);
+    }
     // loads of every kept slot first (raw 16-byte words: few registers, so many
     // warps per SM), then the sum in slot order
     uint4 raw[kMaxK][O16 ? 1 : 2];
@@ -347,8 +368,19 @@ cudaError_t launch_stream_down(const moe_w8a8_weights* w, int T, const int8_t* h
 cudaError_t launch_combine(const void* o, int o_bf16, const int32_t* ts2row, int T, int k, int d,
                            int out_dtype, void* y, cudaStream_t s) {
     dim3 grid(T, (d / 8 + 255) / 256);
-    if (o_bf16) return launch_pdl(combine_kernel<true>, grid, dim3(256), 0, s, o, ts2row, k, d, out_dtype, y);
-    return launch_pdl(combine_kernel<false>, grid, dim3(256), 0, s, o, ts2row, k, d, out_dtype, y);
+    const BlockMap none{};
+    if (o_bf16)
+        return launch_pdl(combine_kernel<true, false>, grid, dim3(256), 0, s, o, ts2row, k, d, out_dtype, y, none);
+    return launch_pdl(combine_kernel<false, false>, grid, dim3(256), 0, s, o, ts2row, k, d, out_dtype, y, none);
+}
+
+cudaError_t launch_combine_blocked(const float* o_blocks, const int32_t* ts2row, const int32_t* offsets,
+                                   const EpRanks& ranks, int world, int block_rows, int T, int k, int d,
+                                   int out_dtype, void* y, cudaStream_t s) {
+    dim3 grid(T, (d / 8 + 255) / 256);
+    const BlockMap bm{offsets, ranks, world, block_rows};
+    return launch_pdl(combine_kernel<false, true>, grid, dim3(256), 0, s, (const void*)o_blocks, ts2row, k, d,
+                      out_dtype, y, bm);
 }
 
 }  // namespace moe

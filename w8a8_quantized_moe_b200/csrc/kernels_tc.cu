@@ -33,6 +33,8 @@
 // returns.
 #include <cuda.h>
 
+#include <climits>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -60,6 +62,12 @@ template <int FMT>
 __host__ __device__ constexpr uint32_t idesc() {
     return (FMT == FMT_E4M3 ? (1u << 4) : ((2u << 4) | (1u << 7) | (1u << 10))) | ((uint32_t)(BN >> 3) << 17) |
            ((uint32_t)(BM >> 4) << 24);
+}
+
+// Row of the tiled weight copy at which k-block kb of the weight rows
+// starting at brow (a multiple of 128) begins: [row tile][k-block][256 rows].
+__device__ __forceinline__ int tiled_row(int brow, int kb, int nkb) {
+    return ((brow / BN) * nkb + kb) * BN + brow % BN;
 }
 
 struct Ctl {
@@ -545,7 +553,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     mbar_arrive_expect_tx(&ctl->full[s], kStageBytes);
                     uint8_t* sa = smem + s * kStageBytes;
                     tma_load_2d(sa, &tm_a, &ctl->full[s], kb * BK, row0);
-                    tma_load_2d(sa + kABytes, &tm_b, &ctl->full[s], kb * BK, brow);
+                    tma_load_2d(sa + kABytes, &tm_b, &ctl->full[s], 0, tiled_row(brow, kb, nkb));
                     issued[s] = true;
                     issued_par[s] = ph;
                     if (++s == kStages) { s = 0; ph ^= 1; }
@@ -827,7 +835,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     const uint32_t bar = leader_addr(&ctl->full[s]);
                     uint8_t* sa = smem + s * kStageBytesP;
                     tma_load_2d_pair(sa, &tm_a, bar, kb * BK, row0);
-                    tma_load_2d_pair(sa + kABytesP, &tm_b, bar, kb * BK, brow);
+                    tma_load_2d_pair(sa + kABytesP, &tm_b, bar, 0, tiled_row(brow, kb, nkb));
                     issued[s] = true;
                     issued_par[s] = ph;
                     if (++s == kStagesP) { s = 0; ph ^= 1; }
@@ -1405,7 +1413,7 @@ template <int EPAD>
 __global__ void __launch_bounds__(kRcThreads, 1)
     router_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_hi,
                      const __grid_constant__ CUtensorMap tm_lo, int T, int d, int E, float* __restrict__ approx,
-                     int32_t* status) {
+                     int32_t* status, int32_t* zero_words, int n_zero) {
     using C = RcCfg<EPAD>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
@@ -1436,6 +1444,9 @@ __global__ void __launch_bounds__(kRcThreads, 1)
     volatile int* abort = &ctl->abort;
     pdl_wait();
     pdl_trigger();
+    // counters the next kernel adds to (the selection's expert histogram)
+    if (blockIdx.x == 0)
+        for (int z = threadIdx.x; z < n_zero; z += blockDim.x) zero_words[z] = 0;
 
     if (warp == 0) {
         if (lane == 0) {
@@ -1637,13 +1648,14 @@ bool make_out_map(CUtensorMap* m, void* base, uint64_t cols, uint64_t rows, bool
 
 template <int EPAD>
 cudaError_t launch_router_tc_pad(const CUtensorMap& mx, const moe_w8a8_weights* w, int T, float* approx,
-                                 cudaStream_t s) {
+                                 int32_t* zero_words, int n_zero, cudaStream_t s) {
     using C = RcCfg<EPAD>;
     static std::atomic<uint64_t> attr{0};
     cudaError_t e = smem_attr_once(router_tc_kernel<EPAD>, C::kSmem, attr);
     if (e != cudaSuccess) return e;
     return launch_pdl(router_tc_kernel<EPAD>, dim3((T + BM - 1) / BM), dim3(kRcThreads), C::kSmem, s, mx,
-                      w->tm_rt_hi, w->tm_rt_lo, T, w->cfg.d, w->cfg.n_experts, approx, w->status);
+                      w->tm_rt_hi, w->tm_rt_lo, T, w->cfg.d, w->cfg.n_experts, approx, w->status, zero_words,
+                      n_zero);
 }
 
 template <int EPI, int FMT>
@@ -1710,9 +1722,39 @@ cudaError_t launch_pair(const CUtensorMap& ta, const CUtensorMap& tb, const CUte
 bool tc_make_weight_maps(moe_w8a8_weights* w) {
     const moe_w8a8_config& c = w->cfg;
     const uint64_t E = w->n_local, d = c.d, f = c.f;   // the experts this handle holds
+    // canonical layout (the fused launch), and the tiled copies as
+    // [rows x k-blocks][128 bytes]: box (0, tiled_row(...)) of 256 (or 128) rows
+    // is one k-block of a tile (or half of it)
+    const uint64_t gu_rows = E * 2 * f * (d / BK), dn_rows = E * d * (f / BK);
     return make_map(&w->tm_w_gu, w->w_gu, d, E * 2 * f, BN) && make_map(&w->tm_w_dn, w->w_dn, f, E * d, BN) &&
-           make_map(&w->tm_w_gu_half, w->w_gu, d, E * 2 * f, BN / 2) &&
-           make_map(&w->tm_w_dn_half, w->w_dn, f, E * d, BN / 2);
+           w->w_gu_t && w->w_dn_t &&
+           make_map(&w->tm_w_gu_t, w->w_gu_t, BK, gu_rows, BN) && make_map(&w->tm_w_dn_t, w->w_dn_t, BK, dn_rows, BN) &&
+           make_map(&w->tm_w_gu_t_half, w->w_gu_t, BK, gu_rows, BN / 2) &&
+           make_map(&w->tm_w_dn_t_half, w->w_dn_t, BK, dn_rows, BN / 2);
+}
+
+namespace {
+// One 32 KB chunk (256 rows x 128 bytes) per block: thread r copies row r's
+// 128 bytes of k-block kb.
+__global__ void __launch_bounds__(256) tile_weights_kernel(const int8_t* __restrict__ src, int K,
+                                                           int8_t* __restrict__ dst) {
+    const int nkb = K / BK;
+    const int64_t chunk = blockIdx.x;
+    const int64_t rt = chunk / nkb;
+    const int kb = (int)(chunk % nkb), r = threadIdx.x;
+    const int4* in = reinterpret_cast<const int4*>(src + (rt * BN + r) * (int64_t)K + kb * BK);
+    int4* out = reinterpret_cast<int4*>(dst + (chunk * BN + r) * BK);
+#pragma unroll
+    for (int j = 0; j < BK / 16; ++j) out[j] = in[j];
+}
+}  // namespace
+
+cudaError_t launch_tile_weights(const int8_t* src, int64_t rows, int K, int8_t* dst, cudaStream_t s) {
+    if (rows % BN || K % BK) return cudaErrorInvalidValue;
+    const int64_t chunks = rows / BN * (K / BK);
+    if (chunks > INT32_MAX) return cudaErrorInvalidValue;
+    tile_weights_kernel<<<(unsigned)chunks, 256, 0, s>>>(src, K, dst);
+    return cudaGetLastError();
 }
 
 template <int FMT>
@@ -1778,13 +1820,14 @@ bool router_tc_make_maps(moe_w8a8_weights* w) {
            make_map_bf16(&w->tm_rt_lo, w->rt_lo, w->cfg.d, w->rt_epad, w->rt_epad);
 }
 
-cudaError_t launch_router_tc(const moe_w8a8_weights* w, const void* x, int T, float* approx, cudaStream_t s) {
+cudaError_t launch_router_tc(const moe_w8a8_weights* w, const void* x, int T, float* approx, int32_t* zero_words,
+                             int n_zero, cudaStream_t s) {
     CUtensorMap mx;
     if (!make_map_bf16(&mx, x, w->cfg.d, T, BM)) return cudaErrorInvalidValue;
     switch (w->rt_epad) {
-        case 64: return launch_router_tc_pad<64>(mx, w, T, approx, s);
-        case 128: return launch_router_tc_pad<128>(mx, w, T, approx, s);
-        case 256: return launch_router_tc_pad<256>(mx, w, T, approx, s);
+        case 64: return launch_router_tc_pad<64>(mx, w, T, approx, zero_words, n_zero, s);
+        case 128: return launch_router_tc_pad<128>(mx, w, T, approx, zero_words, n_zero, s);
+        case 256: return launch_router_tc_pad<256>(mx, w, T, approx, zero_words, n_zero, s);
     }
     return cudaErrorInvalidValue;
 }
@@ -1843,11 +1886,11 @@ cudaError_t launch_tc_gemm1(const moe_w8a8_weights* w, int T, const int8_t* aq, 
     p.tma_c = 1;
     if (pairs) {
         const int max_pt = (rows + 2 * BM - 1) / (2 * BM) + w->n_local;
-        return launch_pair<EPI_SWIGLU>(ta, w->tm_w_gu_half, tc, p, max_pt * p.n_tiles_n, c.expert_format, s);
+        return launch_pair<EPI_SWIGLU>(ta, w->tm_w_gu_t_half, tc, p, max_pt * p.n_tiles_n, c.expert_format, s);
     }
     const int max_mt = (rows + BM - 1) / BM + c.n_experts;
     const int grid = max(1, min(w->num_sms, max_mt * p.n_tiles_n));
-    return launch<EPI_SWIGLU>(ta, w->tm_w_gu, tc, p, grid, c.expert_format, s);
+    return launch<EPI_SWIGLU>(ta, w->tm_w_gu_t, tc, p, grid, c.expert_format, s);
 }
 
 cudaError_t launch_tc_gemm2(const moe_w8a8_weights* w, int T, const int8_t* hq, const float* sh,
@@ -1883,11 +1926,11 @@ cudaError_t launch_tc_gemm2(const moe_w8a8_weights* w, int T, const int8_t* hq, 
     p.tma_c = p.o_bf16;
     if (pairs) {
         const int max_pt = (rows + 2 * BM - 1) / (2 * BM) + w->n_local;
-        return launch_pair<EPI_DOWN>(ta, w->tm_w_dn_half, tc, p, max_pt * p.n_tiles_n, c.expert_format, s);
+        return launch_pair<EPI_DOWN>(ta, w->tm_w_dn_t_half, tc, p, max_pt * p.n_tiles_n, c.expert_format, s);
     }
     const int max_mt = (rows + BM - 1) / BM + c.n_experts;
     const int grid = max(1, min(w->num_sms, max_mt * p.n_tiles_n));
-    return launch<EPI_DOWN>(ta, w->tm_w_dn, tc, p, grid, c.expert_format, s);
+    return launch<EPI_DOWN>(ta, w->tm_w_dn_t, tc, p, grid, c.expert_format, s);
 }
 
 }  // namespace moe

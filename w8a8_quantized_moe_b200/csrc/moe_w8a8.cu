@@ -6,6 +6,7 @@
 #include <algorithm>
 #include <cmath>
 #include <cstdlib>
+#include <climits>
 #include <cstring>
 #include <mutex>
 #include <vector>
@@ -90,6 +91,8 @@ void free_handle(moe_w8a8_weights* w) {
     prof_free(w);
     cudaFree(w->w_gu);
     cudaFree(w->w_dn);
+    cudaFree(w->w_gu_t);
+    cudaFree(w->w_dn_t);
     cudaFree(w->sw_gate);
     cudaFree(w->sw_up);
     cudaFree(w->sw_dn);
@@ -348,7 +351,18 @@ moe_status prepare_impl(const moe_w8a8_config* cfg, int e_first, int n_local, co
             cudaSuccess ||
         cudaStreamSynchronize(s) != cudaSuccess)
         return fail(MOE_ERR_CUDA);
-    w->tmaps_ok = tc_make_weight_maps(w);
+    // the tensor-core kernels' tiled copies (only for layers they serve)
+    if (tc_supported(c)) {
+        if (cudaMalloc(&w->w_gu_t, n_gu) != cudaSuccess || cudaMalloc(&w->w_dn_t, n_dn) != cudaSuccess) {
+            cudaGetLastError();
+            return fail(MOE_ERR_OOM);
+        }
+        if (launch_tile_weights(w->w_gu, (int64_t)E * 2 * f, d, w->w_gu_t, s) != cudaSuccess ||
+            launch_tile_weights(w->w_dn, (int64_t)E * d, f, w->w_dn_t, s) != cudaSuccess ||
+            cudaStreamSynchronize(s) != cudaSuccess)
+            return fail(MOE_ERR_CUDA);
+        w->tmaps_ok = tc_make_weight_maps(w);
+    }
     prepare_router_tc(w, s);
     cudaFree(tmp);
     *out = w;
@@ -424,11 +438,15 @@ moe_status route_stage(Run& r, const void* x, int T, const float* bias, const fl
     if (certified) {
         // approximate logits on the tensor cores, then per token the candidates'
         // logits in the stated order, top-k and gate weights
+        // (the selection also counts the permutation's histogram, which the
+        // approximate-logit kernel zeroes)
+        const int n_hist = (int)(((size_t)T * k + kPermChunk - 1) / kPermChunk) * E;
         r.mark(MOE_STAGE_ROUTER, 0);
-        CUDA_TRY(launch_router_tc(w, x, T, logits, s));
+        CUDA_TRY(launch_router_tc(w, x, T, logits, r.at<int32_t>(L.hist), n_hist, s));
         r.mark(MOE_STAGE_ROUTER, 1);
         r.mark(MOE_STAGE_TOPK, 0);
-        CUDA_TRY(launch_router_select(w, x, T, logits, bias, r.at<float>(L.logits_sel), idx, wts, dbg_logits, s));
+        CUDA_TRY(launch_router_select(w, x, T, logits, bias, r.at<float>(L.logits_sel), idx, wts, dbg_logits,
+                                      r.at<int32_t>(L.hist), s));
         r.mark(MOE_STAGE_TOPK, 1);
         r.launches += 2;
     } else if (!lsrc) {
@@ -446,9 +464,9 @@ moe_status route_stage(Run& r, const void* x, int T, const float* bias, const fl
     if (certified) {
         r.mark(MOE_STAGE_PERMUTE, 0);
         CUDA_TRY(launch_permute(idx, T, k, E, capacity_of(c, T), r.at<int32_t>(L.hist), offsets, row2ts, ts2row,
-                                meta, active, tiles, r.at<int32_t>(L.pairs), s, zero_words, n_zero));
+                                meta, active, tiles, r.at<int32_t>(L.pairs), s, zero_words, n_zero, true));
         r.mark(MOE_STAGE_PERMUTE, 1);
-        r.launches += 2;
+        r.launches += 1;
     } else if (route_small_ok(T, k)) {
         // top-k, histogram, scan and scatter in one block
         r.mark(MOE_STAGE_TOPK, 0);
@@ -919,15 +937,36 @@ moe_status moe_w8a8_ep_dispatch(const moe_w8a8_weights* w, const void* x, int32_
     return MOE_OK;
 }
 
-moe_status moe_w8a8_ep_experts(const moe_w8a8_weights* w, const void* recv, int32_t R, float* o_rows,
-                               void* workspace, size_t workspace_bytes, const moe_w8a8_debug* dbg,
-                               moe_stream_t stream) {
-    if (!w || R < 0) return MOE_ERR_INVALID_ARG;
-    if (R == 0) return MOE_OK;
+namespace moe {
+namespace {
+
+// The expert view of an expert-parallel handle for R received rows; for rows
+// in fixed blocks of block_rows rows (0: contiguous rows), a decode-sized
+// block (capacity within the fused launch's limit) keeps the fused launch for
+// all R rows, most of which are unused slots of the blocks.
+moe_w8a8_weights ep_view(const moe_w8a8_weights* w, int R, int block_rows) {
+    moe_w8a8_weights v = expert_view(w);
+    if (block_rows > 0 && block_rows - 1 <= w->fused_max_rows) v.fused_max_rows = std::max<int64_t>(v.fused_max_rows, R);
+    return v;
+}
+
+bool ep_ranks(const moe_w8a8_weights* w, const int32_t* rank_first, int32_t world, EpRanks& out) {
+    if (!rank_first || world < 1 || world > kEpMaxWorld || rank_first[0] != 0 ||
+        rank_first[world] != w->cfg.n_experts)
+        return false;
+    for (int g = 0; g < world; ++g)
+        if (rank_first[g + 1] <= rank_first[g]) return false;
+    for (int g = 0; g <= kEpMaxWorld; ++g) out.first[g] = g <= world ? rank_first[g] : w->cfg.n_experts;
+    return true;
+}
+
+moe_status ep_experts_impl(const moe_w8a8_weights* w, const void* recv, int32_t R, int block_rows, float* o_rows,
+                           void* workspace, size_t workspace_bytes, const moe_w8a8_debug* dbg,
+                           moe_stream_t stream) {
     if (!recv || !o_rows || !workspace) return MOE_ERR_INVALID_ARG;
     if ((uintptr_t)workspace % kAlign || misaligned16(recv) || misaligned16(o_rows)) return MOE_ERR_INVALID_ARG;
     if (!on_handle_device(w)) return MOE_ERR_INVALID_ARG;
-    const moe_w8a8_weights v = expert_view(w);
+    const moe_w8a8_weights v = ep_view(w, R, block_rows);
     if (!path_ok(&v, R)) return MOE_ERR_UNSUPPORTED_SHAPE;
     const int path = choose_path(&v, R);
     const WsLayout L = ws_layout(&v, R, WS_EXPERTS);
@@ -942,7 +981,8 @@ moe_status moe_w8a8_ep_experts(const moe_w8a8_weights* w, const void* recv, int3
     int32_t* ts2row = r.at<int32_t>(L.ts2row);
     if (L.fused_words > 0) CUDA_TRY(cudaMemsetAsync(r.at<int32_t>(L.fused_sync), 0, (size_t)L.fused_words * 4, s));
     // each received row is one (token, slot) pair with k = 1 of the local experts
-    CUDA_TRY(launch_ep_read_experts(rows, R, rb, d, w->ep_first, w->n_local, idx, w->status, s));
+    // (in fixed blocks: headers and unused rows left out)
+    CUDA_TRY(launch_ep_read_experts(rows, R, rb, d, block_rows, w->ep_first, w->n_local, idx, w->status, s));
     CUDA_TRY(launch_permute(idx, R, 1, v.cfg.n_experts, -1, r.at<int32_t>(L.hist), r.at<int32_t>(L.offsets),
                             r.at<int32_t>(L.row2ts), ts2row, r.at<int32_t>(L.meta), r.at<int32_t>(L.active),
                             r.at<int32_t>(L.tiles), r.at<int32_t>(L.pairs), s));
@@ -952,11 +992,85 @@ moe_status moe_w8a8_ep_experts(const moe_w8a8_weights* w, const void* recv, int3
                               r.at<float>(L.topk_w), s));
     r.launches += 4;
     MOE_TRY(expert_stage(r, R, path));
-    // un-sort: O of received row r to o_rows[r] (k = 1)
+    // un-sort: O of received row r to o_rows[r] (k = 1; rows left out get zeros)
     CUDA_TRY(launch_combine(r.at<void>(L.o), v.cfg.out_dtype == MOE_BF16, ts2row, R, 1, d, MOE_F32, o_rows, s));
     ++r.launches;
     MOE_TRY(debug_stage(r, R, 1, v.cfg.n_experts, false, true));
     const_cast<moe_w8a8_weights*>(w)->last_launches = r.launches;
+    return MOE_OK;
+}
+
+}  // namespace
+}  // namespace moe
+
+moe_status moe_w8a8_ep_experts(const moe_w8a8_weights* w, const void* recv, int32_t R, float* o_rows,
+                               void* workspace, size_t workspace_bytes, const moe_w8a8_debug* dbg,
+                               moe_stream_t stream) {
+    if (!w || R < 0) return MOE_ERR_INVALID_ARG;
+    if (R == 0) return MOE_OK;
+    return ep_experts_impl(w, recv, R, 0, o_rows, workspace, workspace_bytes, dbg, stream);
+}
+
+int32_t moe_w8a8_ep_block_rows(const moe_w8a8_weights* w, int32_t block_tokens) {
+    if (!w || block_tokens < 1 || (int64_t)block_tokens * w->cfg.top_k + 1 > INT32_MAX / 64) return 0;
+    return block_tokens * w->cfg.top_k + 1;
+}
+
+moe_status moe_w8a8_ep_pack(const moe_w8a8_weights* w, const void* send, const int32_t* expert_offsets,
+                            const int32_t* rank_first, int32_t world, int32_t block_tokens, void* blocks,
+                            moe_stream_t stream) {
+    if (!w) return MOE_ERR_INVALID_ARG;
+    const int block_rows = moe_w8a8_ep_block_rows(w, block_tokens);
+    EpRanks ranks;
+    if (block_rows == 0 || !ep_ranks(w, rank_first, world, ranks)) return MOE_ERR_INVALID_ARG;
+    if (!send || !expert_offsets || !blocks || misaligned16(send) || misaligned16(blocks))
+        return MOE_ERR_INVALID_ARG;
+    if (!on_handle_device(w)) return MOE_ERR_INVALID_ARG;
+    CUDA_TRY(launch_ep_pack((const uint8_t*)send, expert_offsets, ranks, world, block_rows,
+                            (int64_t)w->cfg.d + kEpTrailerBytes, (uint8_t*)blocks, (cudaStream_t)stream));
+    const_cast<moe_w8a8_weights*>(w)->last_launches = 1;
+    return MOE_OK;
+}
+
+size_t moe_w8a8_ep_experts_blocked_workspace_size(const moe_w8a8_weights* w, int32_t world,
+                                                  int32_t block_tokens) {
+    if (!w || world < 1 || world > kEpMaxWorld) return 0;
+    const int block_rows = moe_w8a8_ep_block_rows(w, block_tokens);
+    if (block_rows == 0) return 0;
+    const int R = world * block_rows;
+    const moe_w8a8_weights v = ep_view(w, R, block_rows);
+    return ws_layout(&v, R, WS_EXPERTS).total;
+}
+
+moe_status moe_w8a8_ep_experts_blocked(const moe_w8a8_weights* w, const void* blocks, int32_t world,
+                                       int32_t block_tokens, float* o_blocks, void* workspace,
+                                       size_t workspace_bytes, const moe_w8a8_debug* dbg, moe_stream_t stream) {
+    if (!w || world < 1 || world > kEpMaxWorld) return MOE_ERR_INVALID_ARG;
+    const int block_rows = moe_w8a8_ep_block_rows(w, block_tokens);
+    if (block_rows == 0) return MOE_ERR_INVALID_ARG;
+    return ep_experts_impl(w, blocks, world * block_rows, block_rows, o_blocks, workspace, workspace_bytes, dbg,
+                           stream);
+}
+
+moe_status moe_w8a8_ep_combine_blocked(const moe_w8a8_weights* w, const float* o_blocks, int32_t T,
+                                       const int32_t* rank_first, int32_t world, int32_t block_tokens, void* y,
+                                       const void* workspace, size_t workspace_bytes, moe_stream_t stream) {
+    if (!w || T < 0) return MOE_ERR_INVALID_ARG;
+    const int block_rows = moe_w8a8_ep_block_rows(w, block_tokens);
+    EpRanks ranks;
+    if (block_rows == 0 || !ep_ranks(w, rank_first, world, ranks) || T > block_tokens) return MOE_ERR_INVALID_ARG;
+    if (T == 0) return MOE_OK;
+    if (!y || !o_blocks || !workspace) return MOE_ERR_INVALID_ARG;
+    if ((uintptr_t)workspace % kAlign || misaligned16(o_blocks) || misaligned16(y)) return MOE_ERR_INVALID_ARG;
+    if (!on_handle_device(w)) return MOE_ERR_INVALID_ARG;
+    const moe_w8a8_config& c = w->cfg;
+    const WsLayout L = ws_layout(w, T, WS_ROUTE);
+    if (workspace_bytes < L.total) return MOE_ERR_WORKSPACE_TOO_SMALL;
+    const int32_t* ts2row = (const int32_t*)((const char*)workspace + L.ts2row);
+    const int32_t* offsets = (const int32_t*)((const char*)workspace + L.offsets);
+    CUDA_TRY(launch_combine_blocked(o_blocks, ts2row, offsets, ranks, world, block_rows, T, c.top_k, c.d,
+                                    c.out_dtype, y, (cudaStream_t)stream));
+    const_cast<moe_w8a8_weights*>(w)->last_launches = 1;
     return MOE_OK;
 }
 

@@ -13,10 +13,19 @@ sender, and sums its tokens' slots in slot order (``moe_w8a8_ep_combine``).
 Every rank's output equals the single-GPU layer on that rank's tokens.
 
 The exchange is ``all_to_all_single`` of the process group (NCCL over
-NVLink/NVSwitch on GPUs, gloo on CPU for the tests).  Its split sizes follow
-the routing: the per-peer row counts are formed on the device from the row
-offsets, exchanged, and read by the host together, once per layer.  All
-arithmetic of the layer runs in the library's kernels; this module moves
+NVLink/NVSwitch on GPUs, gloo on CPU for the tests), in one of two forms:
+
+- counted (default): split sizes follow the routing; the per-peer row counts
+  are formed on the device from the row offsets, exchanged, and read by the
+  host together, once per layer;
+- fixed blocks (``block_tokens=B``, every rank's T <= B): each rank sends
+  every peer one block of B k + 1 rows, a header row holding the count and
+  then the rows (``moe_w8a8_ep_pack``), and gets one output block back, so
+  both All-to-Alls have sizes known in advance and no count reaches the host;
+  the experts read the counts on the device.  Worst-case bytes on the links
+  for no host round trip: the form for decode-sized batches.
+
+All arithmetic of the layer runs in the library's kernels; this module moves
 buffers and picks split sizes.
 """
 from __future__ import annotations
@@ -75,17 +84,38 @@ class LibraryStages:
     def combine(self, o_rows, T, y, ws):
         M.moe_w8a8_ep_combine(self.w, o_rows, T, y, ws)
 
+    # fixed-block exchange
+    def block_rows(self, B):
+        return M.moe_w8a8_ep_block_rows(self.w, B)
+
+    def pack(self, send, offsets, rank_first, B, blocks):
+        M.moe_w8a8_ep_pack(self.w, send, offsets, rank_first, B, blocks)
+
+    def experts_blocked_workspace(self, world, B):
+        return M.moe_w8a8_ep_experts_blocked_workspace_size(self.w, world, B)
+
+    def experts_blocked(self, blocks, world, B, o_blocks, ws):
+        M.moe_w8a8_ep_experts_blocked(self.w, blocks, world, B, o_blocks, ws)
+
+    def combine_blocked(self, o_blocks, T, rank_first, B, y, ws):
+        M.moe_w8a8_ep_combine_blocked(self.w, o_blocks, T, rank_first, B, y, ws)
+
 
 class ExpertParallelMoE:
     """One rank of the expert-parallel layer.
 
-    stages  the compute steps (``LibraryStages`` on a GPU)
-    ranges  (first expert, count) of every rank, contiguous and ascending;
-            equal ranges by default
+    stages        the compute steps (``LibraryStages`` on a GPU)
+    ranges        (first expert, count) of every rank, contiguous and
+                  ascending; equal ranges by default
+    block_tokens  None: the counted exchange; B: the fixed-block exchange,
+                  every rank's T <= B (all ranks must pass the same B)
     """
 
-    def __init__(self, stages, group=None, ranges=None):
+    def __init__(self, stages, group=None, ranges=None, block_tokens=None):
         self.stages = stages
+        if block_tokens is not None and block_tokens < 1:
+            raise ValueError("block_tokens must be at least 1")
+        self.block_tokens = block_tokens
         self.group = group
         self.rank = dist.get_rank(group)
         self.world = dist.get_world_size(group)
@@ -100,7 +130,8 @@ class ExpertParallelMoE:
         if nxt != stages.E:
             raise ValueError("expert ranges must cover every expert")
         self._bufs: dict[str, torch.Tensor] = {}
-        self.last_rows = (0, 0)   # rows sent, rows received by the last forward
+        self.last_rows = (0, 0)   # rows sent, rows received by the last counted forward
+        self._rank_first = [first for first, _ in self.ranges] + [stages.E]
         # row-offset indices of each destination's first expert and one past its last
         self._lo = torch.tensor([first for first, _ in self.ranges], dtype=torch.long, device=stages.device)
         self._hi = torch.tensor([first + n for first, n in self.ranges], dtype=torch.long, device=stages.device)
@@ -114,6 +145,8 @@ class ExpertParallelMoE:
         return b[:n]
 
     def forward(self, x, T: int, router_bias=None, router_logits=None, y=None):
+        if self.block_tokens is not None:
+            return self._forward_blocked(x, T, router_bias, router_logits, y)
         st = self.stages
         k, E, d, rb = st.k, st.E, st.d, st.row_bytes
         send = self._buf("send", T * k * rb, torch.uint8)
@@ -145,4 +178,31 @@ class ExpertParallelMoE:
             y = torch.empty((T, d), dtype=st.out_dtype, device=st.device)
         st.combine(o_back.view(R_send, d), T, y, ws_route)
         self.last_rows = (R_send, R_recv)
+        return y
+
+    def _forward_blocked(self, x, T: int, router_bias, router_logits, y):
+        """The fixed-block exchange: nothing of this forward is read by the host."""
+        st = self.stages
+        B = self.block_tokens
+        if T > B:
+            raise ValueError(f"T={T} exceeds the exchange's block of {B} tokens")
+        k, E, d, rb, G = st.k, st.E, st.d, st.row_bytes, self.world
+        rows = st.block_rows(B)
+        send = self._buf("send", B * k * rb, torch.uint8)
+        offsets = self._buf("offsets", E + 1, torch.int32)
+        ws_route = self._buf("ws_route", st.dispatch_workspace(B), torch.uint8)
+        st.dispatch(x, T, router_bias, router_logits, send, offsets, ws_route)
+        blocks = self._buf("blocks", G * rows * rb, torch.uint8)
+        st.pack(send, offsets, self._rank_first, B, blocks)
+        recv = self._buf("recv_blocks", G * rows * rb, torch.uint8)
+        dist.all_to_all_single(recv, blocks, group=self.group)            # one block per peer each way
+        o_blocks = self._buf("o_blocks", G * rows * d, torch.float32)
+        ws_exp = self._buf("ws_experts_blocked", st.experts_blocked_workspace(G, B), torch.uint8)
+        st.experts_blocked(recv, G, B, o_blocks, ws_exp)
+        o_back = self._buf("o_back_blocks", G * rows * d, torch.float32)
+        dist.all_to_all_single(o_back, o_blocks, group=self.group)
+        if y is None:
+            y = torch.empty((T, d), dtype=st.out_dtype, device=st.device)
+        st.combine_blocked(o_back, T, self._rank_first, B, y, ws_route)
+        self.last_rows = (None, None)
         return y
