@@ -131,12 +131,10 @@ cudaError_t launch_topk(const float* logits, const float* bias, int T, int E, in
                         int32_t* idx, float* wts, float* logits_out, cudaStream_t s);
 // zero_words[0, n_zero): counters a later kernel of the forward starts from
 // zero (the fused expert launch); block 0 of the scatter clears them.
-// hist_ready: `hist` ([chunks][E], kPermChunk entries per chunk) was already
-// counted (by the certified router's selection); only the scatter runs.
 cudaError_t launch_permute(const int32_t* idx, int T, int k, int E, int cap, int32_t* hist,
                            int32_t* offsets, int32_t* row2ts, int32_t* ts2row, int32_t* meta,
                            int32_t* active, int32_t* tiles, int32_t* pairs, cudaStream_t s,
-                           int32_t* zero_words = nullptr, int n_zero = 0, bool hist_ready = false);
+                           int32_t* zero_words = nullptr, int n_zero = 0);
 bool route_small_ok(int T, int k);
 cudaError_t launch_route_small(const float* logits, const float* bias, int T, int E, int k,
                                int renorm, int cap, int32_t* idx, float* wts, float* logits_out,
@@ -202,14 +200,10 @@ cudaError_t launch_tile_weights(const int8_t* src, int64_t rows, int K, int8_t* 
 // bound, their logits in the stated fp32 order, top-k and gate weights
 // (kernels_route.cu).  sel: [T][E] scratch.
 bool router_tc_make_maps(moe_w8a8_weights* w);
-// Also zeroes zero_words[0, n_zero) (the selection's histogram) before it ends.
-cudaError_t launch_router_tc(const moe_w8a8_weights* w, const void* x, int T, float* approx, int32_t* zero_words,
-                             int n_zero, cudaStream_t s);
-// Also counts the chosen (token, slot) entries per kPermChunk chunk and
-// expert into hist ([chunks][E], zeroed beforehand), for the permutation.
+cudaError_t launch_router_tc(const moe_w8a8_weights* w, const void* x, int T, float* approx, cudaStream_t s);
 cudaError_t launch_router_select(const moe_w8a8_weights* w, const void* x, int T, const float* approx,
                                  const float* bias, float* sel, int32_t* idx, float* wts, float* logits_out,
-                                 int32_t* hist, cudaStream_t s);
+                                 cudaStream_t s);
 constexpr int kRouterTcMinTokens = 1024;   // the certified router runs from this many tokens up
 bool tc_supported(const moe_w8a8_config& c);
 // n_mma back-to-back M=128 N=256 K=32 8-bit MMAs per CTA on `grid` CTAs

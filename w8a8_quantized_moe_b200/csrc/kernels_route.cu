@@ -323,9 +323,8 @@ __device__ __forceinline__ bool better(float v, int i, float v2, int i2) {
 
 // One warp: top-k and gate weights of token t.  lsh: kMaxE floats of shared
 // scratch for this warp (used when the softmax runs over all E experts).
-// When idx_copy is given, the chosen experts are also written there.  Returns
-// the expert of slot `lane` to lanes below k (-1 to the others).
-__device__ __forceinline__ int topk_token(const float* __restrict__ logits,
+// When idx_copy is given, the chosen experts are also written there.
+__device__ __forceinline__ void topk_token(const float* __restrict__ logits,
                                            const float* __restrict__ bias, int t, int E, int k,
                                            int renorm, int32_t* __restrict__ idx,
                                            float* __restrict__ wts, float* __restrict__ logits_out,
@@ -380,7 +379,6 @@ __device__ __forceinline__ int topk_token(const float* __restrict__ logits,
     } else {
         for (int e = 0; e < E; ++e) z = __fadd_rn(z, moe_exp(__fsub_rn(lsh[e], lmax)));
     }
-    int mine = -1;
 #pragma unroll
     for (int s = 0; s < kMaxK; ++s) {
         if (s >= k) break;
@@ -388,10 +386,8 @@ __device__ __forceinline__ int topk_token(const float* __restrict__ logits,
             idx[(int64_t)t * k + s] = sel_i[s];
             wts[(int64_t)t * k + s] = __fdiv_rn(moe_exp(__fsub_rn(sel_v[s], lmax)), z);
             if (idx_copy) idx_copy[t * k + s] = sel_i[s];
-            mine = sel_i[s];
         }
     }
-    return mine;
 }
 
 __global__ void topk_kernel(const float* __restrict__ logits, const float* __restrict__ bias, int T,
@@ -440,8 +436,7 @@ __device__ __forceinline__ float4 ld_lane4(const float* rowbase, int j, int lane
 __global__ void __launch_bounds__(kSelWarps * 32) router_select_kernel(
     const uint16_t* __restrict__ x, const float* __restrict__ approx, const float* __restrict__ bias,
     const float* __restrict__ wt, const float* __restrict__ wmax, int T, int d, int E, int k, float c_err,
-    float* __restrict__ sel, int32_t* __restrict__ idx, float* __restrict__ wts, float* __restrict__ logits_out,
-    int32_t* __restrict__ hist) {
+    float* __restrict__ sel, int32_t* __restrict__ idx, float* __restrict__ wts, float* __restrict__ logits_out) {
     pdl_wait();
     pdl_trigger();
 
@@ -577,9 +572,7 @@ __global__ void __launch_bounds__(kSelWarps * 32) router_select_kernel(
         }
     }
     __syncwarp();
-    const int e = topk_token(sel, nullptr, t, E, k, 1, idx, wts, nullptr, lsh, nullptr, lane);
-    // the permutation's histogram: entry t k + s (expert e of lane s) of chunk (t k + s) / kPermChunk
-    if (lane < k) atomicAdd(&hist[(int64_t)((t * k + lane) / kPermChunk) * E + e], 1);
+    topk_token(sel, nullptr, t, E, k, 1, idx, wts, nullptr, lsh, nullptr, lane);
 }
 
 // ---------------------------------------------------------------------------
@@ -1066,7 +1059,7 @@ cudaError_t launch_router_logits(const void* x, int in_dtype, const float* wr, i
 
 cudaError_t launch_router_select(const moe_w8a8_weights* w, const void* x, int T, const float* approx,
                                  const float* bias, float* sel, int32_t* idx, float* wts, float* logits_out,
-                                 int32_t* hist, cudaStream_t s) {
+                                 cudaStream_t s) {
     const int d = w->cfg.d;
     // bf16 split of W_g (2^-16), the stated order's own rounding ((d/32 + 6) ulps), the
     // tensor cores' accumulation: 2 x (d/16 + 1) MMA steps, 2^-21 of the running sum each
@@ -1079,7 +1072,7 @@ cudaError_t launch_router_select(const moe_w8a8_weights* w, const void* x, int T
     if (e != cudaSuccess) return e;
     return launch_pdl(router_select_kernel, dim3((T + kSelWarps - 1) / kSelWarps), dim3(kSelWarps * 32), smem, s,
                       reinterpret_cast<const uint16_t*>(x), approx, bias, w->rt_wt, w->rt_wmax, T, d,
-                      w->cfg.n_experts, w->cfg.top_k, (float)c_err, sel, idx, wts, logits_out, hist);
+                      w->cfg.n_experts, w->cfg.top_k, (float)c_err, sel, idx, wts, logits_out);
 }
 
 cudaError_t launch_topk(const float* logits, const float* bias, int T, int E, int k, int renorm,
@@ -1091,13 +1084,11 @@ cudaError_t launch_topk(const float* logits, const float* bias, int T, int E, in
 cudaError_t launch_permute(const int32_t* idx, int T, int k, int E, int cap, int32_t* hist,
                            int32_t* offsets, int32_t* row2ts, int32_t* ts2row, int32_t* meta,
                            int32_t* active, int32_t* tiles, int32_t* pairs, cudaStream_t s, int32_t* zero_words,
-                           int n_zero, bool hist_ready) {
+                           int n_zero) {
     const int n = T * k;
     const int nblk = (n + kPermChunk - 1) / kPermChunk;
-    if (!hist_ready) {
-        cudaError_t err = launch_pdl(perm_hist_kernel, dim3(nblk), dim3(256), 0, s, idx, n, E, hist);
-        if (err != cudaSuccess) return err;
-    }
+    cudaError_t err = launch_pdl(perm_hist_kernel, dim3(nblk), dim3(256), 0, s, idx, n, E, hist);
+    if (err != cudaSuccess) return err;
     return launch_pdl(perm_scatter_kernel, dim3(nblk), dim3(kPermThreads), 0, s, idx, n, E, cap, nblk, hist,
                       offsets, row2ts, ts2row, meta, active, tiles, pairs, zero_words, n_zero);
 }

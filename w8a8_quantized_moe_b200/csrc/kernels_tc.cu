@@ -1413,7 +1413,7 @@ template <int EPAD>
 __global__ void __launch_bounds__(kRcThreads, 1)
     router_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_hi,
                      const __grid_constant__ CUtensorMap tm_lo, int T, int d, int E, float* __restrict__ approx,
-                     int32_t* status, int32_t* zero_words, int n_zero) {
+                     int32_t* status) {
     using C = RcCfg<EPAD>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
@@ -1444,9 +1444,6 @@ __global__ void __launch_bounds__(kRcThreads, 1)
     volatile int* abort = &ctl->abort;
     pdl_wait();
     pdl_trigger();
-    // counters the next kernel adds to (the selection's expert histogram)
-    if (blockIdx.x == 0)
-        for (int z = threadIdx.x; z < n_zero; z += blockDim.x) zero_words[z] = 0;
 
     if (warp == 0) {
         if (lane == 0) {
@@ -1648,14 +1645,13 @@ bool make_out_map(CUtensorMap* m, void* base, uint64_t cols, uint64_t rows, bool
 
 template <int EPAD>
 cudaError_t launch_router_tc_pad(const CUtensorMap& mx, const moe_w8a8_weights* w, int T, float* approx,
-                                 int32_t* zero_words, int n_zero, cudaStream_t s) {
+                                 cudaStream_t s) {
     using C = RcCfg<EPAD>;
     static std::atomic<uint64_t> attr{0};
     cudaError_t e = smem_attr_once(router_tc_kernel<EPAD>, C::kSmem, attr);
     if (e != cudaSuccess) return e;
     return launch_pdl(router_tc_kernel<EPAD>, dim3((T + BM - 1) / BM), dim3(kRcThreads), C::kSmem, s, mx,
-                      w->tm_rt_hi, w->tm_rt_lo, T, w->cfg.d, w->cfg.n_experts, approx, w->status, zero_words,
-                      n_zero);
+                      w->tm_rt_hi, w->tm_rt_lo, T, w->cfg.d, w->cfg.n_experts, approx, w->status);
 }
 
 template <int EPI, int FMT>
@@ -1820,14 +1816,13 @@ bool router_tc_make_maps(moe_w8a8_weights* w) {
            make_map_bf16(&w->tm_rt_lo, w->rt_lo, w->cfg.d, w->rt_epad, w->rt_epad);
 }
 
-cudaError_t launch_router_tc(const moe_w8a8_weights* w, const void* x, int T, float* approx, int32_t* zero_words,
-                             int n_zero, cudaStream_t s) {
+cudaError_t launch_router_tc(const moe_w8a8_weights* w, const void* x, int T, float* approx, cudaStream_t s) {
     CUtensorMap mx;
     if (!make_map_bf16(&mx, x, w->cfg.d, T, BM)) return cudaErrorInvalidValue;
     switch (w->rt_epad) {
-        case 64: return launch_router_tc_pad<64>(mx, w, T, approx, zero_words, n_zero, s);
-        case 128: return launch_router_tc_pad<128>(mx, w, T, approx, zero_words, n_zero, s);
-        case 256: return launch_router_tc_pad<256>(mx, w, T, approx, zero_words, n_zero, s);
+        case 64: return launch_router_tc_pad<64>(mx, w, T, approx, s);
+        case 128: return launch_router_tc_pad<128>(mx, w, T, approx, s);
+        case 256: return launch_router_tc_pad<256>(mx, w, T, approx, s);
     }
     return cudaErrorInvalidValue;
 }

@@ -438,15 +438,11 @@ moe_status route_stage(Run& r, const void* x, int T, const float* bias, const fl
     if (certified) {
         // approximate logits on the tensor cores, then per token the candidates'
         // logits in the stated order, top-k and gate weights
-        // (the selection also counts the permutation's histogram, which the
-        // approximate-logit kernel zeroes)
-        const int n_hist = (int)(((size_t)T * k + kPermChunk - 1) / kPermChunk) * E;
         r.mark(MOE_STAGE_ROUTER, 0);
-        CUDA_TRY(launch_router_tc(w, x, T, logits, r.at<int32_t>(L.hist), n_hist, s));
+        CUDA_TRY(launch_router_tc(w, x, T, logits, s));
         r.mark(MOE_STAGE_ROUTER, 1);
         r.mark(MOE_STAGE_TOPK, 0);
-        CUDA_TRY(launch_router_select(w, x, T, logits, bias, r.at<float>(L.logits_sel), idx, wts, dbg_logits,
-                                      r.at<int32_t>(L.hist), s));
+        CUDA_TRY(launch_router_select(w, x, T, logits, bias, r.at<float>(L.logits_sel), idx, wts, dbg_logits, s));
         r.mark(MOE_STAGE_TOPK, 1);
         r.launches += 2;
     } else if (!lsrc) {
@@ -464,9 +460,9 @@ moe_status route_stage(Run& r, const void* x, int T, const float* bias, const fl
     if (certified) {
         r.mark(MOE_STAGE_PERMUTE, 0);
         CUDA_TRY(launch_permute(idx, T, k, E, capacity_of(c, T), r.at<int32_t>(L.hist), offsets, row2ts, ts2row,
-                                meta, active, tiles, r.at<int32_t>(L.pairs), s, zero_words, n_zero, true));
+                                meta, active, tiles, r.at<int32_t>(L.pairs), s, zero_words, n_zero));
         r.mark(MOE_STAGE_PERMUTE, 1);
-        r.launches += 1;
+        r.launches += 2;
     } else if (route_small_ok(T, k)) {
         // top-k, histogram, scan and scatter in one block
         r.mark(MOE_STAGE_TOPK, 0);
