@@ -787,62 +787,6 @@ __global__ void __launch_bounds__(kRouteSmallThreads) route_small_kernel(
     scatter_entries(sm.idx, 0, n, E, cap, sm.pre, sm.off, sm.running, sm.u.wcnt, row2ts, ts2row);
 }
 
-// Decode-sized inputs (T <= 32 tokens, T*k <= kRouteTinyMax entries): the same
-// results as route_small_kernel with three block barriers instead of about ten.
-// Warp t does token t's top-k; thread i then finds entry i's rank among the
-// earlier entries of its expert by a plain count over the entries before it
-// (at most kRouteTinyMax - 1 shared-memory reads, broadcast across the warp),
-// warp 0 places the offsets and lists, and each entry is stored at its row.
-constexpr int kRouteTinyMax = 256;
-
-struct RouteTinySmem {
-    int32_t idx[kRouteTinyMax];
-    int kept[kMaxE], off[kMaxE + 1];
-    float lsh[32][kMaxE];
-};
-
-__global__ void __launch_bounds__(1024) route_tiny_kernel(
-    const float* __restrict__ logits, const float* __restrict__ bias, int T, int E, int k,
-    int renorm, int cap, int32_t* __restrict__ idx, float* __restrict__ wts,
-    float* __restrict__ logits_out, int32_t* __restrict__ offsets, int32_t* __restrict__ row2ts,
-    int32_t* __restrict__ ts2row, int32_t* __restrict__ meta, int32_t* __restrict__ active,
-    int32_t* __restrict__ tiles, int32_t* __restrict__ pairs, int32_t* __restrict__ zero_words, int n_zero) {
-    pdl_wait();
-    pdl_trigger();
-    for (int i = threadIdx.x; i < n_zero; i += blockDim.x) zero_words[i] = 0;
-
-    extern __shared__ __align__(16) uint8_t smem_raw[];
-    RouteTinySmem& sm = *reinterpret_cast<RouteTinySmem*>(smem_raw);
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int n = T * k;
-    for (int e = tid; e < E; e += blockDim.x) sm.kept[e] = 0;
-    if (warp < T) topk_token(logits, bias, warp, E, k, renorm, idx, wts, logits_out, sm.lsh[warp], sm.idx, lane);
-    __syncthreads();
-    int e = -1, rank = 0;
-    if (tid < n) {
-        e = sm.idx[tid];
-        for (int j = 0; j < tid; ++j) rank += sm.idx[j] == e;
-        atomicAdd(&sm.kept[e], 1);
-    }
-    __syncthreads();
-    if (warp == 0) {
-        if (cap >= 0)
-            for (int x = lane; x < E; x += 32) sm.kept[x] = min(sm.kept[x], cap);
-        __syncwarp();
-        write_offsets_and_lists(sm.kept, E, sm.off, offsets, meta, active, tiles, pairs, lane);
-    }
-    __syncthreads();
-    if (tid < n) {
-        if (cap < 0 || rank < cap) {
-            const int row = sm.off[e] + rank;
-            ts2row[tid] = row;
-            row2ts[row] = tid;
-        } else {
-            ts2row[tid] = -1;
-        }
-    }
-}
-
 // ---------------------------------------------------------------------------
 // Smoothed per-token quantisation: x' = fp32(x * inv_s); sx = amax/127;
 // q = rint(x'/sx) clamped to +-127.  One block per token; each thread owns
@@ -850,13 +794,12 @@ __global__ void __launch_bounds__(1024) route_tiny_kernel(
 // given, the copy of the token's codes into every kept (t, slot) row of the
 // expert-sorted matrix.
 // ---------------------------------------------------------------------------
-// One block of 128 threads per token: thread i owns channel groups i, i + 128,
-// ... (8 channels each); all of a thread's loads are issued before the block
+// One block of kSqThreads threads per token: thread i owns channel groups i,
+// i + kSqThreads, ... (8 channels each); all of a thread's loads are issued before the block
 // max (one shared-memory exchange), then the codes are written to xq[t] and,
 // for the tensor-core path, to every kept (t, slot) row of the sorted copy.
-constexpr int kSqThreads = 128;
 
-template <int kSqMaxGroups, int FMT>   // groups of 8 channels per thread: d <= 128 x 8 x kSqMaxGroups
+template <int kSqMaxGroups, int FMT, int kSqThreads>   // groups of 8 channels per thread: d <= kSqThreads x 8 x kSqMaxGroups
 __global__ void __launch_bounds__(kSqThreads) smooth_quant_kernel(
     const void* __restrict__ x, int in_dtype, const float* __restrict__ inv_s, float act_clip, int T, int d,
     int k, const int32_t* __restrict__ ts2row, int8_t* __restrict__ xq, float* __restrict__ sx,
@@ -1100,12 +1043,6 @@ cudaError_t launch_route_small(const float* logits, const float* bias, int T, in
                                int32_t* offsets, int32_t* row2ts, int32_t* ts2row, int32_t* meta,
                                int32_t* active, int32_t* tiles, int32_t* pairs, int32_t* zero_words, int n_zero,
                                cudaStream_t s) {
-    if (T <= 32 && T * k <= kRouteTinyMax) {
-        const int threads = std::max(T * 32, kRouteTinyMax);
-        return launch_pdl(route_tiny_kernel, dim3(1), dim3(threads), sizeof(RouteTinySmem), s, logits, bias, T, E, k,
-                          renorm, cap, idx, wts, logits_out, offsets, row2ts, ts2row, meta, active, tiles, pairs,
-                          zero_words, n_zero);
-    }
     static std::atomic<uint64_t> attr{0};
     cudaError_t e = smem_attr_once(route_small_kernel, sizeof(RouteSmallSmem), attr);
     if (e != cudaSuccess) return e;
@@ -1117,13 +1054,17 @@ cudaError_t launch_route_small(const float* logits, const float* bias, int T, in
 cudaError_t launch_smooth_quant(const void* x, int in_dtype, const float* inv_s, float act_clip, int T,
                                 int d, int k, const int32_t* ts2row, int8_t* xq, float* sx, int8_t* aq,
                                 int64_t aq_ld, const float* wts, const int32_t* idx, int fmt, cudaStream_t s) {
-    const int groups = (d / 8 + kSqThreads - 1) / kSqThreads;
+    // 256 threads per token with few channel groups each: few registers, so
+    // many warps per SM hide the load latency (the kernel is issue- and
+    // latency-bound, not bandwidth-bound)
+    constexpr int NT = 256;
+    const int groups = (d / 8 + NT - 1) / NT;
     auto kern = fmt == FMT_E4M3
-                    ? (groups <= 4 ? smooth_quant_kernel<4, FMT_E4M3>
-                                   : groups <= 8 ? smooth_quant_kernel<8, FMT_E4M3> : smooth_quant_kernel<16, FMT_E4M3>)
-                    : (groups <= 4 ? smooth_quant_kernel<4, FMT_INT8>
-                                   : groups <= 8 ? smooth_quant_kernel<8, FMT_INT8> : smooth_quant_kernel<16, FMT_INT8>);
-    return launch_pdl(kern, dim3(T), dim3(kSqThreads), 0, s, x, in_dtype, inv_s, act_clip, T, d, k, ts2row, xq,
+                    ? (groups <= 2 ? smooth_quant_kernel<2, FMT_E4M3, NT>
+                                   : groups <= 4 ? smooth_quant_kernel<4, FMT_E4M3, NT> : smooth_quant_kernel<8, FMT_E4M3, NT>)
+                    : (groups <= 2 ? smooth_quant_kernel<2, FMT_INT8, NT>
+                                   : groups <= 4 ? smooth_quant_kernel<4, FMT_INT8, NT> : smooth_quant_kernel<8, FMT_INT8, NT>);
+    return launch_pdl(kern, dim3(T), dim3(NT), 0, s, x, in_dtype, inv_s, act_clip, T, d, k, ts2row, xq,
                       sx, aq, aq_ld, wts, idx);
 }
 

@@ -250,7 +250,9 @@ __device__ __forceinline__ int block_row(const BlockMap& bm, int r) {
     return g * bm.block_rows + 1 + r - bm.offsets[bm.ranks.first[g]];
 }
 
-template <bool O16, bool BLOCKED>
+// KM: the largest k the instance serves (4 or kMaxK): the slot arrays live in
+// registers, so a smaller bound leaves room for more warps per SM.
+template <bool O16, bool BLOCKED, int KM>
 __global__ void combine_kernel(const void* __restrict__ o, const int32_t* __restrict__ ts2row,
                                int k, int d, int out_dtype, void* __restrict__ y, const BlockMap bm) {
     pdl_wait();
@@ -259,19 +261,19 @@ __global__ void combine_kernel(const void* __restrict__ o, const int32_t* __rest
     const int t = blockIdx.x;
     const int n8 = blockIdx.y * blockDim.x + threadIdx.x;
     if (n8 * 8 >= d) return;
-    int rows[kMaxK];
+    int rows[KM];
 #pragma unroll
-    for (int s = 0; s < kMaxK; ++s) rows[s] = s < k ? ts2row[(int64_t)t * k + s] : -1;
+    for (int s = 0; s < KM; ++s) rows[s] = s < k ? ts2row[(int64_t)t * k + s] : -1;
     if (BLOCKED) {
 #pragma unroll
-        for (int s = 0; s < kMaxK; ++s)
+        for (int s = 0; s < KM; ++s)
             if (rows[s] >= 0) rows[s] = block_row(bm, rows[s]);
     }
     // loads of every kept slot first (raw 16-byte words: few registers, so many
     // warps per SM), then the sum in slot order
-    uint4 raw[kMaxK][O16 ? 1 : 2];
+    uint4 raw[KM][O16 ? 1 : 2];
 #pragma unroll
-    for (int s = 0; s < kMaxK; ++s) {
+    for (int s = 0; s < KM; ++s) {
         if (rows[s] < 0) continue;
         if (O16) {
             raw[s][0] = reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(o) + (int64_t)rows[s] * d)[n8];
@@ -283,7 +285,7 @@ __global__ void combine_kernel(const void* __restrict__ o, const int32_t* __rest
     }
     float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-    for (int s = 0; s < kMaxK; ++s) {
+    for (int s = 0; s < KM; ++s) {
         if (rows[s] < 0) continue;
         float v[8];
         if (O16) {
@@ -369,9 +371,9 @@ cudaError_t launch_combine(const void* o, int o_bf16, const int32_t* ts2row, int
                            int out_dtype, void* y, cudaStream_t s) {
     dim3 grid(T, (d / 8 + 255) / 256);
     const BlockMap none{};
-    if (o_bf16)
-        return launch_pdl(combine_kernel<true, false>, grid, dim3(256), 0, s, o, ts2row, k, d, out_dtype, y, none);
-    return launch_pdl(combine_kernel<false, false>, grid, dim3(256), 0, s, o, ts2row, k, d, out_dtype, y, none);
+    auto kern = o_bf16 ? (k <= 4 ? combine_kernel<true, false, 4> : combine_kernel<true, false, kMaxK>)
+                       : (k <= 4 ? combine_kernel<false, false, 4> : combine_kernel<false, false, kMaxK>);
+    return launch_pdl(kern, grid, dim3(256), 0, s, o, ts2row, k, d, out_dtype, y, none);
 }
 
 cudaError_t launch_combine_blocked(const float* o_blocks, const int32_t* ts2row, const int32_t* offsets,
@@ -379,8 +381,8 @@ cudaError_t launch_combine_blocked(const float* o_blocks, const int32_t* ts2row,
                                    int out_dtype, void* y, cudaStream_t s) {
     dim3 grid(T, (d / 8 + 255) / 256);
     const BlockMap bm{offsets, ranks, world, block_rows};
-    return launch_pdl(combine_kernel<false, true>, grid, dim3(256), 0, s, (const void*)o_blocks, ts2row, k, d,
-                      out_dtype, y, bm);
+    auto kern = k <= 4 ? combine_kernel<false, true, 4> : combine_kernel<false, true, kMaxK>;
+    return launch_pdl(kern, grid, dim3(256), 0, s, (const void*)o_blocks, ts2row, k, d, out_dtype, y, bm);
 }
 
 }  // namespace moe

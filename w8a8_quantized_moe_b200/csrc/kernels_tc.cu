@@ -1289,7 +1289,9 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
                 epilogue_swiglu<FMT>(p1, taddr, half, e, nt, wrow0, nvalid, stage, sc, r0, &ctl->acc_empty[buf], nullptr,
                                      lane);
                 // this warp's share of the tile is stored: count it; the last arrival requantises
-                __threadfence();
+                // (a warp without valid rows stored nothing, so it has nothing to fence: at decode
+                // sizes most warps of a tile, and the fence was measurable)
+                if (nvalid > 0) __threadfence();
                 __syncwarp();
                 int old = 0;
                 if (lane == 0) old = atom_add_acq_rel(fx.count + mt, 1);
@@ -1380,14 +1382,17 @@ __global__ void __launch_bounds__(kRqThreads) requant_kernel(const float* __rest
 // l~[t][e] = sum_j x[t][j] (hi[e][j] + lo[e][j]) with W_g split into two bf16
 // parts (hi = bf16(w), lo = bf16(w - hi), so |w - hi - lo| <= 2^-16 |w|),
 // tcgen05.mma kind::f16 (bf16 x bf16, fp32 accumulators in TMEM).  One CTA per
-// 128 tokens: warp 0 loads X (128 x 64 bf16) and both W parts (EPAD x 64 bf16)
-// per k-block by TMA into a ring, warp 1 issues two MMAs per 16 channels into
-// one accumulator, warps 2-5 write the EPAD columns of their 32 rows.  These
+// 128 tokens and 64 experts (a 256-expert router is four CTAs per token block,
+// so wide routers still fill the GPU): warp 0 loads X (128 x 64 bf16) and both
+// W parts (EPAD x 64 bf16) per k-block by TMA into a ring, warp 1 issues two
+// MMAs per 16 channels into one accumulator, warps 2-5 write the EPAD columns
+// of their 32 rows.  These
 // values only choose candidates; the logits that decide top-k and the gate
 // weights are recomputed in the stated fp32 order (router_select_kernel).
 constexpr int kRcBK = 64;                     // bf16 channels per k-block (128 bytes)
 constexpr int kRcThreads = 192;
 constexpr int kRcABytes = BM * kRcBK * 2;     // 16 KB
+constexpr int kRcSlice = 64;                  // experts per CTA (the padded router is a multiple)
 
 template <int EPAD>
 struct RcCfg {
@@ -1419,7 +1424,11 @@ __global__ void __launch_bounds__(kRcThreads, 1)
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
     Ctl* ctl = reinterpret_cast<Ctl*>(smem + C::kStages * C::kStage);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int t0 = blockIdx.x * BM;
+    // blockIdx.x: which EPAD experts (a slice of the padded router), blockIdx.y:
+    // which 128 tokens; the slices of one token block are neighbours in launch
+    // order, so they read the block's X from L2
+    const int e0 = blockIdx.x * EPAD;
+    const int t0 = blockIdx.y * BM;
     const int nkb = d / kRcBK;
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::kStages; ++s) {
@@ -1456,8 +1465,8 @@ __global__ void __launch_bounds__(kRcThreads, 1)
                 mbar_arrive_expect_tx(&ctl->full[s], C::kStage);
                 uint8_t* sa = smem + s * C::kStage;
                 tma_load_2d(sa, &tm_x, &ctl->full[s], kb * kRcBK, t0);
-                tma_load_2d(sa + kRcABytes, &tm_hi, &ctl->full[s], kb * kRcBK, 0);
-                tma_load_2d(sa + kRcABytes + C::kBBytes, &tm_lo, &ctl->full[s], kb * kRcBK, 0);
+                tma_load_2d(sa + kRcABytes, &tm_hi, &ctl->full[s], kb * kRcBK, e0);
+                tma_load_2d(sa + kRcABytes + C::kBBytes, &tm_lo, &ctl->full[s], kb * kRcBK, e0);
                 issued[s] = true;
                 issued_par[s] = ph;
                 if (++s == C::kStages) { s = 0; ph ^= 1; }
@@ -1505,7 +1514,7 @@ __global__ void __launch_bounds__(kRcThreads, 1)
                 tmem_ld_wait();
                 if (t < T)
                     for (int j = 0; j < 32; ++j)
-                        if (c0 + j < E) approx[(int64_t)t * E + c0 + j] = __uint_as_float(v[j]);
+                        if (e0 + c0 + j < E) approx[(int64_t)t * E + e0 + c0 + j] = __uint_as_float(v[j]);
             }
         }
     }
@@ -1650,7 +1659,8 @@ cudaError_t launch_router_tc_pad(const CUtensorMap& mx, const moe_w8a8_weights* 
     static std::atomic<uint64_t> attr{0};
     cudaError_t e = smem_attr_once(router_tc_kernel<EPAD>, C::kSmem, attr);
     if (e != cudaSuccess) return e;
-    return launch_pdl(router_tc_kernel<EPAD>, dim3((T + BM - 1) / BM), dim3(kRcThreads), C::kSmem, s, mx,
+    return launch_pdl(router_tc_kernel<EPAD>, dim3(w->rt_epad / EPAD, (T + BM - 1) / BM), dim3(kRcThreads), C::kSmem,
+                      s, mx,
                       w->tm_rt_hi, w->tm_rt_lo, T, w->cfg.d, w->cfg.n_experts, approx, w->status);
 }
 
@@ -1812,19 +1822,16 @@ cudaError_t launch_tc_ffn_fused(const moe_w8a8_weights* w, int T, const int8_t* 
 }
 
 bool router_tc_make_maps(moe_w8a8_weights* w) {
-    return make_map_bf16(&w->tm_rt_hi, w->rt_hi, w->cfg.d, w->rt_epad, w->rt_epad) &&
-           make_map_bf16(&w->tm_rt_lo, w->rt_lo, w->cfg.d, w->rt_epad, w->rt_epad);
+    return make_map_bf16(&w->tm_rt_hi, w->rt_hi, w->cfg.d, w->rt_epad, kRcSlice) &&
+           make_map_bf16(&w->tm_rt_lo, w->rt_lo, w->cfg.d, w->rt_epad, kRcSlice);
 }
 
 cudaError_t launch_router_tc(const moe_w8a8_weights* w, const void* x, int T, float* approx, cudaStream_t s) {
     CUtensorMap mx;
     if (!make_map_bf16(&mx, x, w->cfg.d, T, BM)) return cudaErrorInvalidValue;
-    switch (w->rt_epad) {
-        case 64: return launch_router_tc_pad<64>(mx, w, T, approx, s);
-        case 128: return launch_router_tc_pad<128>(mx, w, T, approx, s);
-        case 256: return launch_router_tc_pad<256>(mx, w, T, approx, s);
-    }
-    return cudaErrorInvalidValue;
+    // 64 experts per CTA whatever the padded count: more CTAs for wide routers
+    if (w->rt_epad % kRcSlice) return cudaErrorInvalidValue;
+    return launch_router_tc_pad<kRcSlice>(mx, w, T, approx, s);
 }
 
 cudaError_t launch_tc_peak(int fmt, int64_t n_mma, int grid, cudaStream_t s) {
