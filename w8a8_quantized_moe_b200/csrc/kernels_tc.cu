@@ -967,9 +967,7 @@ __device__ void requant_rows_warp(const float* h32, const float* pamax, int f, i
             if (j < total) {
                 const float s = scales[j / n4];
                 const float rs = s > 0.0f ? __frcp_rn(s) : 0.0f;
-                q4[j] = s > 0.0f ? pack4((int)fmt_code<FMT>(h[i].x, s, rs), (int)fmt_code<FMT>(h[i].y, s, rs),
-                                         (int)fmt_code<FMT>(h[i].z, s, rs), (int)fmt_code<FMT>(h[i].w, s, rs))
-                                 : 0u;
+                q4[j] = s > 0.0f ? fmt_codes4<FMT>(h[i].x, h[i].y, h[i].z, h[i].w, s, rs) : 0u;
             }
         }
     }
@@ -1324,11 +1322,12 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
 // codes rint(h / sh), ties to even, clamped to +-127 (sh = 0 gives 0).  The
 // scale comes from the partial maxima, not from h, so a row's h loads (up to
 // kRqBatch x 16 bytes per lane) and its partial-maximum loads are issued
-// together; further batches follow (f = 1536: 12 x 16 bytes per lane in two
-// batches).  A small batch keeps the registers, and so the warps per SM that
+// together; further batches follow (f = 1536: 12 x 16 bytes per lane in three
+// batches; 4 per batch measured faster than 6, 8 or 12: 39 registers, so 6
+// blocks of 8 warps per SM).  A small batch keeps the registers, and so the warps per SM that
 // hide the per-element arithmetic, in balance with the bytes in flight.
 constexpr int kRqThreads = 256;
-constexpr int kRqBatch = 8;
+constexpr int kRqBatch = 4;
 
 template <int FMT>
 __global__ void __launch_bounds__(kRqThreads) requant_kernel(const float* __restrict__ h32,
@@ -1369,9 +1368,7 @@ __global__ void __launch_bounds__(kRqThreads) requant_kernel(const float* __rest
         for (int i = 0; i < kRqBatch; ++i) {
             const int c4 = b + lane + 32 * i;
             if (c4 < n4)
-                qrow[c4] = s > 0.0f ? pack4((int)fmt_code<FMT>(h[i].x, s, rs), (int)fmt_code<FMT>(h[i].y, s, rs),
-                                            (int)fmt_code<FMT>(h[i].z, s, rs), (int)fmt_code<FMT>(h[i].w, s, rs))
-                                    : 0u;
+                qrow[c4] = s > 0.0f ? fmt_codes4<FMT>(h[i].x, h[i].y, h[i].z, h[i].w, s, rs) : 0u;
         }
     }
 }
