@@ -112,6 +112,38 @@ __device__ __forceinline__ uint32_t pack4(int a, int b, int c, int d) {
            ((uint32_t)(d & 0xff) << 24);
 }
 
+// The four code bytes of v0..v3 for scale s > 0 (r = fp32(1 / s)), packed low
+// byte first: identical to fmt_code element by element.  For INT8 the four
+// products t = v r are rounded together and the near-half-integer test of
+// quant_code_fast is combined into one branch: if any element needs the IEEE
+// quotient (or 1/s overflowed), all four are formed by quant_code, which gives
+// the same codes for the others (the test's premise).
+template <int FMT>
+__device__ __forceinline__ uint32_t fmt_codes4(float v0, float v1, float v2, float v3, float s, float r) {
+    if (FMT == FMT_E4M3)
+        return pack4((int)fmt_code<FMT>(v0, s, r), (int)fmt_code<FMT>(v1, s, r), (int)fmt_code<FMT>(v2, s, r),
+                     (int)fmt_code<FMT>(v3, s, r));
+    const float v[4] = {v0, v1, v2, v3};
+    float n[4];
+    bool slow = isinf(r);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float t = __fmul_rn(v[i], r);
+        n[i] = rintf(t);
+        const float dist = fabsf(fabsf(__fsub_rn(t, n[i])) - 0.5f);
+        slow |= dist <= 3.0e-5f && fabsf(t) <= 130.0f;
+    }
+    int q[4];
+    if (!slow) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) q[i] = max(-127, min(127, __float2int_rn(n[i])));
+    } else {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) q[i] = quant_code(v[i], s);
+    }
+    return pack4(q[0], q[1], q[2], q[3]);
+}
+
 __device__ __forceinline__ float bf16_bits_to_f32(uint16_t h) {
     return __uint_as_float((uint32_t)h << 16);
 }

@@ -849,10 +849,9 @@ __global__ void __launch_bounds__(kSqThreads) smooth_quant_kernel(
     for (int gi = 0; gi < kSqMaxGroups; ++gi) {
         const int g = tid + kSqThreads * gi;
         if (g >= ng) continue;
-        int q[8];
-#pragma unroll
-        for (int c = 0; c < 8; ++c) q[c] = s > 0.0f ? (int)fmt_code<FMT>(v[gi][c], s, rs) : 0;
-        packed[gi] = make_uint2(pack4(q[0], q[1], q[2], q[3]), pack4(q[4], q[5], q[6], q[7]));
+        packed[gi] = s > 0.0f ? make_uint2(fmt_codes4<FMT>(v[gi][0], v[gi][1], v[gi][2], v[gi][3], s, rs),
+                                           fmt_codes4<FMT>(v[gi][4], v[gi][5], v[gi][6], v[gi][7], s, rs))
+                              : make_uint2(0u, 0u);
         if (xq) *reinterpret_cast<uint2*>(xq + (int64_t)t * d + g * 8) = packed[gi];
     }
     pdl_wait();   // the routing of this forward is complete from here on
