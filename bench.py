@@ -57,6 +57,16 @@ def sources_hash() -> str:
     return h.hexdigest()[:16]
 
 
+def norm_kernel(name: str) -> str:
+    """A kernel's name as the traffic table keys it: no namespaces or parameters, and of
+    its template arguments only the first ("tc_pair_gemm_kernel<0, 0>" -> "tc_pair_gemm_kernel<0>")."""
+    import re
+    name = re.sub(r"\(anonymous namespace\)::|<unnamed>::|unnamed>::", "", name).split("(")[0].strip()
+    name = name.split()[-1].split("::")[-1] if "<" not in name else name.split("<")[0].split()[-1].split("::")[-1] + \
+        "<" + name.split("<", 1)[1].split(",")[0].rstrip(">").strip() + ">"
+    return name
+
+
 def load_traffic() -> dict:
     """{(workload, T, kernel): bytes per launch} for the current sources."""
     out = {}
@@ -87,8 +97,7 @@ def record_traffic(csv_path: str, workload: str, T: int, scale: float = 1.0):
     hdr = rows[0]
     col = {n: hdr.index(n) for n in ("ID", "Kernel Name", "Metric Name", "Metric Unit", "Metric Value")}
     for r in rows[1:]:
-        raw = re.sub(r"\(anonymous namespace\)::", "", r[col["Kernel Name"]]).split("(")[0].split("<")[0]
-        name = raw.split("::")[-1].split()[-1]
+        name = norm_kernel(r[col["Kernel Name"]])
         m = r[col["Metric Name"]]
         if m not in ("dram__bytes_read.sum", "dram__bytes_write.sum"):
             continue
@@ -587,18 +596,21 @@ def measure(args, wl, world, rank, local, e2e_on=True, wts=None):
     if stages:
         dom = max(("gemm1", "gemm2"), key=lambda k: stages[k])
         dom_ms = stages[dom]
-        kernel = (f"tc_gemm_kernel<{0 if dom == 'gemm1' else 1}>" if tensor else
+        # the library's rule for SM pairs (a cta_pairs setting of 2 or the default)
+        cp = getattr(args, "cta_pairs", -1)
+        pairs = cp == 1 or (cp in (-1, 2) and wl.T * wl.k >= 256 * wl.E)
+        kernel = (f"tc_{'pair_' if pairs else ''}gemm_kernel<{0 if dom == 'gemm1' else 1}>" if tensor else
                   ("stream_gateup_kernel" if dom == "gemm1" else "stream_down_kernel"))
         ops = 2 * R * (2 * wl.f if dom == "gemm1" else wl.f) * wl.d
         nbytes = alg[f"{dom}_bytes"]
         if fused:
-            kernel, ops, nbytes = "tc_ffn_fused_kernel", alg["int8_ops"], alg["fused_bytes"]
+            kernel, ops, nbytes = f"tc_ffn_fused_kernel<{1 if fp8 else 0}>", alg["int8_ops"], alg["fused_bytes"]
         # the bound is whichever of the byte time and the INT8 op time is larger
         if ops / (int8_peak * 1e12) > nbytes / (peaks["hbm_gbs"] * 1e9):
             achieved = ops / (dom_ms / 1e3) / 1e12
             roof = {"bound": "tensor", "kernel": f"{dom} ({kernel})", "achieved": achieved,
                     "peak": int8_peak, "unit": "TFLOP/s", "frac": achieved / int8_peak,
-                    "traffic": load_traffic().get((wl.name, wl.T, kernel)),
+                    "traffic": load_traffic().get((wl.name, wl.T, norm_kernel(kernel))),
                     "peak_source": int8_src,
                     "int8_ops_per_launch": ops, "launch_ms": dom_ms,
                     "frac_of_nominal_4500": achieved / NOMINAL_INT8_TOPS}
@@ -608,7 +620,7 @@ def measure(args, wl, world, rank, local, e2e_on=True, wts=None):
             achieved = nbytes / (dom_ms / 1e3) / 1e9
             roof = {"bound": "hbm", "kernel": f"{dom} ({kernel})", "achieved": achieved,
                     "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
-                    "traffic": load_traffic().get((wl.name, wl.T, kernel)),
+                    "traffic": load_traffic().get((wl.name, wl.T, norm_kernel(kernel))),
                     "peak_source": f"hbm_gbs of {peak_src}",
                     "algorithmic_bytes_per_launch": nbytes, "launch_ms": dom_ms}
     step_s = ms_total / K / 1e3

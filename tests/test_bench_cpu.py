@@ -71,7 +71,12 @@ def test_traffic_record_and_lookup(tmp_path, monkeypatch):
     csv_path.write_text("==PROF== noise\n" + hdr + "".join(rows))
     bench.record_traffic(str(csv_path), "decode", 32)
     t = bench.load_traffic()
-    assert abs(t[("decode", 32, "tc_ffn_fused_kernel")] - 1012e6) < 1.0
+    # keyed by the name without namespaces or parameters and its first template argument
+    assert abs(t[("decode", 32, "tc_ffn_fused_kernel<0>")] - 1012e6) < 1.0
+    assert bench.norm_kernel("void moe::<unnamed>::tc_pair_gemm_kernel<1, 0>(CUtensorMap_st)") == \
+        "tc_pair_gemm_kernel<1>"
+    assert bench.norm_kernel("moe::<unnamed>::router_select_kernel(const unsigned short *)") == \
+        "router_select_kernel"
     # a different sources hash: the row is ignored
     monkeypatch.setattr(bench, "sources_hash", lambda: "0" * 16)
     assert bench.load_traffic() == {}

@@ -1226,8 +1226,9 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
             const int e = p1.tiles[2 * mt], row0 = p1.tiles[2 * mt + 1];
             const int nrows = min(BM, p1.offsets[e + 1] - row0);
             requant_rows_warp<FMT>(p1.h32, p1.pamax, p1.f, row0, nrows, fx.hq, fx.sh, scales, lane);
+            // the codes reach the GEMM2 producers' TMA loads (async proxy) and the
+            // epilogues' loads through lane 0's release after the warp barrier
             fence_proxy_async_global();
-            __threadfence();
             __syncwarp();
             if (lane == 0 && mt != fx.skip_ready) st_release(fx.ready + mt, 1);
         }
@@ -1286,10 +1287,11 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
             if (g1) {
                 epilogue_swiglu<FMT>(p1, taddr, half, e, nt, wrow0, nvalid, stage, sc, r0, &ctl->acc_empty[buf], nullptr,
                                      lane);
-                // this warp's share of the tile is stored: count it; the last arrival requantises
-                // (a warp without valid rows stored nothing, so it has nothing to fence: at decode
-                // sizes most warps of a tile, and the fence was measurable)
-                if (nvalid > 0) __threadfence();
+                // this warp's share of the tile is stored: count it; the last arrival requantises.
+                // The lanes' stores are ordered before lane 0's release by the warp barrier (it
+                // orders the participating lanes' memory accesses), and a release publishes
+                // everything ordered before it, so no separate fence is needed (membar.gl here
+                // cost the decode step about 5 us with the requantisation warp's below)
                 __syncwarp();
                 int old = 0;
                 if (lane == 0) old = atom_add_acq_rel(fx.count + mt, 1);
