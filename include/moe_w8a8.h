@@ -335,7 +335,7 @@ moe_status moe_w8a8_check_status(const moe_w8a8_weights* w, moe_stream_t stream)
  * waiting for a full accumulator (words 3-4: tile, awaited phase parity);
  * of the fused expert launch also 6 a down-projection producer waiting for
  * an m-tile's h codes (words 3-4: tile, m-tile), 7 a requantisation warp
- * waiting for a queue slot (word 3: slot), 8-10 the producer, MMA issuer and
+ * waiting for an m-tile's h to be complete (word 3: m-tile), 8-10 the producer, MMA issuer and
  * epilogue waiting on the block's tile ring, 16 a down-projection epilogue
  * waiting for an m-tile's h scales (words 3-4: tile, m-tile); 11-13 the certified router's
  * producer, MMA issuer and epilogue.  Site 14 (with MOE_ERR_INVALID_ARG): a

@@ -228,7 +228,7 @@ cudaError_t launch_tc_ffn_fused(const moe_w8a8_weights* w, int T, const int8_t* 
                                 const float* sx, const float* topk_w, float* h32, float* pamax, int8_t* hq,
                                 float* sh, void* o, int32_t* acc1_dbg, int32_t* acc2_dbg, int32_t* sync_words,
                                 cudaStream_t s);
-inline size_t fused_sync_words(size_t max_mtiles) { return 3 * max_mtiles + 3; }
+inline size_t fused_sync_words(size_t max_mtiles) { return 2 * max_mtiles + 2; }
 constexpr int kFusedMaxRows = 512;   // default: T*k at or below which the tensor path runs the fused launch
 
 // The per-slot rows o (sorted, [rows][d]) are fp32, or bf16 when o_bf16; the

@@ -973,10 +973,9 @@ __device__ void requant_rows_warp(const float* h32, const float* pamax, int f, i
     }
 }
 
-__device__ __forceinline__ int atom_add_acq_rel(int32_t* p, int v) {
-    int old;
-    asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
-    return old;
+// A release add whose old value nobody waits for.
+__device__ __forceinline__ void red_release_add(int32_t* p, int v) {
+    asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 __device__ __forceinline__ int ld_acquire(const int32_t* p) {
     int v;
@@ -996,15 +995,13 @@ __device__ __forceinline__ void fence_proxy_async_global() {
 struct FusedExtra {
     int32_t* count;   // [m-tiles] GEMM1 epilogue-warp arrivals
     int32_t* ready;   // [m-tiles] 1 once the m-tile's h codes are written
-    int32_t* queue;   // [m-tiles] m-tiles whose h is complete, + 1, in completion order
-    int32_t* qtail;   // next free queue slot
-    int32_t* qhead;   // next queue slot a requantisation warp takes
+    int32_t* qhead;   // next m-tile a requantisation warp takes
     int32_t* next;    // next tile to take (dynamic schedule)
     int8_t* hq;       // [rows][f] h codes
     float* sh;        // [rows] h scales
-    uint64_t budget_ns;   // bound on each wait for another block's results (ready flags, queue)
+    uint64_t budget_ns;   // bound on each wait for another block's results (counts, ready flags)
     int skip_ready;       // testing aid: the m-tile whose ready flag is never released (-1: none)
-};                    // (count, ready, queue, qtail, qhead, next zeroed before the launch)
+};                    // (count, ready, qhead, next zeroed before the launch)
 
 constexpr int kFusedThreads = kThreads + 32;   // + one requantisation warp (warp 10)
 constexpr int kTileRing = 8;                   // tiles taken but not yet finished, per CTA
@@ -1029,13 +1026,15 @@ constexpr size_t kFusedSmemBytes = kSmemBytes + kEpiStageBytes + 256;
 // wait depends on has already been taken by a running CTA: the launch makes
 // progress even when not all its CTAs are resident.  Dependencies are per
 // m-tile (one expert's rows): every
-// epilogue warp that finishes a GEMM1 tile adds one to count[m]; the warp that
-// brings it to (GEMM1 column tiles x epilogue warps) appends m to a device-wide
-// queue.  Warp 10 of every CTA takes queue slots in turn, requantises that
-// m-tile's rows and releases ready[m], so requantisation runs on otherwise idle
-// warps of many CTAs and never delays an epilogue (when the epilogue warp that
-// completed an m-tile requantised it itself, it fell behind, became the last
-// arrival again, and the delays piled up).  The producer of a GEMM2 tile waits
+// epilogue warp that finishes a GEMM1 tile adds one to count[m] (a release add
+// whose result it does not wait for).  Warp 10 of every CTA takes m-tiles in
+// index order from a counter, waits until the m-tile's count is complete
+// (GEMM1 column tiles x epilogue warps), requantises its rows and releases
+// ready[m], so requantisation runs on otherwise idle warps of many CTAs and
+// never delays an epilogue (when the epilogue warp that completed an m-tile
+// requantised it itself, it fell behind, became the last arrival again, and
+// the delays piled up; when the last arrival found out by an atomic's result
+// and queued the m-tile, every epilogue warp waited for that result).  The producer of a GEMM2 tile waits
 // for ready[m] (bounded by the handle's wait budget) before loading its h codes.  GEMM1 tiles are all taken
 // before any GEMM2 tile, GEMM1 tiles wait on nothing, and the requant warps
 // wait only on GEMM1 tiles, so the waits always end.  Arithmetic per element
@@ -1199,30 +1198,31 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
             while (!mbar_try_wait(&ctl->drain, 0) && global_timer() - t0 < kWaitBudgetNs) {}
         }
     } else if (warp == kFusedThreads / 32 - 1) {
-        // ---------------- requantisation warp: queue slots in turn
+        // ---------------- requantisation warp: m-tiles in index order
         float* scales = epi_stage + kEpiWarps * (kEpiStageBytes / 4);
         while (true) {
             int i = 0;
             if (lane == 0) i = atomicAdd(fx.qhead, 1);
             i = __shfl_sync(0xffffffffu, i, 0);
             if (i >= n_mt) break;
-            int v = 0;
+            int ok = 1;
             if (lane == 0) {
                 const uint64_t t0 = global_timer();
-                while ((v = ld_acquire(fx.queue + i)) == 0) {
-                    if (*abort) break;
+                while (ld_acquire(fx.count + i) < arrivals) {
+                    if (*abort) { ok = 0; break; }
                     if (global_timer() - t0 > fx.budget_ns) {
                         *abort = 1;
                         report_timeout(p1.status, 7, i, 0);
+                        ok = 0;
                         break;
                     }
                     __nanosleep(64);
                 }
             }
-            v = __shfl_sync(0xffffffffu, v, 0);
-            if (v == 0) break;
-            (void)ld_acquire(fx.queue + i);   // each lane's own acquire of the m-tile's h
-            const int mt = v - 1;
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (!ok) break;
+            (void)ld_acquire(fx.count + i);   // each lane's own acquire of the m-tile's h
+            const int mt = i;
             const int e = p1.tiles[2 * mt], row0 = p1.tiles[2 * mt + 1];
             const int nrows = min(BM, p1.offsets[e + 1] - row0);
             requant_rows_warp<FMT>(p1.h32, p1.pamax, p1.f, row0, nrows, fx.hq, fx.sh, scales, lane);
@@ -1287,20 +1287,13 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
             if (g1) {
                 epilogue_swiglu<FMT>(p1, taddr, half, e, nt, wrow0, nvalid, stage, sc, r0, &ctl->acc_empty[buf], nullptr,
                                      lane);
-                // this warp's share of the tile is stored: count it; the last arrival requantises.
-                // The lanes' stores are ordered before lane 0's release by the warp barrier (it
-                // orders the participating lanes' memory accesses), and a release publishes
-                // everything ordered before it, so no separate fence is needed (membar.gl here
-                // cost the decode step about 5 us with the requantisation warp's below)
+                // this warp's share of the tile is stored: count it.  The lanes' stores are
+                // ordered before lane 0's release by the warp barrier (it orders the
+                // participating lanes' memory accesses), and a release publishes everything
+                // ordered before it, so no separate fence is needed (membar.gl here cost the
+                // decode step about 5 us with the requantisation warp's below)
                 __syncwarp();
-                int old = 0;
-                if (lane == 0) old = atom_add_acq_rel(fx.count + mt, 1);
-                old = __shfl_sync(0xffffffffu, old, 0);
-                if (old == arrivals - 1 && lane == 0) {
-                    // the m-tile's h is complete: hand it to the requantisation warps
-                    const int slot = atomicAdd(fx.qtail, 1);
-                    st_release(fx.queue + slot, mt + 1);
-                }
+                if (lane == 0) red_release_add(fx.count + mt, 1);
             } else {
                 epilogue_down<FMT>(p2, taddr, half, e, nt, wrow0, nvalid, stage, sc, r0, r1, &ctl->acc_empty[buf],
                                    nullptr, lane);
@@ -1811,9 +1804,8 @@ cudaError_t launch_tc_ffn_fused(const moe_w8a8_weights* w, int T, const int8_t* 
     p2.o_bf16 = c.out_dtype == MOE_BF16;
     p2.acc_dbg = acc2_dbg;
     const int max_mt = (rows + BM - 1) / BM + c.n_experts;
-    const FusedExtra fx{sync_words, sync_words + max_mt, sync_words + 2 * max_mt, sync_words + 3 * max_mt,
-                        sync_words + 3 * max_mt + 1, sync_words + 3 * max_mt + 2, hq, sh,
-                        w->wait_budget_ns, w->test_skip_ready};
+    const FusedExtra fx{sync_words, sync_words + max_mt, sync_words + 2 * max_mt, sync_words + 2 * max_mt + 1, hq,
+                        sh, w->wait_budget_ns, w->test_skip_ready};
     const int grid = max(1, min(w->num_sms, max_mt * (p1.n_tiles_n + p2.n_tiles_n)));
     if (c.expert_format == FMT_E4M3)
         return launch_fused_fmt<FMT_E4M3>(a1, w->tm_w_gu, a2, w->tm_w_dn, p1, p2, fx, grid, s);
