@@ -403,9 +403,20 @@ enum {
  */
 moe_status moe_w8a8_profile_start(moe_w8a8_weights* w, int32_t max_forwards);
 
+/*
+ * As moe_w8a8_profile_start, but only the stages whose bit (1 << stage) is set
+ * in stage_mask record their event pair; the others record nothing and read
+ * back as 0 ms.  Bracketing one stage alone leaves every other boundary of the
+ * forward free of events, so the launches run as in a plain forward except at
+ * that stage's own two boundaries.
+ * stage_mask == 0 or with bits at or above MOE_N_STAGES: MOE_ERR_INVALID_ARG.
+ */
+moe_status moe_w8a8_profile_start_stages(moe_w8a8_weights* w, int32_t max_forwards, uint32_t stage_mask);
+
 /* Synchronise the recorded events and write ms_host[i * MOE_N_STAGES + s],
  * the time of stage s in recorded forward i, for up to `capacity` forwards.
- * Returns the number of forwards written (negative on a CUDA error). */
+ * Returns the number of forwards written (negative on a CUDA error).
+ * Stages left out by the mask read 0. */
 int32_t moe_w8a8_profile_read(moe_w8a8_weights* w, float* ms_host, int32_t capacity);
 
 /* Stop recording and free the events. */

@@ -107,6 +107,7 @@ def test_host_side_argument_checks(M):
     assert L.moe_w8a8_calibrate_absmax(z, 4, 16, 5, z, None) == M.MOE_ERR_INVALID_ARG
     assert L.moe_w8a8_calibrate_absmax(z, -1, 16, 0, z, None) == M.MOE_ERR_INVALID_ARG
     assert L.moe_w8a8_last_launch_count(None) == 0
+    assert L.moe_w8a8_profile_start_stages(None, 4, 1 << M.STAGE_NAMES.index("gemm1")) == M.MOE_ERR_INVALID_ARG
     assert L.moe_w8a8_set_act_clip(None, 1.0) == M.MOE_ERR_INVALID_ARG
     clip = ctypes.c_float(0.0)
     assert L.moe_w8a8_calibrate_act_clip(None, z, 4, 1, 99.9, ctypes.byref(clip), None) == M.MOE_ERR_INVALID_ARG

@@ -38,7 +38,7 @@ EXPORTS = (
     "moe_w8a8_forward", "moe_w8a8_forward_host", "moe_w8a8_set_path",
     "moe_w8a8_set_stream_threshold", "moe_w8a8_get_smooth_scales", "moe_w8a8_export_weights",
     "moe_w8a8_check_status", "moe_w8a8_destroy", "moe_status_string",
-    "moe_w8a8_last_launch_count", "moe_w8a8_profile_start", "moe_w8a8_profile_read",
+    "moe_w8a8_last_launch_count", "moe_w8a8_profile_start", "moe_w8a8_profile_start_stages", "moe_w8a8_profile_read",
     "moe_w8a8_profile_stop", "moe_w8a8_stage_name", "moe_w8a8_forward_noalloc",
     "moe_w8a8_status_words", "moe_w8a8_set_act_clip", "moe_w8a8_calibrate_act_clip",
     "moe_w8a8_ep_row_bytes", "moe_w8a8_gateup_absmax", "moe_w8a8_prepare_shard",
@@ -108,6 +108,7 @@ def lib():
             "moe_status_string": ([i32], ctypes.c_char_p),
             "moe_w8a8_last_launch_count": ([vp], i32),
             "moe_w8a8_profile_start": ([vp, i32], i32),
+            "moe_w8a8_profile_start_stages": ([vp, i32, ctypes.c_uint32], i32),
             "moe_w8a8_profile_read": ([vp, vp, i32], i32),
             "moe_w8a8_profile_stop": ([vp], i32),
             "moe_w8a8_stage_name": ([i32], ctypes.c_char_p),
@@ -374,6 +375,15 @@ def moe_w8a8_last_launch_count(w: Weights) -> int:
 
 def moe_w8a8_profile_start(w: Weights, max_forwards: int):
     _check(lib().moe_w8a8_profile_start(w.handle, int(max_forwards)), "moe_w8a8_profile_start")
+
+
+def moe_w8a8_profile_start_stages(w: Weights, max_forwards: int, stages):
+    """Event pairs around the listed stages only (indices into STAGE_NAMES)."""
+    mask = 0
+    for st in stages:
+        mask |= 1 << int(st)
+    _check(lib().moe_w8a8_profile_start_stages(w.handle, int(max_forwards), mask),
+           "moe_w8a8_profile_start_stages")
 
 
 def moe_w8a8_profile_read(w: Weights, capacity: int):

@@ -67,6 +67,7 @@ struct moe_w8a8_weights {
     cudaEvent_t* prof_events;   // [prof_max][MOE_N_STAGES][2]
     int prof_max;
     int prof_n;
+    uint32_t prof_mask;         // stages that record their event pair
 };
 
 namespace moe {

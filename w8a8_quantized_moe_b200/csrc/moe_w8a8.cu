@@ -409,7 +409,8 @@ struct Run {
     template <class V>
     V* at(size_t off) const { return reinterpret_cast<V*>(ws + off); }
     void mark(int stage, int edge) const {
-        if (prof) cudaEventRecord(w->prof_events[(w->prof_n * MOE_N_STAGES + stage) * 2 + edge], s);
+        if (prof && (w->prof_mask >> stage & 1u))
+            cudaEventRecord(w->prof_events[(w->prof_n * MOE_N_STAGES + stage) * 2 + edge], s);
     }
     void empty_stage(int stage) const { mark(stage, 0); mark(stage, 1); }
 };
@@ -831,7 +832,11 @@ moe_status moe_w8a8_status_words(const moe_w8a8_weights* w, int32_t* words_host,
 void moe_w8a8_destroy(moe_w8a8_weights* w) { free_handle(w); }
 
 moe_status moe_w8a8_profile_start(moe_w8a8_weights* w, int32_t max_forwards) {
-    if (!w || max_forwards <= 0) return MOE_ERR_INVALID_ARG;
+    return moe_w8a8_profile_start_stages(w, max_forwards, (1u << MOE_N_STAGES) - 1u);
+}
+
+moe_status moe_w8a8_profile_start_stages(moe_w8a8_weights* w, int32_t max_forwards, uint32_t stage_mask) {
+    if (!w || max_forwards <= 0 || stage_mask == 0 || (stage_mask >> MOE_N_STAGES) != 0) return MOE_ERR_INVALID_ARG;
     prof_free(w);
     const int n = max_forwards * MOE_N_STAGES * 2;
     w->prof_events = new cudaEvent_t[n];
@@ -845,6 +850,7 @@ moe_status moe_w8a8_profile_start(moe_w8a8_weights* w, int32_t max_forwards) {
     }
     w->prof_max = max_forwards;
     w->prof_n = 0;
+    w->prof_mask = stage_mask;
     return MOE_OK;
 }
 
@@ -853,6 +859,10 @@ int32_t moe_w8a8_profile_read(moe_w8a8_weights* w, float* ms_host, int32_t capac
     const int n = w->prof_n < capacity ? w->prof_n : capacity;
     for (int i = 0; i < n; ++i)
         for (int st = 0; st < MOE_N_STAGES; ++st) {
+            if (!(w->prof_mask >> st & 1u)) {
+                ms_host[i * MOE_N_STAGES + st] = 0.0f;
+                continue;
+            }
             cudaEvent_t a = w->prof_events[(i * MOE_N_STAGES + st) * 2];
             cudaEvent_t b = w->prof_events[(i * MOE_N_STAGES + st) * 2 + 1];
             if (cudaEventSynchronize(b) != cudaSuccess) return -1;
