@@ -342,7 +342,9 @@ moe_status moe_w8a8_check_status(const moe_w8a8_weights* w, moe_stream_t stream)
  * received expert-parallel row names an expert outside the handle's range
  * (words 2-3: row index, expert); site 15 (with MOE_ERR_INVALID_ARG): a
  * received fixed block's row count is outside [0, block rows - 1] (words 2-3:
- * block, count).  Does not clear them.
+ * block, count); site 17 (with MOE_ERR_INVALID_ARG): the fused expert launch's
+ * plan for at most 32 tokens met an m-tile of more than 32 rows (words 3-4:
+ * m-tile, rows; an internal consistency check).  Does not clear them.
  */
 moe_status moe_w8a8_status_words(const moe_w8a8_weights* w, int32_t* words_host, int32_t n,
                                  moe_stream_t stream);

@@ -231,6 +231,11 @@ cudaError_t launch_tc_ffn_fused(const moe_w8a8_weights* w, int T, const int8_t* 
                                 cudaStream_t s);
 inline size_t fused_sync_words(size_t max_mtiles) { return 2 * max_mtiles + 2; }
 constexpr int kFusedMaxRows = 512;   // default: T*k at or below which the tensor path runs the fused launch
+// At most this many tokens: the fused launch runs its swapped-operand plan (weights as the MMA's
+// 128-row operand, the m-tile's at most 32 token rows as its N = 32 operand), whose partial row
+// maxima cover 32 channels each ([rows][f / 32]; otherwise 64: [rows][f / 64]).
+constexpr int kFusedSwapTokens = 32;
+inline bool fused_swapped(int T) { return T <= kFusedSwapTokens; }
 
 // The per-slot rows o (sorted, [rows][d]) are fp32, or bf16 when o_bf16; the
 // expert FFN writes them in the layer's output precision.

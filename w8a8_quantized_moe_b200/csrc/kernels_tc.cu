@@ -58,10 +58,10 @@ constexpr size_t kSmemBytes = (size_t)kStages * kStageBytes + (size_t)kEpiWarps 
 // Instruction descriptors (both operands K-major, N>>3 at bit 17, M>>4 at bit 24):
 //   kind::i8     D = s32 (bits 4-5 = 2), A and B signed 8-bit (bits 7-9, 10-12 = 1)
 //   kind::f8f6f4 D = f32 (bits 4-5 = 1), A and B E4M3 (bits 7-9, 10-12 = 0)
-template <int FMT>
+template <int FMT, int M = BM, int N = BN>
 __host__ __device__ constexpr uint32_t idesc() {
-    return (FMT == FMT_E4M3 ? (1u << 4) : ((2u << 4) | (1u << 7) | (1u << 10))) | ((uint32_t)(BN >> 3) << 17) |
-           ((uint32_t)(BM >> 4) << 24);
+    return (FMT == FMT_E4M3 ? (1u << 4) : ((2u << 4) | (1u << 7) | (1u << 10))) | ((uint32_t)(N >> 3) << 17) |
+           ((uint32_t)(M >> 4) << 24);
 }
 
 // Row of the tiled weight copy at which k-block kb of the weight rows
@@ -70,15 +70,17 @@ __device__ __forceinline__ int tiled_row(int brow, int kb, int nkb) {
     return ((brow / BN) * nkb + kb) * BN + brow % BN;
 }
 
-struct Ctl {
-    uint64_t full[kStages];
-    uint64_t empty[kStages];
+template <int NS>
+struct CtlT {
+    uint64_t full[NS];
+    uint64_t empty[NS];
     uint64_t acc_full[2];
     uint64_t acc_empty[2];
     uint64_t drain;
     uint32_t tmem_base;
     int abort;
 };
+using Ctl = CtlT<kStages>;
 
 struct TcParams {
     int N, K, n_tiles_n, f, k;
@@ -205,22 +207,23 @@ __device__ __forceinline__ uint64_t desc_sw128(uint32_t saddr) {
     return d;
 }
 
-// One M=128, N=256, K=32 MMA of 8-bit operands: INT8 (s32 accumulators) or
-// E4M3 (f32 accumulators).
-template <int FMT>
+// One K=32 MMA of 8-bit operands, M x N = 128 x 256 unless the instruction
+// descriptor ID says otherwise: INT8 (s32 accumulators) or E4M3 (f32
+// accumulators).
+template <int FMT, uint32_t ID = idesc<FMT>()>
 __device__ __forceinline__ void mma_8bit(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t accum) {
     if (FMT == FMT_E4M3)
         asm volatile(
             "{\n\t.reg .pred p;\n\t"
             "setp.ne.b32 p, %4, 0;\n\t"
             "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(tmem_d),
-            "l"(adesc), "l"(bdesc), "r"(idesc<FMT>()), "r"(accum));
+            "l"(adesc), "l"(bdesc), "r"(ID), "r"(accum));
     else
         asm volatile(
             "{\n\t.reg .pred p;\n\t"
             "setp.ne.b32 p, %4, 0;\n\t"
             "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(tmem_d),
-            "l"(adesc), "l"(bdesc), "r"(idesc<FMT>()), "r"(accum));
+            "l"(adesc), "l"(bdesc), "r"(ID), "r"(accum));
 }
 
 // Accumulator word as a float: INT32 converted, fp32 reinterpreted.
@@ -490,6 +493,83 @@ __device__ __forceinline__ void epilogue_down(const TcParams& p, uint32_t taddr,
                            (int64_t)d * 2, nvalid, lane);
         } else
             store_rows32(stage, a, reinterpret_cast<float*>(p.o) + (int64_t)wrow0 * d + ch0, d, nvalid, lane);
+    }
+}
+
+// Epilogues of the fused launch's swapped-operand plan (at most 32 rows per
+// m-tile): the weights are the MMAs' A operand and the tile's token rows the
+// B operand (N = 32), so an accumulator holds [weight row][token row]: TMEM
+// lane = channel, column = row.  Two accumulators per tile, 32 columns each:
+// GEMM1 gate (columns 0..31) and up (32..63) of 128 channels; GEMM2 output
+// columns nt*256 + [0, 128) and + [128, 256).  A warp reads its TMEM lane
+// quarter (32 channels); per-row scalars are held by lane r and broadcast.
+// The arithmetic per element is that of epilogue_swiglu / epilogue_down.
+constexpr int kFusedSwapRows = 32;
+
+// GEMM1: warp (quad, half) owns channels nt*128 + 32 quad + lane and rows
+// 16 half .. 16 half + 15 (sxr: lane j's row 16 half + j activation scale; sg,
+// su: the lane's channel scales).  The partial maximum of each row over the
+// warp's 32 channels goes to pamax[row][f / 32].
+template <int FMT>
+__device__ __forceinline__ void epilogue_swiglu_sw(const TcParams& p, uint32_t taddr, int half, int quad, int nt,
+                                                   int row0, int nrows, float sg, float su, float sxr,
+                                                   uint64_t* acc_empty, int lane) {
+    const int f = p.f;
+    const int ch = nt * 128 + 32 * quad + lane;
+    const int npart = f / 32, part = nt * 4 + quad;
+    uint32_t g[16], u[16];
+    tmem_ld16(taddr + 16 * half, g);
+    tmem_ld16(taddr + 32 + 16 * half, u);
+    tmem_ld_wait();
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(acc_empty);
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+        const int r = 16 * half + j;
+        const float sx = __shfl_sync(0xffffffffu, sxr, j);
+        if (r >= nrows) break;   // the same for every lane
+        const int64_t grow = row0 + r;
+        if (p.acc_dbg) {
+            p.acc_dbg[grow * 2 * f + ch] = (int32_t)g[j];
+            p.acc_dbg[grow * 2 * f + f + ch] = (int32_t)u[j];
+        }
+        const float gf = __fmul_rn(__fmul_rn(acc_value<FMT>(g[j]), sx), sg);
+        const float uf = __fmul_rn(__fmul_rn(acc_value<FMT>(u[j]), sx), su);
+        const float h = __fmul_rn(moe_silu(gf), uf);
+        p.h32[grow * f + ch] = h;
+        const float m = warp_max(fabsf(h));
+        if (lane == 0) p.pamax[grow * npart + part] = m;
+    }
+}
+
+// GEMM2: warp (quad, half) owns output column nt*256 + 128 half + 32 quad +
+// lane for all rows (shr, wr: lane r's row h scale and routing weight; sw: the
+// lane's column scale).
+template <int FMT>
+__device__ __forceinline__ void epilogue_down_sw(const TcParams& p, uint32_t taddr, int half, int quad, int nt,
+                                                 int row0, int nrows, float sw, float shr, float wr,
+                                                 uint64_t* acc_empty, int lane) {
+    const int d = p.N;
+    const int col = nt * BN + 128 * half + 32 * quad + lane;
+    uint32_t a[32];
+    tmem_ld32(taddr + 32 * half, a);
+    tmem_ld_wait();
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(acc_empty);
+#pragma unroll
+    for (int r = 0; r < kFusedSwapRows; ++r) {
+        const float s_h = __shfl_sync(0xffffffffu, shr, r);
+        const float w_r = __shfl_sync(0xffffffffu, wr, r);
+        if (r >= nrows) break;   // the same for every lane
+        const int64_t grow = row0 + r;
+        if (p.acc_dbg) p.acc_dbg[grow * d + col] = (int32_t)a[r];
+        const float o = __fmul_rn(__fmul_rn(__fmul_rn(acc_value<FMT>(a[r]), s_h), sw), w_r);
+        if (p.o_bf16)
+            reinterpret_cast<uint16_t*>(p.o)[grow * d + col] = f32_to_bf16_bits(o);
+        else
+            reinterpret_cast<float*>(p.o)[grow * d + col] = o;
     }
 }
 
@@ -934,16 +1014,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 // ------------------------------------------------------------------ fused expert FFN (few rows)
 
 // Requantise the rows [row0, row0 + nrows) of h with one warp: the same
-// arithmetic as requant_kernel (sh = max of the row's partial maxima / qmax,
-// codes of h / sh).  Reads through L2 (other CTAs wrote h and the maxima).
+// arithmetic as requant_kernel (sh = max of the row's npart partial maxima /
+// qmax, codes of h / sh).  Reads through L2 (other CTAs wrote h and the maxima).
 // Lane r finds the scale of rows r, r + 32, ... (kept in `scales`, nrows <=
 // 128); then one flat pass over the rows' h with 8 x 16-byte loads per lane
 // in flight, so a few rows cost a few L2 round trips in total.
 template <int FMT>
-__device__ void requant_rows_warp(const float* h32, const float* pamax, int f, int row0, int nrows, int8_t* hq,
-                                  float* sh, float* scales, int lane) {
+__device__ void requant_rows_warp(const float* h32, const float* pamax, int f, int npart, int row0, int nrows,
+                                  int8_t* hq, float* sh, float* scales, int lane) {
     constexpr int kB = 8;
-    const int npart = f / 64, n4 = f / 4;
+    const int n4 = f / 4;
     for (int r = lane; r < nrows; r += 32) {
         const float* pm = pamax + (int64_t)(row0 + r) * npart;
         float m = 0.0f;
@@ -1012,7 +1092,19 @@ struct TileRing {
     uint64_t empty[kTileRing];   // the MMA thread and the 8 epilogue warps have read it
     int tile[kTileRing];         // tile index, or -1 = no more tiles
 };
-constexpr size_t kFusedSmemBytes = kSmemBytes + kEpiStageBytes + 256;
+// Shared-memory plan of the fused launch: per stage the tile's token rows
+// (128, or 32 in the swapped-operand plan) then its 256 weight rows, each
+// 128 bytes of K.
+template <bool SW>
+struct FusedPlan {
+    static constexpr int kT = (SW ? kFusedSwapRows : BM) * BK;
+    static constexpr int kStage = kT + kBBytes;
+    static constexpr int kNStages = kStages;
+    static constexpr size_t kSmem =
+        (size_t)kNStages * kStage + (size_t)(kEpiWarps + 1) * kEpiStageBytes + 1024 + 256 + 256;
+    static_assert(kSmem <= 232448, "shared memory per block");
+    static_assert(kT % 1024 == 0 && kStage % 1024 == 0, "128-byte swizzle atoms stay aligned");
+};
 
 // GEMM1 (gate/up + SwiGLU), the row-wise requantisation of h and GEMM2 (down)
 // in one persistent launch, for launches with few rows per expert (decode),
@@ -1040,21 +1132,23 @@ constexpr size_t kFusedSmemBytes = kSmemBytes + kEpiStageBytes + 256;
 // wait only on GEMM1 tiles, so the waits always end.  Arithmetic per element
 // is that of the two separate kernels and requant_kernel, so the results are
 // identical.
-template <int FMT>
+template <int FMT, bool SW>
 __global__ void __launch_bounds__(kFusedThreads, 1)
     tc_ffn_fused_kernel(const __grid_constant__ CUtensorMap tm_a1, const __grid_constant__ CUtensorMap tm_b1,
                         const __grid_constant__ CUtensorMap tm_a2, const __grid_constant__ CUtensorMap tm_b2,
                         const TcParams p1, const TcParams p2, const FusedExtra fx) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
-    float* epi_stage = reinterpret_cast<float*>(smem + kStages * kStageBytes);
+    using Plan = FusedPlan<SW>;
+    constexpr int NS = Plan::kNStages;
+    float* epi_stage = reinterpret_cast<float*>(smem + NS * Plan::kStage);
     // the requantisation warp's scale buffer follows the epilogue warps' staging buffers
-    Ctl* ctl = reinterpret_cast<Ctl*>(smem + kStages * kStageBytes + (kEpiWarps + 1) * kEpiStageBytes);
+    CtlT<NS>* ctl = reinterpret_cast<CtlT<NS>*>(smem + NS * Plan::kStage + (kEpiWarps + 1) * kEpiStageBytes);
     TileRing* ring = reinterpret_cast<TileRing*>(reinterpret_cast<uint8_t*>(ctl) + 256);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kStages; ++s) {
+        for (int s = 0; s < NS; ++s) {
             mbar_init(&ctl->full[s], 1);
             mbar_init(&ctl->empty[s], 1);
         }
@@ -1102,9 +1196,9 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
             // ---------------- TMA producer
             int s = 0;
             uint32_t ph = 0;
-            uint32_t issued_par[kStages];
-            bool issued[kStages];
-            for (int i = 0; i < kStages; ++i) issued[i] = false;
+            uint32_t issued_par[NS];
+            bool issued[NS];
+            for (int i = 0; i < NS; ++i) issued[i] = false;
             bool ok = true;
             int q = 0;
             uint32_t rph = 0;
@@ -1140,19 +1234,31 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
                     if (!ok) break;
                     fence_proxy_async_global();
                 }
+                if (SW && p.offsets[e + 1] - row0 > kFusedSwapRows) {
+                    // more rows than the swapped plan's token tile holds (the host's
+                    // choice of plan excludes it): report and stop
+                    atomicExch(p.status, (int32_t)MOE_ERR_INVALID_ARG);
+                    if (atomicCAS(p.status + 1, 0, 17) == 0) {
+                        p.status[2] = (int32_t)blockIdx.x;
+                        p.status[3] = mt;
+                        p.status[4] = p.offsets[e + 1] - row0;
+                    }
+                    *abort = 1;
+                    break;
+                }
                 const int nkb = p.K / BK;
                 for (int kb = 0; kb < nkb; ++kb) {
                     if (!mbar_wait(&ctl->empty[s], ph ^ 1, abort, p.status, 1, t)) { ok = false; break; }
-                    mbar_arrive_expect_tx(&ctl->full[s], kStageBytes);
-                    uint8_t* sa = smem + s * kStageBytes;
+                    mbar_arrive_expect_tx(&ctl->full[s], Plan::kStage);
+                    uint8_t* sa = smem + s * Plan::kStage;
                     tma_load_2d(sa, ma, &ctl->full[s], kb * BK, row0);
-                    tma_load_2d(sa + kABytes, mb, &ctl->full[s], kb * BK, brow);
+                    tma_load_2d(sa + Plan::kT, mb, &ctl->full[s], kb * BK, brow);
                     issued[s] = true;
                     issued_par[s] = ph;
-                    if (++s == kStages) { s = 0; ph ^= 1; }
+                    if (++s == NS) { s = 0; ph ^= 1; }
                 }
             }
-            for (int i = 0; i < kStages; ++i) {
+            for (int i = 0; i < NS; ++i) {
                 if (!issued[i]) continue;
                 const uint64_t t0 = global_timer();
                 while (!mbar_try_wait(&ctl->full[i], issued_par[i]) && global_timer() - t0 < kWaitBudgetNs) {}
@@ -1175,18 +1281,31 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
                 const int nkb = (t < w1 ? p1.K : p2.K) / BK;
                 if (!mbar_wait(&ctl->acc_empty[buf], aph ^ 1, abort, p1.status, 2, t)) break;
                 tc_fence_after();
-                const uint32_t d_tmem = tmem + (uint32_t)(buf * BN);
+                const uint32_t d_tmem = tmem + (uint32_t)(buf * (SW ? 2 * kFusedSwapRows : BN));
                 for (int kb = 0; kb < nkb; ++kb) {
                     if (!mbar_wait(&ctl->full[s], ph, abort, p1.status, 3, t)) { ok = false; break; }
                     tc_fence_after();
-                    const uint32_t a_addr = smem_u32(smem + s * kStageBytes);
-                    const uint32_t b_addr = a_addr + kABytes;
+                    const uint32_t t_addr = smem_u32(smem + s * Plan::kStage);
+                    const uint32_t w_addr = t_addr + Plan::kT;
+                    if (SW) {
+                        // weights as A (two 128-row halves), token rows as B (N = 32)
+                        constexpr uint32_t id = idesc<FMT, BM, kFusedSwapRows>();
 #pragma unroll
-                    for (int kk = 0; kk < BK / 32; ++kk)
-                        mma_8bit<FMT>(d_tmem, desc_sw128(a_addr + kk * 32), desc_sw128(b_addr + kk * 32),
-                                      (kb | kk) != 0 ? 1u : 0u);
+                        for (int kk = 0; kk < BK / 32; ++kk) {
+                            const uint64_t bd = desc_sw128(t_addr + kk * 32);
+                            const uint32_t acc = (kb | kk) != 0 ? 1u : 0u;
+                            mma_8bit<FMT, id>(d_tmem, desc_sw128(w_addr + kk * 32), bd, acc);
+                            mma_8bit<FMT, id>(d_tmem + kFusedSwapRows, desc_sw128(w_addr + BM * BK + kk * 32), bd,
+                                              acc);
+                        }
+                    } else {
+#pragma unroll
+                        for (int kk = 0; kk < BK / 32; ++kk)
+                            mma_8bit<FMT>(d_tmem, desc_sw128(t_addr + kk * 32), desc_sw128(w_addr + kk * 32),
+                                          (kb | kk) != 0 ? 1u : 0u);
+                    }
                     mma_commit(&ctl->empty[s]);
-                    if (++s == kStages) { s = 0; ph ^= 1; }
+                    if (++s == NS) { s = 0; ph ^= 1; }
                 }
                 if (!ok) break;
                 mma_commit(&ctl->acc_full[buf]);
@@ -1225,7 +1344,8 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
             const int mt = i;
             const int e = p1.tiles[2 * mt], row0 = p1.tiles[2 * mt + 1];
             const int nrows = min(BM, p1.offsets[e + 1] - row0);
-            requant_rows_warp<FMT>(p1.h32, p1.pamax, p1.f, row0, nrows, fx.hq, fx.sh, scales, lane);
+            requant_rows_warp<FMT>(p1.h32, p1.pamax, p1.f, p1.f / (SW ? 32 : 64), row0, nrows, fx.hq, fx.sh, scales,
+                                   lane);
             // the codes reach the GEMM2 producers' TMA loads (async proxy) and the
             // epilogues' loads through lane 0's release after the warp barrier
             fence_proxy_async_global();
@@ -1258,9 +1378,19 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
             const int nrows = min(BM, p.offsets[e + 1] - row0);
             const int wrow0 = row0 + quad * 32;
             const int nvalid = max(0, min(32, nrows - quad * 32));
-            float r0, r1;
+            float r0, r1, c0 = 0.0f, c1 = 0.0f;
             if (g1) {
-                epi_prefetch<EPI_SWIGLU>(p1, e, nt, half, wrow0 + lane, lane < nvalid, sc, lane, r0, r1);
+                if (SW) {
+                    // the lane's gate / up channel scales; lane j < 16: row 16 half + j's activation scale
+                    const int ch = nt * 128 + 32 * quad + lane;
+                    c0 = p1.sw0[(int64_t)e * p1.f + ch];
+                    c1 = p1.sw1[(int64_t)e * p1.f + ch];
+                    const int r = 16 * half + lane;
+                    r0 = lane < 16 && r < nrows ? p1.sx[p1.row2ts[row0 + r] / p1.k] : 0.0f;
+                    r1 = 0.0f;
+                } else {
+                    epi_prefetch<EPI_SWIGLU>(p1, e, nt, half, wrow0 + lane, lane < nvalid, sc, lane, r0, r1);
+                }
             } else {
                 // the h scales this epilogue reads are released with the m-tile's ready flag:
                 // wait for it (bounded) before fetching them
@@ -1279,14 +1409,26 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
                 rdy = __shfl_sync(0xffffffffu, rdy, 0);
                 if (rdy == 0) break;
                 (void)ld_acquire(fx.ready + mt);   // each lane's own acquire of the released scales
-                epi_prefetch<EPI_DOWN>(p2, e, nt, half, wrow0 + lane, lane < nvalid, sc, lane, r0, r1);
+                if (SW) {
+                    // the lane's output column scale; lane r: row r's h scale and routing weight
+                    c0 = p2.sw0[(int64_t)e * p2.N + nt * BN + 128 * half + 32 * quad + lane];
+                    r0 = lane < nrows ? p2.sh[row0 + lane] : 0.0f;
+                    r1 = lane < nrows ? p2.topk_w[p2.row2ts[row0 + lane]] : 0.0f;
+                } else {
+                    epi_prefetch<EPI_DOWN>(p2, e, nt, half, wrow0 + lane, lane < nvalid, sc, lane, r0, r1);
+                }
             }
             if (!mbar_wait(&ctl->acc_full[buf], aph, abort, p1.status, 4, t)) break;
             tc_fence_after();
-            const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(buf * BN);
+            const uint32_t taddr =
+                tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(buf * (SW ? 2 * kFusedSwapRows : BN));
             if (g1) {
-                epilogue_swiglu<FMT>(p1, taddr, half, e, nt, wrow0, nvalid, stage, sc, r0, &ctl->acc_empty[buf], nullptr,
-                                     lane);
+                if (SW)
+                    epilogue_swiglu_sw<FMT>(p1, taddr, half, quad, nt, row0, nrows, c0, c1, r0, &ctl->acc_empty[buf],
+                                            lane);
+                else
+                    epilogue_swiglu<FMT>(p1, taddr, half, e, nt, wrow0, nvalid, stage, sc, r0, &ctl->acc_empty[buf],
+                                         nullptr, lane);
                 // this warp's share of the tile is stored: count it.  The lanes' stores are
                 // ordered before lane 0's release by the warp barrier (it orders the
                 // participating lanes' memory accesses), and a release publishes everything
@@ -1294,6 +1436,8 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
                 // decode step about 5 us with the requantisation warp's below)
                 __syncwarp();
                 if (lane == 0) red_release_add(fx.count + mt, 1);
+            } else if (SW) {
+                epilogue_down_sw<FMT>(p2, taddr, half, quad, nt, row0, nrows, c0, r0, r1, &ctl->acc_empty[buf], lane);
             } else {
                 epilogue_down<FMT>(p2, taddr, half, e, nt, wrow0, nvalid, stage, sc, r0, r1, &ctl->acc_empty[buf],
                                    nullptr, lane);
@@ -1755,15 +1899,16 @@ cudaError_t launch_tile_weights(const int8_t* src, int64_t rows, int K, int8_t* 
     return cudaGetLastError();
 }
 
-template <int FMT>
+template <int FMT, bool SW>
 cudaError_t launch_fused_fmt(const CUtensorMap& a1, const CUtensorMap& b1, const CUtensorMap& a2,
                              const CUtensorMap& b2, const TcParams& p1, const TcParams& p2, const FusedExtra& fx,
                              int grid, cudaStream_t s) {
     static std::atomic<uint64_t> attr{0};
-    cudaError_t e = smem_attr_once(tc_ffn_fused_kernel<FMT>, kFusedSmemBytes, attr);
+    constexpr size_t smem = FusedPlan<SW>::kSmem;
+    cudaError_t e = smem_attr_once(tc_ffn_fused_kernel<FMT, SW>, smem, attr);
     if (e != cudaSuccess) return e;
-    return launch_pdl(tc_ffn_fused_kernel<FMT>, dim3(grid), dim3(kFusedThreads), kFusedSmemBytes, s, a1, b1, a2,
-                      b2, p1, p2, fx);
+    return launch_pdl(tc_ffn_fused_kernel<FMT, SW>, dim3(grid), dim3(kFusedThreads), smem, s, a1, b1, a2, b2, p1,
+                      p2, fx);
 }
 
 cudaError_t launch_tc_ffn_fused(const moe_w8a8_weights* w, int T, const int8_t* aq, const int32_t* meta,
@@ -1774,7 +1919,11 @@ cudaError_t launch_tc_ffn_fused(const moe_w8a8_weights* w, int T, const int8_t* 
     const moe_w8a8_config& c = w->cfg;
     const int rows = T * c.top_k;
     CUtensorMap a1, a2;
-    if (!make_map(&a1, aq, c.d, rows, BM) || !make_map(&a2, hq, c.f, rows, BM)) return cudaErrorInvalidValue;
+    // at most kFusedSwapRows tokens: each m-tile holds at most that many rows (a token
+    // adds at most one row per expert), and the swapped-operand plan runs
+    const bool sw = fused_swapped(T);
+    const uint32_t trows = sw ? kFusedSwapRows : BM;
+    if (!make_map(&a1, aq, c.d, rows, trows) || !make_map(&a2, hq, c.f, rows, trows)) return cudaErrorInvalidValue;
     TcParams p1{}, p2{};
     p1.N = 2 * c.f;
     p1.K = c.d;
@@ -1808,8 +1957,10 @@ cudaError_t launch_tc_ffn_fused(const moe_w8a8_weights* w, int T, const int8_t* 
                         sh, w->wait_budget_ns, w->test_skip_ready};
     const int grid = max(1, min(w->num_sms, max_mt * (p1.n_tiles_n + p2.n_tiles_n)));
     if (c.expert_format == FMT_E4M3)
-        return launch_fused_fmt<FMT_E4M3>(a1, w->tm_w_gu, a2, w->tm_w_dn, p1, p2, fx, grid, s);
-    return launch_fused_fmt<FMT_INT8>(a1, w->tm_w_gu, a2, w->tm_w_dn, p1, p2, fx, grid, s);
+        return sw ? launch_fused_fmt<FMT_E4M3, true>(a1, w->tm_w_gu, a2, w->tm_w_dn, p1, p2, fx, grid, s)
+                  : launch_fused_fmt<FMT_E4M3, false>(a1, w->tm_w_gu, a2, w->tm_w_dn, p1, p2, fx, grid, s);
+    return sw ? launch_fused_fmt<FMT_INT8, true>(a1, w->tm_w_gu, a2, w->tm_w_dn, p1, p2, fx, grid, s)
+              : launch_fused_fmt<FMT_INT8, false>(a1, w->tm_w_gu, a2, w->tm_w_dn, p1, p2, fx, grid, s);
 }
 
 bool router_tc_make_maps(moe_w8a8_weights* w) {

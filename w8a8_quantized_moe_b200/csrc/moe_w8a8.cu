@@ -154,8 +154,8 @@ WsLayout ws_layout(const moe_w8a8_weights* w, int T, WsPart part) {
     L.sh = take(ex ? tk * 4 : 0);
     L.o = take(ex ? tk * d * o_bytes(c) : 0);
     L.h32 = take(ex && !stream ? tk * f * 4 : 0);
-    L.pamax = take(ex && !stream ? tk * (f / 64) * 4 : 0);
     const bool fused = ex && !stream && fused_ok(w, T);
+    L.pamax = take(ex && !stream ? tk * (f / (fused && fused_swapped(T) ? 32 : 64)) * 4 : 0);
     L.fused_sync = take(fused ? fused_sync_words(max_tiles) * 4 : 0);
     L.fused_words = fused ? (int)fused_sync_words(max_tiles) : 0;
     L.total = p;
