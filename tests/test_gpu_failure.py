@@ -6,6 +6,7 @@ out.  The launch must then end by itself, report MOE_ERR_TIMEOUT with the
 place it gave up, and leave the GPU usable: the next forward on the same
 handle matches the oracle bit for bit.  ("One night of MoE inference
 optimisation", s6.4: a watchdog that turns a stuck step into an error.)"""
+import dataclasses
 import time
 
 import numpy as np
@@ -38,14 +39,17 @@ def _forward_raw(M, W, wl, data):
     torch.cuda.synchronize()
 
 
-def test_withheld_release_times_out_and_the_gpu_stays_usable(M):
-    wl = synth.WORKLOADS["tiny"]            # 64 tokens x top-2 = 128 rows: the fused launch
+@pytest.mark.parametrize("T", [64, 32], ids=["128-row plan", "swapped-operand plan"])
+def test_withheld_release_times_out_and_the_gpu_stays_usable(M, T):
+    # 64 tokens x top-2 = 128 rows: the fused launch with 128-row MMAs; 32 tokens: its
+    # swapped-operand plan (at most 32 rows per expert)
+    wl = dataclasses.replace(synth.WORKLOADS["tiny"], T=T)
     wts = synth.make_weights(wl)
     data = synth.make_data(wl)
     W = H.gpu_prepare(wl, wts, w_router=data.w_router)
     prep = H.oracle_prepare(wl, wts)
     rt = H.oracle_route(wl, data)
-    assert len(np.unique(rt.idx)) == wl.E    # one 128-row tile per expert, tiles 0..7
+    assert len(np.unique(rt.idx)) == wl.E    # one m-tile per expert, tiles 0..7
     M.moe_w8a8_set_path(W, M.MOE_PATH_TENSOR)
     M.moe_w8a8_set_wait_budget(W, 10_000_000)
     M.moe_w8a8_test_withhold_release(W, 3)
