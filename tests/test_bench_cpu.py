@@ -80,3 +80,27 @@ def test_traffic_record_and_lookup(tmp_path, monkeypatch):
     # a different sources hash: the row is ignored
     monkeypatch.setattr(bench, "sources_hash", lambda: "0" * 16)
     assert bench.load_traffic() == {}
+
+
+def test_reference_arm_line_keeps_the_contract():
+    """`bench.py --impl reference` (the CPU oracle as the reference arm) prints one JSON line
+    with the contract's keys; it needs no GPU."""
+    import json
+    import subprocess
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    out = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--impl", "reference",
+                          "--workload", "tiny", "--steps", "2", "--warmup", "1"],
+                         capture_output=True, text=True, timeout=300, cwd=root, check=True).stdout
+    lines = [json.loads(x) for x in out.splitlines() if x.startswith("{")]
+    assert len(lines) == 1
+    d = lines[0]
+    assert d["impl"] == "reference" and d["value"] > 0 and d["unit"] == "tokens/s"
+    for key in ("metric", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better", "scaling",
+                "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert key in d, key
+    assert (d["steps"], d["warmup"], d["n_gpus"]) == (2, 1, 1)
+    assert all(k in d["config"] for k in ("workload", "T", "d", "E", "k", "f"))
+    cb = d["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == d["value"] and cb["sample"]
+    assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}
